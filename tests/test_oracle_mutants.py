@@ -1,0 +1,100 @@
+"""Planted mistakes in copies of the oracle must each fail at least one pin.
+
+Every mutant below is a plausible slip (a dropped term, a flipped sign, a wrong
+or transposed index, a missing factor).  Each is applied to a copy of
+oracle/lla_oracle.c in a temporary directory, compiled with gcc and loaded in
+place of the real oracle while the pins of test_oracle_pins.py run.  If a
+mutant survives every pin, the pins are too weak and this test fails.  All
+mutants keep every array access in bounds.  CPU only.
+"""
+import ctypes
+import os
+import subprocess
+
+import pytest
+
+import oracle
+import test_oracle_pins as P
+
+SRC = os.path.join(os.path.dirname(oracle.__file__), "lla_oracle.c")
+
+MUTANTS = {
+    "encode_sign_of_mean": ("(x[i * W + k] - mu[k])", "(x[i * W + k] + mu[k])"),
+    "encode_transposed_W_down": ("W_down[(int64_t)k * r + j]", "W_down[(int64_t)j * W + k]"),
+    "reconstruct_drops_mean": ("double acc = mu_t[k];", "double acc = 0.0;"),
+    "reconstruct_transposed_W_up": ("W_up_t[(int64_t)j * d + k]", "W_up_t[(int64_t)k * r + j]"),
+    "softmax_no_max_subtraction": ("p[i] = exp(l[i] - m);", "p[i] = exp(l[i]);"),
+    "softmax_lse_drops_max": ("*lse = m + log(Z);", "*lse = log(Z);"),
+    "softmax_not_normalised": ("p[i] /= Z;", "p[i] /= 1.0;"),
+    "softmax_min_instead_of_max": ("if (l[i] > m)", "if (l[i] < m)"),
+    "reconstruct_attn_reversed_dot": ("dot += q[k] * k_hat[k];", "dot += q[k] * k_hat[d - 1 - k];"),
+    "absorb_drops_scale": ("q_tilde[j] = scale * acc;", "q_tilde[j] = acc;"),
+    "absorb_mean_term_sign": ("l[i] = dot + q_mu;", "l[i] = dot - q_mu;"),
+    "absorb_drops_value_mean": ("double acc = mu_V_t[k];", "double acc = 0.0;"),
+    "absorb_transposed_W_up_K": ("acc += q[k] * W_up_K_t[(int64_t)j * d + k];",
+                                 "acc += q[k] * W_up_K_t[(int64_t)k * r_k + j];"),
+    "absorb_reversed_value_latent": ("o_lat[j] += p[i] * c_V[i * r_v + j];",
+                                     "o_lat[j] += p[i] * c_V[i * r_v + (r_v - 1 - j)];"),
+    "absorb_wrong_key_latent_row": ("dot += q_tilde[j] * c_K[i * r_k + j];",
+                                    "dot += q_tilde[j] * c_K[(n - 1 - i) * r_k + j];"),
+    "bytes_drop_factor_two": ("2ull * (uint64_t)T * (uint64_t)H", "(uint64_t)T * (uint64_t)H"),
+    "bytes_fold_swapped": ("fold2d ? 1u : (uint64_t)H", "fold2d ? (uint64_t)H : 1u"),
+    "bytes_ratio_not_reduced": ("uint64_t g = gcd_u64(per_token_uncompressed, per_token_latent);",
+                                "uint64_t g = 1;"),
+}
+
+
+def _pins():
+    pins = [
+        (P.test_rank_table_golden, {}),
+        (P.test_headline_ratios_golden, {}),
+        (P.test_rho_closed_forms, {}),
+        (P.test_capacity_bytes_exact, {}),
+        (P.test_cache_bytes_linear_and_divided_by_rho, {}),
+        (P.test_full_rank_roundtrip_is_exact, {}),
+        (P.test_encode_of_mean_is_zero_and_affine, {}),
+        (P.test_reconstruct_orientation_one_hot, {}),
+        (P.test_eckart_young_calibration_residual, {"r": 4}),
+        (P.test_absorb_equals_reconstruct_low_rank, {}),
+        (P.test_decode_layer_matches_masked_dense_attention, {"fold2d": True}),
+    ]
+    for v in P.VARIANTS:
+        pins += [
+            (P.test_full_rank_codec_equals_uncompressed_attention, {"variant": v, "scale": 0.125}),
+            (P.test_softmax_weights_sum_to_one, {"variant": v}),
+            (P.test_shift_of_key_mean_is_invisible, {"variant": v}),
+            (P.test_single_token_returns_its_value, {"variant": v}),
+            (P.test_identity_codec_is_textbook_attention, {"variant": v}),
+            (P.test_large_logits_select_the_best_token, {"variant": v}),
+            (P.test_fold2d_full_rank_reproduces_each_head, {"variant": v}),
+        ]
+    return pins
+
+
+def test_unmutated_oracle_passes_every_pin():
+    for fn, kw in _pins():
+        fn(**kw)
+
+
+@pytest.mark.parametrize("name", sorted(MUTANTS))
+def test_mutant_is_caught(name, tmp_path):
+    old, new = MUTANTS[name]
+    src = open(SRC).read()
+    assert src.count(old) == 1, f"mutation site for {name} not unique"
+    path_c = tmp_path / "mutant.c"
+    path_c.write_text(src.replace(old, new))
+    path_so = tmp_path / "mutant.so"
+    subprocess.check_call(["gcc", "-O2", "-std=c11", "-fPIC", "-shared", "-ffp-contract=off",
+                           str(path_c), "-o", str(path_so), "-lm"])
+    saved = oracle._load()
+    oracle._lib = oracle.configure(ctypes.CDLL(str(path_so)))
+    failed = []
+    try:
+        for fn, kw in _pins():
+            try:
+                fn(**kw)
+            except (AssertionError, ValueError, FloatingPointError):
+                failed.append(fn.__name__)
+    finally:
+        oracle._lib = saved
+    assert failed, f"mutant {name} survived every pin"

@@ -1,0 +1,386 @@
+"""Pins for the fp64 CPU oracle: values and identities the pages and the mathematics fix.
+
+Nothing here compares the oracle with itself.  Each test checks it against
+something independent: numbers printed on the pages (golden files), closed forms,
+a library routine for a special case (torch scaled_dot_product_attention in
+float64), or an algebraic identity whose failure a dropped term, a wrong sign,
+a wrong loop index or a transposed operand would expose.
+"""
+import math
+import os
+from fractions import Fraction
+
+import numpy as np
+import pytest
+import torch
+
+import lla_synth as S
+import oracle
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def _rows(name):
+    with open(os.path.join(GOLDEN, name)) as f:
+        return [line.split() for line in f if line.strip() and not line.startswith("#")]
+
+
+def sdpa(q, K, V, scale):
+    """Textbook attention of one query via torch (float64): returns (o, lse)."""
+    qt = torch.as_tensor(q, dtype=torch.float64)[None, None, None, :]
+    Kt = torch.as_tensor(K, dtype=torch.float64)[None, None]
+    Vt = torch.as_tensor(V, dtype=torch.float64)[None, None]
+    o = torch.nn.functional.scaled_dot_product_attention(qt, Kt, Vt, scale=scale)
+    lse = torch.logsumexp(scale * (Kt[0, 0] @ qt[0, 0, 0]), dim=0)
+    return o[0, 0, 0].numpy(), float(lse)
+
+
+# ---------------------------------------------------------------------------
+# Eq. 4 / Figure 10 / Table 8: exact compression ratio and cache bytes
+# ---------------------------------------------------------------------------
+def test_rank_table_golden():
+    rows = _rows("rank_table.txt")
+    assert len(rows) == 6
+    for T, d, rk, rv, printed in rows:
+        lat, unc, num, den = oracle.cache_bytes(int(T), 1, 1, int(d), int(rk), int(rv),
+                                                False, 2, 1)
+        digits = len(printed.split(".")[1]) if "." in printed else 0
+        assert round(num / den, digits) == float(printed)
+        assert Fraction(unc, lat) == Fraction(num, den)
+
+
+def test_headline_ratios_golden():
+    for T, d, rsum, printed, digits in _rows("headline_ratios.txt"):
+        rk = int(rsum) // 3
+        rv = int(rsum) - rk
+        _, _, num, den = oracle.cache_bytes(int(T), 1, 1, int(d), rk, rv, False, 2, 1)
+        assert round(num / den, int(digits)) == float(printed)
+
+
+def test_rho_closed_forms():
+    # per head: 2*T*d/(r_k+r_v), reduced
+    assert oracle.cache_bytes(4, 1, 16, 128, 16, 32, False, 2, 1)[2:] == (64, 3)
+    assert oracle.cache_bytes(4, 1, 2, 64, 8, 16, False, 4, 1)[2:] == (64, 3)
+    assert oracle.cache_bytes(4, 24, 16, 128, 96, 160, False, 2, 1)[2:] == (4, 1)
+    assert oracle.cache_bytes(32, 8, 16, 128, 96, 160, False, 2, 1)[2:] == (32, 1)
+    # LLA-2D folds the H heads into one latent: 2*T*H*d/(r_k+r_v) = 16384/192
+    assert oracle.cache_bytes(4, 24, 16, 128, 64, 128, True, 2, 1)[2:] == (256, 3)
+
+
+def test_capacity_bytes_exact():
+    # 768 sequences x 4096 tokens, 24 layers, 16 heads, r_k+r_v = 48, bf16
+    lat, unc, num, den = oracle.cache_bytes(4, 24, 16, 128, 16, 32, False, 2, 768 * 4096)
+    assert lat == 768 * 4096 * 24 * 16 * 48 * 2 == 115_964_116_992
+    assert unc == 768 * 4096 * 24 * 16 * 2 * 4 * 128 * 2
+    assert lat * num == unc * den
+
+
+def test_cache_bytes_linear_and_divided_by_rho():
+    rng = np.random.default_rng(5)
+    for _ in range(200):
+        T, L, H = (int(v) for v in rng.integers(1, 40, 3))
+        d = int(rng.choice([16, 32, 64, 128, 256]))
+        rk, rv = (int(v) for v in rng.integers(1, 600, 2))
+        fold = bool(rng.integers(0, 2))
+        e = int(rng.choice([2, 4]))
+        n = int(rng.integers(0, 10 ** 7))
+        lat, unc, num, den = oracle.cache_bytes(T, L, H, d, rk, rv, fold, e, n)
+        lat2, unc2, _, _ = oracle.cache_bytes(T, L, H, d, rk, rv, fold, e, 2 * n + 3)
+        assert lat2 * n == lat * (2 * n + 3) and unc2 * n == unc * (2 * n + 3)
+        assert lat * num == unc * den
+        assert math.gcd(num, den) == 1
+        Hs = 1 if fold else H
+        assert Fraction(num, den) == Fraction(2 * T * H * d, Hs * (rk + rv))
+
+
+def test_cache_bytes_rejects_bad_dims():
+    with pytest.raises(ValueError):
+        oracle.cache_bytes(0, 1, 1, 64, 8, 16, False, 2, 1)
+    with pytest.raises(ValueError):
+        oracle.cache_bytes(4, 1, 1, 64, 8, 16, False, 2, -1)
+
+
+# ---------------------------------------------------------------------------
+# Eqs. 2-3: encode and per-loop reconstruction
+# ---------------------------------------------------------------------------
+def test_full_rank_roundtrip_is_exact():
+    T, d = 4, 8
+    codec = S.orthonormal_codec(T * d, T, seed=1)
+    x = np.random.default_rng(2).standard_normal((50, T * d)) * 3 + 1
+    c = oracle.encode(x, codec.mu, codec.W_down)
+    for t in range(T):
+        xt = oracle.reconstruct(c, codec.W_up[t], codec.mu_t()[t])
+        np.testing.assert_allclose(xt, x[:, t * d:(t + 1) * d], atol=1e-12, rtol=0)
+
+
+def test_encode_of_mean_is_zero_and_affine():
+    T, d, r = 3, 8, 5
+    rng = np.random.default_rng(3)
+    W_down = rng.standard_normal((T * d, r))
+    mu = rng.standard_normal(T * d)
+    np.testing.assert_allclose(oracle.encode(mu[None], mu, W_down), 0.0, atol=1e-14)
+    x1, x2 = rng.standard_normal((2, 7, T * d))
+    a = 0.3
+    lhs = oracle.encode(a * x1 + (1 - a) * x2, mu, W_down)
+    rhs = a * oracle.encode(x1, mu, W_down) + (1 - a) * oracle.encode(x2, mu, W_down)
+    np.testing.assert_allclose(lhs, rhs, atol=1e-12)
+    # one-hot tokens pick rows of W_down (checks operand orientation)
+    e = np.zeros((T * d, T * d))
+    np.fill_diagonal(e, 1.0)
+    np.testing.assert_allclose(oracle.encode(e, np.zeros(T * d), W_down), W_down, atol=0)
+
+
+def test_reconstruct_orientation_one_hot():
+    r, d = 5, 7
+    rng = np.random.default_rng(4)
+    W_up = rng.standard_normal((r, d))
+    mu = rng.standard_normal(d)
+    c = np.eye(r)
+    np.testing.assert_allclose(oracle.reconstruct(c, W_up, mu), W_up + mu[None], atol=0)
+
+
+@pytest.mark.parametrize("r", [1, 4, 16, 40])
+def test_eckart_young_calibration_residual(r):
+    """Residual of the SVD codec on its own calibration set = tail singular energy."""
+    w = S.shrink(S.WORKLOADS["tiny-fp32"], d=16)
+    model = S.trajectory_model(11, w.T * w.d)
+    x_cal = S.draw_tokens_np(model, S.N_CALIB, 12)
+    codec = S.fit_codec(x_cal, r, w.T)
+    c = oracle.encode(x_cal, codec.mu, codec.W_down)
+    resid = 0.0
+    for t in range(w.T):
+        xt = oracle.reconstruct(c, codec.W_up[t], codec.mu_t()[t])
+        resid += ((x_cal[:, t * w.d:(t + 1) * w.d] - xt) ** 2).sum()
+    tail = (codec.sigma[r:] ** 2).sum()
+    assert resid == pytest.approx(tail, rel=1e-9, abs=1e-9)
+
+
+# ---------------------------------------------------------------------------
+# Decode attention (reconstruct and absorb forms)
+# ---------------------------------------------------------------------------
+VARIANTS = ["absorb", "reconstruct"]
+
+
+def _codec_pair(T, d, rk, rv, seed, perturb=0.2):
+    rng = np.random.default_rng(seed)
+    out = []
+    for r in (rk, rv):
+        W_up = rng.standard_normal((T, r, d)) / math.sqrt(r)
+        mu = rng.standard_normal((T, d))
+        out.append((W_up * (1 + perturb), mu))
+    return out
+
+
+@pytest.mark.parametrize("variant", VARIANTS)
+@pytest.mark.parametrize("scale", [1.0, 0.125, 3.0])
+def test_full_rank_codec_equals_uncompressed_attention(variant, scale):
+    """Full-rank orthonormal codec: decode over latents == plain attention on K/V."""
+    T, d, n = 3, 8, 20
+    rng = np.random.default_rng(7)
+    cK, cV = S.orthonormal_codec(T * d, T, 8), S.orthonormal_codec(T * d, T, 9)
+    xK = rng.standard_normal((n, T * d))
+    xV = rng.standard_normal((n, T * d)) * 2
+    lK, lV = oracle.encode(xK, cK.mu, cK.W_down), oracle.encode(xV, cV.mu, cV.W_down)
+    for t in range(T):
+        q = rng.standard_normal(d)
+        o, lse = oracle.attend(variant, lK, lV, cK.W_up[t], cK.mu_t()[t], cV.W_up[t],
+                               cV.mu_t()[t], q, scale)
+        o_ref, lse_ref = sdpa(q, xK[:, t * d:(t + 1) * d], xV[:, t * d:(t + 1) * d], scale)
+        np.testing.assert_allclose(o, o_ref, atol=1e-10, rtol=0)
+        assert lse == pytest.approx(lse_ref, abs=1e-10)
+
+
+def test_absorb_equals_reconstruct_low_rank():
+    T, d, rk, rv, n = 4, 16, 3, 6, 33
+    rng = np.random.default_rng(10)
+    (WK, muK), (WV, muV) = _codec_pair(T, d, rk, rv, 11)
+    cK = rng.standard_normal((n, rk))
+    cV = rng.standard_normal((n, rv))
+    for t in range(T):
+        q = rng.standard_normal(d)
+        a = oracle.attend("absorb", cK, cV, WK[t], muK[t], WV[t], muV[t], q, 0.7)
+        b = oracle.attend("reconstruct", cK, cV, WK[t], muK[t], WV[t], muV[t], q, 0.7)
+        np.testing.assert_allclose(a[0], b[0], atol=1e-10, rtol=0)
+        assert a[1] == pytest.approx(b[1], abs=1e-10)
+
+
+@pytest.mark.parametrize("variant", VARIANTS)
+def test_softmax_weights_sum_to_one(variant):
+    """Constant values: o must equal that value exactly when sum_n p_n = 1."""
+    T, d, rk, rv, n = 2, 8, 4, 5, 17
+    rng = np.random.default_rng(12)
+    (WK, muK), (WV, muV) = _codec_pair(T, d, rk, rv, 13)
+    cK = rng.standard_normal((n, rk)) * 3
+    v0 = rng.standard_normal(rv)
+    cV = np.tile(v0, (n, 1))
+    q = rng.standard_normal(d)
+    o, _ = oracle.attend(variant, cK, cV, WK[1], muK[1], WV[1], muV[1], q, 1.0)
+    np.testing.assert_allclose(o, v0 @ WV[1] + muV[1], atol=1e-12)
+    o0, _ = oracle.attend(variant, cK, 0 * cV, WK[1], muK[1], WV[1], muV[1], q, 1.0)
+    np.testing.assert_allclose(o0, muV[1], atol=1e-14)
+
+
+@pytest.mark.parametrize("variant", VARIANTS)
+def test_shift_of_key_mean_is_invisible(variant):
+    T, d, rk, rv, n = 2, 8, 4, 5, 9
+    rng = np.random.default_rng(14)
+    (WK, muK), (WV, muV) = _codec_pair(T, d, rk, rv, 15)
+    cK, cV = rng.standard_normal((n, rk)), rng.standard_normal((n, rv))
+    q = rng.standard_normal(d)
+    delta = rng.standard_normal(d)
+    s = 0.9
+    o1, l1 = oracle.attend(variant, cK, cV, WK[0], muK[0], WV[0], muV[0], q, s)
+    o2, l2 = oracle.attend(variant, cK, cV, WK[0], muK[0] + delta, WV[0], muV[0], q, s)
+    np.testing.assert_allclose(o1, o2, atol=1e-12)
+    assert l2 - l1 == pytest.approx(s * q @ delta, abs=1e-12)
+
+
+@pytest.mark.parametrize("variant", VARIANTS)
+def test_single_token_returns_its_value(variant):
+    T, d, rk, rv = 3, 8, 4, 6
+    rng = np.random.default_rng(16)
+    (WK, muK), (WV, muV) = _codec_pair(T, d, rk, rv, 17)
+    cK, cV = rng.standard_normal((1, rk)), rng.standard_normal((1, rv))
+    q = rng.standard_normal(d)
+    o, lse = oracle.attend(variant, cK, cV, WK[2], muK[2], WV[2], muV[2], q, 0.5)
+    np.testing.assert_allclose(o, cV[0] @ WV[2] + muV[2], atol=1e-12)
+    assert lse == pytest.approx(0.5 * q @ (cK[0] @ WK[2] + muK[2]), abs=1e-12)
+
+
+@pytest.mark.parametrize("variant", VARIANTS)
+def test_identity_codec_is_textbook_attention(variant):
+    """T = 1, r = d, W_down = I, mu = 0: the latents are K and V themselves."""
+    d, n = 8, 25
+    rng = np.random.default_rng(18)
+    K, V, q = rng.standard_normal((n, d)), rng.standard_normal((n, d)), rng.standard_normal(d)
+    I, z = np.eye(d), np.zeros(d)
+    cK, cV = oracle.encode(K, z, I), oracle.encode(V, z, I)
+    o, lse = oracle.attend(variant, cK, cV, I, z, I, z, q, 1 / math.sqrt(d))
+    o_ref, lse_ref = sdpa(q, K, V, 1 / math.sqrt(d))
+    np.testing.assert_allclose(o, o_ref, atol=1e-12)
+    assert lse == pytest.approx(lse_ref, abs=1e-12)
+
+
+@pytest.mark.parametrize("variant", VARIANTS)
+def test_large_logits_select_the_best_token(variant):
+    """Very large scale: softmax becomes argmax and stays finite (max subtraction)."""
+    d, n = 8, 40
+    rng = np.random.default_rng(19)
+    I, z = np.eye(d), np.zeros(d)
+    K, V, q = rng.standard_normal((n, d)), rng.standard_normal((n, d)), rng.standard_normal(d)
+    o, lse = oracle.attend(variant, K, V, I, z, I, z, q, 1e4)
+    best = int(np.argmax(K @ q))
+    assert np.all(np.isfinite(o)) and math.isfinite(lse)
+    np.testing.assert_allclose(o, V[best], atol=1e-9)
+    assert lse == pytest.approx(1e4 * K[best] @ q, rel=1e-12)
+
+
+@pytest.mark.parametrize("variant", VARIANTS)
+def test_empty_context(variant):
+    d = 8
+    o, lse = oracle.attend(variant, np.zeros((0, 3)), np.zeros((0, 4)), np.ones((3, d)),
+                           np.ones(d), np.ones((4, d)), np.ones(d), np.ones(d), 1.0)
+    assert np.all(o == 0) and lse == -math.inf
+
+
+def _ragged_layer(T, H, d, lens, rk, rv, fold2d, seed, gap=3):
+    rng = np.random.default_rng(seed)
+    starts = S.slot_starts(np.asarray(lens), gap=gap)
+    n_slots = int(starts[-1] + lens[-1] + gap)
+    Hs = 1 if fold2d else H
+    c_K = rng.standard_normal((Hs, n_slots, rk))
+    c_V = rng.standard_normal((Hs, n_slots, rv))
+    if fold2d:
+        WK = rng.standard_normal((T, rk, H * d)) / math.sqrt(rk)
+        WV = rng.standard_normal((T, rv, H * d)) / math.sqrt(rv)
+        mK, mV = rng.standard_normal((T, H * d)), rng.standard_normal((T, H * d))
+    else:
+        WK = rng.standard_normal((H, T, rk, d)) / math.sqrt(rk)
+        WV = rng.standard_normal((H, T, rv, d)) / math.sqrt(rv)
+        mK, mV = rng.standard_normal((H, T, d)), rng.standard_normal((H, T, d))
+    return starts, c_K, c_V, WK, mK, WV, mV
+
+
+@pytest.mark.parametrize("fold2d", [False, True])
+def test_decode_layer_matches_masked_dense_attention(fold2d):
+    """Ragged batch: per-sequence slicing checked against dense reconstruct + SDPA."""
+    T, H, d, rk, rv = 3, 2, 8, 4, 6
+    lens = np.array([5, 1, 0, 9], dtype=np.int32)
+    starts, c_K, c_V, WK, mK, WV, mV = _ragged_layer(T, H, d, lens, rk, rv, fold2d, 20)
+    B, Tq, t0, s = len(lens), 2, 1, 0.8
+    q = np.random.default_rng(21).standard_normal((B, Tq, H, d))
+    for variant in VARIANTS:
+        o, lse = oracle.decode_layer(variant, q, c_K, c_V, starts, lens, WK, mK, WV, mV,
+                                     t0, s, fold2d=fold2d, threads=2)
+        for b in range(B):
+            sl = slice(int(starts[b]), int(starts[b] + lens[b]))
+            for tq in range(Tq):
+                t = t0 + tq
+                for h in range(H):
+                    if fold2d:
+                        cols = slice(h * d, (h + 1) * d)
+                        Kh = c_K[0, sl] @ WK[t][:, cols] + mK[t][cols]
+                        Vh = c_V[0, sl] @ WV[t][:, cols] + mV[t][cols]
+                    else:
+                        Kh = c_K[h, sl] @ WK[h, t] + mK[h, t]
+                        Vh = c_V[h, sl] @ WV[h, t] + mV[h, t]
+                    if lens[b] == 0:
+                        assert np.all(o[b, tq, h] == 0) and lse[b, tq, h] == -np.inf
+                        continue
+                    o_ref, lse_ref = sdpa(q[b, tq, h], Kh, Vh, s)
+                    np.testing.assert_allclose(o[b, tq, h], o_ref, atol=1e-11)
+                    assert lse[b, tq, h] == pytest.approx(lse_ref, abs=1e-11)
+
+
+def test_fold2d_with_one_head_equals_per_head():
+    T, H, d, rk, rv = 3, 1, 8, 4, 6
+    lens = np.array([7, 3], dtype=np.int32)
+    starts, c_K, c_V, WK, mK, WV, mV = _ragged_layer(T, H, d, lens, rk, rv, True, 22)
+    q = np.random.default_rng(23).standard_normal((2, 3, H, d))
+    a = oracle.decode_layer("absorb", q, c_K, c_V, starts, lens, WK, mK, WV, mV, 0, 1.0,
+                            fold2d=True, threads=1)
+    b = oracle.decode_layer("absorb", q, c_K, c_V, starts, lens, WK[None], mK[None],
+                            WV[None], mV[None], 0, 1.0, fold2d=False, threads=1)
+    np.testing.assert_array_equal(a[0], b[0])
+    np.testing.assert_array_equal(a[1], b[1])
+
+
+@pytest.mark.parametrize("variant", VARIANTS)
+def test_fold2d_full_rank_reproduces_each_head(variant):
+    """LLA-2D full-rank codec over x in [T][H][d] order: head h's output equals plain
+    attention on head h's own original K/V (pins the head column slicing)."""
+    T, H, d, n = 2, 3, 4, 11
+    W = T * H * d
+    rng = np.random.default_rng(24)
+    cK, cV = S.orthonormal_codec(W, T, 25), S.orthonormal_codec(W, T, 26)
+    xK, xV = rng.standard_normal((n, W)), rng.standard_normal((n, W))
+    lK, lV = oracle.encode(xK, cK.mu, cK.W_down), oracle.encode(xV, cV.mu, cV.W_down)
+    q = rng.standard_normal((1, T, H, d))
+    o, lse = oracle.decode_layer(variant, q, lK[None], lV[None], [0], [n], cK.W_up,
+                                 cK.mu_t(), cV.W_up, cV.mu_t(), 0, 1.0, fold2d=True,
+                                 threads=1)
+    xK4, xV4 = xK.reshape(n, T, H, d), xV.reshape(n, T, H, d)
+    for t in range(T):
+        for h in range(H):
+            o_ref, lse_ref = sdpa(q[0, t, h], xK4[:, t, h], xV4[:, t, h], 1.0)
+            np.testing.assert_allclose(o[0, t, h], o_ref, atol=1e-10)
+            assert lse[0, t, h] == pytest.approx(lse_ref, abs=1e-10)
+
+
+# ---------------------------------------------------------------------------
+# The input generator's stated statistics (pins the recipe, not the oracle)
+# ---------------------------------------------------------------------------
+def test_trajectory_model_energy_split():
+    m = S.trajectory_model(30, 512)
+    e = (m.A ** 2).sum(axis=1) / 512
+    assert e.sum() == pytest.approx(1.0, abs=1e-12)
+    assert e[0] == pytest.approx(S.TOP_ENERGY, abs=1e-12)
+    np.testing.assert_allclose(m.A @ m.A.T, np.diag(e * 512), atol=1e-9)
+    assert np.all(np.diff(e[1:]) < 0)
+
+
+def test_latent_draw_statistics():
+    std = np.array([3.0, 1.0, 0.25])
+    z = S.draw_latents(200_000, std, 31, "cpu", torch.float32).double().numpy()
+    np.testing.assert_allclose(z.std(axis=0), std, rtol=0.01)
+    np.testing.assert_allclose(z.mean(axis=0), 0, atol=0.02)
