@@ -1,0 +1,412 @@
+"""Benchmark: LLA decode step on B200 -- latent-cache GB/s, token-loop reads/s, HBM roofline.
+
+One step = one decode step of an Ouro-1.4B-shaped layer (T=4 loops, H=16 heads,
+d=128, r_k=16 / r_v=32, rho = 21.3, B=64 sequences with context lengths uniform in
+[2048, 4096]): the four loop queries of every sequence attend over the latent cache
+(lla_decode_attn, absorbed form, all loops fused in one pass), then the finished
+token's stacked K/V are encoded into the cache (lla_encode).  Inputs are resident
+in HBM before timing; the latent cache (302 MB) is larger than L2 and the timed
+loop also rotates over 3 independent cache replicas, so no step reads latents
+another recent step left in L2.
+
+Prints ONE JSON line on rank 0.  `python bench.py --gpus N --steps K --warmup W`;
+N > 1 runs under torchrun as independent replicas (weak scaling, no collective on
+the data path; the barrier and the max-over-ranks reduction are the only
+communication).  `--impl reference` times the fp64 CPU oracle instead (the pages
+ship no implementation to run); see `cpu_baseline`.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "LLA decode latent-cache GB/s & token-loop reads/s (% of HBM roofline) at 1 B200"
+WORKLOAD = "ouro1.4b-layer"
+SPEC_HBM_GBS = 8000.0
+PROFILE_TRAFFIC = os.path.join(ROOT, "profiles", "decode_absorb_simt.ouro1.4b-layer.json")
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--workload", default=WORKLOAD)
+    ap.add_argument("--num-splits", type=int, default=0)
+    ap.add_argument("--replicas", type=int, default=3)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=10.0)
+    return ap.parse_args()
+
+
+def measured_peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            return json.load(f), "measured"
+    except OSError:
+        return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0}, "fallback"
+
+
+def kernel_source_hash():
+    h = hashlib.sha256()
+    for rel in ("decode_attention_12_b200/csrc/decode_simt.cu", "decode_attention_12_b200/csrc/decode.cuh",
+                "decode_attention_12_b200/csrc/common.cuh"):
+        with open(os.path.join(ROOT, rel), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def profiled_traffic(units_per_launch):
+    """DRAM bytes per launch from the committed ncu summary, or None if stale/absent."""
+    try:
+        with open(PROFILE_TRAFFIC) as f:
+            prof = json.load(f)
+    except (OSError, ValueError):
+        return None
+    if prof.get("source_hash") != kernel_source_hash():
+        return None
+    per_unit = prof["dram_bytes_per_launch"] / prof["units_per_launch"]
+    return per_unit * units_per_launch
+
+
+# ---------------------------------------------------------------------------
+# clocks: NVML samples during the timed region (read-only queries)
+# ---------------------------------------------------------------------------
+class ClockSampler:
+    REASONS = {
+        "gpu_idle": 0x1, "applications_clocks_setting": 0x2, "sw_power_cap": 0x4,
+        "hw_slowdown": 0x8, "sync_boost": 0x10, "sw_thermal_slowdown": 0x20,
+        "hw_thermal_slowdown": 0x40, "hw_power_brake_slowdown": 0x80,
+        "display_clock_setting": 0x100,
+    }
+
+    def __init__(self, index, period=0.005):
+        self.samples, self.period, self.ok = [], period, False
+        self._stop = threading.Event()
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self.nv = pynvml
+            self.h = pynvml.nvmlDeviceGetHandleByIndex(index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+            self.ok = True
+        except Exception:
+            self.max_mhz = None
+
+    def _run(self):
+        nv = self.nv
+        while not self._stop.is_set():
+            try:
+                mhz = nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM)
+                rs = nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+                self.samples.append((time.perf_counter(), mhz, rs))
+            except Exception:
+                pass
+            time.sleep(self.period)
+
+    def start(self):
+        if self.ok:
+            self.t = threading.Thread(target=self._run, daemon=True)
+            self.t.start()
+        return self
+
+    def stop(self):
+        if self.ok:
+            self._stop.set()
+            self.t.join()
+
+    def summary(self, t0, t1):
+        if not self.ok or not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": [], "samples": 0}
+        inside = [s for s in self.samples if t0 <= s[0] <= t1]
+        if not inside:  # a short timed region: take the samples nearest to it
+            inside = sorted(self.samples, key=lambda s: abs(s[0] - 0.5 * (t0 + t1)))[:3]
+        mhz = statistics.median(s[1] for s in inside)
+        bits = 0
+        for s in inside:
+            bits |= s[2]
+        reasons = [n for n, b in self.REASONS.items() if bits & b and n != "gpu_idle"]
+        return {"sm_mhz": mhz, "sm_max_mhz": self.max_mhz, "reasons": reasons,
+                "samples": len(inside)}
+
+
+# ---------------------------------------------------------------------------
+# the CPU oracle leg (cpu_baseline, and the --impl reference arm)
+# ---------------------------------------------------------------------------
+def oracle_sample_rate(p, w, Tq, max_seconds, units_per_round=None):
+    """Time the fp64 oracle on (b, h) units of the same step; returns (GB/s, info)."""
+    import oracle
+    import torch
+
+    def f64(t):
+        return t.detach().to(torch.float32).cpu().double().numpy()
+
+    q = f64(p["q"])
+    cK, cV = f64(p["k"][0]), f64(p["v"][0])
+    WK, WV, mK, mV = (f64(p[n][0]) for n in ("W_up_k", "W_up_v", "mu_k", "mu_v"))
+    threads = os.cpu_count() or 1
+    all_units = [(b, h) for b in range(w.B) for h in range(w.H)]
+    if units_per_round is None:
+        units_per_round = len(all_units)
+    lens = p["lens"]
+    bytes_done, t_spent, rounds, pos = 0, 0.0, 0, 0
+    while t_spent < max_seconds or rounds == 0:
+        units = [all_units[(pos + i) % len(all_units)] for i in range(units_per_round)]
+        pos += units_per_round
+        t0 = time.perf_counter()
+        oracle.decode_layer("absorb", q, cK, cV, p["starts"], lens, WK, mK, WV, mV, 0, 1.0,
+                            units=units, threads=threads)
+        t_spent += time.perf_counter() - t0
+        bytes_done += sum(int(lens[b]) for b, _ in units) * (w.r_k + w.r_v) * w.elem_bytes
+        rounds += 1
+    info = {"cores": threads, "units": units_per_round, "rounds": rounds, "seconds": t_spent}
+    return bytes_done / t_spent / 1e9, info
+
+
+def run_reference(args, rank):
+    """--impl reference: the oracle, as it stands, on the host cores (rank 0 only)."""
+    if rank != 0:
+        return
+    import torch
+    import lla_synth as S
+    w = S.WORKLOADS[args.workload]
+    p = S.decode_inputs(w, 0, "cpu")
+    units = max(1, (w.B * w.H) // 16)          # each step: 1/16 of the layer's (b, h) units
+    tot_units = w.B * w.H
+    for _ in range(args.warmup):
+        oracle_sample_rate(p, w, w.T, 0.0, units_per_round=units)
+    t0 = time.perf_counter()
+    rates = []
+    for _ in range(args.steps):
+        r, info = oracle_sample_rate(p, w, w.T, 0.0, units_per_round=units)
+        rates.append(r)
+    dt = time.perf_counter() - t0
+    value = statistics.median(rates)
+    S_tot = int(p["lens"].sum())
+    step_bytes = S_tot * w.H * (w.r_k + w.r_v) * w.elem_bytes
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "GB/s",
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": 1e3 * dt / max(1, args.steps), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": w.name, "T": w.T, "H": w.H, "d": w.d, "r_k": w.r_k, "r_v": w.r_v,
+                   "B": w.B, "ctx_len": [w.len_lo, w.len_hi], "Tq": w.T,
+                   "sample": f"{units} of {tot_units} (sequence, head) units per step"},
+        "token_loop_reads_per_s": value * 1e9 / (step_bytes / (S_tot * w.T)),
+        "cpu_baseline": {"value": value, "unit": "GB/s", "cores": info["cores"], "kind": "oracle",
+                         "sample": f"{units} (sequence, head) units x 4 loop queries per step"},
+        "e2e": {"value": value, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+# ---------------------------------------------------------------------------
+# our arm
+# ---------------------------------------------------------------------------
+def main():
+    args = parse()
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        run_reference(args, rank)
+        return
+
+    import torch
+    import torch.distributed as dist
+
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+
+    import decode_attention_12_b200 as lla
+    import lla_synth as S
+
+    w = S.WORKLOADS[args.workload]
+    Tq = w.T
+    p = S.decode_inputs(w, 0, dev, gap=1)          # one free slot per sequence for the new token
+    dims = lla.make_dims(w.T, w.L, w.H, w.d, w.r_k, w.r_v, int(w.fold2d),
+                         lla.F32 if w.dtype == "f32" else lla.BF16)
+    B, H = w.B, w.H
+    lens = p["lens"]
+    max_ctx = int(lens.max())
+    S_tot = int(lens.sum())
+    p["bias_k"] = torch.zeros(w.L, w.heads_stored, w.r_k, device=dev)
+    p["bias_v"] = torch.zeros(w.L, w.heads_stored, w.r_v, device=dev)
+    codec = lla.make_codec(W_down_k=p["W_down_k"], W_down_v=p["W_down_v"], bias_k=p["bias_k"],
+                           bias_v=p["bias_v"], W_up_k=p["W_up_k"], W_up_v=p["W_up_v"],
+                           mu_k=p["mu_k"], mu_v=p["mu_v"])
+    lla.codec_bias(dims, codec, p["bias_k"], p["bias_v"])
+    # independent cache replicas (rotated per step so that no step finds latents in L2)
+    R = max(1, args.replicas)
+    reps = [(p["k"], p["v"])] + [(p["k"].clone(), p["v"].clone()) for _ in range(R - 1)]
+    caches = [lla.make_cache(k, v, p["slots"]) for k, v in reps]
+    x_k = S.draw_encode_tokens(w, 0, "k", B, dev, seed_tag="new")
+    x_v = S.draw_encode_tokens(w, 0, "v", B, dev, seed_tag="new")
+    new_slot = (p["seq_start"] + p["ctx_lens"].to(torch.int64)).contiguous()
+    ws_bytes = lla.decode_workspace_bytes(dims, B, Tq, max_ctx, lla.ABSORB, args.num_splits)
+    ws = torch.zeros(ws_bytes, dtype=torch.uint8, device=dev)
+    q = p["q"]
+    out = torch.empty(B, Tq, H, w.d, dtype=torch.float32, device=dev)
+    lse = torch.empty(B, Tq, H, dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    splits = lla.decode_num_splits(dims, B, Tq, max_ctx, lla.ABSORB, args.num_splits)
+
+    def decode(i, q_in=q, out_buf=out):
+        lla.decode_attn(dims, 0, 0, Tq, q_in, caches[i % R], p["seq_start"], p["ctx_lens"], B,
+                        max_ctx, codec, 1.0, out_buf, lse, ws, ws_bytes, num_splits=args.num_splits,
+                        stream=stream)
+
+    def encode(i, xk=x_k, xv=x_v):
+        lla.encode(dims, 0, 1, xk, xv, B, new_slot, codec, caches[i % R], stream=stream)
+
+    launches_per_step = 3                       # decode + combine + encode kernels
+    # ---- warm-up, then the device-timed region ------------------------------------------------
+    sampler = ClockSampler(local).start()
+    for i in range(args.warmup):
+        decode(i)
+        encode(i)
+    torch.cuda.synchronize()
+    ev_a = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    ev_b = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    t_start = torch.cuda.Event(enable_timing=True)
+    t_end = torch.cuda.Event(enable_timing=True)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    wall0 = time.perf_counter()
+    t_start.record(stream)
+    for i in range(args.steps):
+        ev_a[i].record(stream)
+        decode(i)
+        ev_b[i].record(stream)
+        encode(i)
+    t_end.record(stream)
+    torch.cuda.synchronize()
+    wall1 = time.perf_counter()
+    if world > 1:
+        dist.barrier()
+    sampler.stop()
+    ms_total = t_start.elapsed_time(t_end)
+    decode_ms = [a.elapsed_time(b) for a, b in zip(ev_a, ev_b)]
+    if world > 1:
+        t = torch.tensor([ms_total], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms_total = float(t.item())
+    status = lla.status_fetch(ws)
+    if status != 0:
+        raise RuntimeError(f"device status {status}: {lla.status_string(status)}")
+
+    step_bytes = S_tot * w.heads_stored * (w.r_k + w.r_v) * w.elem_bytes   # latents read per step
+    ms_step = ms_total / args.steps
+    value = world * step_bytes / (ms_step * 1e-3) / 1e9
+    reads = world * S_tot * Tq / (ms_step * 1e-3)       # (token, layer, loop) reads per second
+    peaks, peak_kind = measured_peaks()
+    peak = float(peaks["hbm_gbs"])
+    mean_dec_ms = float(np.mean(decode_ms))
+    achieved = step_bytes / (mean_dec_ms * 1e-3) / 1e9
+
+    # ---- end to end through the public API with host buffers -------------------------------------
+    q_h = torch.empty_like(q, device="cpu").pin_memory()
+    q_h.copy_(q)
+    xk_h = torch.empty_like(x_k, device="cpu").pin_memory()
+    xk_h.copy_(x_k)
+    xv_h = torch.empty_like(x_v, device="cpu").pin_memory()
+    xv_h.copy_(x_v)
+    out_h = torch.empty_like(out, device="cpu").pin_memory()
+    lse_h = torch.empty_like(lse, device="cpu").pin_memory()
+    q_d, xk_d, xv_d = torch.empty_like(q), torch.empty_like(x_k), torch.empty_like(x_v)
+    e2e_steps = max(1, min(args.steps, 1000))
+
+    def e2e_step(i):
+        q_d.copy_(q_h, non_blocking=True)
+        xk_d.copy_(xk_h, non_blocking=True)
+        xv_d.copy_(xv_h, non_blocking=True)
+        decode(i, q_in=q_d)
+        encode(i, xk=xk_d, xv=xv_d)
+        out_h.copy_(out, non_blocking=True)
+        lse_h.copy_(lse, non_blocking=True)
+
+    for i in range(min(args.warmup, 10)):
+        e2e_step(i)
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for i in range(e2e_steps):
+        e2e_step(i)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = e0.elapsed_time(e1)
+    if world > 1:
+        t = torch.tensor([e2e_ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e_ms = float(t.item())
+    e2e_value = world * step_bytes * e2e_steps / (e2e_ms * 1e-3) / 1e9
+    h2d = (q.numel() * q.element_size() + x_k.numel() * x_k.element_size() * 2)
+    d2h = out.numel() * out.element_size() + lse.numel() * lse.element_size()
+
+    if rank != 0:
+        if world > 1:
+            dist.destroy_process_group()
+        return
+
+    cpu = None
+    if world == 1 and not args.no_cpu_baseline:
+        rate, info = oracle_sample_rate(p, w, Tq, args.cpu_seconds, units_per_round=max(1, B * H // 8))
+        cpu = {"value": rate, "unit": "GB/s", "cores": info["cores"], "kind": "oracle",
+               "sample": f"{info['rounds']} rounds of {info['units']} (sequence, head) units x "
+                         f"{Tq} loop queries of this workload, {info['seconds']:.1f} s"}
+
+    units_per_launch = S_tot * w.heads_stored
+    clocks = sampler.summary(wall0, wall1)
+    line = {
+        "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "f32", "storage_dtype": w.dtype, "data": "synthetic",
+        "config": {"workload": w.name, "T": w.T, "L_per_step": 1, "H": H, "d": w.d,
+                   "r_k": w.r_k, "r_v": w.r_v, "rho": "64/3", "B": B,
+                   "ctx_len": [w.len_lo, w.len_hi], "tokens": S_tot, "Tq": Tq,
+                   "variant": "absorb", "num_splits": splits,
+                   "step": "decode_attn(all 4 loop queries) + encode(B new tokens)",
+                   "l2": f"inputs larger than L2 ({step_bytes / 1e6:.0f} MB of latents per step) "
+                         f"and {R} rotating cache replicas",
+                   "parallelism": f"replicas x{world}"},
+        "token_loop_reads_per_s": reads,
+        "hbm_frac_of_8tbs_spec": value / world / SPEC_HBM_GBS,
+        "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+                     "frac": achieved / peak, "peak_kind": peak_kind,
+                     "traffic": profiled_traffic(units_per_launch),
+                     "timed": "lla_decode_attn (decode + combine kernels), CUDA events per call",
+                     "algorithmic_bytes_per_launch": step_bytes},
+        "cpu_baseline": cpu,
+        "e2e": {"value": e2e_value, "unit": "GB/s", "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h, "steps": e2e_steps},
+        "gpu_launches": launches_per_step * args.steps,
+        "clocks": clocks,
+    }
+    print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,189 @@
+"""Python binding of liblla -- Looped Latent Attention decode/encode on B200 (sm_100a).
+
+Argument marshalling only: every step of the path runs in the CUDA kernels of
+``liblla.so`` behind the C ABI declared in ``include/lla.h``.  Tensors are
+passed as raw device pointers (``tensor.data_ptr()``) together with the current
+torch CUDA stream; torch is used for device memory and streams, nothing else.
+There is no CPU path: importing this package fails loudly when the compiled
+library is missing.
+
+Names follow the C ABI: ``cache_bytes``, ``slot_layout``, ``codec_bias``,
+``encode``, ``decode_attn``, ``decode_workspace_bytes``, ``decode_num_splits``,
+``status_fetch``, ``status_string``.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional, Sequence
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "liblla.so")
+
+if not os.path.exists(LIB_PATH):
+    raise ImportError(
+        f"{LIB_PATH} is missing: build the CUDA library first "
+        "(python -m decode_attention_12_b200._build, or __graft_entry__.build())")
+
+_lib = ctypes.CDLL(LIB_PATH)
+
+LLA_OK = 0
+LLA_ERR_INVALID = -1
+LLA_ERR_UNSUPPORTED = -2
+LLA_ERR_MISALIGNED = -3
+LLA_ERR_WORKSPACE = -4
+LLA_ERR_CUDA = -5
+LLA_ERR_DEVICE_TIMEOUT = -6
+PER_HEAD, FOLD_2D = 0, 1
+F32, BF16 = 0, 1
+ABSORB, RECONSTRUCT = 0, 1
+
+EXPORTED = ("lla_cache_bytes", "lla_slot_layout", "lla_codec_bias", "lla_encode",
+            "lla_decode_attn", "lla_decode_workspace_bytes", "lla_decode_num_splits",
+            "lla_status_fetch", "lla_status_string")
+
+
+class Dims(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_int32) for n in ("T", "L", "H", "d_head", "r_k", "r_v", "fold", "dtype",
+                                              "out_dtype")]
+
+
+class Codec(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_void_p) for n in ("W_down_k", "W_down_v", "bias_k", "bias_v",
+                                               "W_up_k", "W_up_v", "mu_k", "mu_v")]
+
+
+class Cache(ctypes.Structure):
+    _fields_ = [("k", ctypes.c_void_p), ("v", ctypes.c_void_p), ("slots", ctypes.c_int64)]
+
+
+_i32, _i64, _u64p = ctypes.c_int32, ctypes.c_int64, ctypes.POINTER(ctypes.c_uint64)
+_vp, _sz = ctypes.c_void_p, ctypes.c_size_t
+_P = ctypes.POINTER
+_lib.lla_cache_bytes.argtypes = [_P(Dims), _P(_i32), _i32, _u64p, _u64p, _u64p, _u64p]
+_lib.lla_slot_layout.argtypes = [_P(_i32), _i32, _i64, _P(_i64), _P(_i64)]
+_lib.lla_codec_bias.argtypes = [_P(Dims), _P(Codec), _vp, _vp, _vp]
+_lib.lla_encode.argtypes = [_P(Dims), _i32, _i32, _vp, _vp, _i64, _vp, _P(Codec), _P(Cache), _vp]
+_lib.lla_decode_attn.argtypes = [_P(Dims), _i32, _i32, _i32, _vp, _P(Cache), _vp, _vp, _i32, _i32,
+                                 _P(Codec), ctypes.c_float, _i32, _i32, _vp, _vp, _vp, _sz, _vp]
+_lib.lla_decode_workspace_bytes.argtypes = [_P(Dims), _i32, _i32, _i32, _i32, _i32]
+_lib.lla_decode_workspace_bytes.restype = _sz
+_lib.lla_decode_num_splits.argtypes = [_P(Dims), _i32, _i32, _i32, _i32, _i32]
+_lib.lla_status_fetch.argtypes = [_vp, _vp, _P(_i32)]
+_lib.lla_status_string.argtypes = [ctypes.c_int]
+_lib.lla_status_string.restype = ctypes.c_char_p
+for _n in ("lla_cache_bytes", "lla_slot_layout", "lla_codec_bias", "lla_encode", "lla_decode_attn",
+           "lla_decode_num_splits", "lla_status_fetch"):
+    getattr(_lib, _n).restype = ctypes.c_int
+
+
+class LLAError(RuntimeError):
+    def __init__(self, code: int, where: str):
+        super().__init__(f"{where}: {status_string(code)} ({code})")
+        self.code = code
+
+
+def status_string(code: int) -> str:
+    return _lib.lla_status_string(code).decode()
+
+
+def _check(rc: int, where: str) -> int:
+    if rc < 0:
+        raise LLAError(rc, where)
+    return rc
+
+
+def make_dims(T, L, H, d_head, r_k, r_v, fold=PER_HEAD, dtype=BF16, out_dtype=F32) -> Dims:
+    return Dims(T, L, H, d_head, r_k, r_v, int(fold), int(dtype), int(out_dtype))
+
+
+def _ptr(t) -> Optional[int]:
+    if t is None:
+        return None
+    if isinstance(t, int):
+        return t
+    return t.data_ptr()
+
+
+def _stream(stream=None) -> Optional[int]:
+    if stream is None:
+        import torch
+        return torch.cuda.current_stream().cuda_stream
+    return stream if isinstance(stream, int) else stream.cuda_stream
+
+
+def make_codec(W_down_k=None, W_down_v=None, bias_k=None, bias_v=None, W_up_k=None, W_up_v=None,
+               mu_k=None, mu_v=None) -> Codec:
+    return Codec(*[_ptr(t) for t in (W_down_k, W_down_v, bias_k, bias_v, W_up_k, W_up_v, mu_k, mu_v)])
+
+
+def make_cache(k, v, slots: int) -> Cache:
+    return Cache(_ptr(k), _ptr(v), int(slots))
+
+
+# ---- a7 -------------------------------------------------------------------------------
+def cache_bytes(dims: Dims, ctx_lens: Sequence[int]):
+    """(latent_bytes, uncompressed_bytes, rho_num, rho_den) -- exact integers."""
+    n = len(ctx_lens)
+    arr = (_i32 * max(n, 1))(*[int(v) for v in ctx_lens])
+    out = [ctypes.c_uint64(0) for _ in range(4)]
+    _check(_lib.lla_cache_bytes(ctypes.byref(dims), arr, n, *[ctypes.byref(o) for o in out]),
+           "lla_cache_bytes")
+    return tuple(int(o.value) for o in out)
+
+
+def slot_layout(ctx_lens: Sequence[int], gap: int = 0):
+    """(seq_start list, total_slots) -- exclusive prefix sum with an optional gap."""
+    n = len(ctx_lens)
+    arr = (_i32 * max(n, 1))(*[int(v) for v in ctx_lens])
+    starts = (_i64 * max(n, 1))()
+    total = _i64(0)
+    _check(_lib.lla_slot_layout(arr, n, int(gap), starts, ctypes.byref(total)), "lla_slot_layout")
+    return [int(starts[i]) for i in range(n)], int(total.value)
+
+
+# ---- a6 -------------------------------------------------------------------------------
+def codec_bias(dims: Dims, codec: Codec, bias_k, bias_v, stream=None) -> None:
+    _check(_lib.lla_codec_bias(ctypes.byref(dims), ctypes.byref(codec), _ptr(bias_k), _ptr(bias_v),
+                               _stream(stream)), "lla_codec_bias")
+
+
+def encode(dims: Dims, layer0: int, n_layers: int, x_k, x_v, n_tok: int, slot_idx, codec: Codec,
+           cache: Cache, stream=None) -> None:
+    _check(_lib.lla_encode(ctypes.byref(dims), layer0, n_layers, _ptr(x_k), _ptr(x_v), int(n_tok),
+                           _ptr(slot_idx), ctypes.byref(codec), ctypes.byref(cache), _stream(stream)),
+           "lla_encode")
+
+
+# ---- a1-a5, a8 ------------------------------------------------------------------------------
+def decode_num_splits(dims: Dims, B: int, Tq: int, max_ctx: int, variant: int = ABSORB,
+                      num_splits: int = 0) -> int:
+    return _check(_lib.lla_decode_num_splits(ctypes.byref(dims), B, Tq, max_ctx, variant, num_splits),
+                  "lla_decode_num_splits")
+
+
+def decode_workspace_bytes(dims: Dims, B: int, Tq: int, max_ctx: int, variant: int = ABSORB,
+                           num_splits: int = 0) -> int:
+    n = _lib.lla_decode_workspace_bytes(ctypes.byref(dims), B, Tq, max_ctx, variant, num_splits)
+    if n == 0:
+        raise LLAError(LLA_ERR_INVALID, "lla_decode_workspace_bytes")
+    return int(n)
+
+
+def decode_attn(dims: Dims, layer: int, t0: int, Tq: int, q, cache: Cache, seq_start, ctx_lens,
+                B: int, max_ctx: int, codec: Codec, softmax_scale: float, out, lse=None,
+                workspace=None, ws_bytes: Optional[int] = None, variant: int = ABSORB,
+                num_splits: int = 0, stream=None) -> None:
+    if ws_bytes is None:
+        ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
+    _check(_lib.lla_decode_attn(ctypes.byref(dims), layer, t0, Tq, _ptr(q), ctypes.byref(cache),
+                                _ptr(seq_start), _ptr(ctx_lens), B, max_ctx, ctypes.byref(codec),
+                                float(softmax_scale), variant, num_splits, _ptr(out), _ptr(lse),
+                                _ptr(workspace), int(ws_bytes), _stream(stream)),
+           "lla_decode_attn")
+
+
+def status_fetch(workspace, stream=None) -> int:
+    v = _i32(0)
+    _check(_lib.lla_status_fetch(_ptr(workspace), _stream(stream), ctypes.byref(v)), "lla_status_fetch")
+    return int(v.value)

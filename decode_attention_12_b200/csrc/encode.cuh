@@ -1,0 +1,22 @@
+// encode.cuh -- shared declarations of the LLA write-path kernels.
+#pragma once
+
+#include "common.cuh"
+
+namespace lla {
+
+struct EncodeArgs {
+    const void *x_k, *x_v;         // T [n_layers][n_tok][T][H][d]
+    const void *W_down_k, *W_down_v; // T [L][H'][r][W]
+    const float *bias_k, *bias_v;  // [L][H'][r]
+    void *cache_k, *cache_v;       // T [L][H'][slots][r]
+    const int64_t *slot_idx;       // [n_tok]
+    int64_t n_tok, slots;
+    int32_t layer0, n_layers, T, H, d, Hs, W, r_k, r_v, fold;
+};
+
+cudaError_t launch_encode_simt(const EncodeArgs &a, int dtype, cudaStream_t stream);
+cudaError_t launch_codec_bias(const void *Wd, const float *mu, float *bias, int64_t groups, int r, int W,
+                              int dtype, cudaStream_t stream);
+
+} // namespace lla

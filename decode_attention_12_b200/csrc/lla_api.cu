@@ -1,0 +1,324 @@
+// lla_api.cu -- the C ABI of liblla (declared in include/lla.h): argument checks,
+// kernel selection, workspace carving, status handling.  Every arithmetic step of
+// the path runs in the kernels; this file only validates and launches.
+#include <climits>
+#include <cstring>
+
+#include "decode.cuh"
+#include "encode.cuh"
+
+using namespace lla;
+
+namespace {
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+int elem_bytes(int dtype) { return dtype == LLA_BF16 ? 2 : 4; }
+
+// Basic validity of the problem description.
+int check_dims(const lla_dims *d)
+{
+    if (d == nullptr)
+        return LLA_ERR_INVALID;
+    if (d->T <= 0 || d->L <= 0 || d->H <= 0 || d->d_head <= 0 || d->r_k <= 0 || d->r_v <= 0)
+        return LLA_ERR_INVALID;
+    if (d->fold != LLA_PER_HEAD && d->fold != LLA_FOLD_2D)
+        return LLA_ERR_INVALID;
+    if (d->dtype != LLA_F32 && d->dtype != LLA_BF16)
+        return LLA_ERR_INVALID;
+    if (d->out_dtype != LLA_F32 && d->out_dtype != LLA_BF16)
+        return LLA_ERR_INVALID;
+    const int64_t W = (int64_t)d->T * d->d_head * (d->fold ? d->H : 1);
+    if (W > INT32_MAX / 2 || d->r_k > W || d->r_v > W)
+        return LLA_ERR_INVALID;
+    // every latent row and every W_down row must be a whole number of 16-byte chunks
+    const int e = elem_bytes(d->dtype);
+    if ((d->r_k * e) % 16 != 0 || (d->r_v * e) % 16 != 0 || (W * e) % 16 != 0)
+        return LLA_ERR_UNSUPPORTED;
+    return LLA_OK;
+}
+
+int heads_stored(const lla_dims *d) { return d->fold ? 1 : d->H; }
+int64_t stack_width(const lla_dims *d) { return (int64_t)d->T * d->d_head * (d->fold ? d->H : 1); }
+int64_t loop_width(const lla_dims *d) { return (int64_t)d->d_head * (d->fold ? d->H : 1); }
+
+int sm_count()
+{
+    static int cached[64] = {0};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64)
+        return 148;
+    if (cached[dev] == 0) {
+        int n = 0;
+        if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
+            n = 148;
+        cached[dev] = n;
+    }
+    return cached[dev];
+}
+
+int choose_splits(const lla_dims *d, int32_t B, int32_t max_ctx, int32_t num_splits)
+{
+    if (num_splits > 0)
+        return num_splits;
+    const int64_t units = (int64_t)B * d->H;
+    if (units <= 0)
+        return 1;
+    const int64_t target = (int64_t)sm_count() * 2 * 4; // ~4 waves at 2 CTAs per SM
+    int64_t s = (target + units - 1) / units;
+    int64_t cap = max_ctx / 1024;
+    if (cap < 1)
+        cap = 1;
+    if (s > cap)
+        s = cap;
+    if (s > 256)
+        s = 256;
+    return (int)(s < 1 ? 1 : s);
+}
+
+size_t part_bytes(const lla_dims *d, int32_t B, int32_t Tq, int splits)
+{
+    return (size_t)B * d->H * Tq * splits * part_stride(d->r_v) * sizeof(float);
+}
+
+} // namespace
+
+extern "C" {
+
+const char *lla_status_string(int code)
+{
+    switch (code) {
+    case LLA_OK: return "ok";
+    case LLA_ERR_INVALID: return "invalid argument";
+    case LLA_ERR_UNSUPPORTED: return "unsupported rank, dtype or shape";
+    case LLA_ERR_MISALIGNED: return "device pointer not 16-byte aligned";
+    case LLA_ERR_WORKSPACE: return "workspace missing or too small";
+    case LLA_ERR_CUDA: return "CUDA launch or copy failed";
+    case LLA_ERR_DEVICE_TIMEOUT: return "a kernel gave up a bounded wait";
+    default: return "unknown status";
+    }
+}
+
+int lla_cache_bytes(const lla_dims *dims, const int32_t *ctx_lens_host, int32_t B,
+                    uint64_t *latent_bytes, uint64_t *uncompressed_bytes, uint64_t *rho_num,
+                    uint64_t *rho_den)
+{
+    if (dims == nullptr || B < 0 || (B > 0 && ctx_lens_host == nullptr))
+        return LLA_ERR_INVALID;
+    if (dims->T <= 0 || dims->L <= 0 || dims->H <= 0 || dims->d_head <= 0 || dims->r_k <= 0 ||
+        dims->r_v <= 0 || (dims->fold != 0 && dims->fold != 1) || (dims->dtype != 0 && dims->dtype != 1))
+        return LLA_ERR_INVALID;
+    unsigned __int128 S = 0;
+    for (int32_t b = 0; b < B; ++b) {
+        if (ctx_lens_host[b] < 0)
+            return LLA_ERR_INVALID;
+        S += (unsigned)ctx_lens_host[b];
+    }
+    const unsigned __int128 e = (unsigned)elem_bytes(dims->dtype);
+    const unsigned __int128 per_unc = (unsigned __int128)2 * dims->T * dims->H * dims->d_head;
+    const unsigned __int128 per_lat = (unsigned __int128)heads_stored(dims) * (dims->r_k + dims->r_v);
+    const unsigned __int128 unc = S * dims->L * per_unc * e;
+    const unsigned __int128 lat = S * dims->L * per_lat * e;
+    if (unc > (unsigned __int128)UINT64_MAX || lat > (unsigned __int128)UINT64_MAX)
+        return LLA_ERR_INVALID;
+    uint64_t a = (uint64_t)per_unc, b = (uint64_t)per_lat;
+    while (b != 0) {
+        const uint64_t t = a % b;
+        a = b;
+        b = t;
+    }
+    if (latent_bytes) *latent_bytes = (uint64_t)lat;
+    if (uncompressed_bytes) *uncompressed_bytes = (uint64_t)unc;
+    if (rho_num) *rho_num = (uint64_t)per_unc / a;
+    if (rho_den) *rho_den = (uint64_t)per_lat / a;
+    return LLA_OK;
+}
+
+int lla_slot_layout(const int32_t *ctx_lens_host, int32_t B, int64_t gap, int64_t *seq_start_host,
+                    int64_t *total_slots)
+{
+    if (B < 0 || gap < 0 || (B > 0 && (ctx_lens_host == nullptr || seq_start_host == nullptr)))
+        return LLA_ERR_INVALID;
+    int64_t pos = 0;
+    for (int32_t b = 0; b < B; ++b) {
+        if (ctx_lens_host[b] < 0)
+            return LLA_ERR_INVALID;
+        seq_start_host[b] = pos;
+        if (pos > INT64_MAX - ctx_lens_host[b] - gap)
+            return LLA_ERR_INVALID;
+        pos += ctx_lens_host[b] + gap;
+    }
+    if (total_slots)
+        *total_slots = pos;
+    return LLA_OK;
+}
+
+int lla_codec_bias(const lla_dims *dims, const lla_codec *codec, float *bias_k_out, float *bias_v_out,
+                   lla_stream_t stream)
+{
+    int rc = check_dims(dims);
+    if (rc != LLA_OK)
+        return rc;
+    if (codec == nullptr || codec->W_down_k == nullptr || codec->W_down_v == nullptr ||
+        codec->mu_k == nullptr || codec->mu_v == nullptr || bias_k_out == nullptr || bias_v_out == nullptr)
+        return LLA_ERR_INVALID;
+    const int64_t groups = (int64_t)dims->L * heads_stored(dims);
+    const int W = (int)stack_width(dims);
+    cudaError_t e = launch_codec_bias(codec->W_down_k, codec->mu_k, bias_k_out, groups, dims->r_k, W,
+                                      dims->dtype, (cudaStream_t)stream);
+    if (e == cudaSuccess)
+        e = launch_codec_bias(codec->W_down_v, codec->mu_v, bias_v_out, groups, dims->r_v, W, dims->dtype,
+                              (cudaStream_t)stream);
+    return e == cudaSuccess ? LLA_OK : LLA_ERR_CUDA;
+}
+
+int lla_encode(const lla_dims *dims, int32_t layer0, int32_t n_layers, const void *x_k, const void *x_v,
+               int64_t n_tok, const int64_t *slot_idx, const lla_codec *codec, const lla_cache *cache,
+               lla_stream_t stream)
+{
+    int rc = check_dims(dims);
+    if (rc != LLA_OK)
+        return rc;
+    if (layer0 < 0 || n_layers < 0 || layer0 + (int64_t)n_layers > dims->L || n_tok < 0)
+        return LLA_ERR_INVALID;
+    if (n_tok == 0 || n_layers == 0)
+        return LLA_OK;
+    if (x_k == nullptr || x_v == nullptr || slot_idx == nullptr || codec == nullptr || cache == nullptr ||
+        codec->W_down_k == nullptr || codec->W_down_v == nullptr || codec->bias_k == nullptr ||
+        codec->bias_v == nullptr || cache->k == nullptr || cache->v == nullptr || cache->slots < 0)
+        return LLA_ERR_INVALID;
+    if (!aligned16(x_k) || !aligned16(x_v) || !aligned16(slot_idx) || !aligned16(codec->W_down_k) ||
+        !aligned16(codec->W_down_v) || !aligned16(codec->bias_k) || !aligned16(codec->bias_v) ||
+        !aligned16(cache->k) || !aligned16(cache->v))
+        return LLA_ERR_MISALIGNED;
+    if (dims->r_k > 256 || dims->r_v > 256)
+        return LLA_ERR_UNSUPPORTED;
+    EncodeArgs a;
+    a.x_k = x_k; a.x_v = x_v;
+    a.W_down_k = codec->W_down_k; a.W_down_v = codec->W_down_v;
+    a.bias_k = codec->bias_k; a.bias_v = codec->bias_v;
+    a.cache_k = cache->k; a.cache_v = cache->v;
+    a.slot_idx = slot_idx;
+    a.n_tok = n_tok; a.slots = cache->slots;
+    a.layer0 = layer0; a.n_layers = n_layers;
+    a.T = dims->T; a.H = dims->H; a.d = dims->d_head; a.Hs = heads_stored(dims);
+    a.W = (int32_t)stack_width(dims);
+    a.r_k = dims->r_k; a.r_v = dims->r_v; a.fold = dims->fold;
+    cudaError_t e = launch_encode_simt(a, dims->dtype, (cudaStream_t)stream);
+    return e == cudaSuccess ? LLA_OK : LLA_ERR_CUDA;
+}
+
+int lla_decode_num_splits(const lla_dims *dims, int32_t B, int32_t Tq, int32_t max_ctx, int32_t variant,
+                          int32_t num_splits)
+{
+    int rc = check_dims(dims);
+    if (rc != LLA_OK)
+        return rc;
+    if (B < 0 || Tq < 1 || max_ctx < 0 || num_splits < 0 ||
+        (variant != LLA_ABSORB && variant != LLA_RECONSTRUCT))
+        return LLA_ERR_INVALID;
+    return choose_splits(dims, B, max_ctx, num_splits);
+}
+
+size_t lla_decode_workspace_bytes(const lla_dims *dims, int32_t B, int32_t Tq, int32_t max_ctx,
+                                  int32_t variant, int32_t num_splits)
+{
+    const int s = lla_decode_num_splits(dims, B, Tq, max_ctx, variant, num_splits);
+    if (s < 1)
+        return 0;
+    return kWorkspaceHeader + part_bytes(dims, B, Tq, s);
+}
+
+int lla_decode_attn(const lla_dims *dims, int32_t layer, int32_t t0, int32_t Tq, const void *q,
+                    const lla_cache *cache, const int64_t *seq_start, const int32_t *ctx_lens, int32_t B,
+                    int32_t max_ctx, const lla_codec *codec, float softmax_scale, int32_t variant,
+                    int32_t num_splits, void *out, float *lse, void *workspace, size_t ws_bytes,
+                    lla_stream_t stream)
+{
+    int rc = check_dims(dims);
+    if (rc != LLA_OK)
+        return rc;
+    if (layer < 0 || layer >= dims->L || t0 < 0 || Tq < 1 || t0 + (int64_t)Tq > dims->T || B < 0 ||
+        max_ctx < 0 || num_splits < 0 || (variant != LLA_ABSORB && variant != LLA_RECONSTRUCT))
+        return LLA_ERR_INVALID;
+    if (B == 0)
+        return LLA_OK;
+    if (q == nullptr || cache == nullptr || cache->k == nullptr || cache->v == nullptr || cache->slots < 0 ||
+        seq_start == nullptr || ctx_lens == nullptr || codec == nullptr || codec->W_up_k == nullptr ||
+        codec->W_up_v == nullptr || codec->mu_k == nullptr || codec->mu_v == nullptr || out == nullptr)
+        return LLA_ERR_INVALID;
+    if (!aligned16(q) || !aligned16(cache->k) || !aligned16(cache->v) || !aligned16(out) ||
+        !aligned16(codec->W_up_k) || !aligned16(codec->W_up_v) || !aligned16(codec->mu_k) ||
+        !aligned16(codec->mu_v) || !aligned16(seq_start) || !aligned16(ctx_lens) ||
+        (lse != nullptr && !aligned16(lse)))
+        return LLA_ERR_MISALIGNED;
+    const int splits = choose_splits(dims, B, max_ctx, num_splits);
+    const size_t need = kWorkspaceHeader + part_bytes(dims, B, Tq, splits);
+    if (workspace == nullptr || ws_bytes < need)
+        return LLA_ERR_WORKSPACE;
+    if (!aligned16(workspace))
+        return LLA_ERR_MISALIGNED;
+    if (variant != LLA_ABSORB)
+        return LLA_ERR_UNSUPPORTED;
+    if (!decode_absorb_simt_supported(dims->dtype, dims->r_k, dims->r_v, dims->d_head, dims->fold))
+        return LLA_ERR_UNSUPPORTED;
+
+    const int Hs = heads_stored(dims);
+    const int64_t Dp = loop_width(dims);
+    const int e = elem_bytes(dims->dtype);
+    DecodeArgs a;
+    a.q = q;
+    a.k = static_cast<const uint8_t *>(cache->k) + (int64_t)layer * Hs * cache->slots * dims->r_k * e;
+    a.v = static_cast<const uint8_t *>(cache->v) + (int64_t)layer * Hs * cache->slots * dims->r_v * e;
+    a.slots = cache->slots;
+    a.seq_start = seq_start;
+    a.ctx_lens = ctx_lens;
+    a.W_up_k = codec->W_up_k + (int64_t)layer * Hs * dims->T * dims->r_k * Dp;
+    a.W_up_v = codec->W_up_v + (int64_t)layer * Hs * dims->T * dims->r_v * Dp;
+    a.mu_k = codec->mu_k + (int64_t)layer * Hs * dims->T * Dp;
+    a.mu_v = codec->mu_v + (int64_t)layer * Hs * dims->T * Dp;
+    a.B = B; a.H = dims->H; a.d = dims->d_head; a.T = dims->T; a.t0 = t0; a.Tq = Tq;
+    a.fold = dims->fold; a.r_k = dims->r_k; a.r_v = dims->r_v;
+    a.num_splits = splits;
+    a.scale = softmax_scale;
+    a.status = static_cast<int32_t *>(workspace);
+    a.part = reinterpret_cast<float *>(static_cast<uint8_t *>(workspace) + kWorkspaceHeader);
+    a.out = out;
+    a.lse = lse;
+
+    a.Tq_all = Tq;
+    a.tq_off = 0;
+    cudaStream_t s = (cudaStream_t)stream;
+    // The SIMT kernel serves up to 4 loop queries per pass over the latents.
+    cudaError_t err = cudaSuccess;
+    for (int32_t c = 0; c < Tq && err == cudaSuccess; c += 4) {
+        DecodeArgs ac = a;
+        ac.tq_off = c;
+        ac.Tq = Tq - c < 4 ? Tq - c : 4;
+        bool supported = false;
+        err = launch_decode_absorb_simt(ac, dims->dtype, s, &supported);
+        if (!supported)
+            return LLA_ERR_UNSUPPORTED;
+        if (err == cudaSuccess)
+            err = launch_decode_combine(ac, dims->dtype, dims->out_dtype, s);
+    }
+    return err == cudaSuccess ? LLA_OK : LLA_ERR_CUDA;
+}
+
+int lla_status_fetch(void *workspace, lla_stream_t stream, int32_t *status_host)
+{
+    if (workspace == nullptr || status_host == nullptr)
+        return LLA_ERR_INVALID;
+    cudaStream_t s = (cudaStream_t)stream;
+    int32_t v = 0;
+    if (cudaMemcpyAsync(&v, workspace, sizeof(int32_t), cudaMemcpyDeviceToHost, s) != cudaSuccess)
+        return LLA_ERR_CUDA;
+    if (cudaStreamSynchronize(s) != cudaSuccess)
+        return LLA_ERR_CUDA;
+    if (cudaMemsetAsync(workspace, 0, sizeof(int32_t), s) != cudaSuccess)
+        return LLA_ERR_CUDA;
+    *status_host = v;
+    return LLA_OK;
+}
+
+} // extern "C"

@@ -1,0 +1,181 @@
+/*
+ * lla.h -- C ABI of liblla: Looped Latent Attention (LLA) decode attention over a
+ * cross-loop latent KV cache, and its write path, on NVIDIA B200 (sm_100a).
+ *
+ * The method ("Looped Latent Attention: Cross-Loop KV Compression for Looped
+ * Transformers", Pith review page, "What carries the argument", Eqs. 2-4):
+ * a looped, weight-tied model runs its L-layer block T times per token and each
+ * loop t yields a key and a value per head (Figure 1).  Instead of T (K_t, V_t)
+ * pairs, the cache keeps, per (token, layer, head) and per axis K / V, one centred
+ * latent  c = (x - mu) W_down  of rank r_k (keys) or r_v (values), where
+ * x = [x_1 .. x_T] stacks the token's T per-loop vectors.  Loop t reads
+ *   x_hat_t = c W_up,t + mu_t                                          (Eq. 3)
+ * either literally (RECONSTRUCT) or through query-side absorption (ABSORB: the
+ * "absorbed-attention variant" of the Pith verdict record's desk-editor letter),
+ * which gives the same attention output when no rotation sits between the
+ * reconstruction and the dot product.  LLA-2D (arXiv abstract) folds the H heads
+ * into one latent per (token, layer): x stacks [T][H][d] and head h reads columns
+ * h*d .. h*d+d-1 of W_up,t and mu_t.  The compression is exact (Eq. 4):
+ *   rho = 2 T d_head / (r_k + r_v) per head per layer  (LLA-2D: 2 T H d / (r_k + r_v)).
+ *
+ * General conventions
+ *  - Every pointer is caller-owned; the library allocates nothing and keeps no
+ *    state between calls.  Pointers named *_host are host memory; all others are
+ *    device memory of the current CUDA device.
+ *  - Device work is enqueued on `stream`, asynchronously; no call synchronises
+ *    the host except lla_status_fetch.  No exception crosses the ABI.
+ *  - Arrays are dense and row-major in the index order written next to them.
+ *    Storage type "T" is the `dtype` of lla_dims (fp32 or bf16); codec tensors
+ *    other than W_down are always fp32.  bf16 values are rounded to nearest-even.
+ *  - Return value: LLA_OK or one of the negative LLA_ERR_* codes below; on an
+ *    error nothing has been enqueued.  Device pointers must be 16-byte aligned.
+ */
+#ifndef LLA_H_
+#define LLA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st *lla_stream_t; /* same type as cudaStream_t; NULL = legacy stream */
+
+/* ---- status codes ---------------------------------------------------------------- */
+#define LLA_OK 0
+#define LLA_ERR_INVALID (-1)     /* bad dimension, loop range, null pointer, ...       */
+#define LLA_ERR_UNSUPPORTED (-2) /* no kernel instantiated for this rank/dtype/shape     */
+#define LLA_ERR_MISALIGNED (-3)  /* a device pointer is not 16-byte aligned              */
+#define LLA_ERR_WORKSPACE (-4)   /* workspace missing or smaller than required           */
+#define LLA_ERR_CUDA (-5)        /* a CUDA launch or copy failed                         */
+#define LLA_ERR_DEVICE_TIMEOUT (-6) /* a kernel gave up a bounded wait (reported via the
+                                       workspace status word, see lla_status_fetch)      */
+
+/* ---- problem description ---------------------------------------------------------- */
+enum { LLA_PER_HEAD = 0, LLA_FOLD_2D = 1 };       /* lla_dims.fold                    */
+enum { LLA_F32 = 0, LLA_BF16 = 1 };               /* lla_dims.dtype                   */
+enum { LLA_ABSORB = 0, LLA_RECONSTRUCT = 1 };     /* decode read variant              */
+
+typedef struct {
+    int32_t T;      /* loops (recurrence steps) of the weight-tied block                   */
+    int32_t L;      /* layers of the block                                                 */
+    int32_t H;      /* attention heads                                                     */
+    int32_t d_head; /* head dimension d                                                    */
+    int32_t r_k;    /* key latent rank                                                     */
+    int32_t r_v;    /* value latent rank                                                   */
+    int32_t fold;   /* LLA_PER_HEAD or LLA_FOLD_2D                                         */
+    int32_t dtype;  /* storage type T of tokens, queries, latents and W_down                */
+    int32_t out_dtype; /* storage type O of decode outputs (LLA_F32 or LLA_BF16).  With bf16
+                          outputs the rounding of |out| >= 4 alone exceeds 1e-2; fp32 output
+                          keeps the attention result at full accumulation precision.        */
+} lla_dims;
+/* H' below = H (per-head) or 1 (LLA-2D); W = T*d (per-head) or T*H*d (LLA-2D);
+ * D' = d (per-head) or H*d (LLA-2D) is the width of one loop block of the stack.  */
+
+typedef struct {
+    const void *W_down_k;  /* T     [L][H'][r_k][W]  W_down^K stored transposed        */
+    const void *W_down_v;  /* T     [L][H'][r_v][W]                                    */
+    const float *bias_k;   /* fp32  [L][H'][r_k]  = -mu^K W_down^K (lla_codec_bias)     */
+    const float *bias_v;   /* fp32  [L][H'][r_v]                                        */
+    const float *W_up_k;   /* fp32  [L][H'][T][r_k][D']  per-loop up-projections W_up,t */
+    const float *W_up_v;   /* fp32  [L][H'][T][r_v][D']                                 */
+    const float *mu_k;     /* fp32  [L][H'][T][D']  = mu^K, loop-major ([L][H'][W])     */
+    const float *mu_v;     /* fp32  [L][H'][T][D']                                      */
+} lla_codec;
+
+typedef struct {
+    void *k;       /* T [L][H'][slots][r_k]  key latents c_K                             */
+    void *v;       /* T [L][H'][slots][r_v]  value latents c_V                           */
+    int64_t slots; /* slot capacity of one (layer, head) plane                          */
+} lla_cache;
+/* A sequence b owns the contiguous slots seq_start[b] .. seq_start[b]+len_b-1 of every
+ * plane, so each (sequence, layer, head) latent stream is one contiguous run.      */
+
+/* ---- a7: exact cache accounting (host only) ----------------------------------------
+ * Eq. 4 and Figure 10 of the review page.  S = sum of ctx_lens_host[0..B).
+ *   latent_bytes       = S * L * H' * (r_k + r_v) * sizeof(T)
+ *   uncompressed_bytes = S * L * H  * 2 * T * d   * sizeof(T)
+ *   rho = rho_num / rho_den = uncompressed / latent, reduced to lowest terms.
+ * Any output pointer may be NULL.  Errors: LLA_ERR_INVALID (dims <= 0, negative
+ * length, B < 0, overflow of 64-bit byte counts).                                     */
+int lla_cache_bytes(const lla_dims *dims, const int32_t *ctx_lens_host, int32_t B,
+                    uint64_t *latent_bytes, uint64_t *uncompressed_bytes,
+                    uint64_t *rho_num, uint64_t *rho_den);
+
+/* Ragged slot layout (host only): seq_start_host[b] = sum_{i<b} (len_i + gap), and
+ * *total_slots = sum_b (len_b + gap).  Exact 64-bit integer arithmetic.            */
+int lla_slot_layout(const int32_t *ctx_lens_host, int32_t B, int64_t gap,
+                    int64_t *seq_start_host, int64_t *total_slots);
+
+/* ---- a6 set-up: encode bias ---------------------------------------------------------
+ * Eq. 2 written as c = x W_down + b with b = -mu W_down.  Computes b for every
+ * (layer, head', axis) from codec->W_down_{k,v} and codec->mu_{k,v} (fp64
+ * accumulation, fp32 result) into bias_k_out [L][H'][r_k] and bias_v_out
+ * [L][H'][r_v].  Run once per codec; lla_encode reads the result through
+ * codec->bias_{k,v}.                                                                 */
+int lla_codec_bias(const lla_dims *dims, const lla_codec *codec, float *bias_k_out,
+                   float *bias_v_out, lla_stream_t stream);
+
+/* ---- a6: encode (write path) ----------------------------------------------------------
+ * Eq. 2: for layers layer0 .. layer0+n_layers-1, tokens i < n_tok, stored heads h',
+ * and both axes:  cache[l][h'][slot_idx[i]] = x_stack(i, h') W_down[l][h'] + bias[l][h'].
+ *   x_k, x_v  T [n_layers][n_tok][T][H][d]   per-loop K (V) of every head, loop-major;
+ *             per-head rows stack x[i][0..T)[h][0..d); LLA-2D rows are x[i] itself.
+ *   slot_idx  int64 [n_tok] destination slot of each token; a slot outside
+ *             [0, cache->slots) is skipped (nothing is written for that token).
+ * bf16 runs on tcgen05 tensor cores (fp32 accumulation in tensor memory, one
+ * rounding to bf16); fp32 runs on CUDA cores in fp32.  Errors: LLA_ERR_INVALID,
+ * LLA_ERR_UNSUPPORTED (rank not a multiple of 16 for bf16, or > 256),
+ * LLA_ERR_MISALIGNED, LLA_ERR_CUDA.                                                   */
+int lla_encode(const lla_dims *dims, int32_t layer0, int32_t n_layers, const void *x_k,
+               const void *x_v, int64_t n_tok, const int64_t *slot_idx,
+               const lla_codec *codec, const lla_cache *cache, lla_stream_t stream);
+
+/* ---- a1-a5, a8: decode attention ------------------------------------------------------
+ * For layer `layer`, loops t = t0 .. t0+Tq-1, sequences b < B and heads h < H, the
+ * loop-t query q[b][t-t0][h] attends over the ctx_lens[b] cached latents of
+ * sequence b (Figure 1 of the review page; the cache holds only latents):
+ *   k_hat_n = c_K[n] W_up,t^K + mu_t^K,  v_hat_n = c_V[n] W_up,t^V + mu_t^V    (Eq. 3)
+ *   l_n = softmax_scale * q . k_hat_n,  out = sum_n softmax(l)_n v_hat_n,
+ *   lse = log sum_n exp(l_n)  (natural log).
+ * variant LLA_ABSORB evaluates l_n = q_tilde . c_K[n] + softmax_scale * q . mu_t^K with
+ * q_tilde = softmax_scale * q W_up,t^K^T and out = (sum_n p_n c_V[n]) W_up,t^V + mu_t^V;
+ * LLA_RECONSTRUCT rebuilds k_hat, v_hat per tile on tensor cores.
+ *   q        T [B][Tq][H][d]            out  O [B][Tq][H][d]  (O = dims->out_dtype)
+ *   lse      fp32 [B][Tq][H] or NULL    (len_b = 0 gives out = 0 and lse = -inf)
+ *   seq_start int64 [B], ctx_lens int32 [B]   (device; slots must lie in the plane)
+ *   max_ctx  host-side upper bound of ctx_lens, used only to choose the split count
+ *   num_splits  split-K factor per (sequence, head); 0 = automatic
+ *   workspace   device scratch of at least lla_decode_workspace_bytes(...) bytes
+ * Errors: LLA_ERR_INVALID (dims, loop range, Tq < 1, pointers), LLA_ERR_UNSUPPORTED,
+ * LLA_ERR_MISALIGNED, LLA_ERR_WORKSPACE, LLA_ERR_CUDA.                                  */
+int lla_decode_attn(const lla_dims *dims, int32_t layer, int32_t t0, int32_t Tq,
+                    const void *q, const lla_cache *cache, const int64_t *seq_start,
+                    const int32_t *ctx_lens, int32_t B, int32_t max_ctx,
+                    const lla_codec *codec, float softmax_scale, int32_t variant,
+                    int32_t num_splits, void *out, float *lse, void *workspace,
+                    size_t ws_bytes, lla_stream_t stream);
+
+/* Workspace bytes lla_decode_attn needs for these sizes (num_splits as passed to it;
+ * 0 = the automatic choice for max_ctx).  Returns 0 for invalid arguments.          */
+size_t lla_decode_workspace_bytes(const lla_dims *dims, int32_t B, int32_t Tq,
+                                  int32_t max_ctx, int32_t variant, int32_t num_splits);
+
+/* The split count lla_decode_attn uses for these arguments (>= 1), or a negative
+ * LLA_ERR_* code.                                                                     */
+int lla_decode_num_splits(const lla_dims *dims, int32_t B, int32_t Tq, int32_t max_ctx,
+                          int32_t variant, int32_t num_splits);
+
+/* ---- status ---------------------------------------------------------------------------
+ * Kernels never trap.  A kernel that gives up a bounded wait records
+ * LLA_ERR_DEVICE_TIMEOUT in the first word of the decode workspace (sticky).
+ * lla_status_fetch synchronises `stream`, copies that word to *status_host and
+ * clears it.  lla_status_string maps any code to a static message.                   */
+int lla_status_fetch(void *workspace, lla_stream_t stream, int32_t *status_host);
+const char *lla_status_string(int code);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* LLA_H_ */

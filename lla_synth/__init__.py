@@ -317,3 +317,54 @@ def draw_encode_tokens(w: Workload, layer: int, axis: str, n_tok: int, device,
             else:
                 out[a:b, :, hs, :] = x.view(b - a, T, d).to(w.torch_dtype)
     return out
+
+
+# ---------------------------------------------------------------------------
+# Everything one decode call needs, in the library's device layouts
+# ---------------------------------------------------------------------------
+def decode_inputs(w: Workload, layers, device, Tq: Optional[int] = None, lens=None, gap: int = 0,
+                  perturb: float = 0.0, q_tag="q") -> dict:
+    """Draw the latent cache, codec and queries for ``layers`` of workload ``w``.
+
+    Returns device tensors in the library layouts (see include/lla.h):
+      k, v        [L][H'][slots][r]      latents (layers not listed stay zero)
+      W_up_k/v    [L][H'][T][r][D']      fp32;  mu_k/v [L][H'][T][D'] fp32
+      W_down_k/v  [L][H'][r][W]          storage dtype
+      seq_start   int64 [B], ctx_lens int32 [B]
+      q           [B][Tq][H][d]          storage dtype
+    plus host copies ``lens`` / ``starts`` and the fitted ``codecs`` per layer.
+    """
+    if isinstance(layers, int):
+        layers = [layers]
+    Tq = w.T if Tq is None else Tq
+    lens = context_lengths(w) if lens is None else np.asarray(lens, dtype=np.int32)
+    starts = slot_starts(lens, gap)
+    slots = int(starts[-1] + lens[-1] + gap) if len(lens) else 1
+    slots = max(slots, 1)
+    Hs, T, Dp = w.heads_stored, w.T, w.d * (w.H if w.fold2d else 1)
+    dt = w.torch_dtype
+    out = {
+        "k": torch.zeros(w.L, Hs, slots, w.r_k, dtype=dt, device=device),
+        "v": torch.zeros(w.L, Hs, slots, w.r_v, dtype=dt, device=device),
+        "W_up_k": torch.zeros(w.L, Hs, T, w.r_k, Dp, dtype=torch.float32, device=device),
+        "W_up_v": torch.zeros(w.L, Hs, T, w.r_v, Dp, dtype=torch.float32, device=device),
+        "mu_k": torch.zeros(w.L, Hs, T, Dp, dtype=torch.float32, device=device),
+        "mu_v": torch.zeros(w.L, Hs, T, Dp, dtype=torch.float32, device=device),
+        "W_down_k": torch.zeros(w.L, Hs, w.r_k, w.W, dtype=dt, device=device),
+        "W_down_v": torch.zeros(w.L, Hs, w.r_v, w.W, dtype=dt, device=device),
+        "seq_start": torch.as_tensor(starts, dtype=torch.int64, device=device),
+        "ctx_lens": torch.as_tensor(lens, dtype=torch.int32, device=device),
+        "lens": lens, "starts": starts, "slots": slots, "codecs": {},
+    }
+    for layer in layers:
+        codecs = layer_codecs(w, layer, perturb=perturb)
+        out["codecs"][layer] = codecs
+        ct = codec_tensors(w, codecs, device)
+        for name in ("W_up_k", "W_up_v", "mu_k", "mu_v", "W_down_k", "W_down_v"):
+            src = ct[name]
+            if w.fold2d and name.startswith(("W_up", "mu")):
+                src = src.unsqueeze(0)
+            out[name][layer].copy_(src)
+        draw_layer_cache(w, layer, codecs, slots, device, out_k=out["k"][layer], out_v=out["v"][layer])
+    out["q"] = draw_queries(w.B, Tq, w.H, w.d, seed_of(w.name, q_tag, Tq), device, dt)
+    return out

@@ -1,0 +1,90 @@
+"""Helpers for GPU parity tests: run the CUDA path through the C ABI, run the fp64
+oracle on the same inputs, compare with the stated tolerances.
+
+Tolerances (attention output stored in bf16 with fp32 accumulation): max-abs <= 1e-2
+and relative L2 <= 5e-3 against the fp64 oracle; encode latents relative L2 <= 5e-3.
+lse is compared with an absolute bound of 2e-3 (it is computed in fp32 from fp32
+scores; -inf must match exactly for empty contexts).
+"""
+import numpy as np
+import torch
+
+import decode_attention_12_b200 as lla
+import oracle
+
+ATOL_MAX = 1e-2
+RTOL_L2 = 5e-3
+LSE_ATOL = 2e-3
+
+
+def to64(t):
+    return t.detach().to(torch.float32).cpu().double().numpy()
+
+
+def dims_of(w, out_dtype=lla.F32):
+    return lla.make_dims(w.T, w.L, w.H, w.d, w.r_k, w.r_v, int(w.fold2d),
+                         lla.F32 if w.dtype == "f32" else lla.BF16, out_dtype)
+
+
+def codec_of(p):
+    return lla.make_codec(W_down_k=p["W_down_k"], W_down_v=p["W_down_v"], bias_k=p.get("bias_k"),
+                          bias_v=p.get("bias_v"), W_up_k=p["W_up_k"], W_up_v=p["W_up_v"],
+                          mu_k=p["mu_k"], mu_v=p["mu_v"])
+
+
+def run_decode(p, w, layer, t0, Tq, scale, num_splits=0, variant=lla.ABSORB, q=None,
+               out_dtype=lla.F32):
+    """Decode through the C ABI; returns (out, lse, device status)."""
+    dims = dims_of(w, out_dtype)
+    q = p["q"] if q is None else q
+    B = len(p["lens"])
+    max_ctx = int(p["lens"].max()) if B else 0
+    ws_bytes = lla.decode_workspace_bytes(dims, B, Tq, max_ctx, variant, num_splits)
+    ws = torch.zeros(ws_bytes, dtype=torch.uint8, device="cuda")
+    odt = torch.float32 if out_dtype == lla.F32 else torch.bfloat16
+    out = torch.full((B, Tq, w.H, w.d), float("nan"), dtype=odt, device="cuda")
+    lse = torch.full((B, Tq, w.H), float("nan"), dtype=torch.float32, device="cuda")
+    lla.decode_attn(dims, layer, t0, Tq, q, lla.make_cache(p["k"], p["v"], p["slots"]),
+                    p["seq_start"], p["ctx_lens"], B, max_ctx, codec_of(p), scale, out, lse,
+                    ws, ws_bytes, variant=variant, num_splits=num_splits)
+    torch.cuda.synchronize()
+    status = lla.status_fetch(ws)
+    return out, lse, status
+
+
+def oracle_decode(p, w, layer, t0, Tq, scale, units=None, variant="absorb", q=None, threads=None):
+    q = p["q"] if q is None else q
+    q64 = to64(q)
+    cK, cV = to64(p["k"][layer]), to64(p["v"][layer])
+    WK, WV = to64(p["W_up_k"][layer]), to64(p["W_up_v"][layer])
+    mK, mV = to64(p["mu_k"][layer]), to64(p["mu_v"][layer])
+    if w.fold2d:
+        WK, WV, mK, mV = WK[0], WV[0], mK[0], mV[0]
+    return oracle.decode_layer(variant, q64, cK, cV, p["starts"], p["lens"], WK, mK, WV, mV,
+                               t0, scale, fold2d=w.fold2d, units=units, threads=threads)
+
+
+def attn_errors(out_gpu, o_ref):
+    o = to64(out_gpu)
+    mask = ~np.isnan(o_ref)
+    err = o[mask] - o_ref[mask]
+    max_abs = float(np.abs(err).max()) if err.size else 0.0
+    den = float(np.linalg.norm(o_ref[mask]))
+    rel = float(np.linalg.norm(err)) / den if den > 0 else float(np.linalg.norm(err))
+    return max_abs, rel
+
+
+def assert_attn_close(out_gpu, lse_gpu, o_ref, lse_ref):
+    assert not torch.isnan(out_gpu.float()).any(), "NaN in GPU output"
+    max_abs, rel = attn_errors(out_gpu, o_ref)
+    assert max_abs <= ATOL_MAX, f"max-abs {max_abs:.3e} > {ATOL_MAX}"
+    assert rel <= RTOL_L2, f"rel-L2 {rel:.3e} > {RTOL_L2}"
+    l = to64(lse_gpu)
+    m = ~np.isnan(lse_ref)
+    inf_ref = np.isinf(lse_ref) & m
+    assert np.array_equal(np.isinf(l) & m, inf_ref), "lse -inf pattern differs"
+    fin = m & ~inf_ref
+    if fin.any():
+        d = np.abs(l[fin] - lse_ref[fin]).max()
+        assert d <= LSE_ATOL, f"lse max-abs {d:.3e}"
+    return max_abs, rel

@@ -1,0 +1,167 @@
+"""CPU tests of the C-ABI library: it loads, exports every declared symbol, its
+integer accounting is bit-exact against the oracle, and argument checks reject bad
+calls before any device work (fake pointers are never dereferenced)."""
+import ctypes
+import glob
+import os
+import re
+
+import numpy as np
+import pytest
+
+import decode_attention_12_b200 as lla
+import lla_synth as S
+import oracle
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def declared_symbols():
+    names = set()
+    for h in glob.glob(os.path.join(ROOT, "include", "*.h")):
+        src = open(h).read()
+        src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+        names |= set(re.findall(r"\b(lla_\w+)\s*\(", src))
+    return sorted(names)
+
+
+def test_every_declared_symbol_is_exported():
+    names = declared_symbols()
+    assert {"lla_cache_bytes", "lla_encode", "lla_decode_attn"} <= set(names)
+    lib = ctypes.CDLL(lla.LIB_PATH)
+    missing = [n for n in names if not hasattr(lib, n)]
+    assert not missing, missing
+
+
+def test_status_strings():
+    for code in (0, -1, -2, -3, -4, -5, -6):
+        assert lla.status_string(code) and lla.status_string(code) != "unknown status"
+    assert lla.status_string(12345) == "unknown status"
+
+
+@pytest.mark.parametrize("name", sorted(S.WORKLOADS))
+def test_cache_bytes_bit_exact_vs_oracle(name):
+    w = S.WORKLOADS[name]
+    lens = S.context_lengths(w)
+    dims = lla.make_dims(w.T, w.L, w.H, w.d, w.r_k, w.r_v, int(w.fold2d),
+                         lla.F32 if w.dtype == "f32" else lla.BF16)
+    got = lla.cache_bytes(dims, lens)
+    ref = oracle.cache_bytes(w.T, w.L, w.H, w.d, w.r_k, w.r_v, w.fold2d, w.elem_bytes,
+                             int(lens.sum()))
+    assert got == ref
+
+
+def test_cache_bytes_random_dims_bit_exact():
+    rng = np.random.default_rng(0)
+    for _ in range(300):
+        T, L, H = (int(v) for v in rng.integers(1, 33, 3))
+        d = int(rng.choice([16, 64, 128, 256]))
+        rk, rv = (int(v) for v in rng.integers(1, 513, 2))
+        fold = int(rng.integers(0, 2))
+        dt = int(rng.integers(0, 2))
+        lens = rng.integers(0, 20000, size=int(rng.integers(0, 50)))
+        dims = lla.make_dims(T, L, H, d, rk, rv, fold, dt)
+        got = lla.cache_bytes(dims, lens)
+        ref = oracle.cache_bytes(T, L, H, d, rk, rv, bool(fold), 4 if dt == 0 else 2,
+                                 int(lens.sum()))
+        assert got == ref
+
+
+def test_capacity_workload_bytes():
+    w = S.WORKLOADS["capacity-768x4k"]
+    dims = lla.make_dims(w.T, w.L, w.H, w.d, w.r_k, w.r_v)
+    lat, unc, num, den = lla.cache_bytes(dims, [4096] * 768)
+    assert lat == 115_964_116_992 and (num, den) == (64, 3)
+
+
+def test_cache_bytes_errors():
+    dims = lla.make_dims(4, 1, 2, 64, 8, 16)
+    with pytest.raises(lla.LLAError):
+        lla.cache_bytes(dims, [5, -1])
+    with pytest.raises(lla.LLAError):
+        lla.cache_bytes(lla.make_dims(0, 1, 2, 64, 8, 16), [5])
+
+
+@pytest.mark.parametrize("gap", [0, 3])
+def test_slot_layout_exact(gap):
+    lens = np.array([5, 0, 7, 1, 4096, 3], dtype=np.int32)
+    starts, total = lla.slot_layout(lens, gap)
+    assert starts == list(S.slot_starts(lens, gap))
+    assert total == int(lens.sum()) + gap * len(lens)
+    big = [2 ** 31 - 1] * 8
+    starts, total = lla.slot_layout(big, 0)
+    assert total == 8 * (2 ** 31 - 1) and starts[-1] == 7 * (2 ** 31 - 1)
+
+
+# ---- argument checks (no device memory is touched: fake aligned pointers) ------------
+FAKE = 1 << 40   # 16-byte aligned, never dereferenced
+
+
+def _decode_args(**over):
+    dims = lla.make_dims(4, 1, 16, 128, 16, 32)
+    codec = lla.make_codec(W_up_k=FAKE, W_up_v=FAKE, mu_k=FAKE, mu_v=FAKE)
+    cache = lla.make_cache(FAKE, FAKE, 1000)
+    a = dict(dims=dims, layer=0, t0=0, Tq=4, q=FAKE, cache=cache, seq_start=FAKE, ctx_lens=FAKE,
+             B=2, max_ctx=100, codec=codec, softmax_scale=1.0, out=FAKE, lse=None,
+             workspace=FAKE, ws_bytes=1 << 30, variant=lla.ABSORB, num_splits=0, stream=0)
+    a.update(over)
+    return a
+
+
+def _rc(**over):
+    try:
+        lla.decode_attn(**_decode_args(**over))
+    except lla.LLAError as e:
+        return e.code
+    return 0
+
+
+def test_decode_argument_errors():
+    assert _rc(layer=1) == lla.LLA_ERR_INVALID
+    assert _rc(t0=1) == lla.LLA_ERR_INVALID          # t0 + Tq > T
+    assert _rc(Tq=0) == lla.LLA_ERR_INVALID
+    assert _rc(max_ctx=-1) == lla.LLA_ERR_INVALID
+    assert _rc(variant=7) == lla.LLA_ERR_INVALID
+    assert _rc(q=0) == lla.LLA_ERR_INVALID
+    assert _rc(q=FAKE + 2) == lla.LLA_ERR_MISALIGNED
+    assert _rc(out=FAKE + 8) == lla.LLA_ERR_MISALIGNED
+    assert _rc(ws_bytes=64) == lla.LLA_ERR_WORKSPACE
+    assert _rc(workspace=0) == lla.LLA_ERR_WORKSPACE
+    assert _rc(dims=lla.make_dims(4, 1, 16, 128, 0, 32)) == lla.LLA_ERR_INVALID
+    assert _rc(dims=lla.make_dims(4, 1, 16, 128, 12, 32)) == lla.LLA_ERR_UNSUPPORTED  # 24 B rows
+    assert _rc(dims=lla.make_dims(4, 1, 16, 128, 16, 32, 0, 5)) == lla.LLA_ERR_INVALID
+    assert _rc(B=0) == 0  # nothing to do, nothing launched
+
+
+def test_workspace_bytes_and_splits():
+    dims = lla.make_dims(4, 1, 16, 128, 16, 32)
+    s = lla.decode_num_splits(dims, 64, 4, 4096)
+    assert s >= 1
+    ws = lla.decode_workspace_bytes(dims, 64, 4, 4096)
+    assert ws >= 256 + 64 * 16 * 4 * s * (32 + 4) * 4
+    assert lla.decode_num_splits(dims, 64, 4, 4096, num_splits=7) == 7
+    with pytest.raises(lla.LLAError):
+        lla.decode_workspace_bytes(dims, 64, 0, 4096)
+
+
+def test_encode_argument_errors():
+    dims = lla.make_dims(4, 2, 16, 128, 96, 160)
+    codec = lla.make_codec(W_down_k=FAKE, W_down_v=FAKE, bias_k=FAKE, bias_v=FAKE)
+    cache = lla.make_cache(FAKE, FAKE, 10)
+
+    def rc(**over):
+        a = dict(dims=dims, layer0=0, n_layers=1, x_k=FAKE, x_v=FAKE, n_tok=4, slot_idx=FAKE,
+                 codec=codec, cache=cache, stream=0)
+        a.update(over)
+        try:
+            lla.encode(**a)
+        except lla.LLAError as e:
+            return e.code
+        return 0
+
+    assert rc(layer0=2) == lla.LLA_ERR_INVALID
+    assert rc(layer0=1, n_layers=2) == lla.LLA_ERR_INVALID
+    assert rc(x_k=FAKE + 4) == lla.LLA_ERR_MISALIGNED
+    assert rc(x_v=0) == lla.LLA_ERR_INVALID
+    assert rc(n_tok=0) == 0
+    assert rc(dims=lla.make_dims(4, 2, 16, 128, 320, 160)) == lla.LLA_ERR_UNSUPPORTED

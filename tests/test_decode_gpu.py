@@ -1,0 +1,141 @@
+"""GPU parity: lla_decode_attn (absorb form) against the fp64 oracle on seeded inputs."""
+import numpy as np
+import pytest
+import torch
+
+import decode_attention_12_b200 as lla
+import lla_synth as S
+from gpu_util import assert_attn_close, oracle_decode, run_decode
+
+pytestmark = pytest.mark.gpu
+DEV = "cuda"
+
+
+@pytest.fixture(scope="module")
+def tiny():
+    w = S.WORKLOADS["tiny-fp32"]
+    return w, S.decode_inputs(w, 0, DEV)
+
+
+@pytest.mark.parametrize("splits", [1, 2, 0])
+def test_tiny_fp32_all_loops_fused(tiny, splits):
+    w, p = tiny
+    out, lse, st = run_decode(p, w, 0, 0, 4, 1.0, num_splits=splits)
+    assert st == 0
+    o_ref, l_ref = oracle_decode(p, w, 0, 0, 4, 1.0)
+    assert_attn_close(out, lse, o_ref, l_ref)
+
+
+@pytest.mark.parametrize("t0", [0, 1, 2, 3])
+def test_tiny_fp32_one_loop_per_call(tiny, t0):
+    w, p = tiny
+    q1 = p["q"][:, t0:t0 + 1].contiguous()
+    out, lse, st = run_decode(p, w, 0, t0, 1, 0.125, q=q1)
+    assert st == 0
+    o_ref, l_ref = oracle_decode(p, w, 0, t0, 1, 0.125, q=q1)
+    assert_attn_close(out, lse, o_ref, l_ref)
+
+
+@pytest.fixture(scope="module")
+def ouro():
+    w = S.WORKLOADS["ouro1.4b-layer"]
+    return w, S.decode_inputs(w, 0, DEV)
+
+
+def test_ouro_layer_fused_loops_full(ouro):
+    """Full Ouro-1.4B-shaped layer, 64 ragged sequences, all 4 loop queries in one
+    pass, the split count the benchmark uses (automatic)."""
+    w, p = ouro
+    out, lse, st = run_decode(p, w, 0, 0, 4, 1.0)
+    assert st == 0
+    o_ref, l_ref = oracle_decode(p, w, 0, 0, 4, 1.0)
+    assert_attn_close(out, lse, o_ref, l_ref)
+
+
+@pytest.mark.parametrize("t0", [0, 3])
+def test_ouro_layer_model_order_single_loop(ouro, t0):
+    w, p = ouro
+    q1 = p["q"][:, t0:t0 + 1].contiguous()
+    out, lse, st = run_decode(p, w, 0, t0, 1, 1.0, q=q1)
+    assert st == 0
+    units = [(b, h) for b in range(0, 64, 5) for h in range(16)]
+    o_ref, l_ref = oracle_decode(p, w, 0, t0, 1, 1.0, q=q1, units=units)
+    assert_attn_close(out, lse, o_ref, l_ref)
+
+
+def test_decode_is_deterministic(ouro):
+    w, p = ouro
+    a = run_decode(p, w, 0, 0, 4, 1.0)
+    b = run_decode(p, w, 0, 0, 4, 1.0)
+    assert torch.equal(a[0], b[0]) and torch.equal(a[1], b[1])
+
+
+# ---- edge cases -------------------------------------------------------------------------
+EDGE_LENS = [0, 1, 2, 31, 255, 256, 257, 1000, 4097]
+
+
+@pytest.mark.parametrize("rk,rv", [(16, 32), (8, 16), (16, 16)])
+@pytest.mark.parametrize("splits", [1, 3, 8])
+def test_ragged_edges_bf16(rk, rv, splits):
+    w = S.shrink(S.WORKLOADS["ouro1.4b-layer"], name=f"edge-{rk}-{rv}", r_k=rk, r_v=rv,
+                 B=len(EDGE_LENS))
+    p = S.decode_inputs(w, 0, DEV, lens=EDGE_LENS, gap=5)
+    out, lse, st = run_decode(p, w, 0, 0, 4, 1.0, num_splits=splits)
+    assert st == 0
+    o_ref, l_ref = oracle_decode(p, w, 0, 0, 4, 1.0)
+    assert_attn_close(out, lse, o_ref, l_ref)
+    # empty context: out == 0 exactly, lse == -inf
+    assert torch.all(out[0] == 0) and torch.all(torch.isneginf(lse[0]))
+
+
+@pytest.mark.parametrize("Tq,t0", [(2, 1), (3, 0), (3, 1)])
+def test_partial_loop_ranges(Tq, t0):
+    w = S.shrink(S.WORKLOADS["ouro1.4b-layer"], name="tq", B=6, len_lo=100, len_hi=3000)
+    p = S.decode_inputs(w, 0, DEV, Tq=Tq)
+    out, lse, st = run_decode(p, w, 0, t0, Tq, 1.0)
+    assert st == 0
+    o_ref, l_ref = oracle_decode(p, w, 0, t0, Tq, 1.0)
+    assert_attn_close(out, lse, o_ref, l_ref)
+
+
+@pytest.mark.parametrize("scale", [30.0, 1.0 / np.sqrt(128)])
+def test_large_and_small_logit_scales(scale):
+    w = S.shrink(S.WORKLOADS["ouro1.4b-layer"], name="scale", B=4, len_lo=500, len_hi=2500)
+    p = S.decode_inputs(w, 0, DEV)
+    out, lse, st = run_decode(p, w, 0, 0, 4, scale, num_splits=2)
+    assert st == 0
+    o_ref, l_ref = oracle_decode(p, w, 0, 0, 4, scale)
+    assert_attn_close(out, lse, o_ref, l_ref)
+
+
+def test_distilled_codec_up_projection_not_transpose():
+    """W_up perturbed away from W_down^T (a distilled codec): still exact attention."""
+    w = S.shrink(S.WORKLOADS["ouro1.4b-layer"], name="perturb", B=4, len_lo=300, len_hi=1500)
+    p = S.decode_inputs(w, 0, DEV, perturb=0.3)
+    out, lse, st = run_decode(p, w, 0, 0, 4, 1.0)
+    assert st == 0
+    o_ref, l_ref = oracle_decode(p, w, 0, 0, 4, 1.0)
+    assert_attn_close(out, lse, o_ref, l_ref)
+
+
+def test_second_layer_of_a_multilayer_cache():
+    w = S.shrink(S.WORKLOADS["capacity-768x4k"], name="ml", L=3, B=5, len_lo=10, len_hi=900)
+    p = S.decode_inputs(w, [0, 2], DEV)
+    for layer in (0, 2):
+        out, lse, st = run_decode(p, w, layer, 0, 4, 1.0)
+        assert st == 0
+        o_ref, l_ref = oracle_decode(p, w, layer, 0, 4, 1.0)
+        assert_attn_close(out, lse, o_ref, l_ref)
+
+
+def test_bf16_output_storage(ouro):
+    """bf16 outputs: the only extra error is the final round-to-nearest-even (<= 2^-9 |o|)."""
+    w, p = ouro
+    out, lse, st = run_decode(p, w, 0, 0, 4, 1.0, out_dtype=lla.BF16)
+    assert st == 0 and out.dtype == torch.bfloat16
+    units = [(b, h) for b in range(0, 64, 7) for h in range(16)]
+    o_ref, _ = oracle_decode(p, w, 0, 0, 4, 1.0, units=units)
+    o = out.float().cpu().double().numpy()
+    m = ~np.isnan(o_ref)
+    bound = np.abs(o_ref[m]) * 2.0 ** -8 + 5e-3
+    assert np.all(np.abs(o[m] - o_ref[m]) <= bound)
