@@ -1,6 +1,6 @@
 """Build liblla.so (the C-ABI library) in-tree with nvcc for sm_100a.
 
-Usage:  python -m decode_attention_12_b200._build   (or __graft_entry__.build())
+Usage:  python decode_attention_12_b200/_build.py [--force] [--ptxas-v]   (or __graft_entry__.build())
 """
 from __future__ import annotations
 
