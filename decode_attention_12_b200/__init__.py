@@ -23,7 +23,7 @@ LIB_PATH = os.path.join(_HERE, "liblla.so")
 if not os.path.exists(LIB_PATH):
     raise ImportError(
         f"{LIB_PATH} is missing: build the CUDA library first "
-        "(python -m decode_attention_12_b200._build, or __graft_entry__.build())")
+        "(python decode_attention_12_b200/_build.py, or __graft_entry__.build())")
 
 _lib = ctypes.CDLL(LIB_PATH)
 
@@ -40,7 +40,8 @@ ABSORB, RECONSTRUCT = 0, 1
 
 EXPORTED = ("lla_cache_bytes", "lla_slot_layout", "lla_codec_bias", "lla_encode",
             "lla_decode_attn", "lla_decode_workspace_bytes", "lla_decode_num_splits",
-            "lla_status_fetch", "lla_status_string")
+            "lla_decode_attn_static", "lla_status_fetch", "lla_status_string")
+STATIC_SCRATCH_BYTES = 8 << 20
 
 
 class Dims(ctypes.Structure):
@@ -66,6 +67,8 @@ _lib.lla_codec_bias.argtypes = [_P(Dims), _P(Codec), _vp, _vp, _vp]
 _lib.lla_encode.argtypes = [_P(Dims), _i32, _i32, _vp, _vp, _i64, _vp, _P(Codec), _P(Cache), _vp]
 _lib.lla_decode_attn.argtypes = [_P(Dims), _i32, _i32, _i32, _vp, _P(Cache), _vp, _vp, _i32, _i32,
                                  _P(Codec), ctypes.c_float, _i32, _i32, _vp, _vp, _vp, _sz, _vp]
+_lib.lla_decode_attn_static.argtypes = [_P(Dims), _i32, _i32, _i32, _vp, _P(Cache), _vp, _vp, _i32,
+                                        _i32, _P(Codec), ctypes.c_float, _i32, _i32, _vp, _vp, _vp]
 _lib.lla_decode_workspace_bytes.argtypes = [_P(Dims), _i32, _i32, _i32, _i32, _i32]
 _lib.lla_decode_workspace_bytes.restype = _sz
 _lib.lla_decode_num_splits.argtypes = [_P(Dims), _i32, _i32, _i32, _i32, _i32]
@@ -73,7 +76,7 @@ _lib.lla_status_fetch.argtypes = [_vp, _vp, _P(_i32)]
 _lib.lla_status_string.argtypes = [ctypes.c_int]
 _lib.lla_status_string.restype = ctypes.c_char_p
 for _n in ("lla_cache_bytes", "lla_slot_layout", "lla_codec_bias", "lla_encode", "lla_decode_attn",
-           "lla_decode_num_splits", "lla_status_fetch"):
+           "lla_decode_attn_static", "lla_decode_num_splits", "lla_status_fetch"):
     getattr(_lib, _n).restype = ctypes.c_int
 
 
@@ -181,6 +184,19 @@ def decode_attn(dims: Dims, layer: int, t0: int, Tq: int, q, cache: Cache, seq_s
                                 float(softmax_scale), variant, num_splits, _ptr(out), _ptr(lse),
                                 _ptr(workspace), int(ws_bytes), _stream(stream)),
            "lla_decode_attn")
+
+
+def decode_attn_static(dims: Dims, layer: int, t0: int, Tq: int, q, cache: Cache, seq_start,
+                       ctx_lens, B: int, max_ctx: int, codec: Codec, softmax_scale: float, out,
+                       lse=None, variant: int = ABSORB, num_splits: int = 0, stream=None) -> None:
+    """lla_decode_attn without a workspace argument: for callers that cannot allocate
+    device memory.  The scratch is an 8 MiB array inside the library, shared by every
+    call (serialise calls that could overlap on the GPU)."""
+    _check(_lib.lla_decode_attn_static(ctypes.byref(dims), layer, t0, Tq, _ptr(q), ctypes.byref(cache),
+                                       _ptr(seq_start), _ptr(ctx_lens), B, max_ctx,
+                                       ctypes.byref(codec), float(softmax_scale), variant, num_splits,
+                                       _ptr(out), _ptr(lse), _stream(stream)),
+           "lla_decode_attn_static")
 
 
 def status_fetch(workspace, stream=None) -> int:

@@ -167,6 +167,31 @@ size_t lla_decode_workspace_bytes(const lla_dims *dims, int32_t B, int32_t Tq,
 int lla_decode_num_splits(const lla_dims *dims, int32_t B, int32_t Tq, int32_t max_ctx,
                           int32_t variant, int32_t num_splits);
 
+/* ---- decode attention with library-owned scratch ----------------------------------------
+ * No counterpart in the paper: a deployment aid.  Some callers cannot allocate device
+ * memory -- for example a plugin whose host framework owns the whole device memory pool
+ * and offers no allocation hook, or a serving loop whose rules forbid any allocation
+ * after start-up.  For them this entry point computes exactly what lla_decode_attn
+ * computes, with the same arguments and errors, but takes no workspace: its scratch is
+ * a file-scope device array of LLA_STATIC_SCRATCH_BYTES (8 MiB) inside the library,
+ * which every GPU that loads the library holds until the process exits.  It calls no
+ * cudaMalloc, no cudaFree and no allocating library routine.
+ *  - The first call on a device, made with that device current, looks up the array's
+ *    device address (cudaGetSymbolAddress) and caches it; make that first call before
+ *    any stream capture.
+ *  - A problem that needs more scratch than LLA_STATIC_SCRATCH_BYTES (compare
+ *    lla_decode_workspace_bytes) is rejected with LLA_ERR_WORKSPACE before any launch.
+ *  - All calls share the one array, which keeps the last call's contents; each call
+ *    clears the array's status word (a 4-byte memset on `stream`) before its launches.
+ *    Calls that overlap on the GPU (other streams, or unordered host threads) race on
+ *    the array: the caller must serialise them.                                            */
+#define LLA_STATIC_SCRATCH_BYTES (8u << 20)
+int lla_decode_attn_static(const lla_dims *dims, int32_t layer, int32_t t0, int32_t Tq,
+                           const void *q, const lla_cache *cache, const int64_t *seq_start,
+                           const int32_t *ctx_lens, int32_t B, int32_t max_ctx,
+                           const lla_codec *codec, float softmax_scale, int32_t variant,
+                           int32_t num_splits, void *out, float *lse, lla_stream_t stream);
+
 /* ---- status ---------------------------------------------------------------------------
  * Kernels never trap.  A kernel that gives up a bounded wait records
  * LLA_ERR_DEVICE_TIMEOUT in the first word of the decode workspace (sticky).
