@@ -385,7 +385,7 @@ def main():
         "config": {"workload": w.name, "T": w.T, "L_per_step": 1, "H": H, "d": w.d,
                    "r_k": w.r_k, "r_v": w.r_v, "rho": "64/3", "B": B,
                    "ctx_len": [w.len_lo, w.len_hi], "tokens": S_tot, "Tq": Tq,
-                   "variant": "absorb", "num_splits": splits,
+                   "variant": "absorb", "seg_max": splits,
                    "step": "decode_attn(all 4 loop queries) + encode(B new tokens)",
                    "l2": f"inputs larger than L2 ({step_bytes / 1e6:.0f} MB of latents per step) "
                          f"and {R} rotating cache replicas",

@@ -5,9 +5,9 @@
 
 namespace lla {
 
-// Arguments of one decode call for one layer (pointers already offset to the layer).
+// Arguments of one decode pass for one layer (pointers already offset to the layer).
 struct DecodeArgs {
-    const void *q;            // T [B][Tq][H][d]
+    const void *q;            // T [B][Tq_all][H][d]
     const void *k;            // T [H'][slots][r_k]
     const void *v;            // T [H'][slots][r_v]
     int64_t slots;
@@ -18,14 +18,17 @@ struct DecodeArgs {
     const float *W_up_v;      // [H'][T][r_v][D']
     const float *mu_v;        // [H'][T][D']
     int32_t B, H, d, T, t0, Tq, fold, r_k, r_v;
-    int32_t Tq_all, tq_off;   // q/out/lse/part hold Tq_all loop queries; this pass
+    int32_t Tq_all, tq_off;   // q/out/lse/records hold Tq_all loop queries; this pass
                               // serves queries tq_off .. tq_off+Tq-1 (loop t0 + tq_off + i)
-    int32_t num_splits;
+    int32_t seg_max;          // partial-record slots per (unit, query)
+    int32_t chunk_min;        // smallest token share of one decode CTA
     float scale;              // softmax scale
-    float *part;              // [B][H][Tq][num_splits][r_v + 4] partial records
+    float *qt;                // [B*H][Tq_all][r_k] absorbed queries, pre-scaled by log2(e)
+    int32_t *counts;          // [B*H] partial records written for each unit by this pass
+    float *part;              // [B*H][Tq_all][seg_max][r_v + 4] partial records
     int32_t *status;          // sticky device status word
-    void *out;                // O [B][Tq][H][d] (O = out_dtype)
-    float *lse;               // [B][Tq][H] or null
+    void *out;                // O [B][Tq_all][H][d] (O = out_dtype)
+    float *lse;               // [B][Tq_all][H] or null
 };
 
 constexpr float kLog2e = 1.4426950408889634f;
@@ -34,18 +37,13 @@ constexpr float kLn2 = 0.6931471805599453f;
 // Partial record stride (floats) for value rank r_v: acc[r_v], m, l, 2 pad.
 __host__ __device__ constexpr int part_stride(int r_v) { return r_v + 4; }
 
-// Token range [n0, n1) of split `s` out of `S` for a context of `len` tokens.
-__device__ __forceinline__ void split_range(int len, int s, int S, int &n0, int &n1)
-{
-    int chunk = (len + S - 1) / S;
-    chunk = (chunk + 31) & ~31;
-    n0 = min(len, s * chunk);
-    n1 = min(len, n0 + chunk);
-}
+// Decode CTAs resident per SM that the persistent kernel is shaped for.
+constexpr int kDecodeCtasPerSm = 4;
 
-cudaError_t launch_decode_absorb_simt(const DecodeArgs &a, int dtype, cudaStream_t stream,
-                                      bool *supported);
+cudaError_t launch_decode_absorb(const DecodeArgs &a, int dtype, int ctas, cudaStream_t stream,
+                                 bool *supported);
+cudaError_t launch_absorb_prologue(const DecodeArgs &a, int dtype, cudaStream_t stream);
 cudaError_t launch_decode_combine(const DecodeArgs &a, int dtype, int out_dtype, cudaStream_t stream);
-bool decode_absorb_simt_supported(int dtype, int r_k, int r_v, int d, int fold);
+bool decode_absorb_supported(int dtype, int r_k, int r_v, int d, int fold);
 
 } // namespace lla

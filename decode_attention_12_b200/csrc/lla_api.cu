@@ -57,28 +57,32 @@ int sm_count()
     return cached[dev];
 }
 
-int choose_splits(const lla_dims *d, int32_t B, int32_t max_ctx, int32_t num_splits)
-{
-    if (num_splits > 0)
-        return num_splits;
-    const int64_t units = (int64_t)B * d->H;
-    if (units <= 0)
-        return 1;
-    const int64_t target = (int64_t)sm_count() * 2 * 4; // ~4 waves at 2 CTAs per SM
-    int64_t s = (target + units - 1) / units;
-    int64_t cap = max_ctx / 1024;
-    if (cap < 1)
-        cap = 1;
-    if (s > cap)
-        s = cap;
-    if (s > 256)
-        s = 256;
-    return (int)(s < 1 ? 1 : s);
-}
+// Plan of one decode call: the work split of the persistent decode kernel and the
+// workspace regions (header | counts | q_tilde | partial records).
+struct Plan {
+    int32_t seg_max, chunk_min;
+    size_t off_counts, off_qt, off_part, bytes;
+};
 
-size_t part_bytes(const lla_dims *d, int32_t B, int32_t Tq, int splits)
+size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
+
+Plan make_plan(const lla_dims *d, int32_t B, int32_t Tq, int32_t max_ctx, int32_t num_splits)
 {
-    return (size_t)B * d->H * Tq * splits * part_stride(d->r_v) * sizeof(float);
+    Plan p;
+    const int64_t units = (int64_t)B * d->H;
+    const int64_t ctas = (int64_t)sm_count() * kDecodeCtasPerSm;
+    int64_t segs = num_splits > 0 ? num_splits : (units > 0 ? (2 * ctas + units - 1) / units : 1);
+    if (segs < 1) segs = 1;
+    if (segs > 64) segs = 64;
+    int64_t chunk_min = (max_ctx + segs - 1) / segs;
+    if (chunk_min < 128) chunk_min = 128;
+    p.chunk_min = (int32_t)chunk_min;
+    p.seg_max = (int32_t)((max_ctx + chunk_min - 1) / chunk_min + 1);
+    p.off_counts = kWorkspaceHeader;
+    p.off_qt = align256(p.off_counts + (size_t)units * sizeof(int32_t));
+    p.off_part = align256(p.off_qt + (size_t)units * Tq * d->r_k * sizeof(float));
+    p.bytes = p.off_part + (size_t)units * Tq * p.seg_max * part_stride(d->r_v) * sizeof(float);
+    return p;
 }
 
 } // namespace
@@ -217,16 +221,15 @@ int lla_decode_num_splits(const lla_dims *dims, int32_t B, int32_t Tq, int32_t m
     if (B < 0 || Tq < 1 || max_ctx < 0 || num_splits < 0 ||
         (variant != LLA_ABSORB && variant != LLA_RECONSTRUCT))
         return LLA_ERR_INVALID;
-    return choose_splits(dims, B, max_ctx, num_splits);
+    return make_plan(dims, B, Tq, max_ctx, num_splits).seg_max;
 }
 
 size_t lla_decode_workspace_bytes(const lla_dims *dims, int32_t B, int32_t Tq, int32_t max_ctx,
                                   int32_t variant, int32_t num_splits)
 {
-    const int s = lla_decode_num_splits(dims, B, Tq, max_ctx, variant, num_splits);
-    if (s < 1)
+    if (lla_decode_num_splits(dims, B, Tq, max_ctx, variant, num_splits) < 1)
         return 0;
-    return kWorkspaceHeader + part_bytes(dims, B, Tq, s);
+    return make_plan(dims, B, Tq, max_ctx, num_splits).bytes;
 }
 
 int lla_decode_attn(const lla_dims *dims, int32_t layer, int32_t t0, int32_t Tq, const void *q,
@@ -252,15 +255,16 @@ int lla_decode_attn(const lla_dims *dims, int32_t layer, int32_t t0, int32_t Tq,
         !aligned16(codec->mu_v) || !aligned16(seq_start) || !aligned16(ctx_lens) ||
         (lse != nullptr && !aligned16(lse)))
         return LLA_ERR_MISALIGNED;
-    const int splits = choose_splits(dims, B, max_ctx, num_splits);
-    const size_t need = kWorkspaceHeader + part_bytes(dims, B, Tq, splits);
-    if (workspace == nullptr || ws_bytes < need)
+    const Plan plan = make_plan(dims, B, Tq, max_ctx, num_splits);
+    if (workspace == nullptr || ws_bytes < plan.bytes)
         return LLA_ERR_WORKSPACE;
     if (!aligned16(workspace))
         return LLA_ERR_MISALIGNED;
     if (variant != LLA_ABSORB)
         return LLA_ERR_UNSUPPORTED;
-    if (!decode_absorb_simt_supported(dims->dtype, dims->r_k, dims->r_v, dims->d_head, dims->fold))
+    if (!decode_absorb_supported(dims->dtype, dims->r_k, dims->r_v, dims->d_head, dims->fold))
+        return LLA_ERR_UNSUPPORTED;
+    if (B > 16384)
         return LLA_ERR_UNSUPPORTED;
 
     const int Hs = heads_stored(dims);
@@ -279,24 +283,30 @@ int lla_decode_attn(const lla_dims *dims, int32_t layer, int32_t t0, int32_t Tq,
     a.mu_v = codec->mu_v + (int64_t)layer * Hs * dims->T * Dp;
     a.B = B; a.H = dims->H; a.d = dims->d_head; a.T = dims->T; a.t0 = t0; a.Tq = Tq;
     a.fold = dims->fold; a.r_k = dims->r_k; a.r_v = dims->r_v;
-    a.num_splits = splits;
+    a.seg_max = plan.seg_max;
+    a.chunk_min = plan.chunk_min;
     a.scale = softmax_scale;
-    a.status = static_cast<int32_t *>(workspace);
-    a.part = reinterpret_cast<float *>(static_cast<uint8_t *>(workspace) + kWorkspaceHeader);
+    uint8_t *ws = static_cast<uint8_t *>(workspace);
+    a.status = reinterpret_cast<int32_t *>(ws);
+    a.counts = reinterpret_cast<int32_t *>(ws + plan.off_counts);
+    a.qt = reinterpret_cast<float *>(ws + plan.off_qt);
+    a.part = reinterpret_cast<float *>(ws + plan.off_part);
     a.out = out;
     a.lse = lse;
 
     a.Tq_all = Tq;
     a.tq_off = 0;
     cudaStream_t s = (cudaStream_t)stream;
-    // The SIMT kernel serves up to 4 loop queries per pass over the latents.
+    // The CUDA-core kernel serves up to 4 loop queries per pass over the latents.
     cudaError_t err = cudaSuccess;
     for (int32_t c = 0; c < Tq && err == cudaSuccess; c += 4) {
         DecodeArgs ac = a;
         ac.tq_off = c;
         ac.Tq = Tq - c < 4 ? Tq - c : 4;
+        err = launch_absorb_prologue(ac, dims->dtype, s);
         bool supported = false;
-        err = launch_decode_absorb_simt(ac, dims->dtype, s, &supported);
+        if (err == cudaSuccess)
+            err = launch_decode_absorb(ac, dims->dtype, 0, s, &supported);
         if (!supported)
             return LLA_ERR_UNSUPPORTED;
         if (err == cudaSuccess)

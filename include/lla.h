@@ -146,7 +146,9 @@ int lla_encode(const lla_dims *dims, int32_t layer0, int32_t n_layers, const voi
  *   lse      fp32 [B][Tq][H] or NULL    (len_b = 0 gives out = 0 and lse = -inf)
  *   seq_start int64 [B], ctx_lens int32 [B]   (device; slots must lie in the plane)
  *   max_ctx  host-side upper bound of ctx_lens, used only to choose the split count
- *   num_splits  split-K factor per (sequence, head); 0 = automatic
+ *   num_splits  target number of token shares (split-K pieces) per (sequence, head);
+ *               0 = automatic.  The work is spread evenly over resident CTAs, so a
+ *               share never holds fewer than ceil(max_ctx / num_splits) tokens
  *   workspace   device scratch of at least lla_decode_workspace_bytes(...) bytes
  * Errors: LLA_ERR_INVALID (dims, loop range, Tq < 1, pointers), LLA_ERR_UNSUPPORTED,
  * LLA_ERR_MISALIGNED, LLA_ERR_WORKSPACE, LLA_ERR_CUDA.                                  */
@@ -162,8 +164,8 @@ int lla_decode_attn(const lla_dims *dims, int32_t layer, int32_t t0, int32_t Tq,
 size_t lla_decode_workspace_bytes(const lla_dims *dims, int32_t B, int32_t Tq,
                                   int32_t max_ctx, int32_t variant, int32_t num_splits);
 
-/* The split count lla_decode_attn uses for these arguments (>= 1), or a negative
- * LLA_ERR_* code.                                                                     */
+/* The largest number of partial records lla_decode_attn writes per (sequence, head,
+ * loop query) for these arguments (>= 1), or a negative LLA_ERR_* code.              */
 int lla_decode_num_splits(const lla_dims *dims, int32_t B, int32_t Tq, int32_t max_ctx,
                           int32_t variant, int32_t num_splits);
 

@@ -139,7 +139,8 @@ def test_workspace_bytes_and_splits():
     assert s >= 1
     ws = lla.decode_workspace_bytes(dims, 64, 4, 4096)
     assert ws >= 256 + 64 * 16 * 4 * s * (32 + 4) * 4
-    assert lla.decode_num_splits(dims, 64, 4, 4096, num_splits=7) == 7
+    # 7 shares of >= ceil(4096/7) = 586 tokens: a context spans at most 8 of them
+    assert lla.decode_num_splits(dims, 64, 4, 4096, num_splits=7) == 8
     with pytest.raises(lla.LLAError):
         lla.decode_workspace_bytes(dims, 64, 0, 4096)
 
