@@ -77,17 +77,48 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity)
     return ok != 0;
 }
 
-// Wait for phase `parity` of `bar` to complete, giving up after kWaitLimitNs.
+// try_wait that may suspend the thread for up to ~`hint_ns` while the phase is pending.
+__device__ __forceinline__ bool mbar_try_wait_hint(uint32_t bar, uint32_t parity, uint32_t hint_ns)
+{
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(bar), "r"(parity), "r"(hint_ns)
+        : "memory");
+    return ok != 0;
+}
+
+// Wait for phase `parity` of `bar` to complete, giving up after kWaitLimitNs.  The
+// clock is read only every 256 polls so that waiting warps cost few issue slots.
 __device__ __forceinline__ bool mbar_wait_bounded(uint32_t bar, uint32_t parity)
 {
     if (mbar_try_wait(bar, parity))
         return true;
     const uint64_t t0 = global_timer_ns();
-    while (!mbar_try_wait(bar, parity)) {
-        if (global_timer_ns() - t0 > kWaitLimitNs)
+    for (uint32_t n = 1;; ++n) {
+        if (mbar_try_wait_hint(bar, parity, 20000u))
+            return true;
+        if ((n & 255u) == 0u && global_timer_ns() - t0 > kWaitLimitNs)
             return false;
     }
-    return true;
+}
+
+// Programmatic dependent launch: allow the next grid in the stream (launched with the
+// programmatic-serialization attribute) to start once every CTA of this grid has run
+// this instruction or exited.
+__device__ __forceinline__ void grid_launch_dependents()
+{
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
+// Programmatic dependent launch: block until the preceding grid in the stream has
+// completed and its memory is visible (no-op when launched without the attribute).
+__device__ __forceinline__ void grid_dependency_wait()
+{
+    asm volatile("griddepcontrol.wait;" ::: "memory");
 }
 
 // ---- 1-D bulk copy global -> shared (TMA engine), completion on an mbarrier -----------

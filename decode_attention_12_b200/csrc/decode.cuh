@@ -45,5 +45,7 @@ cudaError_t launch_decode_absorb(const DecodeArgs &a, int dtype, int ctas, cudaS
 cudaError_t launch_absorb_prologue(const DecodeArgs &a, int dtype, cudaStream_t stream);
 cudaError_t launch_decode_combine(const DecodeArgs &a, int dtype, int out_dtype, cudaStream_t stream);
 bool decode_absorb_supported(int dtype, int r_k, int r_v, int d, int fold);
+bool decode_mma_supported(int dtype, int r_k, int r_v, int fold, int Tq);
+cudaError_t launch_decode_absorb_mma(const DecodeArgs &a, int ctas, cudaStream_t stream);
 
 } // namespace lla

@@ -1,0 +1,509 @@
+// decode_mma.cu -- LLA decode attention, query-absorbed form, on warp-level tensor cores.
+//
+// "Looped Latent Attention: Cross-Loop KV Compression for Looped Transformers": Pith
+// review page, "What carries the argument" (Eq. 3) and the Pith verdict record's
+// desk-editor letter (absorbed-attention variant):
+//     l_n = q_tilde . c_K[n] + scale * q . mu_t^K,   out = (sum_n p_n c_V[n]) W_up,t^V + mu_t^V.
+// Per (sequence, head) unit the Tq <= 16 loop queries form the 16 rows of an m16n8k16
+// tile, so both contractions of one token tile are tensor-core MMAs:
+//     S[16 x 16 tok]   = Q_tilde[16 x r_k] . C_K^T          (bf16 hi + lo parts of q_tilde)
+//     O[16 x r_v]     += P[16 x 16 tok] . C_V[16 tok x r_v]  (bf16 hi + lo parts of p)
+// The hi/lo split keeps about 16 mantissa bits for q_tilde and p, so the result matches
+// fp32 accumulation to within the parity tolerance while the latents stay exact bf16.
+//
+// Scheduling is the persistent, load-balanced split of decode_sched.cuh.  One thread
+// streams tiles of 128 tokens with 2-D TMA tensor copies (boxes of 16 rows) into a
+// 3-stage mbarrier ring; the swizzled shared layout (32 B rows: 32B swizzle, 64 B rows:
+// 64B swizzle) makes every ldmatrix conflict-free.  Each of the 4 warps owns 32 tokens of
+// a tile: 8 (r_k = 16) MMAs for the scores, an online softmax on the accumulator
+// fragments (row max over a quad of lanes, lazy rescale), then 16 (r_v = 32) MMAs for
+// P.C_V with P taken straight from the score fragments.  At a segment end the 4 warp
+// states are merged through shared memory into one partial record (acc, m, l).
+#include "decode_sched.cuh"
+#include "tmap.cuh"
+
+namespace lla {
+namespace {
+
+constexpr int kWarps = 4;                   // consumer warps (32 tokens of a tile each)
+constexpr int kThreads = (kWarps + 1) * 32; // + one producer warp
+constexpr int kConsumers = kWarps * 32;
+constexpr int kTile = 128;                  // tokens per stage
+constexpr int kStages = 3;
+constexpr int kBox = 32;                    // rows per TMA box
+constexpr float kRescaleThreshold = 8.0f;
+
+__host__ __device__ constexpr int align1024(int x) { return (x + 1023) & ~1023; }
+
+template <int RK, int RV> struct MCfg {
+    static constexpr int KB = RK * 2, VB = RV * 2; // bf16 row bytes
+    static constexpr int KS = RK / 16;             // k16 steps of the score MMA
+    static constexpr int NTV = RV / 8;             // n8 tiles of the output
+    static constexpr int K_BYTES = kTile * KB, V_BYTES = kTile * VB;
+    static constexpr int Q_BYTES = 16 * RK * 4;
+    static constexpr int STAGE = align1024(K_BYTES + V_BYTES + Q_BYTES);
+    static constexpr int RING = kStages * STAGE;
+    static constexpr int MRG_OFF = RING;                                  // [warps][16][RV + 2]
+    static constexpr int DESC_OFF = MRG_OFF + kWarps * 16 * (RV + 2) * 4;
+    static constexpr int BAR_OFF = (DESC_OFF + 15) & ~15;               // full[S], empty[S]
+    static constexpr int MISC_OFF = BAR_OFF + 2 * kStages * 8;
+    static constexpr int SCR_OFF = (MISC_OFF + 16 + 15) & ~15;            // int64 [warps + 1]
+    static constexpr int PREF_OFF = SCR_OFF + (kWarps + 1) * 8;           // int64 [B + 1]
+    static_assert(KB == 32 || KB == 64 || KB == 128, "r_k in {16, 32, 64}");
+    static_assert(VB == 32 || VB == 64 || VB == 128, "r_v in {16, 32, 64}");
+};
+
+// Byte offset of (row, 16-byte chunk) in a tile whose rows are RB bytes, stored by TMA
+// with the RB-byte swizzle (16-byte chunk index XOR address bits 7.. of the row).
+template <int RB> __device__ __forceinline__ uint32_t swz(int row, int chunk)
+{
+    return (uint32_t)(row * RB + 16 * (chunk ^ ((row * RB >> 7) & (RB / 16 - 1))));
+}
+
+__device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t (&r)[4])
+{
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+                 : "r"(addr));
+}
+
+__device__ __forceinline__ void ldsm_x4_t(uint32_t addr, uint32_t (&r)[4])
+{
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+                 : "r"(addr));
+}
+
+__device__ __forceinline__ void mma16816(float (&c)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                         uint32_t b0, uint32_t b1)
+{
+    asm volatile("mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, "
+                 "{%8, %9}, {%0, %1, %2, %3};"
+                 : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+                 : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+__device__ __forceinline__ uint32_t pack_bf16(float lo, float hi)
+{
+    const __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+    return *reinterpret_cast<const uint32_t *>(&v);
+}
+
+// x = hi + lo with hi and lo exactly representable in bf16: hi keeps the top 16 bits of x
+// (truncation), lo = x - hi is exact in fp32 and is truncated to bf16 in turn, so hi + lo
+// carries about 15 mantissa bits of x.  Packs (x0, x1) into two bf16x2 words using only
+// integer/FMA-pipe instructions (byte permutes, masks, subtractions).
+__device__ __forceinline__ uint32_t pack_top16(float a, float b)
+{
+    return __byte_perm(__float_as_uint(a), __float_as_uint(b), 0x7632);
+}
+
+// Round-to-nearest split (hi = bf16(x), lo = bf16(x - hi)): about 17 bits, for q_tilde,
+// whose error scales with the logits.  Used once per unit segment, so cost does not matter.
+__device__ __forceinline__ void split_bf16_rn(float x0, float x1, uint32_t &hi, uint32_t &lo)
+{
+    const __nv_bfloat162 h = __floats2bfloat162_rn(x0, x1);
+    const float2 hf = __bfloat1622float2(h);
+    hi = *reinterpret_cast<const uint32_t *>(&h);
+    lo = pack_bf16(x0 - hf.x, x1 - hf.y);
+}
+
+// Truncating split for the softmax weights p in the hot loop (p <= 2^8, relative error
+// below 2^-14 is far inside the tolerance).
+__device__ __forceinline__ void split_bf16(float x0, float x1, uint32_t &hi, uint32_t &lo)
+{
+    hi = pack_top16(x0, x1);
+    const float h0 = __uint_as_float(__float_as_uint(x0) & 0xffff0000u);
+    const float h1 = __uint_as_float(__float_as_uint(x1) & 0xffff0000u);
+    lo = pack_top16(x0 - h0, x1 - h1);
+}
+
+__device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap *map, int x, int y, uint32_t bar)
+{
+    asm volatile("cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+                 " [%0], [%1, {%2, %3}], [%4];" ::"r"(dst),
+                 "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(bar)
+                 : "memory");
+}
+
+// TQ16: the tile carries more than 8 loop queries, so fragment rows g + 8 are real.
+template <int RK, int RV, bool TQ16>
+__global__ void __launch_bounds__(kThreads, kDecodeCtasPerSm)
+    decode_absorb_mma_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant__ CUtensorMap map_v,
+                             const DecodeArgs a)
+{
+    using C = MCfg<RK, RV>;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
+    float *mrg = reinterpret_cast<float *>(smem + C::MRG_OFF);
+    volatile int *misc = reinterpret_cast<volatile int *>(smem + C::MISC_OFF); // [0] error flag
+    int64_t *pref = reinterpret_cast<int64_t *>(smem + C::PREF_OFF);
+    const uint32_t sbase = smem_u32(smem);
+    const uint32_t full0 = sbase + C::BAR_OFF, empty0 = full0 + 8 * kStages;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int g = lane >> 2, tq = lane & 3; // fragment row group / thread-in-group
+    const int B = a.B, H = a.H, Tq = a.Tq;
+
+    if (tid == 0) {
+        for (int s = 0; s < kStages; ++s) {
+            mbar_init(full0 + 8 * s, 1);       // producer's expect_tx + TMA bytes
+            mbar_init(empty0 + 8 * s, kWarps); // one arrival per consumer warp
+        }
+        misc[0] = 0;
+        fence_barrier_init();
+    }
+    block_length_prefix<kThreads>(a.ctx_lens, B, pref, reinterpret_cast<int64_t *>(smem + C::SCR_OFF));
+    int64_t s0, s1, chunk;
+    cta_share(pref, B, H, a.chunk_min, s0, s1, chunk);
+    if (s0 >= s1)
+        return; // uniform: nothing for this CTA
+
+    // Every warp walks the same tile sequence of this CTA's share, so segment ends (and the
+    // consumer-only barriers at them) happen in the same order in every warp.
+    ShareWalk<kTile> walk;
+    walk.start(s0, s1, chunk);
+    TileDesc d;
+    int issued = 0;
+
+    if (warp == kWarps) {
+        // ================= producer warp: one lane streams the tiles =================
+        if (lane == 0) {
+            bool q_ready = false; // q_tilde comes from the preceding (prologue) grid
+            while (walk.next(pref, a.seq_start, B, H, d)) {
+                const int i = issued, stage = i % kStages;
+                if (i >= kStages && !mbar_wait_bounded(empty0 + 8 * stage, ((i / kStages) - 1) & 1)) {
+                    misc[0] = 1;
+                    break;
+                }
+                if (misc[0])
+                    break;
+                const uint32_t st = sbase + stage * C::STAGE;
+                const int nbox = (d.rows + kBox - 1) / kBox;
+                const uint32_t qb = (d.flags & 1) ? (uint32_t)(Tq * RK * 4) : 0u;
+                const uint32_t bar = full0 + 8 * stage;
+                fence_proxy_async_smem(); // consumers' generic writes to this stage come first
+                mbar_arrive_expect_tx(bar, nbox * kBox * (C::KB + C::VB) + qb);
+                const int y0 = (int)((int64_t)d.h * a.slots + d.row);
+                for (int bx = 0; bx < nbox; ++bx) {
+                    tma_load_2d(st + bx * kBox * C::KB, &map_k, 0, y0 + bx * kBox, bar);
+                    tma_load_2d(st + C::K_BYTES + bx * kBox * C::VB, &map_v, 0, y0 + bx * kBox, bar);
+                }
+                if (qb) {
+                    if (!q_ready) {
+                        grid_dependency_wait();
+                        q_ready = true;
+                    }
+                    bulk_copy_g2s(st + C::K_BYTES + C::V_BYTES, a.qt + ((int64_t)d.u * a.Tq_all + a.tq_off) * RK, qb,
+                                  bar);
+                }
+                ++issued;
+            }
+        }
+    } else {
+        // ================= consumer warps =================
+        uint32_t qa[C::KS][2][4]; // q_tilde A fragments, [k16 step][hi/lo][a0..a3]
+        float o[C::NTV][4];       // output accumulator fragments (rows g, g + 8)
+        float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.f, l1 = 0.f;
+        int i = 0;
+        while (walk.next(pref, a.seq_start, B, H, d)) {
+            const int stage = i % kStages;
+            bool ok = misc[0] == 0 && mbar_wait_bounded(full0 + 8 * stage, (i / kStages) & 1);
+            ok = __all_sync(0xffffffffu, ok);
+            if (!ok)
+                misc[0] = 1;
+            const uint32_t sk = sbase + stage * C::STAGE, sv = sk + C::K_BYTES;
+            if (ok) {
+                // Tokens past the segment in the last active warp's 32-token group (loaded
+                // from beyond the segment, or never written): their p is 0, but 0 * NaN is NaN
+                // in the MMA, so that warp zeroes those value rows.
+                const int r0 = d.rows, r1 = (d.rows + 31) & ~31;
+                if (r0 < r1 && warp == (r0 >> 5)) {
+                    uint4 *vz = reinterpret_cast<uint4 *>(smem + stage * C::STAGE + C::K_BYTES + r0 * C::VB);
+                    for (int e = lane; e < (r1 - r0) * C::VB / 16; e += 32)
+                        vz[e] = make_uint4(0u, 0u, 0u, 0u);
+                    __syncwarp();
+                }
+                if (d.flags & 1) { // new unit segment: its q_tilde, fresh state
+                    const float *qs =
+                        reinterpret_cast<const float *>(smem + stage * C::STAGE + C::K_BYTES + C::V_BYTES);
+#pragma unroll
+                    for (int kk = 0; kk < C::KS; ++kk) {
+                        const int c0 = 16 * kk + 2 * tq;
+                        float x[4][2];
+#pragma unroll
+                        for (int r = 0; r < 2; ++r) { // rows g, g + 8
+                            const int row = g + 8 * r;
+                            const bool in = row < Tq;
+                            x[r][0] = in ? qs[row * RK + c0] : 0.f;
+                            x[r][1] = in ? qs[row * RK + c0 + 1] : 0.f;
+                            x[2 + r][0] = in ? qs[row * RK + c0 + 8] : 0.f;
+                            x[2 + r][1] = in ? qs[row * RK + c0 + 9] : 0.f;
+                        }
+                        // a0: (g, c0..), a1: (g+8, c0..), a2: (g, c0+8..), a3: (g+8, c0+8..)
+#pragma unroll
+                        for (int f = 0; f < 4; ++f)
+                            split_bf16_rn(x[f][0], x[f][1], qa[kk][0][f], qa[kk][1][f]);
+                    }
+#pragma unroll
+                    for (int j = 0; j < C::NTV; ++j)
+                        o[j][0] = o[j][1] = o[j][2] = o[j][3] = 0.f;
+                    m0 = m1 = -INFINITY;
+                    l0 = l1 = 0.f;
+                }
+                const int tbase = warp * 32; // this warp's 32 tokens of the tile
+                if (tbase < d.rows) {
+                    // ---- a2: scores for 32 tokens (4 n8 tiles)
+                    float s[4][4];
+#pragma unroll
+                    for (int j = 0; j < 4; ++j)
+                        s[j][0] = s[j][1] = s[j][2] = s[j][3] = 0.f;
+#pragma unroll
+                    for (int half = 0; half < 2; ++half) {
+                        const int t16 = tbase + 16 * half;
+#pragma unroll
+                        for (int kk = 0; kk < C::KS; ++kk) {
+                            uint32_t kb[4];
+                            const int tok = t16 + ((lane >> 4) << 3) + (lane & 7);
+                            const int ch = 2 * kk + ((lane >> 3) & 1);
+                            ldsm_x4(sk + swz<C::KB>(tok, ch), kb);
+#pragma unroll
+                            for (int hl = 0; hl < 2; ++hl) {
+                                mma16816(s[2 * half], qa[kk][hl][0], qa[kk][hl][1], qa[kk][hl][2], qa[kk][hl][3],
+                                         kb[0], kb[1]);
+                                mma16816(s[2 * half + 1], qa[kk][hl][0], qa[kk][hl][1], qa[kk][hl][2],
+                                         qa[kk][hl][3], kb[2], kb[3]);
+                            }
+                        }
+                    }
+                    if (tbase + 32 > d.rows) {
+#pragma unroll
+                        for (int j = 0; j < 4; ++j) { // mask tokens beyond the tile's rows
+                            const int tok = tbase + 8 * j + 2 * tq;
+                            if (tok >= d.rows)
+                                s[j][0] = s[j][2] = -INFINITY;
+                            if (tok + 1 >= d.rows)
+                                s[j][1] = s[j][3] = -INFINITY;
+                        }
+                    }
+                    // ---- a3: online softmax (log2 domain) for rows g (and g + 8)
+                    float mx0 = -INFINITY, mx1 = -INFINITY;
+#pragma unroll
+                    for (int j = 0; j < 4; ++j) {
+                        mx0 = fmaxf(mx0, fmaxf(s[j][0], s[j][1]));
+                        if constexpr (TQ16)
+                            mx1 = fmaxf(mx1, fmaxf(s[j][2], s[j][3]));
+                    }
+                    mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 1));
+                    mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 2));
+                    if constexpr (TQ16) {
+                        mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 1));
+                        mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 2));
+                    }
+                    if (mx0 > m0 + kRescaleThreshold) {
+                        const float al = fast_exp2(m0 - mx0);
+                        l0 *= al;
+#pragma unroll
+                        for (int j = 0; j < C::NTV; ++j)
+                            o[j][0] *= al, o[j][1] *= al;
+                        m0 = mx0;
+                    }
+                    if constexpr (TQ16) {
+                        if (mx1 > m1 + kRescaleThreshold) {
+                            const float al = fast_exp2(m1 - mx1);
+                            l1 *= al;
+#pragma unroll
+                            for (int j = 0; j < C::NTV; ++j)
+                                o[j][2] *= al, o[j][3] *= al;
+                            m1 = mx1;
+                        }
+                    }
+                    uint32_t pa[2][2][4]; // [k16 step][hi/lo][a0..a3]
+#pragma unroll
+                    for (int j = 0; j < 4; ++j) {
+                        const float p0 = fast_exp2(s[j][0] - m0), p1 = fast_exp2(s[j][1] - m0);
+                        l0 += p0 + p1;
+                        // n8 tile j -> k16 step j/2: a0/a1 for the first tile, a2/a3 for the second
+                        const int ks = j >> 1, f = (j & 1) * 2;
+                        split_bf16(p0, p1, pa[ks][0][f], pa[ks][1][f]);
+                        if constexpr (TQ16) {
+                            const float p2 = fast_exp2(s[j][2] - m1), p3 = fast_exp2(s[j][3] - m1);
+                            l1 += p2 + p3;
+                            split_bf16(p2, p3, pa[ks][0][f + 1], pa[ks][1][f + 1]);
+                        } else {
+                            pa[ks][0][f + 1] = pa[ks][1][f + 1] = 0u; // rows 8..15 are padding
+                        }
+                    }
+                    // ---- O += P . C_V for the 32 tokens
+#pragma unroll
+                    for (int ks = 0; ks < 2; ++ks) {
+                        const int t16 = tbase + 16 * ks;
+#pragma unroll
+                        for (int pr = 0; pr < C::NTV / 2; ++pr) {
+                            uint32_t vb[4];
+                            const int tok = t16 + (((lane >> 3) & 1) << 3) + (lane & 7);
+                            const int ch = 2 * pr + (lane >> 4);
+                            ldsm_x4_t(sv + swz<C::VB>(tok, ch), vb);
+#pragma unroll
+                            for (int hl = 0; hl < 2; ++hl) {
+                                mma16816(o[2 * pr], pa[ks][hl][0], pa[ks][hl][1], pa[ks][hl][2], pa[ks][hl][3], vb[0],
+                                         vb[1]);
+                                mma16816(o[2 * pr + 1], pa[ks][hl][0], pa[ks][hl][1], pa[ks][hl][2], pa[ks][hl][3],
+                                         vb[2], vb[3]);
+                            }
+                        }
+                    }
+                }
+            }
+            __syncwarp();
+            if (lane == 0)
+                mbar_arrive(empty0 + 8 * stage); // this warp is done with the stage
+            if (d.flags & 2) {
+                // ---- segment end: merge the 4 consumer warps' states into one record
+                float lq0 = l0 + __shfl_xor_sync(0xffffffffu, l0, 1);
+                lq0 += __shfl_xor_sync(0xffffffffu, lq0, 2);
+                float lq1 = l1 + __shfl_xor_sync(0xffffffffu, l1, 1);
+                lq1 += __shfl_xor_sync(0xffffffffu, lq1, 2);
+                float *mw = mrg + warp * 16 * (RV + 2);
+#pragma unroll
+                for (int r = 0; r < 2; ++r) {
+                    const int row = g + 8 * r;
+                    if (row < Tq) {
+#pragma unroll
+                        for (int j = 0; j < C::NTV; ++j) {
+                            mw[row * (RV + 2) + 8 * j + 2 * tq] = o[j][2 * r];
+                            mw[row * (RV + 2) + 8 * j + 2 * tq + 1] = o[j][2 * r + 1];
+                        }
+                        if (tq == 0) {
+                            mw[row * (RV + 2) + RV] = r ? m1 : m0;
+                            mw[row * (RV + 2) + RV + 1] = r ? lq1 : lq0;
+                        }
+                    }
+                }
+                asm volatile("bar.sync 1, %0;" ::"r"(kConsumers) : "memory");
+                if (misc[0] == 0 && d.j < a.seg_max) {
+                    for (int idx = tid; idx < Tq * (RV + 2); idx += kConsumers) {
+                        const int row = idx / (RV + 2), jj = idx - row * (RV + 2);
+                        float M = -INFINITY;
+#pragma unroll
+                        for (int w = 0; w < kWarps; ++w)
+                            M = fmaxf(M, mrg[(w * 16 + row) * (RV + 2) + RV]);
+                        float val = 0.f;
+                        if (jj == RV) {
+                            val = M;
+                        } else {
+#pragma unroll
+                            for (int w = 0; w < kWarps; ++w) {
+                                const float mwv = mrg[(w * 16 + row) * (RV + 2) + RV];
+                                if (mwv != -INFINITY)
+                                    val += fast_exp2(mwv - M) * mrg[(w * 16 + row) * (RV + 2) + jj];
+                            }
+                        }
+                        a.part[(((int64_t)d.u * a.Tq_all + a.tq_off + row) * a.seg_max + d.j) * part_stride(RV) + jj] =
+                            val;
+                    }
+                    if (tid == 0 && d.j == 0)
+                        a.counts[d.u] = d.n_u;
+                } else if (tid == 0 && d.j >= a.seg_max) {
+                    report_status(a.status, LLA_ERR_INVALID); // a context longer than max_ctx
+                }
+                asm volatile("bar.sync 1, %0;" ::"r"(kConsumers) : "memory"); // mrg free again
+            }
+            ++i;
+        }
+    }
+    __syncwarp(); // the producer warp's lanes reconverge before the CTA barrier
+    __syncthreads();
+    if (misc[0] != 0 && warp == kWarps && lane == 0) {
+        // wind down: wait (bounded) for this CTA's own copies still in flight
+        report_status(a.status, LLA_ERR_DEVICE_TIMEOUT);
+        for (int i = issued - kStages < 0 ? 0 : issued - kStages; i < issued; ++i)
+            (void)mbar_wait_bounded(full0 + 8 * (i % kStages), (i / kStages) & 1);
+    }
+}
+
+// ---- host ------------------------------------------------------------------------------
+// 2-D map over one layer's latent plane [H' * slots rows][r bf16], boxes of 16 rows.
+bool plane_map(CUtensorMap *map, const void *base, int r, int64_t rows)
+{
+    auto fn = tensor_map_encoder();
+    if (fn == nullptr)
+        return false;
+    const int rb = r * 2;
+    const CUtensorMapSwizzle sw = rb == 32 ? CU_TENSOR_MAP_SWIZZLE_32B
+                                           : (rb == 64 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_128B);
+    const cuuint64_t dims[2] = {(cuuint64_t)r, (cuuint64_t)rows};
+    const cuuint64_t strides[1] = {(cuuint64_t)rb};
+    const cuuint32_t box[2] = {(cuuint32_t)r, (cuuint32_t)kBox};
+    const cuuint32_t estr[2] = {1, 1};
+    return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(base), dims, strides, box, estr,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <int RK, int RV, bool TQ16>
+cudaError_t launch_mma_t(const DecodeArgs &a, int ctas, cudaStream_t stream)
+{
+    using C = MCfg<RK, RV>;
+    const int Hs = a.fold ? 1 : a.H;
+    CUtensorMap mk, mv;
+    if (!plane_map(&mk, a.k, RK, (int64_t)Hs * a.slots) || !plane_map(&mv, a.v, RV, (int64_t)Hs * a.slots))
+        return cudaErrorInvalidValue;
+    auto kern = decode_absorb_mma_kernel<RK, RV, TQ16>;
+    const int smem = C::PREF_OFF + 8 * (a.B + 1) + 1024;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e != cudaSuccess)
+        return e;
+    int dev = 0, sms = 148, occ = 0;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, kern, kThreads, smem);
+    if (e != cudaSuccess)
+        return e;
+    if (occ < 1)
+        return cudaErrorInvalidConfiguration;
+    int grid = sms * occ;
+    if (ctas > 0 && ctas < grid)
+        grid = ctas;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(grid);
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization; // overlap the prologue's tail
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kern, mk, mv, a);
+}
+
+template <int RK, int RV>
+cudaError_t launch_mma(const DecodeArgs &a, int ctas, cudaStream_t stream)
+{
+    return a.Tq > 8 ? launch_mma_t<RK, RV, true>(a, ctas, stream) : launch_mma_t<RK, RV, false>(a, ctas, stream);
+}
+
+} // namespace
+
+bool decode_mma_supported(int dtype, int r_k, int r_v, int fold, int Tq)
+{
+    auto ok = [](int r) { return r == 16 || r == 32 || r == 64; };
+    return dtype == LLA_BF16 && fold == LLA_PER_HEAD && ok(r_k) && ok(r_v) && Tq <= 16 && tensor_map_encoder() != nullptr;
+}
+
+cudaError_t launch_decode_absorb_mma(const DecodeArgs &a, int ctas, cudaStream_t stream)
+{
+#define LLA_MMA_CASE(RK, RV) \
+    if (a.r_k == RK && a.r_v == RV) \
+        return launch_mma<RK, RV>(a, ctas, stream);
+    LLA_MMA_CASE(16, 32)
+    LLA_MMA_CASE(16, 16)
+    LLA_MMA_CASE(32, 32)
+    LLA_MMA_CASE(32, 64)
+    LLA_MMA_CASE(16, 64)
+    LLA_MMA_CASE(64, 64)
+#undef LLA_MMA_CASE
+    return cudaErrorNotSupported;
+}
+
+} // namespace lla

@@ -24,7 +24,7 @@
 //      rotated chunk order so every 16-byte shared load is conflict-free.
 //  a4  decode_combine_kernel: log-sum-exp merge of a unit's records, then
 //      out = o_lat W_up,t^V + mu_t^V and lse.
-#include "decode.cuh"
+#include "decode_sched.cuh"
 
 namespace lla {
 namespace {
@@ -35,20 +35,6 @@ constexpr int kTokensPerThread = 2;
 constexpr int kStages = 3;
 constexpr int kTile = kThreads * kTokensPerThread;
 constexpr float kRescaleThreshold = 8.0f; // log2 units
-
-__device__ __forceinline__ float fast_exp2(float x)
-{
-    float y;
-    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
-    return y;
-}
-
-struct TileDesc {
-    int64_t row;            // first cache row of the tile within the head's plane
-    int32_t b, h, n0, rows; // sequence, head, first token (within the sequence), rows
-    int32_t u, j, n_u;      // unit id, record slot within the unit, records of the unit
-    int32_t flags;          // bit 0: first tile of a segment, bit 1: last tile of a segment
-};
 
 template <typename T, int RK, int RV, int TQ> struct Cfg {
     static constexpr int KB = RK * (int)sizeof(T); // bytes per key-latent row
@@ -78,75 +64,6 @@ __device__ __forceinline__ int chunk_rotation(int row, int nc)
     return nc <= 1 ? 0 : (row / (8 / nc)) % nc;
 }
 
-// Largest b in [0, B) with H * pref[b] <= pos (pref is the exclusive prefix of lengths).
-__device__ __forceinline__ int find_seq(const int64_t *pref, int B, int H, int64_t pos)
-{
-    int lo = 0, hi = B - 1;
-    while (lo < hi) {
-        const int mid = (lo + hi + 1) >> 1;
-        if ((int64_t)H * pref[mid] <= pos)
-            lo = mid;
-        else
-            hi = mid - 1;
-    }
-    return lo;
-}
-
-// Walks the token share [pos, end) of one CTA, unit segment by unit segment, tile by tile.
-struct ShareWalk {
-    int64_t pos, end, chunk, seq0;
-    int32_t b, h, n, seg_end, u, j, n_u;
-    bool in_seg;
-
-    __device__ void start(int64_t p, int64_t e, int64_t ch)
-    {
-        pos = p;
-        end = e;
-        chunk = ch;
-        in_seg = false;
-    }
-    // Next tile; false when the share is exhausted.
-    __device__ bool next(const int64_t *pref, const int64_t *starts, int B, int H, TileDesc &d)
-    {
-        if (!in_seg) {
-            if (pos >= end)
-                return false;
-            b = find_seq(pref, B, H, pos);
-            const int len = (int)(pref[b + 1] - pref[b]);
-            seq0 = starts[b];
-            const int64_t off = pos - (int64_t)H * pref[b];
-            h = (int)(off / len);
-            n = (int)(off - (int64_t)h * len);
-            const int64_t take = min((int64_t)(len - n), end - pos);
-            seg_end = n + (int)take;
-            pos += take;
-            u = b * H + h;
-            const int64_t U = (int64_t)H * pref[b] + (int64_t)h * len; // unit start in the stream
-            const int64_t c_first = U / chunk, c_last = (U + len - 1) / chunk;
-            j = (int)(blockIdx.x - c_first);
-            n_u = (int)(c_last - c_first + 1);
-            in_seg = true;
-            d.flags = 1;
-        } else {
-            d.flags = 0;
-        }
-        d.row = seq0 + n;
-        d.b = b;
-        d.h = h;
-        d.n0 = n;
-        d.rows = min(kTile, seg_end - n);
-        d.u = u;
-        d.j = j;
-        d.n_u = n_u;
-        n += d.rows;
-        if (n >= seg_end) {
-            d.flags |= 2;
-            in_seg = false;
-        }
-        return true;
-    }
-};
-
 template <typename T, int RK, int RV, int TQ>
 __global__ void __launch_bounds__(kThreads, kDecodeCtasPerSm) decode_absorb_kernel(const DecodeArgs a)
 {
@@ -163,55 +80,23 @@ __global__ void __launch_bounds__(kThreads, kDecodeCtasPerSm) decode_absorb_kern
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int B = a.B, H = a.H;
 
-    // ---- exclusive prefix of the context lengths (work split of the token stream):
-    // each thread sums a contiguous slice, a warp scan and a cross-warp offset follow.
-    {
-        const int per = (B + kThreads - 1) / kThreads;
-        const int b0 = min(B, tid * per), b1 = min(B, b0 + per);
-        int64_t local = 0;
-        for (int b = b0; b < b1; ++b)
-            local += a.ctx_lens[b];
-        int64_t x = local;
-#pragma unroll
-        for (int off = 1; off < 32; off <<= 1) {
-            const int64_t y = __shfl_up_sync(0xffffffffu, x, off);
-            if (lane >= off)
-                x += y;
-        }
-        int64_t *wtot = reinterpret_cast<int64_t *>(red);
-        if (lane == 31)
-            wtot[warp] = x;
-        if (tid == 0) {
-            for (int s2 = 0; s2 < kStages; ++s2)
-                mbar_init(bar0 + 8 * s2, 1);
-            misc[1] = 0;
-            fence_barrier_init();
-        }
-        __syncthreads();
-        int64_t run = x - local;
-        for (int w = 0; w < warp; ++w)
-            run += wtot[w];
-        for (int b = b0; b < b1; ++b) {
-            pref[b] = run;
-            run += a.ctx_lens[b];
-        }
-        if (tid == kThreads - 1)
-            pref[B] = run;
+    // ---- work split: prefix of the context lengths, this CTA's token share
+    if (tid == 0) {
+        for (int s2 = 0; s2 < kStages; ++s2)
+            mbar_init(bar0 + 8 * s2, 1);
+        misc[1] = 0;
+        fence_barrier_init();
     }
-    __syncthreads();
-    const int64_t total = (int64_t)H * pref[B];
-    int64_t chunk = (total + gridDim.x - 1) / gridDim.x;
-    if (chunk < a.chunk_min)
-        chunk = a.chunk_min;
-    const int64_t s0 = (int64_t)blockIdx.x * chunk;
-    const int64_t s1 = min(total, s0 + chunk);
+    block_length_prefix<kThreads>(a.ctx_lens, B, pref, reinterpret_cast<int64_t *>(red));
+    int64_t s0, s1, chunk;
+    cta_share(pref, B, H, a.chunk_min, s0, s1, chunk);
     if (s0 >= s1)
         return; // uniform: nothing for this CTA
 
     const T *gk = static_cast<const T *>(a.k);
     const T *gv = static_cast<const T *>(a.v);
     uint8_t *ring = smem;
-    ShareWalk walk; // producer state (thread 0 only)
+    ShareWalk<kTile> walk; // producer state (thread 0 only)
     auto issue = [&](int stage) -> bool {
         TileDesc d;
         if (!walk.next(pref, a.seq_start, B, H, d))
@@ -254,9 +139,17 @@ __global__ void __launch_bounds__(kThreads, kDecodeCtasPerSm) decode_absorb_kern
     int failed_at = -1;
     for (int i = 0; i < ntiles; ++i) {
         const int stage = i % kStages;
-        if (!mbar_wait_bounded(bar0 + 8 * stage, (i / kStages) & 1)) {
+        __syncthreads(); // every thread is done with tile i - 1: its stage may be refilled
+        if (tid == 0 && i >= 1 && i - 1 + kStages < ntiles)
+            issue((i - 1) % kStages);
+        if (!mbar_wait_bounded(bar0 + 8 * stage, (i / kStages) & 1))
             misc[1] = 1; // every writer stores 1
-        } else {
+        __syncthreads(); // all threads agree on the outcome before reading the descriptor
+        if (misc[1]) {
+            failed_at = i;
+            break;
+        }
+        {
             const TileDesc d = descs[stage];
             const uint8_t *sK = ring + stage * C::STAGE;
             const uint8_t *sV = sK + kTile * C::KB;
@@ -409,13 +302,6 @@ __global__ void __launch_bounds__(kThreads, kDecodeCtasPerSm) decode_absorb_kern
                 }
             }
         }
-        __syncthreads();
-        if (misc[1]) {
-            failed_at = i;
-            break;
-        }
-        if (tid == 0 && i + kStages < ntiles)
-            issue(stage);
     }
     if (failed_at >= 0 && tid == 0) {
         // wind down: wait (bounded) for this CTA's own copies still in flight
@@ -461,117 +347,207 @@ cudaError_t launch_tq(const DecodeArgs &a, int ctas, cudaStream_t stream)
 
 // ---------------------------------------------------------------------------------
 // a1: q_tilde[u][tq_off + t][j] = scale * log2(e) * sum_k q[b][t][h][k] W_up,t^K[j][k]
-// grid (B*H, Tq); one warp per latent dimension j.  LLA-2D reads head h's columns.
+// Batched per (head, loop query, chunk of 32 sequences): the loop's W_up,t^K slice of
+// the head (r_k x d, LLA-2D: head h's columns) is staged in shared memory once and
+// serves all 32 sequences.  Thread (sequence, j) runs a d-long dot product.
 // ---------------------------------------------------------------------------------
-template <typename T>
-__global__ void absorb_prologue_kernel(const DecodeArgs a)
+// Copy a rows x cols fp32 matrix (16-byte aligned rows of stride src_ld floats) into
+// shared memory (row stride dst_ld) with all of a thread's loads issued before its stores.
+template <int NT>
+__device__ __forceinline__ void stage_f32(float *dst, int dst_ld, const float *src, int64_t src_ld, int rows, int cols)
 {
-    const int u = blockIdx.x, t = blockIdx.y;
-    const int b = u / a.H, h = u - b * a.H;
-    const int j = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    if (j >= a.r_k)
-        return;
-    const int tg = a.t0 + a.tq_off + t;
-    const int ld = a.fold ? a.H * a.d : a.d;
-    const float *w = a.W_up_k + (a.fold ? ((int64_t)tg * a.r_k + j) * ld + (int64_t)h * a.d
-                                        : (((int64_t)h * a.T + tg) * a.r_k + j) * ld);
-    const T *qrow = static_cast<const T *>(a.q) + (((int64_t)b * a.Tq_all + a.tq_off + t) * a.H + h) * a.d;
-    float acc = 0.f;
-    for (int k = lane; k < a.d; k += 32)
-        acc = fmaf(Elem<T>::to_f(qrow[k]), w[k], acc);
+    const int c4 = cols >> 2, n = rows * c4;
+    for (int base = threadIdx.x; base < n; base += 4 * NT) {
+        float4 v[4];
 #pragma unroll
-    for (int off = 16; off > 0; off >>= 1)
-        acc += __shfl_xor_sync(0xffffffffu, acc, off);
-    if (lane == 0)
-        a.qt[((int64_t)u * a.Tq_all + a.tq_off + t) * a.r_k + j] = acc * a.scale * kLog2e;
+        for (int u = 0; u < 4; ++u) {
+            const int e = base + u * NT;
+            if (e < n) {
+                const int r = e / c4, c = e - r * c4;
+                v[u] = *reinterpret_cast<const float4 *>(src + r * src_ld + 4 * c);
+            }
+        }
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            const int e = base + u * NT;
+            if (e < n) {
+                const int r = e / c4, c = e - r * c4;
+                float *o = dst + r * dst_ld + 4 * c;
+                o[0] = v[u].x, o[1] = v[u].y, o[2] = v[u].z, o[3] = v[u].w;
+            }
+        }
+    }
+}
+
+constexpr int kBatchSeqs = 8;
+constexpr int kPrologueThreads = 128;
+
+template <typename T>
+__global__ void __launch_bounds__(kPrologueThreads) absorb_prologue_kernel(const DecodeArgs a)
+{
+    extern __shared__ float psm[];
+    grid_launch_dependents(); // the decode grid may start streaming latents right away
+    const int h = blockIdx.x, t = blockIdx.y, b0 = blockIdx.z * kBatchSeqs;
+    const int RK = a.r_k, d = a.d, ldw = d + 1;
+    float *W = psm;                       // [RK][d + 1]
+    float *qs = W + RK * ldw;             // [kBatchSeqs][d]
+    const int tg = a.t0 + a.tq_off + t;
+    const int ld = a.fold ? a.H * d : d;
+    const float *wsrc = a.W_up_k + (a.fold ? (int64_t)tg * RK * ld + (int64_t)h * d
+                                           : ((int64_t)h * a.T + tg) * RK * ld);
+    stage_f32<kPrologueThreads>(W, ldw, wsrc, ld, RK, d);
+    const int nb = min(kBatchSeqs, a.B - b0);
+    {
+        // query rows of the chunk, 16-byte loads (8 bf16 or 4 fp32), all issued first
+        constexpr int V = 16 / (int)sizeof(T);
+        const int dv = d / V, n = nb * dv;
+        for (int base = threadIdx.x; base < n; base += 2 * kPrologueThreads) {
+            uint4 raw[2];
+#pragma unroll
+            for (int u = 0; u < 2; ++u) {
+                const int e = base + u * kPrologueThreads;
+                if (e < n) {
+                    const int bl = e / dv, c = e - bl * dv;
+                    raw[u] = *reinterpret_cast<const uint4 *>(
+                        static_cast<const T *>(a.q) + (((int64_t)(b0 + bl) * a.Tq_all + a.tq_off + t) * a.H + h) * d + V * c);
+                }
+            }
+#pragma unroll
+            for (int u = 0; u < 2; ++u) {
+                const int e = base + u * kPrologueThreads;
+                if (e < n) {
+                    const int bl = e / dv, c = e - bl * dv;
+                    const T *vals = reinterpret_cast<const T *>(&raw[u]);
+#pragma unroll
+                    for (int k = 0; k < V; ++k)
+                        qs[bl * d + V * c + k] = Elem<T>::to_f(vals[k]);
+                }
+            }
+        }
+    }
+    __syncthreads();
+    for (int o = threadIdx.x; o < nb * RK; o += kPrologueThreads) {
+        const int bl = o / RK, j = o - bl * RK;
+        const float *qr = qs + bl * d;
+        const float *wr = W + j * ldw;
+        float s0 = 0.f, s1 = 0.f, s2 = 0.f, s3 = 0.f;
+        for (int k = 0; k < d; k += 4) {
+            s0 = fmaf(qr[k], wr[k], s0);
+            s1 = fmaf(qr[k + 1], wr[k + 1], s1);
+            s2 = fmaf(qr[k + 2], wr[k + 2], s2);
+            s3 = fmaf(qr[k + 3], wr[k + 3], s3);
+        }
+        const int64_t u = (int64_t)(b0 + bl) * a.H + h;
+        a.qt[(u * a.Tq_all + a.tq_off + t) * RK + j] = ((s0 + s1) + (s2 + s3)) * a.scale * kLog2e;
+    }
 }
 
 // ---------------------------------------------------------------------------------
-// a4: cross-segment combine + output projection.
-//   M = max_s m_s,  L = sum_s l_s 2^(m_s - M),  o_lat = sum_s acc_s 2^(m_s - M) / L
-//   out = o_lat W_up,t^V + mu_t^V,   lse = ln2 (M + log2 L) + scale * q . mu_t^K
-// One CTA per (loop query, head, sequence); thread k owns output dims k, k+128, ...
+// a4: cross-segment combine + output projection, batched per (head, loop query, chunk
+// of 32 sequences).  For each sequence b of the chunk (one warp per sequence):
+//   M = max_s m_s,  L = sum_s l_s 2^(m_s - M),  o_lat = sum_s acc_s 2^(m_s - M) / L,
+//   lse = ln2 (M + log2 L) + scale * q . mu_t^K   (-inf and out = 0 for an empty context)
+// then out[b] = o_lat[b] W_up,t^V + mu_t^V with W_up,t^V (r_v x d) staged in shared memory.
 // ---------------------------------------------------------------------------------
-constexpr int kCombineThreads = 128;
+constexpr int kCombineThreads = 256; // 8 warps: one sequence each
 
 template <typename T, typename O>
 __global__ void __launch_bounds__(kCombineThreads) decode_combine_kernel(const DecodeArgs a)
 {
-    extern __shared__ float csm[]; // o_lat [r_v], w [seg_max], red [8]
-    const int t = a.tq_off + blockIdx.x, h = blockIdx.y, b = blockIdx.z; // t indexes q/out/lse
-    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const int RV = a.r_v, ps = part_stride(RV);
-    const int u = b * a.H + h;
-    const int len = a.ctx_lens[b];
-    const int S = len > 0 ? min(a.counts[u], a.seg_max) : 0;
-    float *olat = csm;
-    float *w = csm + RV;
-    float *red = w + a.seg_max;
-    const float *rec0 = a.part + ((int64_t)u * a.Tq_all + t) * a.seg_max * ps;
-
-    float Mloc = -INFINITY;
-    for (int s = tid; s < S; s += kCombineThreads)
-        Mloc = fmaxf(Mloc, rec0[s * ps + RV]);
-    for (int off = 16; off > 0; off >>= 1)
-        Mloc = fmaxf(Mloc, __shfl_xor_sync(0xffffffffu, Mloc, off));
-    if (lane == 0)
-        red[warp] = Mloc;
-    __syncthreads();
-    const float M = fmaxf(fmaxf(red[0], red[1]), fmaxf(red[2], red[3]));
-    __syncthreads();
-    float Lloc = 0.f;
-    for (int s = tid; s < S; s += kCombineThreads) {
-        const float ms = rec0[s * ps + RV];
-        const float ws = (ms == -INFINITY) ? 0.f : exp2f(ms - M);
-        w[s] = ws;
-        Lloc += ws * rec0[s * ps + RV + 1];
-    }
-    for (int off = 16; off > 0; off >>= 1)
-        Lloc += __shfl_xor_sync(0xffffffffu, Lloc, off);
-    if (lane == 0)
-        red[warp] = Lloc;
-    __syncthreads();
-    const float L = red[0] + red[1] + red[2] + red[3];
-    const float invL = L > 0.f ? 1.f / L : 0.f;
-    for (int j = tid; j < RV; j += kCombineThreads) {
-        float sum = 0.f;
-        for (int s = 0; s < S; ++s)
-            sum = fmaf(w[s], rec0[s * ps + j], sum);
-        olat[j] = sum * invL;
-    }
-    __syncthreads();
-
-    // output projection; per-head: W_up [H][T][RV][d]; LLA-2D: [T][RV][H*d], cols h*d..
+    extern __shared__ float csm[];
+    const int h = blockIdx.x, tl = blockIdx.y, b0 = blockIdx.z * kBatchSeqs;
+    const int t = a.tq_off + tl; // indexes q / out / lse / records
+    const int RV = a.r_v, d = a.d, ps = part_stride(RV);
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    float *W = csm;                        // [RV][d]
+    float *muv = W + RV * d;               // [d]
+    float *muk = muv + d;                  // [d]
+    float *olat = muk + d;                 // [kBatchSeqs][RV]
+    float *valid = olat + kBatchSeqs * RV; // [kBatchSeqs]
     const int tg = a.t0 + t;
-    const int ld = a.fold ? a.H * a.d : a.d;
-    const int64_t wbase = a.fold ? (int64_t)tg * RV * ld + (int64_t)h * a.d
-                                 : ((int64_t)h * a.T + tg) * RV * ld;
-    const int64_t mbase = a.fold ? (int64_t)tg * ld + (int64_t)h * a.d : ((int64_t)h * a.T + tg) * ld;
-    const T *qrow = static_cast<const T *>(a.q) + (((int64_t)b * a.Tq_all + t) * a.H + h) * a.d;
-    O *orow = static_cast<O *>(a.out) + (((int64_t)b * a.Tq_all + t) * a.H + h) * a.d;
-    float qmu = 0.f;
-    for (int k = tid; k < a.d; k += kCombineThreads) {
-        float o = 0.f;
-        if (L > 0.f) {
-            o = a.mu_v[mbase + k];
-            for (int j = 0; j < RV; ++j)
-                o = fmaf(olat[j], a.W_up_v[wbase + (int64_t)j * ld + k], o);
-        }
-        orow[k] = Elem<O>::from_f(o);
-        qmu = fmaf(Elem<T>::to_f(qrow[k]), a.mu_k[mbase + k], qmu);
+    const int ld = a.fold ? a.H * d : d;
+    const int64_t wbase = a.fold ? (int64_t)tg * RV * ld + (int64_t)h * d : ((int64_t)h * a.T + tg) * RV * ld;
+    const int64_t mbase = a.fold ? (int64_t)tg * ld + (int64_t)h * d : ((int64_t)h * a.T + tg) * ld;
+    stage_f32<kCombineThreads>(W, d, a.W_up_v + wbase, ld, RV, d);
+    for (int k = threadIdx.x; k < d; k += kCombineThreads) {
+        muv[k] = a.mu_v[mbase + k];
+        muk[k] = a.mu_k[mbase + k];
     }
-    if (a.lse != nullptr) {
+    grid_dependency_wait(); // partial records come from the preceding decode grid
+    __syncthreads();
+    const int nb = min(kBatchSeqs, a.B - b0);
+    for (int bl = warp; bl < nb; bl += kCombineThreads / 32) {
+        const int b = b0 + bl;
+        const int64_t u = (int64_t)b * a.H + h;
+        const int len = a.ctx_lens[b];
+        const int S = len > 0 ? min(a.counts[u], a.seg_max) : 0;
+        const float *rec0 = a.part + (u * a.Tq_all + t) * a.seg_max * ps;
+        // lane s holds record s's reference and sum (records beyond 32 folded in a loop)
+        float M = -INFINITY;
+        for (int s = lane; s < S; s += 32)
+            M = fmaxf(M, rec0[s * ps + RV]);
         for (int off = 16; off > 0; off >>= 1)
-            qmu += __shfl_xor_sync(0xffffffffu, qmu, off);
-        __syncthreads();
-        if (lane == 0)
-            red[warp] = qmu;
-        __syncthreads();
-        if (tid == 0) {
-            const float qm = red[0] + red[1] + red[2] + red[3];
-            a.lse[((int64_t)b * a.Tq_all + t) * a.H + h] =
-                L > 0.f ? kLn2 * (M + log2f(L)) + a.scale * qm : -INFINITY;
+            M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, off));
+        float L = 0.f;
+        float acc[8]; // r_v / 32 values per lane (r_v <= 256)
+#pragma unroll
+        for (int q = 0; q < 8; ++q)
+            acc[q] = 0.f;
+        for (int s0 = 0; s0 < S; s0 += 32) {
+            const int s = s0 + lane;
+            float ws = 0.f;
+            if (s < S) {
+                const float ms = rec0[s * ps + RV];
+                ws = ms == -INFINITY ? 0.f : exp2f(ms - M);
+                L += ws * rec0[s * ps + RV + 1];
+            }
+            const int ns = min(32, S - s0);
+            for (int i = 0; i < ns; ++i) {
+                const float wi = __shfl_sync(0xffffffffu, ws, i);
+                const float *ri = rec0 + (s0 + i) * ps;
+#pragma unroll
+                for (int q = 0; q < 8; ++q)
+                    if (lane + 32 * q < RV)
+                        acc[q] = fmaf(wi, ri[lane + 32 * q], acc[q]);
+            }
         }
+        for (int off = 16; off > 0; off >>= 1)
+            L += __shfl_xor_sync(0xffffffffu, L, off);
+        const float invL = L > 0.f ? 1.f / L : 0.f;
+#pragma unroll
+        for (int q = 0; q < 8; ++q)
+            if (lane + 32 * q < RV)
+                olat[bl * RV + lane + 32 * q] = acc[q] * invL;
+        // lse with the constant key-mean term scale * q . mu_t^K
+        const T *qrow = static_cast<const T *>(a.q) + (((int64_t)b * a.Tq_all + t) * a.H + h) * d;
+        float qm = 0.f;
+        for (int k = lane; k < d; k += 32)
+            qm = fmaf(Elem<T>::to_f(qrow[k]), muk[k], qm);
+        for (int off = 16; off > 0; off >>= 1)
+            qm += __shfl_xor_sync(0xffffffffu, qm, off);
+        if (lane == 0) {
+            valid[bl] = L > 0.f ? 1.f : 0.f;
+            if (a.lse != nullptr)
+                a.lse[((int64_t)b * a.Tq_all + t) * a.H + h] = L > 0.f ? kLn2 * (M + log2f(L)) + a.scale * qm : -INFINITY;
+        }
+    }
+    __syncthreads();
+    for (int e = threadIdx.x; e < nb * d; e += kCombineThreads) {
+        const int bl = e / d, k = e - bl * d;
+        float o = 0.f;
+        if (valid[bl] != 0.f) {
+            const float *ol = olat + bl * RV;
+            float o0 = muv[k], o1 = 0.f;
+            int j = 0;
+            for (; j + 1 < RV; j += 2) {
+                o0 = fmaf(ol[j], W[j * d + k], o0);
+                o1 = fmaf(ol[j + 1], W[(j + 1) * d + k], o1);
+            }
+            for (; j < RV; ++j)
+                o0 = fmaf(ol[j], W[j * d + k], o0);
+            o = o0 + o1;
+        }
+        static_cast<O *>(a.out)[(((int64_t)(b0 + bl) * a.Tq_all + t) * a.H + h) * d + k] = Elem<O>::from_f(o);
     }
 }
 
@@ -606,33 +582,57 @@ cudaError_t launch_decode_absorb(const DecodeArgs &a, int dtype, int ctas, cudaS
 
 cudaError_t launch_absorb_prologue(const DecodeArgs &a, int dtype, cudaStream_t stream)
 {
-    if (a.r_k > 32)
+    dim3 grid(a.H, a.Tq, (a.B + kBatchSeqs - 1) / kBatchSeqs);
+    const size_t smem = sizeof(float) * ((size_t)a.r_k * (a.d + 1) + (size_t)kBatchSeqs * a.d);
+    if (smem > 200 * 1024)
         return cudaErrorInvalidValue;
-    dim3 grid(a.B * a.H, a.Tq);
-    const int threads = 32 * a.r_k;
-    if (dtype == LLA_BF16)
-        absorb_prologue_kernel<__nv_bfloat16><<<grid, threads, 0, stream>>>(a);
-    else
-        absorb_prologue_kernel<float><<<grid, threads, 0, stream>>>(a);
+    if (dtype == LLA_BF16) {
+        auto k = absorb_prologue_kernel<__nv_bfloat16>;
+        cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        k<<<grid, kPrologueThreads, smem, stream>>>(a);
+    } else {
+        auto k = absorb_prologue_kernel<float>;
+        cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        k<<<grid, kPrologueThreads, smem, stream>>>(a);
+    }
     return cudaGetLastError();
+}
+
+template <typename T, typename O>
+static cudaError_t launch_combine_t(const DecodeArgs &a, size_t smem, cudaStream_t stream)
+{
+    auto k = decode_combine_kernel<T, O>;
+    cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess)
+        return e;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(a.H, a.Tq, (a.B + kBatchSeqs - 1) / kBatchSeqs);
+    cfg.blockDim = dim3(kCombineThreads);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization; // stage W_up while decode ends
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, k, a);
 }
 
 cudaError_t launch_decode_combine(const DecodeArgs &a, int dtype, int out_dtype, cudaStream_t stream)
 {
-    dim3 grid(a.Tq, a.H, a.B);
-    const size_t smem = sizeof(float) * (a.r_v + a.seg_max + 8);
-    if (smem > 48 * 1024)
+    if (a.r_v > 256)
+        return cudaErrorInvalidValue; // one warp holds r_v / 32 <= 8 values per lane
+    const size_t smem = sizeof(float) * ((size_t)a.r_v * a.d + 2 * a.d + (size_t)kBatchSeqs * (a.r_v + 1));
+    if (smem > 200 * 1024)
         return cudaErrorInvalidValue;
     using BF = __nv_bfloat16;
     if (dtype == LLA_BF16 && out_dtype == LLA_BF16)
-        decode_combine_kernel<BF, BF><<<grid, kCombineThreads, smem, stream>>>(a);
-    else if (dtype == LLA_BF16)
-        decode_combine_kernel<BF, float><<<grid, kCombineThreads, smem, stream>>>(a);
-    else if (out_dtype == LLA_BF16)
-        decode_combine_kernel<float, BF><<<grid, kCombineThreads, smem, stream>>>(a);
-    else
-        decode_combine_kernel<float, float><<<grid, kCombineThreads, smem, stream>>>(a);
-    return cudaGetLastError();
+        return launch_combine_t<BF, BF>(a, smem, stream);
+    if (dtype == LLA_BF16)
+        return launch_combine_t<BF, float>(a, smem, stream);
+    if (out_dtype == LLA_BF16)
+        return launch_combine_t<float, BF>(a, smem, stream);
+    return launch_combine_t<float, float>(a, smem, stream);
 }
 
 } // namespace lla

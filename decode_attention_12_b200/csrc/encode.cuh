@@ -16,6 +16,9 @@ struct EncodeArgs {
 };
 
 cudaError_t launch_encode_simt(const EncodeArgs &a, int dtype, cudaStream_t stream);
+bool encode_tc_supported(const EncodeArgs &a);
+cudaError_t launch_encode_tc(const EncodeArgs &a, cudaStream_t stream);
+void *encode_status_address(); // device address of the encode status word, current device
 cudaError_t launch_codec_bias(const void *Wd, const float *mu, float *bias, int64_t groups, int r, int W,
                               int dtype, cudaStream_t stream);
 

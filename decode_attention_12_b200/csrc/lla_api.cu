@@ -208,7 +208,11 @@ int lla_encode(const lla_dims *dims, int32_t layer0, int32_t n_layers, const voi
     a.T = dims->T; a.H = dims->H; a.d = dims->d_head; a.Hs = heads_stored(dims);
     a.W = (int32_t)stack_width(dims);
     a.r_k = dims->r_k; a.r_v = dims->r_v; a.fold = dims->fold;
-    cudaError_t e = launch_encode_simt(a, dims->dtype, (cudaStream_t)stream);
+    cudaError_t e;
+    if (dims->dtype == LLA_BF16 && encode_tc_supported(a))
+        e = launch_encode_tc(a, (cudaStream_t)stream);   // tcgen05 tensor cores
+    else
+        e = launch_encode_simt(a, dims->dtype, (cudaStream_t)stream);
     return e == cudaSuccess ? LLA_OK : LLA_ERR_CUDA;
 }
 
@@ -255,6 +259,8 @@ int lla_decode_attn(const lla_dims *dims, int32_t layer, int32_t t0, int32_t Tq,
         !aligned16(codec->mu_v) || !aligned16(seq_start) || !aligned16(ctx_lens) ||
         (lse != nullptr && !aligned16(lse)))
         return LLA_ERR_MISALIGNED;
+    if ((dims->d_head * elem_bytes(dims->dtype)) % 16 != 0)
+        return LLA_ERR_UNSUPPORTED; // query / output rows are moved in 16-byte pieces
     const Plan plan = make_plan(dims, B, Tq, max_ctx, num_splits);
     if (workspace == nullptr || ws_bytes < plan.bytes)
         return LLA_ERR_WORKSPACE;
@@ -262,7 +268,8 @@ int lla_decode_attn(const lla_dims *dims, int32_t layer, int32_t t0, int32_t Tq,
         return LLA_ERR_MISALIGNED;
     if (variant != LLA_ABSORB)
         return LLA_ERR_UNSUPPORTED;
-    if (!decode_absorb_supported(dims->dtype, dims->r_k, dims->r_v, dims->d_head, dims->fold))
+    const bool use_mma = decode_mma_supported(dims->dtype, dims->r_k, dims->r_v, dims->fold, Tq);
+    if (!use_mma && !decode_absorb_supported(dims->dtype, dims->r_k, dims->r_v, dims->d_head, dims->fold))
         return LLA_ERR_UNSUPPORTED;
     if (B > 16384)
         return LLA_ERR_UNSUPPORTED;
@@ -297,8 +304,17 @@ int lla_decode_attn(const lla_dims *dims, int32_t layer, int32_t t0, int32_t Tq,
     a.Tq_all = Tq;
     a.tq_off = 0;
     cudaStream_t s = (cudaStream_t)stream;
-    // The CUDA-core kernel serves up to 4 loop queries per pass over the latents.
     cudaError_t err = cudaSuccess;
+    if (use_mma) {
+        // tensor-core kernel: all Tq (<= 16) loop queries in one pass over the latents
+        err = launch_absorb_prologue(a, dims->dtype, s);
+        if (err == cudaSuccess)
+            err = launch_decode_absorb_mma(a, 0, s);
+        if (err == cudaSuccess)
+            err = launch_decode_combine(a, dims->dtype, dims->out_dtype, s);
+        return err == cudaSuccess ? LLA_OK : LLA_ERR_CUDA;
+    }
+    // The CUDA-core kernel serves up to 4 loop queries per pass over the latents.
     for (int32_t c = 0; c < Tq && err == cudaSuccess; c += 4) {
         DecodeArgs ac = a;
         ac.tq_off = c;
@@ -317,8 +333,13 @@ int lla_decode_attn(const lla_dims *dims, int32_t layer, int32_t t0, int32_t Tq,
 
 int lla_status_fetch(void *workspace, lla_stream_t stream, int32_t *status_host)
 {
-    if (workspace == nullptr || status_host == nullptr)
+    if (status_host == nullptr)
         return LLA_ERR_INVALID;
+    if (workspace == nullptr) { // the encode kernels' status word of the current device
+        workspace = encode_status_address();
+        if (workspace == nullptr)
+            return LLA_ERR_CUDA;
+    }
     cudaStream_t s = (cudaStream_t)stream;
     int32_t v = 0;
     if (cudaMemcpyAsync(&v, workspace, sizeof(int32_t), cudaMemcpyDeviceToHost, s) != cudaSuccess)

@@ -195,9 +195,11 @@ int lla_decode_attn_static(const lla_dims *dims, int32_t layer, int32_t t0, int3
                            int32_t num_splits, void *out, float *lse, lla_stream_t stream);
 
 /* ---- status ---------------------------------------------------------------------------
- * Kernels never trap.  A kernel that gives up a bounded wait records
- * LLA_ERR_DEVICE_TIMEOUT in the first word of the decode workspace (sticky).
- * lla_status_fetch synchronises `stream`, copies that word to *status_host and
+ * Kernels never trap.  A decode kernel that gives up a bounded wait records
+ * LLA_ERR_DEVICE_TIMEOUT in the first word of the decode workspace (sticky); the encode
+ * kernels record theirs in a status word inside the library (one per device).
+ * lla_status_fetch synchronises `stream`, copies the decode workspace's word (or, with
+ * workspace == NULL, the current device's encode status word) to *status_host and
  * clears it.  lla_status_string maps any code to a static message.                   */
 int lla_status_fetch(void *workspace, lla_stream_t stream, int32_t *status_host);
 const char *lla_status_string(int code);
