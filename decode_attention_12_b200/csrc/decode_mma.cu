@@ -25,40 +25,65 @@
 namespace lla {
 namespace {
 
-constexpr int kWarps = 4;                   // consumer warps (32 tokens of a tile each)
-constexpr int kThreads = (kWarps + 1) * 32; // + one producer warp
-constexpr int kConsumers = kWarps * 32;
-constexpr int kTile = 128;                  // tokens per stage
-constexpr int kStages = 3;
-constexpr int kBox = 32;                    // rows per TMA box
+constexpr int kBox = 32; // rows per TMA box
 constexpr float kRescaleThreshold = 8.0f;
 
 __host__ __device__ constexpr int align1024(int x) { return (x + 1023) & ~1023; }
 
-template <int RK, int RV> struct MCfg {
-    static constexpr int KB = RK * 2, VB = RV * 2; // bf16 row bytes
-    static constexpr int KS = RK / 16;             // k16 steps of the score MMA
-    static constexpr int NTV = RV / 8;             // n8 tiles of the output
-    static constexpr int K_BYTES = kTile * KB, V_BYTES = kTile * VB;
-    static constexpr int Q_BYTES = 16 * RK * 4;
-    static constexpr int STAGE = align1024(K_BYTES + V_BYTES + Q_BYTES);
-    static constexpr int RING = kStages * STAGE;
-    static constexpr int MRG_OFF = RING;                                  // [warps][16][RV + 2]
-    static constexpr int DESC_OFF = MRG_OFF + kWarps * 16 * (RV + 2) * 4;
-    static constexpr int BAR_OFF = (DESC_OFF + 15) & ~15;               // full[S], empty[S]
-    static constexpr int MISC_OFF = BAR_OFF + 2 * kStages * 8;
-    static constexpr int SCR_OFF = (MISC_OFF + 16 + 15) & ~15;            // int64 [warps + 1]
-    static constexpr int PREF_OFF = SCR_OFF + (kWarps + 1) * 8;           // int64 [B + 1]
-    static_assert(KB == 32 || KB == 64 || KB == 128, "r_k in {16, 32, 64}");
-    static_assert(VB == 32 || VB == 64 || VB == 128, "r_v in {16, 32, 64}");
+// Shared-memory layout of a tile of TILE rows of R bf16 latents.  The columns are cut
+// into NBLK blocks of 64 (128-byte rows, 128B swizzle) and a tail of TAIL = R % 64
+// columns (32- or 64-byte rows with the matching swizzle); each block is a separate
+// TMA box, so every ldmatrix row group touches 8 distinct bank groups.
+template <int R, int TILE> struct TileLayout {
+    static constexpr int NBLK = R / 64;
+    static constexpr int TAIL = R % 64;
+    static constexpr int TB = TAIL * 2; // tail row bytes
+    static constexpr int BYTES = TILE * R * 2;
+    static_assert(TAIL == 0 || TAIL == 16 || TAIL == 32, "rank must be 64k, 64k + 16 or 64k + 32");
+    // byte offset of (row, 16-byte chunk c) in the tile
+    __device__ static __forceinline__ uint32_t off(int row, int c)
+    {
+        if (c < 8 * NBLK)
+            return (uint32_t)((c >> 3) * TILE * 128 + row * 128 + 16 * ((c & 7) ^ (row & 7)));
+        const int cc = c - 8 * NBLK;
+        return (uint32_t)(NBLK * TILE * 128 + row * TB + 16 * (cc ^ ((row * TB >> 7) & (TB / 16 - 1))));
+    }
+    // zero rows [r0, r1) of the tile (all column blocks), lane-strided over one warp
+    __device__ static __forceinline__ void zero_rows(uint8_t *tile, int r0, int r1, int lane)
+    {
+        for (int blk = 0; blk < NBLK; ++blk) {
+            uint4 *z = reinterpret_cast<uint4 *>(tile + blk * TILE * 128 + r0 * 128);
+            for (int e = lane; e < (r1 - r0) * 8; e += 32)
+                z[e] = make_uint4(0u, 0u, 0u, 0u);
+        }
+        if (TAIL) {
+            uint4 *z = reinterpret_cast<uint4 *>(tile + NBLK * TILE * 128 + r0 * TB);
+            for (int e = lane; e < (r1 - r0) * TB / 16; e += 32)
+                z[e] = make_uint4(0u, 0u, 0u, 0u);
+        }
+    }
 };
 
-// Byte offset of (row, 16-byte chunk) in a tile whose rows are RB bytes, stored by TMA
-// with the RB-byte swizzle (16-byte chunk index XOR address bits 7.. of the row).
-template <int RB> __device__ __forceinline__ uint32_t swz(int row, int chunk)
-{
-    return (uint32_t)(row * RB + 16 * (chunk ^ ((row * RB >> 7) & (RB / 16 - 1))));
-}
+// NW consumer warps (32 tokens of a tile each) + one producer warp.
+template <int RK, int RV, int NW> struct MCfg {
+    static constexpr int TILE = 32 * NW;
+    static constexpr int THREADS = (NW + 1) * 32;
+    static constexpr int CONSUMERS = NW * 32;
+    static constexpr int STAGES = (RK + RV) * 2 * TILE > 24 * 1024 ? 2 : 3;
+    using LK = TileLayout<RK, TILE>;
+    using LV = TileLayout<RV, TILE>;
+    static constexpr int KS = RK / 16;  // k16 steps of the score MMA
+    static constexpr int NTV = RV / 8;  // n8 tiles of the output
+    static constexpr int K_BYTES = LK::BYTES, V_BYTES = LV::BYTES;
+    static constexpr int Q_BYTES = 16 * RK * 4;
+    static constexpr int STAGE = align1024(K_BYTES + V_BYTES + Q_BYTES);
+    static constexpr int RING = STAGES * STAGE;
+    static constexpr int MRG_OFF = RING;                              // [NW][16][RV + 2]
+    static constexpr int BAR_OFF = (MRG_OFF + NW * 16 * (RV + 2) * 4 + 15) & ~15; // full[S], empty[S]
+    static constexpr int MISC_OFF = BAR_OFF + 2 * STAGES * 8;
+    static constexpr int SCR_OFF = (MISC_OFF + 16 + 15) & ~15;        // int64 [NW + 1]
+    static constexpr int PREF_OFF = SCR_OFF + (NW + 1) * 8;           // int64 [B + 1]
+};
 
 __device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t (&r)[4])
 {
@@ -127,12 +152,15 @@ __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap *map
 }
 
 // TQ16: the tile carries more than 8 loop queries, so fragment rows g + 8 are real.
-template <int RK, int RV, bool TQ16>
-__global__ void __launch_bounds__(kThreads, kDecodeCtasPerSm)
-    decode_absorb_mma_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant__ CUtensorMap map_v,
+template <int RK, int RV, bool TQ16, int NW, int MINB>
+__global__ void __launch_bounds__((NW + 1) * 32, MINB)
+    decode_absorb_mma_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant__ CUtensorMap map_kt,
+                             const __grid_constant__ CUtensorMap map_v, const __grid_constant__ CUtensorMap map_vt,
                              const DecodeArgs a)
 {
-    using C = MCfg<RK, RV>;
+    using C = MCfg<RK, RV, NW>;
+    constexpr int kWarps = NW, kThreads = C::THREADS, kConsumers = C::CONSUMERS, kTile = C::TILE;
+    constexpr int kStages = C::STAGES;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
     float *mrg = reinterpret_cast<float *>(smem + C::MRG_OFF);
@@ -182,11 +210,24 @@ __global__ void __launch_bounds__(kThreads, kDecodeCtasPerSm)
                 const uint32_t qb = (d.flags & 1) ? (uint32_t)(Tq * RK * 4) : 0u;
                 const uint32_t bar = full0 + 8 * stage;
                 fence_proxy_async_smem(); // consumers' generic writes to this stage come first
-                mbar_arrive_expect_tx(bar, nbox * kBox * (C::KB + C::VB) + qb);
-                const int y0 = (int)((int64_t)d.h * a.slots + d.row);
+                mbar_arrive_expect_tx(bar, nbox * kBox * (RK + RV) * 2 + qb);
+                const int hs = a.fold ? 0 : d.h; // LLA-2D: every head reads the one folded plane
+                const int y0 = (int)((int64_t)hs * a.slots + d.row);
                 for (int bx = 0; bx < nbox; ++bx) {
-                    tma_load_2d(st + bx * kBox * C::KB, &map_k, 0, y0 + bx * kBox, bar);
-                    tma_load_2d(st + C::K_BYTES + bx * kBox * C::VB, &map_v, 0, y0 + bx * kBox, bar);
+                    const int y = y0 + bx * kBox;
+#pragma unroll
+                    for (int blk = 0; blk < C::LK::NBLK; ++blk)
+                        tma_load_2d(st + blk * kTile * 128 + bx * kBox * 128, &map_k, 64 * blk, y, bar);
+                    if (C::LK::TAIL)
+                        tma_load_2d(st + C::LK::NBLK * kTile * 128 + bx * kBox * C::LK::TB, &map_kt,
+                                    64 * C::LK::NBLK, y, bar);
+                    const uint32_t sv0 = st + C::K_BYTES;
+#pragma unroll
+                    for (int blk = 0; blk < C::LV::NBLK; ++blk)
+                        tma_load_2d(sv0 + blk * kTile * 128 + bx * kBox * 128, &map_v, 64 * blk, y, bar);
+                    if (C::LV::TAIL)
+                        tma_load_2d(sv0 + C::LV::NBLK * kTile * 128 + bx * kBox * C::LV::TB, &map_vt,
+                                    64 * C::LV::NBLK, y, bar);
                 }
                 if (qb) {
                     if (!q_ready) {
@@ -218,9 +259,7 @@ __global__ void __launch_bounds__(kThreads, kDecodeCtasPerSm)
                 // in the MMA, so that warp zeroes those value rows.
                 const int r0 = d.rows, r1 = (d.rows + 31) & ~31;
                 if (r0 < r1 && warp == (r0 >> 5)) {
-                    uint4 *vz = reinterpret_cast<uint4 *>(smem + stage * C::STAGE + C::K_BYTES + r0 * C::VB);
-                    for (int e = lane; e < (r1 - r0) * C::VB / 16; e += 32)
-                        vz[e] = make_uint4(0u, 0u, 0u, 0u);
+                    C::LV::zero_rows(smem + stage * C::STAGE + C::K_BYTES, r0, r1, lane);
                     __syncwarp();
                 }
                 if (d.flags & 1) { // new unit segment: its q_tilde, fresh state
@@ -265,7 +304,7 @@ __global__ void __launch_bounds__(kThreads, kDecodeCtasPerSm)
                             uint32_t kb[4];
                             const int tok = t16 + ((lane >> 4) << 3) + (lane & 7);
                             const int ch = 2 * kk + ((lane >> 3) & 1);
-                            ldsm_x4(sk + swz<C::KB>(tok, ch), kb);
+                            ldsm_x4(sk + C::LK::off(tok, ch), kb);
 #pragma unroll
                             for (int hl = 0; hl < 2; ++hl) {
                                 mma16816(s[2 * half], qa[kk][hl][0], qa[kk][hl][1], qa[kk][hl][2], qa[kk][hl][3],
@@ -342,7 +381,7 @@ __global__ void __launch_bounds__(kThreads, kDecodeCtasPerSm)
                             uint32_t vb[4];
                             const int tok = t16 + (((lane >> 3) & 1) << 3) + (lane & 7);
                             const int ch = 2 * pr + (lane >> 4);
-                            ldsm_x4_t(sv + swz<C::VB>(tok, ch), vb);
+                            ldsm_x4_t(sv + C::LV::off(tok, ch), vb);
 #pragma unroll
                             for (int hl = 0; hl < 2; ++hl) {
                                 mma16816(o[2 * pr], pa[ks][hl][0], pa[ks][hl][1], pa[ks][hl][2], pa[ks][hl][3], vb[0],
@@ -422,33 +461,51 @@ __global__ void __launch_bounds__(kThreads, kDecodeCtasPerSm)
 }
 
 // ---- host ------------------------------------------------------------------------------
-// 2-D map over one layer's latent plane [H' * slots rows][r bf16], boxes of 16 rows.
-bool plane_map(CUtensorMap *map, const void *base, int r, int64_t rows)
+// 2-D map over one layer's latent plane [rows][r bf16]: boxes of `cols` columns x 32 rows
+// with the swizzle that matches the box's row bytes.
+bool plane_map(CUtensorMap *map, const void *base, int r, int64_t rows, int cols)
 {
     auto fn = tensor_map_encoder();
     if (fn == nullptr)
         return false;
-    const int rb = r * 2;
+    const int rb = cols * 2;
     const CUtensorMapSwizzle sw = rb == 32 ? CU_TENSOR_MAP_SWIZZLE_32B
                                            : (rb == 64 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_128B);
     const cuuint64_t dims[2] = {(cuuint64_t)r, (cuuint64_t)rows};
-    const cuuint64_t strides[1] = {(cuuint64_t)rb};
-    const cuuint32_t box[2] = {(cuuint32_t)r, (cuuint32_t)kBox};
+    const cuuint64_t strides[1] = {(cuuint64_t)r * 2};
+    const cuuint32_t box[2] = {(cuuint32_t)cols, (cuuint32_t)kBox};
     const cuuint32_t estr[2] = {1, 1};
     return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(base), dims, strides, box, estr,
               CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <int RK, int RV, bool TQ16>
+// Maps for the 64-column blocks and the tail of one plane (an unused map is a copy).
+bool plane_maps(CUtensorMap *main, CUtensorMap *tail, const void *base, int r, int64_t rows)
+{
+    const int nblk = r / 64, t = r % 64;
+    bool ok = true;
+    if (nblk > 0)
+        ok = ok && plane_map(main, base, r, rows, 64);
+    if (t > 0)
+        ok = ok && plane_map(tail, base, r, rows, t);
+    if (nblk == 0)
+        *main = *tail;
+    if (t == 0)
+        *tail = *main;
+    return ok;
+}
+
+template <int RK, int RV, bool TQ16, int NW, int MINB>
 cudaError_t launch_mma_t(const DecodeArgs &a, int ctas, cudaStream_t stream)
 {
-    using C = MCfg<RK, RV>;
+    using C = MCfg<RK, RV, NW>;
     const int Hs = a.fold ? 1 : a.H;
-    CUtensorMap mk, mv;
-    if (!plane_map(&mk, a.k, RK, (int64_t)Hs * a.slots) || !plane_map(&mv, a.v, RV, (int64_t)Hs * a.slots))
+    CUtensorMap mk, mkt, mv, mvt;
+    if (!plane_maps(&mk, &mkt, a.k, RK, (int64_t)Hs * a.slots) ||
+        !plane_maps(&mv, &mvt, a.v, RV, (int64_t)Hs * a.slots))
         return cudaErrorInvalidValue;
-    auto kern = decode_absorb_mma_kernel<RK, RV, TQ16>;
+    auto kern = decode_absorb_mma_kernel<RK, RV, TQ16, NW, MINB>;
     const int smem = C::PREF_OFF + 8 * (a.B + 1) + 1024;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess)
@@ -456,7 +513,7 @@ cudaError_t launch_mma_t(const DecodeArgs &a, int ctas, cudaStream_t stream)
     int dev = 0, sms = 148, occ = 0;
     cudaGetDevice(&dev);
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, kern, kThreads, smem);
+    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, kern, C::THREADS, smem);
     if (e != cudaSuccess)
         return e;
     if (occ < 1)
@@ -466,7 +523,7 @@ cudaError_t launch_mma_t(const DecodeArgs &a, int ctas, cudaStream_t stream)
         grid = ctas;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(grid);
-    cfg.blockDim = dim3(kThreads);
+    cfg.blockDim = dim3(C::THREADS);
     cfg.dynamicSmemBytes = smem;
     cfg.stream = stream;
     cudaLaunchAttribute attr[1];
@@ -474,21 +531,28 @@ cudaError_t launch_mma_t(const DecodeArgs &a, int ctas, cudaStream_t stream)
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, kern, mk, mv, a);
+    return cudaLaunchKernelEx(&cfg, kern, mk, mkt, mv, mvt, a);
 }
 
+// Small ranks: 128-token tiles, 4 consumer warps, 4 CTAs per SM.  Ranks >= 64: 64-token
+// tiles, 2 consumer warps, 2 CTAs per SM (larger register and shared-memory footprint).
 template <int RK, int RV>
 cudaError_t launch_mma(const DecodeArgs &a, int ctas, cudaStream_t stream)
 {
-    return a.Tq > 8 ? launch_mma_t<RK, RV, true>(a, ctas, stream) : launch_mma_t<RK, RV, false>(a, ctas, stream);
+    constexpr bool big = RK >= 64 || RV >= 64;
+    constexpr int NW = big ? 2 : 4, MINB = big ? 2 : 4;
+    return a.Tq > 8 ? launch_mma_t<RK, RV, true, NW, MINB>(a, ctas, stream)
+                    : launch_mma_t<RK, RV, false, NW, MINB>(a, ctas, stream);
 }
 
 } // namespace
 
 bool decode_mma_supported(int dtype, int r_k, int r_v, int fold, int Tq)
 {
-    auto ok = [](int r) { return r == 16 || r == 32 || r == 64; };
-    return dtype == LLA_BF16 && fold == LLA_PER_HEAD && ok(r_k) && ok(r_v) && Tq <= 16 && tensor_map_encoder() != nullptr;
+    (void)Tq; // more than 16 loop queries run as passes of 16
+    const bool pair = (r_k == 16 && r_v == 32) || (r_k == 16 && r_v == 16) || (r_k == 32 && r_v == 32) ||
+                      (r_k == 64 && r_v == 128) || (r_k == 96 && r_v == 160) || (r_k == 128 && r_v == 128);
+    return dtype == LLA_BF16 && pair && tensor_map_encoder() != nullptr;
 }
 
 cudaError_t launch_decode_absorb_mma(const DecodeArgs &a, int ctas, cudaStream_t stream)
@@ -499,9 +563,9 @@ cudaError_t launch_decode_absorb_mma(const DecodeArgs &a, int ctas, cudaStream_t
     LLA_MMA_CASE(16, 32)
     LLA_MMA_CASE(16, 16)
     LLA_MMA_CASE(32, 32)
-    LLA_MMA_CASE(32, 64)
-    LLA_MMA_CASE(16, 64)
-    LLA_MMA_CASE(64, 64)
+    LLA_MMA_CASE(64, 128)
+    LLA_MMA_CASE(96, 160)
+    LLA_MMA_CASE(128, 128)
 #undef LLA_MMA_CASE
     return cudaErrorNotSupported;
 }

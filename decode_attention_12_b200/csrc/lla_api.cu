@@ -306,12 +306,17 @@ int lla_decode_attn(const lla_dims *dims, int32_t layer, int32_t t0, int32_t Tq,
     cudaStream_t s = (cudaStream_t)stream;
     cudaError_t err = cudaSuccess;
     if (use_mma) {
-        // tensor-core kernel: all Tq (<= 16) loop queries in one pass over the latents
-        err = launch_absorb_prologue(a, dims->dtype, s);
-        if (err == cudaSuccess)
-            err = launch_decode_absorb_mma(a, 0, s);
-        if (err == cudaSuccess)
-            err = launch_decode_combine(a, dims->dtype, dims->out_dtype, s);
+        // tensor-core kernel: up to 16 loop queries (one m16 tile) per pass over the latents
+        for (int32_t c = 0; c < Tq && err == cudaSuccess; c += 16) {
+            DecodeArgs ac = a;
+            ac.tq_off = c;
+            ac.Tq = Tq - c < 16 ? Tq - c : 16;
+            err = launch_absorb_prologue(ac, dims->dtype, s);
+            if (err == cudaSuccess)
+                err = launch_decode_absorb_mma(ac, 0, s);
+            if (err == cudaSuccess)
+                err = launch_decode_combine(ac, dims->dtype, dims->out_dtype, s);
+        }
         return err == cudaSuccess ? LLA_OK : LLA_ERR_CUDA;
     }
     // The CUDA-core kernel serves up to 4 loop queries per pass over the latents.

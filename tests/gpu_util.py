@@ -88,3 +88,46 @@ def assert_attn_close(out_gpu, lse_gpu, o_ref, lse_ref):
         d = np.abs(l[fin] - lse_ref[fin]).max()
         assert d <= LSE_ATOL, f"lse max-abs {d:.3e}"
     return max_abs, rel
+
+
+def oracle_decode_units(p, w, layer, t0, Tq, scale, units, variant="absorb", q=None, threads=None):
+    """Oracle on sampled (b, h) units only: their latent rows are gathered to the host.
+
+    Works for caches far larger than host memory; the result arrays are NaN outside
+    ``units``.  Uses the same stored inputs as the GPU run.
+    """
+    q = p["q"] if q is None else q
+    q64 = to64(q)
+    B, _, H, d = q64.shape
+    o = np.full((B, Tq, H, d), np.nan)
+    lse = np.full((B, Tq, H), np.nan)
+    WK, WV = to64(p["W_up_k"][layer]), to64(p["W_up_v"][layer])
+    mK, mV = to64(p["mu_k"][layer]), to64(p["mu_v"][layer])
+    if w.fold2d:
+        WK, WV, mK, mV = WK[0], WV[0], mK[0], mV[0]
+    for (b, h) in units:
+        s0, n = int(p["starts"][b]), int(p["lens"][b])
+        hp = 0 if w.fold2d else h
+        cK = to64(p["k"][layer, hp, s0:s0 + n])[None]
+        cV = to64(p["v"][layer, hp, s0:s0 + n])[None]
+        if w.fold2d:
+            ob, lb = oracle.decode_layer(variant, q64[b:b + 1], cK, cV, [0], [n], WK, mK, WV, mV, t0, scale,
+                                         fold2d=True, units=[(0, h)], threads=1)
+        else:
+            sel = [h]
+            ob, lb = oracle.decode_layer(variant, q64[b:b + 1, :, sel], cK, cV, [0], [n], WK[sel], mK[sel],
+                                         WV[sel], mV[sel], t0, scale, fold2d=False, threads=1)
+            o[b, :, h] = ob[0, :, 0]
+            lse[b, :, h] = lb[0, :, 0]
+            continue
+        o[b, :, h] = ob[0, :, h]
+        lse[b, :, h] = lb[0, :, h]
+    return o, lse
+
+
+def sample_units(B, H, n, seed=0):
+    rng = np.random.default_rng(seed)
+    units = {(0, 0), (B - 1, H - 1)}
+    while len(units) < min(n, B * H):
+        units.add((int(rng.integers(0, B)), int(rng.integers(0, H))))
+    return sorted(units)

@@ -52,7 +52,7 @@ def _check(w, p, layer, x, axis, rows, slot_of_row):
     return err
 
 
-@pytest.mark.parametrize("name", ["tiny-fp32", "ouro1.4b-layer", "rho4-prefill"])
+@pytest.mark.parametrize("name", ["tiny-fp32", "ouro1.4b-layer", "rho4-prefill", "deep-T32", "lla2d"])
 def test_encode_matches_oracle(name):
     w = S.WORKLOADS[name]
     if w.L > 1:
@@ -122,3 +122,21 @@ def test_codec_bias_matches_definition():
                 ref = oracle.encode(np.zeros((1, Wd.shape[-1])), mu[l, h], Wd[l, h].T)[0]
                 got = to64(p[f"bias_{axis}"][l, h])
                 np.testing.assert_allclose(got, ref, rtol=1e-6, atol=1e-6)
+
+
+def test_prefill_encode_full_layer_sampled_rows():
+    """rho4-prefill: one layer of the full prefill (32 x 4096 tokens x 16 heads, K and V),
+    checked on sampled token rows."""
+    w = S.WORKLOADS["rho4-prefill"]
+    n_tok = w.B * 4096
+    layer = w.L - 1
+    p = _setup(w, [layer], n_tok)
+    xk = S.draw_encode_tokens(w, layer, "k", n_tok, DEV)
+    xv = S.draw_encode_tokens(w, layer, "v", n_tok, DEV)
+    slot_idx = torch.arange(n_tok, device=DEV)
+    lla.encode(dims_of(w), layer, 1, xk, xv, n_tok, slot_idx, _codec(p), _cache(p, n_tok))
+    torch.cuda.synchronize()
+    assert lla.status_fetch(None) == 0
+    rows = np.unique(np.concatenate([[0, n_tok - 1], np.random.default_rng(5).integers(0, n_tok, 62)]))
+    for axis, x in (("k", xk), ("v", xv)):
+        _check(w, p, layer, x, axis, rows, rows)
