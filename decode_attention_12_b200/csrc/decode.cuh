@@ -20,6 +20,7 @@ struct DecodeArgs {
     int32_t B, H, d, T, t0, Tq, fold, r_k, r_v;
     int32_t Tq_all, tq_off;   // q/out/lse/records hold Tq_all loop queries; this pass
                               // serves queries tq_off .. tq_off+Tq-1 (loop t0 + tq_off + i)
+    int32_t recon;            // records hold d-wide reconstruct-form outputs (no projection)
     int32_t seg_max;          // partial-record slots per (unit, query)
     int32_t chunk_min;        // smallest token share of one decode CTA
     float scale;              // softmax scale
@@ -47,5 +48,7 @@ cudaError_t launch_decode_combine(const DecodeArgs &a, int dtype, int out_dtype,
 bool decode_absorb_supported(int dtype, int r_k, int r_v, int d, int fold);
 bool decode_mma_supported(int dtype, int r_k, int r_v, int fold, int Tq);
 cudaError_t launch_decode_absorb_mma(const DecodeArgs &a, int ctas, cudaStream_t stream);
+bool decode_reconstruct_supported(int dtype, int r_k, int r_v, int d);
+cudaError_t launch_decode_reconstruct(const DecodeArgs &a, cudaStream_t stream);
 
 } // namespace lla

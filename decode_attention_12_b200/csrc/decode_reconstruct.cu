@@ -1,0 +1,418 @@
+// decode_reconstruct.cu -- LLA decode attention, reconstruct-on-read form.
+//
+// "Looped Latent Attention: Cross-Loop KV Compression for Looped Transformers": Pith
+// review page, "What carries the argument" (Eq. 3: loop t reads x_hat_t = c W_up,t + mu_t)
+// and arXiv abstract (K/V vectors are reconstructed only when attention reads them).
+// For one loop t this kernel rebuilds, per 32-token slice of every latent tile,
+//     K_hat^T [d x 32] = W_up,t^K^T [d x r_k] . C_K^T   (+ mu_t^K),
+//     V_hat^T [d x 32] = W_up,t^V^T [d x r_v] . C_V^T   (+ mu_t^V)
+// on warp-level tensor cores (m16n8k16, d rows as M, bf16 hi/lo parts of W_up,t), and
+// runs plain flash decoding on the rebuilt vectors: the scores q . k_hat come from the
+// K_hat fragments, and O^T [d x 1] += V_hat^T . p is another MMA (V_hat and p split
+// into bf16 hi/lo parts).  It costs about d flop per latent byte per loop against the
+// absorbed form's ~1, which is the Pith verdict record's desk-editor point that the
+// latent store read this way is compute-bound.  It exists for that comparison.
+//
+// One launch serves one loop query (Tq = 1); the host launches it per loop.  The
+// scheduling (persistent token shares, producer warp, swizzled TMA tiles) is the one
+// of the absorbed kernel; each CTA stages W_up,t (transposed, bf16 hi/lo), mu_t and q_t
+// of a unit in shared memory when a segment of that unit starts.  Records hold the
+// d-wide output, so the combine kernel only merges them.
+#include "mma_common.cuh"
+
+namespace lla {
+namespace {
+using namespace mma;
+
+constexpr int kWarps = 4;
+constexpr int kThreads = (kWarps + 1) * 32;
+constexpr int kConsumers = kWarps * 32;
+constexpr int kTile = 128;
+constexpr int kStages = 3;
+
+template <int RK, int RV, int D> struct RCfg {
+    using LK = TileLayout<RK, kTile>;
+    using LV = TileLayout<RV, kTile>;
+    static constexpr int MD = D / 16;       // m16 tiles over the head dimension
+    static constexpr int KSK = RK / 16, KSV = RV / 16;
+    static constexpr int WK_LD = RK * 2 + 16; // padded bf16 row bytes of W_up^K^T (conflict-free ldmatrix)
+    static constexpr int WV_LD = RV * 2 + 16;
+    static constexpr int STAGE = align1024(LK::BYTES + LV::BYTES);
+    static constexpr int RING = kStages * STAGE;
+    static constexpr int WK_OFF = RING;                      // [2 hi/lo][D][WK_LD bytes]
+    static constexpr int WV_OFF = WK_OFF + 2 * D * WK_LD;    // [2 hi/lo][D][WV_LD bytes]
+    static constexpr int VEC_OFF = WV_OFF + 2 * D * WV_LD;   // q[D], mu_k[D], mu_v[D] fp32, qmu
+    static constexpr int MRG_OFF = VEC_OFF + (3 * D + 4) * 4; // [warps][D + 2]
+    static constexpr int BAR_OFF = (MRG_OFF + kWarps * (D + 2) * 4 + 15) & ~15;
+    static constexpr int MISC_OFF = BAR_OFF + 2 * kStages * 8;
+    static constexpr int SCR_OFF = (MISC_OFF + 16 + 15) & ~15;
+    static constexpr int PREF_OFF = SCR_OFF + (kWarps + 1) * 8;
+};
+
+template <int RK, int RV, int D>
+__global__ void __launch_bounds__(kThreads, 2)
+    decode_reconstruct_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant__ CUtensorMap map_kt,
+                              const __grid_constant__ CUtensorMap map_v, const __grid_constant__ CUtensorMap map_vt,
+                              const DecodeArgs a)
+{
+    using C = RCfg<RK, RV, D>;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
+    float *vq = reinterpret_cast<float *>(smem + C::VEC_OFF);
+    float *vmk = vq + D, *vmv = vq + 2 * D, *vqmu = vq + 3 * D;
+    float *mrg = reinterpret_cast<float *>(smem + C::MRG_OFF);
+    volatile int *misc = reinterpret_cast<volatile int *>(smem + C::MISC_OFF);
+    int64_t *pref = reinterpret_cast<int64_t *>(smem + C::PREF_OFF);
+    const uint32_t sbase = smem_u32(smem);
+    const uint32_t full0 = sbase + C::BAR_OFF, empty0 = full0 + 8 * kStages;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int g = lane >> 2, tq = lane & 3;
+    const int B = a.B, H = a.H;
+    const int tl = a.t0 + a.tq_off; // the loop this launch serves
+
+    if (tid == 0) {
+        for (int s = 0; s < kStages; ++s) {
+            mbar_init(full0 + 8 * s, 1);
+            mbar_init(empty0 + 8 * s, kWarps);
+        }
+        misc[0] = 0;
+        fence_barrier_init();
+    }
+    block_length_prefix<kThreads>(a.ctx_lens, B, pref, reinterpret_cast<int64_t *>(smem + C::SCR_OFF));
+    int64_t s0, s1, chunk;
+    cta_share(pref, B, H, a.chunk_min, s0, s1, chunk);
+    if (s0 >= s1)
+        return;
+
+    ShareWalk<kTile> walk;
+    walk.start(s0, s1, chunk);
+    TileDesc d;
+    int issued = 0;
+
+    if (warp == kWarps) {
+        if (lane == 0) { // producer: stream the latent tiles
+            while (walk.next(pref, a.seq_start, B, H, d)) {
+                const int i = issued, stage = i % kStages;
+                if (i >= kStages && !mbar_wait_bounded(empty0 + 8 * stage, ((i / kStages) - 1) & 1)) {
+                    misc[0] = 1;
+                    break;
+                }
+                if (misc[0])
+                    break;
+                const uint32_t st = sbase + stage * C::STAGE, sv0 = st + C::LK::BYTES;
+                const int nbox = (d.rows + kBox - 1) / kBox;
+                const uint32_t bar = full0 + 8 * stage;
+                fence_proxy_async_smem();
+                mbar_arrive_expect_tx(bar, nbox * kBox * (RK + RV) * 2);
+                const int y0 = (int)((int64_t)(a.fold ? 0 : d.h) * a.slots + d.row);
+                for (int bx = 0; bx < nbox; ++bx) {
+                    const int y = y0 + bx * kBox;
+#pragma unroll
+                    for (int blk = 0; blk < C::LK::NBLK; ++blk)
+                        tma_load_2d(st + blk * kTile * 128 + bx * kBox * 128, &map_k, 64 * blk, y, bar);
+                    if (C::LK::TAIL)
+                        tma_load_2d(st + C::LK::NBLK * kTile * 128 + bx * kBox * C::LK::TB, &map_kt, 64 * C::LK::NBLK,
+                                    y, bar);
+#pragma unroll
+                    for (int blk = 0; blk < C::LV::NBLK; ++blk)
+                        tma_load_2d(sv0 + blk * kTile * 128 + bx * kBox * 128, &map_v, 64 * blk, y, bar);
+                    if (C::LV::TAIL)
+                        tma_load_2d(sv0 + C::LV::NBLK * kTile * 128 + bx * kBox * C::LV::TB, &map_vt, 64 * C::LV::NBLK,
+                                    y, bar);
+                }
+                ++issued;
+            }
+        }
+    } else {
+        float o[C::MD][4]; // O^T fragments: rows d = 16 md + g (+8), column 0 real (tq == 0)
+        float m = -INFINITY, l = 0.f;
+        int i = 0;
+        while (walk.next(pref, a.seq_start, B, H, d)) {
+            const int stage = i % kStages;
+            if (d.flags & 1) {
+                // ---- new unit segment: stage W_up,t^T (bf16 hi/lo), mu_t, scaled q_t
+                const int ld = a.fold ? a.H * D : D;
+                const int64_t col0 = a.fold ? (int64_t)d.h * D : 0;
+                const float *wk = a.W_up_k + (a.fold ? (int64_t)tl * RK * ld : ((int64_t)d.h * a.T + tl) * RK * ld) + col0;
+                const float *wv = a.W_up_v + (a.fold ? (int64_t)tl * RV * ld : ((int64_t)d.h * a.T + tl) * RV * ld) + col0;
+                const float *mk = a.mu_k + (a.fold ? (int64_t)tl * ld : ((int64_t)d.h * a.T + tl) * ld) + col0;
+                const float *mv = a.mu_v + (a.fold ? (int64_t)tl * ld : ((int64_t)d.h * a.T + tl) * ld) + col0;
+                for (int e = tid; e < D * RK; e += kConsumers) { // read [j][k] coalesced, store [k][j]
+                    const int j = e / D, k = e - j * D;
+                    const float x = wk[(int64_t)j * ld + k];
+                    const __nv_bfloat16 hi = __float2bfloat16_rn(x);
+                    const __nv_bfloat16 lo = __float2bfloat16_rn(x - __bfloat162float(hi));
+                    *reinterpret_cast<__nv_bfloat16 *>(smem + C::WK_OFF + k * C::WK_LD + 2 * j) = hi;
+                    *reinterpret_cast<__nv_bfloat16 *>(smem + C::WK_OFF + D * C::WK_LD + k * C::WK_LD + 2 * j) = lo;
+                }
+                for (int e = tid; e < D * RV; e += kConsumers) {
+                    const int j = e / D, k = e - j * D;
+                    const float x = wv[(int64_t)j * ld + k];
+                    const __nv_bfloat16 hi = __float2bfloat16_rn(x);
+                    const __nv_bfloat16 lo = __float2bfloat16_rn(x - __bfloat162float(hi));
+                    *reinterpret_cast<__nv_bfloat16 *>(smem + C::WV_OFF + k * C::WV_LD + 2 * j) = hi;
+                    *reinterpret_cast<__nv_bfloat16 *>(smem + C::WV_OFF + D * C::WV_LD + k * C::WV_LD + 2 * j) = lo;
+                }
+                const __nv_bfloat16 *qrow =
+                    static_cast<const __nv_bfloat16 *>(a.q) + (((int64_t)d.b * a.Tq_all + a.tq_off) * a.H + d.h) * D;
+                for (int k = tid; k < D; k += kConsumers) {
+                    vq[k] = __bfloat162float(qrow[k]) * a.scale * kLog2e;
+                    vmk[k] = mk[k];
+                    vmv[k] = mv[k];
+                }
+                asm volatile("bar.sync 1, %0;" ::"r"(kConsumers) : "memory");
+                if (warp == 0) { // constant score term q . mu_t^K (log2 units)
+                    float qm = 0.f;
+                    for (int k = lane; k < D; k += 32)
+                        qm = fmaf(vq[k], vmk[k], qm);
+#pragma unroll
+                    for (int off = 16; off > 0; off >>= 1)
+                        qm += __shfl_xor_sync(0xffffffffu, qm, off);
+                    if (lane == 0)
+                        vqmu[0] = qm;
+                }
+                asm volatile("bar.sync 1, %0;" ::"r"(kConsumers) : "memory");
+#pragma unroll
+                for (int md = 0; md < C::MD; ++md)
+                    o[md][0] = o[md][1] = o[md][2] = o[md][3] = 0.f;
+                m = -INFINITY;
+                l = 0.f;
+            }
+            bool ok = misc[0] == 0 && mbar_wait_bounded(full0 + 8 * stage, (i / kStages) & 1);
+            ok = __all_sync(0xffffffffu, ok);
+            if (!ok)
+                misc[0] = 1;
+            const uint32_t sk = sbase + stage * C::STAGE, sv = sk + C::LK::BYTES;
+            const int tbase = warp * 32;
+            if (ok && tbase < d.rows) {
+                const int r0 = d.rows, r1 = (d.rows + 31) & ~31;
+                if (r0 < r1 && warp == (r0 >> 5)) { // 0 * NaN guard for rows past the segment
+                    C::LV::zero_rows(smem + stage * C::STAGE + C::LK::BYTES, r0, r1, lane);
+                    C::LK::zero_rows(smem + stage * C::STAGE, r0, r1, lane);
+                    __syncwarp();
+                }
+                // B fragments of C_K^T and C_V^T for the warp's 32 tokens
+                uint32_t kb[2][C::KSK][4], vb[2][C::KSV][4];
+#pragma unroll
+                for (int half = 0; half < 2; ++half) {
+                    const int tok = tbase + 16 * half + ((lane >> 4) << 3) + (lane & 7);
+#pragma unroll
+                    for (int kk = 0; kk < C::KSK; ++kk)
+                        ldsm_x4(sk + C::LK::off(tok, 2 * kk + ((lane >> 3) & 1)), kb[half][kk]);
+#pragma unroll
+                    for (int kv = 0; kv < C::KSV; ++kv)
+                        ldsm_x4(sv + C::LV::off(tok, 2 * kv + ((lane >> 3) & 1)), vb[half][kv]);
+                }
+                // ---- scores: s[tok] = q . (K_hat[tok]) over d, from K_hat^T fragments
+                float sp[4][2];
+#pragma unroll
+                for (int n = 0; n < 4; ++n)
+                    sp[n][0] = sp[n][1] = 0.f;
+#pragma unroll
+                for (int md = 0; md < C::MD; ++md) {
+                    float acc[4][4];
+#pragma unroll
+                    for (int n = 0; n < 4; ++n)
+                        acc[n][0] = acc[n][1] = acc[n][2] = acc[n][3] = 0.f;
+#pragma unroll
+                    for (int kk = 0; kk < C::KSK; ++kk) {
+#pragma unroll
+                        for (int hl = 0; hl < 2; ++hl) {
+                            uint32_t wa[4];
+                            const int row = 16 * md + (lane & 15);
+                            ldsm_x4(sbase + C::WK_OFF + hl * D * C::WK_LD + row * C::WK_LD + 32 * kk + 16 * (lane >> 4), wa);
+                            // ldmatrix x4 order: (rows 0-7, k 0-7), (rows 8-15, k 0-7), (rows 0-7, k 8-15), (rows 8-15, k 8-15)
+#pragma unroll
+                            for (int half = 0; half < 2; ++half) {
+                                mma16816(acc[2 * half], wa[0], wa[1], wa[2], wa[3], kb[half][kk][0], kb[half][kk][1]);
+                                mma16816(acc[2 * half + 1], wa[0], wa[1], wa[2], wa[3], kb[half][kk][2], kb[half][kk][3]);
+                            }
+                        }
+                    }
+                    const float q0 = vq[16 * md + g], q1 = vq[16 * md + g + 8];
+#pragma unroll
+                    for (int n = 0; n < 4; ++n) {
+                        sp[n][0] = fmaf(q0, acc[n][0], fmaf(q1, acc[n][2], sp[n][0]));
+                        sp[n][1] = fmaf(q0, acc[n][1], fmaf(q1, acc[n][3], sp[n][1]));
+                    }
+                }
+#pragma unroll
+                for (int n = 0; n < 4; ++n)
+#pragma unroll
+                    for (int c = 0; c < 2; ++c) {
+                        float x = sp[n][c];
+                        x += __shfl_xor_sync(0xffffffffu, x, 4);
+                        x += __shfl_xor_sync(0xffffffffu, x, 8);
+                        x += __shfl_xor_sync(0xffffffffu, x, 16);
+                        sp[n][c] = x + vqmu[0];
+                        if (tbase + 8 * n + 2 * tq + c >= d.rows)
+                            sp[n][c] = -INFINITY;
+                    }
+                // ---- online softmax over the 32 scores (one query row)
+                float mx = -INFINITY;
+#pragma unroll
+                for (int n = 0; n < 4; ++n)
+                    mx = fmaxf(mx, fmaxf(sp[n][0], sp[n][1]));
+                mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
+                mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
+                if (mx > m + 8.0f) {
+                    const float al = fast_exp2(m - mx);
+                    l *= al;
+#pragma unroll
+                    for (int md = 0; md < C::MD; ++md)
+                        o[md][0] *= al, o[md][1] *= al, o[md][2] *= al, o[md][3] *= al;
+                    m = mx;
+                }
+                uint32_t pb[2][2][2]; // [k16 step][hi/lo][b0/b1], column 0 only (lanes g == 0)
+#pragma unroll
+                for (int n = 0; n < 4; ++n) {
+                    const float p0 = fast_exp2(sp[n][0] - m), p1 = fast_exp2(sp[n][1] - m);
+                    l += p0 + p1;
+                    uint32_t h, lo;
+                    split_bf16(p0, p1, h, lo);
+                    pb[n >> 1][0][n & 1] = g == 0 ? h : 0u;
+                    pb[n >> 1][1][n & 1] = g == 0 ? lo : 0u;
+                }
+                // ---- V_hat^T per d tile, then O^T += V_hat^T . p
+#pragma unroll
+                for (int md = 0; md < C::MD; ++md) {
+                    float acc[4][4];
+#pragma unroll
+                    for (int n = 0; n < 4; ++n)
+                        acc[n][0] = acc[n][1] = acc[n][2] = acc[n][3] = 0.f;
+#pragma unroll
+                    for (int kv = 0; kv < C::KSV; ++kv) {
+#pragma unroll
+                        for (int hl = 0; hl < 2; ++hl) {
+                            uint32_t wa[4];
+                            const int row = 16 * md + (lane & 15);
+                            ldsm_x4(sbase + C::WV_OFF + hl * D * C::WV_LD + row * C::WV_LD + 32 * kv + 16 * (lane >> 4), wa);
+#pragma unroll
+                            for (int half = 0; half < 2; ++half) {
+                                mma16816(acc[2 * half], wa[0], wa[1], wa[2], wa[3], vb[half][kv][0], vb[half][kv][1]);
+                                mma16816(acc[2 * half + 1], wa[0], wa[1], wa[2], wa[3], vb[half][kv][2], vb[half][kv][3]);
+                            }
+                        }
+                    }
+                    const float mu0 = vmv[16 * md + g], mu1 = vmv[16 * md + g + 8];
+#pragma unroll
+                    for (int ks = 0; ks < 2; ++ks) {
+                        uint32_t ah[4], al[4]; // V_hat^T A fragments (rows d, cols tokens of k16 step ks)
+                        split_bf16(acc[2 * ks][0] + mu0, acc[2 * ks][1] + mu0, ah[0], al[0]);
+                        split_bf16(acc[2 * ks][2] + mu1, acc[2 * ks][3] + mu1, ah[1], al[1]);
+                        split_bf16(acc[2 * ks + 1][0] + mu0, acc[2 * ks + 1][1] + mu0, ah[2], al[2]);
+                        split_bf16(acc[2 * ks + 1][2] + mu1, acc[2 * ks + 1][3] + mu1, ah[3], al[3]);
+                        mma16816(o[md], ah[0], ah[1], ah[2], ah[3], pb[ks][0][0], pb[ks][0][1]);
+                        mma16816(o[md], ah[0], ah[1], ah[2], ah[3], pb[ks][1][0], pb[ks][1][1]);
+                        mma16816(o[md], al[0], al[1], al[2], al[3], pb[ks][0][0], pb[ks][0][1]);
+                    }
+                }
+            }
+            __syncwarp();
+            if (lane == 0)
+                mbar_arrive(empty0 + 8 * stage);
+            if (d.flags & 2) {
+                // ---- segment end: merge the warps into one d-wide record
+                float lq = l + __shfl_xor_sync(0xffffffffu, l, 1);
+                lq += __shfl_xor_sync(0xffffffffu, lq, 2);
+                float *mw = mrg + warp * (D + 2);
+                if (tq == 0) {
+#pragma unroll
+                    for (int md = 0; md < C::MD; ++md) {
+                        mw[16 * md + g] = o[md][0];
+                        mw[16 * md + g + 8] = o[md][2];
+                    }
+                }
+                if (lane == 0) {
+                    mw[D] = m;
+                    mw[D + 1] = lq;
+                }
+                asm volatile("bar.sync 1, %0;" ::"r"(kConsumers) : "memory");
+                if (misc[0] == 0 && d.j < a.seg_max) {
+                    float M = -INFINITY;
+#pragma unroll
+                    for (int w = 0; w < kWarps; ++w)
+                        M = fmaxf(M, mrg[w * (D + 2) + D]);
+                    for (int jj = tid; jj < D + 2; jj += kConsumers) {
+                        float val = 0.f;
+                        if (jj == D) {
+                            val = M;
+                        } else {
+#pragma unroll
+                            for (int w = 0; w < kWarps; ++w) {
+                                const float mwv = mrg[w * (D + 2) + D];
+                                if (mwv != -INFINITY)
+                                    val += fast_exp2(mwv - M) * mrg[w * (D + 2) + jj];
+                            }
+                        }
+                        a.part[(((int64_t)d.u * a.Tq_all + a.tq_off) * a.seg_max + d.j) * part_stride(D) + jj] = val;
+                    }
+                    if (tid == 0 && d.j == 0)
+                        a.counts[d.u] = d.n_u;
+                } else if (tid == 0 && d.j >= a.seg_max) {
+                    report_status(a.status, LLA_ERR_INVALID);
+                }
+                asm volatile("bar.sync 1, %0;" ::"r"(kConsumers) : "memory");
+            }
+            ++i;
+        }
+    }
+    __syncwarp();
+    __syncthreads();
+    if (misc[0] != 0 && warp == kWarps && lane == 0) {
+        report_status(a.status, LLA_ERR_DEVICE_TIMEOUT);
+        for (int i = issued - kStages < 0 ? 0 : issued - kStages; i < issued; ++i)
+            (void)mbar_wait_bounded(full0 + 8 * (i % kStages), (i / kStages) & 1);
+    }
+}
+
+template <int RK, int RV, int D>
+cudaError_t launch_rec(const DecodeArgs &a, cudaStream_t stream)
+{
+    using C = RCfg<RK, RV, D>;
+    const int Hs = a.fold ? 1 : a.H;
+    CUtensorMap mk, mkt, mv, mvt;
+    if (!plane_maps(&mk, &mkt, a.k, RK, (int64_t)Hs * a.slots) ||
+        !plane_maps(&mv, &mvt, a.v, RV, (int64_t)Hs * a.slots))
+        return cudaErrorInvalidValue;
+    auto kern = decode_reconstruct_kernel<RK, RV, D>;
+    const int smem = C::PREF_OFF + 8 * (a.B + 1) + 1024;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e != cudaSuccess)
+        return e;
+    int dev = 0, sms = 148, occ = 0;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, kern, kThreads, smem);
+    if (e != cudaSuccess)
+        return e;
+    if (occ < 1)
+        return cudaErrorInvalidConfiguration;
+    kern<<<sms * occ, kThreads, smem, stream>>>(mk, mkt, mv, mvt, a);
+    return cudaGetLastError();
+}
+
+} // namespace
+
+bool decode_reconstruct_supported(int dtype, int r_k, int r_v, int d)
+{
+    return dtype == LLA_BF16 && (r_k == 16 || r_k == 32) && (r_v == 16 || r_v == 32) && (d == 64 || d == 128) &&
+           tensor_map_encoder() != nullptr;
+}
+
+cudaError_t launch_decode_reconstruct(const DecodeArgs &a, cudaStream_t stream)
+{
+#define LLA_REC_CASE(RK, RV, D) \
+    if (a.r_k == RK && a.r_v == RV && a.d == D) \
+        return launch_rec<RK, RV, D>(a, stream);
+    LLA_REC_CASE(16, 32, 128)
+    LLA_REC_CASE(16, 16, 128)
+    LLA_REC_CASE(32, 32, 128)
+    LLA_REC_CASE(16, 32, 64)
+    LLA_REC_CASE(32, 32, 64)
+    LLA_REC_CASE(16, 16, 64)
+#undef LLA_REC_CASE
+    return cudaErrorNotSupported;
+}
+
+} // namespace lla

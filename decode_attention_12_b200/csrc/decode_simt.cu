@@ -451,13 +451,15 @@ __global__ void __launch_bounds__(kPrologueThreads) absorb_prologue_kernel(const
 // ---------------------------------------------------------------------------------
 constexpr int kCombineThreads = 256; // 8 warps: one sequence each
 
-template <typename T, typename O>
+// REC: records carry d-wide outputs of the reconstruct form (mu and the q.mu_t^K score term
+// already included), so the output is the merged record itself.
+template <typename T, typename O, bool REC>
 __global__ void __launch_bounds__(kCombineThreads) decode_combine_kernel(const DecodeArgs a)
 {
     extern __shared__ float csm[];
     const int h = blockIdx.x, tl = blockIdx.y, b0 = blockIdx.z * kBatchSeqs;
     const int t = a.tq_off + tl; // indexes q / out / lse / records
-    const int RV = a.r_v, d = a.d, ps = part_stride(RV);
+    const int d = a.d, RV = REC ? a.d : a.r_v, ps = part_stride(RV);
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     float *W = csm;                        // [RV][d]
     float *muv = W + RV * d;               // [d]
@@ -468,10 +470,12 @@ __global__ void __launch_bounds__(kCombineThreads) decode_combine_kernel(const D
     const int ld = a.fold ? a.H * d : d;
     const int64_t wbase = a.fold ? (int64_t)tg * RV * ld + (int64_t)h * d : ((int64_t)h * a.T + tg) * RV * ld;
     const int64_t mbase = a.fold ? (int64_t)tg * ld + (int64_t)h * d : ((int64_t)h * a.T + tg) * ld;
-    stage_f32<kCombineThreads>(W, d, a.W_up_v + wbase, ld, RV, d);
-    for (int k = threadIdx.x; k < d; k += kCombineThreads) {
-        muv[k] = a.mu_v[mbase + k];
-        muk[k] = a.mu_k[mbase + k];
+    if (!REC) {
+        stage_f32<kCombineThreads>(W, d, a.W_up_v + wbase, ld, RV, d);
+        for (int k = threadIdx.x; k < d; k += kCombineThreads) {
+            muv[k] = a.mu_v[mbase + k];
+            muk[k] = a.mu_k[mbase + k];
+        }
     }
     grid_dependency_wait(); // partial records come from the preceding decode grid
     __syncthreads();
@@ -518,13 +522,15 @@ __global__ void __launch_bounds__(kCombineThreads) decode_combine_kernel(const D
         for (int q = 0; q < 8; ++q)
             if (lane + 32 * q < RV)
                 olat[bl * RV + lane + 32 * q] = acc[q] * invL;
-        // lse with the constant key-mean term scale * q . mu_t^K
-        const T *qrow = static_cast<const T *>(a.q) + (((int64_t)b * a.Tq_all + t) * a.H + h) * d;
+        // lse with the constant key-mean term scale * q . mu_t^K (absorbed form only)
         float qm = 0.f;
-        for (int k = lane; k < d; k += 32)
-            qm = fmaf(Elem<T>::to_f(qrow[k]), muk[k], qm);
-        for (int off = 16; off > 0; off >>= 1)
-            qm += __shfl_xor_sync(0xffffffffu, qm, off);
+        if (!REC) {
+            const T *qrow = static_cast<const T *>(a.q) + (((int64_t)b * a.Tq_all + t) * a.H + h) * d;
+            for (int k = lane; k < d; k += 32)
+                qm = fmaf(Elem<T>::to_f(qrow[k]), muk[k], qm);
+            for (int off = 16; off > 0; off >>= 1)
+                qm += __shfl_xor_sync(0xffffffffu, qm, off);
+        }
         if (lane == 0) {
             valid[bl] = L > 0.f ? 1.f : 0.f;
             if (a.lse != nullptr)
@@ -535,7 +541,9 @@ __global__ void __launch_bounds__(kCombineThreads) decode_combine_kernel(const D
     for (int e = threadIdx.x; e < nb * d; e += kCombineThreads) {
         const int bl = e / d, k = e - bl * d;
         float o = 0.f;
-        if (valid[bl] != 0.f) {
+        if (REC) {
+            o = valid[bl] != 0.f ? olat[bl * RV + k] : 0.f;
+        } else if (valid[bl] != 0.f) {
             const float *ol = olat + bl * RV;
             float o0 = muv[k], o1 = 0.f;
             int j = 0;
@@ -601,7 +609,7 @@ cudaError_t launch_absorb_prologue(const DecodeArgs &a, int dtype, cudaStream_t 
 template <typename T, typename O>
 static cudaError_t launch_combine_t(const DecodeArgs &a, size_t smem, cudaStream_t stream)
 {
-    auto k = decode_combine_kernel<T, O>;
+    auto k = a.recon ? decode_combine_kernel<T, O, true> : decode_combine_kernel<T, O, false>;
     cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess)
         return e;
@@ -620,9 +628,10 @@ static cudaError_t launch_combine_t(const DecodeArgs &a, size_t smem, cudaStream
 
 cudaError_t launch_decode_combine(const DecodeArgs &a, int dtype, int out_dtype, cudaStream_t stream)
 {
-    if (a.r_v > 256)
-        return cudaErrorInvalidValue; // one warp holds r_v / 32 <= 8 values per lane
-    const size_t smem = sizeof(float) * ((size_t)a.r_v * a.d + 2 * a.d + (size_t)kBatchSeqs * (a.r_v + 1));
+    const int rv = a.recon ? a.d : a.r_v;
+    if (rv > 256)
+        return cudaErrorInvalidValue; // one warp holds (record width) / 32 <= 8 values per lane
+    const size_t smem = sizeof(float) * ((size_t)rv * a.d + 2 * a.d + (size_t)kBatchSeqs * (rv + 1));
     if (smem > 200 * 1024)
         return cudaErrorInvalidValue;
     using BF = __nv_bfloat16;

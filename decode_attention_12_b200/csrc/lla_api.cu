@@ -66,7 +66,7 @@ struct Plan {
 
 size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
 
-Plan make_plan(const lla_dims *d, int32_t B, int32_t Tq, int32_t max_ctx, int32_t num_splits)
+Plan make_plan(const lla_dims *d, int32_t B, int32_t Tq, int32_t max_ctx, int32_t num_splits, int32_t variant)
 {
     Plan p;
     const int64_t units = (int64_t)B * d->H;
@@ -81,7 +81,9 @@ Plan make_plan(const lla_dims *d, int32_t B, int32_t Tq, int32_t max_ctx, int32_
     p.off_counts = kWorkspaceHeader;
     p.off_qt = align256(p.off_counts + (size_t)units * sizeof(int32_t));
     p.off_part = align256(p.off_qt + (size_t)units * Tq * d->r_k * sizeof(float));
-    p.bytes = p.off_part + (size_t)units * Tq * p.seg_max * part_stride(d->r_v) * sizeof(float);
+    // reconstruct-form records carry d-wide outputs, absorbed-form records r_v-wide latents
+    const int rec_w = variant == LLA_RECONSTRUCT ? d->d_head : d->r_v;
+    p.bytes = p.off_part + (size_t)units * Tq * p.seg_max * part_stride(rec_w) * sizeof(float);
     return p;
 }
 
@@ -225,7 +227,7 @@ int lla_decode_num_splits(const lla_dims *dims, int32_t B, int32_t Tq, int32_t m
     if (B < 0 || Tq < 1 || max_ctx < 0 || num_splits < 0 ||
         (variant != LLA_ABSORB && variant != LLA_RECONSTRUCT))
         return LLA_ERR_INVALID;
-    return make_plan(dims, B, Tq, max_ctx, num_splits).seg_max;
+    return make_plan(dims, B, Tq, max_ctx, num_splits, variant).seg_max;
 }
 
 size_t lla_decode_workspace_bytes(const lla_dims *dims, int32_t B, int32_t Tq, int32_t max_ctx,
@@ -233,7 +235,7 @@ size_t lla_decode_workspace_bytes(const lla_dims *dims, int32_t B, int32_t Tq, i
 {
     if (lla_decode_num_splits(dims, B, Tq, max_ctx, variant, num_splits) < 1)
         return 0;
-    return make_plan(dims, B, Tq, max_ctx, num_splits).bytes;
+    return make_plan(dims, B, Tq, max_ctx, num_splits, variant).bytes;
 }
 
 int lla_decode_attn(const lla_dims *dims, int32_t layer, int32_t t0, int32_t Tq, const void *q,
@@ -261,12 +263,13 @@ int lla_decode_attn(const lla_dims *dims, int32_t layer, int32_t t0, int32_t Tq,
         return LLA_ERR_MISALIGNED;
     if ((dims->d_head * elem_bytes(dims->dtype)) % 16 != 0)
         return LLA_ERR_UNSUPPORTED; // query / output rows are moved in 16-byte pieces
-    const Plan plan = make_plan(dims, B, Tq, max_ctx, num_splits);
+    const Plan plan = make_plan(dims, B, Tq, max_ctx, num_splits, variant);
     if (workspace == nullptr || ws_bytes < plan.bytes)
         return LLA_ERR_WORKSPACE;
     if (!aligned16(workspace))
         return LLA_ERR_MISALIGNED;
-    if (variant != LLA_ABSORB)
+    if (variant == LLA_RECONSTRUCT &&
+        !decode_reconstruct_supported(dims->dtype, dims->r_k, dims->r_v, dims->d_head))
         return LLA_ERR_UNSUPPORTED;
     const bool use_mma = decode_mma_supported(dims->dtype, dims->r_k, dims->r_v, dims->fold, Tq);
     if (!use_mma && !decode_absorb_supported(dims->dtype, dims->r_k, dims->r_v, dims->d_head, dims->fold))
@@ -290,6 +293,7 @@ int lla_decode_attn(const lla_dims *dims, int32_t layer, int32_t t0, int32_t Tq,
     a.mu_v = codec->mu_v + (int64_t)layer * Hs * dims->T * Dp;
     a.B = B; a.H = dims->H; a.d = dims->d_head; a.T = dims->T; a.t0 = t0; a.Tq = Tq;
     a.fold = dims->fold; a.r_k = dims->r_k; a.r_v = dims->r_v;
+    a.recon = variant == LLA_RECONSTRUCT;
     a.seg_max = plan.seg_max;
     a.chunk_min = plan.chunk_min;
     a.scale = softmax_scale;
@@ -305,6 +309,18 @@ int lla_decode_attn(const lla_dims *dims, int32_t layer, int32_t t0, int32_t Tq,
     a.tq_off = 0;
     cudaStream_t s = (cudaStream_t)stream;
     cudaError_t err = cudaSuccess;
+    if (variant == LLA_RECONSTRUCT) {
+        // one pass over the latents per loop query, then one merge of all records
+        for (int32_t c = 0; c < Tq && err == cudaSuccess; ++c) {
+            DecodeArgs ac = a;
+            ac.tq_off = c;
+            ac.Tq = 1;
+            err = launch_decode_reconstruct(ac, s);
+        }
+        if (err == cudaSuccess)
+            err = launch_decode_combine(a, dims->dtype, dims->out_dtype, s);
+        return err == cudaSuccess ? LLA_OK : LLA_ERR_CUDA;
+    }
     if (use_mma) {
         // tensor-core kernel: up to 16 loop queries (one m16 tile) per pass over the latents
         for (int32_t c = 0; c < Tq && err == cudaSuccess; c += 16) {
