@@ -35,7 +35,14 @@ sys.path.insert(0, ROOT)
 METRIC = "LLA decode latent-cache GB/s & token-loop reads/s (% of HBM roofline) at 1 B200"
 WORKLOAD = "ouro1.4b-layer"
 SPEC_HBM_GBS = 8000.0
-PROFILE_TRAFFIC = os.path.join(ROOT, "profiles", "decode_absorb_simt.ouro1.4b-layer.json")
+PROFILE_TRAFFIC = {
+    "absorb": os.path.join(ROOT, "profiles", "decode_absorb_mma.ouro1.4b-layer.json"),
+    "reconstruct": os.path.join(ROOT, "profiles", "decode_reconstruct.ouro1.4b-layer.json"),
+}
+KERNEL_SOURCES = {
+    "absorb": ("decode_mma.cu", "mma_common.cuh", "decode_sched.cuh", "decode.cuh", "common.cuh"),
+    "reconstruct": ("decode_reconstruct.cu", "mma_common.cuh", "decode_sched.cuh", "decode.cuh", "common.cuh"),
+}
 
 
 def parse():
@@ -49,6 +56,12 @@ def parse():
     ap.add_argument("--replicas", type=int, default=3)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
+    ap.add_argument("--variant", default="absorb", choices=["absorb", "reconstruct"],
+                    help="decode read form (the headline uses absorb)")
+    ap.add_argument("--phase", default="step", choices=["step", "encode"],
+                    help="step: decode step (headline); encode: prefill encode of one layer")
+    ap.add_argument("--encode-seqs", type=int, default=0,
+                    help="--phase encode: sequences of len_hi tokens to encode (default: B)")
     return ap.parse_args()
 
 
@@ -60,26 +73,37 @@ def measured_peaks():
         return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0}, "fallback"
 
 
-def kernel_source_hash():
+def kernel_source_hash(variant="absorb"):
+    """Hash of the decode kernel's sources: a profile taken on other sources is stale."""
     h = hashlib.sha256()
-    for rel in ("decode_attention_12_b200/csrc/decode_simt.cu", "decode_attention_12_b200/csrc/decode.cuh",
-                "decode_attention_12_b200/csrc/common.cuh"):
-        with open(os.path.join(ROOT, rel), "rb") as f:
+    for name in KERNEL_SOURCES[variant]:
+        with open(os.path.join(ROOT, "decode_attention_12_b200", "csrc", name), "rb") as f:
             h.update(f.read())
     return h.hexdigest()[:16]
 
 
-def profiled_traffic(units_per_launch):
+def profiled_traffic(units_per_launch, variant="absorb"):
     """DRAM bytes per launch from the committed ncu summary, or None if stale/absent."""
     try:
-        with open(PROFILE_TRAFFIC) as f:
+        with open(PROFILE_TRAFFIC[variant]) as f:
             prof = json.load(f)
     except (OSError, ValueError):
         return None
-    if prof.get("source_hash") != kernel_source_hash():
+    if prof.get("source_hash") != kernel_source_hash(variant):
         return None
     per_unit = prof["dram_bytes_per_launch"] / prof["units_per_launch"]
     return per_unit * units_per_launch
+
+
+def max_over_ranks(value: float, device) -> float:
+    """Largest value over all ranks of the default process group (plain value at N = 1)."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return float(value)
+    t = torch.tensor([float(value)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
 
 
 # ---------------------------------------------------------------------------
@@ -214,6 +238,73 @@ def run_reference(args, rank):
 
 
 # ---------------------------------------------------------------------------
+# --phase encode: prefill encode of one layer (write path, tcgen05 for bf16)
+# ---------------------------------------------------------------------------
+def run_encode_phase(args, dev):
+    import torch
+    import decode_attention_12_b200 as lla
+    import lla_synth as S
+
+    w = S.WORKLOADS[args.workload]
+    n_seq = args.encode_seqs or w.B
+    n_tok = n_seq * w.len_hi
+    layer = w.L - 1
+    p = S.decode_inputs(w, layer, dev, lens=[1], Tq=1)
+    dims = lla.make_dims(w.T, w.L, w.H, w.d, w.r_k, w.r_v, int(w.fold2d),
+                         lla.F32 if w.dtype == "f32" else lla.BF16)
+    bias_k = torch.zeros(w.L, w.heads_stored, w.r_k, device=dev)
+    bias_v = torch.zeros(w.L, w.heads_stored, w.r_v, device=dev)
+    codec = lla.make_codec(W_down_k=p["W_down_k"], W_down_v=p["W_down_v"], bias_k=bias_k, bias_v=bias_v,
+                           mu_k=p["mu_k"], mu_v=p["mu_v"])
+    lla.codec_bias(dims, codec, bias_k, bias_v)
+    ck = torch.empty(w.L, w.heads_stored, n_tok, w.r_k, dtype=w.torch_dtype, device=dev)
+    cv = torch.empty(w.L, w.heads_stored, n_tok, w.r_v, dtype=w.torch_dtype, device=dev)
+    cache = lla.make_cache(ck, cv, n_tok)
+    xk = S.draw_encode_tokens(w, layer, "k", n_tok, dev)
+    xv = S.draw_encode_tokens(w, layer, "v", n_tok, dev)
+    slot_idx = torch.arange(n_tok, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step():
+        lla.encode(dims, layer, 1, xk, xv, n_tok, slot_idx, codec, cache, stream=stream)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    sampler = ClockSampler(dev.index or 0).start()
+    wall0 = time.perf_counter()
+    e0.record(stream)
+    for _ in range(args.steps):
+        step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    wall1 = time.perf_counter()
+    sampler.stop()
+    assert lla.status_fetch(None) == 0
+    ms = e0.elapsed_time(e1) / args.steps
+    e = w.elem_bytes
+    bytes_moved = 2 * n_tok * w.H * w.T * w.d * e + n_tok * w.heads_stored * (w.r_k + w.r_v) * e
+    flops = 2.0 * n_tok * w.heads_stored * w.W * (w.r_k + w.r_v)
+    peaks, kind = measured_peaks()
+    gbs = bytes_moved / (ms * 1e-3) / 1e9
+    tfl = flops / (ms * 1e-3) / 1e12
+    print(json.dumps({
+        "metric": "LLA prefill encode GB/s (one layer, K and V)", "value": gbs, "unit": "GB/s",
+        "n_gpus": 1, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+        "higher_is_better": True, "dtype": "bf16 x bf16 -> f32" if w.dtype == "bf16" else "f32",
+        "data": "synthetic",
+        "config": {"workload": w.name, "tokens": n_tok, "H": w.H, "T": w.T, "d": w.d, "r_k": w.r_k,
+                   "r_v": w.r_v, "fold2d": w.fold2d},
+        "roofline": {"bound": "hbm", "achieved": gbs, "peak": float(peaks["hbm_gbs"]), "unit": "GB/s",
+                     "frac": gbs / float(peaks["hbm_gbs"]), "peak_kind": kind},
+        "tensor": {"achieved_tflops": tfl, "peak_tflops": float(peaks.get("bf16_tflops", 1590.0)),
+                   "frac": tfl / float(peaks.get("bf16_tflops", 1590.0))},
+        "clocks": sampler.summary(wall0, wall1),
+    }), flush=True)
+
+
+# ---------------------------------------------------------------------------
 # our arm
 # ---------------------------------------------------------------------------
 def main():
@@ -237,6 +328,9 @@ def main():
     import decode_attention_12_b200 as lla
     import lla_synth as S
 
+    if args.phase == "encode":
+        run_encode_phase(args, dev)
+        return
     w = S.WORKLOADS[args.workload]
     Tq = w.T
     p = S.decode_inputs(w, 0, dev, gap=1)          # one free slot per sequence for the new token
@@ -259,23 +353,25 @@ def main():
     x_k = S.draw_encode_tokens(w, 0, "k", B, dev, seed_tag="new")
     x_v = S.draw_encode_tokens(w, 0, "v", B, dev, seed_tag="new")
     new_slot = (p["seq_start"] + p["ctx_lens"].to(torch.int64)).contiguous()
-    ws_bytes = lla.decode_workspace_bytes(dims, B, Tq, max_ctx, lla.ABSORB, args.num_splits)
+    variant = lla.RECONSTRUCT if args.variant == "reconstruct" else lla.ABSORB
+    ws_bytes = lla.decode_workspace_bytes(dims, B, Tq, max_ctx, variant, args.num_splits)
     ws = torch.zeros(ws_bytes, dtype=torch.uint8, device=dev)
     q = p["q"]
     out = torch.empty(B, Tq, H, w.d, dtype=torch.float32, device=dev)
     lse = torch.empty(B, Tq, H, dtype=torch.float32, device=dev)
     stream = torch.cuda.current_stream(dev)
-    splits = lla.decode_num_splits(dims, B, Tq, max_ctx, lla.ABSORB, args.num_splits)
+    splits = lla.decode_num_splits(dims, B, Tq, max_ctx, variant, args.num_splits)
 
     def decode(i, q_in=q, out_buf=out):
         lla.decode_attn(dims, 0, 0, Tq, q_in, caches[i % R], p["seq_start"], p["ctx_lens"], B,
-                        max_ctx, codec, 1.0, out_buf, lse, ws, ws_bytes, num_splits=args.num_splits,
-                        stream=stream)
+                        max_ctx, codec, 1.0, out_buf, lse, ws, ws_bytes, variant=variant,
+                        num_splits=args.num_splits, stream=stream)
 
     def encode(i, xk=x_k, xv=x_v):
         lla.encode(dims, 0, 1, xk, xv, B, new_slot, codec, caches[i % R], stream=stream)
 
-    launches_per_step = 3                       # decode + combine + encode kernels
+    # prologue + decode + combine + 2 encode (K, V) kernels; reconstruct: Tq decode passes
+    launches_per_step = (3 if args.variant == "absorb" else Tq + 1) + 2
     # ---- warm-up, then the device-timed region ------------------------------------------------
     sampler = ClockSampler(local).start()
     for i in range(args.warmup):
@@ -302,12 +398,8 @@ def main():
     if world > 1:
         dist.barrier()
     sampler.stop()
-    ms_total = t_start.elapsed_time(t_end)
+    ms_total = max_over_ranks(t_start.elapsed_time(t_end), dev)
     decode_ms = [a.elapsed_time(b) for a, b in zip(ev_a, ev_b)]
-    if world > 1:
-        t = torch.tensor([ms_total], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms_total = float(t.item())
     status = lla.status_fetch(ws)
     if status != 0:
         raise RuntimeError(f"device status {status}: {lla.status_string(status)}")
@@ -354,11 +446,7 @@ def main():
         e2e_step(i)
     e1.record(stream)
     torch.cuda.synchronize()
-    e2e_ms = e0.elapsed_time(e1)
-    if world > 1:
-        t = torch.tensor([e2e_ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_ms = float(t.item())
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1), dev)
     e2e_value = world * step_bytes * e2e_steps / (e2e_ms * 1e-3) / 1e9
     h2d = (q.numel() * q.element_size() + x_k.numel() * x_k.element_size() * 2)
     d2h = out.numel() * out.element_size() + lse.numel() * lse.element_size()
@@ -385,7 +473,7 @@ def main():
         "config": {"workload": w.name, "T": w.T, "L_per_step": 1, "H": H, "d": w.d,
                    "r_k": w.r_k, "r_v": w.r_v, "rho": "64/3", "B": B,
                    "ctx_len": [w.len_lo, w.len_hi], "tokens": S_tot, "Tq": Tq,
-                   "variant": "absorb", "seg_max": splits,
+                   "variant": args.variant, "seg_max": splits,
                    "step": "decode_attn(all 4 loop queries) + encode(B new tokens)",
                    "l2": f"inputs larger than L2 ({step_bytes / 1e6:.0f} MB of latents per step) "
                          f"and {R} rotating cache replicas",
@@ -394,8 +482,9 @@ def main():
         "hbm_frac_of_8tbs_spec": value / world / SPEC_HBM_GBS,
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                      "frac": achieved / peak, "peak_kind": peak_kind,
-                     "traffic": profiled_traffic(units_per_launch),
-                     "timed": "lla_decode_attn (decode + combine kernels), CUDA events per call",
+                     "traffic": profiled_traffic(units_per_launch, args.variant),
+                     "timed": "one lla_decode_attn call (q_tilde prologue + decode + combine "
+                              "kernels), CUDA events per call on the launch stream",
                      "algorithmic_bytes_per_launch": step_bytes},
         "cpu_baseline": cpu,
         "e2e": {"value": e2e_value, "unit": "GB/s", "h2d_bytes_per_step": h2d,
