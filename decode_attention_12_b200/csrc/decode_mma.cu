@@ -57,7 +57,7 @@ __global__ void __launch_bounds__((NW + 1) * 32, MINB)
     constexpr int kWarps = NW, kThreads = C::THREADS, kConsumers = C::CONSUMERS, kTile = C::TILE;
     constexpr int kStages = C::STAGES;
     extern __shared__ uint8_t smem_raw[];
-    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
+    uint8_t *smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
     float *mrg = reinterpret_cast<float *>(smem + C::MRG_OFF);
     volatile int *misc = reinterpret_cast<volatile int *>(smem + C::MISC_OFF); // [0] error flag
     int64_t *pref = reinterpret_cast<int64_t *>(smem + C::PREF_OFF);

@@ -57,7 +57,8 @@ __global__ void __launch_bounds__(kThreads, 2)
 {
     using C = RCfg<RK, RV, D>;
     extern __shared__ uint8_t smem_raw[];
-    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
+    // aligned by arithmetic on the shared array itself, so accesses stay shared-space loads
+    uint8_t *smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
     float *vq = reinterpret_cast<float *>(smem + C::VEC_OFF);
     float *vmk = vq + D, *vmv = vq + 2 * D, *vqmu = vq + 3 * D;
     float *mrg = reinterpret_cast<float *>(smem + C::MRG_OFF);

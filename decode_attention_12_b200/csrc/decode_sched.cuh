@@ -40,10 +40,12 @@ __device__ __forceinline__ int find_seq(const int64_t *pref, int B, int H, int64
     return lo;
 }
 
-// Walks the token share [pos, end) of one CTA, unit segment by unit segment, tile by tile.
+// Walks the token share [pos, end) of one CTA (shares of `chunk` tokens), unit segment by
+// unit segment, tile by tile; each segment's record slot j = share - first share of the
+// unit and the unit's record count n_u come from the share geometry.
 template <int TILE> struct ShareWalk {
     int64_t pos, end, chunk, seq0;
-    int32_t b, h, n, seg_end, u, j, n_u;
+    int32_t b = 0, h, n, seg_end, u, j, n_u;
     bool in_seg;
 
     __device__ void start(int64_t p, int64_t e, int64_t ch)
@@ -59,17 +61,29 @@ template <int TILE> struct ShareWalk {
         if (!in_seg) {
             if (pos >= end)
                 return false;
-            b = find_seq(pref, B, H, pos);
+            // the sequence holding pos: the previous one or its successor, else bisect
+            const int64_t HH = H;
+            if (!(HH * pref[b] <= pos && pos < HH * pref[b + 1])) {
+                if (b + 2 <= B && HH * pref[b + 1] <= pos && pos < HH * pref[b + 2])
+                    ++b;
+                else
+                    b = find_seq(pref, B, H, pos);
+            }
             const int len = (int)(pref[b + 1] - pref[b]);
             seq0 = starts[b];
-            const int64_t off = pos - (int64_t)H * pref[b];
-            h = (int)(off / len);
-            n = (int)(off - (int64_t)h * len);
+            const int64_t off = pos - HH * pref[b];
+            if (off < 0x7fffffff) {
+                h = (int)off / len;
+                n = (int)off - h * len;
+            } else {
+                h = (int)(off / len);
+                n = (int)(off - (int64_t)h * len);
+            }
             const int64_t take = min((int64_t)(len - n), end - pos);
             seg_end = n + (int)take;
             pos += take;
             u = b * H + h;
-            const int64_t U = (int64_t)H * pref[b] + (int64_t)h * len; // unit start in the stream
+            const int64_t U = HH * pref[b] + (int64_t)h * len; // unit start in the stream
             const int64_t c_first = U / chunk, c_last = (U + len - 1) / chunk;
             j = (int)(blockIdx.x - c_first);
             n_u = (int)(c_last - c_first + 1);

@@ -443,119 +443,218 @@ __global__ void __launch_bounds__(kPrologueThreads) absorb_prologue_kernel(const
 }
 
 // ---------------------------------------------------------------------------------
-// a4: cross-segment combine + output projection, batched per (head, loop query, chunk
-// of 32 sequences).  For each sequence b of the chunk (one warp per sequence):
+// a4: cross-segment combine + output projection.  One warp per (sequence b, head h,
+// loop query t); a CTA holds 8 sequences of one (h, t) and stages W_up,t^V (r_v x d)
+// in shared memory once:
 //   M = max_s m_s,  L = sum_s l_s 2^(m_s - M),  o_lat = sum_s acc_s 2^(m_s - M) / L,
 //   lse = ln2 (M + log2 L) + scale * q . mu_t^K   (-inf and out = 0 for an empty context)
-// then out[b] = o_lat[b] W_up,t^V + mu_t^V with W_up,t^V (r_v x d) staged in shared memory.
+//   out[b] = o_lat W_up,t^V + mu_t^V.
+// Latency design: everything that does not come from the decode grid (W_up,t^V,
+// mu_t^V, mu_t^K, q, ctx_lens) is fetched before the programmatic-launch wait; after
+// it, the unit's record count and its first kSpecRecords records are loaded in one
+// round (slots past the count lie inside the workspace and are ignored), so the
+// combine adds two dependent global-load latencies to the end of the decode.
+// Lane c owns record / output columns 4c + 128 i (16-byte groups).
 // ---------------------------------------------------------------------------------
 constexpr int kCombineThreads = 256; // 8 warps: one sequence each
+constexpr int kSpecRecords = 4;      // records fetched before the count is known
+constexpr int kMaxOutGroups = 4;     // d <= 512
+
+template <typename T> struct Vec4;
+template <> struct Vec4<float> {
+    static __device__ __forceinline__ float4 load(const float *p) { return *reinterpret_cast<const float4 *>(p); }
+    static __device__ __forceinline__ void store(float *p, float4 v) { *reinterpret_cast<float4 *>(p) = v; }
+};
+template <> struct Vec4<__nv_bfloat16> {
+    static __device__ __forceinline__ float4 load(const __nv_bfloat16 *p)
+    {
+        const uint2 u = *reinterpret_cast<const uint2 *>(p);
+        return make_float4(bf16_lo(u.x), bf16_hi(u.x), bf16_lo(u.y), bf16_hi(u.y));
+    }
+    static __device__ __forceinline__ void store(__nv_bfloat16 *p, float4 v)
+    {
+        const __nv_bfloat162 lo = __floats2bfloat162_rn(v.x, v.y), hi = __floats2bfloat162_rn(v.z, v.w);
+        uint2 u;
+        u.x = *reinterpret_cast<const uint32_t *>(&lo);
+        u.y = *reinterpret_cast<const uint32_t *>(&hi);
+        *reinterpret_cast<uint2 *>(p) = u;
+    }
+};
+
+__device__ __forceinline__ float4 f4_fma(float s, float4 x, float4 y)
+{
+    return make_float4(fmaf(s, x.x, y.x), fmaf(s, x.y, y.y), fmaf(s, x.z, y.z), fmaf(s, x.w, y.w));
+}
+__device__ __forceinline__ float4 f4_scale(float s, float4 x) { return make_float4(s * x.x, s * x.y, s * x.z, s * x.w); }
+
+// Records [s0, s0 + n) of one unit in registers: (m, l) and this lane's RG column groups.
+template <int RG> struct RecBatch {
+    float2 ml[kSpecRecords];
+    float4 rv[kSpecRecords][RG];
+
+    // Loads the records s0 + k < lim (k < kSpecRecords); lane c holds columns 4c + 128 g.
+    __device__ __forceinline__ void load(const float *rec0, int s0, int lim, int ps, int RV, int lane)
+    {
+#pragma unroll
+        for (int k = 0; k < kSpecRecords; ++k) {
+            const int s = s0 + k;
+            ml[k] = make_float2(-INFINITY, 0.f);
+#pragma unroll
+            for (int g = 0; g < RG; ++g)
+                rv[k][g] = make_float4(0.f, 0.f, 0.f, 0.f);
+            if (s < lim) {
+                ml[k] = *reinterpret_cast<const float2 *>(rec0 + (int64_t)s * ps + RV);
+#pragma unroll
+                for (int g = 0; g < RG; ++g) {
+                    const int c = 4 * lane + 128 * g;
+                    if (c < RV)
+                        rv[k][g] = Vec4<float>::load(rec0 + (int64_t)s * ps + c);
+                }
+            }
+        }
+    }
+
+    // Folds records k < n into the running (M, L, acc).
+    __device__ __forceinline__ void merge(int n, float &M, float &L, float4 (&acc)[RG]) const
+    {
+        float Mn = M;
+#pragma unroll
+        for (int k = 0; k < kSpecRecords; ++k)
+            if (k < n)
+                Mn = fmaxf(Mn, ml[k].x);
+        if (Mn == -INFINITY)
+            return; // nothing but empty records so far
+        const float al = M == -INFINITY ? 0.f : exp2f(M - Mn);
+        L *= al;
+#pragma unroll
+        for (int g = 0; g < RG; ++g)
+            acc[g] = f4_scale(al, acc[g]);
+#pragma unroll
+        for (int k = 0; k < kSpecRecords; ++k) {
+            if (k < n && ml[k].x != -INFINITY) {
+                const float w = exp2f(ml[k].x - Mn);
+                L = fmaf(w, ml[k].y, L);
+#pragma unroll
+                for (int g = 0; g < RG; ++g)
+                    acc[g] = f4_fma(w, rv[k][g], acc[g]);
+            }
+        }
+        M = Mn;
+    }
+};
 
 // REC: records carry d-wide outputs of the reconstruct form (mu and the q.mu_t^K score term
-// already included), so the output is the merged record itself.
-template <typename T, typename O, bool REC>
-__global__ void __launch_bounds__(kCombineThreads) decode_combine_kernel(const DecodeArgs a)
+// already included), so the output is the merged record itself.  RG = record width / 128,
+// rounded up.
+template <typename T, typename O, bool REC, int RG>
+__global__ void __launch_bounds__(kCombineThreads, RG == 1 ? 4 : 2) decode_combine_kernel(const DecodeArgs a)
 {
-    extern __shared__ float csm[];
+    extern __shared__ __align__(16) float csm[];
     const int h = blockIdx.x, tl = blockIdx.y, b0 = blockIdx.z * kBatchSeqs;
     const int t = a.tq_off + tl; // indexes q / out / lse / records
     const int d = a.d, RV = REC ? a.d : a.r_v, ps = part_stride(RV);
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    float *W = csm;                        // [RV][d]
-    float *muv = W + RV * d;               // [d]
-    float *muk = muv + d;                  // [d]
-    float *olat = muk + d;                 // [kBatchSeqs][RV]
-    float *valid = olat + kBatchSeqs * RV; // [kBatchSeqs]
+    const int b = b0 + warp;
+    const bool active = b < a.B;
+    float *W = csm;          // [RV][d]
+    float *muv = W + RV * d; // [d]
     const int tg = a.t0 + t;
     const int ld = a.fold ? a.H * d : d;
     const int64_t wbase = a.fold ? (int64_t)tg * RV * ld + (int64_t)h * d : ((int64_t)h * a.T + tg) * RV * ld;
     const int64_t mbase = a.fold ? (int64_t)tg * ld + (int64_t)h * d : ((int64_t)h * a.T + tg) * ld;
+    const int64_t u = (int64_t)b * a.H + h;
+
+    // ---- inputs of the call (not written by the decode grid)
     if (!REC) {
         stage_f32<kCombineThreads>(W, d, a.W_up_v + wbase, ld, RV, d);
-        for (int k = threadIdx.x; k < d; k += kCombineThreads) {
+        for (int k = threadIdx.x; k < d; k += kCombineThreads)
             muv[k] = a.mu_v[mbase + k];
-            muk[k] = a.mu_k[mbase + k];
-        }
     }
-    grid_dependency_wait(); // partial records come from the preceding decode grid
-    __syncthreads();
-    const int nb = min(kBatchSeqs, a.B - b0);
-    for (int bl = warp; bl < nb; bl += kCombineThreads / 32) {
-        const int b = b0 + bl;
-        const int64_t u = (int64_t)b * a.H + h;
-        const int len = a.ctx_lens[b];
-        const int S = len > 0 ? min(a.counts[u], a.seg_max) : 0;
-        const float *rec0 = a.part + (u * a.Tq_all + t) * a.seg_max * ps;
-        // lane s holds record s's reference and sum (records beyond 32 folded in a loop)
-        float M = -INFINITY;
-        for (int s = lane; s < S; s += 32)
-            M = fmaxf(M, rec0[s * ps + RV]);
-        for (int off = 16; off > 0; off >>= 1)
-            M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, off));
-        float L = 0.f;
-        float acc[8]; // r_v / 32 values per lane (r_v <= 256)
-#pragma unroll
-        for (int q = 0; q < 8; ++q)
-            acc[q] = 0.f;
-        for (int s0 = 0; s0 < S; s0 += 32) {
-            const int s = s0 + lane;
-            float ws = 0.f;
-            if (s < S) {
-                const float ms = rec0[s * ps + RV];
-                ws = ms == -INFINITY ? 0.f : exp2f(ms - M);
-                L += ws * rec0[s * ps + RV + 1];
-            }
-            const int ns = min(32, S - s0);
-            for (int i = 0; i < ns; ++i) {
-                const float wi = __shfl_sync(0xffffffffu, ws, i);
-                const float *ri = rec0 + (s0 + i) * ps;
-#pragma unroll
-                for (int q = 0; q < 8; ++q)
-                    if (lane + 32 * q < RV)
-                        acc[q] = fmaf(wi, ri[lane + 32 * q], acc[q]);
-            }
-        }
-        for (int off = 16; off > 0; off >>= 1)
-            L += __shfl_xor_sync(0xffffffffu, L, off);
-        const float invL = L > 0.f ? 1.f / L : 0.f;
-#pragma unroll
-        for (int q = 0; q < 8; ++q)
-            if (lane + 32 * q < RV)
-                olat[bl * RV + lane + 32 * q] = acc[q] * invL;
-        // lse with the constant key-mean term scale * q . mu_t^K (absorbed form only)
-        float qm = 0.f;
+    int len = 0;
+    float qm = 0.f;
+    if (active) {
+        len = a.ctx_lens[b];
         if (!REC) {
             const T *qrow = static_cast<const T *>(a.q) + (((int64_t)b * a.Tq_all + t) * a.H + h) * d;
-            for (int k = lane; k < d; k += 32)
-                qm = fmaf(Elem<T>::to_f(qrow[k]), muk[k], qm);
+            for (int c = 4 * lane; c < d; c += 128) {
+                const float4 qv = Vec4<T>::load(qrow + c);
+                const float4 mk = Vec4<float>::load(a.mu_k + mbase + c);
+                qm = fmaf(qv.x, mk.x, fmaf(qv.y, mk.y, fmaf(qv.z, mk.z, fmaf(qv.w, mk.w, qm))));
+            }
+#pragma unroll
             for (int off = 16; off > 0; off >>= 1)
                 qm += __shfl_xor_sync(0xffffffffu, qm, off);
         }
-        if (lane == 0) {
-            valid[bl] = L > 0.f ? 1.f : 0.f;
-            if (a.lse != nullptr)
-                a.lse[((int64_t)b * a.Tq_all + t) * a.H + h] = L > 0.f ? kLn2 * (M + log2f(L)) + a.scale * qm : -INFINITY;
+    }
+
+    grid_dependency_wait(); // records and counts come from the preceding decode grid
+
+    float M = -INFINITY, L = 0.f;
+    float4 acc[RG];
+#pragma unroll
+    for (int g = 0; g < RG; ++g)
+        acc[g] = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (active && len > 0) {
+        const float *rec0 = a.part + (u * a.Tq_all + t) * a.seg_max * ps;
+        const int cnt = a.counts[u];
+        RecBatch<RG> rb;
+        rb.load(rec0, 0, a.seg_max, ps, RV, lane); // issued together with the count
+        const int S = min(cnt, a.seg_max);
+        rb.merge(min(S, kSpecRecords), M, L, acc);
+        for (int s0 = kSpecRecords; s0 < S; s0 += kSpecRecords) { // long contexts / many splits
+            rb.load(rec0, s0, S, ps, RV, lane);
+            rb.merge(min(S - s0, kSpecRecords), M, L, acc);
         }
     }
-    __syncthreads();
-    for (int e = threadIdx.x; e < nb * d; e += kCombineThreads) {
-        const int bl = e / d, k = e - bl * d;
-        float o = 0.f;
-        if (REC) {
-            o = valid[bl] != 0.f ? olat[bl * RV + k] : 0.f;
-        } else if (valid[bl] != 0.f) {
-            const float *ol = olat + bl * RV;
-            float o0 = muv[k], o1 = 0.f;
-            int j = 0;
-            for (; j + 1 < RV; j += 2) {
-                o0 = fmaf(ol[j], W[j * d + k], o0);
-                o1 = fmaf(ol[j + 1], W[(j + 1) * d + k], o1);
+    const float invL = L > 0.f ? 1.f / L : 0.f;
+#pragma unroll
+    for (int g = 0; g < RG; ++g)
+        acc[g] = f4_scale(invL, acc[g]); // o_lat (or the output itself for REC)
+    if (active && lane == 0 && a.lse != nullptr)
+        a.lse[((int64_t)b * a.Tq_all + t) * a.H + h] =
+            L > 0.f ? kLn2 * (M + log2f(L)) + (REC ? 0.f : a.scale * qm) : -INFINITY;
+
+    O *orow = static_cast<O *>(a.out) + (((int64_t)b * a.Tq_all + t) * a.H + h) * d;
+    if (REC) {
+        if (active) {
+#pragma unroll
+            for (int g = 0; g < RG; ++g) {
+                const int c = 4 * lane + 128 * g;
+                if (c < d)
+                    Vec4<O>::store(orow + c, acc[g]);
             }
-            for (; j < RV; ++j)
-                o0 = fmaf(ol[j], W[j * d + k], o0);
-            o = o0 + o1;
         }
-        static_cast<O *>(a.out)[(((int64_t)(b0 + bl) * a.Tq_all + t) * a.H + h) * d + k] = Elem<O>::from_f(o);
+        return;
+    }
+    __syncthreads(); // W_up,t^V and mu_t^V staged
+    if (!active)
+        return;
+    const bool valid = L > 0.f;
+    for (int c = 4 * lane, gi = 0; gi < kMaxOutGroups && c - 4 * lane < d; c += 128, ++gi) {
+        // every lane takes part in the shuffles; lanes past d only skip the math
+        const bool mine = c < d;
+        float4 o = valid && mine ? *reinterpret_cast<const float4 *>(muv + c) : make_float4(0.f, 0.f, 0.f, 0.f);
+        if (valid) {
+            // o_lat[j] sits in lane (j / 4) % 32, group j / 128, component j % 4
+#pragma unroll 2
+            for (int j4 = 0; j4 < RV; j4 += 4) {
+                const int src = (j4 >> 2) & 31;
+                const float4 sel = (RG > 1 && j4 >= 128) ? acc[RG - 1] : acc[0];
+                const float ox = __shfl_sync(0xffffffffu, sel.x, src);
+                const float oy = __shfl_sync(0xffffffffu, sel.y, src);
+                const float oz = __shfl_sync(0xffffffffu, sel.z, src);
+                const float ow = __shfl_sync(0xffffffffu, sel.w, src);
+                if (mine) {
+                    const float *wr = W + j4 * d + c;
+                    o = f4_fma(ox, *reinterpret_cast<const float4 *>(wr), o);
+                    o = f4_fma(oy, *reinterpret_cast<const float4 *>(wr + d), o);
+                    o = f4_fma(oz, *reinterpret_cast<const float4 *>(wr + 2 * d), o);
+                    o = f4_fma(ow, *reinterpret_cast<const float4 *>(wr + 3 * d), o);
+                }
+            }
+        }
+        if (mine)
+            Vec4<O>::store(orow + c, o);
     }
 }
 
@@ -606,10 +705,10 @@ cudaError_t launch_absorb_prologue(const DecodeArgs &a, int dtype, cudaStream_t 
     return cudaGetLastError();
 }
 
-template <typename T, typename O>
+template <typename T, typename O, int RG>
 static cudaError_t launch_combine_t(const DecodeArgs &a, size_t smem, cudaStream_t stream)
 {
-    auto k = a.recon ? decode_combine_kernel<T, O, true> : decode_combine_kernel<T, O, false>;
+    auto k = a.recon ? decode_combine_kernel<T, O, true, RG> : decode_combine_kernel<T, O, false, RG>;
     cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess)
         return e;
@@ -626,22 +725,28 @@ static cudaError_t launch_combine_t(const DecodeArgs &a, size_t smem, cudaStream
     return cudaLaunchKernelEx(&cfg, k, a);
 }
 
+template <typename T, typename O>
+static cudaError_t launch_combine_rg(const DecodeArgs &a, int rv, size_t smem, cudaStream_t stream)
+{
+    return rv > 128 ? launch_combine_t<T, O, 2>(a, smem, stream) : launch_combine_t<T, O, 1>(a, smem, stream);
+}
+
 cudaError_t launch_decode_combine(const DecodeArgs &a, int dtype, int out_dtype, cudaStream_t stream)
 {
     const int rv = a.recon ? a.d : a.r_v;
-    if (rv > 256)
-        return cudaErrorInvalidValue; // one warp holds (record width) / 32 <= 8 values per lane
-    const size_t smem = sizeof(float) * ((size_t)rv * a.d + 2 * a.d + (size_t)kBatchSeqs * (rv + 1));
+    if (rv > 256 || a.d > 128 * kMaxOutGroups || rv % 4 != 0 || a.d % 4 != 0)
+        return cudaErrorInvalidValue; // a lane holds 16-byte groups of a record / output row
+    const size_t smem = a.recon ? 16 : sizeof(float) * ((size_t)rv * a.d + a.d);
     if (smem > 200 * 1024)
         return cudaErrorInvalidValue;
     using BF = __nv_bfloat16;
     if (dtype == LLA_BF16 && out_dtype == LLA_BF16)
-        return launch_combine_t<BF, BF>(a, smem, stream);
+        return launch_combine_rg<BF, BF>(a, rv, smem, stream);
     if (dtype == LLA_BF16)
-        return launch_combine_t<BF, float>(a, smem, stream);
+        return launch_combine_rg<BF, float>(a, rv, smem, stream);
     if (out_dtype == LLA_BF16)
-        return launch_combine_t<float, BF>(a, smem, stream);
-    return launch_combine_t<float, float>(a, smem, stream);
+        return launch_combine_rg<float, BF>(a, rv, smem, stream);
+    return launch_combine_rg<float, float>(a, rv, smem, stream);
 }
 
 } // namespace lla

@@ -18,6 +18,7 @@
 //    its cache slot.
 // Every wait is bounded; a timeout records LLA_ERR_DEVICE_TIMEOUT in the library's
 // encode status word and the CTA winds down (tensor memory is always released).
+#include <cstring>
 #include <mutex>
 
 #include "encode.cuh"
@@ -103,19 +104,28 @@ __device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&r)[16])
     asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 }
 
-struct EncTcArgs {
+struct EncTcAxis {
     const float *bias;     // [L][H'][N]
     void *plane;           // [L][H'][slots][N]
-    const int64_t *slot_idx;
-    int64_t n_tok, slots;
-    int32_t layer0, Hs, nk, d_slabs, fold;
 };
 
-template <int N> struct EncCfg {
+struct EncTcArgs {
+    EncTcAxis ax[2];       // K, V
+    const int64_t *slot_idx;
+    int64_t n_tok, slots;
+    int32_t layer0, Hs, nk, d_slabs, fold, axis0;
+};
+
+// Ring depth: a shallow ring (~110 KB) leaves room for two CTAs per SM on large grids;
+// a grid smaller than the GPU gets every K slab in flight at once (<= 8 stages).
+template <int N, bool DEEP> struct EncCfg {
     static constexpr int A_BYTES = kBlockM * 128;
     static constexpr int B_BYTES = N * 128;
     static constexpr int STAGE = (A_BYTES + B_BYTES + 1023) & ~1023;
-    static constexpr int STAGES = (110 * 1024) / STAGE >= 4 ? 4 : ((110 * 1024) / STAGE >= 3 ? 3 : 2);
+    static constexpr int BUDGET = DEEP ? 200 * 1024 : 110 * 1024;
+    static constexpr int FIT = BUDGET / STAGE;
+    static constexpr int CAP = DEEP ? 8 : 4;
+    static constexpr int STAGES = FIT >= CAP ? CAP : (FIT >= 2 ? FIT : 2);
     static constexpr int TMEM_COLS = N <= 32 ? 32 : (N <= 64 ? 64 : (N <= 128 ? 128 : 256));
     static constexpr int BAR_OFF = STAGES * STAGE;         // full[S], empty[S], acc
     static constexpr int HOLD_OFF = BAR_OFF + (2 * STAGES + 1) * 8;
@@ -124,22 +134,27 @@ template <int N> struct EncCfg {
     static_assert(N % 16 == 0 && N >= 16 && N <= 256, "tcgen05 N for M = 128");
 };
 
-template <int N>
-__global__ void __launch_bounds__(kThreads, 1)
-    encode_tc_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CUtensorMap map_b,
-                     const EncTcArgs a)
+// One 128-token x N tile of one (layer, stored head, axis).
+template <int N, bool DEEP>
+__device__ __forceinline__ void encode_tile(uint8_t *smem, const CUtensorMap *map_a, const CUtensorMap *map_b,
+                                            const EncTcArgs &a, const EncTcAxis &ax, int m0, int hs, int li)
 {
-    using C = EncCfg<N>;
-    extern __shared__ uint8_t smem_raw[];
-    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
+    using C = EncCfg<N, DEEP>;
     const uint32_t sbase = smem_u32(smem);
     const uint32_t full0 = sbase + C::BAR_OFF, empty0 = full0 + 8 * C::STAGES, accb = empty0 + 8 * C::STAGES;
     uint32_t *hold = reinterpret_cast<uint32_t *>(smem + C::HOLD_OFF);
     float *bias_s = reinterpret_cast<float *>(smem + C::BIAS_OFF);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int m0 = blockIdx.x * kBlockM, hs = blockIdx.y, li = blockIdx.z;
     const int l = a.layer0 + li;
 
+    // destination slot of this thread's token (accumulator lane), fetched up front
+    const int64_t tok = (int64_t)m0 + warp * 32 + lane;
+    int64_t slot = -1;
+    if (tok < a.n_tok) {
+        slot = a.slot_idx[tok];
+        if (slot < 0 || slot >= a.slots)
+            slot = -1;
+    }
     if (threadIdx.x == 0) {
         for (int s = 0; s < C::STAGES; ++s) {
             mbar_init(full0 + 8 * s, 1);
@@ -156,8 +171,6 @@ __global__ void __launch_bounds__(kThreads, 1)
                      : "memory");
         asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
     }
-    for (int j = threadIdx.x; j < N; j += kThreads)
-        bias_s[j] = a.bias[((int64_t)l * a.Hs + hs) * N + j];
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
@@ -174,10 +187,10 @@ __global__ void __launch_bounds__(kThreads, 1)
             const uint32_t dst = sbase + s * C::STAGE;
             mbar_arrive_expect_tx(full0 + 8 * s, C::A_BYTES + C::B_BYTES);
             if (a.fold)
-                tma_load_3d(dst, &map_a, kb * kSlabK, m0, li, full0 + 8 * s);
+                tma_load_3d(dst, map_a, kb * kSlabK, m0, li, full0 + 8 * s);
             else
-                tma_load_5d(dst, &map_a, (kb % a.d_slabs) * kSlabK, hs, kb / a.d_slabs, m0, li, full0 + 8 * s);
-            tma_load_3d(dst + C::A_BYTES, &map_b, kb * kSlabK, 0, l * a.Hs + hs, full0 + 8 * s);
+                tma_load_5d(dst, map_a, (kb % a.d_slabs) * kSlabK, hs, kb / a.d_slabs, m0, li, full0 + 8 * s);
+            tma_load_3d(dst + C::A_BYTES, map_b, kb * kSlabK, 0, l * a.Hs + hs, full0 + 8 * s);
         }
     } else if (warp == 1 && lane == 0) {
         // ---- MMA issuer
@@ -202,8 +215,13 @@ __global__ void __launch_bounds__(kThreads, 1)
             tc_commit(accb); // accumulator complete
         else
             mbar_arrive(accb);
+    } else if (warp >= 2) {
+        // the bias row, while the tiles stream in
+        for (int j = threadIdx.x - 64; j < N; j += kThreads - 64)
+            bias_s[j] = ax.bias[((int64_t)l * a.Hs + hs) * N + j];
     }
     __syncwarp();
+    __syncthreads(); // bias staged; roles done issuing
 
     // ---- epilogue: all 4 warps, warp w owns accumulator lanes (tokens) 32w .. 32w+31
     const bool acc_ok = mbar_wait_bounded(accb, 0);
@@ -212,14 +230,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (threadIdx.x == 0)
             report_status(&g_encode_status, LLA_ERR_DEVICE_TIMEOUT);
     } else {
-        const int64_t tok = (int64_t)m0 + warp * 32 + lane;
-        int64_t slot = -1;
-        if (tok < a.n_tok) {
-            slot = a.slot_idx[tok];
-            if (slot < 0 || slot >= a.slots)
-                slot = -1;
-        }
-        __nv_bfloat16 *dst = static_cast<__nv_bfloat16 *>(a.plane) + (((int64_t)l * a.Hs + hs) * a.slots) * N;
+        __nv_bfloat16 *dst = static_cast<__nv_bfloat16 *>(ax.plane) + (((int64_t)l * a.Hs + hs) * a.slots) * N;
 #pragma unroll 1
         for (int c = 0; c < N / 16; ++c) {
             uint32_t r[16];
@@ -246,6 +257,24 @@ __global__ void __launch_bounds__(kThreads, 1)
                      : "memory");
 }
 
+// grid (token tiles, axes x stored heads, layers); blockIdx.y / Hs selects K (rank NK) or
+// V (rank NV) counted from a.axis0, so one launch can cover both axes.
+template <int NK, int NV, bool DEEP>
+__global__ void __launch_bounds__(kThreads, 1)
+    encode_tc_kernel(const __grid_constant__ CUtensorMap map_ak, const __grid_constant__ CUtensorMap map_bk,
+                     const __grid_constant__ CUtensorMap map_av, const __grid_constant__ CUtensorMap map_bv,
+                     const EncTcArgs a)
+{
+    extern __shared__ uint8_t smem_raw[];
+    // aligned by arithmetic on the shared array itself, so accesses stay shared-space loads
+    uint8_t *smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
+    const int axis = a.axis0 + (int)blockIdx.y / a.Hs, hs = (int)blockIdx.y % a.Hs;
+    if (axis == 0)
+        encode_tile<NK, DEEP>(smem, &map_ak, &map_bk, a, a.ax[0], blockIdx.x * kBlockM, hs, blockIdx.z);
+    else
+        encode_tile<NV, DEEP>(smem, &map_av, &map_bv, a, a.ax[1], blockIdx.x * kBlockM, hs, blockIdx.z);
+}
+
 // ---- host: tensor maps ------------------------------------------------------------------------
 bool make_map(CUtensorMap *map, const void *base, int rank, const uint64_t *dims, const uint64_t *strides_bytes,
               const uint32_t *box)
@@ -260,40 +289,51 @@ bool make_map(CUtensorMap *map, const void *base, int rank, const uint64_t *dims
     return r == CUDA_SUCCESS;
 }
 
-template <int N>
-cudaError_t launch_tc_axis(const EncodeArgs &e, int axis, cudaStream_t stream)
+bool axis_maps(const EncodeArgs &e, int axis, int N, CUtensorMap *ma, CUtensorMap *mb)
 {
-    using C = EncCfg<N>;
     const void *x = axis ? e.x_v : e.x_k;
     const void *wd = axis ? e.W_down_v : e.W_down_k;
-    CUtensorMap ma, mb;
     const uint64_t el = 2;
     if (e.fold) {
         const uint64_t dims[3] = {(uint64_t)e.W, (uint64_t)e.n_tok, (uint64_t)e.n_layers};
         const uint64_t str[2] = {(uint64_t)e.W * el, (uint64_t)e.n_tok * e.W * el};
         const uint32_t box[3] = {kSlabK, kBlockM, 1};
-        if (!make_map(&ma, x, 3, dims, str, box))
-            return cudaErrorInvalidValue;
+        if (!make_map(ma, x, 3, dims, str, box))
+            return false;
     } else {
         const uint64_t dims[5] = {(uint64_t)e.d, (uint64_t)e.H, (uint64_t)e.T, (uint64_t)e.n_tok,
                                   (uint64_t)e.n_layers};
         const uint64_t str[4] = {(uint64_t)e.d * el, (uint64_t)e.H * e.d * el, (uint64_t)e.T * e.H * e.d * el,
                                  (uint64_t)e.n_tok * e.T * e.H * e.d * el};
         const uint32_t box[5] = {kSlabK, 1, 1, kBlockM, 1};
-        if (!make_map(&ma, x, 5, dims, str, box))
-            return cudaErrorInvalidValue;
+        if (!make_map(ma, x, 5, dims, str, box))
+            return false;
     }
-    {
-        const int L_total = e.layer0 + e.n_layers; // rows of W_down needed: up to the last layer used
-        const uint64_t dims[3] = {(uint64_t)e.W, (uint64_t)N, (uint64_t)L_total * e.Hs};
-        const uint64_t str[2] = {(uint64_t)e.W * el, (uint64_t)N * e.W * el};
-        const uint32_t box[3] = {kSlabK, (uint32_t)N, 1};
-        if (!make_map(&mb, wd, 3, dims, str, box))
-            return cudaErrorInvalidValue;
-    }
+    const int L_total = e.layer0 + e.n_layers; // rows of W_down needed: up to the last layer used
+    const uint64_t dims[3] = {(uint64_t)e.W, (uint64_t)N, (uint64_t)L_total * e.Hs};
+    const uint64_t str[2] = {(uint64_t)e.W * el, (uint64_t)N * e.W * el};
+    const uint32_t box[3] = {kSlabK, (uint32_t)N, 1};
+    return make_map(mb, wd, 3, dims, str, box);
+}
+
+// Launch axes [axis0, axis0 + n_axes) of one encode in one grid.
+template <int NK, int NV, bool DEEP>
+cudaError_t launch_tc(const EncodeArgs &e, int axis0, int n_axes, cudaStream_t stream)
+{
+    CUtensorMap mak, mbk, mav, mbv;
+    std::memset(&mak, 0, sizeof(mak));
+    std::memset(&mbk, 0, sizeof(mbk));
+    std::memset(&mav, 0, sizeof(mav));
+    std::memset(&mbv, 0, sizeof(mbv));
+    if (axis0 == 0 && !axis_maps(e, 0, NK, &mak, &mbk))
+        return cudaErrorInvalidValue;
+    if (axis0 + n_axes > 1 && !axis_maps(e, 1, NV, &mav, &mbv))
+        return cudaErrorInvalidValue;
     EncTcArgs a;
-    a.bias = axis ? e.bias_v : e.bias_k;
-    a.plane = axis ? e.cache_v : e.cache_k;
+    a.ax[0].bias = e.bias_k;
+    a.ax[0].plane = e.cache_k;
+    a.ax[1].bias = e.bias_v;
+    a.ax[1].plane = e.cache_v;
     a.slot_idx = e.slot_idx;
     a.n_tok = e.n_tok;
     a.slots = e.slots;
@@ -302,32 +342,59 @@ cudaError_t launch_tc_axis(const EncodeArgs &e, int axis, cudaStream_t stream)
     a.nk = e.W / kSlabK;
     a.d_slabs = e.d / kSlabK;
     a.fold = e.fold;
-    auto kern = encode_tc_kernel<N>;
-    cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
+    a.axis0 = axis0;
+    auto kern = encode_tc_kernel<NK, NV, DEEP>;
+    const int smem = EncCfg<NK, DEEP>::SMEM > EncCfg<NV, DEEP>::SMEM ? EncCfg<NK, DEEP>::SMEM
+                                                                       : EncCfg<NV, DEEP>::SMEM;
+    cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (err != cudaSuccess)
         return err;
-    dim3 grid((unsigned)((e.n_tok + kBlockM - 1) / kBlockM), e.Hs, e.n_layers);
-    kern<<<grid, kThreads, C::SMEM, stream>>>(ma, mb, a);
+    dim3 grid((unsigned)((e.n_tok + kBlockM - 1) / kBlockM), n_axes * e.Hs, e.n_layers);
+    kern<<<grid, kThreads, smem, stream>>>(mak, mbk, mav, mbv, a);
     return cudaGetLastError();
 }
 
-cudaError_t launch_tc_rank(const EncodeArgs &e, int axis, int r, cudaStream_t stream)
+template <bool DEEP> cudaError_t launch_tc_single(const EncodeArgs &e, int axis, int r, cudaStream_t stream)
 {
     switch (r) {
-    case 16: return launch_tc_axis<16>(e, axis, stream);
-    case 32: return launch_tc_axis<32>(e, axis, stream);
-    case 48: return launch_tc_axis<48>(e, axis, stream);
-    case 64: return launch_tc_axis<64>(e, axis, stream);
-    case 96: return launch_tc_axis<96>(e, axis, stream);
-    case 128: return launch_tc_axis<128>(e, axis, stream);
-    case 160: return launch_tc_axis<160>(e, axis, stream);
-    case 192: return launch_tc_axis<192>(e, axis, stream);
-    case 256: return launch_tc_axis<256>(e, axis, stream);
+    case 16: return launch_tc<16, 16, DEEP>(e, axis, 1, stream);
+    case 32: return launch_tc<32, 32, DEEP>(e, axis, 1, stream);
+    case 48: return launch_tc<48, 48, DEEP>(e, axis, 1, stream);
+    case 64: return launch_tc<64, 64, DEEP>(e, axis, 1, stream);
+    case 96: return launch_tc<96, 96, DEEP>(e, axis, 1, stream);
+    case 128: return launch_tc<128, 128, DEEP>(e, axis, 1, stream);
+    case 160: return launch_tc<160, 160, DEEP>(e, axis, 1, stream);
+    case 192: return launch_tc<192, 192, DEEP>(e, axis, 1, stream);
+    case 256: return launch_tc<256, 256, DEEP>(e, axis, 1, stream);
     default: return cudaErrorNotSupported;
     }
 }
 
+// Both axes in one grid for the rank pairs of the decode kernels; otherwise one grid per axis.
+template <bool DEEP> cudaError_t launch_tc_pair(const EncodeArgs &e, cudaStream_t stream)
+{
+    const int rk = e.r_k, rv = e.r_v;
+    if (rk == 16 && rv == 32) return launch_tc<16, 32, DEEP>(e, 0, 2, stream);
+    if (rk == 16 && rv == 16) return launch_tc<16, 16, DEEP>(e, 0, 2, stream);
+    if (rk == 32 && rv == 32) return launch_tc<32, 32, DEEP>(e, 0, 2, stream);
+    if (rk == 64 && rv == 128) return launch_tc<64, 128, DEEP>(e, 0, 2, stream);
+    if (rk == 96 && rv == 160) return launch_tc<96, 160, DEEP>(e, 0, 2, stream);
+    if (rk == 128 && rv == 128) return launch_tc<128, 128, DEEP>(e, 0, 2, stream);
+    cudaError_t err = launch_tc_single<DEEP>(e, 0, rk, stream);
+    if (err == cudaSuccess)
+        err = launch_tc_single<DEEP>(e, 1, rv, stream);
+    return err;
+}
+
 bool tc_rank_ok(int r) { return r == 16 || r == 32 || r == 48 || r == 64 || r == 96 || r == 128 || r == 160 || r == 192 || r == 256; }
+
+int device_sms()
+{
+    int dev = 0, n = 148;
+    if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+        return 148;
+    return n;
+}
 
 } // namespace
 
@@ -339,10 +406,9 @@ bool encode_tc_supported(const EncodeArgs &e)
 
 cudaError_t launch_encode_tc(const EncodeArgs &e, cudaStream_t stream)
 {
-    cudaError_t err = launch_tc_rank(e, 0, e.r_k, stream);
-    if (err == cudaSuccess)
-        err = launch_tc_rank(e, 1, e.r_v, stream);
-    return err;
+    // a grid that does not fill the GPU twice over gets the deep ring (latency-bound)
+    const int64_t ctas = ((e.n_tok + kBlockM - 1) / kBlockM) * (int64_t)e.Hs * e.n_layers * 2;
+    return ctas < 2 * device_sms() ? launch_tc_pair<true>(e, stream) : launch_tc_pair<false>(e, stream);
 }
 
 namespace {

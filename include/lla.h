@@ -147,9 +147,13 @@ int lla_encode(const lla_dims *dims, int32_t layer0, int32_t n_layers, const voi
  *   seq_start int64 [B], ctx_lens int32 [B]   (device; slots must lie in the plane)
  *   max_ctx  host-side upper bound of ctx_lens, used only to choose the split count
  *   num_splits  target number of token shares (split-K pieces) per (sequence, head);
- *               0 = automatic.  The work is spread evenly over resident CTAs, so a
- *               share never holds fewer than ceil(max_ctx / num_splits) tokens
- *   workspace   device scratch of at least lla_decode_workspace_bytes(...) bytes
+ *               0 = automatic.  The token stream of all (sequence, head) pairs is cut
+ *               into one equal share per resident CTA, never fewer than
+ *               ceil(max_ctx / num_splits) tokens.  Results are bitwise reproducible
+ *               for equal arguments.
+ *   workspace   device scratch of at least lla_decode_workspace_bytes(...) bytes; its
+ *               contents need not be initialised (the first word, the status, must be
+ *               zero -- lla_status_fetch leaves it so)
  * Errors: LLA_ERR_INVALID (dims, loop range, Tq < 1, pointers), LLA_ERR_UNSUPPORTED,
  * LLA_ERR_MISALIGNED, LLA_ERR_WORKSPACE, LLA_ERR_CUDA.                                  */
 int lla_decode_attn(const lla_dims *dims, int32_t layer, int32_t t0, int32_t Tq,

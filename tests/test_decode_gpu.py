@@ -5,7 +5,7 @@ import torch
 
 import decode_attention_12_b200 as lla
 import lla_synth as S
-from gpu_util import assert_attn_close, oracle_decode, run_decode
+from gpu_util import assert_attn_close, codec_of, dims_of, oracle_decode, run_decode
 
 pytestmark = pytest.mark.gpu
 DEV = "cuda"
@@ -63,11 +63,33 @@ def test_ouro_layer_model_order_single_loop(ouro, t0):
     assert_attn_close(out, lse, o_ref, l_ref)
 
 
-def test_decode_is_deterministic(ouro):
+@pytest.mark.parametrize("splits", [0, 3])
+def test_decode_is_deterministic(ouro, splits):
     w, p = ouro
-    a = run_decode(p, w, 0, 0, 4, 1.0)
-    b = run_decode(p, w, 0, 0, 4, 1.0)
+    a = run_decode(p, w, 0, 0, 4, 1.0, num_splits=splits)
+    b = run_decode(p, w, 0, 0, 4, 1.0, num_splits=splits)
+    assert a[2] == 0 and b[2] == 0
     assert torch.equal(a[0], b[0]) and torch.equal(a[1], b[1])
+
+
+def test_decode_with_dirty_workspace(ouro):
+    """The workspace needs no initialisation beyond its status word: one full of stale
+    bytes (here 0xff) gives the same result."""
+    w, p = ouro
+    dims = dims_of(w)
+    B, Tq = len(p["lens"]), 4
+    max_ctx = int(p["lens"].max())
+    nb = lla.decode_workspace_bytes(dims, B, Tq, max_ctx, lla.ABSORB, 0)
+    ws = torch.full((nb,), 255, dtype=torch.uint8, device="cuda")
+    ws[:4] = 0  # status word
+    out = torch.empty(B, Tq, w.H, w.d, device="cuda")
+    lse = torch.empty(B, Tq, w.H, device="cuda")
+    lla.decode_attn(dims, 0, 0, Tq, p["q"], lla.make_cache(p["k"], p["v"], p["slots"]), p["seq_start"],
+                    p["ctx_lens"], B, max_ctx, codec_of(p), 1.0, out, lse, ws, nb)
+    torch.cuda.synchronize()
+    assert lla.status_fetch(ws) == 0
+    ref = run_decode(p, w, 0, 0, 4, 1.0)
+    assert torch.equal(out, ref[0]) and torch.equal(lse, ref[1])
 
 
 # ---- edge cases -------------------------------------------------------------------------
@@ -75,7 +97,7 @@ EDGE_LENS = [0, 1, 2, 31, 255, 256, 257, 1000, 4097]
 
 
 @pytest.mark.parametrize("rk,rv", [(16, 32), (8, 16), (16, 16)])
-@pytest.mark.parametrize("splits", [1, 3, 8])
+@pytest.mark.parametrize("splits", [0, 1, 3, 8])
 def test_ragged_edges_bf16(rk, rv, splits):
     w = S.shrink(S.WORKLOADS["ouro1.4b-layer"], name=f"edge-{rk}-{rv}", r_k=rk, r_v=rv,
                  B=len(EDGE_LENS))
