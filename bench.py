@@ -62,6 +62,8 @@ def parse():
                     help="step: decode step (headline); encode: prefill encode of one layer")
     ap.add_argument("--encode-seqs", type=int, default=0,
                     help="--phase encode: sequences of len_hi tokens to encode (default: B)")
+    ap.add_argument("--model-order", action="store_true",
+                    help="one decode call per loop (Tq = 1, t = 0..T-1) instead of all loops fused")
     return ap.parse_args()
 
 
@@ -181,6 +183,8 @@ def oracle_sample_rate(p, w, Tq, max_seconds, units_per_round=None):
     q = f64(p["q"])
     cK, cV = f64(p["k"][0]), f64(p["v"][0])
     WK, WV, mK, mV = (f64(p[n][0]) for n in ("W_up_k", "W_up_v", "mu_k", "mu_v"))
+    if w.fold2d:  # one folded codec for all heads
+        WK, WV, mK, mV = WK[0], WV[0], mK[0], mV[0]
     threads = os.cpu_count() or 1
     all_units = [(b, h) for b in range(w.B) for h in range(w.H)]
     if units_per_round is None:
@@ -192,9 +196,11 @@ def oracle_sample_rate(p, w, Tq, max_seconds, units_per_round=None):
         pos += units_per_round
         t0 = time.perf_counter()
         oracle.decode_layer("absorb", q, cK, cV, p["starts"], lens, WK, mK, WV, mV, 0, 1.0,
-                            units=units, threads=threads)
+                            fold2d=w.fold2d, units=units, threads=threads)
         t_spent += time.perf_counter() - t0
-        bytes_done += sum(int(lens[b]) for b, _ in units) * (w.r_k + w.r_v) * w.elem_bytes
+        # latent bytes this share of the step covers (a folded latent serves all H heads)
+        bytes_done += (sum(int(lens[b]) for b, _ in units) * (w.r_k + w.r_v) * w.elem_bytes
+                       * w.heads_stored / w.H)
         rounds += 1
     info = {"cores": threads, "units": units_per_round, "rounds": rounds, "seconds": t_spent}
     return bytes_done / t_spent / 1e9, info
@@ -220,7 +226,7 @@ def run_reference(args, rank):
     dt = time.perf_counter() - t0
     value = statistics.median(rates)
     S_tot = int(p["lens"].sum())
-    step_bytes = S_tot * w.H * (w.r_k + w.r_v) * w.elem_bytes
+    step_bytes = S_tot * w.heads_stored * (w.r_k + w.r_v) * w.elem_bytes
     line = {
         "impl": "reference", "metric": METRIC, "value": value, "unit": "GB/s",
         "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
@@ -354,24 +360,34 @@ def main():
     x_v = S.draw_encode_tokens(w, 0, "v", B, dev, seed_tag="new")
     new_slot = (p["seq_start"] + p["ctx_lens"].to(torch.int64)).contiguous()
     variant = lla.RECONSTRUCT if args.variant == "reconstruct" else lla.ABSORB
-    ws_bytes = lla.decode_workspace_bytes(dims, B, Tq, max_ctx, variant, args.num_splits)
+    # decode calls of one step: all T loop queries fused (t0 = 0, Tq = T), or in model
+    # order one call per loop (t0 = t, Tq = 1) with each loop's queries and outputs in
+    # buffers of their own
+    calls = [(t, 1) for t in range(w.T)] if args.model_order else [(0, w.T)]
+    Tq_call = calls[0][1]
+    q_full = p["q"]
+    qs = [q_full[:, t0:t0 + n].contiguous() for t0, n in calls]
+    outs = [torch.empty(B, n, H, w.d, dtype=torch.float32, device=dev) for _, n in calls]
+    lses = [torch.empty(B, n, H, dtype=torch.float32, device=dev) for _, n in calls]
+    q, out, lse = q_full, outs[0], lses[0]
+    ws_bytes = lla.decode_workspace_bytes(dims, B, Tq_call, max_ctx, variant, args.num_splits)
     ws = torch.zeros(ws_bytes, dtype=torch.uint8, device=dev)
-    q = p["q"]
-    out = torch.empty(B, Tq, H, w.d, dtype=torch.float32, device=dev)
-    lse = torch.empty(B, Tq, H, dtype=torch.float32, device=dev)
     stream = torch.cuda.current_stream(dev)
-    splits = lla.decode_num_splits(dims, B, Tq, max_ctx, variant, args.num_splits)
+    splits = lla.decode_num_splits(dims, B, Tq_call, max_ctx, variant, args.num_splits)
 
-    def decode(i, q_in=q, out_buf=out, lse_buf=lse):
-        lla.decode_attn(dims, 0, 0, Tq, q_in, caches[i % R], p["seq_start"], p["ctx_lens"], B,
-                        max_ctx, codec, 1.0, out_buf, lse_buf, ws, ws_bytes, variant=variant,
-                        num_splits=args.num_splits, stream=stream)
+    def decode(i, q_in=None, out_buf=None, lse_buf=None):
+        for c, (t0, n) in enumerate(calls):
+            lla.decode_attn(dims, 0, t0, n, (q_in or qs)[c], caches[i % R], p["seq_start"], p["ctx_lens"], B,
+                            max_ctx, codec, 1.0, (out_buf or outs)[c], (lse_buf or lses)[c], ws, ws_bytes,
+                            variant=variant, num_splits=args.num_splits, stream=stream)
 
     def encode(i, xk=x_k, xv=x_v):
         lla.encode(dims, 0, 1, xk, xv, B, new_slot, codec, caches[i % R], stream=stream)
 
-    # prologue + decode + combine + 2 encode (K, V) kernels; reconstruct: Tq decode passes
-    launches_per_step = (3 if args.variant == "absorb" else Tq + 1) + 2
+    # per decode call: prologue + decode + combine (reconstruct: one decode pass per loop
+    # query + combine); the encode of K and V is one launch
+    per_call = 3 if args.variant == "absorb" else Tq_call + 1
+    launches_per_step = per_call * len(calls) + 1
     # ---- warm-up, then the device-timed region ------------------------------------------------
     sampler = ClockSampler(local).start()
     for i in range(args.warmup):
@@ -404,7 +420,8 @@ def main():
     if status != 0:
         raise RuntimeError(f"device status {status}: {lla.status_string(status)}")
 
-    step_bytes = S_tot * w.heads_stored * (w.r_k + w.r_v) * w.elem_bytes   # latents read per step
+    # latents read per step: one pass over the layer's latents per decode call
+    step_bytes = len(calls) * S_tot * w.heads_stored * (w.r_k + w.r_v) * w.elem_bytes
     ms_step = ms_total / args.steps
     value = world * step_bytes / (ms_step * 1e-3) / 1e9
     reads = world * S_tot * Tq / (ms_step * 1e-3)       # (token, layer, loop) reads per second
@@ -419,19 +436,20 @@ def main():
     # i+1's inputs and step i-1's results while step i computes (copy streams ordered by
     # events); the timed region runs from before the first input copy to after the last
     # result copy.
-    q_h = torch.empty_like(q, device="cpu").pin_memory()
-    q_h.copy_(q)
-    xk_h = torch.empty_like(x_k, device="cpu").pin_memory()
-    xk_h.copy_(x_k)
-    xv_h = torch.empty_like(x_v, device="cpu").pin_memory()
-    xv_h.copy_(x_v)
-    out_h = [torch.empty_like(out, device="cpu").pin_memory() for _ in range(2)]
-    lse_h = [torch.empty_like(lse, device="cpu").pin_memory() for _ in range(2)]
-    q_d = [torch.empty_like(q) for _ in range(2)]
+    def pinned(t):
+        h = torch.empty_like(t, device="cpu").pin_memory()
+        h.copy_(t)
+        return h
+
+    q_h = [pinned(t) for t in qs]
+    xk_h, xv_h = pinned(x_k), pinned(x_v)
+    out_h = [[torch.empty_like(t, device="cpu").pin_memory() for t in outs] for _ in range(2)]
+    lse_h = [[torch.empty_like(t, device="cpu").pin_memory() for t in lses] for _ in range(2)]
+    q_d = [[torch.empty_like(t) for t in qs] for _ in range(2)]
     xk_d = [torch.empty_like(x_k) for _ in range(2)]
     xv_d = [torch.empty_like(x_v) for _ in range(2)]
-    out_d = [torch.empty_like(out) for _ in range(2)]
-    lse_d = [torch.empty_like(lse) for _ in range(2)]
+    out_d = [[torch.empty_like(t) for t in outs] for _ in range(2)]
+    lse_d = [[torch.empty_like(t) for t in lses] for _ in range(2)]
     s_in, s_out = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
     in_ready = [torch.cuda.Event() for _ in range(2)]
     comp_done = [torch.cuda.Event() for _ in range(2)]
@@ -443,7 +461,8 @@ def main():
         if i >= 2:
             s_in.wait_event(comp_done[sl])      # step i-2 is done with this input slot
         with torch.cuda.stream(s_in):
-            q_d[sl].copy_(q_h, non_blocking=True)
+            for dq, hq in zip(q_d[sl], q_h):
+                dq.copy_(hq, non_blocking=True)
             xk_d[sl].copy_(xk_h, non_blocking=True)
             xv_d[sl].copy_(xv_h, non_blocking=True)
         in_ready[sl].record(s_in)
@@ -455,8 +474,10 @@ def main():
         comp_done[sl].record(stream)
         s_out.wait_event(comp_done[sl])
         with torch.cuda.stream(s_out):
-            out_h[sl].copy_(out_d[sl], non_blocking=True)
-            lse_h[sl].copy_(lse_d[sl], non_blocking=True)
+            for ho, do in zip(out_h[sl], out_d[sl]):
+                ho.copy_(do, non_blocking=True)
+            for hl, dl in zip(lse_h[sl], lse_d[sl]):
+                hl.copy_(dl, non_blocking=True)
         out_read[sl].record(s_out)
 
     for i in range(min(args.warmup, 10)):
@@ -477,8 +498,8 @@ def main():
     torch.cuda.synchronize()
     e2e_ms = max_over_ranks(e0.elapsed_time(e1), dev)
     e2e_value = world * step_bytes * e2e_steps / (e2e_ms * 1e-3) / 1e9
-    h2d = (q.numel() * q.element_size() + x_k.numel() * x_k.element_size() * 2)
-    d2h = out.numel() * out.element_size() + lse.numel() * lse.element_size()
+    h2d = sum(t.numel() * t.element_size() for t in qs) + x_k.numel() * x_k.element_size() * 2
+    d2h = sum(t.numel() * t.element_size() for t in outs + lses)
     status = lla.status_fetch(ws)
     if status != 0:
         raise RuntimeError(f"device status after the end-to-end steps {status}: {lla.status_string(status)}")
@@ -504,9 +525,11 @@ def main():
         "dtype": "f32", "storage_dtype": w.dtype, "data": "synthetic",
         "config": {"workload": w.name, "T": w.T, "L_per_step": 1, "H": H, "d": w.d,
                    "r_k": w.r_k, "r_v": w.r_v, "rho": "64/3", "B": B,
-                   "ctx_len": [w.len_lo, w.len_hi], "tokens": S_tot, "Tq": Tq,
+                   "ctx_len": [w.len_lo, w.len_hi], "tokens": S_tot, "Tq": Tq_call, "decode_calls_per_step": len(calls),
                    "variant": args.variant, "seg_max": splits,
-                   "step": "decode_attn(all 4 loop queries) + encode(B new tokens)",
+                   "step": (f"{len(calls)} x decode_attn(Tq = 1, one loop each, model order)"
+                            if args.model_order else f"decode_attn(all {w.T} loop queries fused)")
+                           + " + encode(B new tokens)",
                    "l2": f"inputs larger than L2 ({step_bytes / 1e6:.0f} MB of latents per step) "
                          f"and {R} rotating cache replicas",
                    "parallelism": f"replicas x{world}"},

@@ -76,6 +76,9 @@ __global__ void __launch_bounds__((NW + 1) * 32, MINB)
         fence_barrier_init();
     }
     block_length_prefix<kThreads>(a.ctx_lens, B, pref, reinterpret_cast<int64_t *>(smem + C::SCR_OFF));
+    // The combine grid may take SM slots (and stage its inputs) as this grid's CTAs exit;
+    // it reads nothing of ours before its own programmatic-launch wait.
+    grid_launch_dependents();
     int64_t s0, s1, chunk;
     cta_share(pref, B, H, a.chunk_min, s0, s1, chunk);
     if (s0 >= s1)
