@@ -49,6 +49,11 @@ bool decode_absorb_supported(int dtype, int r_k, int r_v, int d, int fold);
 bool decode_mma_supported(int dtype, int r_k, int r_v, int fold, int Tq);
 cudaError_t launch_decode_absorb_mma(const DecodeArgs &a, int ctas, cudaStream_t stream);
 bool decode_reconstruct_supported(int dtype, int r_k, int r_v, int d);
+// LLA-2D: every latent tile read once for all heads of a sequence (H * loops <= 64 rows
+// per pass); records in the per-(sequence, head) layout of the other kernels.
+bool decode_mma2d_supported(int dtype, int r_k, int r_v, int fold, int H);
+int decode_mma2d_loops_per_pass(int H);
+cudaError_t launch_decode_absorb_2d(const DecodeArgs &a, cudaStream_t stream);
 cudaError_t launch_decode_reconstruct(const DecodeArgs &a, cudaStream_t stream);
 
 } // namespace lla

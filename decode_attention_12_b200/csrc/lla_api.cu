@@ -76,6 +76,11 @@ Plan make_plan(const lla_dims *d, int32_t B, int32_t Tq, int32_t max_ctx, int32_
     if (segs > 64) segs = 64;
     int64_t chunk_min = (max_ctx + segs - 1) / segs;
     if (chunk_min < 128) chunk_min = 128;
+    // LLA-2D: units are whole sequences and each segment writes H x Tq records, so by
+    // default a share holds at least 384 tokens (records stay a small part of the traffic)
+    if (num_splits == 0 && variant == LLA_ABSORB &&
+        decode_mma2d_supported(d->dtype, d->r_k, d->r_v, d->fold, d->H))
+        chunk_min = 384;
     p.chunk_min = (int32_t)chunk_min;
     p.seg_max = (int32_t)((max_ctx + chunk_min - 1) / chunk_min + 1);
     p.off_counts = kWorkspaceHeader;
@@ -319,6 +324,22 @@ int lla_decode_attn(const lla_dims *dims, int32_t layer, int32_t t0, int32_t Tq,
         }
         if (err == cudaSuccess)
             err = launch_decode_combine(a, dims->dtype, dims->out_dtype, s);
+        return err == cudaSuccess ? LLA_OK : LLA_ERR_CUDA;
+    }
+    if (decode_mma2d_supported(dims->dtype, dims->r_k, dims->r_v, dims->fold, dims->H)) {
+        // LLA-2D: all heads of a sequence share each latent tile; passes of H * loops <= 64
+        // query rows
+        const int per = decode_mma2d_loops_per_pass(dims->H);
+        for (int32_t c = 0; c < Tq && err == cudaSuccess; c += per) {
+            DecodeArgs ac = a;
+            ac.tq_off = c;
+            ac.Tq = Tq - c < per ? Tq - c : per;
+            err = launch_absorb_prologue(ac, dims->dtype, s);
+            if (err == cudaSuccess)
+                err = launch_decode_absorb_2d(ac, s);
+            if (err == cudaSuccess)
+                err = launch_decode_combine(ac, dims->dtype, dims->out_dtype, s);
+        }
         return err == cudaSuccess ? LLA_OK : LLA_ERR_CUDA;
     }
     if (use_mma) {

@@ -42,7 +42,7 @@ def test_deep_recurrence_T32(Tq, t0):
     assert_attn_close(out, lse, o_ref, l_ref)
 
 
-@pytest.mark.parametrize("Tq,t0", [(4, 0), (1, 2)])
+@pytest.mark.parametrize("Tq,t0", [(4, 0), (1, 2), (2, 1), (3, 1)])
 def test_lla2d_folded_heads(Tq, t0):
     w = S.WORKLOADS["lla2d"]
     layer = 23
@@ -78,3 +78,22 @@ def test_long_context_8x16k_full_layer():
     assert st == 0
     o_ref, l_ref = oracle_decode(p, w, layer, 0, 4, 1.0)
     assert_attn_close(out, lse, o_ref, l_ref)
+
+
+LLA2D_EDGE_LENS = [0, 1, 31, 64, 65, 383, 384, 385, 1000, 4096]
+
+
+@pytest.mark.parametrize("Tq,t0", [(4, 0), (1, 3)])
+def test_lla2d_ragged_and_empty_contexts(Tq, t0):
+    """LLA-2D with ragged contexts (empty, one token, tile and share boundaries +-1):
+    every head of every sequence against the oracle; an empty context gives out = 0 and
+    lse = -inf."""
+    w = S.shrink(S.WORKLOADS["lla2d"], name="lla2d-edge", L=2, B=len(LLA2D_EDGE_LENS))
+    layer = 1
+    p = S.decode_inputs(w, layer, DEV, Tq=Tq, lens=LLA2D_EDGE_LENS, gap=3)
+    out, lse, st = run_decode(p, w, layer, t0, Tq, 1.0)
+    assert st == 0
+    units = [(b, h) for b in range(w.B) for h in range(w.H)]
+    o_ref, l_ref = oracle_decode_units(p, w, layer, t0, Tq, 1.0, units)
+    assert_attn_close(out, lse, o_ref, l_ref)
+    assert torch.all(out[0] == 0) and torch.all(torch.isneginf(lse[0]))
