@@ -114,7 +114,30 @@ struct EncTcArgs {
     const int64_t *slot_idx;
     int64_t n_tok, slots;
     int32_t layer0, Hs, nk, d_slabs, fold, axis0;
+    int32_t ksplit;        // CTAs of a cluster sharing one tile's K slabs (1: no split)
 };
+
+__device__ __forceinline__ uint32_t cluster_ctarank()
+{
+    uint32_t r;
+    asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+    return r;
+}
+__device__ __forceinline__ void cluster_sync_all()
+{
+    asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+__device__ __forceinline__ float4 ld_peer_f4(uint32_t local_addr, uint32_t rank)
+{
+    uint32_t remote;
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(remote) : "r"(local_addr), "r"(rank));
+    float4 v;
+    asm volatile("ld.shared::cluster.v4.f32 {%0, %1, %2, %3}, [%4];"
+                 : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
+                 : "r"(remote)
+                 : "memory");
+    return v;
+}
 
 // Ring depth: a shallow ring (~110 KB) leaves room for two CTAs per SM on large grids;
 // a grid smaller than the GPU gets every K slab in flight at once (<= 8 stages).
@@ -134,7 +157,10 @@ template <int N, bool DEEP> struct EncCfg {
     static_assert(N % 16 == 0 && N >= 16 && N <= 256, "tcgen05 N for M = 128");
 };
 
-// One 128-token x N tile of one (layer, stored head, axis).
+// One 128-token x N tile of one (layer, stored head, axis).  With a.ksplit > 1 the CTAs of
+// a cluster each take a contiguous share of the K slabs; their fp32 partial tiles meet in
+// shared memory (the idle ring) and every CTA reduces a share of the rows across the
+// cluster (distributed shared memory) before the bias and the bf16 store.
 template <int N, bool DEEP>
 __device__ __forceinline__ void encode_tile(uint8_t *smem, const CUtensorMap *map_a, const CUtensorMap *map_b,
                                             const EncTcArgs &a, const EncTcAxis &ax, int m0, int hs, int li)
@@ -175,12 +201,15 @@ __device__ __forceinline__ void encode_tile(uint8_t *smem, const CUtensorMap *ma
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = hold[0];
+    const int krank = a.ksplit > 1 ? (int)cluster_ctarank() : 0;
+    const int kper = (a.nk + a.ksplit - 1) / a.ksplit;
+    const int kb0 = krank * kper, nkl = min(a.nk, kb0 + kper) - kb0; // this CTA's K slabs
 
     if (warp == 0 && lane == 0) {
         // ---- TMA producer
-        for (int kb = 0; kb < a.nk; ++kb) {
-            const int s = kb % C::STAGES;
-            if (kb >= C::STAGES && !mbar_wait_bounded(empty0 + 8 * s, ((kb / C::STAGES) - 1) & 1)) {
+        for (int kl = 0; kl < nkl; ++kl) {
+            const int kb = kb0 + kl, s = kl % C::STAGES;
+            if (kl >= C::STAGES && !mbar_wait_bounded(empty0 + 8 * s, ((kl / C::STAGES) - 1) & 1)) {
                 hold[1] = 1;
                 break;
             }
@@ -196,9 +225,9 @@ __device__ __forceinline__ void encode_tile(uint8_t *smem, const CUtensorMap *ma
         // ---- MMA issuer
         constexpr uint32_t idesc = idesc_bf16_f32(N);
         bool ok = true;
-        for (int kb = 0; kb < a.nk; ++kb) {
-            const int s = kb % C::STAGES;
-            if (!mbar_wait_bounded(full0 + 8 * s, (kb / C::STAGES) & 1)) {
+        for (int kl = 0; kl < nkl; ++kl) {
+            const int s = kl % C::STAGES;
+            if (!mbar_wait_bounded(full0 + 8 * s, (kl / C::STAGES) & 1)) {
                 hold[1] = 1;
                 ok = false;
                 break;
@@ -208,7 +237,7 @@ __device__ __forceinline__ void encode_tile(uint8_t *smem, const CUtensorMap *ma
 #pragma unroll
             for (int k = 0; k < kSlabK / 16; ++k)
                 tc_mma(tmem, smem_desc_sw128(a_addr + 32 * k), smem_desc_sw128(b_addr + 32 * k), idesc,
-                       (kb | k) != 0);
+                       (kl | k) != 0);
             tc_commit(empty0 + 8 * s); // frees the stage once these MMAs have read it
         }
         if (ok)
@@ -226,10 +255,48 @@ __device__ __forceinline__ void encode_tile(uint8_t *smem, const CUtensorMap *ma
     // ---- epilogue: all 4 warps, warp w owns accumulator lanes (tokens) 32w .. 32w+31
     const bool acc_ok = mbar_wait_bounded(accb, 0);
     tc_fence_after();
-    if (!acc_ok || hold[1]) {
-        if (threadIdx.x == 0)
-            report_status(&g_encode_status, LLA_ERR_DEVICE_TIMEOUT);
-    } else {
+    const bool good = acc_ok && !hold[1] && nkl > 0;
+    if (!good && nkl > 0 && threadIdx.x == 0)
+        report_status(&g_encode_status, LLA_ERR_DEVICE_TIMEOUT);
+    if (a.ksplit > 1) {
+        // ---- split K: partial rows into the (idle) ring, reduction across the cluster
+        static_assert(!DEEP || C::STAGES * C::STAGE >= kBlockM * N * 4, "ring holds the fp32 partial tile");
+        float *red = reinterpret_cast<float *>(smem); // [128][N]
+        const int row = warp * 32 + lane;
+#pragma unroll 1
+        for (int c = 0; c < N / 16; ++c) {
+            uint32_t r[16];
+            tmem_ld16(tmem + ((uint32_t)(warp * 32) << 16) + c * 16, r);
+#pragma unroll
+            for (int e = 0; e < 16; e += 4)
+                *reinterpret_cast<float4 *>(red + row * N + c * 16 + e) =
+                    good ? make_float4(__uint_as_float(r[e]), __uint_as_float(r[e + 1]), __uint_as_float(r[e + 2]),
+                                       __uint_as_float(r[e + 3]))
+                         : make_float4(0.f, 0.f, 0.f, 0.f);
+        }
+        cluster_sync_all(); // every partial tile is written
+        const int rows = (int)min((int64_t)kBlockM, a.n_tok - m0);
+        const int per = (rows + a.ksplit - 1) / a.ksplit, r0 = krank * per, r1 = min(rows, r0 + per);
+        __nv_bfloat16 *dst = static_cast<__nv_bfloat16 *>(ax.plane) + (((int64_t)l * a.Hs + hs) * a.slots) * N;
+        const uint32_t red_addr = smem_u32(red);
+        for (int it = threadIdx.x; it < (r1 - r0) * (N / 4); it += kThreads) {
+            const int rr = r0 + it / (N / 4), c4 = 4 * (it % (N / 4));
+            float4 acc = make_float4(bias_s[c4], bias_s[c4 + 1], bias_s[c4 + 2], bias_s[c4 + 3]);
+            for (int p = 0; p < a.ksplit; ++p) {
+                const float4 v = ld_peer_f4(red_addr + (uint32_t)(rr * N + c4) * 4u, (uint32_t)p);
+                acc.x += v.x, acc.y += v.y, acc.z += v.z, acc.w += v.w;
+            }
+            int64_t sl = a.slot_idx[m0 + rr];
+            if (sl >= 0 && sl < a.slots) {
+                const __nv_bfloat162 lo = __floats2bfloat162_rn(acc.x, acc.y), hi = __floats2bfloat162_rn(acc.z, acc.w);
+                uint2 w;
+                w.x = *reinterpret_cast<const uint32_t *>(&lo);
+                w.y = *reinterpret_cast<const uint32_t *>(&hi);
+                *reinterpret_cast<uint2 *>(dst + sl * N + c4) = w;
+            }
+        }
+        cluster_sync_all(); // peers are done reading this CTA's partial tile
+    } else if (good) {
         __nv_bfloat16 *dst = static_cast<__nv_bfloat16 *>(ax.plane) + (((int64_t)l * a.Hs + hs) * a.slots) * N;
 #pragma unroll 1
         for (int c = 0; c < N / 16; ++c) {
@@ -269,10 +336,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     // aligned by arithmetic on the shared array itself, so accesses stay shared-space loads
     uint8_t *smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
     const int axis = a.axis0 + (int)blockIdx.y / a.Hs, hs = (int)blockIdx.y % a.Hs;
+    const int m0 = (int)(blockIdx.x / a.ksplit) * kBlockM; // a cluster of ksplit CTAs per tile
     if (axis == 0)
-        encode_tile<NK, DEEP>(smem, &map_ak, &map_bk, a, a.ax[0], blockIdx.x * kBlockM, hs, blockIdx.z);
+        encode_tile<NK, DEEP>(smem, &map_ak, &map_bk, a, a.ax[0], m0, hs, blockIdx.z);
     else
-        encode_tile<NV, DEEP>(smem, &map_av, &map_bv, a, a.ax[1], blockIdx.x * kBlockM, hs, blockIdx.z);
+        encode_tile<NV, DEEP>(smem, &map_av, &map_bv, a, a.ax[1], m0, hs, blockIdx.z);
 }
 
 // ---- host: tensor maps ------------------------------------------------------------------------
@@ -316,9 +384,10 @@ bool axis_maps(const EncodeArgs &e, int axis, int N, CUtensorMap *ma, CUtensorMa
     return make_map(mb, wd, 3, dims, str, box);
 }
 
-// Launch axes [axis0, axis0 + n_axes) of one encode in one grid.
+// Launch axes [axis0, axis0 + n_axes) of one encode in one grid; ksplit > 1 runs every tile
+// as a cluster of ksplit CTAs that share its K slabs (deep ring only).
 template <int NK, int NV, bool DEEP>
-cudaError_t launch_tc(const EncodeArgs &e, int axis0, int n_axes, cudaStream_t stream)
+cudaError_t launch_tc(const EncodeArgs &e, int axis0, int n_axes, cudaStream_t stream, int ksplit = 1)
 {
     CUtensorMap mak, mbk, mav, mbv;
     std::memset(&mak, 0, sizeof(mak));
@@ -343,46 +412,58 @@ cudaError_t launch_tc(const EncodeArgs &e, int axis0, int n_axes, cudaStream_t s
     a.d_slabs = e.d / kSlabK;
     a.fold = e.fold;
     a.axis0 = axis0;
+    a.ksplit = DEEP ? ksplit : 1;
     auto kern = encode_tc_kernel<NK, NV, DEEP>;
     const int smem = EncCfg<NK, DEEP>::SMEM > EncCfg<NV, DEEP>::SMEM ? EncCfg<NK, DEEP>::SMEM
                                                                        : EncCfg<NV, DEEP>::SMEM;
     cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (err != cudaSuccess)
         return err;
-    dim3 grid((unsigned)((e.n_tok + kBlockM - 1) / kBlockM), n_axes * e.Hs, e.n_layers);
-    kern<<<grid, kThreads, smem, stream>>>(mak, mbk, mav, mbv, a);
-    return cudaGetLastError();
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)((e.n_tok + kBlockM - 1) / kBlockM) * a.ksplit, n_axes * e.Hs, e.n_layers);
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = a.ksplit;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = a.ksplit > 1 ? 1 : 0;
+    return cudaLaunchKernelEx(&cfg, kern, mak, mbk, mav, mbv, a);
 }
 
-template <bool DEEP> cudaError_t launch_tc_single(const EncodeArgs &e, int axis, int r, cudaStream_t stream)
+template <bool DEEP>
+cudaError_t launch_tc_single(const EncodeArgs &e, int axis, int r, cudaStream_t stream, int ks)
 {
     switch (r) {
-    case 16: return launch_tc<16, 16, DEEP>(e, axis, 1, stream);
-    case 32: return launch_tc<32, 32, DEEP>(e, axis, 1, stream);
-    case 48: return launch_tc<48, 48, DEEP>(e, axis, 1, stream);
-    case 64: return launch_tc<64, 64, DEEP>(e, axis, 1, stream);
-    case 96: return launch_tc<96, 96, DEEP>(e, axis, 1, stream);
-    case 128: return launch_tc<128, 128, DEEP>(e, axis, 1, stream);
-    case 160: return launch_tc<160, 160, DEEP>(e, axis, 1, stream);
-    case 192: return launch_tc<192, 192, DEEP>(e, axis, 1, stream);
-    case 256: return launch_tc<256, 256, DEEP>(e, axis, 1, stream);
+    case 16: return launch_tc<16, 16, DEEP>(e, axis, 1, stream, ks);
+    case 32: return launch_tc<32, 32, DEEP>(e, axis, 1, stream, ks);
+    case 48: return launch_tc<48, 48, DEEP>(e, axis, 1, stream, ks);
+    case 64: return launch_tc<64, 64, DEEP>(e, axis, 1, stream, ks);
+    case 96: return launch_tc<96, 96, DEEP>(e, axis, 1, stream, ks);
+    case 128: return launch_tc<128, 128, DEEP>(e, axis, 1, stream, ks);
+    case 160: return launch_tc<160, 160, DEEP>(e, axis, 1, stream, ks);
+    case 192: return launch_tc<192, 192, DEEP>(e, axis, 1, stream, ks);
+    case 256: return launch_tc<256, 256, DEEP>(e, axis, 1, stream, ks);
     default: return cudaErrorNotSupported;
     }
 }
 
 // Both axes in one grid for the rank pairs of the decode kernels; otherwise one grid per axis.
-template <bool DEEP> cudaError_t launch_tc_pair(const EncodeArgs &e, cudaStream_t stream)
+template <bool DEEP> cudaError_t launch_tc_pair(const EncodeArgs &e, cudaStream_t stream, int ks)
 {
     const int rk = e.r_k, rv = e.r_v;
-    if (rk == 16 && rv == 32) return launch_tc<16, 32, DEEP>(e, 0, 2, stream);
-    if (rk == 16 && rv == 16) return launch_tc<16, 16, DEEP>(e, 0, 2, stream);
-    if (rk == 32 && rv == 32) return launch_tc<32, 32, DEEP>(e, 0, 2, stream);
-    if (rk == 64 && rv == 128) return launch_tc<64, 128, DEEP>(e, 0, 2, stream);
-    if (rk == 96 && rv == 160) return launch_tc<96, 160, DEEP>(e, 0, 2, stream);
-    if (rk == 128 && rv == 128) return launch_tc<128, 128, DEEP>(e, 0, 2, stream);
-    cudaError_t err = launch_tc_single<DEEP>(e, 0, rk, stream);
+    if (rk == 16 && rv == 32) return launch_tc<16, 32, DEEP>(e, 0, 2, stream, ks);
+    if (rk == 16 && rv == 16) return launch_tc<16, 16, DEEP>(e, 0, 2, stream, ks);
+    if (rk == 32 && rv == 32) return launch_tc<32, 32, DEEP>(e, 0, 2, stream, ks);
+    if (rk == 64 && rv == 128) return launch_tc<64, 128, DEEP>(e, 0, 2, stream, ks);
+    if (rk == 96 && rv == 160) return launch_tc<96, 160, DEEP>(e, 0, 2, stream, ks);
+    if (rk == 128 && rv == 128) return launch_tc<128, 128, DEEP>(e, 0, 2, stream, ks);
+    cudaError_t err = launch_tc_single<DEEP>(e, 0, rk, stream, ks);
     if (err == cudaSuccess)
-        err = launch_tc_single<DEEP>(e, 1, rv, stream);
+        err = launch_tc_single<DEEP>(e, 1, rv, stream, ks);
     return err;
 }
 
@@ -406,9 +487,17 @@ bool encode_tc_supported(const EncodeArgs &e)
 
 cudaError_t launch_encode_tc(const EncodeArgs &e, cudaStream_t stream)
 {
-    // a grid that does not fill the GPU twice over gets the deep ring (latency-bound)
+    // A grid that does not fill the GPU twice over gets the deep ring (latency-bound).  One
+    // that leaves most SMs idle, with more K slabs than one ring pass (8), also splits each
+    // tile's slabs over a cluster of up to 8 CTAs, so every CTA's slabs are in flight at once.
     const int64_t ctas = ((e.n_tok + kBlockM - 1) / kBlockM) * (int64_t)e.Hs * e.n_layers * 2;
-    return ctas < 2 * device_sms() ? launch_tc_pair<true>(e, stream) : launch_tc_pair<false>(e, stream);
+    const int sms = device_sms();
+    if (ctas >= 2 * sms)
+        return launch_tc_pair<false>(e, stream, 1);
+    const int nk = e.W / kSlabK, passes = (nk + 7) / 8;
+    int ks = ctas < sms ? (int)(sms / ctas < 8 ? sms / ctas : 8) : 1;
+    ks = ks < passes ? ks : passes;
+    return launch_tc_pair<true>(e, stream, ks < 1 ? 1 : ks);
 }
 
 namespace {
