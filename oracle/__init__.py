@@ -65,6 +65,9 @@ def configure(lib):
         f.argtypes = [i64, i32, i32, i32, _dp, _dp, _dp, _dp, _dp, _dp, _dp,
                       ctypes.c_double, _dp, _dp]
         f.restype = i32
+    lib.oracle_attend_hybrid.argtypes = [i64, i64, i32, i32, i32, _dp, _dp, _dp, _dp, _dp, _dp, _dp, _dp,
+                                         _dp, ctypes.c_double, _dp, _dp]
+    lib.oracle_attend_hybrid.restype = i32
     return lib
 
 
@@ -151,11 +154,37 @@ def attend(variant, c_K, c_V, W_up_K_t, mu_K_t, W_up_V_t, mu_V_t, q, scale):
     return o, float(lse.value)
 
 
+def attend_hybrid(c_K, c_V, W_up_K_t, mu_K_t, W_up_V_t, mu_V_t, k_win, v_win, q, scale):
+    """One loop query over n older tokens (latents) and w window tokens (exact K/V).
+
+    c_K [n, r_k], c_V [n, r_v], codec slices as in ``attend``, k_win / v_win [w, d],
+    q [d]  ->  (o [d], lse).
+    """
+    c_K, c_V = _f64(c_K), _f64(c_V)
+    W_up_K_t, mu_K_t, W_up_V_t, mu_V_t, q = map(_f64, (W_up_K_t, mu_K_t, W_up_V_t, mu_V_t, q))
+    k_win, v_win = _f64(k_win), _f64(v_win)
+    n, w = c_K.shape[0], k_win.shape[0]
+    r_k, r_v, d = W_up_K_t.shape[0], W_up_V_t.shape[0], q.shape[0]
+    if n == 0:
+        c_K = np.zeros((1, r_k)); c_V = np.zeros((1, r_v))
+    if w == 0:
+        k_win = np.zeros((1, d)); v_win = np.zeros((1, d))
+    assert k_win.shape[1] == d and v_win.shape == k_win.shape
+    o = np.empty(d, dtype=np.float64)
+    lse = ctypes.c_double(0.0)
+    rc = _load().oracle_attend_hybrid(n, w, r_k, r_v, d, _ptr(c_K), _ptr(c_V), _ptr(W_up_K_t),
+                                      _ptr(mu_K_t), _ptr(W_up_V_t), _ptr(mu_V_t), _ptr(k_win),
+                                      _ptr(v_win), _ptr(q), float(scale), _ptr(o), ctypes.byref(lse))
+    if rc != 0:
+        raise MemoryError("oracle scratch allocation failed")
+    return o, float(lse.value)
+
+
 # --------------------------------------------------------------------------
 # A whole decode call for one layer: loop over (b, loop t, head) instances
 # --------------------------------------------------------------------------
 def decode_layer(variant, q, c_K, c_V, seq_start, ctx_lens, W_up_K, mu_K, W_up_V, mu_V,
-                 t0, scale, fold2d=False, units=None, threads=None):
+                 t0, scale, fold2d=False, units=None, threads=None, window=None):
     """Decode attention of every (b, tq, h) query of one layer.
 
     q        [B, Tq, H, d]           loop queries t0 .. t0+Tq-1
@@ -164,6 +193,10 @@ def decode_layer(variant, q, c_K, c_V, seq_start, ctx_lens, W_up_K, mu_K, W_up_V
     W_up_K   per-head [H, T, r_k, d]    LLA-2D [T, r_k, H*d]   (same for V)
     mu_K     per-head [H, T, d]         LLA-2D [T, H*d]
     units    optional iterable of (b, h) pairs to evaluate (default: all)
+    window   optional (win_k, win_v, win_len): exact loop keys / values of each
+             sequence's window tokens, win_k [B, H, T, w_max, d], win_len [B]; the
+             hybrid form then attends over the ctx_lens[b] latents and the
+             win_len[b] window tokens together (variant is ignored)
     Returns (o [B, Tq, H, d], lse [B, Tq, H]); entries outside ``units`` are NaN.
     """
     q = np.asarray(q)
@@ -187,8 +220,15 @@ def decode_layer(variant, q, c_K, c_V, seq_start, ctx_lens, W_up_K, mu_K, W_up_V
         cV = c_V[hp, s0:s0 + n]
         for tq in range(Tq):
             wk, mk, wv, mv = slices(h, t0 + tq)
-            o[b, tq, h], lse[b, tq, h] = attend(variant, cK, cV, wk, mk, wv, mv,
-                                                q[b, tq, h], scale)
+            if window is None:
+                o[b, tq, h], lse[b, tq, h] = attend(variant, cK, cV, wk, mk, wv, mv,
+                                                    q[b, tq, h], scale)
+            else:
+                win_k, win_v, win_len = window
+                nw = int(win_len[b])
+                o[b, tq, h], lse[b, tq, h] = attend_hybrid(
+                    cK, cV, wk, mk, wv, mv, win_k[b, h, t0 + tq, :nw], win_v[b, h, t0 + tq, :nw],
+                    q[b, tq, h], scale)
 
     units = list(units)
     if threads is None:

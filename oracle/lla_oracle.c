@@ -18,6 +18,9 @@
  *       "absorbed-attention variant") and key_machinery.
  *  [A]  Same paper, arXiv abstract -- LLA-2D folds the heads into one latent;
  *       K/V are reconstructed "only when attention reads them".
+ *  [HLA] "Hybrid Latent Attention for Looped Language Models", abstract -- exact
+ *       keys and values for a sliding window of W recent tokens, latents for the
+ *       older tokens, read by every loop's query.
  *
  * Conventions (all arrays row-major, caller-owned, doubles):
  *  - one stacked vector per token x in R^W with W = T*d (per-head) or W = T*H*d
@@ -226,5 +229,64 @@ int oracle_attend_absorb(int64_t n, int r_k, int r_v, int d,
         o[k] = acc;
     }
     free(q_tilde); free(o_lat); free(l); free(p);
+    return 0;
+}
+
+/* ---------------------------------------------------------------------------
+ * Hybrid decode attention ([HLA] abstract): the sequence's w most recent tokens
+ * keep their exact loop-t keys and values (the sliding window), its n older
+ * tokens are latents.  The loop-t query attends over all n + w tokens at once:
+ *   older token i:   k_i = c_K[i] W_up,t^K + mu_t^K,   v_i = c_V[i] W_up,t^V + mu_t^V
+ *   window token m:  k = k_win[m],                    v = v_win[m]
+ *   l = scale * q . k over the n + w tokens, p = softmax(l), o = sum p v,
+ *   lse = log sum exp(l).
+ *   k_win, v_win [w][d].  n + w = 0 gives o = 0 and lse = -inf.
+ * Returns 0, or -1 if scratch memory could not be allocated.
+ * ------------------------------------------------------------------------- */
+int oracle_attend_hybrid(int64_t n, int64_t w, int r_k, int r_v, int d,
+                         const double *c_K, const double *c_V,
+                         const double *W_up_K_t, const double *mu_K_t,
+                         const double *W_up_V_t, const double *mu_V_t,
+                         const double *k_win, const double *v_win,
+                         const double *q, double scale, double *o, double *lse)
+{
+    const int64_t total = n + w;
+    for (int k = 0; k < d; ++k)
+        o[k] = 0.0;
+    if (total == 0) {
+        *lse = -INFINITY;
+        return 0;
+    }
+    double *k_hat = malloc(sizeof(double) * (size_t)d);
+    double *v_hat = malloc(sizeof(double) * (size_t)d);
+    double *l = malloc(sizeof(double) * (size_t)total);
+    double *p = malloc(sizeof(double) * (size_t)total);
+    if (!k_hat || !v_hat || !l || !p) {
+        free(k_hat); free(v_hat); free(l); free(p);
+        return -1;
+    }
+    for (int64_t i = 0; i < n; ++i) { /* older tokens: rebuilt loop-t keys */
+        oracle_reconstruct(1, r_k, d, c_K + i * r_k, W_up_K_t, mu_K_t, k_hat);
+        double dotc = 0.0;
+        for (int k = 0; k < d; ++k)
+            dotc += q[k] * k_hat[k];
+        l[i] = scale * dotc;
+    }
+    for (int64_t m = 0; m < w; ++m) { /* window tokens: exact loop-t keys */
+        double dotw = 0.0;
+        for (int k = 0; k < d; ++k)
+            dotw += q[k] * k_win[m * d + k];
+        l[n + m] = scale * dotw;
+    }
+    softmax_rows(total, l, p, lse);
+    for (int64_t i = 0; i < n; ++i) {
+        oracle_reconstruct(1, r_v, d, c_V + i * r_v, W_up_V_t, mu_V_t, v_hat);
+        for (int k = 0; k < d; ++k)
+            o[k] += v_hat[k] * p[i];
+    }
+    for (int64_t m = 0; m < w; ++m)
+        for (int k = 0; k < d; ++k)
+            o[k] += p[n + m] * v_win[m * d + k];
+    free(k_hat); free(v_hat); free(l); free(p);
     return 0;
 }

@@ -37,6 +37,12 @@ MUTANTS = {
                                      "o_lat[j] += p[i] * c_V[i * r_v + (r_v - 1 - j)];"),
     "absorb_wrong_key_latent_row": ("dot += q_tilde[j] * c_K[i * r_k + j];",
                                     "dot += q_tilde[j] * c_K[(n - 1 - i) * r_k + j];"),
+    "hybrid_latent_key_reversed": ("dotc += q[k] * k_hat[k];", "dotc += q[k] * k_hat[d - 1 - k];"),
+    "hybrid_window_drops_scale": ("l[n + m] = scale * dotw;", "l[n + m] = dotw;"),
+    "hybrid_window_values_are_keys": ("o[k] += p[n + m] * v_win[m * d + k];",
+                                      "o[k] += p[n + m] * k_win[m * d + k];"),
+    "hybrid_window_key_reversed": ("dotw += q[k] * k_win[m * d + k];",
+                                   "dotw += q[k] * k_win[m * d + (d - 1 - k)];"),
     "bytes_drop_factor_two": ("2ull * (uint64_t)T * (uint64_t)H", "(uint64_t)T * (uint64_t)H"),
     "bytes_fold_swapped": ("fold2d ? 1u : (uint64_t)H", "fold2d ? (uint64_t)H : 1u"),
     "bytes_ratio_not_reduced": ("uint64_t g = gcd_u64(per_token_uncompressed, per_token_latent);",
@@ -57,6 +63,9 @@ def _pins():
         (P.test_eckart_young_calibration_residual, {"r": 4}),
         (P.test_absorb_equals_reconstruct_low_rank, {}),
         (P.test_decode_layer_matches_masked_dense_attention, {"fold2d": True}),
+        (P.test_hybrid_full_rank_equals_attention_over_all_tokens, {"n": 20, "w": 5}),
+        (P.test_hybrid_window_order_is_irrelevant_and_empty_is_neutral, {}),
+        (P.test_decode_layer_hybrid_matches_dense_attention_over_both_parts, {"fold2d": False}),
     ]
     for v in P.VARIANTS:
         pins += [

@@ -384,3 +384,86 @@ def test_latent_draw_statistics():
     z = S.draw_latents(200_000, std, 31, "cpu", torch.float32).double().numpy()
     np.testing.assert_allclose(z.std(axis=0), std, rtol=0.01)
     np.testing.assert_allclose(z.mean(axis=0), 0, atol=0.02)
+
+
+# ---------------------------------------------------------------------------
+# Hybrid form ("Hybrid Latent Attention for Looped Language Models", abstract):
+# exact K/V for the window tokens, latents for the older ones, one softmax
+# ---------------------------------------------------------------------------
+@pytest.mark.parametrize("n,w", [(20, 5), (0, 7), (13, 0), (1, 1)])
+def test_hybrid_full_rank_equals_attention_over_all_tokens(n, w):
+    """A full-rank orthonormal codec rebuilds the older tokens exactly, so the hybrid
+    result is textbook attention over all n + w original tokens (torch SDPA)."""
+    T, d = 3, 8
+    rng = np.random.default_rng(31 + n + 7 * w)
+    cK, cV = S.orthonormal_codec(T * d, T, 18), S.orthonormal_codec(T * d, T, 19)
+    xK = rng.standard_normal((n + w, T * d))
+    xV = rng.standard_normal((n + w, T * d)) * 1.5
+    lK = oracle.encode(xK[:n], cK.mu, cK.W_down) if n else np.zeros((0, T * d))
+    lV = oracle.encode(xV[:n], cV.mu, cV.W_down) if n else np.zeros((0, T * d))
+    for t in range(T):
+        q = rng.standard_normal(d)
+        sl = slice(t * d, (t + 1) * d)
+        o, lse = oracle.attend_hybrid(lK, lV, cK.W_up[t], cK.mu_t()[t], cV.W_up[t], cV.mu_t()[t],
+                                      xK[n:, sl], xV[n:, sl], q, 0.7)
+        o_ref, lse_ref = sdpa(q, xK[:, sl], xV[:, sl], 0.7)
+        np.testing.assert_allclose(o, o_ref, atol=1e-10, rtol=0)
+        assert lse == pytest.approx(lse_ref, abs=1e-10)
+
+
+def test_hybrid_window_order_is_irrelevant_and_empty_is_neutral():
+    """The window is a set: its row order does not matter; and with no window the hybrid
+    form is the latent-only decode attention (absorbed form, written separately)."""
+    T, d, rk, rv, n, w = 4, 16, 3, 6, 17, 9
+    rng = np.random.default_rng(40)
+    (WK, muK), (WV, muV) = _codec_pair(T, d, rk, rv, 41)
+    cK, cV = rng.standard_normal((n, rk)), rng.standard_normal((n, rv))
+    kw, vw = rng.standard_normal((w, d)), rng.standard_normal((w, d))
+    perm = rng.permutation(w)
+    for t in range(T):
+        q = rng.standard_normal(d)
+        a = oracle.attend_hybrid(cK, cV, WK[t], muK[t], WV[t], muV[t], kw, vw, q, 0.5)
+        b = oracle.attend_hybrid(cK, cV, WK[t], muK[t], WV[t], muV[t], kw[perm], vw[perm], q, 0.5)
+        np.testing.assert_allclose(a[0], b[0], atol=1e-12, rtol=0)
+        assert a[1] == pytest.approx(b[1], abs=1e-12)
+        e = oracle.attend_hybrid(cK, cV, WK[t], muK[t], WV[t], muV[t], kw[:0], vw[:0], q, 0.5)
+        ref = oracle.attend("absorb", cK, cV, WK[t], muK[t], WV[t], muV[t], q, 0.5)
+        np.testing.assert_allclose(e[0], ref[0], atol=1e-12, rtol=0)
+        assert e[1] == pytest.approx(ref[1], abs=1e-12)
+
+
+@pytest.mark.parametrize("fold2d", [False, True])
+def test_decode_layer_hybrid_matches_dense_attention_over_both_parts(fold2d):
+    """Ragged batch with ragged windows (one sequence with no latents, one with no
+    window, one with neither): each unit against SDPA over [rebuilt older tokens; window]."""
+    T, H, d, rk, rv = 3, 2, 8, 4, 6
+    lens = np.array([5, 0, 4, 0], dtype=np.int32)
+    wins = np.array([3, 2, 0, 0], dtype=np.int32)
+    starts, c_K, c_V, WK, mK, WV, mV = _ragged_layer(T, H, d, lens, rk, rv, fold2d, 24)
+    B, Tq, t0, s, wmax = len(lens), 2, 1, 0.6, 4
+    rng = np.random.default_rng(25)
+    q = rng.standard_normal((B, Tq, H, d))
+    win_k = rng.standard_normal((B, H, T, wmax, d))
+    win_v = rng.standard_normal((B, H, T, wmax, d))
+    o, lse = oracle.decode_layer("absorb", q, c_K, c_V, starts, lens, WK, mK, WV, mV, t0, s,
+                                 fold2d=fold2d, threads=2, window=(win_k, win_v, wins))
+    for b in range(B):
+        sl = slice(int(starts[b]), int(starts[b] + lens[b]))
+        for tq in range(Tq):
+            t = t0 + tq
+            for h in range(H):
+                if fold2d:
+                    cols = slice(h * d, (h + 1) * d)
+                    Kh = c_K[0, sl] @ WK[t][:, cols] + mK[t][cols]
+                    Vh = c_V[0, sl] @ WV[t][:, cols] + mV[t][cols]
+                else:
+                    Kh = c_K[h, sl] @ WK[h, t] + mK[h, t]
+                    Vh = c_V[h, sl] @ WV[h, t] + mV[h, t]
+                Kh = np.concatenate([Kh, win_k[b, h, t, :wins[b]]])
+                Vh = np.concatenate([Vh, win_v[b, h, t, :wins[b]]])
+                if Kh.shape[0] == 0:
+                    assert np.all(o[b, tq, h] == 0) and lse[b, tq, h] == -np.inf
+                    continue
+                o_ref, lse_ref = sdpa(q[b, tq, h], Kh, Vh, s)
+                np.testing.assert_allclose(o[b, tq, h], o_ref, atol=1e-11)
+                assert lse[b, tq, h] == pytest.approx(lse_ref, abs=1e-11)
