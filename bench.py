@@ -62,6 +62,9 @@ def parse():
                     help="step: decode step (headline); encode: prefill encode of one layer")
     ap.add_argument("--encode-seqs", type=int, default=0,
                     help="--phase encode: sequences of len_hi tokens to encode (default: B)")
+    ap.add_argument("--window", type=int, default=0,
+                    help="hybrid form: W exact window rows per sequence (all in use) besides the "
+                         "latents; 0 = latents only")
     ap.add_argument("--model-order", action="store_true",
                     help="one decode call per loop (Tq = 1, t = 0..T-1) instead of all loops fused")
     return ap.parse_args()
@@ -356,6 +359,14 @@ def main():
     R = max(1, args.replicas)
     reps = [(p["k"], p["v"])] + [(p["k"].clone(), p["v"].clone()) for _ in range(R - 1)]
     caches = [lla.make_cache(k, v, p["slots"]) for k, v in reps]
+    # hybrid form: every sequence holds a full window of W exact rows (steady state)
+    Wn = max(0, args.window)
+    windows = []
+    if Wn:
+        win = S.window_inputs(w, 0, B, Wn, dev, win_lens=np.full(B, Wn, dtype=np.int32))
+        wreps = [(win["win_k"], win["win_v"])] + [(win["win_k"].clone(), win["win_v"].clone())
+                                                  for _ in range(R - 1)]
+        windows = [lla.make_window(k, v, win["win_len"], Wn, B) for k, v in wreps]
     x_k = S.draw_encode_tokens(w, 0, "k", B, dev, seed_tag="new")
     x_v = S.draw_encode_tokens(w, 0, "v", B, dev, seed_tag="new")
     new_slot = (p["seq_start"] + p["ctx_lens"].to(torch.int64)).contiguous()
@@ -370,13 +381,20 @@ def main():
     outs = [torch.empty(B, n, H, w.d, dtype=torch.float32, device=dev) for _, n in calls]
     lses = [torch.empty(B, n, H, dtype=torch.float32, device=dev) for _, n in calls]
     q, out, lse = q_full, outs[0], lses[0]
-    ws_bytes = lla.decode_workspace_bytes(dims, B, Tq_call, max_ctx, variant, args.num_splits)
+    ws_fn = lla.decode_hybrid_workspace_bytes if Wn else lla.decode_workspace_bytes
+    ws_bytes = ws_fn(dims, B, Tq_call, max_ctx, variant, args.num_splits)
     ws = torch.zeros(ws_bytes, dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream(dev)
     splits = lla.decode_num_splits(dims, B, Tq_call, max_ctx, variant, args.num_splits)
 
     def decode(i, q_in=None, out_buf=None, lse_buf=None):
         for c, (t0, n) in enumerate(calls):
+            if Wn:
+                lla.decode_attn_hybrid(dims, 0, t0, n, (q_in or qs)[c], caches[i % R], p["seq_start"],
+                                       p["ctx_lens"], B, max_ctx, codec, windows[i % R], 1.0,
+                                       (out_buf or outs)[c], (lse_buf or lses)[c], ws, ws_bytes,
+                                       variant=variant, num_splits=args.num_splits, stream=stream)
+                continue
             lla.decode_attn(dims, 0, t0, n, (q_in or qs)[c], caches[i % R], p["seq_start"], p["ctx_lens"], B,
                             max_ctx, codec, 1.0, (out_buf or outs)[c], (lse_buf or lses)[c], ws, ws_bytes,
                             variant=variant, num_splits=args.num_splits, stream=stream)
@@ -386,7 +404,7 @@ def main():
 
     # per decode call: prologue + decode + combine (reconstruct: one decode pass per loop
     # query + combine); the encode of K and V is one launch
-    per_call = 3 if args.variant == "absorb" else Tq_call + 1
+    per_call = (3 if args.variant == "absorb" else Tq_call + 1) + (1 if Wn else 0)  # + window pass
     launches_per_step = per_call * len(calls) + 1
     # ---- warm-up, then the device-timed region ------------------------------------------------
     sampler = ClockSampler(local).start()
@@ -422,6 +440,9 @@ def main():
 
     # latents read per step: one pass over the layer's latents per decode call
     step_bytes = len(calls) * S_tot * w.heads_stored * (w.r_k + w.r_v) * w.elem_bytes
+    # hybrid form: each loop query also reads its own loop's exact window keys and values once
+    win_bytes = B * H * Tq * Wn * w.d * 2 * w.elem_bytes
+    step_bytes += win_bytes
     ms_step = ms_total / args.steps
     value = world * step_bytes / (ms_step * 1e-3) / 1e9
     reads = world * S_tot * Tq / (ms_step * 1e-3)       # (token, layer, loop) reads per second
@@ -510,7 +531,7 @@ def main():
         return
 
     cpu = None
-    if world == 1 and not args.no_cpu_baseline:
+    if world == 1 and not args.no_cpu_baseline and not Wn:
         rate, info = oracle_sample_rate(p, w, Tq, args.cpu_seconds, units_per_round=max(1, B * H // 8))
         cpu = {"value": rate, "unit": "GB/s", "cores": info["cores"], "kind": "oracle",
                "sample": f"{info['rounds']} rounds of {info['units']} (sequence, head) units x "
@@ -523,12 +544,14 @@ def main():
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": "f32", "storage_dtype": w.dtype, "data": "synthetic",
-        "config": {"workload": w.name, "T": w.T, "L_per_step": 1, "H": H, "d": w.d,
+        "config": {"workload": w.name + (f"+window{Wn}" if Wn else ""), "T": w.T, "L_per_step": 1,
+                   "H": H, "d": w.d, "window_rows": Wn, "window_bytes_per_step": win_bytes,
                    "r_k": w.r_k, "r_v": w.r_v, "rho": "64/3", "B": B,
                    "ctx_len": [w.len_lo, w.len_hi], "tokens": S_tot, "Tq": Tq_call, "decode_calls_per_step": len(calls),
                    "variant": args.variant, "seg_max": splits,
                    "step": (f"{len(calls)} x decode_attn(Tq = 1, one loop each, model order)"
                             if args.model_order else f"decode_attn(all {w.T} loop queries fused)")
+                           + (f" with {Wn} exact window rows per sequence (decode_attn_hybrid)" if Wn else "")
                            + " + encode(B new tokens)",
                    "l2": f"inputs larger than L2 ({step_bytes / 1e6:.0f} MB of latents per step) "
                          f"and {R} rotating cache replicas",

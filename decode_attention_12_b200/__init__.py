@@ -9,6 +9,7 @@ library is missing.
 
 Names follow the C ABI: ``cache_bytes``, ``slot_layout``, ``codec_bias``,
 ``encode``, ``decode_attn``, ``decode_workspace_bytes``, ``decode_num_splits``,
+``decode_attn_static``, ``decode_attn_hybrid``, ``decode_hybrid_workspace_bytes``,
 ``status_fetch``, ``status_string``.
 """
 from __future__ import annotations
@@ -40,7 +41,8 @@ ABSORB, RECONSTRUCT = 0, 1
 
 EXPORTED = ("lla_cache_bytes", "lla_slot_layout", "lla_codec_bias", "lla_encode",
             "lla_decode_attn", "lla_decode_workspace_bytes", "lla_decode_num_splits",
-            "lla_decode_attn_static", "lla_status_fetch", "lla_status_string")
+            "lla_decode_attn_static", "lla_decode_attn_hybrid", "lla_decode_hybrid_workspace_bytes",
+            "lla_status_fetch", "lla_status_string")
 STATIC_SCRATCH_BYTES = 8 << 20
 
 
@@ -58,6 +60,11 @@ class Cache(ctypes.Structure):
     _fields_ = [("k", ctypes.c_void_p), ("v", ctypes.c_void_p), ("slots", ctypes.c_int64)]
 
 
+class Window(ctypes.Structure):
+    _fields_ = [("k", ctypes.c_void_p), ("v", ctypes.c_void_p), ("len", ctypes.c_void_p),
+                ("w_max", ctypes.c_int32), ("seqs", ctypes.c_int32)]
+
+
 _i32, _i64, _u64p = ctypes.c_int32, ctypes.c_int64, ctypes.POINTER(ctypes.c_uint64)
 _vp, _sz = ctypes.c_void_p, ctypes.c_size_t
 _P = ctypes.POINTER
@@ -69,6 +76,11 @@ _lib.lla_decode_attn.argtypes = [_P(Dims), _i32, _i32, _i32, _vp, _P(Cache), _vp
                                  _P(Codec), ctypes.c_float, _i32, _i32, _vp, _vp, _vp, _sz, _vp]
 _lib.lla_decode_attn_static.argtypes = [_P(Dims), _i32, _i32, _i32, _vp, _P(Cache), _vp, _vp, _i32,
                                         _i32, _P(Codec), ctypes.c_float, _i32, _i32, _vp, _vp, _vp]
+_lib.lla_decode_attn_hybrid.argtypes = [_P(Dims), _i32, _i32, _i32, _vp, _P(Cache), _vp, _vp, _i32,
+                                        _i32, _P(Codec), _P(Window), ctypes.c_float, _i32, _i32, _vp,
+                                        _vp, _vp, _sz, _vp]
+_lib.lla_decode_hybrid_workspace_bytes.argtypes = [_P(Dims), _i32, _i32, _i32, _i32, _i32]
+_lib.lla_decode_hybrid_workspace_bytes.restype = _sz
 _lib.lla_decode_workspace_bytes.argtypes = [_P(Dims), _i32, _i32, _i32, _i32, _i32]
 _lib.lla_decode_workspace_bytes.restype = _sz
 _lib.lla_decode_num_splits.argtypes = [_P(Dims), _i32, _i32, _i32, _i32, _i32]
@@ -76,7 +88,8 @@ _lib.lla_status_fetch.argtypes = [_vp, _vp, _P(_i32)]
 _lib.lla_status_string.argtypes = [ctypes.c_int]
 _lib.lla_status_string.restype = ctypes.c_char_p
 for _n in ("lla_cache_bytes", "lla_slot_layout", "lla_codec_bias", "lla_encode", "lla_decode_attn",
-           "lla_decode_attn_static", "lla_decode_num_splits", "lla_status_fetch"):
+           "lla_decode_attn_static", "lla_decode_attn_hybrid", "lla_decode_num_splits",
+           "lla_status_fetch"):
     getattr(_lib, _n).restype = ctypes.c_int
 
 
@@ -122,6 +135,11 @@ def make_codec(W_down_k=None, W_down_v=None, bias_k=None, bias_v=None, W_up_k=No
 
 def make_cache(k, v, slots: int) -> Cache:
     return Cache(_ptr(k), _ptr(v), int(slots))
+
+
+def make_window(k, v, win_len, w_max: int, seqs: int) -> Window:
+    """Exact window planes k, v [L][seqs][H][T][w_max][d] and rows in use win_len [seqs]."""
+    return Window(_ptr(k), _ptr(v), _ptr(win_len), int(w_max), int(seqs))
 
 
 # ---- a7 -------------------------------------------------------------------------------
@@ -184,6 +202,29 @@ def decode_attn(dims: Dims, layer: int, t0: int, Tq: int, q, cache: Cache, seq_s
                                 float(softmax_scale), variant, num_splits, _ptr(out), _ptr(lse),
                                 _ptr(workspace), int(ws_bytes), _stream(stream)),
            "lla_decode_attn")
+
+
+def decode_hybrid_workspace_bytes(dims: Dims, B: int, Tq: int, max_ctx: int, variant: int = ABSORB,
+                                  num_splits: int = 0) -> int:
+    n = _lib.lla_decode_hybrid_workspace_bytes(ctypes.byref(dims), B, Tq, max_ctx, variant, num_splits)
+    if n == 0:
+        raise LLAError(LLA_ERR_INVALID, "lla_decode_hybrid_workspace_bytes")
+    return int(n)
+
+
+def decode_attn_hybrid(dims: Dims, layer: int, t0: int, Tq: int, q, cache: Cache, seq_start, ctx_lens,
+                       B: int, max_ctx: int, codec: Codec, window: Window, softmax_scale: float, out,
+                       lse=None, workspace=None, ws_bytes: Optional[int] = None, variant: int = ABSORB,
+                       num_splits: int = 0, stream=None) -> None:
+    """Hybrid latent attention: one softmax over the latent tokens and the exact window rows."""
+    if ws_bytes is None:
+        ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
+    _check(_lib.lla_decode_attn_hybrid(ctypes.byref(dims), layer, t0, Tq, _ptr(q), ctypes.byref(cache),
+                                       _ptr(seq_start), _ptr(ctx_lens), B, max_ctx, ctypes.byref(codec),
+                                       ctypes.byref(window), float(softmax_scale), variant, num_splits,
+                                       _ptr(out), _ptr(lse), _ptr(workspace), int(ws_bytes),
+                                       _stream(stream)),
+           "lla_decode_attn_hybrid")
 
 
 def decode_attn_static(dims: Dims, layer: int, t0: int, Tq: int, q, cache: Cache, seq_start,

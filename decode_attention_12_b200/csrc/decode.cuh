@@ -30,6 +30,13 @@ struct DecodeArgs {
     int32_t *status;          // sticky device status word
     void *out;                // O [B][Tq_all][H][d] (O = out_dtype)
     float *lse;               // [B][Tq_all][H] or null
+    // hybrid form: exact loop keys / values of each sequence's window tokens
+    const void *win_k;        // T [B][H][T][w_max][d] (layer already selected) or null
+    const void *win_v;        // T [B][H][T][w_max][d]
+    const int32_t *win_len;   // [B] window rows in use
+    int32_t w_max;
+    float *win_part;          // [B*H][Tq_all][d + 4] window output and lse (log2 units);
+                              // null: no window, the combine writes the latent result alone
 };
 
 constexpr float kLog2e = 1.4426950408889634f;
@@ -55,5 +62,9 @@ bool decode_mma2d_supported(int dtype, int r_k, int r_v, int fold, int H);
 int decode_mma2d_loops_per_pass(int H);
 cudaError_t launch_decode_absorb_2d(const DecodeArgs &a, cudaStream_t stream);
 cudaError_t launch_decode_reconstruct(const DecodeArgs &a, cudaStream_t stream);
+// Hybrid form: attention of every loop query over its exact window rows, written to
+// a.win_part for the combine to merge (launched between the decode and the combine).
+bool decode_window_supported(int dtype, int d);
+cudaError_t launch_decode_window(const DecodeArgs &a, int dtype, cudaStream_t stream);
 
 } // namespace lla

@@ -545,9 +545,10 @@ template <int RG> struct RecBatch {
 
 // REC: records carry d-wide outputs of the reconstruct form (mu and the q.mu_t^K score term
 // already included), so the output is the merged record itself.  RG = record width / 128,
-// rounded up.
-template <typename T, typename O, bool REC, int RG>
-__global__ void __launch_bounds__(kCombineThreads, RG == 1 ? 4 : 2) decode_combine_kernel(const DecodeArgs a)
+// rounded up.  WIN: hybrid form, merge the window part (a.win_part) as well.
+template <typename T, typename O, bool REC, int RG, bool WIN>
+__global__ void __launch_bounds__(kCombineThreads, RG == 1 && !WIN ? 4 : RG == 1 ? 3 : 2)
+    decode_combine_kernel(const DecodeArgs a)
 {
     extern __shared__ __align__(16) float csm[];
     const int h = blockIdx.x, tl = blockIdx.y, b0 = blockIdx.z * kBatchSeqs;
@@ -589,6 +590,18 @@ __global__ void __launch_bounds__(kCombineThreads, RG == 1 ? 4 : 2) decode_combi
 
     grid_dependency_wait(); // records and counts come from the preceding decode grid
 
+    // hybrid form: the window part of this (unit, query), complete before this grid's wait
+    // returns; its first column group is fetched here, wider rows group by group below
+    constexpr bool win = WIN;
+    const float *wrec = win ? a.win_part + (u * a.Tq_all + t) * part_stride(d) : nullptr;
+    float wl = -INFINITY;
+    float4 wo0 = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (win && active) {
+        wl = wrec[d];
+        if (4 * lane < d)
+            wo0 = Vec4<float>::load(wrec + 4 * lane);
+    }
+
     float M = -INFINITY, L = 0.f;
     float4 acc[RG];
 #pragma unroll
@@ -610,9 +623,23 @@ __global__ void __launch_bounds__(kCombineThreads, RG == 1 ? 4 : 2) decode_combi
 #pragma unroll
     for (int g = 0; g < RG; ++g)
         acc[g] = f4_scale(invL, acc[g]); // o_lat (or the output itself for REC)
+    float lse = L > 0.f ? kLn2 * (M + log2f(L)) + (REC ? 0.f : a.scale * qm) : -INFINITY;
+    // hybrid form: out = fa * out_lat + fw * out_win, weights from the two log-sum-exps
+    float fa = 1.f, fw = 0.f;
+    if (win) {
+        const float l2 = L > 0.f ? M + log2f(L) + (REC ? 0.f : a.scale * qm * kLog2e) : -INFINITY;
+        const float mm = fmaxf(l2, wl);
+        fa = 0.f;
+        lse = -INFINITY;
+        if (mm != -INFINITY) {
+            const float ea = exp2f(l2 - mm), ew = exp2f(wl - mm), sum = ea + ew;
+            fa = ea / sum;
+            fw = ew / sum;
+            lse = kLn2 * (mm + log2f(sum));
+        }
+    }
     if (active && lane == 0 && a.lse != nullptr)
-        a.lse[((int64_t)b * a.Tq_all + t) * a.H + h] =
-            L > 0.f ? kLn2 * (M + log2f(L)) + (REC ? 0.f : a.scale * qm) : -INFINITY;
+        a.lse[((int64_t)b * a.Tq_all + t) * a.H + h] = lse;
 
     O *orow = static_cast<O *>(a.out) + (((int64_t)b * a.Tq_all + t) * a.H + h) * d;
     if (REC) {
@@ -620,8 +647,12 @@ __global__ void __launch_bounds__(kCombineThreads, RG == 1 ? 4 : 2) decode_combi
 #pragma unroll
             for (int g = 0; g < RG; ++g) {
                 const int c = 4 * lane + 128 * g;
-                if (c < d)
-                    Vec4<O>::store(orow + c, acc[g]);
+                if (c < d) {
+                    float4 o = acc[g];
+                    if (win)
+                        o = f4_fma(fw, g == 0 ? wo0 : Vec4<float>::load(wrec + c), f4_scale(fa, o));
+                    Vec4<O>::store(orow + c, o);
+                }
             }
         }
         return;
@@ -653,6 +684,8 @@ __global__ void __launch_bounds__(kCombineThreads, RG == 1 ? 4 : 2) decode_combi
                 }
             }
         }
+        if (win && mine)
+            o = f4_fma(fw, gi == 0 ? wo0 : Vec4<float>::load(wrec + c), f4_scale(fa, o));
         if (mine)
             Vec4<O>::store(orow + c, o);
     }
@@ -708,7 +741,9 @@ cudaError_t launch_absorb_prologue(const DecodeArgs &a, int dtype, cudaStream_t 
 template <typename T, typename O, int RG>
 static cudaError_t launch_combine_t(const DecodeArgs &a, size_t smem, cudaStream_t stream)
 {
-    auto k = a.recon ? decode_combine_kernel<T, O, true, RG> : decode_combine_kernel<T, O, false, RG>;
+    const bool win = a.win_part != nullptr;
+    auto k = a.recon ? (win ? decode_combine_kernel<T, O, true, RG, true> : decode_combine_kernel<T, O, true, RG, false>)
+                     : (win ? decode_combine_kernel<T, O, false, RG, true> : decode_combine_kernel<T, O, false, RG, false>);
     cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess)
         return e;

@@ -61,12 +61,13 @@ int sm_count()
 // workspace regions (header | counts | q_tilde | partial records).
 struct Plan {
     int32_t seg_max, chunk_min;
-    size_t off_counts, off_qt, off_part, bytes;
+    size_t off_counts, off_qt, off_part, off_win, bytes;
 };
 
 size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
 
-Plan make_plan(const lla_dims *d, int32_t B, int32_t Tq, int32_t max_ctx, int32_t num_splits, int32_t variant)
+Plan make_plan(const lla_dims *d, int32_t B, int32_t Tq, int32_t max_ctx, int32_t num_splits, int32_t variant,
+               bool window = false)
 {
     Plan p;
     const int64_t units = (int64_t)B * d->H;
@@ -89,6 +90,11 @@ Plan make_plan(const lla_dims *d, int32_t B, int32_t Tq, int32_t max_ctx, int32_
     // reconstruct-form records carry d-wide outputs, absorbed-form records r_v-wide latents
     const int rec_w = variant == LLA_RECONSTRUCT ? d->d_head : d->r_v;
     p.bytes = p.off_part + (size_t)units * Tq * p.seg_max * part_stride(rec_w) * sizeof(float);
+    p.off_win = 0;
+    if (window) { // hybrid form: one d-wide window record per (unit, loop query)
+        p.off_win = align256(p.bytes);
+        p.bytes = p.off_win + (size_t)units * Tq * part_stride(d->d_head) * sizeof(float);
+    }
     return p;
 }
 
@@ -243,11 +249,16 @@ size_t lla_decode_workspace_bytes(const lla_dims *dims, int32_t B, int32_t Tq, i
     return make_plan(dims, B, Tq, max_ctx, num_splits, variant).bytes;
 }
 
-int lla_decode_attn(const lla_dims *dims, int32_t layer, int32_t t0, int32_t Tq, const void *q,
-                    const lla_cache *cache, const int64_t *seq_start, const int32_t *ctx_lens, int32_t B,
-                    int32_t max_ctx, const lla_codec *codec, float softmax_scale, int32_t variant,
-                    int32_t num_splits, void *out, float *lse, void *workspace, size_t ws_bytes,
-                    lla_stream_t stream)
+} // extern "C"
+
+namespace {
+
+// Body of lla_decode_attn and lla_decode_attn_hybrid (window == NULL: latents only).
+int decode_call(const lla_dims *dims, int32_t layer, int32_t t0, int32_t Tq, const void *q,
+                const lla_cache *cache, const int64_t *seq_start, const int32_t *ctx_lens, int32_t B,
+                int32_t max_ctx, const lla_codec *codec, const lla_window *window, float softmax_scale,
+                int32_t variant, int32_t num_splits, void *out, float *lse, void *workspace,
+                size_t ws_bytes, lla_stream_t stream)
 {
     int rc = check_dims(dims);
     if (rc != LLA_OK)
@@ -268,7 +279,16 @@ int lla_decode_attn(const lla_dims *dims, int32_t layer, int32_t t0, int32_t Tq,
         return LLA_ERR_MISALIGNED;
     if ((dims->d_head * elem_bytes(dims->dtype)) % 16 != 0)
         return LLA_ERR_UNSUPPORTED; // query / output rows are moved in 16-byte pieces
-    const Plan plan = make_plan(dims, B, Tq, max_ctx, num_splits, variant);
+    if (window != nullptr) {
+        if (window->w_max < 0 || window->seqs < B || window->len == nullptr ||
+            (window->w_max > 0 && (window->k == nullptr || window->v == nullptr)))
+            return LLA_ERR_INVALID;
+        if (!aligned16(window->len) || !aligned16(window->k) || !aligned16(window->v))
+            return LLA_ERR_MISALIGNED;
+        if (!decode_window_supported(dims->dtype, dims->d_head))
+            return LLA_ERR_UNSUPPORTED;
+    }
+    const Plan plan = make_plan(dims, B, Tq, max_ctx, num_splits, variant, window != nullptr);
     if (workspace == nullptr || ws_bytes < plan.bytes)
         return LLA_ERR_WORKSPACE;
     if (!aligned16(workspace))
@@ -309,11 +329,28 @@ int lla_decode_attn(const lla_dims *dims, int32_t layer, int32_t t0, int32_t Tq,
     a.part = reinterpret_cast<float *>(ws + plan.off_part);
     a.out = out;
     a.lse = lse;
+    a.win_k = a.win_v = nullptr;
+    a.win_len = nullptr;
+    a.w_max = 0;
+    a.win_part = nullptr;
+    if (window != nullptr) {
+        // window planes [L][seqs][H][T][w_max][d]: select the layer
+        const int64_t plane = (int64_t)window->seqs * dims->H * dims->T * window->w_max * dims->d_head * e;
+        a.win_k = window->w_max > 0 ? static_cast<const uint8_t *>(window->k) + layer * plane : nullptr;
+        a.win_v = window->w_max > 0 ? static_cast<const uint8_t *>(window->v) + layer * plane : nullptr;
+        a.win_len = window->len;
+        a.w_max = window->w_max;
+        a.win_part = reinterpret_cast<float *>(ws + plan.off_win);
+    }
 
     a.Tq_all = Tq;
     a.tq_off = 0;
     cudaStream_t s = (cudaStream_t)stream;
     cudaError_t err = cudaSuccess;
+    // hybrid form: the window pass runs after the decode grid, before the combine
+    auto window_pass = [&](const DecodeArgs &ac) -> cudaError_t {
+        return window != nullptr ? launch_decode_window(ac, dims->dtype, s) : cudaSuccess;
+    };
     if (variant == LLA_RECONSTRUCT) {
         // one pass over the latents per loop query, then one merge of all records
         for (int32_t c = 0; c < Tq && err == cudaSuccess; ++c) {
@@ -322,6 +359,8 @@ int lla_decode_attn(const lla_dims *dims, int32_t layer, int32_t t0, int32_t Tq,
             ac.Tq = 1;
             err = launch_decode_reconstruct(ac, s);
         }
+        if (err == cudaSuccess)
+            err = window_pass(a);
         if (err == cudaSuccess)
             err = launch_decode_combine(a, dims->dtype, dims->out_dtype, s);
         return err == cudaSuccess ? LLA_OK : LLA_ERR_CUDA;
@@ -338,6 +377,8 @@ int lla_decode_attn(const lla_dims *dims, int32_t layer, int32_t t0, int32_t Tq,
             if (err == cudaSuccess)
                 err = launch_decode_absorb_2d(ac, s);
             if (err == cudaSuccess)
+                err = window_pass(ac);
+            if (err == cudaSuccess)
                 err = launch_decode_combine(ac, dims->dtype, dims->out_dtype, s);
         }
         return err == cudaSuccess ? LLA_OK : LLA_ERR_CUDA;
@@ -351,6 +392,8 @@ int lla_decode_attn(const lla_dims *dims, int32_t layer, int32_t t0, int32_t Tq,
             err = launch_absorb_prologue(ac, dims->dtype, s);
             if (err == cudaSuccess)
                 err = launch_decode_absorb_mma(ac, 0, s);
+            if (err == cudaSuccess)
+                err = window_pass(ac);
             if (err == cudaSuccess)
                 err = launch_decode_combine(ac, dims->dtype, dims->out_dtype, s);
         }
@@ -368,9 +411,45 @@ int lla_decode_attn(const lla_dims *dims, int32_t layer, int32_t t0, int32_t Tq,
         if (!supported)
             return LLA_ERR_UNSUPPORTED;
         if (err == cudaSuccess)
+            err = window_pass(ac);
+        if (err == cudaSuccess)
             err = launch_decode_combine(ac, dims->dtype, dims->out_dtype, s);
     }
     return err == cudaSuccess ? LLA_OK : LLA_ERR_CUDA;
+}
+
+} // namespace
+
+extern "C" {
+
+int lla_decode_attn(const lla_dims *dims, int32_t layer, int32_t t0, int32_t Tq, const void *q,
+                    const lla_cache *cache, const int64_t *seq_start, const int32_t *ctx_lens, int32_t B,
+                    int32_t max_ctx, const lla_codec *codec, float softmax_scale, int32_t variant,
+                    int32_t num_splits, void *out, float *lse, void *workspace, size_t ws_bytes,
+                    lla_stream_t stream)
+{
+    return decode_call(dims, layer, t0, Tq, q, cache, seq_start, ctx_lens, B, max_ctx, codec, nullptr,
+                       softmax_scale, variant, num_splits, out, lse, workspace, ws_bytes, stream);
+}
+
+int lla_decode_attn_hybrid(const lla_dims *dims, int32_t layer, int32_t t0, int32_t Tq, const void *q,
+                           const lla_cache *cache, const int64_t *seq_start, const int32_t *ctx_lens,
+                           int32_t B, int32_t max_ctx, const lla_codec *codec, const lla_window *window,
+                           float softmax_scale, int32_t variant, int32_t num_splits, void *out, float *lse,
+                           void *workspace, size_t ws_bytes, lla_stream_t stream)
+{
+    if (window == nullptr)
+        return LLA_ERR_INVALID;
+    return decode_call(dims, layer, t0, Tq, q, cache, seq_start, ctx_lens, B, max_ctx, codec, window,
+                       softmax_scale, variant, num_splits, out, lse, workspace, ws_bytes, stream);
+}
+
+size_t lla_decode_hybrid_workspace_bytes(const lla_dims *dims, int32_t B, int32_t Tq, int32_t max_ctx,
+                                         int32_t variant, int32_t num_splits)
+{
+    if (lla_decode_num_splits(dims, B, Tq, max_ctx, variant, num_splits) < 1)
+        return 0;
+    return make_plan(dims, B, Tq, max_ctx, num_splits, variant, true).bytes;
 }
 
 int lla_status_fetch(void *workspace, lla_stream_t stream, int32_t *status_host)

@@ -173,6 +173,46 @@ size_t lla_decode_workspace_bytes(const lla_dims *dims, int32_t B, int32_t Tq,
 int lla_decode_num_splits(const lla_dims *dims, int32_t B, int32_t Tq, int32_t max_ctx,
                           int32_t variant, int32_t num_splits);
 
+/* ---- NEXT-2: hybrid latent attention (exact window + latents) ---------------------------
+ * "Hybrid Latent Attention for Looped Language Models", abstract: the keys and values
+ * of each sequence's most recent tokens (a sliding window) are kept exact, one K_t, V_t
+ * pair per loop t; older tokens are cached only as latents, which every loop's query
+ * reads directly.  Loop query t of sequence b and head h attends, with ONE softmax, over
+ * the ctx_lens[b] latent tokens (read exactly as lla_decode_attn reads them) and the
+ * len[b] window tokens (plain dot products with their exact loop-t keys):
+ *   l = [ latent logits of lla_decode_attn ; softmax_scale * q . k_win[m] ]
+ *   out = sum softmax(l) * [ v_hat ; v_win[m] ],   lse = log sum exp(l).
+ * The window is a set: its row order does not matter, so a ring buffer may be used
+ * as it is.  Which tokens the caller keeps in the window (the page fixes W recent ones,
+ * the current token among them) and when an aged-out token is encoded into the latent
+ * cache (lla_encode) is the caller's; the two parts must not hold the same token.
+ * Computation: the latent part runs as in lla_decode_attn; a streaming kernel computes
+ * each query's window part (out_win, lse_win), and the combine step merges the two by
+ * their log-sum-exps.  An empty context (ctx_lens[b] = 0) with a non-empty window gives
+ * the window attention alone; both empty give out = 0, lse = -inf.                      */
+typedef struct {
+    const void *k;       /* T [L][seqs][H][T][w_max][d]  exact loop keys of window rows   */
+    const void *v;       /* T [L][seqs][H][T][w_max][d]  exact loop values                */
+    const int32_t *len;  /* int32 [seqs] (device) rows in use for sequence b, clamped to
+                            [0, w_max]; rows len[b] .. w_max-1 are never read              */
+    int32_t w_max;       /* row capacity per (layer, sequence, head, loop); 0 = no window  */
+    int32_t seqs;        /* sequence capacity of one layer plane (>= B of the call)        */
+} lla_window;
+/* Same arguments, errors and workspace rules as lla_decode_attn, plus `window` (required,
+ * host struct of device pointers; sequence b of the call uses window row-block b).  The
+ * workspace must hold lla_decode_hybrid_workspace_bytes(...) bytes.  Additional errors:
+ * LLA_ERR_INVALID (window NULL, w_max < 0, seqs < B, null arrays),
+ * LLA_ERR_UNSUPPORTED (d_head * sizeof(T) > 512 bytes).                                   */
+int lla_decode_attn_hybrid(const lla_dims *dims, int32_t layer, int32_t t0, int32_t Tq,
+                           const void *q, const lla_cache *cache, const int64_t *seq_start,
+                           const int32_t *ctx_lens, int32_t B, int32_t max_ctx,
+                           const lla_codec *codec, const lla_window *window,
+                           float softmax_scale, int32_t variant, int32_t num_splits,
+                           void *out, float *lse, void *workspace, size_t ws_bytes,
+                           lla_stream_t stream);
+size_t lla_decode_hybrid_workspace_bytes(const lla_dims *dims, int32_t B, int32_t Tq,
+                                         int32_t max_ctx, int32_t variant, int32_t num_splits);
+
 /* ---- decode attention with library-owned scratch ----------------------------------------
  * No counterpart in the paper: a deployment aid.  Some callers cannot allocate device
  * memory -- for example a plugin whose host framework owns the whole device memory pool

@@ -28,6 +28,11 @@ whose weights are not available):
   values).  Queries q ~ N(0, 1) / sqrt(d).  Context lengths uniform inclusive.
 * Encode inputs: trajectory tokens laid out [n_tok][T][H][d] (loop-major, as a
   looped model produces them loop by loop).
+* Hybrid-window inputs ("Hybrid Latent Attention for Looped Language Models",
+  abstract: exact keys and values of the most recent tokens): fresh trajectory
+  tokens of the same model, drawn as encode inputs and laid out per window row,
+  [B][H][T][w_max][d] per layer and axis; rows in use per sequence uniform in
+  [0, w_max] unless given.
 """
 from __future__ import annotations
 
@@ -367,4 +372,39 @@ def decode_inputs(w: Workload, layers, device, Tq: Optional[int] = None, lens=No
             out[name][layer].copy_(src)
         draw_layer_cache(w, layer, codecs, slots, device, out_k=out["k"][layer], out_v=out["v"][layer])
     out["q"] = draw_queries(w.B, Tq, w.H, w.d, seed_of(w.name, q_tag, Tq), device, dt)
+    return out
+
+
+# ---------------------------------------------------------------------------
+# Hybrid form: exact window rows of every sequence
+# ---------------------------------------------------------------------------
+def window_lengths(B: int, w_max: int, seed_tag="win_len") -> np.ndarray:
+    rng = np.random.default_rng(seed_of("window", B, w_max, seed_tag))
+    return rng.integers(0, w_max + 1, size=B).astype(np.int32)
+
+
+def window_inputs(w: Workload, layers, B: int, w_max: int, device, win_lens=None,
+                  seed_tag="window") -> dict:
+    """Exact window keys / values in the library layout [L][B][H][T][w_max][d].
+
+    Rows of a layer are trajectory tokens of that layer's K (V) model (the tokens a
+    looped model would emit), one token per (sequence, row); layers not listed stay
+    zero.  Returns device tensors ``win_k``, ``win_v``, ``win_len`` (int32 [B]) and the
+    host copy ``win_lens``.
+    """
+    if isinstance(layers, int):
+        layers = [layers]
+    win_lens = window_lengths(B, w_max) if win_lens is None else np.asarray(win_lens, dtype=np.int32)
+    shape = (w.L, B, w.H, w.T, w_max, w.d)
+    out = {"win_k": torch.zeros(shape, dtype=w.torch_dtype, device=device),
+           "win_v": torch.zeros(shape, dtype=w.torch_dtype, device=device),
+           "win_len": torch.as_tensor(win_lens, dtype=torch.int32, device=device),
+           "win_lens": win_lens, "w_max": w_max}
+    if B * w_max == 0:
+        return out
+    for layer in layers:
+        for axis, name in (("k", "win_k"), ("v", "win_v")):
+            tok = draw_encode_tokens(w, layer, axis, B * w_max, device, seed_tag=seed_tag)
+            # [B*w_max, T, H, d] -> [B, H, T, w_max, d]
+            out[name][layer].copy_(tok.view(B, w_max, w.T, w.H, w.d).permute(0, 3, 2, 1, 4))
     return out

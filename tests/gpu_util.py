@@ -52,7 +52,8 @@ def run_decode(p, w, layer, t0, Tq, scale, num_splits=0, variant=lla.ABSORB, q=N
     return out, lse, status
 
 
-def oracle_decode(p, w, layer, t0, Tq, scale, units=None, variant="absorb", q=None, threads=None):
+def oracle_decode(p, w, layer, t0, Tq, scale, units=None, variant="absorb", q=None, threads=None,
+                  win=None):
     q = p["q"] if q is None else q
     q64 = to64(q)
     cK, cV = to64(p["k"][layer]), to64(p["v"][layer])
@@ -60,8 +61,34 @@ def oracle_decode(p, w, layer, t0, Tq, scale, units=None, variant="absorb", q=No
     mK, mV = to64(p["mu_k"][layer]), to64(p["mu_v"][layer])
     if w.fold2d:
         WK, WV, mK, mV = WK[0], WV[0], mK[0], mV[0]
+    window = None
+    if win is not None:
+        window = (to64(win["win_k"][layer]), to64(win["win_v"][layer]), win["win_lens"])
     return oracle.decode_layer(variant, q64, cK, cV, p["starts"], p["lens"], WK, mK, WV, mV,
-                               t0, scale, fold2d=w.fold2d, units=units, threads=threads)
+                               t0, scale, fold2d=w.fold2d, units=units, threads=threads,
+                               window=window)
+
+
+def run_decode_hybrid(p, win, w, layer, t0, Tq, scale, num_splits=0, variant=lla.ABSORB, q=None,
+                      out_dtype=lla.F32):
+    """Hybrid decode through the C ABI; returns (out, lse, device status)."""
+    dims = dims_of(w, out_dtype)
+    q = p["q"] if q is None else q
+    B = len(p["lens"])
+    max_ctx = int(p["lens"].max()) if B else 0
+    ws_bytes = lla.decode_hybrid_workspace_bytes(dims, B, Tq, max_ctx, variant, num_splits)
+    ws = torch.zeros(ws_bytes, dtype=torch.uint8, device="cuda")
+    odt = torch.float32 if out_dtype == lla.F32 else torch.bfloat16
+    out = torch.full((B, Tq, w.H, w.d), float("nan"), dtype=odt, device="cuda")
+    lse = torch.full((B, Tq, w.H), float("nan"), dtype=torch.float32, device="cuda")
+    window = lla.make_window(win["win_k"], win["win_v"], win["win_len"], win["w_max"],
+                             win["win_k"].shape[1])
+    lla.decode_attn_hybrid(dims, layer, t0, Tq, q, lla.make_cache(p["k"], p["v"], p["slots"]),
+                           p["seq_start"], p["ctx_lens"], B, max_ctx, codec_of(p), window, scale,
+                           out, lse, ws, ws_bytes, variant=variant, num_splits=num_splits)
+    torch.cuda.synchronize()
+    status = lla.status_fetch(ws)
+    return out, lse, status
 
 
 def attn_errors(out_gpu, o_ref):
@@ -90,7 +117,8 @@ def assert_attn_close(out_gpu, lse_gpu, o_ref, lse_ref):
     return max_abs, rel
 
 
-def oracle_decode_units(p, w, layer, t0, Tq, scale, units, variant="absorb", q=None, threads=None):
+def oracle_decode_units(p, w, layer, t0, Tq, scale, units, variant="absorb", q=None, threads=None,
+                        win=None):
     """Oracle on sampled (b, h) units only: their latent rows are gathered to the host.
 
     Works for caches far larger than host memory; the result arrays are NaN outside
@@ -110,13 +138,20 @@ def oracle_decode_units(p, w, layer, t0, Tq, scale, units, variant="absorb", q=N
         hp = 0 if w.fold2d else h
         cK = to64(p["k"][layer, hp, s0:s0 + n])[None]
         cV = to64(p["v"][layer, hp, s0:s0 + n])[None]
+        window = None
+        if win is not None:
+            nw = int(win["win_lens"][b])
+            hsel = slice(None) if w.fold2d else slice(h, h + 1)
+            window = (to64(win["win_k"][layer, b:b + 1, hsel, :, :nw]),
+                      to64(win["win_v"][layer, b:b + 1, hsel, :, :nw]), [nw])
         if w.fold2d:
             ob, lb = oracle.decode_layer(variant, q64[b:b + 1], cK, cV, [0], [n], WK, mK, WV, mV, t0, scale,
-                                         fold2d=True, units=[(0, h)], threads=1)
+                                         fold2d=True, units=[(0, h)], threads=1, window=window)
         else:
             sel = [h]
             ob, lb = oracle.decode_layer(variant, q64[b:b + 1, :, sel], cK, cV, [0], [n], WK[sel], mK[sel],
-                                         WV[sel], mV[sel], t0, scale, fold2d=False, threads=1)
+                                         WV[sel], mV[sel], t0, scale, fold2d=False, threads=1,
+                                         window=window)
             o[b, :, h] = ob[0, :, 0]
             lse[b, :, h] = lb[0, :, 0]
             continue

@@ -133,6 +133,42 @@ def test_decode_argument_errors():
     assert _rc(B=0) == 0  # nothing to do, nothing launched
 
 
+def _hybrid_rc(window=None, **over):
+    a = _decode_args(**over)
+    if window is None:
+        window = lla.make_window(FAKE, FAKE, FAKE, 128, a["B"])
+    try:
+        lla.decode_attn_hybrid(window=window, **a)
+    except lla.LLAError as e:
+        return e.code
+    return 0
+
+
+def test_hybrid_argument_errors():
+    assert _hybrid_rc(layer=1) == lla.LLA_ERR_INVALID
+    assert _hybrid_rc(window=lla.make_window(FAKE, FAKE, FAKE, -1, 2)) == lla.LLA_ERR_INVALID
+    assert _hybrid_rc(window=lla.make_window(FAKE, FAKE, FAKE, 128, 1)) == lla.LLA_ERR_INVALID  # seqs < B
+    assert _hybrid_rc(window=lla.make_window(FAKE, FAKE, 0, 128, 2)) == lla.LLA_ERR_INVALID
+    assert _hybrid_rc(window=lla.make_window(0, FAKE, FAKE, 128, 2)) == lla.LLA_ERR_INVALID
+    assert _hybrid_rc(window=lla.make_window(FAKE + 8, FAKE, FAKE, 128, 2)) == lla.LLA_ERR_MISALIGNED
+    assert _hybrid_rc(window=lla.make_window(FAKE, FAKE, FAKE + 4, 128, 2)) == lla.LLA_ERR_MISALIGNED
+    # bf16 rows of 512 bytes at most (d_head <= 256)
+    assert _hybrid_rc(dims=lla.make_dims(4, 1, 16, 512, 16, 32)) == lla.LLA_ERR_UNSUPPORTED
+    assert _hybrid_rc(B=0) == 0
+    # a NULL window is rejected by the hybrid entry itself
+    rc = lla._lib.lla_decode_attn_hybrid(None, 0, 0, 4, None, None, None, None, 2, 100, None, None,
+                                         1.0, 0, 0, None, None, None, 0, None)
+    assert rc == lla.LLA_ERR_INVALID
+
+
+def test_hybrid_workspace_adds_one_window_record_per_query():
+    dims = lla.make_dims(4, 1, 16, 128, 16, 32)
+    base = lla.decode_workspace_bytes(dims, 64, 4, 4096)
+    hyb = lla.decode_hybrid_workspace_bytes(dims, 64, 4, 4096)
+    assert hyb >= base + 64 * 16 * 4 * (128 + 4) * 4
+    assert hyb - base < 64 * 16 * 4 * (128 + 4) * 4 + 256
+
+
 def test_workspace_bytes_and_splits():
     dims = lla.make_dims(4, 1, 16, 128, 16, 32)
     s = lla.decode_num_splits(dims, 64, 4, 4096)
