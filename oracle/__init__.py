@@ -68,6 +68,10 @@ def configure(lib):
     lib.oracle_attend_hybrid.argtypes = [i64, i64, i32, i32, i32, _dp, _dp, _dp, _dp, _dp, _dp, _dp, _dp,
                                          _dp, ctypes.c_double, _dp, _dp]
     lib.oracle_attend_hybrid.restype = i32
+    lib.oracle_attend_rope.argtypes = [i64, i32, i32, i32, _dp, _dp, _dp, _dp, _dp, _dp, _dp,
+                                       ctypes.c_double, i32, ctypes.c_double, ctypes.c_double,
+                                       ctypes.c_double, _dp, _dp]
+    lib.oracle_attend_rope.restype = i32
     return lib
 
 
@@ -180,11 +184,36 @@ def attend_hybrid(c_K, c_V, W_up_K_t, mu_K_t, W_up_V_t, mu_V_t, k_win, v_win, q,
     return o, float(lse.value)
 
 
+ROPE_HALF, ROPE_INTERLEAVED = 0, 1
+
+
+def attend_rope(c_K, c_V, W_up_K_t, mu_K_t, W_up_V_t, mu_V_t, q, scale, style, base, q_pos,
+                k_pos0=0):
+    """Faithful read: rebuilt keys and the query rotated at their positions (token i of
+    the context at k_pos0 + i, the query at q_pos), then plain attention.  -> (o, lse)."""
+    c_K, c_V = _f64(c_K), _f64(c_V)
+    W_up_K_t, mu_K_t, W_up_V_t, mu_V_t, q = map(_f64, (W_up_K_t, mu_K_t, W_up_V_t, mu_V_t, q))
+    n = c_K.shape[0]
+    r_k, r_v, d = W_up_K_t.shape[0], W_up_V_t.shape[0], q.shape[0]
+    if d % 2:
+        raise ValueError("rotary embedding needs an even head dimension")
+    if n == 0:
+        c_K = np.zeros((1, r_k)); c_V = np.zeros((1, r_v))
+    o = np.empty(d, dtype=np.float64)
+    lse = ctypes.c_double(0.0)
+    rc = _load().oracle_attend_rope(n, r_k, r_v, d, _ptr(c_K), _ptr(c_V), _ptr(W_up_K_t), _ptr(mu_K_t),
+                                    _ptr(W_up_V_t), _ptr(mu_V_t), _ptr(q), float(scale), int(style),
+                                    float(base), float(q_pos), float(k_pos0), _ptr(o), ctypes.byref(lse))
+    if rc != 0:
+        raise MemoryError("oracle scratch allocation failed")
+    return o, float(lse.value)
+
+
 # --------------------------------------------------------------------------
 # A whole decode call for one layer: loop over (b, loop t, head) instances
 # --------------------------------------------------------------------------
 def decode_layer(variant, q, c_K, c_V, seq_start, ctx_lens, W_up_K, mu_K, W_up_V, mu_V,
-                 t0, scale, fold2d=False, units=None, threads=None, window=None):
+                 t0, scale, fold2d=False, units=None, threads=None, window=None, rope=None):
     """Decode attention of every (b, tq, h) query of one layer.
 
     q        [B, Tq, H, d]           loop queries t0 .. t0+Tq-1
@@ -197,6 +226,9 @@ def decode_layer(variant, q, c_K, c_V, seq_start, ctx_lens, W_up_K, mu_K, W_up_V
              sequence's window tokens, win_k [B, H, T, w_max, d], win_len [B]; the
              hybrid form then attends over the ctx_lens[b] latents and the
              win_len[b] window tokens together (variant is ignored)
+    rope     optional (q_pos [B], base, style): the faithful read with rotary embedding,
+             cached token i of sequence b at position i, its queries at q_pos[b]
+             (variant is ignored)
     Returns (o [B, Tq, H, d], lse [B, Tq, H]); entries outside ``units`` are NaN.
     """
     q = np.asarray(q)
@@ -220,7 +252,11 @@ def decode_layer(variant, q, c_K, c_V, seq_start, ctx_lens, W_up_K, mu_K, W_up_V
         cV = c_V[hp, s0:s0 + n]
         for tq in range(Tq):
             wk, mk, wv, mv = slices(h, t0 + tq)
-            if window is None:
+            if rope is not None:
+                q_pos, base, style = rope
+                o[b, tq, h], lse[b, tq, h] = attend_rope(cK, cV, wk, mk, wv, mv, q[b, tq, h], scale,
+                                                         style, base, float(q_pos[b]))
+            elif window is None:
                 o[b, tq, h], lse[b, tq, h] = attend(variant, cK, cV, wk, mk, wv, mv,
                                                     q[b, tq, h], scale)
             else:

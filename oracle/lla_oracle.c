@@ -21,6 +21,12 @@
  *  [HLA] "Hybrid Latent Attention for Looped Language Models", abstract -- exact
  *       keys and values for a sliding window of W recent tokens, latents for the
  *       older tokens, read by every loop's query.
+ *  [P]  Same LLA paper, Pith verdict record -- key_machinery (the codec leaves the
+ *       attention computation and RoPE unchanged) and the domain assumptions (the
+ *       codec is fitted on pre-RoPE K; a token has the same position at every loop,
+ *       so RoPE can be applied after reconstruction); rotary embedding as defined by
+ *       RoFormer (arXiv:2104.09864), which the paper cites: a pair of components is
+ *       rotated by pos * base^(-2i/d).
  *
  * Conventions (all arrays row-major, caller-owned, doubles):
  *  - one stacked vector per token x in R^W with W = T*d (per-head) or W = T*H*d
@@ -288,5 +294,71 @@ int oracle_attend_hybrid(int64_t n, int64_t w, int r_k, int r_v, int d,
         for (int k = 0; k < d; ++k)
             o[k] += p[n + m] * v_win[m * d + k];
     free(k_hat); free(v_hat); free(l); free(p);
+    return 0;
+}
+
+/* ---------------------------------------------------------------------------
+ * [P]: the faithful read with rotary position embedding.  Keys are rebuilt
+ * (Eq. 3) as pre-RoPE vectors, then both the query and every rebuilt key are
+ * rotated at their own positions, and attention proceeds as usual; values are
+ * not rotated.  Component pairs: style 0 pairs i with i + d/2 (the half-split
+ * layout), style 1 pairs 2i with 2i+1 (RoFormer's layout); pair i turns by the
+ * angle pos * base^(-2i/d), counter-clockwise:
+ *   (a, b) -> (a cos - b sin, a sin + b cos).
+ * The cached token i of the sequence sits at position k_pos0 + i.
+ * ------------------------------------------------------------------------- */
+static void rope_rotate(int d, int style, double base, double pos, double *x)
+{
+    for (int i = 0; i < d / 2; ++i) {
+        const double angle = pos * pow(base, -2.0 * i / d);
+        const double cs = cos(angle), sn = sin(angle);
+        const int ia = style == 0 ? i : 2 * i;
+        const int ib = style == 0 ? i + d / 2 : 2 * i + 1;
+        const double xa = x[ia], xb = x[ib];
+        x[ia] = xa * cs - xb * sn;
+        x[ib] = xa * sn + xb * cs;
+    }
+}
+
+int oracle_attend_rope(int64_t n, int r_k, int r_v, int d,
+                       const double *c_K, const double *c_V,
+                       const double *W_up_K_t, const double *mu_K_t,
+                       const double *W_up_V_t, const double *mu_V_t,
+                       const double *q, double scale, int style, double base,
+                       double q_pos, double k_pos0, double *o, double *lse)
+{
+    for (int k = 0; k < d; ++k)
+        o[k] = 0.0;
+    if (n == 0) {
+        *lse = -INFINITY;
+        return 0;
+    }
+    double *q_rot = malloc(sizeof(double) * (size_t)d);
+    double *k_rot = malloc(sizeof(double) * (size_t)d);
+    double *v_hat = malloc(sizeof(double) * (size_t)d);
+    double *l = malloc(sizeof(double) * (size_t)n);
+    double *p = malloc(sizeof(double) * (size_t)n);
+    if (!q_rot || !k_rot || !v_hat || !l || !p) {
+        free(q_rot); free(k_rot); free(v_hat); free(l); free(p);
+        return -1;
+    }
+    for (int k = 0; k < d; ++k)
+        q_rot[k] = q[k];
+    rope_rotate(d, style, base, q_pos, q_rot);
+    for (int64_t i = 0; i < n; ++i) {
+        oracle_reconstruct(1, r_k, d, c_K + i * r_k, W_up_K_t, mu_K_t, k_rot);
+        rope_rotate(d, style, base, k_pos0 + (double)i, k_rot);
+        double dotr = 0.0;
+        for (int k = 0; k < d; ++k)
+            dotr += q_rot[k] * k_rot[k];
+        l[i] = scale * dotr;
+    }
+    softmax_rows(n, l, p, lse);
+    for (int64_t i = 0; i < n; ++i) {
+        oracle_reconstruct(1, r_v, d, c_V + i * r_v, W_up_V_t, mu_V_t, v_hat);
+        for (int k = 0; k < d; ++k)
+            o[k] += p[i] * v_hat[k];
+    }
+    free(q_rot); free(k_rot); free(v_hat); free(l); free(p);
     return 0;
 }

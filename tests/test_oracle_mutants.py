@@ -43,6 +43,11 @@ MUTANTS = {
                                       "o[k] += p[n + m] * k_win[m * d + k];"),
     "hybrid_window_key_reversed": ("dotw += q[k] * k_win[m * d + k];",
                                    "dotw += q[k] * k_win[m * d + (d - 1 - k)];"),
+    "rope_not_a_rotation": ("x[ib] = xa * sn + xb * cs;", "x[ib] = -xa * sn + xb * cs;"),
+    "rope_frequency_exponent": ("pow(base, -2.0 * i / d)", "pow(base, -1.0 * i / d)"),
+    "rope_keys_ignore_offset": ("k_pos0 + (double)i", "(double)i"),
+    "rope_query_not_rotated": ("rope_rotate(d, style, base, q_pos, q_rot);", ""),
+    "rope_half_pairs_adjacent": ("style == 0 ? i + d / 2 : 2 * i + 1", "style == 0 ? i + 1 : 2 * i + 1"),
     "bytes_drop_factor_two": ("2ull * (uint64_t)T * (uint64_t)H", "(uint64_t)T * (uint64_t)H"),
     "bytes_fold_swapped": ("fold2d ? 1u : (uint64_t)H", "fold2d ? (uint64_t)H : 1u"),
     "bytes_ratio_not_reduced": ("uint64_t g = gcd_u64(per_token_uncompressed, per_token_latent);",
@@ -66,6 +71,11 @@ def _pins():
         (P.test_hybrid_full_rank_equals_attention_over_all_tokens, {"n": 20, "w": 5}),
         (P.test_hybrid_window_order_is_irrelevant_and_empty_is_neutral, {}),
         (P.test_decode_layer_hybrid_matches_dense_attention_over_both_parts, {"fold2d": False}),
+        (P.test_rope_matches_roformer_complex_form, {"style": 0, "q_pos": 9, "k_pos0": 0}),
+        (P.test_rope_matches_roformer_complex_form, {"style": 1, "q_pos": 3000, "k_pos0": 17}),
+        (P.test_rope_depends_on_relative_position_only, {}),
+        (P.test_rope_pairings_are_one_permutation_apart, {}),
+        (P.test_decode_layer_rope_matches_dense_rotated_attention, {"style": 0}),
     ]
     for v in P.VARIANTS:
         pins += [

@@ -467,3 +467,124 @@ def test_decode_layer_hybrid_matches_dense_attention_over_both_parts(fold2d):
                 o_ref, lse_ref = sdpa(q[b, tq, h], Kh, Vh, s)
                 np.testing.assert_allclose(o[b, tq, h], o_ref, atol=1e-11)
                 assert lse[b, tq, h] == pytest.approx(lse_ref, abs=1e-11)
+
+
+# ---------------------------------------------------------------------------
+# Faithful read with rotary embedding (RoPE after reconstruction: LLA paper, Pith
+# verdict record, key_machinery and domain assumptions; RoFormer arXiv:2104.09864)
+# ---------------------------------------------------------------------------
+def _complex_pairs(x, style):
+    d = x.shape[-1]
+    if style == oracle.ROPE_HALF:
+        return x[..., :d // 2] + 1j * x[..., d // 2:]
+    return x[..., 0::2] + 1j * x[..., 1::2]
+
+
+@pytest.mark.parametrize("style", [oracle.ROPE_HALF, oracle.ROPE_INTERLEAVED])
+@pytest.mark.parametrize("q_pos,k_pos0", [(9, 0), (0, 0), (3000, 17)])
+def test_rope_matches_roformer_complex_form(style, q_pos, k_pos0):
+    """RoFormer writes the rotary map as complex multiplication, f(x, m) = x e^{i m theta_j}
+    per component pair, so the score of query m and key n is
+    Re sum_j z_q,j conj(z_k,j) e^{i (m - n) theta_j}, theta_j = base^(-2j/d).  With an
+    identity codec (W_up = I, mu = 0) the latents are the keys themselves."""
+    d, n, base, scale = 8, 11, 100.0, 0.7
+    rng = np.random.default_rng(50 + style)
+    K, V = rng.standard_normal((n, d)), rng.standard_normal((n, d))
+    q = rng.standard_normal(d)
+    I, z = np.eye(d), np.zeros(d)
+    o, lse = oracle.attend_rope(K, V, I, z, I, z, q, scale, style, base, q_pos, k_pos0)
+    theta = base ** (-2.0 * np.arange(d // 2) / d)
+    pos = k_pos0 + np.arange(n)
+    rot = np.exp(1j * (q_pos - pos)[:, None] * theta[None, :])
+    scores = scale * np.real((_complex_pairs(q, style)[None, :] * np.conj(_complex_pairs(K, style)) * rot).sum(1))
+    lse_ref = float(np.log(np.exp(scores - scores.max()).sum()) + scores.max())
+    o_ref = np.exp(scores - lse_ref) @ V
+    np.testing.assert_allclose(o, o_ref, atol=1e-11, rtol=0)
+    assert lse == pytest.approx(lse_ref, abs=1e-11)
+
+
+def test_rope_depends_on_relative_position_only():
+    """Shifting the query and every key by the same offset leaves the result unchanged."""
+    T, d, rk, rv, n = 3, 16, 4, 6, 23
+    rng = np.random.default_rng(52)
+    (WK, muK), (WV, muV) = _codec_pair(T, d, rk, rv, 53)
+    cK, cV = rng.standard_normal((n, rk)), rng.standard_normal((n, rv))
+    q = rng.standard_normal(d)
+    for style in (oracle.ROPE_HALF, oracle.ROPE_INTERLEAVED):
+        a = oracle.attend_rope(cK, cV, WK[1], muK[1], WV[1], muV[1], q, 0.5, style, 10000.0, 40, 0)
+        b = oracle.attend_rope(cK, cV, WK[1], muK[1], WV[1], muV[1], q, 0.5, style, 10000.0, 40 + 1234, 1234)
+        np.testing.assert_allclose(a[0], b[0], atol=1e-10, rtol=0)
+        assert a[1] == pytest.approx(b[1], abs=1e-10)
+        # and the rotation matters: another query position gives another result
+        c = oracle.attend_rope(cK, cV, WK[1], muK[1], WV[1], muV[1], q, 0.5, style, 10000.0, 41, 0)
+        assert np.abs(c[0] - a[0]).max() > 1e-4
+
+
+def test_rope_pairings_are_one_permutation_apart():
+    """Interleaved pairs (2i, 2i+1) become half-split pairs (i, i + d/2) once the key and
+    query components are reordered even-first; values are not rotated."""
+    T, d, rk, rv, n = 2, 12, 5, 3, 14
+    rng = np.random.default_rng(54)
+    (WK, muK), (WV, muV) = _codec_pair(T, d, rk, rv, 55)
+    cK, cV = rng.standard_normal((n, rk)), rng.standard_normal((n, rv))
+    q = rng.standard_normal(d)
+    P = np.concatenate([np.arange(0, d, 2), np.arange(1, d, 2)])
+    a = oracle.attend_rope(cK, cV, WK[0], muK[0], WV[0], muV[0], q, 1.0, oracle.ROPE_INTERLEAVED, 500.0, 30)
+    b = oracle.attend_rope(cK, cV, WK[0][:, P], muK[0][P], WV[0], muV[0], q[P], 1.0, oracle.ROPE_HALF, 500.0, 30)
+    np.testing.assert_allclose(a[0], b[0], atol=1e-12, rtol=0)
+    assert a[1] == pytest.approx(b[1], abs=1e-12)
+
+
+def test_rope_at_position_zero_is_the_plain_read():
+    """One cached token at position 0 and the query at position 0: every angle is zero."""
+    T, d, rk, rv = 2, 8, 3, 5
+    rng = np.random.default_rng(56)
+    (WK, muK), (WV, muV) = _codec_pair(T, d, rk, rv, 57)
+    cK, cV = rng.standard_normal((1, rk)), rng.standard_normal((1, rv))
+    q = rng.standard_normal(d)
+    for style in (oracle.ROPE_HALF, oracle.ROPE_INTERLEAVED):
+        a = oracle.attend_rope(cK, cV, WK[0], muK[0], WV[0], muV[0], q, 0.9, style, 10000.0, 0, 0)
+        ref = oracle.attend("reconstruct", cK, cV, WK[0], muK[0], WV[0], muV[0], q, 0.9)
+        np.testing.assert_allclose(a[0], ref[0], atol=1e-13, rtol=0)
+        assert a[1] == pytest.approx(ref[1], abs=1e-13)
+
+
+def _rotate_complex(x, pos, base, style):
+    """Rotary map in RoFormer's complex form, returned in the real layout of ``style``."""
+    d = x.shape[-1]
+    theta = base ** (-2.0 * np.arange(d // 2) / d)
+    z = _complex_pairs(x, style) * np.exp(1j * np.asarray(pos, dtype=float)[..., None] * theta)
+    out = np.empty_like(x)
+    if style == oracle.ROPE_HALF:
+        out[..., :d // 2], out[..., d // 2:] = z.real, z.imag
+    else:
+        out[..., 0::2], out[..., 1::2] = z.real, z.imag
+    return out
+
+
+@pytest.mark.parametrize("style", [oracle.ROPE_HALF, oracle.ROPE_INTERLEAVED])
+def test_decode_layer_rope_matches_dense_rotated_attention(style):
+    """Ragged batch with per-sequence query positions: each unit against SDPA over the
+    rebuilt keys rotated at positions 0..len-1 and the query rotated at q_pos[b]."""
+    T, H, d, rk, rv = 3, 2, 8, 4, 6
+    lens = np.array([5, 1, 0, 9], dtype=np.int32)
+    q_pos = np.array([5, 700, 0, 12], dtype=np.int64)
+    starts, c_K, c_V, WK, mK, WV, mV = _ragged_layer(T, H, d, lens, rk, rv, False, 26)
+    B, Tq, t0, s, base = len(lens), 2, 1, 0.8, 1000.0
+    q = np.random.default_rng(27).standard_normal((B, Tq, H, d))
+    o, lse = oracle.decode_layer("reconstruct", q, c_K, c_V, starts, lens, WK, mK, WV, mV, t0, s,
+                                 threads=2, rope=(q_pos, base, style))
+    for b in range(B):
+        sl = slice(int(starts[b]), int(starts[b] + lens[b]))
+        for tq in range(Tq):
+            for h in range(H):
+                Kh = c_K[h, sl] @ WK[h, t0 + tq] + mK[h, t0 + tq]
+                Vh = c_V[h, sl] @ WV[h, t0 + tq] + mV[h, t0 + tq]
+                if lens[b] == 0:
+                    assert np.all(o[b, tq, h] == 0) and lse[b, tq, h] == -np.inf
+                    continue
+                Kr = _rotate_complex(Kh, np.arange(lens[b]), base, style)
+                qr = _rotate_complex(q[b, tq, h], q_pos[b], base, style)
+                o_ref, lse_ref = sdpa(qr, Kr, Vh, s)
+                np.testing.assert_allclose(o[b, tq, h], o_ref, atol=1e-11)
+                assert lse[b, tq, h] == pytest.approx(lse_ref, abs=1e-11)
