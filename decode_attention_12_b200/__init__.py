@@ -9,7 +9,7 @@ library is missing.
 
 Names follow the C ABI: ``cache_bytes``, ``slot_layout``, ``codec_bias``,
 ``encode``, ``decode_attn``, ``decode_workspace_bytes``, ``decode_num_splits``,
-``decode_attn_static``, ``decode_attn_hybrid``, ``decode_hybrid_workspace_bytes``,
+``decode_attn_static``, ``decode_attn_hybrid``, ``decode_hybrid_workspace_bytes``, ``decode_attn_rope``,
 ``status_fetch``, ``status_string``.
 """
 from __future__ import annotations
@@ -38,10 +38,12 @@ LLA_ERR_DEVICE_TIMEOUT = -6
 PER_HEAD, FOLD_2D = 0, 1
 F32, BF16 = 0, 1
 ABSORB, RECONSTRUCT = 0, 1
+ROPE_HALF, ROPE_INTERLEAVED = 0, 1
 
 EXPORTED = ("lla_cache_bytes", "lla_slot_layout", "lla_codec_bias", "lla_encode",
             "lla_decode_attn", "lla_decode_workspace_bytes", "lla_decode_num_splits",
             "lla_decode_attn_static", "lla_decode_attn_hybrid", "lla_decode_hybrid_workspace_bytes",
+            "lla_decode_attn_rope",
             "lla_status_fetch", "lla_status_string")
 STATIC_SCRATCH_BYTES = 8 << 20
 
@@ -65,6 +67,10 @@ class Window(ctypes.Structure):
                 ("w_max", ctypes.c_int32), ("seqs", ctypes.c_int32)]
 
 
+class Rope(ctypes.Structure):
+    _fields_ = [("q_pos", ctypes.c_void_p), ("base", ctypes.c_float), ("style", ctypes.c_int32)]
+
+
 _i32, _i64, _u64p = ctypes.c_int32, ctypes.c_int64, ctypes.POINTER(ctypes.c_uint64)
 _vp, _sz = ctypes.c_void_p, ctypes.c_size_t
 _P = ctypes.POINTER
@@ -79,6 +85,8 @@ _lib.lla_decode_attn_static.argtypes = [_P(Dims), _i32, _i32, _i32, _vp, _P(Cach
 _lib.lla_decode_attn_hybrid.argtypes = [_P(Dims), _i32, _i32, _i32, _vp, _P(Cache), _vp, _vp, _i32,
                                         _i32, _P(Codec), _P(Window), ctypes.c_float, _i32, _i32, _vp,
                                         _vp, _vp, _sz, _vp]
+_lib.lla_decode_attn_rope.argtypes = [_P(Dims), _i32, _i32, _i32, _vp, _P(Cache), _vp, _vp, _i32, _i32,
+                                      _P(Codec), _P(Rope), ctypes.c_float, _i32, _vp, _vp, _vp, _sz, _vp]
 _lib.lla_decode_hybrid_workspace_bytes.argtypes = [_P(Dims), _i32, _i32, _i32, _i32, _i32]
 _lib.lla_decode_hybrid_workspace_bytes.restype = _sz
 _lib.lla_decode_workspace_bytes.argtypes = [_P(Dims), _i32, _i32, _i32, _i32, _i32]
@@ -88,7 +96,7 @@ _lib.lla_status_fetch.argtypes = [_vp, _vp, _P(_i32)]
 _lib.lla_status_string.argtypes = [ctypes.c_int]
 _lib.lla_status_string.restype = ctypes.c_char_p
 for _n in ("lla_cache_bytes", "lla_slot_layout", "lla_codec_bias", "lla_encode", "lla_decode_attn",
-           "lla_decode_attn_static", "lla_decode_attn_hybrid", "lla_decode_num_splits",
+           "lla_decode_attn_static", "lla_decode_attn_hybrid", "lla_decode_attn_rope", "lla_decode_num_splits",
            "lla_status_fetch"):
     getattr(_lib, _n).restype = ctypes.c_int
 
@@ -225,6 +233,25 @@ def decode_attn_hybrid(dims: Dims, layer: int, t0: int, Tq: int, q, cache: Cache
                                        _ptr(out), _ptr(lse), _ptr(workspace), int(ws_bytes),
                                        _stream(stream)),
            "lla_decode_attn_hybrid")
+
+
+def make_rope(q_pos, base: float = 10000.0, style: int = ROPE_HALF) -> Rope:
+    """Query positions q_pos int32 [B] (device), rotary base and pairing style."""
+    return Rope(_ptr(q_pos), float(base), int(style))
+
+
+def decode_attn_rope(dims: Dims, layer: int, t0: int, Tq: int, q, cache: Cache, seq_start, ctx_lens,
+                     B: int, max_ctx: int, codec: Codec, rope: Rope, softmax_scale: float, out, lse=None,
+                     workspace=None, ws_bytes: Optional[int] = None, num_splits: int = 0,
+                     stream=None) -> None:
+    """Faithful read: rebuilt keys and the query rotated at their positions (reconstruct form)."""
+    if ws_bytes is None:
+        ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
+    _check(_lib.lla_decode_attn_rope(ctypes.byref(dims), layer, t0, Tq, _ptr(q), ctypes.byref(cache),
+                                     _ptr(seq_start), _ptr(ctx_lens), B, max_ctx, ctypes.byref(codec),
+                                     ctypes.byref(rope), float(softmax_scale), num_splits, _ptr(out),
+                                     _ptr(lse), _ptr(workspace), int(ws_bytes), _stream(stream)),
+           "lla_decode_attn_rope")
 
 
 def decode_attn_static(dims: Dims, layer: int, t0: int, Tq: int, q, cache: Cache, seq_start,

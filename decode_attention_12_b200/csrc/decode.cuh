@@ -37,6 +37,10 @@ struct DecodeArgs {
     int32_t w_max;
     float *win_part;          // [B*H][Tq_all][d + 4] window output and lse (log2 units);
                               // null: no window, the combine writes the latent result alone
+    // faithful read (reconstruct form only): rotary embedding after reconstruction
+    const int32_t *q_pos;     // [B] query position of each sequence; null: no rotation
+    float rope_base;          // pair i turns by pos * rope_base^(-2i/d)
+    int32_t rope_style;       // LLA_ROPE_HALF or LLA_ROPE_INTERLEAVED
 };
 
 constexpr float kLog2e = 1.4426950408889634f;

@@ -13,6 +13,18 @@
 // absorbed form's ~1, which is the Pith verdict record's desk-editor point that the
 // latent store read this way is compute-bound.  It exists for that comparison.
 //
+// Faithful read (ROPE): the pages' model applies rotary embedding after reconstruction
+// (Pith verdict record: the codec is fitted on pre-RoPE K and a token has one position at
+// every loop).  Query and rebuilt key are rotated at their positions, which for the score
+// is one rotation of the key by the relative angle (pos_n - pos_q) * omega_i per component
+// pair.  Both elements of a pair sit in the same thread: the staged W_up,t^K rows (and q,
+// mu_t^K) are ordered so that pair i is (row i, row i + d/2) -- the identity for the
+// half-split pairing, an even-first reordering for RoFormer's (2i, 2i+1) -- and row i of
+// m16 tile md pairs with the same fragment slot of tile md + d/32.  Angles: the warp's
+// first token gets its base angle in double precision (reduced to [-pi, pi]), the 32
+// tokens of a block add a per-CTA table of cos/sin(j * omega_i); mu_t^K is rotated with
+// the key, so the constant q . mu term is not used.
+//
 // One launch serves one loop query (Tq = 1); the host launches it per loop.  The
 // scheduling (persistent token shares, producer warp, swizzled TMA tiles) is the one
 // of the absorbed kernel; each CTA stages W_up,t (transposed, bf16 hi/lo), mu_t and q_t
@@ -30,7 +42,7 @@ constexpr int kConsumers = kWarps * 32;
 constexpr int kTile = 128;
 constexpr int kStages = 3;
 
-template <int RK, int RV, int D> struct RCfg {
+template <int RK, int RV, int D, bool ROPE> struct RCfg {
     using LK = TileLayout<RK, kTile>;
     using LV = TileLayout<RV, kTile>;
     static constexpr int MD = D / 16;       // m16 tiles over the head dimension
@@ -46,16 +58,25 @@ template <int RK, int RV, int D> struct RCfg {
     static constexpr int BAR_OFF = (MRG_OFF + kWarps * (D + 2) * 4 + 15) & ~15;
     static constexpr int MISC_OFF = BAR_OFF + 2 * kStages * 8;
     static constexpr int SCR_OFF = (MISC_OFF + 16 + 15) & ~15;
-    static constexpr int PREF_OFF = SCR_OFF + (kWarps + 1) * 8;
+    static constexpr int ROT_LD = D / 2 + 4;                  // float2 per table row (bank spread)
+    static constexpr int ROT_OFF = (SCR_OFF + (kWarps + 1) * 8 + 15) & ~15; // [32][ROT_LD] cos/sin(j w_i)
+    static constexpr int OMG_OFF = ROT_OFF + (ROPE ? 32 * ROT_LD * 8 : 0); // double w_i [D/2]
+    static constexpr int PREF_OFF = OMG_OFF + (ROPE ? D / 2 * 8 : 0);
 };
 
-template <int RK, int RV, int D>
+// Kernel row of d-index k in the staged K side: pair i is (row i, row i + D/2).
+template <int D> __device__ __forceinline__ int rope_row(int k, int style)
+{
+    return style == LLA_ROPE_INTERLEAVED ? (k & 1) * (D / 2) + (k >> 1) : k;
+}
+
+template <int RK, int RV, int D, bool ROPE>
 __global__ void __launch_bounds__(kThreads, 2)
     decode_reconstruct_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant__ CUtensorMap map_kt,
                               const __grid_constant__ CUtensorMap map_v, const __grid_constant__ CUtensorMap map_vt,
                               const DecodeArgs a)
 {
-    using C = RCfg<RK, RV, D>;
+    using C = RCfg<RK, RV, D, ROPE>;
     extern __shared__ uint8_t smem_raw[];
     // aligned by arithmetic on the shared array itself, so accesses stay shared-space loads
     uint8_t *smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
@@ -78,6 +99,20 @@ __global__ void __launch_bounds__(kThreads, 2)
         }
         misc[0] = 0;
         fence_barrier_init();
+    }
+    if (ROPE) { // cos/sin(j w_i) for the 32 token offsets of a block, and w_i in double
+        float2 *rot = reinterpret_cast<float2 *>(smem + C::ROT_OFF);
+        double *omg = reinterpret_cast<double *>(smem + C::OMG_OFF);
+        const float lb = log2f(a.rope_base);
+        for (int e = tid; e < 32 * (D / 2); e += kThreads) {
+            const int j = e / (D / 2), i = e - j * (D / 2);
+            float sn, cs;
+            sincosf((float)j * exp2f(-2.0f * (float)i / (float)D * lb), &sn, &cs);
+            rot[j * C::ROT_LD + i] = make_float2(cs, sn);
+        }
+        for (int i = tid; i < D / 2; i += kThreads)
+            omg[i] = pow((double)a.rope_base, -2.0 * i / D);
+        __syncthreads();
     }
     block_length_prefix<kThreads>(a.ctx_lens, B, pref, reinterpret_cast<int64_t *>(smem + C::SCR_OFF));
     int64_t s0, s1, chunk;
@@ -127,6 +162,7 @@ __global__ void __launch_bounds__(kThreads, 2)
     } else {
         float o[C::MD][4]; // O^T fragments: rows d = 16 md + g (+8), column 0 real (tq == 0)
         float m = -INFINITY, l = 0.f;
+        int64_t rope_off = 0; // seq_start[b] + q_pos[b]: a tile row's relative position is row - rope_off
         int i = 0;
         while (walk.next(pref, a.seq_start, B, H, d)) {
             const int stage = i % kStages;
@@ -140,11 +176,12 @@ __global__ void __launch_bounds__(kThreads, 2)
                 const float *mv = a.mu_v + (a.fold ? (int64_t)tl * ld : ((int64_t)d.h * a.T + tl) * ld) + col0;
                 for (int e = tid; e < D * RK; e += kConsumers) { // read [j][k] coalesced, store [k][j]
                     const int j = e / D, k = e - j * D;
+                    const int kr = ROPE ? rope_row<D>(k, a.rope_style) : k;
                     const float x = wk[(int64_t)j * ld + k];
                     const __nv_bfloat16 hi = __float2bfloat16_rn(x);
                     const __nv_bfloat16 lo = __float2bfloat16_rn(x - __bfloat162float(hi));
-                    *reinterpret_cast<__nv_bfloat16 *>(smem + C::WK_OFF + k * C::WK_LD + 2 * j) = hi;
-                    *reinterpret_cast<__nv_bfloat16 *>(smem + C::WK_OFF + D * C::WK_LD + k * C::WK_LD + 2 * j) = lo;
+                    *reinterpret_cast<__nv_bfloat16 *>(smem + C::WK_OFF + kr * C::WK_LD + 2 * j) = hi;
+                    *reinterpret_cast<__nv_bfloat16 *>(smem + C::WK_OFF + D * C::WK_LD + kr * C::WK_LD + 2 * j) = lo;
                 }
                 for (int e = tid; e < D * RV; e += kConsumers) {
                     const int j = e / D, k = e - j * D;
@@ -157,10 +194,13 @@ __global__ void __launch_bounds__(kThreads, 2)
                 const __nv_bfloat16 *qrow =
                     static_cast<const __nv_bfloat16 *>(a.q) + (((int64_t)d.b * a.Tq_all + a.tq_off) * a.H + d.h) * D;
                 for (int k = tid; k < D; k += kConsumers) {
-                    vq[k] = __bfloat162float(qrow[k]) * a.scale * kLog2e;
-                    vmk[k] = mk[k];
+                    const int kr = ROPE ? rope_row<D>(k, a.rope_style) : k;
+                    vq[kr] = __bfloat162float(qrow[k]) * a.scale * kLog2e;
+                    vmk[kr] = mk[k];
                     vmv[k] = mv[k];
                 }
+                if (ROPE)
+                    rope_off = a.seq_start[d.b] + (int64_t)a.q_pos[d.b];
                 asm volatile("bar.sync 1, %0;" ::"r"(kConsumers) : "memory");
                 if (warp == 0) { // constant score term q . mu_t^K (log2 units)
                     float qm = 0.f;
@@ -209,9 +249,8 @@ __global__ void __launch_bounds__(kThreads, 2)
 #pragma unroll
                 for (int n = 0; n < 4; ++n)
                     sp[n][0] = sp[n][1] = 0.f;
-#pragma unroll
-                for (int md = 0; md < C::MD; ++md) {
-                    float acc[4][4];
+                // K_hat^T tile md (rows d = 16 md + g (+8), 32 token columns), without mu
+                auto k_tile = [&](int md, float (&acc)[4][4]) {
 #pragma unroll
                     for (int n = 0; n < 4; ++n)
                         acc[n][0] = acc[n][1] = acc[n][2] = acc[n][3] = 0.f;
@@ -230,11 +269,49 @@ __global__ void __launch_bounds__(kThreads, 2)
                             }
                         }
                     }
-                    const float q0 = vq[16 * md + g], q1 = vq[16 * md + g + 8];
+                };
+                if (!ROPE) {
 #pragma unroll
-                    for (int n = 0; n < 4; ++n) {
-                        sp[n][0] = fmaf(q0, acc[n][0], fmaf(q1, acc[n][2], sp[n][0]));
-                        sp[n][1] = fmaf(q0, acc[n][1], fmaf(q1, acc[n][3], sp[n][1]));
+                    for (int md = 0; md < C::MD; ++md) {
+                        float acc[4][4];
+                        k_tile(md, acc);
+                        const float q0 = vq[16 * md + g], q1 = vq[16 * md + g + 8];
+#pragma unroll
+                        for (int n = 0; n < 4; ++n) {
+                            sp[n][0] = fmaf(q0, acc[n][0], fmaf(q1, acc[n][2], sp[n][0]));
+                            sp[n][1] = fmaf(q0, acc[n][1], fmaf(q1, acc[n][3], sp[n][1]));
+                        }
+                    }
+                } else {
+                    // pair (row i, row i + D/2): tile mp and tile mp + MD/2, same fragment slot
+                    const float2 *rot = reinterpret_cast<const float2 *>(smem + C::ROT_OFF);
+                    const double *omg = reinterpret_cast<const double *>(smem + C::OMG_OFF);
+                    const int64_t rel0 = d.row + tbase - rope_off; // relative position of token 0
+#pragma unroll
+                    for (int mp = 0; mp < C::MD / 2; ++mp) {
+                        float ka[4][4], kc[4][4];
+                        k_tile(mp, ka);
+                        k_tile(mp + C::MD / 2, kc);
+#pragma unroll
+                        for (int e = 0; e < 2; ++e) {
+                            const int i = 16 * mp + g + 8 * e;
+                            const double ang = (double)rel0 * omg[i];
+                            const float red = (float)(ang - 6.283185307179586 * rint(ang * 0.15915494309189535));
+                            float s0, c0;
+                            sincosf(red, &s0, &c0);
+                            const float qa = vq[i], qb = vq[i + D / 2];
+                            const float ma = vmk[i], mb = vmk[i + D / 2];
+#pragma unroll
+                            for (int n = 0; n < 4; ++n)
+#pragma unroll
+                                for (int c = 0; c < 2; ++c) {
+                                    const float2 cj = rot[(8 * n + 2 * tq + c) * C::ROT_LD + i];
+                                    const float cp = c0 * cj.x - s0 * cj.y, sp_ = s0 * cj.x + c0 * cj.y;
+                                    const float x = ka[n][c + 2 * e] + ma, y = kc[n][c + 2 * e] + mb;
+                                    // q_a (x cos - y sin) + q_b (x sin + y cos)
+                                    sp[n][c] = fmaf(x, fmaf(qa, cp, qb * sp_), fmaf(y, fmaf(qb, cp, -qa * sp_), sp[n][c]));
+                                }
+                        }
                     }
                 }
 #pragma unroll
@@ -245,7 +322,7 @@ __global__ void __launch_bounds__(kThreads, 2)
                         x += __shfl_xor_sync(0xffffffffu, x, 4);
                         x += __shfl_xor_sync(0xffffffffu, x, 8);
                         x += __shfl_xor_sync(0xffffffffu, x, 16);
-                        sp[n][c] = x + vqmu[0];
+                        sp[n][c] = ROPE ? x : x + vqmu[0]; // ROPE: mu_t^K was rotated with the key
                         if (tbase + 8 * n + 2 * tq + c >= d.rows)
                             sp[n][c] = -INFINITY;
                     }
@@ -367,16 +444,16 @@ __global__ void __launch_bounds__(kThreads, 2)
     }
 }
 
-template <int RK, int RV, int D>
+template <int RK, int RV, int D, bool ROPE>
 cudaError_t launch_rec(const DecodeArgs &a, cudaStream_t stream)
 {
-    using C = RCfg<RK, RV, D>;
+    using C = RCfg<RK, RV, D, ROPE>;
     const int Hs = a.fold ? 1 : a.H;
     CUtensorMap mk, mkt, mv, mvt;
     if (!plane_maps(&mk, &mkt, a.k, RK, (int64_t)Hs * a.slots) ||
         !plane_maps(&mv, &mvt, a.v, RV, (int64_t)Hs * a.slots))
         return cudaErrorInvalidValue;
-    auto kern = decode_reconstruct_kernel<RK, RV, D>;
+    auto kern = decode_reconstruct_kernel<RK, RV, D, ROPE>;
     const int smem = C::PREF_OFF + 8 * (a.B + 1) + 1024;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess)
@@ -405,7 +482,7 @@ cudaError_t launch_decode_reconstruct(const DecodeArgs &a, cudaStream_t stream)
 {
 #define LLA_REC_CASE(RK, RV, D) \
     if (a.r_k == RK && a.r_v == RV && a.d == D) \
-        return launch_rec<RK, RV, D>(a, stream);
+        return a.q_pos != nullptr ? launch_rec<RK, RV, D, true>(a, stream) : launch_rec<RK, RV, D, false>(a, stream);
     LLA_REC_CASE(16, 32, 128)
     LLA_REC_CASE(16, 16, 128)
     LLA_REC_CASE(32, 32, 128)

@@ -105,18 +105,25 @@ __global__ void __launch_bounds__(kWinThreads) decode_window_kernel(const Decode
     for (int i = 0; i < N; ++i)
         acc[i] = 0.f;
 
-    for (int r0 = 0; r0 < len; r0 += ROWS) {
-        uint4 kk[kWinUnroll], vv[kWinUnroll];
-        int row[kWinUnroll];
+    // Row block r0 covers rows r0 + (warp * kWinUnroll + u) * RPW + g.  The loads of block
+    // r0 + ROWS are issued before block r0 is computed (register double buffering), so a
+    // lane always has a block of K and V chunks in flight.
+    uint4 kk[kWinUnroll], vv[kWinUnroll];
+    auto load_block = [&](int r0, uint4 (&kb)[kWinUnroll], uint4 (&vb)[kWinUnroll]) {
 #pragma unroll
         for (int u = 0; u < kWinUnroll; ++u) {
-            row[u] = r0 + (warp * kWinUnroll + u) * RPW + g;
-            kk[u] = vv[u] = make_uint4(0u, 0u, 0u, 0u);
-            if (row[u] < len && has_chunk) {
-                kk[u] = ld_stream_u4(K + (int64_t)row[u] * d);
-                vv[u] = ld_stream_u4(V + (int64_t)row[u] * d);
+            const int row = r0 + (warp * kWinUnroll + u) * RPW + g;
+            kb[u] = vb[u] = make_uint4(0u, 0u, 0u, 0u);
+            if (row < len && has_chunk) {
+                kb[u] = ld_stream_u4(K + (int64_t)row * d);
+                vb[u] = ld_stream_u4(V + (int64_t)row * d);
             }
         }
+    };
+    load_block(0, kk, vv);
+    for (int r0 = 0; r0 < len; r0 += ROWS) {
+        uint4 nk[kWinUnroll], nv[kWinUnroll];
+        load_block(r0 + ROWS, nk, nv); // rows past len load nothing
         float s[kWinUnroll];
         float mx = m;
 #pragma unroll
@@ -130,27 +137,32 @@ __global__ void __launch_bounds__(kWinThreads) decode_window_kernel(const Decode
 #pragma unroll
             for (int off = LPR / 2; off > 0; off >>= 1)
                 p += __shfl_xor_sync(0xffffffffu, p, off);
-            s[u] = row[u] < len ? p : -INFINITY;
+            s[u] = r0 + (warp * kWinUnroll + u) * RPW + g < len ? p : -INFINITY;
             mx = fmaxf(mx, s[u]);
         }
-        if (mx == -INFINITY)
-            continue; // this group had no rows in this block (m is still -inf)
-        const float al = exp2f(m - mx);
-        l *= al;
-#pragma unroll
-        for (int i = 0; i < N; ++i)
-            acc[i] *= al;
-#pragma unroll
-        for (int u = 0; u < kWinUnroll; ++u) {
-            const float p = exp2f(s[u] - mx);
-            float vf[N];
-            Chunk<T>::unpack(vv[u], vf);
-            l += p;
+        if (mx != -INFINITY) { // else this group had no rows in this block (m stays -inf)
+            const float al = exp2f(m - mx);
+            l *= al;
 #pragma unroll
             for (int i = 0; i < N; ++i)
-                acc[i] = fmaf(p, vf[i], acc[i]);
+                acc[i] *= al;
+#pragma unroll
+            for (int u = 0; u < kWinUnroll; ++u) {
+                const float p = exp2f(s[u] - mx);
+                float vf[N];
+                Chunk<T>::unpack(vv[u], vf);
+                l += p;
+#pragma unroll
+                for (int i = 0; i < N; ++i)
+                    acc[i] = fmaf(p, vf[i], acc[i]);
+            }
+            m = mx;
         }
-        m = mx;
+#pragma unroll
+        for (int u = 0; u < kWinUnroll; ++u) {
+            kk[u] = nk[u];
+            vv[u] = nv[u];
+        }
     }
 
     // merge the lane groups of this warp (lanes sub, sub + LPR, ... hold the same columns)

@@ -2,6 +2,7 @@
 // kernel selection, workspace carving, status handling.  Every arithmetic step of
 // the path runs in the kernels; this file only validates and launches.
 #include <climits>
+#include <cmath>
 #include <cstring>
 
 #include "decode.cuh"
@@ -256,9 +257,9 @@ namespace {
 // Body of lla_decode_attn and lla_decode_attn_hybrid (window == NULL: latents only).
 int decode_call(const lla_dims *dims, int32_t layer, int32_t t0, int32_t Tq, const void *q,
                 const lla_cache *cache, const int64_t *seq_start, const int32_t *ctx_lens, int32_t B,
-                int32_t max_ctx, const lla_codec *codec, const lla_window *window, float softmax_scale,
-                int32_t variant, int32_t num_splits, void *out, float *lse, void *workspace,
-                size_t ws_bytes, lla_stream_t stream)
+                int32_t max_ctx, const lla_codec *codec, const lla_window *window, const lla_rope *rope,
+                float softmax_scale, int32_t variant, int32_t num_splits, void *out, float *lse,
+                void *workspace, size_t ws_bytes, lla_stream_t stream)
 {
     int rc = check_dims(dims);
     if (rc != LLA_OK)
@@ -279,6 +280,13 @@ int decode_call(const lla_dims *dims, int32_t layer, int32_t t0, int32_t Tq, con
         return LLA_ERR_MISALIGNED;
     if ((dims->d_head * elem_bytes(dims->dtype)) % 16 != 0)
         return LLA_ERR_UNSUPPORTED; // query / output rows are moved in 16-byte pieces
+    if (rope != nullptr) {
+        if (variant != LLA_RECONSTRUCT || rope->q_pos == nullptr || !std::isfinite(rope->base) ||
+            rope->base <= 1.0f || (rope->style != LLA_ROPE_HALF && rope->style != LLA_ROPE_INTERLEAVED))
+            return LLA_ERR_INVALID;
+        if (!aligned16(rope->q_pos))
+            return LLA_ERR_MISALIGNED;
+    }
     if (window != nullptr) {
         if (window->w_max < 0 || window->seqs < B || window->len == nullptr ||
             (window->w_max > 0 && (window->k == nullptr || window->v == nullptr)))
@@ -333,6 +341,9 @@ int decode_call(const lla_dims *dims, int32_t layer, int32_t t0, int32_t Tq, con
     a.win_len = nullptr;
     a.w_max = 0;
     a.win_part = nullptr;
+    a.q_pos = rope != nullptr ? rope->q_pos : nullptr;
+    a.rope_base = rope != nullptr ? rope->base : 0.f;
+    a.rope_style = rope != nullptr ? rope->style : 0;
     if (window != nullptr) {
         // window planes [L][seqs][H][T][w_max][d]: select the layer
         const int64_t plane = (int64_t)window->seqs * dims->H * dims->T * window->w_max * dims->d_head * e;
@@ -429,7 +440,19 @@ int lla_decode_attn(const lla_dims *dims, int32_t layer, int32_t t0, int32_t Tq,
                     lla_stream_t stream)
 {
     return decode_call(dims, layer, t0, Tq, q, cache, seq_start, ctx_lens, B, max_ctx, codec, nullptr,
-                       softmax_scale, variant, num_splits, out, lse, workspace, ws_bytes, stream);
+                       nullptr, softmax_scale, variant, num_splits, out, lse, workspace, ws_bytes, stream);
+}
+
+int lla_decode_attn_rope(const lla_dims *dims, int32_t layer, int32_t t0, int32_t Tq, const void *q,
+                         const lla_cache *cache, const int64_t *seq_start, const int32_t *ctx_lens, int32_t B,
+                         int32_t max_ctx, const lla_codec *codec, const lla_rope *rope, float softmax_scale,
+                         int32_t num_splits, void *out, float *lse, void *workspace, size_t ws_bytes,
+                         lla_stream_t stream)
+{
+    if (rope == nullptr)
+        return LLA_ERR_INVALID;
+    return decode_call(dims, layer, t0, Tq, q, cache, seq_start, ctx_lens, B, max_ctx, codec, nullptr, rope,
+                       softmax_scale, LLA_RECONSTRUCT, num_splits, out, lse, workspace, ws_bytes, stream);
 }
 
 int lla_decode_attn_hybrid(const lla_dims *dims, int32_t layer, int32_t t0, int32_t Tq, const void *q,
@@ -440,7 +463,7 @@ int lla_decode_attn_hybrid(const lla_dims *dims, int32_t layer, int32_t t0, int3
 {
     if (window == nullptr)
         return LLA_ERR_INVALID;
-    return decode_call(dims, layer, t0, Tq, q, cache, seq_start, ctx_lens, B, max_ctx, codec, window,
+    return decode_call(dims, layer, t0, Tq, q, cache, seq_start, ctx_lens, B, max_ctx, codec, window, nullptr,
                        softmax_scale, variant, num_splits, out, lse, workspace, ws_bytes, stream);
 }
 

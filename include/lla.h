@@ -56,6 +56,7 @@ typedef struct CUstream_st *lla_stream_t; /* same type as cudaStream_t; NULL = l
 enum { LLA_PER_HEAD = 0, LLA_FOLD_2D = 1 };       /* lla_dims.fold                    */
 enum { LLA_F32 = 0, LLA_BF16 = 1 };               /* lla_dims.dtype                   */
 enum { LLA_ABSORB = 0, LLA_RECONSTRUCT = 1 };     /* decode read variant              */
+enum { LLA_ROPE_HALF = 0, LLA_ROPE_INTERLEAVED = 1 }; /* lla_rope.style                 */
 
 typedef struct {
     int32_t T;      /* loops (recurrence steps) of the weight-tied block                   */
@@ -212,6 +213,36 @@ int lla_decode_attn_hybrid(const lla_dims *dims, int32_t layer, int32_t t0, int3
                            lla_stream_t stream);
 size_t lla_decode_hybrid_workspace_bytes(const lla_dims *dims, int32_t B, int32_t Tq,
                                          int32_t max_ctx, int32_t variant, int32_t num_splits);
+
+/* ---- NEXT-1: faithful read with rotary position embedding --------------------------------
+ * The paper's codec is fitted on pre-RoPE keys and leaves RoPE unchanged; because a token
+ * has the same position at every loop, RoPE is applied after reconstruction (Pith verdict
+ * record, key_machinery and domain assumptions; rotary map of RoFormer, arXiv:2104.09864).
+ * For loop t of sequence b and head h:
+ *   k_hat_n = RoPE(c_K[n] W_up,t^K + mu_t^K, pos = n),   q_rot = RoPE(q, pos = q_pos[b]),
+ *   l_n = softmax_scale * q_rot . k_hat_n,   out = sum_n softmax(l)_n v_hat_n  (v not rotated)
+ * where cached token n (0-based within the sequence) sits at position n, and RoPE turns
+ * component pair i by pos * base^(-2i/d) counter-clockwise, (a, b) -> (a cos - b sin,
+ * a sin + b cos).  Pairs are (i, i + d/2) for LLA_ROPE_HALF and (2i, 2i+1) for
+ * LLA_ROPE_INTERLEAVED (RoFormer's layout).  The rotation cannot be absorbed into the
+ * query, so this runs the reconstruct-form kernels (tensor-core rebuild per tile) with the
+ * rotation applied to the rebuilt key fragments.  Angles are formed in double precision
+ * per 32-token block and in fp32 within it (about 1e-6 rad).
+ * Same arguments, errors and workspace (lla_decode_workspace_bytes with LLA_RECONSTRUCT)
+ * as lla_decode_attn with variant = LLA_RECONSTRUCT, plus `rope` (required, host struct).
+ * Additional errors: LLA_ERR_INVALID (rope NULL, q_pos NULL, style unknown, base not a
+ * finite number > 1), LLA_ERR_UNSUPPORTED (shapes the reconstruct kernels do not cover).   */
+typedef struct {
+    const int32_t *q_pos; /* int32 [B] (device): position of sequence b's query token      */
+    float base;           /* rotary base (10000 in RoFormer)                              */
+    int32_t style;        /* LLA_ROPE_HALF or LLA_ROPE_INTERLEAVED                        */
+} lla_rope;
+int lla_decode_attn_rope(const lla_dims *dims, int32_t layer, int32_t t0, int32_t Tq,
+                         const void *q, const lla_cache *cache, const int64_t *seq_start,
+                         const int32_t *ctx_lens, int32_t B, int32_t max_ctx,
+                         const lla_codec *codec, const lla_rope *rope, float softmax_scale,
+                         int32_t num_splits, void *out, float *lse, void *workspace,
+                         size_t ws_bytes, lla_stream_t stream);
 
 /* ---- decode attention with library-owned scratch ----------------------------------------
  * No counterpart in the paper: a deployment aid.  Some callers cannot allocate device

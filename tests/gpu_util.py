@@ -53,7 +53,7 @@ def run_decode(p, w, layer, t0, Tq, scale, num_splits=0, variant=lla.ABSORB, q=N
 
 
 def oracle_decode(p, w, layer, t0, Tq, scale, units=None, variant="absorb", q=None, threads=None,
-                  win=None):
+                  win=None, rope=None):
     q = p["q"] if q is None else q
     q64 = to64(q)
     cK, cV = to64(p["k"][layer]), to64(p["v"][layer])
@@ -66,7 +66,29 @@ def oracle_decode(p, w, layer, t0, Tq, scale, units=None, variant="absorb", q=No
         window = (to64(win["win_k"][layer]), to64(win["win_v"][layer]), win["win_lens"])
     return oracle.decode_layer(variant, q64, cK, cV, p["starts"], p["lens"], WK, mK, WV, mV,
                                t0, scale, fold2d=w.fold2d, units=units, threads=threads,
-                               window=window)
+                               window=window, rope=rope)
+
+
+def run_decode_rope(p, w, layer, t0, Tq, scale, q_pos, base, style, num_splits=0, q=None,
+                    out_dtype=lla.F32):
+    """Faithful (rotary) decode through the C ABI; returns (out, lse, device status)."""
+    dims = dims_of(w, out_dtype)
+    q = p["q"] if q is None else q
+    B = len(p["lens"])
+    max_ctx = int(p["lens"].max()) if B else 0
+    ws_bytes = lla.decode_workspace_bytes(dims, B, Tq, max_ctx, lla.RECONSTRUCT, num_splits)
+    ws = torch.zeros(ws_bytes, dtype=torch.uint8, device="cuda")
+    odt = torch.float32 if out_dtype == lla.F32 else torch.bfloat16
+    out = torch.full((B, Tq, w.H, w.d), float("nan"), dtype=odt, device="cuda")
+    lse = torch.full((B, Tq, w.H), float("nan"), dtype=torch.float32, device="cuda")
+    qp = torch.as_tensor(np.asarray(q_pos, dtype=np.int32), device="cuda")
+    lla.decode_attn_rope(dims, layer, t0, Tq, q, lla.make_cache(p["k"], p["v"], p["slots"]),
+                         p["seq_start"], p["ctx_lens"], B, max_ctx, codec_of(p),
+                         lla.make_rope(qp, base, style), scale, out, lse, ws, ws_bytes,
+                         num_splits=num_splits)
+    torch.cuda.synchronize()
+    status = lla.status_fetch(ws)
+    return out, lse, status
 
 
 def run_decode_hybrid(p, win, w, layer, t0, Tq, scale, num_splits=0, variant=lla.ABSORB, q=None,
@@ -118,7 +140,7 @@ def assert_attn_close(out_gpu, lse_gpu, o_ref, lse_ref):
 
 
 def oracle_decode_units(p, w, layer, t0, Tq, scale, units, variant="absorb", q=None, threads=None,
-                        win=None):
+                        win=None, rope=None):
     """Oracle on sampled (b, h) units only: their latent rows are gathered to the host.
 
     Works for caches far larger than host memory; the result arrays are NaN outside
@@ -144,14 +166,16 @@ def oracle_decode_units(p, w, layer, t0, Tq, scale, units, variant="absorb", q=N
             hsel = slice(None) if w.fold2d else slice(h, h + 1)
             window = (to64(win["win_k"][layer, b:b + 1, hsel, :, :nw]),
                       to64(win["win_v"][layer, b:b + 1, hsel, :, :nw]), [nw])
+        rope_b = None if rope is None else ([rope[0][b]], rope[1], rope[2])
         if w.fold2d:
             ob, lb = oracle.decode_layer(variant, q64[b:b + 1], cK, cV, [0], [n], WK, mK, WV, mV, t0, scale,
-                                         fold2d=True, units=[(0, h)], threads=1, window=window)
+                                         fold2d=True, units=[(0, h)], threads=1, window=window,
+                                         rope=rope_b)
         else:
             sel = [h]
             ob, lb = oracle.decode_layer(variant, q64[b:b + 1, :, sel], cK, cV, [0], [n], WK[sel], mK[sel],
                                          WV[sel], mV[sel], t0, scale, fold2d=False, threads=1,
-                                         window=window)
+                                         window=window, rope=rope_b)
             o[b, :, h] = ob[0, :, 0]
             lse[b, :, h] = lb[0, :, 0]
             continue

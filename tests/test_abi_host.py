@@ -161,6 +161,33 @@ def test_hybrid_argument_errors():
     assert rc == lla.LLA_ERR_INVALID
 
 
+def _rope_rc(rope=None, **over):
+    a = _decode_args(**over)
+    a.pop("variant")
+    if rope is None:
+        rope = lla.make_rope(FAKE, 10000.0, lla.ROPE_HALF)
+    try:
+        lla.decode_attn_rope(rope=rope, **a)
+    except lla.LLAError as e:
+        return e.code
+    return 0
+
+
+def test_rope_argument_errors():
+    assert _rope_rc(layer=1) == lla.LLA_ERR_INVALID
+    assert _rope_rc(rope=lla.make_rope(0, 10000.0, lla.ROPE_HALF)) == lla.LLA_ERR_INVALID
+    assert _rope_rc(rope=lla.make_rope(FAKE, 10000.0, 7)) == lla.LLA_ERR_INVALID
+    assert _rope_rc(rope=lla.make_rope(FAKE, 1.0, lla.ROPE_HALF)) == lla.LLA_ERR_INVALID
+    assert _rope_rc(rope=lla.make_rope(FAKE, float("nan"), lla.ROPE_HALF)) == lla.LLA_ERR_INVALID
+    assert _rope_rc(rope=lla.make_rope(FAKE + 4, 10000.0, lla.ROPE_HALF)) == lla.LLA_ERR_MISALIGNED
+    # ranks the reconstruct kernels do not cover
+    assert _rope_rc(dims=lla.make_dims(4, 1, 16, 128, 96, 160)) == lla.LLA_ERR_UNSUPPORTED
+    assert _rope_rc(B=0) == 0
+    rc = lla._lib.lla_decode_attn_rope(None, 0, 0, 4, None, None, None, None, 2, 100, None, None,
+                                       1.0, 0, None, None, None, 0, None)
+    assert rc == lla.LLA_ERR_INVALID
+
+
 def test_hybrid_workspace_adds_one_window_record_per_query():
     dims = lla.make_dims(4, 1, 16, 128, 16, 32)
     base = lla.decode_workspace_bytes(dims, 64, 4, 4096)
