@@ -38,10 +38,12 @@ SPEC_HBM_GBS = 8000.0
 PROFILE_TRAFFIC = {
     "absorb": os.path.join(ROOT, "profiles", "decode_absorb_mma.ouro1.4b-layer.json"),
     "reconstruct": os.path.join(ROOT, "profiles", "decode_reconstruct.ouro1.4b-layer.json"),
+    "rope": os.path.join(ROOT, "profiles", "decode_reconstruct_rope.ouro1.4b-layer.json"),
 }
 KERNEL_SOURCES = {
     "absorb": ("decode_mma.cu", "mma_common.cuh", "decode_sched.cuh", "decode.cuh", "common.cuh"),
     "reconstruct": ("decode_reconstruct.cu", "mma_common.cuh", "decode_sched.cuh", "decode.cuh", "common.cuh"),
+    "rope": ("decode_reconstruct.cu", "mma_common.cuh", "decode_sched.cuh", "decode.cuh", "common.cuh"),
 }
 
 
@@ -62,6 +64,9 @@ def parse():
                     help="step: decode step (headline); encode: prefill encode of one layer")
     ap.add_argument("--encode-seqs", type=int, default=0,
                     help="--phase encode: sequences of len_hi tokens to encode (default: B)")
+    ap.add_argument("--rope", action="store_true",
+                    help="faithful read: rotary embedding after reconstruction (reconstruct form, "
+                         "query positions = context lengths, half-split pairs, base 10000)")
     ap.add_argument("--window", type=int, default=0,
                     help="hybrid form: W exact window rows per sequence (all in use) besides the "
                          "latents; 0 = latents only")
@@ -370,7 +375,11 @@ def main():
     x_k = S.draw_encode_tokens(w, 0, "k", B, dev, seed_tag="new")
     x_v = S.draw_encode_tokens(w, 0, "v", B, dev, seed_tag="new")
     new_slot = (p["seq_start"] + p["ctx_lens"].to(torch.int64)).contiguous()
+    if args.rope:
+        args.variant = "reconstruct"
     variant = lla.RECONSTRUCT if args.variant == "reconstruct" else lla.ABSORB
+    # faithful read: each sequence's query sits right after its context
+    rope = lla.make_rope(p["ctx_lens"].clone(), 10000.0, lla.ROPE_HALF) if args.rope else None
     # decode calls of one step: all T loop queries fused (t0 = 0, Tq = T), or in model
     # order one call per loop (t0 = t, Tq = 1) with each loop's queries and outputs in
     # buffers of their own
@@ -389,6 +398,12 @@ def main():
 
     def decode(i, q_in=None, out_buf=None, lse_buf=None):
         for c, (t0, n) in enumerate(calls):
+            if rope is not None:
+                lla.decode_attn_rope(dims, 0, t0, n, (q_in or qs)[c], caches[i % R], p["seq_start"],
+                                     p["ctx_lens"], B, max_ctx, codec, rope, 1.0, (out_buf or outs)[c],
+                                     (lse_buf or lses)[c], ws, ws_bytes, num_splits=args.num_splits,
+                                     stream=stream)
+                continue
             if Wn:
                 lla.decode_attn_hybrid(dims, 0, t0, n, (q_in or qs)[c], caches[i % R], p["seq_start"],
                                        p["ctx_lens"], B, max_ctx, codec, windows[i % R], 1.0,
@@ -450,6 +465,24 @@ def main():
     peak = float(peaks["hbm_gbs"])
     mean_dec_ms = float(np.mean(decode_ms))
     achieved = step_bytes / (mean_dec_ms * 1e-3) / 1e9
+    roofline = {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+                "frac": achieved / peak, "peak_kind": peak_kind,
+                "traffic": profiled_traffic(S_tot * w.heads_stored, args.variant),
+                "timed": "one lla_decode_attn call (q_tilde prologue + decode + combine "
+                         "kernels), CUDA events per call on the launch stream",
+                "algorithmic_bytes_per_launch": step_bytes}
+    if args.variant == "reconstruct":
+        # the reconstruct form rebuilds K_hat and V_hat on tensor cores: per (token, head,
+        # loop) 2 d (r_k + r_v) flop for the rebuild and 4 d for the score and the P.V sum
+        flop = S_tot * w.heads_stored * Tq * (2 * w.d * (w.r_k + w.r_v) + 4 * w.d) * (w.H if w.fold2d else 1)
+        tf_peak = float(peaks.get("bf16_tflops_sustained", peaks.get("bf16_tflops", 1590.0)))
+        tfl = flop / (mean_dec_ms * 1e-3) / 1e12
+        roofline = {"bound": "tensor", "achieved": tfl, "peak": tf_peak, "unit": "TFLOP/s",
+                    "frac": tfl / tf_peak, "peak_kind": peak_kind + " (sustained bf16)",
+                    "traffic": profiled_traffic(S_tot * w.heads_stored, "rope" if args.rope else args.variant),
+                    "timed": "one decode call (one reconstruct pass per loop query + combine), "
+                             "CUDA events per call on the launch stream",
+                    "algorithmic_flop_per_call": flop, "hbm_gbs": achieved, "hbm_frac": achieved / peak}
 
     # ---- end to end through the public API with host buffers -------------------------------------
     # Every step copies its inputs (q and the new tokens' K/V) from pinned host memory and
@@ -531,7 +564,7 @@ def main():
         return
 
     cpu = None
-    if world == 1 and not args.no_cpu_baseline and not Wn:
+    if world == 1 and not args.no_cpu_baseline and not Wn and not args.rope:
         rate, info = oracle_sample_rate(p, w, Tq, args.cpu_seconds, units_per_round=max(1, B * H // 8))
         cpu = {"value": rate, "unit": "GB/s", "cores": info["cores"], "kind": "oracle",
                "sample": f"{info['rounds']} rounds of {info['units']} (sequence, head) units x "
@@ -548,7 +581,7 @@ def main():
                    "H": H, "d": w.d, "window_rows": Wn, "window_bytes_per_step": win_bytes,
                    "r_k": w.r_k, "r_v": w.r_v, "rho": "64/3", "B": B,
                    "ctx_len": [w.len_lo, w.len_hi], "tokens": S_tot, "Tq": Tq_call, "decode_calls_per_step": len(calls),
-                   "variant": args.variant, "seg_max": splits,
+                   "variant": args.variant + (" + rope" if args.rope else ""), "seg_max": splits,
                    "step": (f"{len(calls)} x decode_attn(Tq = 1, one loop each, model order)"
                             if args.model_order else f"decode_attn(all {w.T} loop queries fused)")
                            + (f" with {Wn} exact window rows per sequence (decode_attn_hybrid)" if Wn else "")
@@ -558,12 +591,7 @@ def main():
                    "parallelism": f"replicas x{world}"},
         "token_loop_reads_per_s": reads,
         "hbm_frac_of_8tbs_spec": value / world / SPEC_HBM_GBS,
-        "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
-                     "frac": achieved / peak, "peak_kind": peak_kind,
-                     "traffic": profiled_traffic(units_per_launch, args.variant),
-                     "timed": "one lla_decode_attn call (q_tilde prologue + decode + combine "
-                              "kernels), CUDA events per call on the launch stream",
-                     "algorithmic_bytes_per_launch": step_bytes},
+        "roofline": roofline,
         "cpu_baseline": cpu,
         "e2e": {"value": e2e_value, "unit": "GB/s", "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "steps": e2e_steps,

@@ -33,7 +33,7 @@ namespace {
 
 constexpr int kWinWarps = 4;
 constexpr int kWinThreads = 32 * kWinWarps;
-constexpr int kWinUnroll = 4; // 16-byte K and V chunks in flight per lane and iteration
+constexpr int kWinUnroll = 2; // rows per lane group and block (x2 in flight: double buffered)
 
 // Streaming 16-byte load: the data is read once, keep it out of L1.
 __device__ __forceinline__ uint4 ld_stream_u4(const void *p)
