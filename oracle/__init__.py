@@ -72,6 +72,8 @@ def configure(lib):
                                        ctypes.c_double, i32, ctypes.c_double, ctypes.c_double,
                                        ctypes.c_double, _dp, _dp]
     lib.oracle_attend_rope.restype = i32
+    lib.oracle_codec_residual.argtypes = [i64, i32, i32, i32, _dp, _dp, _dp, _dp, _dp, _dp]
+    lib.oracle_codec_residual.restype = i32
     return lib
 
 
@@ -182,6 +184,26 @@ def attend_hybrid(c_K, c_V, W_up_K_t, mu_K_t, W_up_V_t, mu_V_t, k_win, v_win, q,
     if rc != 0:
         raise MemoryError("oracle scratch allocation failed")
     return o, float(lse.value)
+
+
+def codec_residual(x, mu, W_down, W_up):
+    """Per-token reconstruction residual of a codec.
+
+    x [n, W] stacked vectors (W = T * Dp, loop-major), mu [W], W_down [W, r],
+    W_up [T, r, Dp]  ->  (err [n], norm [n]) with err = ||x - x_hat||, norm = ||x||.
+    """
+    x, mu, W_down, W_up = _f64(x), _f64(mu), _f64(W_down), _f64(W_up)
+    n, W = x.shape
+    T, r, Dp = W_up.shape
+    assert W == T * Dp and mu.shape == (W,) and W_down.shape == (W, r)
+    err = np.empty(n, dtype=np.float64)
+    norm = np.empty(n, dtype=np.float64)
+    if n:
+        rc = _load().oracle_codec_residual(n, T, Dp, r, _ptr(x), _ptr(mu), _ptr(W_down), _ptr(W_up),
+                                           _ptr(err), _ptr(norm))
+        if rc != 0:
+            raise MemoryError("oracle scratch allocation failed")
+    return err, norm
 
 
 ROPE_HALF, ROPE_INTERLEAVED = 0, 1

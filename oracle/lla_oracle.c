@@ -21,6 +21,9 @@
  *  [HLA] "Hybrid Latent Attention for Looped Language Models", abstract -- exact
  *       keys and values for a sliding window of W recent tokens, latents for the
  *       older tokens, read by every loop's query.
+ *  [S]  Same LLA paper, Pith verdict record -- the skeptic's concrete test: the
+ *       per-token reconstruction residual ||x - (x - mu) W_down W_up^T - mu|| / ||x||
+ *       on held-out tokens.
  *  [P]  Same LLA paper, Pith verdict record -- key_machinery (the codec leaves the
  *       attention computation and RoPE unchanged) and the domain assumptions (the
  *       codec is fitted on pre-RoPE K; a token has the same position at every loop,
@@ -360,5 +363,42 @@ int oracle_attend_rope(int64_t n, int r_k, int r_v, int d,
             o[k] += p[i] * v_hat[k];
     }
     free(q_rot); free(k_rot); free(v_hat); free(l); free(p);
+    return 0;
+}
+
+/* ---------------------------------------------------------------------------
+ * [S]: per-token reconstruction residual of a codec.  For each of the n stacked
+ * vectors x (width W = T * Dp, loop t occupying x[t*Dp .. t*Dp+Dp-1]):
+ *   c = (x - mu) W_down                     (Eq. 2)
+ *   x_hat_t = c W_up,t + mu_t for every t   (Eq. 3)
+ *   err = ||x - x_hat||,  norm = ||x||      (Euclidean, over all W components).
+ * W_up holds the T per-loop up-projections, [T][r][Dp].  The caller divides.
+ * ------------------------------------------------------------------------- */
+int oracle_codec_residual(int64_t n, int T, int Dp, int r, const double *x, const double *mu,
+                          const double *W_down, const double *W_up, double *err, double *norm)
+{
+    const int W = T * Dp;
+    double *c = malloc(sizeof(double) * (size_t)r);
+    double *x_hat = malloc(sizeof(double) * (size_t)Dp);
+    if (!c || !x_hat) {
+        free(c); free(x_hat);
+        return -1;
+    }
+    for (int64_t i = 0; i < n; ++i) {
+        const double *xi = x + i * W;
+        oracle_encode(1, W, r, xi, mu, W_down, c);
+        double e2 = 0.0, n2 = 0.0;
+        for (int t = 0; t < T; ++t) {
+            oracle_reconstruct(1, r, Dp, c, W_up + (int64_t)t * r * Dp, mu + (int64_t)t * Dp, x_hat);
+            for (int k = 0; k < Dp; ++k) {
+                const double diff = xi[t * Dp + k] - x_hat[k];
+                e2 += diff * diff;
+                n2 += xi[t * Dp + k] * xi[t * Dp + k];
+            }
+        }
+        err[i] = sqrt(e2);
+        norm[i] = sqrt(n2);
+    }
+    free(c); free(x_hat);
     return 0;
 }

@@ -48,6 +48,10 @@ MUTANTS = {
     "rope_keys_ignore_offset": ("k_pos0 + (double)i", "(double)i"),
     "rope_query_not_rotated": ("rope_rotate(d, style, base, q_pos, q_rot);", ""),
     "rope_half_pairs_adjacent": ("style == 0 ? i + d / 2 : 2 * i + 1", "style == 0 ? i + 1 : 2 * i + 1"),
+    "residual_mean_of_loop_zero": ("mu + (int64_t)t * Dp, x_hat", "mu, x_hat"),
+    "residual_first_loop_block_only": ("W_up + (int64_t)t * r * Dp", "W_up"),
+    "residual_norm_of_rebuilt": ("n2 += xi[t * Dp + k] * xi[t * Dp + k];", "n2 += x_hat[k] * x_hat[k];"),
+    "residual_squared": ("err[i] = sqrt(e2);", "err[i] = e2;"),
     "bytes_drop_factor_two": ("2ull * (uint64_t)T * (uint64_t)H", "(uint64_t)T * (uint64_t)H"),
     "bytes_fold_swapped": ("fold2d ? 1u : (uint64_t)H", "fold2d ? (uint64_t)H : 1u"),
     "bytes_ratio_not_reduced": ("uint64_t g = gcd_u64(per_token_uncompressed, per_token_latent);",
@@ -76,6 +80,10 @@ def _pins():
         (P.test_rope_depends_on_relative_position_only, {}),
         (P.test_rope_pairings_are_one_permutation_apart, {}),
         (P.test_decode_layer_rope_matches_dense_rotated_attention, {"style": 0}),
+        (P.test_residual_full_rank_codec_is_zero_and_norm_is_euclidean, {}),
+        (P.test_residual_energy_on_calibration_set_is_the_svd_tail, {"r": 5}),
+        (P.test_residual_of_in_span_and_orthogonal_offsets, {}),
+        (P.test_residual_is_homogeneous_in_the_centred_vector, {}),
     ]
     for v in P.VARIANTS:
         pins += [

@@ -588,3 +588,63 @@ def test_decode_layer_rope_matches_dense_rotated_attention(style):
                 o_ref, lse_ref = sdpa(qr, Kr, Vh, s)
                 np.testing.assert_allclose(o[b, tq, h], o_ref, atol=1e-11)
                 assert lse[b, tq, h] == pytest.approx(lse_ref, abs=1e-11)
+
+
+# ---------------------------------------------------------------------------
+# Per-token reconstruction residual (LLA paper, Pith verdict record: the skeptic's
+# concrete test, ||x - (x - mu) W_down W_up^T - mu|| / ||x||)
+# ---------------------------------------------------------------------------
+def test_residual_full_rank_codec_is_zero_and_norm_is_euclidean():
+    T, d = 4, 8
+    cod = S.orthonormal_codec(T * d, T, seed=60)
+    x = np.random.default_rng(61).standard_normal((30, T * d)) * 2 + 0.5
+    err, norm = oracle.codec_residual(x, cod.mu, cod.W_down, cod.W_up)
+    np.testing.assert_allclose(err, 0.0, atol=1e-12)
+    np.testing.assert_allclose(norm, np.linalg.norm(x, axis=1), rtol=1e-14)
+
+
+@pytest.mark.parametrize("r", [1, 5, 16, 40])
+def test_residual_energy_on_calibration_set_is_the_svd_tail(r):
+    """Eckart-Young: the SVD codec's summed squared residual on its own calibration set
+    equals the energy of the discarded singular values."""
+    w = S.shrink(S.WORKLOADS["tiny-fp32"], d=16)
+    model = S.trajectory_model(62, w.T * w.d)
+    x_cal = S.draw_tokens_np(model, S.N_CALIB, 63)
+    cod = S.fit_codec(x_cal, r, w.T)
+    err, _ = oracle.codec_residual(x_cal, cod.mu, cod.W_down, cod.W_up)
+    assert float((err ** 2).sum()) == pytest.approx(float((cod.sigma[r:] ** 2).sum()), rel=1e-9, abs=1e-9)
+
+
+def test_residual_of_in_span_and_orthogonal_offsets():
+    """Orthonormal rank-r codec with W_up = W_down^T: x = mu + (span vector) is rebuilt
+    exactly; x = mu + v with v orthogonal to the span leaves exactly ||v||."""
+    T, d, r = 3, 8, 5
+    rng = np.random.default_rng(64)
+    Q, _ = np.linalg.qr(rng.standard_normal((T * d, T * d)))
+    Wd = Q[:, :r]
+    Wu = Wd.reshape(T, d, r).transpose(0, 2, 1)
+    mu = rng.standard_normal(T * d)
+    a = rng.standard_normal((6, r))
+    b = rng.standard_normal((6, T * d - r))
+    x_in = mu + a @ Wd.T
+    v = b @ Q[:, r:].T
+    err_in, _ = oracle.codec_residual(x_in, mu, Wd, Wu)
+    err_out, norm_out = oracle.codec_residual(mu + v, mu, Wd, Wu)
+    np.testing.assert_allclose(err_in, 0.0, atol=1e-12)
+    np.testing.assert_allclose(err_out, np.linalg.norm(b, axis=1), rtol=1e-12)
+    np.testing.assert_allclose(norm_out, np.linalg.norm(mu + v, axis=1), rtol=1e-13)
+
+
+def test_residual_is_homogeneous_in_the_centred_vector():
+    """x - x_hat is linear in y = x - mu for any codec (W_up need not be W_down^T), so
+    scaling y by s scales the residual by |s|."""
+    T, d, r = 4, 8, 3
+    rng = np.random.default_rng(65)
+    Wd = rng.standard_normal((T * d, r))
+    Wu = rng.standard_normal((T, r, d))
+    mu = rng.standard_normal(T * d)
+    y = rng.standard_normal((7, T * d))
+    e1, _ = oracle.codec_residual(mu + y, mu, Wd, Wu)
+    e3, _ = oracle.codec_residual(mu - 3.0 * y, mu, Wd, Wu)
+    np.testing.assert_allclose(e3, 3.0 * e1, rtol=1e-12)
+    assert np.all(e1 > 0.1)
