@@ -10,6 +10,7 @@ library is missing.
 Names follow the C ABI: ``cache_bytes``, ``slot_layout``, ``codec_bias``,
 ``encode``, ``decode_attn``, ``decode_workspace_bytes``, ``decode_num_splits``,
 ``decode_attn_static``, ``decode_attn_hybrid``, ``decode_hybrid_workspace_bytes``, ``decode_attn_rope``,
+``codec_residual``,
 ``status_fetch``, ``status_string``.
 """
 from __future__ import annotations
@@ -43,7 +44,7 @@ ROPE_HALF, ROPE_INTERLEAVED = 0, 1
 EXPORTED = ("lla_cache_bytes", "lla_slot_layout", "lla_codec_bias", "lla_encode",
             "lla_decode_attn", "lla_decode_workspace_bytes", "lla_decode_num_splits",
             "lla_decode_attn_static", "lla_decode_attn_hybrid", "lla_decode_hybrid_workspace_bytes",
-            "lla_decode_attn_rope",
+            "lla_decode_attn_rope", "lla_codec_residual",
             "lla_status_fetch", "lla_status_string")
 STATIC_SCRATCH_BYTES = 8 << 20
 
@@ -85,6 +86,7 @@ _lib.lla_decode_attn_static.argtypes = [_P(Dims), _i32, _i32, _i32, _vp, _P(Cach
 _lib.lla_decode_attn_hybrid.argtypes = [_P(Dims), _i32, _i32, _i32, _vp, _P(Cache), _vp, _vp, _i32,
                                         _i32, _P(Codec), _P(Window), ctypes.c_float, _i32, _i32, _vp,
                                         _vp, _vp, _sz, _vp]
+_lib.lla_codec_residual.argtypes = [_P(Dims), _i32, _i32, _vp, _vp, _i64, _P(Codec), _vp, _vp, _vp, _vp, _vp]
 _lib.lla_decode_attn_rope.argtypes = [_P(Dims), _i32, _i32, _i32, _vp, _P(Cache), _vp, _vp, _i32, _i32,
                                       _P(Codec), _P(Rope), ctypes.c_float, _i32, _vp, _vp, _vp, _sz, _vp]
 _lib.lla_decode_hybrid_workspace_bytes.argtypes = [_P(Dims), _i32, _i32, _i32, _i32, _i32]
@@ -96,7 +98,8 @@ _lib.lla_status_fetch.argtypes = [_vp, _vp, _P(_i32)]
 _lib.lla_status_string.argtypes = [ctypes.c_int]
 _lib.lla_status_string.restype = ctypes.c_char_p
 for _n in ("lla_cache_bytes", "lla_slot_layout", "lla_codec_bias", "lla_encode", "lla_decode_attn",
-           "lla_decode_attn_static", "lla_decode_attn_hybrid", "lla_decode_attn_rope", "lla_decode_num_splits",
+           "lla_decode_attn_static", "lla_decode_attn_hybrid", "lla_decode_attn_rope", "lla_codec_residual",
+           "lla_decode_num_splits",
            "lla_status_fetch"):
     getattr(_lib, _n).restype = ctypes.c_int
 
@@ -182,6 +185,15 @@ def encode(dims: Dims, layer0: int, n_layers: int, x_k, x_v, n_tok: int, slot_id
     _check(_lib.lla_encode(ctypes.byref(dims), layer0, n_layers, _ptr(x_k), _ptr(x_v), int(n_tok),
                            _ptr(slot_idx), ctypes.byref(codec), ctypes.byref(cache), _stream(stream)),
            "lla_encode")
+
+
+def codec_residual(dims: Dims, layer0: int, n_layers: int, x_k, x_v, n_tok: int, codec: Codec,
+                   err_k, norm_k, err_v, norm_v, stream=None) -> None:
+    """Per-token reconstruction residual ||x - x_hat|| and norm ||x|| per (layer, token, head')."""
+    _check(_lib.lla_codec_residual(ctypes.byref(dims), layer0, n_layers, _ptr(x_k), _ptr(x_v), n_tok,
+                                   ctypes.byref(codec), _ptr(err_k), _ptr(norm_k), _ptr(err_v),
+                                   _ptr(norm_v), _stream(stream)),
+           "lla_codec_residual")
 
 
 # ---- a1-a5, a8 ------------------------------------------------------------------------------

@@ -230,6 +230,43 @@ int lla_encode(const lla_dims *dims, int32_t layer0, int32_t n_layers, const voi
     return e == cudaSuccess ? LLA_OK : LLA_ERR_CUDA;
 }
 
+int lla_codec_residual(const lla_dims *dims, int32_t layer0, int32_t n_layers, const void *x_k, const void *x_v,
+                       int64_t n_tok, const lla_codec *codec, float *err_k, float *norm_k, float *err_v,
+                       float *norm_v, lla_stream_t stream)
+{
+    int rc = check_dims(dims);
+    if (rc != LLA_OK)
+        return rc;
+    if (layer0 < 0 || n_layers < 0 || layer0 + (int64_t)n_layers > dims->L || n_tok < 0)
+        return LLA_ERR_INVALID;
+    if (n_tok == 0 || n_layers == 0)
+        return LLA_OK;
+    if (x_k == nullptr || x_v == nullptr || codec == nullptr || codec->W_down_k == nullptr ||
+        codec->W_down_v == nullptr || codec->bias_k == nullptr || codec->bias_v == nullptr ||
+        codec->W_up_k == nullptr || codec->W_up_v == nullptr || codec->mu_k == nullptr || codec->mu_v == nullptr ||
+        err_k == nullptr || norm_k == nullptr || err_v == nullptr || norm_v == nullptr)
+        return LLA_ERR_INVALID;
+    if (!aligned16(x_k) || !aligned16(x_v) || !aligned16(codec->W_down_k) || !aligned16(codec->W_down_v) ||
+        !aligned16(codec->bias_k) || !aligned16(codec->bias_v) || !aligned16(codec->W_up_k) ||
+        !aligned16(codec->W_up_v) || !aligned16(codec->mu_k) || !aligned16(codec->mu_v))
+        return LLA_ERR_MISALIGNED;
+    const int Dp = (int)loop_width(dims);
+    if (!codec_residual_supported(dims->dtype, dims->r_k, dims->r_v, Dp))
+        return LLA_ERR_UNSUPPORTED;
+    CodecResidualArgs a;
+    a.x_k = x_k; a.x_v = x_v;
+    a.W_down_k = codec->W_down_k; a.W_down_v = codec->W_down_v;
+    a.bias_k = codec->bias_k; a.bias_v = codec->bias_v;
+    a.W_up_k = codec->W_up_k; a.W_up_v = codec->W_up_v;
+    a.mu_k = codec->mu_k; a.mu_v = codec->mu_v;
+    a.err_k = err_k; a.norm_k = norm_k; a.err_v = err_v; a.norm_v = norm_v;
+    a.n_tok = n_tok;
+    a.layer0 = layer0; a.n_layers = n_layers;
+    a.T = dims->T; a.H = dims->H; a.d = dims->d_head; a.Dp = Dp; a.Hs = heads_stored(dims);
+    a.W = (int32_t)stack_width(dims); a.fold = dims->fold; a.r_k = dims->r_k; a.r_v = dims->r_v;
+    return launch_codec_residual(a, (cudaStream_t)stream) == cudaSuccess ? LLA_OK : LLA_ERR_CUDA;
+}
+
 int lla_decode_num_splits(const lla_dims *dims, int32_t B, int32_t Tq, int32_t max_ctx, int32_t variant,
                           int32_t num_splits)
 {

@@ -133,6 +133,27 @@ int lla_encode(const lla_dims *dims, int32_t layer0, int32_t n_layers, const voi
                const void *x_v, int64_t n_tok, const int64_t *slot_idx,
                const lla_codec *codec, const lla_cache *cache, lla_stream_t stream);
 
+/* ---- NEXT-3: per-token reconstruction residual (codec diagnostic) ------------------------
+ * The Pith verdict record's concrete test for the shared-subspace assumption: on held-out
+ * tokens, how much of each stacked T-loop trajectory does the codec lose?  For layers
+ * layer0 .. layer0+n_layers-1, tokens i < n_tok and stored heads h', per axis:
+ *   c = (x - mu) W_down = x W_down + b             (Eq. 2; b from lla_codec_bias)
+ *   x_hat_t = c W_up,t + mu_t for every loop t     (Eq. 3)
+ *   err = ||x - x_hat||,  norm = ||x||             (over all T * d, or T * H * d, values)
+ * and the residual fraction is err / norm.  c is kept in fp32 (never rounded to the
+ * storage type) and the rebuild runs in 3xTF32, so the result measures the codec, not
+ * the cache's bf16 rounding.
+ *   x_k, x_v   bf16 [n_layers][n_tok][T][H][d]  (the lla_encode input layout)
+ *   codec      W_down_{k,v}, bias_{k,v}, W_up_{k,v}, mu_{k,v} (all required)
+ *   err_k, norm_k, err_v, norm_v  fp32 [n_layers][n_tok][H'] (device)
+ * Runs on tensor cores (bf16 MMAs for the encode product, exact since x and W_down are
+ * bf16; tf32 hi/lo MMAs for the rebuild).  Errors: LLA_ERR_INVALID, LLA_ERR_MISALIGNED,
+ * LLA_ERR_UNSUPPORTED (dtype not bf16, a rank outside {16, 32, 64, 96, 128, 160}, or a
+ * loop width d (per head) / H * d (LLA-2D) not a multiple of 64), LLA_ERR_CUDA.        */
+int lla_codec_residual(const lla_dims *dims, int32_t layer0, int32_t n_layers, const void *x_k,
+                       const void *x_v, int64_t n_tok, const lla_codec *codec, float *err_k,
+                       float *norm_k, float *err_v, float *norm_v, lla_stream_t stream);
+
 /* ---- a1-a5, a8: decode attention ------------------------------------------------------
  * For layer `layer`, loops t = t0 .. t0+Tq-1, sequences b < B and heads h < H, the
  * loop-t query q[b][t-t0][h] attends over the ctx_lens[b] cached latents of

@@ -188,6 +188,33 @@ def test_rope_argument_errors():
     assert rc == lla.LLA_ERR_INVALID
 
 
+def test_codec_residual_argument_errors():
+    codec = lla.make_codec(W_down_k=FAKE, W_down_v=FAKE, bias_k=FAKE, bias_v=FAKE, W_up_k=FAKE,
+                           W_up_v=FAKE, mu_k=FAKE, mu_v=FAKE)
+
+    def rc(dims=None, codec=codec, **over):
+        dims = dims or lla.make_dims(4, 2, 16, 128, 16, 32)
+        a = dict(layer0=0, n_layers=1, x_k=FAKE, x_v=FAKE, n_tok=10, err_k=FAKE, norm_k=FAKE,
+                 err_v=FAKE, norm_v=FAKE, stream=0)
+        a.update(over)
+        try:
+            lla.codec_residual(dims, codec=codec, **a)
+        except lla.LLAError as e:
+            return e.code
+        return 0
+
+    assert rc(layer0=2) == lla.LLA_ERR_INVALID
+    assert rc(n_tok=-1) == lla.LLA_ERR_INVALID
+    assert rc(x_k=0) == lla.LLA_ERR_INVALID
+    assert rc(err_v=0) == lla.LLA_ERR_INVALID
+    assert rc(codec=lla.make_codec(W_down_k=FAKE, W_down_v=FAKE)) == lla.LLA_ERR_INVALID
+    assert rc(x_v=FAKE + 2) == lla.LLA_ERR_MISALIGNED
+    assert rc(dims=lla.make_dims(4, 2, 16, 128, 16, 24)) == lla.LLA_ERR_UNSUPPORTED   # rank 24
+    assert rc(dims=lla.make_dims(4, 2, 16, 96, 16, 32)) == lla.LLA_ERR_UNSUPPORTED    # d = 96
+    assert rc(dims=lla.make_dims(4, 2, 16, 128, 16, 32, 0, lla.F32)) == lla.LLA_ERR_UNSUPPORTED
+    assert rc(n_tok=0) == 0 and rc(n_layers=0) == 0
+
+
 def test_hybrid_workspace_adds_one_window_record_per_query():
     dims = lla.make_dims(4, 1, 16, 128, 16, 32)
     base = lla.decode_workspace_bytes(dims, 64, 4, 4096)

@@ -1,0 +1,70 @@
+"""GPU parity of the per-token codec reconstruction residual (LLA paper, Pith verdict
+record: the skeptic's concrete test, ||x - x_hat|| / ||x|| on held-out tokens) against
+the fp64 oracle on the same stored tokens and codec.
+
+The kernel keeps c in fp32 and rebuilds in 3xTF32, so err agrees with the fp64 oracle to
+about 1e-5 relative (it is a difference of nearly equal vectors: the bound is 1e-4);
+norm to 1e-6.  Cases: the per-head ranks 16/32 (double-buffered path) and 96/160
+(single-buffered), LLA-2D (W = 8192), token counts around the 64-token CTA tile, and a
+layer offset.
+"""
+import numpy as np
+import pytest
+import torch
+
+import decode_attention_12_b200 as lla
+import lla_synth as S
+import oracle
+from gpu_util import dims_of, to64
+
+pytestmark = pytest.mark.gpu
+DEV = "cuda"
+
+
+def _run(w, layer0, n_layers, n_tok, seed_tag="held-out"):
+    layers = list(range(layer0, layer0 + n_layers))
+    p = S.decode_inputs(w, layers, DEV, lens=[1], Tq=1)
+    p["bias_k"] = torch.zeros(w.L, w.heads_stored, w.r_k, device=DEV)
+    p["bias_v"] = torch.zeros(w.L, w.heads_stored, w.r_v, device=DEV)
+    dims = dims_of(w)
+    codec = lla.make_codec(W_down_k=p["W_down_k"], W_down_v=p["W_down_v"], bias_k=p["bias_k"],
+                           bias_v=p["bias_v"], W_up_k=p["W_up_k"], W_up_v=p["W_up_v"],
+                           mu_k=p["mu_k"], mu_v=p["mu_v"])
+    lla.codec_bias(dims, codec, p["bias_k"], p["bias_v"])
+    xs = {ax: torch.stack([S.draw_encode_tokens(w, l, ax, n_tok, DEV, seed_tag=seed_tag) for l in layers])
+          for ax in ("k", "v")}
+    out = {k: torch.full((n_layers, n_tok, w.heads_stored), float("nan"), device=DEV)
+           for k in ("err_k", "norm_k", "err_v", "norm_v")}
+    lla.codec_residual(dims, layer0, n_layers, xs["k"], xs["v"], n_tok, codec, out["err_k"], out["norm_k"],
+                       out["err_v"], out["norm_v"])
+    torch.cuda.synchronize()
+    T, Dp = w.T, w.d * (w.H if w.fold2d else 1)
+    for li, l in enumerate(layers):
+        for ax in ("k", "v"):
+            x = to64(xs[ax][li])                                   # [n, T, H, d]
+            Wd = to64(p[f"W_down_{ax}"][l])                        # [H', r, W]
+            mu = to64(p[f"mu_{ax}"][l]).reshape(w.heads_stored, -1)
+            Wu = to64(p[f"W_up_{ax}"][l])                          # [H', T, r, Dp]
+            for hs in range(w.heads_stored):
+                xr = x.reshape(n_tok, -1) if w.fold2d else x[:, :, hs, :].reshape(n_tok, -1)
+                err, norm = oracle.codec_residual(xr, mu[hs], Wd[hs].T, Wu[hs])
+                got_e = to64(out[f"err_{ax}"][li, :, hs])
+                got_n = to64(out[f"norm_{ax}"][li, :, hs])
+                np.testing.assert_allclose(got_n, norm, rtol=1e-6, atol=0)
+                np.testing.assert_allclose(got_e, err, rtol=1e-4, atol=1e-6 * float(norm.max()))
+    return out
+
+
+@pytest.mark.parametrize("n_tok", [1, 63, 64, 65, 300])
+def test_residual_per_head_small_ranks(n_tok):
+    _run(S.shrink(S.WORKLOADS["ouro1.4b-layer"], L=2), 1, 1, n_tok)
+
+
+def test_residual_per_head_large_ranks_two_layers():
+    _run(S.shrink(S.WORKLOADS["rho4-prefill"], L=4), 1, 2, 130)
+
+
+def test_residual_lla2d():
+    out = _run(S.shrink(S.WORKLOADS["lla2d"], L=2), 0, 1, 70)
+    frac = (out["err_k"] / out["norm_k"]).float()
+    assert torch.all(frac > 0) and torch.all(frac < 1)
