@@ -60,7 +60,7 @@ def parse():
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--variant", default="absorb", choices=["absorb", "reconstruct"],
                     help="decode read form (the headline uses absorb)")
-    ap.add_argument("--phase", default="step", choices=["step", "encode"],
+    ap.add_argument("--phase", default="step", choices=["step", "encode", "residual"],
                     help="step: decode step (headline); encode: prefill encode of one layer")
     ap.add_argument("--encode-seqs", type=int, default=0,
                     help="--phase encode: sequences of len_hi tokens to encode (default: B)")
@@ -318,6 +318,70 @@ def run_encode_phase(args, dev):
     }), flush=True)
 
 
+def run_residual_phase(args, dev):
+    """Codec reconstruction residual of held-out tokens (one layer, K and V)."""
+    import torch
+    import decode_attention_12_b200 as lla
+    import lla_synth as S
+
+    w = S.WORKLOADS[args.workload]
+    n_seq = args.encode_seqs or w.B
+    n_tok = n_seq * w.len_hi
+    layer = w.L - 1
+    p = S.decode_inputs(w, layer, dev, lens=[1], Tq=1)
+    dims = lla.make_dims(w.T, w.L, w.H, w.d, w.r_k, w.r_v, int(w.fold2d), lla.BF16)
+    bias_k = torch.zeros(w.L, w.heads_stored, w.r_k, device=dev)
+    bias_v = torch.zeros(w.L, w.heads_stored, w.r_v, device=dev)
+    codec = lla.make_codec(W_down_k=p["W_down_k"], W_down_v=p["W_down_v"], bias_k=bias_k, bias_v=bias_v,
+                           W_up_k=p["W_up_k"], W_up_v=p["W_up_v"], mu_k=p["mu_k"], mu_v=p["mu_v"])
+    lla.codec_bias(dims, codec, bias_k, bias_v)
+    xk = S.draw_encode_tokens(w, layer, "k", n_tok, dev, seed_tag="held-out")
+    xv = S.draw_encode_tokens(w, layer, "v", n_tok, dev, seed_tag="held-out")
+    outs = [torch.empty(1, n_tok, w.heads_stored, device=dev) for _ in range(4)]
+    stream = torch.cuda.current_stream(dev)
+
+    def step():
+        lla.codec_residual(dims, layer, 1, xk, xv, n_tok, codec, *outs, stream=stream)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    sampler = ClockSampler(dev.index or 0).start()
+    wall0 = time.perf_counter()
+    e0.record(stream)
+    for _ in range(args.steps):
+        step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    wall1 = time.perf_counter()
+    sampler.stop()
+    ms = e0.elapsed_time(e1) / args.steps
+    e = w.elem_bytes
+    # algorithmic bytes: each token's K and V stacks read once, 4 fp32 results written
+    bytes_moved = 2 * n_tok * w.H * w.T * w.d * e + 4 * n_tok * w.heads_stored * 4
+    # per (token, stored head, axis): 2 W r for c = x W_down and 2 r W for x_hat = c W_up
+    flops = 4.0 * n_tok * w.heads_stored * w.W * (w.r_k + w.r_v)
+    peaks, kind = measured_peaks()
+    gbs = bytes_moved / (ms * 1e-3) / 1e9
+    tfl = flops / (ms * 1e-3) / 1e12
+    frac = (outs[0] / outs[1]).double()
+    print(json.dumps({
+        "metric": "LLA codec reconstruction residual GB/s (one layer, K and V)", "value": gbs, "unit": "GB/s",
+        "n_gpus": 1, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+        "higher_is_better": True, "dtype": "bf16 x bf16 -> f32, 3xtf32", "data": "synthetic",
+        "config": {"workload": w.name, "tokens": n_tok, "H": w.H, "T": w.T, "d": w.d, "r_k": w.r_k,
+                   "r_v": w.r_v, "fold2d": w.fold2d},
+        "roofline": {"bound": "hbm", "achieved": gbs, "peak": float(peaks["hbm_gbs"]), "unit": "GB/s",
+                     "frac": gbs / float(peaks["hbm_gbs"]), "peak_kind": kind},
+        "tensor": {"achieved_tflops": tfl, "peak_tflops": float(peaks.get("bf16_tflops", 1590.0)),
+                   "frac": tfl / float(peaks.get("bf16_tflops", 1590.0)),
+                   "note": "algorithmic flop; the tf32 hi/lo rebuild issues 3 MMAs per product"},
+        "residual_fraction_k": {"mean": float(frac.mean()), "max": float(frac.max())},
+        "clocks": sampler.summary(wall0, wall1),
+    }), flush=True)
+
+
 # ---------------------------------------------------------------------------
 # our arm
 # ---------------------------------------------------------------------------
@@ -344,6 +408,9 @@ def main():
 
     if args.phase == "encode":
         run_encode_phase(args, dev)
+        return
+    if args.phase == "residual":
+        run_residual_phase(args, dev)
         return
     w = S.WORKLOADS[args.workload]
     Tq = w.T

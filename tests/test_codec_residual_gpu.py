@@ -3,8 +3,9 @@ record: the skeptic's concrete test, ||x - x_hat|| / ||x|| on held-out tokens) a
 the fp64 oracle on the same stored tokens and codec.
 
 The kernel keeps c in fp32 and rebuilds in 3xTF32, so err agrees with the fp64 oracle to
-about 1e-5 relative (it is a difference of nearly equal vectors: the bound is 1e-4);
-norm to 1e-6.  Cases: the per-head ranks 16/32 (double-buffered path) and 96/160
+about 1e-5 relative (it is a difference of nearly equal vectors: the bound is 1e-4).  Each
+lane sums W/4 squared terms in fp32, so norm carries about sqrt(W/4) * 2^-24 relative
+rounding (3e-6 at the LLA-2D width W = 8192); its bound is 8 times that.  Cases: the per-head ranks 16/32 (double-buffered path) and 96/160
 (single-buffered), LLA-2D (W = 8192), token counts around the 64-token CTA tile, and a
 layer offset.
 """
@@ -50,7 +51,8 @@ def _run(w, layer0, n_layers, n_tok, seed_tag="held-out"):
                 err, norm = oracle.codec_residual(xr, mu[hs], Wd[hs].T, Wu[hs])
                 got_e = to64(out[f"err_{ax}"][li, :, hs])
                 got_n = to64(out[f"norm_{ax}"][li, :, hs])
-                np.testing.assert_allclose(got_n, norm, rtol=1e-6, atol=0)
+                rtol_n = 8.0 * np.sqrt(w.W / 4) * 2.0 ** -24
+                np.testing.assert_allclose(got_n, norm, rtol=rtol_n, atol=0)
                 np.testing.assert_allclose(got_e, err, rtol=1e-4, atol=1e-6 * float(norm.max()))
     return out
 
