@@ -72,6 +72,10 @@ def configure(lib):
                                        ctypes.c_double, i32, ctypes.c_double, ctypes.c_double,
                                        ctypes.c_double, _dp, _dp]
     lib.oracle_attend_rope.restype = i32
+    lib.oracle_attend_decoupled.argtypes = [i64, i32, i32, i32, i32, _dp, _dp, _dp, _dp, _dp, _dp, _dp, _dp,
+                                            _dp, ctypes.c_double, i32, ctypes.c_double, ctypes.c_double,
+                                            _dp, _dp]
+    lib.oracle_attend_decoupled.restype = i32
     lib.oracle_codec_residual.argtypes = [i64, i32, i32, i32, _dp, _dp, _dp, _dp, _dp, _dp]
     lib.oracle_codec_residual.restype = i32
     return lib
@@ -186,6 +190,31 @@ def attend_hybrid(c_K, c_V, W_up_K_t, mu_K_t, W_up_V_t, mu_V_t, k_win, v_win, q,
     return o, float(lse.value)
 
 
+def attend_decoupled(c_K, c_V, W_up_K_t, mu_K_t, W_up_V_t, mu_V_t, k_rope, q, q_rope, scale, style,
+                     base, q_pos):
+    """Decoupled rotary sub-key: k_rope [n, d_r] stored rotated, q_rope [d_r] rotated at
+    q_pos here; score = scale (q . k_hat + rope(q_rope) . k_rope).  -> (o [d], lse)."""
+    c_K, c_V, k_rope = _f64(c_K), _f64(c_V), _f64(k_rope)
+    W_up_K_t, mu_K_t, W_up_V_t, mu_V_t, q, q_rope = map(_f64, (W_up_K_t, mu_K_t, W_up_V_t, mu_V_t, q, q_rope))
+    n = c_K.shape[0]
+    r_k, r_v, d, d_r = W_up_K_t.shape[0], W_up_V_t.shape[0], q.shape[0], q_rope.shape[0]
+    if d_r % 2:
+        raise ValueError("the rotary part needs an even width")
+    if n == 0:
+        c_K = np.zeros((1, r_k)); c_V = np.zeros((1, r_v)); k_rope = np.zeros((1, max(d_r, 1)))
+    if d_r == 0:
+        q_rope = np.zeros(1); k_rope = np.zeros((max(n, 1), 1))
+    o = np.empty(d, dtype=np.float64)
+    lse = ctypes.c_double(0.0)
+    rc = _load().oracle_attend_decoupled(n, r_k, r_v, d, d_r, _ptr(c_K), _ptr(c_V), _ptr(W_up_K_t),
+                                         _ptr(mu_K_t), _ptr(W_up_V_t), _ptr(mu_V_t), _ptr(k_rope), _ptr(q),
+                                         _ptr(q_rope), float(scale), int(style), float(base), float(q_pos),
+                                         _ptr(o), ctypes.byref(lse))
+    if rc != 0:
+        raise MemoryError("oracle scratch allocation failed")
+    return o, float(lse.value)
+
+
 def codec_residual(x, mu, W_down, W_up):
     """Per-token reconstruction residual of a codec.
 
@@ -235,7 +264,8 @@ def attend_rope(c_K, c_V, W_up_K_t, mu_K_t, W_up_V_t, mu_V_t, q, scale, style, b
 # A whole decode call for one layer: loop over (b, loop t, head) instances
 # --------------------------------------------------------------------------
 def decode_layer(variant, q, c_K, c_V, seq_start, ctx_lens, W_up_K, mu_K, W_up_V, mu_V,
-                 t0, scale, fold2d=False, units=None, threads=None, window=None, rope=None):
+                 t0, scale, fold2d=False, units=None, threads=None, window=None, rope=None,
+                 decoupled=None):
     """Decode attention of every (b, tq, h) query of one layer.
 
     q        [B, Tq, H, d]           loop queries t0 .. t0+Tq-1
@@ -251,6 +281,9 @@ def decode_layer(variant, q, c_K, c_V, seq_start, ctx_lens, W_up_K, mu_K, W_up_V
     rope     optional (q_pos [B], base, style): the faithful read with rotary embedding,
              cached token i of sequence b at position i, its queries at q_pos[b]
              (variant is ignored)
+    decoupled optional (k_rope [H', S, d_r], q_rope [B, Tq, H, d_r], q_pos [B], base, style):
+             the decoupled rotary sub-key beside each latent (stored rotated), the
+             queries' rotary parts rotated at q_pos[b] (variant is ignored)
     Returns (o [B, Tq, H, d], lse [B, Tq, H]); entries outside ``units`` are NaN.
     """
     q = np.asarray(q)
@@ -274,7 +307,12 @@ def decode_layer(variant, q, c_K, c_V, seq_start, ctx_lens, W_up_K, mu_K, W_up_V
         cV = c_V[hp, s0:s0 + n]
         for tq in range(Tq):
             wk, mk, wv, mv = slices(h, t0 + tq)
-            if rope is not None:
+            if decoupled is not None:
+                k_rope, q_rope, q_pos, base, style = decoupled
+                o[b, tq, h], lse[b, tq, h] = attend_decoupled(
+                    cK, cV, wk, mk, wv, mv, k_rope[hp, s0:s0 + n], q[b, tq, h], q_rope[b, tq, h], scale,
+                    style, base, float(q_pos[b]))
+            elif rope is not None:
                 q_pos, base, style = rope
                 o[b, tq, h], lse[b, tq, h] = attend_rope(cK, cV, wk, mk, wv, mv, q[b, tq, h], scale,
                                                          style, base, float(q_pos[b]))

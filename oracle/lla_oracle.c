@@ -24,6 +24,10 @@
  *  [S]  Same LLA paper, Pith verdict record -- the skeptic's concrete test: the
  *       per-token reconstruction residual ||x - (x - mu) W_down W_up^T - mu|| / ||x||
  *       on held-out tokens.
+ *  [D]  Same LLA paper, Pith verdict record -- desk-editor letter: the absorbed-attention
+ *       variant needs decoupled RoPE (a rotary sub-key kept exact beside the latent,
+ *       as in multi-head latent attention), which the paper measures with a fidelity
+ *       floor.
  *  [P]  Same LLA paper, Pith verdict record -- key_machinery (the codec leaves the
  *       attention computation and RoPE unchanged) and the domain assumptions (the
  *       codec is fitted on pre-RoPE K; a token has the same position at every loop,
@@ -400,5 +404,58 @@ int oracle_codec_residual(int64_t n, int T, int Dp, int r, const double *x, cons
         norm[i] = sqrt(n2);
     }
     free(c); free(x_hat);
+    return 0;
+}
+
+/* ---------------------------------------------------------------------------
+ * [D]: decoupled rotary sub-key.  Beside its latent, cached token i keeps an exact
+ * sub-key k_rope[i] (d_r values), stored already rotated at the token's position;
+ * the query brings a rotary part q_rope (d_r values), rotated here at q_pos.  The
+ * loop-t score adds the two dot products:
+ *   l_i = scale * (q . k_hat_i + rope(q_rope, q_pos) . k_rope[i]),
+ * with k_hat_i rebuilt by Eq. 3; values are rebuilt as usual and not rotated.
+ * ------------------------------------------------------------------------- */
+int oracle_attend_decoupled(int64_t n, int r_k, int r_v, int d, int d_r,
+                            const double *c_K, const double *c_V,
+                            const double *W_up_K_t, const double *mu_K_t,
+                            const double *W_up_V_t, const double *mu_V_t,
+                            const double *k_rope, const double *q, const double *q_rope,
+                            double scale, int style, double base, double q_pos,
+                            double *o, double *lse)
+{
+    for (int k = 0; k < d; ++k)
+        o[k] = 0.0;
+    if (n == 0) {
+        *lse = -INFINITY;
+        return 0;
+    }
+    double *qr = malloc(sizeof(double) * (size_t)(d_r > 0 ? d_r : 1));
+    double *k_hat = malloc(sizeof(double) * (size_t)d);
+    double *v_hat = malloc(sizeof(double) * (size_t)d);
+    double *l = malloc(sizeof(double) * (size_t)n);
+    double *p = malloc(sizeof(double) * (size_t)n);
+    if (!qr || !k_hat || !v_hat || !l || !p) {
+        free(qr); free(k_hat); free(v_hat); free(l); free(p);
+        return -1;
+    }
+    for (int k = 0; k < d_r; ++k)
+        qr[k] = q_rope[k];
+    rope_rotate(d_r, style, base, q_pos, qr);
+    for (int64_t i = 0; i < n; ++i) {
+        oracle_reconstruct(1, r_k, d, c_K + i * r_k, W_up_K_t, mu_K_t, k_hat);
+        double dn = 0.0, dr = 0.0;
+        for (int k = 0; k < d; ++k)
+            dn += q[k] * k_hat[k];
+        for (int k = 0; k < d_r; ++k)
+            dr += qr[k] * k_rope[i * d_r + k];
+        l[i] = scale * (dn + dr);
+    }
+    softmax_rows(n, l, p, lse);
+    for (int64_t i = 0; i < n; ++i) {
+        oracle_reconstruct(1, r_v, d, c_V + i * r_v, W_up_V_t, mu_V_t, v_hat);
+        for (int k = 0; k < d; ++k)
+            o[k] += p[i] * v_hat[k];
+    }
+    free(qr); free(k_hat); free(v_hat); free(l); free(p);
     return 0;
 }

@@ -52,6 +52,10 @@ MUTANTS = {
     "residual_first_loop_block_only": ("W_up + (int64_t)t * r * Dp", "W_up"),
     "residual_norm_of_rebuilt": ("n2 += xi[t * Dp + k] * xi[t * Dp + k];", "n2 += x_hat[k] * x_hat[k];"),
     "residual_squared": ("err[i] = sqrt(e2);", "err[i] = e2;"),
+    "decoupled_drops_rope_term": ("l[i] = scale * (dn + dr);", "l[i] = scale * dn;"),
+    "decoupled_query_not_rotated": ("rope_rotate(d_r, style, base, q_pos, qr);", ""),
+    "decoupled_rope_term_unscaled": ("l[i] = scale * (dn + dr);", "l[i] = scale * dn + dr;"),
+    "decoupled_wrong_subkey_row": ("dr += qr[k] * k_rope[i * d_r + k];", "dr += qr[k] * k_rope[k];"),
     "bytes_drop_factor_two": ("2ull * (uint64_t)T * (uint64_t)H", "(uint64_t)T * (uint64_t)H"),
     "bytes_fold_swapped": ("fold2d ? 1u : (uint64_t)H", "fold2d ? (uint64_t)H : 1u"),
     "bytes_ratio_not_reduced": ("uint64_t g = gcd_u64(per_token_uncompressed, per_token_latent);",
@@ -80,6 +84,9 @@ def _pins():
         (P.test_rope_depends_on_relative_position_only, {}),
         (P.test_rope_pairings_are_one_permutation_apart, {}),
         (P.test_decode_layer_rope_matches_dense_rotated_attention, {"style": 0}),
+        (P.test_decoupled_identity_codec_is_attention_over_concatenated_keys, {"style": 1}),
+        (P.test_decoupled_rope_part_depends_on_relative_position, {}),
+        (P.test_decoupled_without_rope_part_is_the_plain_read, {}),
         (P.test_residual_full_rank_codec_is_zero_and_norm_is_euclidean, {}),
         (P.test_residual_energy_on_calibration_set_is_the_svd_tail, {"r": 5}),
         (P.test_residual_of_in_span_and_orthogonal_offsets, {}),

@@ -648,3 +648,87 @@ def test_residual_is_homogeneous_in_the_centred_vector():
     e3, _ = oracle.codec_residual(mu - 3.0 * y, mu, Wd, Wu)
     np.testing.assert_allclose(e3, 3.0 * e1, rtol=1e-12)
     assert np.all(e1 > 0.1)
+
+
+# ---------------------------------------------------------------------------
+# Decoupled rotary sub-key beside the latent (LLA paper, Pith verdict record, desk-editor
+# letter: the absorbed variant needs decoupled RoPE)
+# ---------------------------------------------------------------------------
+@pytest.mark.parametrize("style", [oracle.ROPE_HALF, oracle.ROPE_INTERLEAVED])
+def test_decoupled_identity_codec_is_attention_over_concatenated_keys(style):
+    """Identity codec (W_up = I, mu = 0): the result is textbook attention of the query
+    [q ; rope(q_rope, q_pos)] (rotated in RoFormer's complex form) over the keys
+    [k ; k_rope] (SDPA)."""
+    d, d_r, n, base, q_pos = 8, 4, 13, 200.0, 37
+    rng = np.random.default_rng(70 + style)
+    K, V = rng.standard_normal((n, d)), rng.standard_normal((n, d))
+    K_r = rng.standard_normal((n, d_r))
+    q, q_r = rng.standard_normal(d), rng.standard_normal(d_r)
+    I, z = np.eye(d), np.zeros(d)
+    o, lse = oracle.attend_decoupled(K, V, I, z, I, z, K_r, q, q_r, 0.8, style, base, q_pos)
+    q_full = np.concatenate([q, _rotate_complex(q_r, q_pos, base, style)])
+    o_ref, lse_ref = sdpa(q_full, np.concatenate([K, K_r], axis=1), V, 0.8)
+    np.testing.assert_allclose(o, o_ref, atol=1e-11, rtol=0)
+    assert lse == pytest.approx(lse_ref, abs=1e-11)
+
+
+def test_decoupled_rope_part_depends_on_relative_position():
+    """Sub-keys stored rotated at their positions p_i: shifting every p_i and q_pos by the
+    same offset leaves the result unchanged; the latent part is unaffected."""
+    T, d, rk, rv, n, d_r = 2, 8, 3, 5, 9, 6
+    rng = np.random.default_rng(72)
+    (WK, muK), (WV, muV) = _codec_pair(T, d, rk, rv, 73)
+    cK, cV = rng.standard_normal((n, rk)), rng.standard_normal((n, rv))
+    raw = rng.standard_normal((n, d_r))
+    q, q_r = rng.standard_normal(d), rng.standard_normal(d_r)
+    out = []
+    for off in (0, 4321):
+        stored = _rotate_complex(raw, off + np.arange(n), 10000.0, oracle.ROPE_HALF)
+        out.append(oracle.attend_decoupled(cK, cV, WK[1], muK[1], WV[1], muV[1], stored, q, q_r, 0.5,
+                                           oracle.ROPE_HALF, 10000.0, off + 20))
+    np.testing.assert_allclose(out[0][0], out[1][0], atol=1e-10, rtol=0)
+    assert out[0][1] == pytest.approx(out[1][1], abs=1e-10)
+
+
+def test_decoupled_without_rope_part_is_the_plain_read():
+    """d_r = 0: nothing beside the latent, the result is the plain (unrotated) read."""
+    T, d, rk, rv, n = 2, 8, 3, 5, 11
+    rng = np.random.default_rng(74)
+    (WK, muK), (WV, muV) = _codec_pair(T, d, rk, rv, 75)
+    cK, cV = rng.standard_normal((n, rk)), rng.standard_normal((n, rv))
+    q = rng.standard_normal(d)
+    a = oracle.attend_decoupled(cK, cV, WK[0], muK[0], WV[0], muV[0], np.zeros((n, 0)), q, np.zeros(0), 0.7,
+                                oracle.ROPE_HALF, 10000.0, 5)
+    ref = oracle.attend("absorb", cK, cV, WK[0], muK[0], WV[0], muV[0], q, 0.7)
+    np.testing.assert_allclose(a[0], ref[0], atol=1e-12, rtol=0)
+    assert a[1] == pytest.approx(ref[1], abs=1e-12)
+
+
+def test_decode_layer_decoupled_matches_dense_attention():
+    """Ragged batch: each unit against SDPA over [rebuilt keys | stored sub-keys] with the
+    query [q ; rope(q_rope, q_pos[b])] (complex form)."""
+    T, H, d, rk, rv, d_r = 3, 2, 8, 4, 6, 4
+    lens = np.array([5, 1, 0, 9], dtype=np.int32)
+    q_pos = np.array([5, 900, 0, 9])
+    starts, c_K, c_V, WK, mK, WV, mV = _ragged_layer(T, H, d, lens, rk, rv, False, 28)
+    rng = np.random.default_rng(29)
+    B, Tq, t0, s, base = len(lens), 2, 1, 0.8, 1000.0
+    k_rope = rng.standard_normal((H, c_K.shape[1], d_r))
+    q = rng.standard_normal((B, Tq, H, d))
+    q_r = rng.standard_normal((B, Tq, H, d_r))
+    o, lse = oracle.decode_layer("absorb", q, c_K, c_V, starts, lens, WK, mK, WV, mV, t0, s, threads=2,
+                                 decoupled=(k_rope, q_r, q_pos, base, oracle.ROPE_INTERLEAVED))
+    for b in range(B):
+        sl = slice(int(starts[b]), int(starts[b] + lens[b]))
+        for tq in range(Tq):
+            for h in range(H):
+                if lens[b] == 0:
+                    assert np.all(o[b, tq, h] == 0) and lse[b, tq, h] == -np.inf
+                    continue
+                Kh = c_K[h, sl] @ WK[h, t0 + tq] + mK[h, t0 + tq]
+                Vh = c_V[h, sl] @ WV[h, t0 + tq] + mV[h, t0 + tq]
+                qf = np.concatenate([q[b, tq, h], _rotate_complex(q_r[b, tq, h], q_pos[b], base,
+                                                                  oracle.ROPE_INTERLEAVED)])
+                o_ref, lse_ref = sdpa(qf, np.concatenate([Kh, k_rope[h, sl]], axis=1), Vh, s)
+                np.testing.assert_allclose(o[b, tq, h], o_ref, atol=1e-11)
+                assert lse[b, tq, h] == pytest.approx(lse_ref, abs=1e-11)
