@@ -10,7 +10,7 @@ library is missing.
 Names follow the C ABI: ``cache_bytes``, ``slot_layout``, ``codec_bias``,
 ``encode``, ``decode_attn``, ``decode_workspace_bytes``, ``decode_num_splits``,
 ``decode_attn_static``, ``decode_attn_hybrid``, ``decode_hybrid_workspace_bytes``, ``decode_attn_rope``,
-``codec_residual``,
+``codec_residual``, ``decode_attn_decoupled``, ``decode_decoupled_workspace_bytes``,
 ``status_fetch``, ``status_string``.
 """
 from __future__ import annotations
@@ -44,7 +44,8 @@ ROPE_HALF, ROPE_INTERLEAVED = 0, 1
 EXPORTED = ("lla_cache_bytes", "lla_slot_layout", "lla_codec_bias", "lla_encode",
             "lla_decode_attn", "lla_decode_workspace_bytes", "lla_decode_num_splits",
             "lla_decode_attn_static", "lla_decode_attn_hybrid", "lla_decode_hybrid_workspace_bytes",
-            "lla_decode_attn_rope", "lla_codec_residual",
+            "lla_decode_attn_rope", "lla_codec_residual", "lla_decode_attn_decoupled",
+            "lla_decode_decoupled_workspace_bytes",
             "lla_status_fetch", "lla_status_string")
 STATIC_SCRATCH_BYTES = 8 << 20
 
@@ -72,6 +73,10 @@ class Rope(ctypes.Structure):
     _fields_ = [("q_pos", ctypes.c_void_p), ("base", ctypes.c_float), ("style", ctypes.c_int32)]
 
 
+class Decoupled(ctypes.Structure):
+    _fields_ = [("k_rope", ctypes.c_void_p), ("q_rope", ctypes.c_void_p), ("d_rope", ctypes.c_int32)]
+
+
 _i32, _i64, _u64p = ctypes.c_int32, ctypes.c_int64, ctypes.POINTER(ctypes.c_uint64)
 _vp, _sz = ctypes.c_void_p, ctypes.c_size_t
 _P = ctypes.POINTER
@@ -86,6 +91,11 @@ _lib.lla_decode_attn_static.argtypes = [_P(Dims), _i32, _i32, _i32, _vp, _P(Cach
 _lib.lla_decode_attn_hybrid.argtypes = [_P(Dims), _i32, _i32, _i32, _vp, _P(Cache), _vp, _vp, _i32,
                                         _i32, _P(Codec), _P(Window), ctypes.c_float, _i32, _i32, _vp,
                                         _vp, _vp, _sz, _vp]
+_lib.lla_decode_attn_decoupled.argtypes = [_P(Dims), _i32, _i32, _i32, _vp, _P(Cache), _vp, _vp, _i32, _i32,
+                                           _P(Codec), _P(Decoupled), _P(Rope), ctypes.c_float, _i32, _vp, _vp,
+                                           _vp, _sz, _vp]
+_lib.lla_decode_decoupled_workspace_bytes.argtypes = [_P(Dims), _i32, _i32, _i32, _i32, _i32]
+_lib.lla_decode_decoupled_workspace_bytes.restype = _sz
 _lib.lla_codec_residual.argtypes = [_P(Dims), _i32, _i32, _vp, _vp, _i64, _P(Codec), _vp, _vp, _vp, _vp, _vp]
 _lib.lla_decode_attn_rope.argtypes = [_P(Dims), _i32, _i32, _i32, _vp, _P(Cache), _vp, _vp, _i32, _i32,
                                       _P(Codec), _P(Rope), ctypes.c_float, _i32, _vp, _vp, _vp, _sz, _vp]
@@ -99,6 +109,7 @@ _lib.lla_status_string.argtypes = [ctypes.c_int]
 _lib.lla_status_string.restype = ctypes.c_char_p
 for _n in ("lla_cache_bytes", "lla_slot_layout", "lla_codec_bias", "lla_encode", "lla_decode_attn",
            "lla_decode_attn_static", "lla_decode_attn_hybrid", "lla_decode_attn_rope", "lla_codec_residual",
+           "lla_decode_attn_decoupled",
            "lla_decode_num_splits",
            "lla_status_fetch"):
     getattr(_lib, _n).restype = ctypes.c_int
@@ -264,6 +275,31 @@ def decode_attn_rope(dims: Dims, layer: int, t0: int, Tq: int, q, cache: Cache, 
                                      ctypes.byref(rope), float(softmax_scale), num_splits, _ptr(out),
                                      _ptr(lse), _ptr(workspace), int(ws_bytes), _stream(stream)),
            "lla_decode_attn_rope")
+
+
+def decode_decoupled_workspace_bytes(dims: Dims, B: int, Tq: int, max_ctx: int, d_rope: int,
+                                     num_splits: int = 0) -> int:
+    n = _lib.lla_decode_decoupled_workspace_bytes(ctypes.byref(dims), B, Tq, max_ctx, d_rope, num_splits)
+    if n == 0:
+        raise LLAError(LLA_ERR_INVALID, "lla_decode_decoupled_workspace_bytes")
+    return int(n)
+
+
+def decode_attn_decoupled(dims: Dims, layer: int, t0: int, Tq: int, q, cache: Cache, seq_start, ctx_lens,
+                          B: int, max_ctx: int, codec: Codec, k_rope, q_rope, d_rope: int, rope: Rope,
+                          softmax_scale: float, out, lse=None, workspace=None, ws_bytes: Optional[int] = None,
+                          num_splits: int = 0, stream=None) -> None:
+    """Absorbed read with a decoupled rotary sub-key plane k_rope [L][H][slots][d_rope] (stored
+    rotated) and the queries' rotary parts q_rope [B][Tq][H][d_rope] (rotated at rope.q_pos)."""
+    if ws_bytes is None:
+        ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
+    dec = Decoupled(_ptr(k_rope), _ptr(q_rope), int(d_rope))
+    _check(_lib.lla_decode_attn_decoupled(ctypes.byref(dims), layer, t0, Tq, _ptr(q), ctypes.byref(cache),
+                                          _ptr(seq_start), _ptr(ctx_lens), B, max_ctx, ctypes.byref(codec),
+                                          ctypes.byref(dec), ctypes.byref(rope), float(softmax_scale),
+                                          num_splits, _ptr(out), _ptr(lse), _ptr(workspace), int(ws_bytes),
+                                          _stream(stream)),
+           "lla_decode_attn_decoupled")
 
 
 def decode_attn_static(dims: Dims, layer: int, t0: int, Tq: int, q, cache: Cache, seq_start,

@@ -41,6 +41,10 @@ struct DecodeArgs {
     const int32_t *q_pos;     // [B] query position of each sequence; null: no rotation
     float rope_base;          // pair i turns by pos * rope_base^(-2i/d)
     int32_t rope_style;       // LLA_ROPE_HALF or LLA_ROPE_INTERLEAVED
+    // decoupled rotary sub-key beside the latent (absorbed form, tensor-core kernel)
+    const void *k_rope;       // T [H'][slots][d_rope], stored rotated at each token's position
+    const void *q_rope;       // T [B][Tq_all][H][d_rope], rotated at q_pos by the prologue
+    int32_t d_rope;           // 0: none; q_tilde rows then hold r_k + d_rope values
 };
 
 constexpr float kLog2e = 1.4426950408889634f;
@@ -58,6 +62,7 @@ cudaError_t launch_absorb_prologue(const DecodeArgs &a, int dtype, cudaStream_t 
 cudaError_t launch_decode_combine(const DecodeArgs &a, int dtype, int out_dtype, cudaStream_t stream);
 bool decode_absorb_supported(int dtype, int r_k, int r_v, int d, int fold);
 bool decode_mma_supported(int dtype, int r_k, int r_v, int fold, int Tq);
+bool decode_mma_rope_supported(int dtype, int r_k, int r_v, int d_rope, int fold);
 cudaError_t launch_decode_absorb_mma(const DecodeArgs &a, int ctas, cudaStream_t stream);
 bool decode_reconstruct_supported(int dtype, int r_k, int r_v, int d);
 // LLA-2D: every latent tile read once for all heads of a sequence (H * loops <= 64 rows

@@ -25,19 +25,27 @@ namespace lla {
 namespace {
 using namespace mma;
 
-// NW consumer warps (32 tokens of a tile each) + one producer warp.
-template <int RK, int RV, int NW> struct MCfg {
+// NW consumer warps (32 tokens of a tile each) + one producer warp.  DR > 0: every cached
+// token also carries a decoupled rotary sub-key of DR values in a plane of its own (the
+// Pith verdict record's decoupled RoPE for the absorbed variant); its tile sits beside
+// the key tile and adds DR / 16 k16 steps to the score MMA, with the rotated rotary query
+// part appended to q_tilde (rows of RK + DR).
+template <int RK, int RV, int NW, int DR = 0> struct MCfg {
     static constexpr int TILE = 32 * NW;
     static constexpr int THREADS = (NW + 1) * 32;
     static constexpr int CONSUMERS = NW * 32;
-    static constexpr int STAGES = (RK + RV) * 2 * TILE > 24 * 1024 ? 2 : 3;
+    static constexpr int STAGES = (RK + RV + DR) * 2 * TILE > 24 * 1024 ? 2 : 3;
     using LK = TileLayout<RK, TILE>;
     using LV = TileLayout<RV, TILE>;
-    static constexpr int KS = RK / 16;  // k16 steps of the score MMA
+    using LR = TileLayout<(DR > 0 ? DR : 16), TILE>;
+    static constexpr int RKT = RK + DR; // q_tilde row
+    static constexpr int KS = RK / 16;  // k16 steps of the score MMA over the latent
+    static constexpr int KSR = DR / 16; // k16 steps over the rotary sub-key
     static constexpr int NTV = RV / 8;  // n8 tiles of the output
-    static constexpr int K_BYTES = LK::BYTES, V_BYTES = LV::BYTES;
-    static constexpr int Q_BYTES = 16 * RK * 4;
-    static constexpr int STAGE = align1024(K_BYTES + V_BYTES + Q_BYTES);
+    static constexpr int K_BYTES = LK::BYTES, V_BYTES = LV::BYTES, R_BYTES = DR > 0 ? LR::BYTES : 0;
+    static constexpr int Q_OFF = K_BYTES + V_BYTES + R_BYTES;
+    static constexpr int Q_BYTES = 16 * RKT * 4;
+    static constexpr int STAGE = align1024(Q_OFF + Q_BYTES);
     static constexpr int RING = STAGES * STAGE;
     static constexpr int MRG_OFF = RING;                              // [NW][16][RV + 2]
     static constexpr int BAR_OFF = (MRG_OFF + NW * 16 * (RV + 2) * 4 + 15) & ~15; // full[S], empty[S]
@@ -47,13 +55,13 @@ template <int RK, int RV, int NW> struct MCfg {
 };
 
 // TQ16: the tile carries more than 8 loop queries, so fragment rows g + 8 are real.
-template <int RK, int RV, bool TQ16, int NW, int MINB>
-__global__ void __launch_bounds__((NW + 1) * 32, MINB)
-    decode_absorb_mma_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant__ CUtensorMap map_kt,
-                             const __grid_constant__ CUtensorMap map_v, const __grid_constant__ CUtensorMap map_vt,
-                             const DecodeArgs a)
+template <int RK, int RV, bool TQ16, int NW, int DR>
+__device__ __forceinline__ void decode_mma_body(const CUtensorMap *map_k, const CUtensorMap *map_kt,
+                                                const CUtensorMap *map_v, const CUtensorMap *map_vt,
+                                                const CUtensorMap *map_r, const CUtensorMap *map_rt,
+                                                const DecodeArgs &a)
 {
-    using C = MCfg<RK, RV, NW>;
+    using C = MCfg<RK, RV, NW, DR>;
     constexpr int kWarps = NW, kThreads = C::THREADS, kConsumers = C::CONSUMERS, kTile = C::TILE;
     constexpr int kStages = C::STAGES;
     extern __shared__ uint8_t smem_raw[];
@@ -105,42 +113,50 @@ __global__ void __launch_bounds__((NW + 1) * 32, MINB)
                     break;
                 const uint32_t st = sbase + stage * C::STAGE;
                 const int nbox = (d.rows + kBox - 1) / kBox;
-                const uint32_t qb = (d.flags & 1) ? (uint32_t)(Tq * RK * 4) : 0u;
+                const uint32_t qb = (d.flags & 1) ? (uint32_t)(Tq * C::RKT * 4) : 0u;
                 const uint32_t bar = full0 + 8 * stage;
                 fence_proxy_async_smem(); // consumers' generic writes to this stage come first
-                mbar_arrive_expect_tx(bar, nbox * kBox * (RK + RV) * 2 + qb);
+                mbar_arrive_expect_tx(bar, nbox * kBox * (RK + RV + DR) * 2 + qb);
                 const int hs = a.fold ? 0 : d.h; // LLA-2D: every head reads the one folded plane
                 const int y0 = (int)((int64_t)hs * a.slots + d.row);
                 for (int bx = 0; bx < nbox; ++bx) {
                     const int y = y0 + bx * kBox;
 #pragma unroll
                     for (int blk = 0; blk < C::LK::NBLK; ++blk)
-                        tma_load_2d(st + blk * kTile * 128 + bx * kBox * 128, &map_k, 64 * blk, y, bar);
+                        tma_load_2d(st + blk * kTile * 128 + bx * kBox * 128, map_k, 64 * blk, y, bar);
                     if (C::LK::TAIL)
-                        tma_load_2d(st + C::LK::NBLK * kTile * 128 + bx * kBox * C::LK::TB, &map_kt,
+                        tma_load_2d(st + C::LK::NBLK * kTile * 128 + bx * kBox * C::LK::TB, map_kt,
                                     64 * C::LK::NBLK, y, bar);
                     const uint32_t sv0 = st + C::K_BYTES;
 #pragma unroll
                     for (int blk = 0; blk < C::LV::NBLK; ++blk)
-                        tma_load_2d(sv0 + blk * kTile * 128 + bx * kBox * 128, &map_v, 64 * blk, y, bar);
+                        tma_load_2d(sv0 + blk * kTile * 128 + bx * kBox * 128, map_v, 64 * blk, y, bar);
                     if (C::LV::TAIL)
-                        tma_load_2d(sv0 + C::LV::NBLK * kTile * 128 + bx * kBox * C::LV::TB, &map_vt,
+                        tma_load_2d(sv0 + C::LV::NBLK * kTile * 128 + bx * kBox * C::LV::TB, map_vt,
                                     64 * C::LV::NBLK, y, bar);
+                    if constexpr (DR > 0) { // the rotary sub-key plane, same rows
+                        const uint32_t sr0 = sv0 + C::V_BYTES;
+#pragma unroll
+                        for (int blk = 0; blk < C::LR::NBLK; ++blk)
+                            tma_load_2d(sr0 + blk * kTile * 128 + bx * kBox * 128, map_r, 64 * blk, y, bar);
+                        if (C::LR::TAIL)
+                            tma_load_2d(sr0 + C::LR::NBLK * kTile * 128 + bx * kBox * C::LR::TB, map_rt,
+                                        64 * C::LR::NBLK, y, bar);
+                    }
                 }
                 if (qb) {
                     if (!q_ready) {
                         grid_dependency_wait();
                         q_ready = true;
                     }
-                    bulk_copy_g2s(st + C::K_BYTES + C::V_BYTES, a.qt + ((int64_t)d.u * a.Tq_all + a.tq_off) * RK, qb,
-                                  bar);
+                    bulk_copy_g2s(st + C::Q_OFF, a.qt + ((int64_t)d.u * a.Tq_all + a.tq_off) * C::RKT, qb, bar);
                 }
                 ++issued;
             }
         }
     } else {
         // ================= consumer warps =================
-        uint32_t qa[C::KS][2][4]; // q_tilde A fragments, [k16 step][hi/lo][a0..a3]
+        uint32_t qa[C::KS + C::KSR][2][4]; // q_tilde A fragments, [k16 step][hi/lo][a0..a3]
         float o[C::NTV][4];       // output accumulator fragments (rows g, g + 8)
         float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.f, l1 = 0.f;
         int i = 0;
@@ -161,20 +177,20 @@ __global__ void __launch_bounds__((NW + 1) * 32, MINB)
                     __syncwarp();
                 }
                 if (d.flags & 1) { // new unit segment: its q_tilde, fresh state
-                    const float *qs =
-                        reinterpret_cast<const float *>(smem + stage * C::STAGE + C::K_BYTES + C::V_BYTES);
+                    const float *qs = reinterpret_cast<const float *>(smem + stage * C::STAGE + C::Q_OFF);
+                    constexpr int QL = C::RKT;
 #pragma unroll
-                    for (int kk = 0; kk < C::KS; ++kk) {
+                    for (int kk = 0; kk < C::KS + C::KSR; ++kk) {
                         const int c0 = 16 * kk + 2 * tq;
                         float x[4][2];
 #pragma unroll
                         for (int r = 0; r < 2; ++r) { // rows g, g + 8
                             const int row = g + 8 * r;
                             const bool in = row < Tq;
-                            x[r][0] = in ? qs[row * RK + c0] : 0.f;
-                            x[r][1] = in ? qs[row * RK + c0 + 1] : 0.f;
-                            x[2 + r][0] = in ? qs[row * RK + c0 + 8] : 0.f;
-                            x[2 + r][1] = in ? qs[row * RK + c0 + 9] : 0.f;
+                            x[r][0] = in ? qs[row * QL + c0] : 0.f;
+                            x[r][1] = in ? qs[row * QL + c0 + 1] : 0.f;
+                            x[2 + r][0] = in ? qs[row * QL + c0 + 8] : 0.f;
+                            x[2 + r][1] = in ? qs[row * QL + c0 + 9] : 0.f;
                         }
                         // a0: (g, c0..), a1: (g+8, c0..), a2: (g, c0+8..), a3: (g+8, c0+8..)
 #pragma unroll
@@ -209,6 +225,24 @@ __global__ void __launch_bounds__((NW + 1) * 32, MINB)
                                          kb[0], kb[1]);
                                 mma16816(s[2 * half + 1], qa[kk][hl][0], qa[kk][hl][1], qa[kk][hl][2],
                                          qa[kk][hl][3], kb[2], kb[3]);
+                            }
+                        }
+                        if constexpr (DR > 0) { // + rotated q_rope . k_rope
+                            const uint32_t sr = sv + C::V_BYTES;
+#pragma unroll
+                            for (int kr = 0; kr < C::KSR; ++kr) {
+                                uint32_t rb[4];
+                                const int tok = t16 + ((lane >> 4) << 3) + (lane & 7);
+                                const int ch = 2 * kr + ((lane >> 3) & 1);
+                                ldsm_x4(sr + C::LR::off(tok, ch), rb);
+                                const int kq = C::KS + kr;
+#pragma unroll
+                                for (int hl = 0; hl < 2; ++hl) {
+                                    mma16816(s[2 * half], qa[kq][hl][0], qa[kq][hl][1], qa[kq][hl][2],
+                                             qa[kq][hl][3], rb[0], rb[1]);
+                                    mma16816(s[2 * half + 1], qa[kq][hl][0], qa[kq][hl][1], qa[kq][hl][2],
+                                             qa[kq][hl][3], rb[2], rb[3]);
+                                }
                             }
                         }
                     }
@@ -358,17 +392,42 @@ __global__ void __launch_bounds__((NW + 1) * 32, MINB)
     }
 }
 
-// ---- host ------------------------------------------------------------------------------
 template <int RK, int RV, bool TQ16, int NW, int MINB>
+__global__ void __launch_bounds__((NW + 1) * 32, MINB)
+    decode_absorb_mma_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant__ CUtensorMap map_kt,
+                             const __grid_constant__ CUtensorMap map_v, const __grid_constant__ CUtensorMap map_vt,
+                             const DecodeArgs a)
+{
+    decode_mma_body<RK, RV, TQ16, NW, 0>(&map_k, &map_kt, &map_v, &map_vt, nullptr, nullptr, a);
+}
+
+// With the decoupled rotary sub-key plane (two more tensor maps).
+template <int RK, int RV, bool TQ16, int NW, int MINB, int DR>
+__global__ void __launch_bounds__((NW + 1) * 32, MINB)
+    decode_absorb_mma_rope_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant__ CUtensorMap map_kt,
+                                  const __grid_constant__ CUtensorMap map_v, const __grid_constant__ CUtensorMap map_vt,
+                                  const __grid_constant__ CUtensorMap map_r, const __grid_constant__ CUtensorMap map_rt,
+                                  const DecodeArgs a)
+{
+    decode_mma_body<RK, RV, TQ16, NW, DR>(&map_k, &map_kt, &map_v, &map_vt, &map_r, &map_rt, a);
+}
+
+// ---- host ------------------------------------------------------------------------------
+template <int RK, int RV, bool TQ16, int NW, int MINB, int DR>
 cudaError_t launch_mma_t(const DecodeArgs &a, int ctas, cudaStream_t stream)
 {
-    using C = MCfg<RK, RV, NW>;
+    using C = MCfg<RK, RV, NW, DR>;
     const int Hs = a.fold ? 1 : a.H;
-    CUtensorMap mk, mkt, mv, mvt;
+    CUtensorMap mk, mkt, mv, mvt, mr, mrt;
     if (!plane_maps(&mk, &mkt, a.k, RK, (int64_t)Hs * a.slots) ||
-        !plane_maps(&mv, &mvt, a.v, RV, (int64_t)Hs * a.slots))
+        !plane_maps(&mv, &mvt, a.v, RV, (int64_t)Hs * a.slots) ||
+        (DR > 0 && !plane_maps(&mr, &mrt, a.k_rope, DR, (int64_t)Hs * a.slots)))
         return cudaErrorInvalidValue;
-    auto kern = decode_absorb_mma_kernel<RK, RV, TQ16, NW, MINB>;
+    const void *kern;
+    if constexpr (DR > 0)
+        kern = (const void *)decode_absorb_mma_rope_kernel<RK, RV, TQ16, NW, MINB, DR>;
+    else
+        kern = (const void *)decode_absorb_mma_kernel<RK, RV, TQ16, NW, MINB>;
     const int smem = C::PREF_OFF + 8 * (a.B + 1) + 1024;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess)
@@ -394,18 +453,23 @@ cudaError_t launch_mma_t(const DecodeArgs &a, int ctas, cudaStream_t stream)
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, kern, mk, mkt, mv, mvt, a);
+    if constexpr (DR > 0)
+        return cudaLaunchKernelEx(&cfg, decode_absorb_mma_rope_kernel<RK, RV, TQ16, NW, MINB, DR>, mk, mkt, mv, mvt,
+                                  mr, mrt, a);
+    else
+        return cudaLaunchKernelEx(&cfg, decode_absorb_mma_kernel<RK, RV, TQ16, NW, MINB>, mk, mkt, mv, mvt, a);
 }
 
 // Small ranks: 128-token tiles, 4 consumer warps, 4 CTAs per SM.  Ranks >= 64: 64-token
 // tiles, 2 consumer warps, 2 CTAs per SM (larger register and shared-memory footprint).
-template <int RK, int RV>
+template <int RK, int RV, int DR = 0>
 cudaError_t launch_mma(const DecodeArgs &a, int ctas, cudaStream_t stream)
 {
     constexpr bool big = RK >= 64 || RV >= 64;
-    constexpr int NW = big ? 2 : 4, MINB = big ? 2 : 4;
-    return a.Tq > 8 ? launch_mma_t<RK, RV, true, NW, MINB>(a, ctas, stream)
-                    : launch_mma_t<RK, RV, false, NW, MINB>(a, ctas, stream);
+    // a 64-wide rotary sub-key adds 32 registers of q_tilde fragments: 3 CTAs per SM
+    constexpr int NW = big ? 2 : 4, MINB = big ? 2 : (DR >= 64 ? 3 : 4);
+    return a.Tq > 8 ? launch_mma_t<RK, RV, true, NW, MINB, DR>(a, ctas, stream)
+                    : launch_mma_t<RK, RV, false, NW, MINB, DR>(a, ctas, stream);
 }
 
 } // namespace
@@ -418,8 +482,21 @@ bool decode_mma_supported(int dtype, int r_k, int r_v, int fold, int Tq)
     return dtype == LLA_BF16 && pair && tensor_map_encoder() != nullptr;
 }
 
+bool decode_mma_rope_supported(int dtype, int r_k, int r_v, int d_rope, int fold)
+{
+    return dtype == LLA_BF16 && fold == LLA_PER_HEAD && r_k == 16 && r_v == 32 && (d_rope == 32 || d_rope == 64) &&
+           tensor_map_encoder() != nullptr;
+}
+
 cudaError_t launch_decode_absorb_mma(const DecodeArgs &a, int ctas, cudaStream_t stream)
 {
+    if (a.d_rope > 0) {
+        if (a.r_k == 16 && a.r_v == 32 && a.d_rope == 32)
+            return launch_mma<16, 32, 32>(a, ctas, stream);
+        if (a.r_k == 16 && a.r_v == 32 && a.d_rope == 64)
+            return launch_mma<16, 32, 64>(a, ctas, stream);
+        return cudaErrorNotSupported;
+    }
 #define LLA_MMA_CASE(RK, RV) \
     if (a.r_k == RK && a.r_v == RV) \
         return launch_mma<RK, RV>(a, ctas, stream);

@@ -438,7 +438,29 @@ __global__ void __launch_bounds__(kPrologueThreads) absorb_prologue_kernel(const
             s3 = fmaf(qr[k + 3], wr[k + 3], s3);
         }
         const int64_t u = (int64_t)(b0 + bl) * a.H + h;
-        a.qt[(u * a.Tq_all + a.tq_off + t) * RK + j] = ((s0 + s1) + (s2 + s3)) * a.scale * kLog2e;
+        a.qt[(u * a.Tq_all + a.tq_off + t) * (RK + a.d_rope) + j] = ((s0 + s1) + (s2 + s3)) * a.scale * kLog2e;
+    }
+    if (a.d_rope > 0) {
+        // decoupled rotary part: q_rope rotated at the query position, appended to q_tilde;
+        // pair i (i, i + d_r/2 or 2i, 2i+1) turns by q_pos * base^(-2i/d_r), angle in fp64
+        const int dr = a.d_rope, np = dr / 2;
+        for (int o = threadIdx.x; o < nb * np; o += kPrologueThreads) {
+            const int bl = o / np, i = o - bl * np;
+            const int b = b0 + bl;
+            const int ia = a.rope_style == LLA_ROPE_INTERLEAVED ? 2 * i : i;
+            const int ib = a.rope_style == LLA_ROPE_INTERLEAVED ? 2 * i + 1 : i + np;
+            const T *qr = static_cast<const T *>(a.q_rope) + (((int64_t)b * a.Tq_all + a.tq_off + t) * a.H + h) * dr;
+            const float xa = Elem<T>::to_f(qr[ia]), xb = Elem<T>::to_f(qr[ib]);
+            const double ang = (double)a.q_pos[b] * pow((double)a.rope_base, -2.0 * i / dr);
+            const float red = (float)(ang - 6.283185307179586 * rint(ang * 0.15915494309189535));
+            float sn, cs;
+            sincosf(red, &sn, &cs);
+            const int64_t u = (int64_t)b * a.H + h;
+            float *dst = a.qt + (u * a.Tq_all + a.tq_off + t) * (RK + dr) + RK;
+            const float sc = a.scale * kLog2e;
+            dst[ia] = (xa * cs - xb * sn) * sc;
+            dst[ib] = (xa * sn + xb * cs) * sc;
+        }
     }
 }
 

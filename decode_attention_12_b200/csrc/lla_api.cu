@@ -68,7 +68,7 @@ struct Plan {
 size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
 
 Plan make_plan(const lla_dims *d, int32_t B, int32_t Tq, int32_t max_ctx, int32_t num_splits, int32_t variant,
-               bool window = false)
+               bool window = false, int32_t d_rope = 0)
 {
     Plan p;
     const int64_t units = (int64_t)B * d->H;
@@ -87,7 +87,7 @@ Plan make_plan(const lla_dims *d, int32_t B, int32_t Tq, int32_t max_ctx, int32_
     p.seg_max = (int32_t)((max_ctx + chunk_min - 1) / chunk_min + 1);
     p.off_counts = kWorkspaceHeader;
     p.off_qt = align256(p.off_counts + (size_t)units * sizeof(int32_t));
-    p.off_part = align256(p.off_qt + (size_t)units * Tq * d->r_k * sizeof(float));
+    p.off_part = align256(p.off_qt + (size_t)units * Tq * (d->r_k + d_rope) * sizeof(float));
     // reconstruct-form records carry d-wide outputs, absorbed-form records r_v-wide latents
     const int rec_w = variant == LLA_RECONSTRUCT ? d->d_head : d->r_v;
     p.bytes = p.off_part + (size_t)units * Tq * p.seg_max * part_stride(rec_w) * sizeof(float);
@@ -296,7 +296,7 @@ int decode_call(const lla_dims *dims, int32_t layer, int32_t t0, int32_t Tq, con
                 const lla_cache *cache, const int64_t *seq_start, const int32_t *ctx_lens, int32_t B,
                 int32_t max_ctx, const lla_codec *codec, const lla_window *window, const lla_rope *rope,
                 float softmax_scale, int32_t variant, int32_t num_splits, void *out, float *lse,
-                void *workspace, size_t ws_bytes, lla_stream_t stream)
+                void *workspace, size_t ws_bytes, lla_stream_t stream, const lla_decoupled *dec = nullptr)
 {
     int rc = check_dims(dims);
     if (rc != LLA_OK)
@@ -317,13 +317,21 @@ int decode_call(const lla_dims *dims, int32_t layer, int32_t t0, int32_t Tq, con
         return LLA_ERR_MISALIGNED;
     if ((dims->d_head * elem_bytes(dims->dtype)) % 16 != 0)
         return LLA_ERR_UNSUPPORTED; // query / output rows are moved in 16-byte pieces
+    if (dec != nullptr) {
+        if (rope == nullptr || dec->k_rope == nullptr || dec->q_rope == nullptr || dec->d_rope <= 0)
+            return LLA_ERR_INVALID;
+        if (!aligned16(dec->k_rope) || !aligned16(dec->q_rope))
+            return LLA_ERR_MISALIGNED;
+    }
     if (rope != nullptr) {
-        if (variant != LLA_RECONSTRUCT || rope->q_pos == nullptr || !std::isfinite(rope->base) ||
+        if (variant != (dec != nullptr ? LLA_ABSORB : LLA_RECONSTRUCT) || rope->q_pos == nullptr || !std::isfinite(rope->base) ||
             rope->base <= 1.0f || (rope->style != LLA_ROPE_HALF && rope->style != LLA_ROPE_INTERLEAVED))
             return LLA_ERR_INVALID;
         if (!aligned16(rope->q_pos))
             return LLA_ERR_MISALIGNED;
     }
+    if (dec != nullptr && !decode_mma_rope_supported(dims->dtype, dims->r_k, dims->r_v, dec->d_rope, dims->fold))
+        return LLA_ERR_UNSUPPORTED;
     if (window != nullptr) {
         if (window->w_max < 0 || window->seqs < B || window->len == nullptr ||
             (window->w_max > 0 && (window->k == nullptr || window->v == nullptr)))
@@ -333,7 +341,8 @@ int decode_call(const lla_dims *dims, int32_t layer, int32_t t0, int32_t Tq, con
         if (!decode_window_supported(dims->dtype, dims->d_head))
             return LLA_ERR_UNSUPPORTED;
     }
-    const Plan plan = make_plan(dims, B, Tq, max_ctx, num_splits, variant, window != nullptr);
+    const Plan plan = make_plan(dims, B, Tq, max_ctx, num_splits, variant, window != nullptr,
+                                dec != nullptr ? dec->d_rope : 0);
     if (workspace == nullptr || ws_bytes < plan.bytes)
         return LLA_ERR_WORKSPACE;
     if (!aligned16(workspace))
@@ -381,6 +390,13 @@ int decode_call(const lla_dims *dims, int32_t layer, int32_t t0, int32_t Tq, con
     a.q_pos = rope != nullptr ? rope->q_pos : nullptr;
     a.rope_base = rope != nullptr ? rope->base : 0.f;
     a.rope_style = rope != nullptr ? rope->style : 0;
+    a.k_rope = a.q_rope = nullptr;
+    a.d_rope = 0;
+    if (dec != nullptr) {
+        a.k_rope = static_cast<const uint8_t *>(dec->k_rope) + (int64_t)layer * Hs * cache->slots * dec->d_rope * e;
+        a.q_rope = dec->q_rope;
+        a.d_rope = dec->d_rope;
+    }
     if (window != nullptr) {
         // window planes [L][seqs][H][T][w_max][d]: select the layer
         const int64_t plane = (int64_t)window->seqs * dims->H * dims->T * window->w_max * dims->d_head * e;
@@ -502,6 +518,26 @@ int lla_decode_attn_hybrid(const lla_dims *dims, int32_t layer, int32_t t0, int3
         return LLA_ERR_INVALID;
     return decode_call(dims, layer, t0, Tq, q, cache, seq_start, ctx_lens, B, max_ctx, codec, window, nullptr,
                        softmax_scale, variant, num_splits, out, lse, workspace, ws_bytes, stream);
+}
+
+int lla_decode_attn_decoupled(const lla_dims *dims, int32_t layer, int32_t t0, int32_t Tq, const void *q,
+                              const lla_cache *cache, const int64_t *seq_start, const int32_t *ctx_lens, int32_t B,
+                              int32_t max_ctx, const lla_codec *codec, const lla_decoupled *dec,
+                              const lla_rope *rope, float softmax_scale, int32_t num_splits, void *out, float *lse,
+                              void *workspace, size_t ws_bytes, lla_stream_t stream)
+{
+    if (dec == nullptr || rope == nullptr)
+        return LLA_ERR_INVALID;
+    return decode_call(dims, layer, t0, Tq, q, cache, seq_start, ctx_lens, B, max_ctx, codec, nullptr, rope,
+                       softmax_scale, LLA_ABSORB, num_splits, out, lse, workspace, ws_bytes, stream, dec);
+}
+
+size_t lla_decode_decoupled_workspace_bytes(const lla_dims *dims, int32_t B, int32_t Tq, int32_t max_ctx,
+                                            int32_t d_rope, int32_t num_splits)
+{
+    if (d_rope <= 0 || lla_decode_num_splits(dims, B, Tq, max_ctx, LLA_ABSORB, num_splits) < 1)
+        return 0;
+    return make_plan(dims, B, Tq, max_ctx, num_splits, LLA_ABSORB, false, d_rope).bytes;
 }
 
 size_t lla_decode_hybrid_workspace_bytes(const lla_dims *dims, int32_t B, int32_t Tq, int32_t max_ctx,

@@ -265,6 +265,42 @@ int lla_decode_attn_rope(const lla_dims *dims, int32_t layer, int32_t t0, int32_
                          int32_t num_splits, void *out, float *lse, void *workspace,
                          size_t ws_bytes, lla_stream_t stream);
 
+/* ---- NEXT-4: absorbed read with a decoupled rotary sub-key ------------------------------
+ * Query absorption cannot carry a rotation (RoPE sits between the rebuilt key and the dot
+ * product), so the paper's absorbed variant keeps positional information in a decoupled
+ * rotary sub-key beside the latent (Pith verdict record, desk-editor letter; the paper
+ * reports a fidelity floor for it, which needs trained weights to measure).  Reading taken
+ * (multi-head latent attention's layout): each cached token keeps, per (layer, stored head),
+ * an exact sub-key k_rope of d_rope values, one for all loops, stored already rotated at the
+ * token's position; each loop query brings a rotary part q_rope of d_rope values, which the
+ * library rotates at q_pos (lla_rope conventions).  For loop t:
+ *   l_n = softmax_scale * (q . k_hat_n + rope(q_rope, q_pos) . k_rope[n]),
+ *   out = sum_n softmax(l)_n v_hat_n,
+ * with k_hat, v_hat as in lla_decode_attn and the q . k_hat term absorbed (q_tilde . c_K +
+ * scale * q . mu_t^K).  The tensor-core kernel streams the sub-key plane as a second key
+ * tile beside the latent tile: the score MMA runs over r_k + d_rope columns.
+ *   dec->k_rope  T [L][H][slots][d_rope]   (the latent cache's slots)
+ *   dec->q_rope  T [B][Tq][H][d_rope]
+ *   dec->d_rope  32 or 64
+ * Per-head layout, bf16, r_k = 16 and r_v = 32 only (LLA_ERR_UNSUPPORTED otherwise).  The
+ * workspace must hold lla_decode_decoupled_workspace_bytes(...) bytes; otherwise the
+ * arguments, errors and outputs are those of lla_decode_attn (variant LLA_ABSORB), plus
+ * `rope` (required: q_pos, base, style of the rotary part).                              */
+typedef struct {
+    const void *k_rope;
+    const void *q_rope;
+    int32_t d_rope;
+} lla_decoupled;
+int lla_decode_attn_decoupled(const lla_dims *dims, int32_t layer, int32_t t0, int32_t Tq,
+                              const void *q, const lla_cache *cache, const int64_t *seq_start,
+                              const int32_t *ctx_lens, int32_t B, int32_t max_ctx,
+                              const lla_codec *codec, const lla_decoupled *dec,
+                              const lla_rope *rope, float softmax_scale, int32_t num_splits,
+                              void *out, float *lse, void *workspace, size_t ws_bytes,
+                              lla_stream_t stream);
+size_t lla_decode_decoupled_workspace_bytes(const lla_dims *dims, int32_t B, int32_t Tq,
+                                            int32_t max_ctx, int32_t d_rope, int32_t num_splits);
+
 /* ---- decode attention with library-owned scratch ----------------------------------------
  * No counterpart in the paper: a deployment aid.  Some callers cannot allocate device
  * memory -- for example a plugin whose host framework owns the whole device memory pool

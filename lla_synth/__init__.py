@@ -28,6 +28,9 @@ whose weights are not available):
   values).  Queries q ~ N(0, 1) / sqrt(d).  Context lengths uniform inclusive.
 * Encode inputs: trajectory tokens laid out [n_tok][T][H][d] (loop-major, as a
   looped model produces them loop by loop).
+* Decoupled rotary sub-keys (LLA paper, Pith verdict record, desk-editor letter):
+  raw sub-keys N(0, 1) per (layer, head, slot) and rotary query parts N(0, 1) / sqrt(d),
+  drawn here unrotated; the tests rotate the stored sub-keys at their positions.
 * Hybrid-window inputs ("Hybrid Latent Attention for Looped Language Models",
   abstract: exact keys and values of the most recent tokens): fresh trajectory
   tokens of the same model, drawn as encode inputs and laid out per window row,
@@ -408,3 +411,19 @@ def window_inputs(w: Workload, layers, B: int, w_max: int, device, win_lens=None
             # [B*w_max, T, H, d] -> [B, H, T, w_max, d]
             out[name][layer].copy_(tok.view(B, w_max, w.T, w.H, w.d).permute(0, 3, 2, 1, 4))
     return out
+
+
+# ---------------------------------------------------------------------------
+# Decoupled rotary sub-keys beside the latents (drawn unrotated)
+# ---------------------------------------------------------------------------
+def rope_subkeys(w: Workload, layer: int, n_slots: int, d_rope: int, device) -> torch.Tensor:
+    """Raw sub-keys [H', n_slots, d_rope], N(0, 1), float32."""
+    g = _gen(device, seed_of(w.name, layer, "k_rope", d_rope))
+    return torch.randn(w.heads_stored, n_slots, d_rope, generator=g, device=device, dtype=torch.float32)
+
+
+def rope_queries(w: Workload, B: int, Tq: int, d_rope: int, device) -> torch.Tensor:
+    """Rotary query parts [B, Tq, H, d_rope], N(0, 1) / sqrt(d), in the storage type."""
+    g = _gen(device, seed_of(w.name, "q_rope", B, Tq, d_rope))
+    q = torch.randn(B, Tq, w.H, d_rope, generator=g, device=device, dtype=torch.float32)
+    return (q / math.sqrt(w.d)).to(w.torch_dtype)

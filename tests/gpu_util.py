@@ -91,6 +91,57 @@ def run_decode_rope(p, w, layer, t0, Tq, scale, q_pos, base, style, num_splits=0
     return out, lse, status
 
 
+def rotate_pairs(x, pos, base, style):
+    """Rotary map in RoFormer's complex form, fp64 numpy, in the real layout of ``style``."""
+    x = np.asarray(x, dtype=np.float64)
+    dr = x.shape[-1]
+    theta = base ** (-2.0 * np.arange(dr // 2) / dr)
+    ang = np.asarray(pos, dtype=np.float64)[..., None] * theta
+    if style == lla.ROPE_HALF:
+        a, b = x[..., :dr // 2], x[..., dr // 2:]
+    else:
+        a, b = x[..., 0::2], x[..., 1::2]
+    z = (a + 1j * b) * np.exp(1j * ang)
+    out = np.empty_like(x)
+    if style == lla.ROPE_HALF:
+        out[..., :dr // 2], out[..., dr // 2:] = z.real, z.imag
+    else:
+        out[..., 0::2], out[..., 1::2] = z.real, z.imag
+    return out
+
+
+def stored_subkeys(raw, starts, lens, base, style, dtype):
+    """Sub-key plane as the cache stores it: slot seq_start[b] + n rotated at position n."""
+    raw = np.asarray(raw, dtype=np.float64)         # [H', slots, d_r]
+    pos = np.zeros(raw.shape[1])
+    for s0, n in zip(starts, lens):
+        pos[int(s0):int(s0) + int(n)] = np.arange(int(n))
+    rot = rotate_pairs(raw, pos[None, :], base, style)
+    return torch.as_tensor(rot, dtype=torch.float32).to(dtype)
+
+
+def run_decode_decoupled(p, w, layer, t0, Tq, scale, k_rope, q_rope, q_pos, base, style, num_splits=0,
+                         out_dtype=lla.F32):
+    """Decoupled-RoPE absorbed decode through the C ABI; k_rope [L][H][slots][d_r] on the device."""
+    dims = dims_of(w, out_dtype)
+    B = len(p["lens"])
+    d_r = k_rope.shape[-1]
+    max_ctx = int(p["lens"].max()) if B else 0
+    ws_bytes = lla.decode_decoupled_workspace_bytes(dims, B, Tq, max_ctx, d_r, num_splits)
+    ws = torch.zeros(ws_bytes, dtype=torch.uint8, device="cuda")
+    odt = torch.float32 if out_dtype == lla.F32 else torch.bfloat16
+    out = torch.full((B, Tq, w.H, w.d), float("nan"), dtype=odt, device="cuda")
+    lse = torch.full((B, Tq, w.H), float("nan"), dtype=torch.float32, device="cuda")
+    qp = torch.as_tensor(np.asarray(q_pos, dtype=np.int32), device="cuda")
+    lla.decode_attn_decoupled(dims, layer, t0, Tq, p["q"], lla.make_cache(p["k"], p["v"], p["slots"]),
+                              p["seq_start"], p["ctx_lens"], B, max_ctx, codec_of(p), k_rope, q_rope, d_r,
+                              lla.make_rope(qp, base, style), scale, out, lse, ws, ws_bytes,
+                              num_splits=num_splits)
+    torch.cuda.synchronize()
+    status = lla.status_fetch(ws)
+    return out, lse, status
+
+
 def run_decode_hybrid(p, win, w, layer, t0, Tq, scale, num_splits=0, variant=lla.ABSORB, q=None,
                       out_dtype=lla.F32):
     """Hybrid decode through the C ABI; returns (out, lse, device status)."""
@@ -140,7 +191,7 @@ def assert_attn_close(out_gpu, lse_gpu, o_ref, lse_ref):
 
 
 def oracle_decode_units(p, w, layer, t0, Tq, scale, units, variant="absorb", q=None, threads=None,
-                        win=None, rope=None):
+                        win=None, rope=None, decoupled=None):
     """Oracle on sampled (b, h) units only: their latent rows are gathered to the host.
 
     Works for caches far larger than host memory; the result arrays are NaN outside
@@ -167,6 +218,10 @@ def oracle_decode_units(p, w, layer, t0, Tq, scale, units, variant="absorb", q=N
             window = (to64(win["win_k"][layer, b:b + 1, hsel, :, :nw]),
                       to64(win["win_v"][layer, b:b + 1, hsel, :, :nw]), [nw])
         rope_b = None if rope is None else ([rope[0][b]], rope[1], rope[2])
+        dec_b = None
+        if decoupled is not None:  # (k_rope plane [H', slots, d_r] of the layer, q_rope, q_pos, base, style)
+            kr, qr, qpos, base_, style_ = decoupled
+            dec_b = (to64(kr[hp:hp + 1, s0:s0 + n]), to64(qr[b:b + 1, :, h:h + 1]), [qpos[b]], base_, style_)
         if w.fold2d:
             ob, lb = oracle.decode_layer(variant, q64[b:b + 1], cK, cV, [0], [n], WK, mK, WV, mV, t0, scale,
                                          fold2d=True, units=[(0, h)], threads=1, window=window,
@@ -175,7 +230,7 @@ def oracle_decode_units(p, w, layer, t0, Tq, scale, units, variant="absorb", q=N
             sel = [h]
             ob, lb = oracle.decode_layer(variant, q64[b:b + 1, :, sel], cK, cV, [0], [n], WK[sel], mK[sel],
                                          WV[sel], mV[sel], t0, scale, fold2d=False, threads=1,
-                                         window=window, rope=rope_b)
+                                         window=window, rope=rope_b, decoupled=dec_b)
             o[b, :, h] = ob[0, :, 0]
             lse[b, :, h] = lb[0, :, 0]
             continue

@@ -215,6 +215,30 @@ def test_codec_residual_argument_errors():
     assert rc(n_tok=0) == 0 and rc(n_layers=0) == 0
 
 
+def test_decoupled_argument_errors():
+    def rc(d_rope=64, k_rope=FAKE, q_rope=FAKE, rope=None, **over):
+        a = _decode_args(**over)
+        a.pop("variant")
+        rope = rope if rope is not None else lla.make_rope(FAKE, 10000.0, lla.ROPE_HALF)
+        try:
+            lla.decode_attn_decoupled(k_rope=k_rope, q_rope=q_rope, d_rope=d_rope, rope=rope, **a)
+        except lla.LLAError as e:
+            return e.code
+        return 0
+
+    assert rc(layer=1) == lla.LLA_ERR_INVALID
+    assert rc(k_rope=0) == lla.LLA_ERR_INVALID
+    assert rc(d_rope=0) == lla.LLA_ERR_INVALID
+    assert rc(q_rope=FAKE + 2) == lla.LLA_ERR_MISALIGNED
+    assert rc(d_rope=48) == lla.LLA_ERR_UNSUPPORTED
+    assert rc(dims=lla.make_dims(4, 1, 16, 128, 32, 32)) == lla.LLA_ERR_UNSUPPORTED
+    assert rc(rope=lla.make_rope(0, 10000.0, lla.ROPE_HALF)) == lla.LLA_ERR_INVALID
+    assert rc(B=0) == 0
+    dims = lla.make_dims(4, 1, 16, 128, 16, 32)
+    base = lla.decode_workspace_bytes(dims, 64, 4, 4096)
+    assert lla.decode_decoupled_workspace_bytes(dims, 64, 4, 4096, 64) >= base + 64 * 16 * 4 * 64 * 4
+
+
 def test_hybrid_workspace_adds_one_window_record_per_query():
     dims = lla.make_dims(4, 1, 16, 128, 16, 32)
     base = lla.decode_workspace_bytes(dims, 64, 4, 4096)
