@@ -67,6 +67,9 @@ def parse():
     ap.add_argument("--rope", action="store_true",
                     help="faithful read: rotary embedding after reconstruction (reconstruct form, "
                          "query positions = context lengths, half-split pairs, base 10000)")
+    ap.add_argument("--decoupled", type=int, default=0,
+                    help="absorbed read with a decoupled rotary sub-key of this width (32 or 64) beside "
+                         "each latent; queries placed after their contexts")
     ap.add_argument("--window", type=int, default=0,
                     help="hybrid form: W exact window rows per sequence (all in use) besides the "
                          "latents; 0 = latents only")
@@ -451,20 +454,38 @@ def main():
     # order one call per loop (t0 = t, Tq = 1) with each loop's queries and outputs in
     # buffers of their own
     calls = [(t, 1) for t in range(w.T)] if args.model_order else [(0, w.T)]
+    # decoupled rotary sub-key planes (drawn unrotated: rotation does not change the timing)
+    DRn = max(0, args.decoupled)
+    if DRn:
+        rope = lla.make_rope(p["ctx_lens"].clone(), 10000.0, lla.ROPE_HALF)
+        kr0 = S.rope_subkeys(w, 0, p["slots"], DRn, dev).to(w.torch_dtype).unsqueeze(0)
+        k_ropes = [kr0] + [kr0.clone() for _ in range(R - 1)]
+        q_rope = S.rope_queries(w, B, w.T, DRn, dev)
+        q_ropes = [q_rope[:, t0:t0 + n].contiguous() for t0, n in calls]
     Tq_call = calls[0][1]
     q_full = p["q"]
     qs = [q_full[:, t0:t0 + n].contiguous() for t0, n in calls]
     outs = [torch.empty(B, n, H, w.d, dtype=torch.float32, device=dev) for _, n in calls]
     lses = [torch.empty(B, n, H, dtype=torch.float32, device=dev) for _, n in calls]
     q, out, lse = q_full, outs[0], lses[0]
-    ws_fn = lla.decode_hybrid_workspace_bytes if Wn else lla.decode_workspace_bytes
-    ws_bytes = ws_fn(dims, B, Tq_call, max_ctx, variant, args.num_splits)
+    if DRn:
+        ws_bytes = lla.decode_decoupled_workspace_bytes(dims, B, Tq_call, max_ctx, DRn, args.num_splits)
+    else:
+        ws_fn = lla.decode_hybrid_workspace_bytes if Wn else lla.decode_workspace_bytes
+        ws_bytes = ws_fn(dims, B, Tq_call, max_ctx, variant, args.num_splits)
     ws = torch.zeros(ws_bytes, dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream(dev)
     splits = lla.decode_num_splits(dims, B, Tq_call, max_ctx, variant, args.num_splits)
 
     def decode(i, q_in=None, out_buf=None, lse_buf=None):
         for c, (t0, n) in enumerate(calls):
+            if DRn:
+                lla.decode_attn_decoupled(dims, 0, t0, n, (q_in or qs)[c], caches[i % R], p["seq_start"],
+                                          p["ctx_lens"], B, max_ctx, codec, k_ropes[i % R],
+                                          q_ropes[c], DRn,
+                                          rope, 1.0, (out_buf or outs)[c], (lse_buf or lses)[c], ws, ws_bytes,
+                                          num_splits=args.num_splits, stream=stream)
+                continue
             if rope is not None:
                 lla.decode_attn_rope(dims, 0, t0, n, (q_in or qs)[c], caches[i % R], p["seq_start"],
                                      p["ctx_lens"], B, max_ctx, codec, rope, 1.0, (out_buf or outs)[c],
@@ -525,6 +546,8 @@ def main():
     # hybrid form: each loop query also reads its own loop's exact window keys and values once
     win_bytes = B * H * Tq * Wn * w.d * 2 * w.elem_bytes
     step_bytes += win_bytes
+    # decoupled form: each call also reads every token's rotary sub-key once
+    step_bytes += len(calls) * S_tot * w.heads_stored * DRn * w.elem_bytes
     ms_step = ms_total / args.steps
     value = world * step_bytes / (ms_step * 1e-3) / 1e9
     reads = world * S_tot * Tq / (ms_step * 1e-3)       # (token, layer, loop) reads per second
@@ -631,7 +654,7 @@ def main():
         return
 
     cpu = None
-    if world == 1 and not args.no_cpu_baseline and not Wn and not args.rope:
+    if world == 1 and not args.no_cpu_baseline and not Wn and not args.rope and not DRn:
         rate, info = oracle_sample_rate(p, w, Tq, args.cpu_seconds, units_per_round=max(1, B * H // 8))
         cpu = {"value": rate, "unit": "GB/s", "cores": info["cores"], "kind": "oracle",
                "sample": f"{info['rounds']} rounds of {info['units']} (sequence, head) units x "
@@ -644,11 +667,13 @@ def main():
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": "f32", "storage_dtype": w.dtype, "data": "synthetic",
-        "config": {"workload": w.name + (f"+window{Wn}" if Wn else ""), "T": w.T, "L_per_step": 1,
+        "config": {"workload": w.name + (f"+window{Wn}" if Wn else "") + (f"+ropekey{DRn}" if DRn else ""),
+                   "T": w.T, "L_per_step": 1,
                    "H": H, "d": w.d, "window_rows": Wn, "window_bytes_per_step": win_bytes,
                    "r_k": w.r_k, "r_v": w.r_v, "rho": "64/3", "B": B,
                    "ctx_len": [w.len_lo, w.len_hi], "tokens": S_tot, "Tq": Tq_call, "decode_calls_per_step": len(calls),
-                   "variant": args.variant + (" + rope" if args.rope else ""), "seg_max": splits,
+                   "variant": args.variant + (" + rope" if args.rope else "")
+                              + (f" + decoupled rotary sub-key {DRn}" if DRn else ""), "seg_max": splits,
                    "step": (f"{len(calls)} x decode_attn(Tq = 1, one loop each, model order)"
                             if args.model_order else f"decode_attn(all {w.T} loop queries fused)")
                            + (f" with {Wn} exact window rows per sequence (decode_attn_hybrid)" if Wn else "")
