@@ -379,24 +379,26 @@ __device__ __forceinline__ void stage_f32(float *dst, int dst_ld, const float *s
     }
 }
 
-constexpr int kBatchSeqs = 8;
+constexpr int kBatchSeqs = 8;    // sequences per combine CTA (one warp each)
+constexpr int kPrologueSeqs = 8; // sequences per prologue CTA
 constexpr int kPrologueThreads = 128;
 
-template <typename T>
+// ROPEQ: also append the rotated rotary query part (decoupled sub-key form).
+template <typename T, bool ROPEQ>
 __global__ void __launch_bounds__(kPrologueThreads) absorb_prologue_kernel(const DecodeArgs a)
 {
     extern __shared__ float psm[];
     grid_launch_dependents(); // the decode grid may start streaming latents right away
-    const int h = blockIdx.x, t = blockIdx.y, b0 = blockIdx.z * kBatchSeqs;
+    const int h = blockIdx.x, t = blockIdx.y, b0 = blockIdx.z * kPrologueSeqs;
     const int RK = a.r_k, d = a.d, ldw = d + 1;
     float *W = psm;                       // [RK][d + 1]
-    float *qs = W + RK * ldw;             // [kBatchSeqs][d]
+    float *qs = W + RK * ldw;             // [kPrologueSeqs][d]
     const int tg = a.t0 + a.tq_off + t;
     const int ld = a.fold ? a.H * d : d;
     const float *wsrc = a.W_up_k + (a.fold ? (int64_t)tg * RK * ld + (int64_t)h * d
                                            : ((int64_t)h * a.T + tg) * RK * ld);
     stage_f32<kPrologueThreads>(W, ldw, wsrc, ld, RK, d);
-    const int nb = min(kBatchSeqs, a.B - b0);
+    const int nb = min(kPrologueSeqs, a.B - b0);
     {
         // query rows of the chunk, 16-byte loads (8 bf16 or 4 fp32), all issued first
         constexpr int V = 16 / (int)sizeof(T);
@@ -440,7 +442,7 @@ __global__ void __launch_bounds__(kPrologueThreads) absorb_prologue_kernel(const
         const int64_t u = (int64_t)(b0 + bl) * a.H + h;
         a.qt[(u * a.Tq_all + a.tq_off + t) * (RK + a.d_rope) + j] = ((s0 + s1) + (s2 + s3)) * a.scale * kLog2e;
     }
-    if (a.d_rope > 0) {
+    if (ROPEQ) {
         // decoupled rotary part: q_rope rotated at the query position, appended to q_tilde;
         // pair i (i, i + d_r/2 or 2i, 2i+1) turns by q_pos * base^(-2i/d_r), angle in fp64
         const int dr = a.d_rope, np = dr / 2;
@@ -744,16 +746,16 @@ cudaError_t launch_decode_absorb(const DecodeArgs &a, int dtype, int ctas, cudaS
 
 cudaError_t launch_absorb_prologue(const DecodeArgs &a, int dtype, cudaStream_t stream)
 {
-    dim3 grid(a.H, a.Tq, (a.B + kBatchSeqs - 1) / kBatchSeqs);
-    const size_t smem = sizeof(float) * ((size_t)a.r_k * (a.d + 1) + (size_t)kBatchSeqs * a.d);
+    dim3 grid(a.H, a.Tq, (a.B + kPrologueSeqs - 1) / kPrologueSeqs);
+    const size_t smem = sizeof(float) * ((size_t)a.r_k * (a.d + 1) + (size_t)kPrologueSeqs * a.d);
     if (smem > 200 * 1024)
         return cudaErrorInvalidValue;
     if (dtype == LLA_BF16) {
-        auto k = absorb_prologue_kernel<__nv_bfloat16>;
+        auto k = a.d_rope > 0 ? absorb_prologue_kernel<__nv_bfloat16, true> : absorb_prologue_kernel<__nv_bfloat16, false>;
         cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
         k<<<grid, kPrologueThreads, smem, stream>>>(a);
     } else {
-        auto k = absorb_prologue_kernel<float>;
+        auto k = a.d_rope > 0 ? absorb_prologue_kernel<float, true> : absorb_prologue_kernel<float, false>;
         cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
         k<<<grid, kPrologueThreads, smem, stream>>>(a);
     }
