@@ -44,7 +44,7 @@ ROPE_HALF, ROPE_INTERLEAVED = 0, 1
 EXPORTED = ("lla_cache_bytes", "lla_slot_layout", "lla_codec_bias", "lla_encode",
             "lla_decode_attn", "lla_decode_workspace_bytes", "lla_decode_num_splits",
             "lla_decode_attn_static", "lla_decode_attn_hybrid", "lla_decode_hybrid_workspace_bytes",
-            "lla_decode_attn_rope", "lla_codec_residual", "lla_decode_attn_decoupled",
+            "lla_decode_attn_rope", "lla_codec_residual", "lla_decode_attn_decoupled", "lla_decode_attn_timed",
             "lla_decode_decoupled_workspace_bytes",
             "lla_status_fetch", "lla_status_string")
 STATIC_SCRATCH_BYTES = 8 << 20
@@ -91,6 +91,8 @@ _lib.lla_decode_attn_static.argtypes = [_P(Dims), _i32, _i32, _i32, _vp, _P(Cach
 _lib.lla_decode_attn_hybrid.argtypes = [_P(Dims), _i32, _i32, _i32, _vp, _P(Cache), _vp, _vp, _i32,
                                         _i32, _P(Codec), _P(Window), ctypes.c_float, _i32, _i32, _vp,
                                         _vp, _vp, _sz, _vp]
+_lib.lla_decode_attn_timed.argtypes = [_P(Dims), _i32, _i32, _i32, _vp, _P(Cache), _vp, _vp, _i32, _i32,
+                                       _P(Codec), ctypes.c_float, _i32, _i32, _vp, _vp, _vp, _sz, _vp, _vp, _vp]
 _lib.lla_decode_attn_decoupled.argtypes = [_P(Dims), _i32, _i32, _i32, _vp, _P(Cache), _vp, _vp, _i32, _i32,
                                            _P(Codec), _P(Decoupled), _P(Rope), ctypes.c_float, _i32, _vp, _vp,
                                            _vp, _sz, _vp]
@@ -109,7 +111,7 @@ _lib.lla_status_string.argtypes = [ctypes.c_int]
 _lib.lla_status_string.restype = ctypes.c_char_p
 for _n in ("lla_cache_bytes", "lla_slot_layout", "lla_codec_bias", "lla_encode", "lla_decode_attn",
            "lla_decode_attn_static", "lla_decode_attn_hybrid", "lla_decode_attn_rope", "lla_codec_residual",
-           "lla_decode_attn_decoupled",
+           "lla_decode_attn_decoupled", "lla_decode_attn_timed",
            "lla_decode_num_splits",
            "lla_status_fetch"):
     getattr(_lib, _n).restype = ctypes.c_int
@@ -300,6 +302,20 @@ def decode_attn_decoupled(dims: Dims, layer: int, t0: int, Tq: int, q, cache: Ca
                                           num_splits, _ptr(out), _ptr(lse), _ptr(workspace), int(ws_bytes),
                                           _stream(stream)),
            "lla_decode_attn_decoupled")
+
+
+def decode_attn_timed(dims: Dims, layer: int, t0: int, Tq: int, q, cache: Cache, seq_start, ctx_lens,
+                      B: int, max_ctx: int, codec: Codec, softmax_scale: float, out, lse, workspace,
+                      ws_bytes: int, ev_start, ev_end, variant: int = ABSORB, num_splits: int = 0,
+                      stream=None) -> None:
+    """lla_decode_attn with CUDA events around the latent-streaming grid alone (timing aid).
+    ev_start / ev_end: torch.cuda.Event(enable_timing=True), already created (recorded once)."""
+    _check(_lib.lla_decode_attn_timed(ctypes.byref(dims), layer, t0, Tq, _ptr(q), ctypes.byref(cache),
+                                      _ptr(seq_start), _ptr(ctx_lens), B, max_ctx, ctypes.byref(codec),
+                                      float(softmax_scale), variant, num_splits, _ptr(out), _ptr(lse),
+                                      _ptr(workspace), int(ws_bytes), _stream(stream), ev_start.cuda_event,
+                                      ev_end.cuda_event),
+           "lla_decode_attn_timed")
 
 
 def decode_attn_static(dims: Dims, layer: int, t0: int, Tq: int, q, cache: Cache, seq_start,

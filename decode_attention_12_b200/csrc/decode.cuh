@@ -45,6 +45,7 @@ struct DecodeArgs {
     const void *k_rope;       // T [H'][slots][d_rope], stored rotated at each token's position
     const void *q_rope;       // T [B][Tq_all][H][d_rope], rotated at q_pos by the prologue
     int32_t d_rope;           // 0: none; q_tilde rows then hold r_k + d_rope values
+    int32_t serial;           // launch every grid without programmatic overlap (timing aid)
 };
 
 constexpr float kLog2e = 1.4426950408889634f;

@@ -450,7 +450,7 @@ cudaError_t launch_mma_t(const DecodeArgs &a, int ctas, cudaStream_t stream)
     cfg.stream = stream;
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization; // overlap the prologue's tail
-    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    attr[0].val.programmaticStreamSerializationAllowed = a.serial ? 0 : 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
     if constexpr (DR > 0)

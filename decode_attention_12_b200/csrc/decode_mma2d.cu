@@ -400,7 +400,7 @@ cudaError_t launch_2d_t(const DecodeArgs &a, cudaStream_t stream)
     cfg.stream = stream;
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization; // overlap the prologue
-    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    attr[0].val.programmaticStreamSerializationAllowed = a.serial ? 0 : 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
     return cudaLaunchKernelEx(&cfg, kern, mk, mkt, mv, mvt, a);

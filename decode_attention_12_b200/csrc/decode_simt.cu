@@ -778,7 +778,7 @@ static cudaError_t launch_combine_t(const DecodeArgs &a, size_t smem, cudaStream
     cfg.stream = stream;
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization; // stage W_up while decode ends
-    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    attr[0].val.programmaticStreamSerializationAllowed = a.serial ? 0 : 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
     return cudaLaunchKernelEx(&cfg, k, a);

@@ -225,7 +225,7 @@ cudaError_t launch_window_t(const DecodeArgs &a, cudaStream_t stream)
     cfg.stream = stream;
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization; // fill the decode's tail
-    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    attr[0].val.programmaticStreamSerializationAllowed = a.serial ? 0 : 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
     return cudaLaunchKernelEx(&cfg, decode_window_kernel<T, LPR>, a);

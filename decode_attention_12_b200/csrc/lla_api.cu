@@ -296,7 +296,8 @@ int decode_call(const lla_dims *dims, int32_t layer, int32_t t0, int32_t Tq, con
                 const lla_cache *cache, const int64_t *seq_start, const int32_t *ctx_lens, int32_t B,
                 int32_t max_ctx, const lla_codec *codec, const lla_window *window, const lla_rope *rope,
                 float softmax_scale, int32_t variant, int32_t num_splits, void *out, float *lse,
-                void *workspace, size_t ws_bytes, lla_stream_t stream, const lla_decoupled *dec = nullptr)
+                void *workspace, size_t ws_bytes, lla_stream_t stream, const lla_decoupled *dec = nullptr,
+                lla_event_t ev_start = nullptr, lla_event_t ev_end = nullptr)
 {
     int rc = check_dims(dims);
     if (rc != LLA_OK)
@@ -392,6 +393,10 @@ int decode_call(const lla_dims *dims, int32_t layer, int32_t t0, int32_t Tq, con
     a.rope_style = rope != nullptr ? rope->style : 0;
     a.k_rope = a.q_rope = nullptr;
     a.d_rope = 0;
+    // timing aid: events around the latent-streaming grid, every grid launched in order
+    a.serial = ev_start != nullptr || ev_end != nullptr;
+    cudaEvent_t e0 = reinterpret_cast<cudaEvent_t>(ev_start), e1 = reinterpret_cast<cudaEvent_t>(ev_end);
+    auto mark = [&](cudaEvent_t ev) -> cudaError_t { return ev != nullptr ? cudaEventRecord(ev, (cudaStream_t)stream) : cudaSuccess; };
     if (dec != nullptr) {
         a.k_rope = static_cast<const uint8_t *>(dec->k_rope) + (int64_t)layer * Hs * cache->slots * dec->d_rope * e;
         a.q_rope = dec->q_rope;
@@ -421,7 +426,11 @@ int decode_call(const lla_dims *dims, int32_t layer, int32_t t0, int32_t Tq, con
             DecodeArgs ac = a;
             ac.tq_off = c;
             ac.Tq = 1;
-            err = launch_decode_reconstruct(ac, s);
+            err = mark(c == 0 ? e0 : nullptr);
+            if (err == cudaSuccess)
+                err = launch_decode_reconstruct(ac, s);
+            if (err == cudaSuccess && c == Tq - 1)
+                err = mark(e1);
         }
         if (err == cudaSuccess)
             err = window_pass(a);
@@ -438,8 +447,12 @@ int decode_call(const lla_dims *dims, int32_t layer, int32_t t0, int32_t Tq, con
             ac.tq_off = c;
             ac.Tq = Tq - c < per ? Tq - c : per;
             err = launch_absorb_prologue(ac, dims->dtype, s);
+            if (err == cudaSuccess && c == 0)
+                err = mark(e0);
             if (err == cudaSuccess)
                 err = launch_decode_absorb_2d(ac, s);
+            if (err == cudaSuccess && c + per >= Tq)
+                err = mark(e1);
             if (err == cudaSuccess)
                 err = window_pass(ac);
             if (err == cudaSuccess)
@@ -454,8 +467,12 @@ int decode_call(const lla_dims *dims, int32_t layer, int32_t t0, int32_t Tq, con
             ac.tq_off = c;
             ac.Tq = Tq - c < 16 ? Tq - c : 16;
             err = launch_absorb_prologue(ac, dims->dtype, s);
+            if (err == cudaSuccess && c == 0)
+                err = mark(e0);
             if (err == cudaSuccess)
                 err = launch_decode_absorb_mma(ac, 0, s);
+            if (err == cudaSuccess && c + 16 >= Tq)
+                err = mark(e1);
             if (err == cudaSuccess)
                 err = window_pass(ac);
             if (err == cudaSuccess)
@@ -470,8 +487,12 @@ int decode_call(const lla_dims *dims, int32_t layer, int32_t t0, int32_t Tq, con
         ac.Tq = Tq - c < 4 ? Tq - c : 4;
         err = launch_absorb_prologue(ac, dims->dtype, s);
         bool supported = false;
+        if (err == cudaSuccess && c == 0)
+            err = mark(e0);
         if (err == cudaSuccess)
             err = launch_decode_absorb(ac, dims->dtype, 0, s, &supported);
+        if (err == cudaSuccess && c + 4 >= Tq)
+            err = mark(e1);
         if (!supported)
             return LLA_ERR_UNSUPPORTED;
         if (err == cudaSuccess)
@@ -506,6 +527,19 @@ int lla_decode_attn_rope(const lla_dims *dims, int32_t layer, int32_t t0, int32_
         return LLA_ERR_INVALID;
     return decode_call(dims, layer, t0, Tq, q, cache, seq_start, ctx_lens, B, max_ctx, codec, nullptr, rope,
                        softmax_scale, LLA_RECONSTRUCT, num_splits, out, lse, workspace, ws_bytes, stream);
+}
+
+int lla_decode_attn_timed(const lla_dims *dims, int32_t layer, int32_t t0, int32_t Tq, const void *q,
+                          const lla_cache *cache, const int64_t *seq_start, const int32_t *ctx_lens, int32_t B,
+                          int32_t max_ctx, const lla_codec *codec, float softmax_scale, int32_t variant,
+                          int32_t num_splits, void *out, float *lse, void *workspace, size_t ws_bytes,
+                          lla_stream_t stream, lla_event_t ev_start, lla_event_t ev_end)
+{
+    if (ev_start == nullptr || ev_end == nullptr)
+        return LLA_ERR_INVALID;
+    return decode_call(dims, layer, t0, Tq, q, cache, seq_start, ctx_lens, B, max_ctx, codec, nullptr, nullptr,
+                       softmax_scale, variant, num_splits, out, lse, workspace, ws_bytes, stream, nullptr, ev_start,
+                       ev_end);
 }
 
 int lla_decode_attn_hybrid(const lla_dims *dims, int32_t layer, int32_t t0, int32_t Tq, const void *q,

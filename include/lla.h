@@ -41,6 +41,7 @@ extern "C" {
 #endif
 
 typedef struct CUstream_st *lla_stream_t; /* same type as cudaStream_t; NULL = legacy stream */
+typedef struct CUevent_st *lla_event_t;   /* same type as cudaEvent_t                         */
 
 /* ---- status codes ---------------------------------------------------------------- */
 #define LLA_OK 0
@@ -184,6 +185,20 @@ int lla_decode_attn(const lla_dims *dims, int32_t layer, int32_t t0, int32_t Tq,
                     const lla_codec *codec, float softmax_scale, int32_t variant,
                     int32_t num_splits, void *out, float *lse, void *workspace,
                     size_t ws_bytes, lla_stream_t stream);
+
+/* Timing aid (no counterpart in the paper): exactly lla_decode_attn, but ev_start is
+ * recorded on `stream` immediately before the latent-streaming decode grid and ev_end
+ * immediately after it (for Tq above one pass: before the first and after the last), and
+ * every grid of the call is launched without programmatic overlap, so that
+ * cudaEventElapsedTime(ev_start, ev_end) is that grid's own duration.  Both events are
+ * required (LLA_ERR_INVALID otherwise).                                                 */
+int lla_decode_attn_timed(const lla_dims *dims, int32_t layer, int32_t t0, int32_t Tq,
+                          const void *q, const lla_cache *cache, const int64_t *seq_start,
+                          const int32_t *ctx_lens, int32_t B, int32_t max_ctx,
+                          const lla_codec *codec, float softmax_scale, int32_t variant,
+                          int32_t num_splits, void *out, float *lse, void *workspace,
+                          size_t ws_bytes, lla_stream_t stream, lla_event_t ev_start,
+                          lla_event_t ev_end);
 
 /* Workspace bytes lla_decode_attn needs for these sizes (num_splits as passed to it;
  * 0 = the automatic choice for max_ctx).  Returns 0 for invalid arguments.          */

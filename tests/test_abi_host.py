@@ -247,6 +247,14 @@ def test_hybrid_workspace_adds_one_window_record_per_query():
     assert hyb - base < 64 * 16 * 4 * (128 + 4) * 4 + 256
 
 
+def test_timed_entry_needs_both_events():
+    a = _decode_args()
+    rc = lla._lib.lla_decode_attn_timed(ctypes.byref(a["dims"]), 0, 0, 4, FAKE, ctypes.byref(a["cache"]), FAKE,
+                                        FAKE, 2, 100, ctypes.byref(a["codec"]), 1.0, 0, 0, FAKE, None, FAKE,
+                                        1 << 30, None, None, FAKE)
+    assert rc == lla.LLA_ERR_INVALID
+
+
 def test_workspace_bytes_and_splits():
     dims = lla.make_dims(4, 1, 16, 128, 16, 32)
     s = lla.decode_num_splits(dims, 64, 4, 4096)

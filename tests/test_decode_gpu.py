@@ -161,3 +161,32 @@ def test_bf16_output_storage(ouro):
     m = ~np.isnan(o_ref)
     bound = np.abs(o_ref[m]) * 2.0 ** -8 + 5e-3
     assert np.all(np.abs(o[m] - o_ref[m]) <= bound)
+
+
+def test_timed_entry_matches_decode_and_times_the_grid():
+    """lla_decode_attn_timed: the same results, bit for bit, and a positive event interval
+    around the decode grid that is shorter than the whole call."""
+    import torch
+    w = S.shrink(S.WORKLOADS["ouro1.4b-layer"], name="timed", B=8, len_lo=500, len_hi=3000)
+    p = S.decode_inputs(w, 0, "cuda")
+    out, lse, st = run_decode(p, w, 0, 0, 4, 1.0)
+    assert st == 0
+    dims = dims_of(w)
+    B, max_ctx = w.B, int(p["lens"].max())
+    wsb = lla.decode_workspace_bytes(dims, B, 4, max_ctx)
+    ws = torch.zeros(wsb, dtype=torch.uint8, device="cuda")
+    out2 = torch.empty_like(out)
+    lse2 = torch.empty_like(lse)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    c0, c1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    for e in (e0, e1):
+        e.record()
+    torch.cuda.synchronize()
+    c0.record()
+    lla.decode_attn_timed(dims, 0, 0, 4, p["q"], lla.make_cache(p["k"], p["v"], p["slots"]), p["seq_start"],
+                          p["ctx_lens"], B, max_ctx, codec_of(p), 1.0, out2, lse2, ws, wsb, e0, e1)
+    c1.record()
+    torch.cuda.synchronize()
+    assert lla.status_fetch(ws) == 0
+    assert torch.equal(out2, out) and torch.equal(lse2, lse)
+    assert 0 < e0.elapsed_time(e1) < c0.elapsed_time(c1)
