@@ -80,7 +80,7 @@ def test_long_context_8x16k_full_layer():
     assert_attn_close(out, lse, o_ref, l_ref)
 
 
-LLA2D_EDGE_LENS = [0, 1, 31, 64, 65, 383, 384, 385, 1000, 4096]
+LLA2D_EDGE_LENS = [0, 1, 31, 64, 65, 255, 256, 257, 383, 384, 385, 1000, 4096]
 
 
 @pytest.mark.parametrize("Tq,t0", [(4, 0), (1, 3)])
