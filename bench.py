@@ -35,6 +35,7 @@ sys.path.insert(0, ROOT)
 METRIC = "LLA decode latent-cache GB/s & token-loop reads/s (% of HBM roofline) at 1 B200"
 WORKLOAD = "ouro1.4b-layer"
 SPEC_HBM_GBS = 8000.0
+L2_BYTES = 126 * 1000 * 1000
 PROFILE_TRAFFIC = {
     "absorb": os.path.join(ROOT, "profiles", "decode_absorb_mma.ouro1.4b-layer.json"),
     "reconstruct": os.path.join(ROOT, "profiles", "decode_reconstruct.ouro1.4b-layer.json"),
@@ -430,8 +431,11 @@ def main():
                            bias_v=p["bias_v"], W_up_k=p["W_up_k"], W_up_v=p["W_up_v"],
                            mu_k=p["mu_k"], mu_v=p["mu_v"])
     lla.codec_bias(dims, codec, p["bias_k"], p["bias_v"])
-    # independent cache replicas (rotated per step so that no step finds latents in L2)
-    R = max(1, args.replicas)
+    # independent cache replicas, rotated per step so that no step finds latents in L2: at
+    # least enough that the replicas together span twice the 126 MB L2 (small planes, such
+    # as the LLA-2D layer's 25 MB, need more than the default 3)
+    plane_bytes = (p["k"].numel() + p["v"].numel()) * p["k"].element_size()
+    R = max(1, args.replicas, math.ceil(2 * L2_BYTES / max(plane_bytes, 1)) if args.replicas > 1 else 1)
     reps = [(p["k"], p["v"])] + [(p["k"].clone(), p["v"].clone()) for _ in range(R - 1)]
     caches = [lla.make_cache(k, v, p["slots"]) for k, v in reps]
     # hybrid form: every sequence holds a full window of W exact rows (steady state)
@@ -712,8 +716,9 @@ def main():
                             if args.model_order else f"decode_attn(all {w.T} loop queries fused)")
                            + (f" with {Wn} exact window rows per sequence (decode_attn_hybrid)" if Wn else "")
                            + " + encode(B new tokens)",
-                   "l2": f"inputs larger than L2 ({step_bytes / 1e6:.0f} MB of latents per step) "
-                         f"and {R} rotating cache replicas",
+                   "l2": f"{R} rotating cache replicas of {plane_bytes / 1e6:.0f} MB "
+                         f"({R * plane_bytes / 1e6:.0f} MB together, L2 is 126 MB); "
+                         f"{step_bytes / 1e6:.0f} MB read per step",
                    "parallelism": f"replicas x{world}"},
         "token_loop_reads_per_s": reads,
         "hbm_frac_of_8tbs_spec": value / world / SPEC_HBM_GBS,
