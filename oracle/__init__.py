@@ -215,6 +215,32 @@ def attend_decoupled(c_K, c_V, W_up_K_t, mu_K_t, W_up_V_t, mu_V_t, k_rope, q, q_
     return o, float(lse.value)
 
 
+def codec_fit(x_cal, r, T):
+    """SVD initialisation of the codec from calibration tokens ("Looped Latent Attention",
+    review page, What carries the argument: the codec starts from the top right singular
+    vectors of the centred teacher activations).
+
+    x_cal [n, W] stacked vectors (W = T * Dp, loop-major), rank r ->
+    (mu [W], W_down [W, r], W_up [T, r, Dp], sigma [min(n, W)]):
+      mu = column mean; Y = x_cal - mu = U diag(sigma) V^T (numpy SVD, fp64);
+      W_down = V[:, :r], each column signed so that its largest-magnitude entry (the first
+      one on a tie) is positive; W_up,t = transpose of the loop-t row block of W_down.
+    """
+    x = _f64(x_cal)
+    n, W = x.shape
+    if W % T or not (0 < r <= min(n, W)):
+        raise ValueError("bad rank or width")
+    mu = x.mean(axis=0)
+    _, sigma, Vt = np.linalg.svd(x - mu[None, :], full_matrices=False)
+    W_down = Vt[:r].T.copy()
+    lead = np.argmax(np.abs(W_down), axis=0)
+    sign = np.sign(W_down[lead, np.arange(r)])
+    sign[sign == 0] = 1.0
+    W_down *= sign[None, :]
+    W_up = W_down.reshape(T, W // T, r).transpose(0, 2, 1).copy()
+    return mu, W_down, W_up, sigma
+
+
 def codec_residual(x, mu, W_down, W_up):
     """Per-token reconstruction residual of a codec.
 

@@ -132,3 +132,39 @@ def test_mutant_is_caught(name, tmp_path):
     finally:
         oracle._lib = saved
     assert failed, f"mutant {name} survived every pin"
+
+
+# Mutants of the numpy-level codec fit: the function's source is edited, compiled in the
+# oracle module's namespace and swapped in while the fit pins run.
+PY_MUTANTS = {
+    "fit_not_centred": ("np.linalg.svd(x - mu[None, :], full_matrices=False)",
+                        "np.linalg.svd(x, full_matrices=False)"),
+    "fit_left_vectors": ("W_down = Vt[:r].T.copy()", "W_down = _[:, :r].copy()"),
+    "fit_no_sign_convention": ("W_down *= sign[None, :]", "pass"),
+    "fit_up_layout": ("W_up = W_down.reshape(T, W // T, r).transpose(0, 2, 1).copy()",
+                      "W_up = W_down.reshape(r, T, W // T).transpose(1, 0, 2).copy()"),
+}
+
+
+@pytest.mark.parametrize("name", sorted(PY_MUTANTS))
+def test_python_mutant_is_caught(name):
+    import inspect
+    import textwrap
+    old, new = PY_MUTANTS[name]
+    src = textwrap.dedent(inspect.getsource(oracle.codec_fit))
+    assert src.count(old) == 1, f"mutation site for {name} not unique"
+    ns = dict(vars(oracle))
+    exec(compile(src.replace(old, new), "<mutant>", "exec"), ns)
+    saved = oracle.codec_fit
+    oracle.codec_fit = ns["codec_fit"]
+    failed = []
+    try:
+        for fn in (P.test_codec_fit_recovers_planted_orthogonal_directions,
+                   P.test_codec_fit_energy_and_orthonormality, P.test_codec_fit_shift_moves_only_the_mean):
+            try:
+                fn()
+            except (AssertionError, ValueError, IndexError, FloatingPointError):
+                failed.append(fn.__name__)
+    finally:
+        oracle.codec_fit = saved
+    assert failed, f"mutant {name} survived every pin"

@@ -732,3 +732,56 @@ def test_decode_layer_decoupled_matches_dense_attention():
                 o_ref, lse_ref = sdpa(qf, np.concatenate([Kh, k_rope[h, sl]], axis=1), Vh, s)
                 np.testing.assert_allclose(o[b, tq, h], o_ref, atol=1e-11)
                 assert lse[b, tq, h] == pytest.approx(lse_ref, abs=1e-11)
+
+
+# ---------------------------------------------------------------------------
+# Codec fit (SVD initialisation; LLA review page, What carries the argument)
+# ---------------------------------------------------------------------------
+def test_codec_fit_recovers_planted_orthogonal_directions():
+    """x = mu0 + Z A with orthogonal columns of Z and orthonormal rows of A, distinct
+    weights: the right singular vectors are A's rows (up to the sign convention), the
+    singular values the weights, and the mean mu0 (Z's columns sum to zero)."""
+    T, d, r, n = 4, 8, 3, 40
+    W = T * d
+    rng = np.random.default_rng(80)
+    Qa, _ = np.linalg.qr(rng.standard_normal((W, W)))
+    A = Qa[:, :r].T                                   # [r, W], orthonormal rows
+    Z0 = rng.standard_normal((n, r))
+    Z0 -= Z0.mean(axis=0)
+    Qz, _ = np.linalg.qr(Z0)                         # orthonormal, zero-mean columns
+    weights = np.array([9.0, 4.0, 2.5])
+    mu0 = rng.standard_normal(W)
+    x = mu0 + (Qz * weights) @ A
+    mu, Wd, Wu, sigma = oracle.codec_fit(x, r, T)
+    np.testing.assert_allclose(mu, mu0, atol=1e-12)
+    np.testing.assert_allclose(sigma[:r], weights, rtol=1e-12)
+    assert np.all(sigma[r:] < 1e-10)
+    for j in range(r):
+        v = A[j] * np.sign(A[j][np.argmax(np.abs(A[j]))])
+        np.testing.assert_allclose(Wd[:, j], v, atol=1e-10)
+    np.testing.assert_allclose(Wu[2], Wd[2 * d:3 * d].T, atol=0)
+
+
+def test_codec_fit_energy_and_orthonormality():
+    """Orthonormal W_down; the fitted codec's residual energy on its calibration set is
+    the tail of the singular values (Eckart-Young), through the pinned residual oracle."""
+    w = S.shrink(S.WORKLOADS["tiny-fp32"], d=16)
+    model = S.trajectory_model(81, w.T * w.d)
+    x = S.draw_tokens_np(model, 100, 82)
+    for r in (1, 7, 30):
+        mu, Wd, Wu, sigma = oracle.codec_fit(x, r, w.T)
+        np.testing.assert_allclose(Wd.T @ Wd, np.eye(r), atol=1e-12)
+        err, _ = oracle.codec_residual(x, mu, Wd, Wu)
+        assert float((err ** 2).sum()) == pytest.approx(float((sigma[r:] ** 2).sum()), rel=1e-9)
+        assert np.all(np.diff(sigma) <= 0)
+
+
+def test_codec_fit_shift_moves_only_the_mean():
+    w = S.shrink(S.WORKLOADS["tiny-fp32"], d=16)
+    x = S.draw_tokens_np(S.trajectory_model(83, w.T * w.d), 60, 84)
+    shift = np.random.default_rng(85).standard_normal(w.T * w.d) * 5
+    a = oracle.codec_fit(x, 6, w.T)
+    b = oracle.codec_fit(x + shift, 6, w.T)
+    np.testing.assert_allclose(b[0], a[0] + shift, atol=1e-12)
+    np.testing.assert_allclose(b[1], a[1], atol=1e-9)
+    np.testing.assert_allclose(b[3], a[3], rtol=1e-10, atol=1e-10 * a[3][0])  # last one is ~0 (rank n-1)
