@@ -10,7 +10,7 @@ library is missing.
 Names follow the C ABI: ``cache_bytes``, ``slot_layout``, ``codec_bias``,
 ``encode``, ``decode_attn``, ``decode_workspace_bytes``, ``decode_num_splits``,
 ``decode_attn_static``, ``decode_attn_hybrid``, ``decode_hybrid_workspace_bytes``, ``decode_attn_rope``,
-``codec_residual``, ``decode_attn_decoupled``, ``decode_decoupled_workspace_bytes``,
+``codec_residual``, ``codec_fit``, ``codec_fit_workspace_bytes``, ``decode_attn_decoupled``, ``decode_decoupled_workspace_bytes``,
 ``status_fetch``, ``status_string``.
 """
 from __future__ import annotations
@@ -36,6 +36,7 @@ LLA_ERR_MISALIGNED = -3
 LLA_ERR_WORKSPACE = -4
 LLA_ERR_CUDA = -5
 LLA_ERR_DEVICE_TIMEOUT = -6
+LLA_ERR_NO_CONVERGENCE = -7
 PER_HEAD, FOLD_2D = 0, 1
 F32, BF16 = 0, 1
 ABSORB, RECONSTRUCT = 0, 1
@@ -45,6 +46,7 @@ EXPORTED = ("lla_cache_bytes", "lla_slot_layout", "lla_codec_bias", "lla_encode"
             "lla_decode_attn", "lla_decode_workspace_bytes", "lla_decode_num_splits",
             "lla_decode_attn_static", "lla_decode_attn_hybrid", "lla_decode_hybrid_workspace_bytes",
             "lla_decode_attn_rope", "lla_codec_residual", "lla_decode_attn_decoupled", "lla_decode_attn_timed",
+            "lla_codec_fit", "lla_codec_fit_workspace_bytes",
             "lla_decode_decoupled_workspace_bytes",
             "lla_status_fetch", "lla_status_string")
 STATIC_SCRATCH_BYTES = 8 << 20
@@ -91,6 +93,9 @@ _lib.lla_decode_attn_static.argtypes = [_P(Dims), _i32, _i32, _i32, _vp, _P(Cach
 _lib.lla_decode_attn_hybrid.argtypes = [_P(Dims), _i32, _i32, _i32, _vp, _P(Cache), _vp, _vp, _i32,
                                         _i32, _P(Codec), _P(Window), ctypes.c_float, _i32, _i32, _vp,
                                         _vp, _vp, _sz, _vp]
+_lib.lla_codec_fit.argtypes = [_P(Dims), _i32, _i32, _vp, _vp, _i64, _P(Codec), _vp, _vp, _vp, _sz, _vp]
+_lib.lla_codec_fit_workspace_bytes.argtypes = [_P(Dims), _i32, _i64]
+_lib.lla_codec_fit_workspace_bytes.restype = _sz
 _lib.lla_decode_attn_timed.argtypes = [_P(Dims), _i32, _i32, _i32, _vp, _P(Cache), _vp, _vp, _i32, _i32,
                                        _P(Codec), ctypes.c_float, _i32, _i32, _vp, _vp, _vp, _sz, _vp, _vp, _vp]
 _lib.lla_decode_attn_decoupled.argtypes = [_P(Dims), _i32, _i32, _i32, _vp, _P(Cache), _vp, _vp, _i32, _i32,
@@ -111,7 +116,7 @@ _lib.lla_status_string.argtypes = [ctypes.c_int]
 _lib.lla_status_string.restype = ctypes.c_char_p
 for _n in ("lla_cache_bytes", "lla_slot_layout", "lla_codec_bias", "lla_encode", "lla_decode_attn",
            "lla_decode_attn_static", "lla_decode_attn_hybrid", "lla_decode_attn_rope", "lla_codec_residual",
-           "lla_decode_attn_decoupled", "lla_decode_attn_timed",
+           "lla_decode_attn_decoupled", "lla_decode_attn_timed", "lla_codec_fit",
            "lla_decode_num_splits",
            "lla_status_fetch"):
     getattr(_lib, _n).restype = ctypes.c_int
@@ -198,6 +203,24 @@ def encode(dims: Dims, layer0: int, n_layers: int, x_k, x_v, n_tok: int, slot_id
     _check(_lib.lla_encode(ctypes.byref(dims), layer0, n_layers, _ptr(x_k), _ptr(x_v), int(n_tok),
                            _ptr(slot_idx), ctypes.byref(codec), ctypes.byref(cache), _stream(stream)),
            "lla_encode")
+
+
+def codec_fit_workspace_bytes(dims: Dims, n_layers: int, n_cal: int) -> int:
+    n = _lib.lla_codec_fit_workspace_bytes(ctypes.byref(dims), n_layers, n_cal)
+    if n == 0:
+        raise LLAError(LLA_ERR_INVALID, "lla_codec_fit_workspace_bytes")
+    return int(n)
+
+
+def codec_fit(dims: Dims, layer0: int, n_layers: int, x_k, x_v, n_cal: int, codec: Codec, workspace,
+              ws_bytes: Optional[int] = None, sigma_k=None, sigma_v=None, stream=None) -> None:
+    """SVD initialisation of the codec on the GPU: writes codec.W_down_{k,v}, W_up_{k,v}, mu_{k,v}."""
+    if ws_bytes is None:
+        ws_bytes = workspace.numel() * workspace.element_size()
+    _check(_lib.lla_codec_fit(ctypes.byref(dims), layer0, n_layers, _ptr(x_k), _ptr(x_v), n_cal,
+                              ctypes.byref(codec), _ptr(sigma_k), _ptr(sigma_v), _ptr(workspace), int(ws_bytes),
+                              _stream(stream)),
+           "lla_codec_fit")
 
 
 def codec_residual(dims: Dims, layer0: int, n_layers: int, x_k, x_v, n_tok: int, codec: Codec,

@@ -33,6 +33,21 @@ struct CodecResidualArgs {
 bool codec_residual_supported(int dtype, int r_k, int r_v, int Dp);
 cudaError_t launch_codec_residual(const CodecResidualArgs &a, cudaStream_t stream);
 
+// SVD initialisation of the codec (lla_codec_fit).
+struct CodecFitArgs {
+    const void *x_k, *x_v;             // T [n_layers][n][T][H][d]
+    void *W_down_k, *W_down_v;         // T [L][H'][r][W] (written)
+    float *W_up_k, *W_up_v;            // [L][H'][T][r][Dp] (written)
+    float *mu_k, *mu_v;                // [L][H'][T][Dp] (written)
+    float *sigma_k, *sigma_v;          // [n_layers][H'][n] or null
+    void *scratch;                     // codec_fit_scratch_bytes(...)
+    int32_t *status;
+    int64_t n;
+    int32_t layer0, n_layers, T, H, d, Dp, Hs, W, fold, r_k, r_v, dtype;
+};
+size_t codec_fit_scratch_bytes(int64_t groups, int64_t n, int64_t W, int64_t r_max);
+cudaError_t launch_codec_fit(const CodecFitArgs &a, cudaStream_t stream);
+
 cudaError_t launch_codec_bias(const void *Wd, const float *mu, float *bias, int64_t groups, int r, int W,
                               int dtype, cudaStream_t stream);
 

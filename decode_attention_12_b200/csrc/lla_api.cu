@@ -115,6 +115,7 @@ const char *lla_status_string(int code)
     case LLA_ERR_WORKSPACE: return "workspace missing or too small";
     case LLA_ERR_CUDA: return "CUDA launch or copy failed";
     case LLA_ERR_DEVICE_TIMEOUT: return "a kernel gave up a bounded wait";
+    case LLA_ERR_NO_CONVERGENCE: return "the codec fit's eigen-solver did not converge";
     default: return "unknown status";
     }
 }
@@ -230,6 +231,58 @@ int lla_encode(const lla_dims *dims, int32_t layer0, int32_t n_layers, const voi
     else
         e = launch_encode_simt(a, dims->dtype, (cudaStream_t)stream);
     return e == cudaSuccess ? LLA_OK : LLA_ERR_CUDA;
+}
+
+size_t lla_codec_fit_workspace_bytes(const lla_dims *dims, int32_t n_layers, int64_t n_cal)
+{
+    if (check_dims(dims) != LLA_OK || n_layers <= 0 || n_cal < 2)
+        return 0;
+    const int r_max = dims->r_k > dims->r_v ? dims->r_k : dims->r_v;
+    return kWorkspaceHeader +
+           codec_fit_scratch_bytes((int64_t)n_layers * heads_stored(dims), n_cal, stack_width(dims), r_max) + 1536;
+}
+
+int lla_codec_fit(const lla_dims *dims, int32_t layer0, int32_t n_layers, const void *x_k, const void *x_v,
+                  int64_t n_cal, const lla_codec *codec, float *sigma_k, float *sigma_v, void *workspace,
+                  size_t ws_bytes, lla_stream_t stream)
+{
+    int rc = check_dims(dims);
+    if (rc != LLA_OK)
+        return rc;
+    if (layer0 < 0 || n_layers < 0 || layer0 + (int64_t)n_layers > dims->L)
+        return LLA_ERR_INVALID;
+    if (n_layers == 0)
+        return LLA_OK;
+    if (n_cal < 2 || n_cal > 1024 || (n_cal & 1) || dims->r_k > n_cal - 1 || dims->r_v > n_cal - 1)
+        return LLA_ERR_INVALID;
+    if (x_k == nullptr || x_v == nullptr || codec == nullptr || codec->W_down_k == nullptr ||
+        codec->W_down_v == nullptr || codec->W_up_k == nullptr || codec->W_up_v == nullptr ||
+        codec->mu_k == nullptr || codec->mu_v == nullptr)
+        return LLA_ERR_INVALID;
+    if (!aligned16(x_k) || !aligned16(x_v) || !aligned16(codec->W_down_k) || !aligned16(codec->W_down_v) ||
+        !aligned16(codec->W_up_k) || !aligned16(codec->W_up_v) || !aligned16(codec->mu_k) ||
+        !aligned16(codec->mu_v))
+        return LLA_ERR_MISALIGNED;
+    const size_t need = lla_codec_fit_workspace_bytes(dims, n_layers, n_cal);
+    if (workspace == nullptr || ws_bytes < need)
+        return LLA_ERR_WORKSPACE;
+    if (!aligned16(workspace))
+        return LLA_ERR_MISALIGNED;
+    CodecFitArgs a;
+    a.x_k = x_k; a.x_v = x_v;
+    a.W_down_k = const_cast<void *>(codec->W_down_k); a.W_down_v = const_cast<void *>(codec->W_down_v);
+    a.W_up_k = const_cast<float *>(codec->W_up_k); a.W_up_v = const_cast<float *>(codec->W_up_v);
+    a.mu_k = const_cast<float *>(codec->mu_k); a.mu_v = const_cast<float *>(codec->mu_v);
+    a.sigma_k = sigma_k; a.sigma_v = sigma_v;
+    uint8_t *ws = static_cast<uint8_t *>(workspace);
+    a.status = reinterpret_cast<int32_t *>(ws);
+    a.scratch = ws + kWorkspaceHeader;
+    a.n = n_cal;
+    a.layer0 = layer0; a.n_layers = n_layers;
+    a.T = dims->T; a.H = dims->H; a.d = dims->d_head; a.Dp = (int32_t)loop_width(dims); a.Hs = heads_stored(dims);
+    a.W = (int32_t)stack_width(dims); a.fold = dims->fold; a.r_k = dims->r_k; a.r_v = dims->r_v;
+    a.dtype = dims->dtype;
+    return launch_codec_fit(a, (cudaStream_t)stream) == cudaSuccess ? LLA_OK : LLA_ERR_CUDA;
 }
 
 int lla_codec_residual(const lla_dims *dims, int32_t layer0, int32_t n_layers, const void *x_k, const void *x_v,

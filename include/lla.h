@@ -52,6 +52,8 @@ typedef struct CUevent_st *lla_event_t;   /* same type as cudaEvent_t           
 #define LLA_ERR_CUDA (-5)        /* a CUDA launch or copy failed                         */
 #define LLA_ERR_DEVICE_TIMEOUT (-6) /* a kernel gave up a bounded wait (reported via the
                                        workspace status word, see lla_status_fetch)      */
+#define LLA_ERR_NO_CONVERGENCE (-7) /* lla_codec_fit: the eigen-solver did not converge
+                                       (reported via the workspace status word)         */
 
 /* ---- problem description ---------------------------------------------------------- */
 enum { LLA_PER_HEAD = 0, LLA_FOLD_2D = 1 };       /* lla_dims.fold                    */
@@ -133,6 +135,30 @@ int lla_codec_bias(const lla_dims *dims, const lla_codec *codec, float *bias_k_o
 int lla_encode(const lla_dims *dims, int32_t layer0, int32_t n_layers, const void *x_k,
                const void *x_v, int64_t n_tok, const int64_t *slot_idx,
                const lla_codec *codec, const lla_cache *cache, lla_stream_t stream);
+
+/* ---- NEXT-3: codec fit on the GPU (SVD initialisation) -----------------------------------
+ * Review page, "What carries the argument": the codec starts from the top right singular
+ * vectors of the centred teacher activations.  For layers layer0 .. layer0+n_layers-1,
+ * every stored head h' and both axes, from n calibration vectors x_i (bf16 or fp32, the
+ * lla_encode input layout [n_layers][n][T][H][d]):
+ *   mu = mean_i x_i,  Y = X - mu = U diag(sigma) V^T,
+ *   W_down = V[:, :r] with each column signed so its largest-magnitude entry is positive
+ *            (the first on a tie), stored transposed in T: codec->W_down_{k,v} [L][H'][r][W]
+ *   W_up,t = transpose of the loop-t row block of W_down: codec->W_up_{k,v} (fp32)
+ *   mu_t   = loop-t slice of mu: codec->mu_{k,v} (fp32)
+ * The codec pointers are written (the const in lla_codec is the read paths' view).
+ * sigma_k / sigma_v, if not NULL, receive all n singular values per group, descending
+ * (fp32 [n_layers][H'][n]).  Method: the dual Gram matrix K = Y Y^T (n x n) in fp64,
+ * parallel cyclic Jacobi on K (one CTA per group), v_j = Y^T u_j / sigma_j.
+ * Requirements: n even, 2 <= n <= 1024, r_k, r_v <= n - 1.  The workspace holds
+ * lla_codec_fit_workspace_bytes(...) bytes; its first word is a status word (must be zero
+ * on entry; lla_status_fetch reads it): LLA_ERR_NO_CONVERGENCE if a group's Jacobi sweeps
+ * did not converge (results then approximate).  Errors: LLA_ERR_INVALID,
+ * LLA_ERR_MISALIGNED, LLA_ERR_WORKSPACE, LLA_ERR_CUDA.                                 */
+size_t lla_codec_fit_workspace_bytes(const lla_dims *dims, int32_t n_layers, int64_t n_cal);
+int lla_codec_fit(const lla_dims *dims, int32_t layer0, int32_t n_layers, const void *x_k,
+                  const void *x_v, int64_t n_cal, const lla_codec *codec, float *sigma_k,
+                  float *sigma_v, void *workspace, size_t ws_bytes, lla_stream_t stream);
 
 /* ---- NEXT-3: per-token reconstruction residual (codec diagnostic) ------------------------
  * The Pith verdict record's concrete test for the shared-subspace assumption: on held-out

@@ -255,6 +255,32 @@ def test_timed_entry_needs_both_events():
     assert rc == lla.LLA_ERR_INVALID
 
 
+def test_codec_fit_argument_errors():
+    codec = lla.make_codec(W_down_k=FAKE, W_down_v=FAKE, W_up_k=FAKE, W_up_v=FAKE, mu_k=FAKE, mu_v=FAKE)
+    dims = lla.make_dims(4, 2, 16, 128, 16, 32)
+
+    def rc(n_cal=256, **over):
+        a = dict(layer0=0, n_layers=1, x_k=FAKE, x_v=FAKE, workspace=FAKE, ws_bytes=1 << 40, stream=0)
+        a.update(over)
+        try:
+            lla.codec_fit(over.pop("dims", dims), a["layer0"], a["n_layers"], a["x_k"], a["x_v"], n_cal,
+                          over.get("codec", codec), a["workspace"], a["ws_bytes"], stream=0)
+        except lla.LLAError as e:
+            return e.code
+        return 0
+
+    assert rc(layer0=2) == lla.LLA_ERR_INVALID
+    assert rc(n_cal=255) == lla.LLA_ERR_INVALID          # odd
+    assert rc(n_cal=2048) == lla.LLA_ERR_INVALID         # above 1024
+    assert rc(n_cal=32) == lla.LLA_ERR_INVALID           # r_v = 32 > n - 1
+    assert rc(x_v=0) == lla.LLA_ERR_INVALID
+    assert rc(x_k=FAKE + 8) == lla.LLA_ERR_MISALIGNED
+    assert rc(ws_bytes=1024) == lla.LLA_ERR_WORKSPACE
+    assert rc(n_layers=0) == 0
+    n = lla.codec_fit_workspace_bytes(dims, 1, 256)
+    assert n >= 16 * (2 * 256 * 256 * 8)
+
+
 def test_workspace_bytes_and_splits():
     dims = lla.make_dims(4, 1, 16, 128, 16, 32)
     s = lla.decode_num_splits(dims, 64, 4, 4096)
