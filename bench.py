@@ -61,7 +61,7 @@ def parse():
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--variant", default="absorb", choices=["absorb", "reconstruct"],
                     help="decode read form (the headline uses absorb)")
-    ap.add_argument("--phase", default="step", choices=["step", "encode", "residual"],
+    ap.add_argument("--phase", default="step", choices=["step", "encode", "residual", "fit"],
                     help="step: decode step (headline); encode: prefill encode of one layer")
     ap.add_argument("--encode-seqs", type=int, default=0,
                     help="--phase encode: sequences of len_hi tokens to encode (default: B)")
@@ -386,6 +386,71 @@ def run_residual_phase(args, dev):
     }), flush=True)
 
 
+def run_fit_phase(args, dev):
+    """Codec fit (SVD initialisation) of every layer, head and axis from 256 calibration tokens."""
+    import torch
+    import decode_attention_12_b200 as lla
+    import lla_synth as S
+
+    w = S.WORKLOADS[args.workload]
+    n = 256
+    dims = lla.make_dims(w.T, w.L, w.H, w.d, w.r_k, w.r_v, int(w.fold2d), lla.BF16)
+    Hs, Dp = w.heads_stored, w.d * (w.H if w.fold2d else 1)
+    xs = {ax: torch.stack([S.draw_encode_tokens(w, l, ax, n, dev, seed_tag="calib") for l in range(w.L)])
+          for ax in ("k", "v")}
+    outs = {}
+    for ax, r in (("k", w.r_k), ("v", w.r_v)):
+        outs[f"W_down_{ax}"] = torch.empty(w.L, Hs, r, w.W, dtype=w.torch_dtype, device=dev)
+        outs[f"W_up_{ax}"] = torch.empty(w.L, Hs, w.T, r, Dp, device=dev)
+        outs[f"mu_{ax}"] = torch.empty(w.L, Hs, w.T, Dp, device=dev)
+    codec = lla.make_codec(**outs)
+    wsb = lla.codec_fit_workspace_bytes(dims, w.L, n)
+    ws = torch.zeros(wsb, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step():
+        lla.codec_fit(dims, 0, w.L, xs["k"], xs["v"], n, codec, ws, wsb, stream=stream)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    ws[:8].zero_()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    sampler = ClockSampler(dev.index or 0).start()
+    wall0 = time.perf_counter()
+    e0.record(stream)
+    for _ in range(args.steps):
+        step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    wall1 = time.perf_counter()
+    sampler.stop()
+    head = ws[:8].view(torch.int32).cpu().tolist()
+    assert head[0] == 0, "eigen-solver did not converge"
+    sweeps_per_group = head[1] / (args.steps * 2 * w.L * Hs)
+    ms = e0.elapsed_time(e1) / args.steps
+    groups = 2 * w.L * Hs
+    # algorithmic fp64 flop per group: Gram n^2 W and v_j = Y^T u_j (2 n W r) as FMAs (x2),
+    # each Jacobi sweep (n - 1 rounds: 24 flop per 2x2 block of K, 6 per pair of U entries)
+    r_avg = (w.r_k + w.r_v) / 2
+    flop = groups * (2.0 * n * n * w.W + 2.0 * n * w.W * r_avg
+                     + sweeps_per_group * (n - 1) * (24.0 * (n / 2) ** 2 + 6.0 * n * (n / 2)))
+    # fp64 peak from unit counts and clocks: 148 SMs x 64 fp64 FMA lanes x 2 flop x 1.965 GHz
+    fp64_peak = 148 * 64 * 2 * 1.965e9 / 1e12
+    tfl = flop / (ms * 1e-3) / 1e12
+    print(json.dumps({
+        "metric": "LLA codec fit ms per model (SVD initialisation of K and V, every layer and head)",
+        "value": ms, "unit": "ms", "n_gpus": 1, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+        "higher_is_better": False, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": w.name, "layers": w.L, "heads_stored": Hs, "W": w.W, "r_k": w.r_k,
+                   "r_v": w.r_v, "calibration_tokens": n, "groups": groups,
+                   "jacobi_sweeps_per_group": sweeps_per_group},
+        "roofline": {"bound": "alu", "achieved": tfl, "peak": fp64_peak, "unit": "TFLOP/s",
+                     "frac": tfl / fp64_peak, "peak_kind": "fp64 units x clock (derived, not measured)"},
+        "clocks": sampler.summary(wall0, wall1),
+    }), flush=True)
+
+
 # ---------------------------------------------------------------------------
 # our arm
 # ---------------------------------------------------------------------------
@@ -415,6 +480,9 @@ def main():
         return
     if args.phase == "residual":
         run_residual_phase(args, dev)
+        return
+    if args.phase == "fit":
+        run_fit_phase(args, dev)
         return
     w = S.WORKLOADS[args.workload]
     Tq = w.T

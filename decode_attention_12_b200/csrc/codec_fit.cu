@@ -41,7 +41,7 @@ struct FitArgs {
     double *lam;            // [G][n] eigenvalues, descending
     int32_t *order;         // [G][n] index of the j-th largest eigenvalue
     double *V;              // [G][r][W]
-    int32_t *status;        // sticky: LLA_ERR_NO_CONVERGENCE
+    int32_t *status;        // sticky: LLA_ERR_NO_CONVERGENCE; status[1] += sweeps of every group
     void *W_down;           // T [L][H'][r][W]
     float *W_up;            // [L][H'][T][r][Dp]
     float *mu;              // [L][H'][T][Dp]
@@ -141,7 +141,8 @@ __global__ void __launch_bounds__(kJacobiThreads) fit_jacobi_kernel(const FitArg
     }
     __syncthreads();
     bool converged = false;
-    for (int sweep = 0; sweep < kFitMaxSweeps && !converged; ++sweep) {
+    int sweeps = 0;
+    for (int sweep = 0; sweep < kFitMaxSweeps && !converged; ++sweep, ++sweeps) {
         if (threadIdx.x == 0)
             rotated = 0;
         __syncthreads();
@@ -193,8 +194,11 @@ __global__ void __launch_bounds__(kJacobiThreads) fit_jacobi_kernel(const FitArg
         converged = rotated == 0;
         __syncthreads();
     }
-    if (!converged && threadIdx.x == 0)
-        report_status(a.status, LLA_ERR_NO_CONVERGENCE);
+    if (threadIdx.x == 0) {
+        atomicAdd(a.status + 1, sweeps);
+        if (!converged)
+            report_status(a.status, LLA_ERR_NO_CONVERGENCE);
+    }
 }
 
 // Eigenvalues of K (its diagonal after Jacobi) ranked descending; sigma = sqrt(lambda).

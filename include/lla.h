@@ -153,7 +153,9 @@ int lla_encode(const lla_dims *dims, int32_t layer0, int32_t n_layers, const voi
  * Requirements: n even, 2 <= n <= 1024, r_k, r_v <= n - 1.  The workspace holds
  * lla_codec_fit_workspace_bytes(...) bytes; its first word is a status word (must be zero
  * on entry; lla_status_fetch reads it): LLA_ERR_NO_CONVERGENCE if a group's Jacobi sweeps
- * did not converge (results then approximate).  Errors: LLA_ERR_INVALID,
+ * did not converge (results then approximate); its second 32-bit word accumulates the
+ * Jacobi sweeps of every group (zero it before the call to count one call's sweeps; each
+ * sweep is n - 1 rounds over all n/2 index pairs).  Errors: LLA_ERR_INVALID,
  * LLA_ERR_MISALIGNED, LLA_ERR_WORKSPACE, LLA_ERR_CUDA.                                 */
 size_t lla_codec_fit_workspace_bytes(const lla_dims *dims, int32_t n_layers, int64_t n_cal);
 int lla_codec_fit(const lla_dims *dims, int32_t layer0, int32_t n_layers, const void *x_k,
