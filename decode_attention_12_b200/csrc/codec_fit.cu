@@ -30,6 +30,7 @@ namespace {
 
 constexpr int kFitMaxSweeps = 40;
 constexpr int kJacobiThreads = 512;
+constexpr int kJacobiUnroll = 4; // blocks / entries per thread and pass (loads first)
 
 struct FitArgs {
     const void *x;          // T [n_layers][n][T][H][d] (one axis)
@@ -167,27 +168,73 @@ __global__ void __launch_bounds__(kJacobiThreads) fit_jacobi_kernel(const FitArg
                 sn[k] = s;
             }
             __syncthreads();
-            // K <- J^T K J, one 2 x 2 block (pair a rows, pair b columns) per step
-            for (int64_t e = threadIdx.x; e < (int64_t)np * np; e += blockDim.x) {
-                const int ia = (int)(e / np), ib = (int)(e - (int64_t)ia * np);
-                const int pa = P[ia], qa = Q[ia], pb = P[ib], qb = Q[ib];
-                const double ca = cs[ia], sa = sn[ia], cb = cs[ib], sb = sn[ib];
-                double *r0 = K + (int64_t)pa * n, *r1 = K + (int64_t)qa * n;
-                const double m00 = r0[pb], m01 = r0[qb], m10 = r1[pb], m11 = r1[qb];
-                const double t00 = m00 * cb - m01 * sb, t01 = m00 * sb + m01 * cb;
-                const double t10 = m10 * cb - m11 * sb, t11 = m10 * sb + m11 * cb;
-                r0[pb] = ca * t00 - sa * t10;
-                r0[qb] = ca * t01 - sa * t11;
-                r1[pb] = sa * t00 + ca * t10;
-                r1[qb] = sa * t01 + ca * t11;
+            // K <- J^T K J, one 2 x 2 block (pair a rows, pair b columns) per step;
+            // kJacobiUnroll blocks per thread and pass, all loads issued before the stores (the
+            // blocks are disjoint, but the compiler cannot know it)
+            const int64_t nblk = (int64_t)np * np;
+            for (int64_t e0 = threadIdx.x; e0 < nblk; e0 += kJacobiUnroll * (int64_t)blockDim.x) {
+                double m[kJacobiUnroll][4];
+                int r0i[kJacobiUnroll], r1i[kJacobiUnroll], c0i[kJacobiUnroll], c1i[kJacobiUnroll], pi[kJacobiUnroll],
+                    pj[kJacobiUnroll];
+                bool ok[kJacobiUnroll];
+#pragma unroll
+                for (int u = 0; u < kJacobiUnroll; ++u) {
+                    const int64_t e = e0 + (int64_t)u * blockDim.x;
+                    ok[u] = e < nblk;
+                    const int ia = ok[u] ? (int)(e / np) : 0, ib = ok[u] ? (int)(e - (int64_t)ia * np) : 0;
+                    pi[u] = ia;
+                    pj[u] = ib;
+                    r0i[u] = P[ia];
+                    r1i[u] = Q[ia];
+                    c0i[u] = P[ib];
+                    c1i[u] = Q[ib];
+                    if (ok[u]) {
+                        m[u][0] = K[(int64_t)r0i[u] * n + c0i[u]];
+                        m[u][1] = K[(int64_t)r0i[u] * n + c1i[u]];
+                        m[u][2] = K[(int64_t)r1i[u] * n + c0i[u]];
+                        m[u][3] = K[(int64_t)r1i[u] * n + c1i[u]];
+                    }
+                }
+#pragma unroll
+                for (int u = 0; u < kJacobiUnroll; ++u) {
+                    if (!ok[u])
+                        continue;
+                    const double ca = cs[pi[u]], sa = sn[pi[u]], cb = cs[pj[u]], sb = sn[pj[u]];
+                    const double t00 = m[u][0] * cb - m[u][1] * sb, t01 = m[u][0] * sb + m[u][1] * cb;
+                    const double t10 = m[u][2] * cb - m[u][3] * sb, t11 = m[u][2] * sb + m[u][3] * cb;
+                    K[(int64_t)r0i[u] * n + c0i[u]] = ca * t00 - sa * t10;
+                    K[(int64_t)r0i[u] * n + c1i[u]] = ca * t01 - sa * t11;
+                    K[(int64_t)r1i[u] * n + c0i[u]] = sa * t00 + ca * t10;
+                    K[(int64_t)r1i[u] * n + c1i[u]] = sa * t01 + ca * t11;
+                }
             }
-            // U <- U J
-            for (int64_t e = threadIdx.x; e < (int64_t)n * np; e += blockDim.x) {
-                const int row = (int)(e / np), k = (int)(e - (int64_t)row * np);
-                double *ur = U + (int64_t)row * n;
-                const double up = ur[P[k]], uq = ur[Q[k]];
-                ur[P[k]] = cs[k] * up - sn[k] * uq;
-                ur[Q[k]] = sn[k] * up + cs[k] * uq;
+            // U <- U J, kJacobiUnroll (row, pair) entries per thread and pass
+            const int64_t nup = (int64_t)n * np;
+            for (int64_t e0 = threadIdx.x; e0 < nup; e0 += kJacobiUnroll * (int64_t)blockDim.x) {
+                double up[kJacobiUnroll], uq[kJacobiUnroll];
+                int64_t ip[kJacobiUnroll], iq[kJacobiUnroll];
+                int kk[kJacobiUnroll];
+                bool ok[kJacobiUnroll];
+#pragma unroll
+                for (int u = 0; u < kJacobiUnroll; ++u) {
+                    const int64_t e = e0 + (int64_t)u * blockDim.x;
+                    ok[u] = e < nup;
+                    const int row = ok[u] ? (int)(e / np) : 0, k = ok[u] ? (int)(e - (int64_t)row * np) : 0;
+                    kk[u] = k;
+                    ip[u] = (int64_t)row * n + P[k];
+                    iq[u] = (int64_t)row * n + Q[k];
+                    if (ok[u]) {
+                        up[u] = U[ip[u]];
+                        uq[u] = U[iq[u]];
+                    }
+                }
+#pragma unroll
+                for (int u = 0; u < kJacobiUnroll; ++u) {
+                    if (!ok[u])
+                        continue;
+                    U[ip[u]] = cs[kk[u]] * up[u] - sn[kk[u]] * uq[u];
+                    U[iq[u]] = sn[kk[u]] * up[u] + cs[kk[u]] * uq[u];
+                }
             }
             __syncthreads();
         }
