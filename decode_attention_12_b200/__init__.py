@@ -46,7 +46,7 @@ EXPORTED = ("lla_cache_bytes", "lla_slot_layout", "lla_codec_bias", "lla_encode"
             "lla_decode_attn", "lla_decode_workspace_bytes", "lla_decode_num_splits",
             "lla_decode_attn_static", "lla_decode_attn_hybrid", "lla_decode_hybrid_workspace_bytes",
             "lla_decode_attn_rope", "lla_codec_residual", "lla_decode_attn_decoupled", "lla_decode_attn_timed",
-            "lla_codec_fit", "lla_codec_fit_workspace_bytes",
+            "lla_codec_fit", "lla_codec_fit_workspace_bytes", "lla_selftest_wait_timeout",
             "lla_decode_decoupled_workspace_bytes",
             "lla_status_fetch", "lla_status_string")
 STATIC_SCRATCH_BYTES = 8 << 20
@@ -112,6 +112,8 @@ _lib.lla_decode_workspace_bytes.argtypes = [_P(Dims), _i32, _i32, _i32, _i32, _i
 _lib.lla_decode_workspace_bytes.restype = _sz
 _lib.lla_decode_num_splits.argtypes = [_P(Dims), _i32, _i32, _i32, _i32, _i32]
 _lib.lla_status_fetch.argtypes = [_vp, _vp, _P(_i32)]
+_lib.lla_selftest_wait_timeout.argtypes = [_vp, _vp]
+_lib.lla_selftest_wait_timeout.restype = ctypes.c_int
 _lib.lla_status_string.argtypes = [ctypes.c_int]
 _lib.lla_status_string.restype = ctypes.c_char_p
 for _n in ("lla_cache_bytes", "lla_slot_layout", "lla_codec_bias", "lla_encode", "lla_decode_attn",
@@ -352,6 +354,12 @@ def decode_attn_static(dims: Dims, layer: int, t0: int, Tq: int, q, cache: Cache
                                        ctypes.byref(codec), float(softmax_scale), variant, num_splits,
                                        _ptr(out), _ptr(lse), _stream(stream)),
            "lla_decode_attn_static")
+
+
+def selftest_wait_timeout(workspace, stream=None) -> None:
+    """Run the bounded-wait self-test: a wait that nothing completes gives up (about 2 s)
+    and records LLA_ERR_DEVICE_TIMEOUT in the workspace's status word."""
+    _check(_lib.lla_selftest_wait_timeout(_ptr(workspace), _stream(stream)), "lla_selftest_wait_timeout")
 
 
 def status_fetch(workspace, stream=None) -> int:

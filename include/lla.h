@@ -379,6 +379,14 @@ int lla_decode_attn_static(const lla_dims *dims, int32_t layer, int32_t t0, int3
 int lla_status_fetch(void *workspace, lla_stream_t stream, int32_t *status_host);
 const char *lla_status_string(int code);
 
+/* Failure-detection self-test (no counterpart in the paper): launches one kernel whose only
+ * wait, bounded exactly like the decode and encode kernels' waits, is on a barrier that
+ * nothing completes.  After about two seconds the wait gives up, LLA_ERR_DEVICE_TIMEOUT is
+ * recorded in the first word of `workspace` (read it with lla_status_fetch) and the kernel
+ * returns; nothing traps and the context stays usable.  workspace: 16-byte aligned device
+ * memory of at least 4 bytes whose first word is zero.                                  */
+int lla_selftest_wait_timeout(void *workspace, lla_stream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

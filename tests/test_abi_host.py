@@ -281,6 +281,11 @@ def test_codec_fit_argument_errors():
     assert n >= 16 * (2 * 256 * 256 * 8)
 
 
+def test_selftest_argument_errors():
+    assert lla._lib.lla_selftest_wait_timeout(None, None) == lla.LLA_ERR_INVALID
+    assert lla._lib.lla_selftest_wait_timeout(FAKE + 4, None) == lla.LLA_ERR_MISALIGNED
+
+
 def test_workspace_bytes_and_splits():
     dims = lla.make_dims(4, 1, 16, 128, 16, 32)
     s = lla.decode_num_splits(dims, 64, 4, 4096)
