@@ -502,7 +502,7 @@ def main():
     # independent cache replicas, rotated per step so that no step finds latents in L2: at
     # least enough that the replicas together span twice the 126 MB L2 (small planes, such
     # as the LLA-2D layer's 25 MB, need more than the default 3)
-    plane_bytes = (p["k"].numel() + p["v"].numel()) * p["k"].element_size()
+    plane_bytes = (p["k"][0].numel() + p["v"][0].numel()) * p["k"].element_size()  # the layer a step reads
     R = max(1, args.replicas, math.ceil(2 * L2_BYTES / max(plane_bytes, 1)) if args.replicas > 1 else 1)
     reps = [(p["k"], p["v"])] + [(p["k"].clone(), p["v"].clone()) for _ in range(R - 1)]
     caches = [lla.make_cache(k, v, p["slots"]) for k, v in reps]
@@ -784,7 +784,7 @@ def main():
                             if args.model_order else f"decode_attn(all {w.T} loop queries fused)")
                            + (f" with {Wn} exact window rows per sequence (decode_attn_hybrid)" if Wn else "")
                            + " + encode(B new tokens)",
-                   "l2": f"{R} rotating cache replicas of {plane_bytes / 1e6:.0f} MB "
+                   "l2": f"{R} rotating cache replicas; the layer read per step is {plane_bytes / 1e6:.0f} MB "
                          f"({R * plane_bytes / 1e6:.0f} MB together, L2 is 126 MB); "
                          f"{step_bytes / 1e6:.0f} MB read per step",
                    "parallelism": f"replicas x{world}"},

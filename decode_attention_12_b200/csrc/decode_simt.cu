@@ -512,15 +512,15 @@ __device__ __forceinline__ float4 f4_fma(float s, float4 x, float4 y)
 __device__ __forceinline__ float4 f4_scale(float s, float4 x) { return make_float4(s * x.x, s * x.y, s * x.z, s * x.w); }
 
 // Records [s0, s0 + n) of one unit in registers: (m, l) and this lane's RG column groups.
-template <int RG> struct RecBatch {
-    float2 ml[kSpecRecords];
-    float4 rv[kSpecRecords][RG];
+template <int RG, int SPEC> struct RecBatch {
+    float2 ml[SPEC];
+    float4 rv[SPEC][RG];
 
-    // Loads the records s0 + k < lim (k < kSpecRecords); lane c holds columns 4c + 128 g.
+    // Loads the records s0 + k < lim (k < SPEC); lane c holds columns 4c + 128 g.
     __device__ __forceinline__ void load(const float *rec0, int s0, int lim, int ps, int RV, int lane)
     {
 #pragma unroll
-        for (int k = 0; k < kSpecRecords; ++k) {
+        for (int k = 0; k < SPEC; ++k) {
             const int s = s0 + k;
             ml[k] = make_float2(-INFINITY, 0.f);
 #pragma unroll
@@ -543,7 +543,7 @@ template <int RG> struct RecBatch {
     {
         float Mn = M;
 #pragma unroll
-        for (int k = 0; k < kSpecRecords; ++k)
+        for (int k = 0; k < SPEC; ++k)
             if (k < n)
                 Mn = fmaxf(Mn, ml[k].x);
         if (Mn == -INFINITY)
@@ -554,7 +554,7 @@ template <int RG> struct RecBatch {
         for (int g = 0; g < RG; ++g)
             acc[g] = f4_scale(al, acc[g]);
 #pragma unroll
-        for (int k = 0; k < kSpecRecords; ++k) {
+        for (int k = 0; k < SPEC; ++k) {
             if (k < n && ml[k].x != -INFINITY) {
                 const float w = exp2f(ml[k].x - Mn);
                 L = fmaf(w, ml[k].y, L);
@@ -570,8 +570,8 @@ template <int RG> struct RecBatch {
 // REC: records carry d-wide outputs of the reconstruct form (mu and the q.mu_t^K score term
 // already included), so the output is the merged record itself.  RG = record width / 128,
 // rounded up.  WIN: hybrid form, merge the window part (a.win_part) as well.
-template <typename T, typename O, bool REC, int RG, bool WIN>
-__global__ void __launch_bounds__(kCombineThreads, RG == 1 && !WIN ? 4 : RG == 1 ? 3 : 2)
+template <typename T, typename O, bool REC, int RG, bool WIN, int SPEC>
+__global__ void __launch_bounds__(kCombineThreads, RG == 1 && !WIN && SPEC == kSpecRecords ? 4 : RG == 1 ? 3 : 2)
     decode_combine_kernel(const DecodeArgs a)
 {
     extern __shared__ __align__(16) float csm[];
@@ -634,13 +634,13 @@ __global__ void __launch_bounds__(kCombineThreads, RG == 1 && !WIN ? 4 : RG == 1
     if (active && len > 0) {
         const float *rec0 = a.part + (u * a.Tq_all + t) * a.seg_max * ps;
         const int cnt = a.counts[u];
-        RecBatch<RG> rb;
+        RecBatch<RG, SPEC> rb;
         rb.load(rec0, 0, a.seg_max, ps, RV, lane); // issued together with the count
         const int S = min(cnt, a.seg_max);
-        rb.merge(min(S, kSpecRecords), M, L, acc);
-        for (int s0 = kSpecRecords; s0 < S; s0 += kSpecRecords) { // long contexts / many splits
+        rb.merge(min(S, SPEC), M, L, acc);
+        for (int s0 = SPEC; s0 < S; s0 += SPEC) { // long contexts / many splits
             rb.load(rec0, s0, S, ps, RV, lane);
-            rb.merge(min(S - s0, kSpecRecords), M, L, acc);
+            rb.merge(min(S - s0, SPEC), M, L, acc);
         }
     }
     const float invL = L > 0.f ? 1.f / L : 0.f;
@@ -762,12 +762,14 @@ cudaError_t launch_absorb_prologue(const DecodeArgs &a, int dtype, cudaStream_t 
     return cudaGetLastError();
 }
 
-template <typename T, typename O, int RG>
+template <typename T, typename O, int RG, int SPEC>
 static cudaError_t launch_combine_t(const DecodeArgs &a, size_t smem, cudaStream_t stream)
 {
     const bool win = a.win_part != nullptr;
-    auto k = a.recon ? (win ? decode_combine_kernel<T, O, true, RG, true> : decode_combine_kernel<T, O, true, RG, false>)
-                     : (win ? decode_combine_kernel<T, O, false, RG, true> : decode_combine_kernel<T, O, false, RG, false>);
+    auto k = a.recon ? (win ? decode_combine_kernel<T, O, true, RG, true, SPEC>
+                            : decode_combine_kernel<T, O, true, RG, false, SPEC>)
+                     : (win ? decode_combine_kernel<T, O, false, RG, true, SPEC>
+                            : decode_combine_kernel<T, O, false, RG, false, SPEC>);
     cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess)
         return e;
@@ -787,7 +789,13 @@ static cudaError_t launch_combine_t(const DecodeArgs &a, size_t smem, cudaStream
 template <typename T, typename O>
 static cudaError_t launch_combine_rg(const DecodeArgs &a, int rv, size_t smem, cudaStream_t stream)
 {
-    return rv > 128 ? launch_combine_t<T, O, 2>(a, smem, stream) : launch_combine_t<T, O, 1>(a, smem, stream);
+    // many record slots per unit (LLA-2D's short shares, long contexts): 8 records per load
+    // round instead of 4, so fewer dependent rounds; the small batch keeps the register count
+    // (and the CTAs resident beside a finishing decode grid) when a unit has <= 4 records
+    if (rv > 128)
+        return launch_combine_t<T, O, 2, kSpecRecords>(a, smem, stream);
+    return a.seg_max > kSpecRecords ? launch_combine_t<T, O, 1, 2 * kSpecRecords>(a, smem, stream)
+                                    : launch_combine_t<T, O, 1, kSpecRecords>(a, smem, stream);
 }
 
 cudaError_t launch_decode_combine(const DecodeArgs &a, int dtype, int out_dtype, cudaStream_t stream)
