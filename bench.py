@@ -504,7 +504,8 @@ def main():
     # as the LLA-2D layer's 25 MB, need more than the default 3)
     plane_bytes = (p["k"][0].numel() + p["v"][0].numel()) * p["k"].element_size()  # the layer a step reads
     R = max(1, args.replicas, math.ceil(2 * L2_BYTES / max(plane_bytes, 1)) if args.replicas > 1 else 1)
-    reps = [(p["k"], p["v"])] + [(p["k"].clone(), p["v"].clone()) for _ in range(R - 1)]
+    # (a step reads layer 0 only, so the extra replicas hold that layer alone)
+    reps = [(p["k"], p["v"])] + [(p["k"][:1].clone(), p["v"][:1].clone()) for _ in range(R - 1)]
     caches = [lla.make_cache(k, v, p["slots"]) for k, v in reps]
     # hybrid form: every sequence holds a full window of W exact rows (steady state)
     Wn = max(0, args.window)
