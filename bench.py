@@ -550,35 +550,33 @@ def main():
     stream = torch.cuda.current_stream(dev)
     splits = lla.decode_num_splits(dims, B, Tq_call, max_ctx, variant, args.num_splits)
 
-    def decode(i, q_in=None, out_buf=None, lse_buf=None, strm=None):
-        stream_ = strm if strm is not None else stream
+    def decode(i, q_in=None, out_buf=None, lse_buf=None):
         for c, (t0, n) in enumerate(calls):
             if DRn:
                 lla.decode_attn_decoupled(dims, 0, t0, n, (q_in or qs)[c], caches[i % R], p["seq_start"],
                                           p["ctx_lens"], B, max_ctx, codec, k_ropes[i % R],
                                           q_ropes[c], DRn,
                                           rope, 1.0, (out_buf or outs)[c], (lse_buf or lses)[c], ws, ws_bytes,
-                                          num_splits=args.num_splits, stream=stream_)
+                                          num_splits=args.num_splits, stream=stream)
                 continue
             if rope is not None:
                 lla.decode_attn_rope(dims, 0, t0, n, (q_in or qs)[c], caches[i % R], p["seq_start"],
                                      p["ctx_lens"], B, max_ctx, codec, rope, 1.0, (out_buf or outs)[c],
                                      (lse_buf or lses)[c], ws, ws_bytes, num_splits=args.num_splits,
-                                     stream=stream_)
+                                     stream=stream)
                 continue
             if Wn:
                 lla.decode_attn_hybrid(dims, 0, t0, n, (q_in or qs)[c], caches[i % R], p["seq_start"],
                                        p["ctx_lens"], B, max_ctx, codec, windows[i % R], 1.0,
                                        (out_buf or outs)[c], (lse_buf or lses)[c], ws, ws_bytes,
-                                       variant=variant, num_splits=args.num_splits, stream=stream_)
+                                       variant=variant, num_splits=args.num_splits, stream=stream)
                 continue
             lla.decode_attn(dims, 0, t0, n, (q_in or qs)[c], caches[i % R], p["seq_start"], p["ctx_lens"], B,
                             max_ctx, codec, 1.0, (out_buf or outs)[c], (lse_buf or lses)[c], ws, ws_bytes,
-                            variant=variant, num_splits=args.num_splits, stream=stream_)
+                            variant=variant, num_splits=args.num_splits, stream=stream)
 
-    def encode(i, xk=x_k, xv=x_v, strm=None):
-        lla.encode(dims, 0, 1, xk, xv, B, new_slot, codec, caches[i % R],
-                   stream=strm if strm is not None else stream)
+    def encode(i, xk=x_k, xv=x_v):
+        lla.encode(dims, 0, 1, xk, xv, B, new_slot, codec, caches[i % R], stream=stream)
 
     # per decode call: prologue + decode + combine (reconstruct: one decode pass per loop
     # query + combine); the encode of K and V is one launch
@@ -709,8 +707,6 @@ def main():
     out_read = [torch.cuda.Event() for _ in range(2)]
     e2e_steps = max(1, min(args.steps, 1000))
 
-    c_e2e = torch.cuda.Stream(dev)  # compute stream of the end-to-end steps (capturable)
-
     def e2e_step(i):
         sl = i % 2
         if i >= 2:
@@ -721,12 +717,12 @@ def main():
             xk_d[sl].copy_(xk_h, non_blocking=True)
             xv_d[sl].copy_(xv_h, non_blocking=True)
         in_ready[sl].record(s_in)
-        c_e2e.wait_event(in_ready[sl])
+        stream.wait_event(in_ready[sl])
         if i >= 2:
-            c_e2e.wait_event(out_read[sl])     # step i-2's results have left this slot
-        decode(i, q_in=q_d[sl], out_buf=out_d[sl], lse_buf=lse_d[sl], strm=c_e2e)
-        encode(i, xk=xk_d[sl], xv=xv_d[sl], strm=c_e2e)
-        comp_done[sl].record(c_e2e)
+            stream.wait_event(out_read[sl])    # step i-2's results have left this slot
+        decode(i, q_in=q_d[sl], out_buf=out_d[sl], lse_buf=lse_d[sl])
+        encode(i, xk=xk_d[sl], xv=xv_d[sl])
+        comp_done[sl].record(stream)
         s_out.wait_event(comp_done[sl])
         with torch.cuda.stream(s_out):
             for ho, do in zip(out_h[sl], out_d[sl]):
@@ -735,49 +731,21 @@ def main():
                 hl.copy_(dl, non_blocking=True)
         out_read[sl].record(s_out)
 
-    def e2e_block(n_steps, first):
-        # the copy streams fork from and join back to the compute stream
-        s_in.wait_stream(c_e2e)
-        s_out.wait_stream(c_e2e)
-        for j in range(n_steps):
-            e2e_step(first + j)
-        c_e2e.wait_stream(s_in)
-        c_e2e.wait_stream(s_out)
-
     for i in range(min(args.warmup, 10)):
         e2e_step(i)
     torch.cuda.synchronize()
-    # Replay the steps from a CUDA graph (G steps per graph: copies, kernels, cross-stream
-    # ordering), so the host issues one launch per G steps instead of ~15 calls per step.
-    G = 8
-    graph = None
-    try:
-        graph = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(graph, stream=c_e2e):
-            e2e_block(G, 0)
-        torch.cuda.synchronize()
-    except Exception as exc:  # capture unavailable: fall back to issuing the steps one by one
-        graph = None
-        graph_error = f"{type(exc).__name__}: {exc}"[:200]
-        torch.cuda.synchronize()
     if world > 1:
         dist.barrier()
     e0 = torch.cuda.Event(enable_timing=True)
     e1 = torch.cuda.Event(enable_timing=True)
-    if graph is not None:
-        n_rep = max(1, e2e_steps // G)
-        e2e_steps = n_rep * G
-        graph.replay()  # warm the graph
-        torch.cuda.synchronize()
-        e0.record(c_e2e)
-        with torch.cuda.stream(c_e2e):
-            for _ in range(n_rep):
-                graph.replay()
-        e1.record(c_e2e)
-    else:
-        e0.record(c_e2e)
-        e2e_block(e2e_steps, 0)
-        e1.record(c_e2e)
+    e0.record(s_in)
+    stream.wait_event(e0)
+    s_out.wait_event(e0)
+    for i in range(e2e_steps):
+        e2e_step(i)
+    s_out.wait_stream(s_in)
+    s_out.wait_stream(stream)
+    e1.record(s_out)
     torch.cuda.synchronize()
     e2e_ms = max_over_ranks(e0.elapsed_time(e1), dev)
     e2e_value = world * step_bytes * e2e_steps / (e2e_ms * 1e-3) / 1e9
@@ -828,9 +796,7 @@ def main():
         "e2e": {"value": e2e_value, "unit": "GB/s", "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "steps": e2e_steps,
                 "copies": "pinned host buffers; two device slots, input and result copies on "
-                          "their own streams overlap the neighbouring steps' kernels",
-                "issue": (f"CUDA graph of {G} steps, replayed" if graph is not None
-                          else f"steps issued one by one (graph capture failed: {graph_error})")},
+                          "their own streams overlap the neighbouring steps' kernels"},
         "gpu_launches": launches_per_step * args.steps,
         "clocks": clocks,
     }
