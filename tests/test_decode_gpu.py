@@ -190,3 +190,15 @@ def test_timed_entry_matches_decode_and_times_the_grid():
     assert lla.status_fetch(ws) == 0
     assert torch.equal(out2, out) and torch.equal(lse2, lse)
     assert 0 < e0.elapsed_time(e1) < c0.elapsed_time(c1)
+
+
+@pytest.mark.parametrize("Tq,t0", [(12, 0), (9, 3)])
+def test_more_than_eight_loop_queries_small_ranks(Tq, t0):
+    """T = 12 loops at ranks 16/32: fragment rows g + 8 of the tensor-core tile carry loop
+    queries (the 16-row variant of the small-rank kernel)."""
+    w = S.shrink(S.WORKLOADS["ouro1.4b-layer"], name="T12", T=12, L=1, B=6, len_lo=100, len_hi=2000)
+    p = S.decode_inputs(w, 0, "cuda", Tq=Tq)
+    out, lse, st = run_decode(p, w, 0, t0, Tq, 1.0)
+    assert st == 0
+    o_ref, l_ref = oracle_decode(p, w, 0, t0, Tq, 1.0)
+    assert_attn_close(out, lse, o_ref, l_ref)

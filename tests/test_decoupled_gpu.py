@@ -54,3 +54,10 @@ def test_decoupled_full_layer_sampled():
     w = S.WORKLOADS["ouro1.4b-layer"]
     lens = S.context_lengths(w)
     _case(w, lens, 64, 10000.0, lla.ROPE_HALF, Tq=4, t0=0, q_pos=lens, units_per_seq=1)
+
+
+def test_decoupled_more_than_eight_loop_queries():
+    """T = 12 loops, all 12 loop queries in one pass: the fragment rows g + 8 carry queries
+    (the kernel's 16-row variant)."""
+    w = S.shrink(S.WORKLOADS["ouro1.4b-layer"], name="dec-T12", T=12, L=2, B=len(CTX_LENS))
+    _case(w, CTX_LENS, 32, 10000.0, lla.ROPE_HALF, Tq=12, t0=0, q_pos=CTX_LENS, units_per_seq=2)
