@@ -319,3 +319,30 @@ def test_encode_argument_errors():
     assert rc(x_v=0) == lla.LLA_ERR_INVALID
     assert rc(n_tok=0) == 0
     assert rc(dims=lla.make_dims(4, 2, 16, 128, 320, 160)) == lla.LLA_ERR_UNSUPPORTED
+
+
+def test_plain_c_program_links_and_calls_the_library(tmp_path):
+    """The header is plain C99 and a C program linked against liblla.so gets the exact
+    accounting of the 768 x 4096-token capacity case (no device needed)."""
+    import subprocess
+    src = tmp_path / "main.c"
+    src.write_text(r'''
+#include <stdio.h>
+#include "lla.h"
+int main(void)
+{
+    lla_dims d = {4, 24, 16, 128, 16, 32, LLA_PER_HEAD, LLA_BF16, LLA_F32};
+    int32_t lens[768];
+    for (int i = 0; i < 768; ++i) lens[i] = 4096;
+    uint64_t lat = 0, unc = 0, num = 0, den = 0;
+    int rc = lla_cache_bytes(&d, lens, 768, &lat, &unc, &num, &den);
+    printf("%d %llu %llu %llu\n", rc, (unsigned long long)lat, (unsigned long long)num, (unsigned long long)den);
+    return rc;
+}
+''')
+    exe = tmp_path / "main"
+    libdir = os.path.dirname(lla.LIB_PATH)
+    subprocess.check_call(["gcc", "-std=c99", "-Wall", "-Wextra", "-pedantic", "-I", os.path.join(ROOT, "include"),
+                           str(src), "-L", libdir, "-llla", "-Wl,-rpath," + libdir, "-o", str(exe)])
+    out = subprocess.check_output([str(exe)], text=True).split()
+    assert out == ["0", "115964116992", "64", "3"]
