@@ -46,11 +46,7 @@ template <int R> struct ResCfg {
     static constexpr int STAGE = P1 > P2 ? P1 : P2;
     static constexpr int CS_LD = R + 4;                     // fp32 row stride of c
     static constexpr int CS_OFF = STAGES * STAGE;
-    // small ranks: each W_up chunk is split into tf32 (hi, lo) pairs once per CTA and
-    // shared by the four warps (room for it only when R <= 64)
-    static constexpr bool PRESPLIT = R <= 64;
-    static constexpr int WS_OFF = CS_OFF + kResWarps * 16 * CS_LD * 4;
-    static constexpr int SMEM = WS_OFF + (PRESPLIT ? R * WU_LD * 8 : 0);
+    static constexpr int SMEM = CS_OFF + kResWarps * 16 * CS_LD * 4;
 };
 
 struct ResArgs {
@@ -207,23 +203,10 @@ __global__ void __launch_bounds__(kResThreads) codec_residual_kernel(const ResAr
         const uint8_t *xg = rsm + (xs - sb);
         const float *wu = reinterpret_cast<const float *>(xg + C::X_BYTES);
         const float *mus = reinterpret_cast<const float *>(xg + C::X_BYTES + C::WU_BYTES);
-        uint2 *wsplit = reinterpret_cast<uint2 *>(rsm + C::WS_OFF);
-        if (C::PRESPLIT) {
-            for (int e = tid; e < R * kChunk; e += kResThreads) {
-                const int j = e / kChunk, c = e - j * kChunk;
-                uint32_t hi, lo;
-                split_tf32(wu[j * C::WU_LD + c], hi, lo);
-                wsplit[j * C::WU_LD + c] = make_uint2(hi, lo);
-            }
-            __syncthreads();
-        }
-        float o[8][4]; // accumulators start at mu_t: the MMAs add c W_up on top
+        float o[8][4];
 #pragma unroll
-        for (int n = 0; n < 8; ++n) {
-            const float2 m2 = *reinterpret_cast<const float2 *>(mus + 8 * n + 2 * tq);
-            o[n][0] = o[n][2] = m2.x;
-            o[n][1] = o[n][3] = m2.y;
-        }
+        for (int n = 0; n < 8; ++n)
+            o[n][0] = o[n][1] = o[n][2] = o[n][3] = 0.f;
 #pragma unroll 2
         for (int ks = 0; ks < R / 8; ++ks) {
             uint32_t ah[4], al[4];
@@ -234,14 +217,8 @@ __global__ void __launch_bounds__(kResThreads) codec_residual_kernel(const ResAr
 #pragma unroll
             for (int n = 0; n < 8; ++n) {
                 uint32_t bh0, bl0, bh1, bl1;
-                if (C::PRESPLIT) {
-                    const uint2 b0 = wsplit[(8 * ks + tq) * C::WU_LD + 8 * n + g];
-                    const uint2 b1 = wsplit[(8 * ks + tq + 4) * C::WU_LD + 8 * n + g];
-                    bh0 = b0.x, bl0 = b0.y, bh1 = b1.x, bl1 = b1.y;
-                } else {
-                    split_tf32(wu[(8 * ks + tq) * C::WU_LD + 8 * n + g], bh0, bl0);
-                    split_tf32(wu[(8 * ks + tq + 4) * C::WU_LD + 8 * n + g], bh1, bl1);
-                }
+                split_tf32(wu[(8 * ks + tq) * C::WU_LD + 8 * n + g], bh0, bl0);
+                split_tf32(wu[(8 * ks + tq + 4) * C::WU_LD + 8 * n + g], bh1, bl1);
                 mma1688(o[n], ah, bh0, bh1);
                 mma1688(o[n], ah, bl0, bl1);
                 mma1688(o[n], al, bh0, bh1);
@@ -249,12 +226,13 @@ __global__ void __launch_bounds__(kResThreads) codec_residual_kernel(const ResAr
         }
 #pragma unroll
         for (int n = 0; n < 8; ++n) {
+            const int c = 8 * n + 2 * tq;
 #pragma unroll
             for (int hrow = 0; hrow < 2; ++hrow) {
                 const int r = 16 * warp + g + 8 * hrow;
                 const uint32_t xv = *reinterpret_cast<const uint32_t *>(xg + swz(r, n) + 4 * tq);
                 const float x0 = bf16_lo(xv), x1 = bf16_hi(xv);
-                const float d0 = x0 - o[n][2 * hrow], d1 = x1 - o[n][2 * hrow + 1];
+                const float d0 = x0 - (o[n][2 * hrow] + mus[c]), d1 = x1 - (o[n][2 * hrow + 1] + mus[c + 1]);
                 e2[hrow] = fmaf(d0, d0, fmaf(d1, d1, e2[hrow]));
                 n2s[hrow] = fmaf(x0, x0, fmaf(x1, x1, n2s[hrow]));
             }
