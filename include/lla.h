@@ -200,8 +200,10 @@ int lla_codec_residual(const lla_dims *dims, int32_t layer0, int32_t n_layers, c
  *   num_splits  target number of token shares (split-K pieces) per (sequence, head);
  *               0 = automatic.  The token stream of all (sequence, head) pairs is cut
  *               into one equal share per resident CTA, never fewer than
- *               ceil(max_ctx / num_splits) tokens.  Results are bitwise reproducible
- *               for equal arguments.
+ *               ceil(max_ctx / num_splits) tokens (automatic: ceil(max_ctx / s) with s
+ *               about twice the resident CTAs per unit, and at least 128 tokens, or 256
+ *               for the LLA-2D kernel, whose units are whole sequences).  Results are
+ *               bitwise reproducible for equal arguments.
  *   workspace   device scratch of at least lla_decode_workspace_bytes(...) bytes; its
  *               contents need not be initialised (the first word, the status, must be
  *               zero -- lla_status_fetch leaves it so)
