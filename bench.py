@@ -575,8 +575,24 @@ def main():
                             max_ctx, codec, 1.0, (out_buf or outs)[c], (lse_buf or lses)[c], ws, ws_bytes,
                             variant=variant, num_splits=args.num_splits, stream=stream)
 
-    def encode(i, xk=x_k, xv=x_v):
-        lla.encode(dims, 0, 1, xk, xv, B, new_slot, codec, caches[i % R], stream=stream)
+    def encode(i, xk=x_k, xv=x_v, strm=None):
+        lla.encode(dims, 0, 1, xk, xv, B, new_slot, codec, caches[i % R],
+                   stream=strm if strm is not None else stream)
+
+    # The encode of the finished tokens writes each sequence's next slot, which no decode
+    # of the step reads: it runs on a side stream forked at the step's start and joined at
+    # its end, so its CTAs can take the SM slots the decode grid frees.
+    s_enc = torch.cuda.Stream(dev)
+
+    def step(i, q_in=None, out_buf=None, lse_buf=None, xk=x_k, xv=x_v, ev_a=None, ev_b=None):
+        if ev_a is not None:
+            ev_a.record(stream)
+        s_enc.wait_stream(stream)
+        encode(i, xk=xk, xv=xv, strm=s_enc)
+        decode(i, q_in=q_in, out_buf=out_buf, lse_buf=lse_buf)
+        if ev_b is not None:
+            ev_b.record(stream)
+        stream.wait_stream(s_enc)
 
     # per decode call: prologue + decode + combine (reconstruct: one decode pass per loop
     # query + combine); the encode of K and V is one launch
@@ -585,8 +601,7 @@ def main():
     # ---- warm-up, then the device-timed region ------------------------------------------------
     sampler = ClockSampler(local).start()
     for i in range(args.warmup):
-        decode(i)
-        encode(i)
+        step(i)
     torch.cuda.synchronize()
     ev_a = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
     ev_b = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
@@ -598,10 +613,7 @@ def main():
     wall0 = time.perf_counter()
     t_start.record(stream)
     for i in range(args.steps):
-        ev_a[i].record(stream)
-        decode(i)
-        ev_b[i].record(stream)
-        encode(i)
+        step(i, ev_a=ev_a[i], ev_b=ev_b[i])
     t_end.record(stream)
     torch.cuda.synchronize()
     wall1 = time.perf_counter()
@@ -734,8 +746,7 @@ def main():
         stream.wait_event(in_ready[sl])
         if i >= 2:
             stream.wait_event(out_read[sl])    # step i-2's results have left this slot
-        decode(i, q_in=q_d[sl], out_buf=out_d[sl], lse_buf=lse_d[sl])
-        encode(i, xk=xk_d[sl], xv=xv_d[sl])
+        step(i, q_in=q_d[sl], out_buf=out_d[sl], lse_buf=lse_d[sl], xk=xk_d[sl], xv=xv_d[sl])
         comp_done[sl].record(stream)
         s_out.wait_event(comp_done[sl])
         with torch.cuda.stream(s_out):
