@@ -785,3 +785,31 @@ def test_codec_fit_shift_moves_only_the_mean():
     np.testing.assert_allclose(b[0], a[0] + shift, atol=1e-12)
     np.testing.assert_allclose(b[1], a[1], atol=1e-9)
     np.testing.assert_allclose(b[3], a[3], rtol=1e-10, atol=1e-10 * a[3][0])  # last one is ~0 (rank n-1)
+
+
+def test_decode_layer_rope_with_folded_heads():
+    """LLA-2D codec with the faithful read: head h rebuilds its column slice of the folded
+    up-projection, then rotates it; against dense SDPA over keys rotated in complex form."""
+    T, H, d, rk, rv = 2, 3, 8, 5, 7
+    lens = np.array([6, 0, 3], dtype=np.int32)
+    q_pos = np.array([6, 2, 40])
+    starts, c_K, c_V, WK, mK, WV, mV = _ragged_layer(T, H, d, lens, rk, rv, True, 30)
+    B, Tq, t0, s, base = len(lens), 2, 0, 0.9, 300.0
+    q = np.random.default_rng(31).standard_normal((B, Tq, H, d))
+    o, lse = oracle.decode_layer("reconstruct", q, c_K, c_V, starts, lens, WK, mK, WV, mV, t0, s,
+                                 fold2d=True, threads=2, rope=(q_pos, base, oracle.ROPE_INTERLEAVED))
+    for b in range(B):
+        sl = slice(int(starts[b]), int(starts[b] + lens[b]))
+        for tq in range(Tq):
+            for h in range(H):
+                if lens[b] == 0:
+                    assert np.all(o[b, tq, h] == 0) and lse[b, tq, h] == -np.inf
+                    continue
+                cols = slice(h * d, (h + 1) * d)
+                Kh = c_K[0, sl] @ WK[t0 + tq][:, cols] + mK[t0 + tq][cols]
+                Vh = c_V[0, sl] @ WV[t0 + tq][:, cols] + mV[t0 + tq][cols]
+                Kr = _rotate_complex(Kh, np.arange(lens[b]), base, oracle.ROPE_INTERLEAVED)
+                qr = _rotate_complex(q[b, tq, h], q_pos[b], base, oracle.ROPE_INTERLEAVED)
+                o_ref, lse_ref = sdpa(qr, Kr, Vh, s)
+                np.testing.assert_allclose(o[b, tq, h], o_ref, atol=1e-11)
+                assert lse[b, tq, h] == pytest.approx(lse_ref, abs=1e-11)
