@@ -134,37 +134,73 @@ def test_mutant_is_caught(name, tmp_path):
     assert failed, f"mutant {name} survived every pin"
 
 
-# Mutants of the numpy-level codec fit: the function's source is edited, compiled in the
-# oracle module's namespace and swapped in while the fit pins run.
+# Mutants of the numpy-level oracle functions (the codec fit, and the per-sequence, per-loop
+# and per-head slicing of a decode layer): the function's source is edited, compiled in the
+# oracle module's namespace and swapped in while that function's pins run.
 PY_MUTANTS = {
-    "fit_not_centred": ("np.linalg.svd(x - mu[None, :], full_matrices=False)",
+    "fit_not_centred": ("codec_fit", "np.linalg.svd(x - mu[None, :], full_matrices=False)",
                         "np.linalg.svd(x, full_matrices=False)"),
-    "fit_left_vectors": ("W_down = Vt[:r].T.copy()", "W_down = _[:, :r].copy()"),
-    "fit_no_sign_convention": ("W_down *= sign[None, :]", "pass"),
-    "fit_up_layout": ("W_up = W_down.reshape(T, W // T, r).transpose(0, 2, 1).copy()",
+    "fit_left_vectors": ("codec_fit", "W_down = Vt[:r].T.copy()", "W_down = _[:, :r].copy()"),
+    "fit_no_sign_convention": ("codec_fit", "W_down *= sign[None, :]", "pass"),
+    "fit_up_layout": ("codec_fit", "W_up = W_down.reshape(T, W // T, r).transpose(0, 2, 1).copy()",
                       "W_up = W_down.reshape(r, T, W // T).transpose(1, 0, 2).copy()"),
+    "layer_ignores_first_loop": ("decode_layer", "wk, mk, wv, mv = slices(h, t0 + tq)",
+                                 "wk, mk, wv, mv = slices(h, tq)"),
+    "layer_ignores_seq_start": ("decode_layer", "cK = c_K[hp, s0:s0 + n]", "cK = c_K[hp, :n]"),
+    "layer_values_ignore_seq_start": ("decode_layer", "cV = c_V[hp, s0:s0 + n]", "cV = c_V[hp, :n]"),
+    "layer_always_plane_zero": ("decode_layer", "hp = 0 if fold2d else h", "hp = 0"),
+    "layer_fold2d_column_slice": ("decode_layer", "cols = slice(h * d, (h + 1) * d)",
+                                  "cols = slice(h, h + d)"),
+    "layer_per_head_index_swapped": ("decode_layer", "return W_up_K[h][t], mu_K[h][t]",
+                                     "return W_up_K[t % len(W_up_K)][h % len(W_up_K[0])], mu_K[h][t]"),
+    "layer_window_loop_index": ("decode_layer", "win_k[b, h, t0 + tq, :nw]", "win_k[b, h, tq, :nw]"),
+    "layer_window_values_are_keys": ("decode_layer", "win_v[b, h, t0 + tq, :nw]",
+                                     "win_k[b, h, t0 + tq, :nw]"),
+    "layer_subkeys_ignore_seq_start": ("decode_layer", "k_rope[hp, s0:s0 + n]", "k_rope[hp, :n]"),
+    "layer_decoupled_position_of_sequence_zero": ("decode_layer", "float(q_pos[b]))\n            elif rope",
+                                                  "float(q_pos[0]))\n            elif rope"),
+    "layer_rope_position_of_sequence_zero": ("decode_layer", "float(q_pos[b]))\n            elif window",
+                                             "float(q_pos[0]))\n            elif window"),
 }
+
+PY_PINS = {
+    "codec_fit": [(P.test_codec_fit_recovers_planted_orthogonal_directions, {}),
+                  (P.test_codec_fit_energy_and_orthonormality, {}),
+                  (P.test_codec_fit_shift_moves_only_the_mean, {})],
+    "decode_layer": [(P.test_decode_layer_matches_masked_dense_attention, {"fold2d": False}),
+                     (P.test_decode_layer_matches_masked_dense_attention, {"fold2d": True}),
+                     (P.test_decode_layer_hybrid_matches_dense_attention_over_both_parts, {"fold2d": False}),
+                     (P.test_decode_layer_rope_matches_dense_rotated_attention, {"style": 1}),
+                     (P.test_decode_layer_rope_with_folded_heads, {}),
+                     (P.test_decode_layer_decoupled_matches_dense_attention, {}),
+                     (P.test_fold2d_full_rank_reproduces_each_head, {"variant": "absorb"})],
+}
+
+
+def test_unmutated_python_oracle_passes_its_pins():
+    for pins in PY_PINS.values():
+        for fn, kw in pins:
+            fn(**kw)
 
 
 @pytest.mark.parametrize("name", sorted(PY_MUTANTS))
 def test_python_mutant_is_caught(name):
     import inspect
     import textwrap
-    old, new = PY_MUTANTS[name]
-    src = textwrap.dedent(inspect.getsource(oracle.codec_fit))
+    target, old, new = PY_MUTANTS[name]
+    src = textwrap.dedent(inspect.getsource(getattr(oracle, target)))
     assert src.count(old) == 1, f"mutation site for {name} not unique"
     ns = dict(vars(oracle))
     exec(compile(src.replace(old, new), "<mutant>", "exec"), ns)
-    saved = oracle.codec_fit
-    oracle.codec_fit = ns["codec_fit"]
+    saved = getattr(oracle, target)
+    setattr(oracle, target, ns[target])
     failed = []
     try:
-        for fn in (P.test_codec_fit_recovers_planted_orthogonal_directions,
-                   P.test_codec_fit_energy_and_orthonormality, P.test_codec_fit_shift_moves_only_the_mean):
+        for fn, kw in PY_PINS[target]:
             try:
-                fn()
+                fn(**kw)
             except (AssertionError, ValueError, IndexError, FloatingPointError):
                 failed.append(fn.__name__)
     finally:
-        oracle.codec_fit = saved
+        setattr(oracle, target, saved)
     assert failed, f"mutant {name} survived every pin"
