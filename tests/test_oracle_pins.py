@@ -813,3 +813,31 @@ def test_decode_layer_rope_with_folded_heads():
                 o_ref, lse_ref = sdpa(qr, Kr, Vh, s)
                 np.testing.assert_allclose(o[b, tq, h], o_ref, atol=1e-11)
                 assert lse[b, tq, h] == pytest.approx(lse_ref, abs=1e-11)
+
+
+@pytest.mark.parametrize("variant", VARIANTS)
+def test_tiny_workload_against_brute_force_without_max_subtraction(variant):
+    """The 64-token fp32 workload exactly as generated (fitted low-rank codec, all four
+    loops): the oracle against a third expression written with Python loops and exact
+    sums, exp of the raw logits with no max subtraction, normalised at the end."""
+    w = S.WORKLOADS["tiny-fp32"]
+    p = S.decode_inputs(w, 0, "cpu")
+    to64 = lambda t: t.double().numpy()
+    cK, cV = to64(p["k"][0]), to64(p["v"][0])
+    WK, WV, mK, mV = (to64(p[k][0]) for k in ("W_up_k", "W_up_v", "mu_k", "mu_v"))
+    q = to64(p["q"])
+    n = int(p["lens"][0])
+    s0 = int(p["starts"][0])
+    o, lse = oracle.decode_layer(variant, q, cK, cV, p["starts"], p["lens"], WK, mK, WV, mV,
+                                 0, 1.0, threads=1)
+    for t in range(w.T):
+        for h in range(w.H):
+            Kh = [[math.fsum([cK[h, s0 + i, j] * WK[h, t, j, k] for j in range(w.r_k)]) + mK[h, t, k]
+                   for k in range(w.d)] for i in range(n)]
+            Vh = [[math.fsum([cV[h, s0 + i, j] * WV[h, t, j, k] for j in range(w.r_v)]) + mV[h, t, k]
+                   for k in range(w.d)] for i in range(n)]
+            e = [math.exp(math.fsum([q[0, t, h, k] * Kh[i][k] for k in range(w.d)])) for i in range(n)]
+            Z = math.fsum(e)
+            o_ref = [math.fsum([e[i] * Vh[i][k] for i in range(n)]) / Z for k in range(w.d)]
+            np.testing.assert_allclose(o[0, t, h], o_ref, atol=1e-12, rtol=0)
+            assert lse[0, t, h] == pytest.approx(math.log(Z), abs=1e-12)
