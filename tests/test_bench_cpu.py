@@ -1,6 +1,8 @@
 """CPU tests of the benchmark's host logic: the max-over-ranks reduction on a
-world-size-2 gloo group, and the reference arm (the fp64 oracle) in one process and
-under torchrun with two ranks (rank 0 alone prints its one JSON line)."""
+world-size-2 gloo group, the reference arm (the fp64 oracle) in one process and
+under torchrun with two ranks (rank 0 alone prints its one JSON line), the clock
+record (median SM clock and throttle reasons of the samples inside the timed region),
+the stale-profile check of the traffic figure, and the peak lookup with its fallback."""
 import json
 import os
 import socket
@@ -76,3 +78,76 @@ def test_reference_arm_two_ranks_torchrun():
     assert r.returncode == 0, r.stderr[-2000:]
     lines = _json_lines(r.stdout)
     assert len(lines) == 1 and lines[0]["impl"] == "reference" and lines[0]["n_gpus"] == 2
+
+
+# ---------------------------------------------------------------------------
+# clock record, stale-profile detection and peak lookup (pure host logic)
+# ---------------------------------------------------------------------------
+def _sampler_with(samples, max_mhz=1965):
+    import bench
+    s = bench.ClockSampler.__new__(bench.ClockSampler)
+    s.samples, s.ok, s.max_mhz = samples, True, max_mhz
+    return s
+
+
+def test_clock_summary_median_and_reasons_inside_the_region():
+    R = __import__("bench").ClockSampler.REASONS
+    samples = [(0.5, 900, R["hw_slowdown"]),                # before the region: ignored
+               (1.0, 1800, R["gpu_idle"]), (1.1, 1900, R["sw_power_cap"]), (1.2, 1950, 0),
+               (3.0, 700, R["sw_thermal_slowdown"])]         # after: ignored
+    out = _sampler_with(samples).summary(1.0, 1.2)
+    assert out["sm_mhz"] == 1900 and out["sm_max_mhz"] == 1965 and out["samples"] == 3
+    assert out["reasons"] == ["sw_power_cap"]                # gpu_idle is not a throttle reason
+
+
+def test_clock_summary_short_region_takes_the_nearest_samples():
+    R = __import__("bench").ClockSampler.REASONS
+    samples = [(0.0, 1000, 0), (1.0, 1500, R["hw_thermal_slowdown"]), (1.01, 1600, 0),
+               (1.02, 1700, 0), (5.0, 500, R["hw_slowdown"])]
+    out = _sampler_with(samples).summary(1.004, 1.006)       # no sample inside
+    assert out["samples"] == 3 and out["sm_mhz"] == 1600
+    assert out["reasons"] == ["hw_thermal_slowdown"]
+
+
+def test_clock_summary_without_nvml():
+    s = _sampler_with([], max_mhz=None)
+    s.ok = False
+    assert s.summary(0.0, 1.0) == {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+
+
+def test_profiled_traffic_scales_per_unit_and_rejects_stale_profiles(tmp_path, monkeypatch):
+    import bench
+    path = tmp_path / "prof.json"
+    prof = {"source_hash": bench.kernel_source_hash("absorb"), "dram_bytes_per_launch": 3.0e8,
+            "units_per_launch": 1.0e6}
+    path.write_text(json.dumps(prof))
+    monkeypatch.setitem(bench.PROFILE_TRAFFIC, "absorb", str(path))
+    assert bench.profiled_traffic(2.0e6, "absorb") == pytest.approx(6.0e8)
+    prof["source_hash"] = "0" * 16                            # taken on other kernel sources
+    path.write_text(json.dumps(prof))
+    assert bench.profiled_traffic(2.0e6, "absorb") is None
+    path.write_text("not json")
+    assert bench.profiled_traffic(2.0e6, "absorb") is None
+    monkeypatch.setitem(bench.PROFILE_TRAFFIC, "absorb", str(tmp_path / "absent.json"))
+    assert bench.profiled_traffic(2.0e6, "absorb") is None
+
+
+def test_committed_traffic_summaries_are_well_formed():
+    """Each committed traffic summary names the hash of the sources it was taken on; the
+    bench reports traffic only while they match (otherwise null)."""
+    import bench
+    for variant, path in bench.PROFILE_TRAFFIC.items():
+        with open(path) as f:
+            prof = json.load(f)
+        assert prof["units_per_launch"] > 0 and prof["dram_bytes_per_launch"] > 0
+        assert len(prof["source_hash"]) == 16
+
+
+def test_measured_peaks_fall_back_when_the_file_is_absent(tmp_path, monkeypatch):
+    import bench
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    peaks, kind = bench.measured_peaks()
+    assert kind == "fallback" and peaks["hbm_gbs"] == 6650.0 and peaks["bf16_tflops"] == 1590.0
+    (tmp_path / "MEASURED_PEAKS.json").write_text(json.dumps({"hbm_gbs": 6543.1}))
+    peaks, kind = bench.measured_peaks()
+    assert kind == "measured" and peaks["hbm_gbs"] == 6543.1
