@@ -145,10 +145,16 @@ def make_dims(T, L, H, d_head, r_k, r_v, fold=PER_HEAD, dtype=BF16, out_dtype=F3
 
 
 def _ptr(t) -> Optional[int]:
+    """Device address of a buffer: None, a raw address, or a tensor.  The library takes
+    dense row-major buffers (no strides cross the ABI), so a strided view is refused
+    rather than read as if it were dense."""
     if t is None:
         return None
     if isinstance(t, int):
         return t
+    if not t.is_contiguous():
+        raise ValueError(f"liblla takes dense row-major buffers; got a strided view of shape "
+                         f"{tuple(t.shape)} with strides {tuple(t.stride())} (call .contiguous())")
     return t.data_ptr()
 
 

@@ -346,3 +346,18 @@ int main(void)
                            str(src), "-L", libdir, "-llla", "-Wl,-rpath," + libdir, "-o", str(exe)])
     out = subprocess.check_output([str(exe)], text=True).split()
     assert out == ["0", "115964116992", "64", "3"]
+
+
+def test_binding_refuses_strided_views():
+    """No strides cross the ABI: the binding passes dense buffers' addresses and refuses a
+    strided view instead of letting the library read it as dense."""
+    import torch
+    dense = torch.zeros(4, 6)
+    assert lla._ptr(dense) == dense.data_ptr()
+    assert lla._ptr(dense[1:3]) == dense[1:3].data_ptr()       # a row range is still dense
+    assert lla._ptr(None) is None and lla._ptr(12345) == 12345
+    for view in (dense.t(), dense[:, 1:3], dense[:, None].expand(4, 2, 6)):
+        with pytest.raises(ValueError, match="dense row-major"):
+            lla._ptr(view)
+    with pytest.raises(ValueError):
+        lla.make_cache(dense.t(), dense, 4)
