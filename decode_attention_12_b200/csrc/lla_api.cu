@@ -1,6 +1,7 @@
 // lla_api.cu -- the C ABI of liblla (declared in include/lla.h): argument checks,
 // kernel selection, workspace carving, status handling.  Every arithmetic step of
 // the path runs in the kernels; this file only validates and launches.
+#include <atomic>
 #include <climits>
 #include <cmath>
 #include <cstring>
@@ -43,19 +44,21 @@ int heads_stored(const lla_dims *d) { return d->fold ? 1 : d->H; }
 int64_t stack_width(const lla_dims *d) { return (int64_t)d->T * d->d_head * (d->fold ? d->H : 1); }
 int64_t loop_width(const lla_dims *d) { return (int64_t)d->d_head * (d->fold ? d->H : 1); }
 
+// SM count of the current device, looked up once per device (atomic: the library may be
+// called from several host threads at once).
 int sm_count()
 {
-    static int cached[64] = {0};
+    static std::atomic<int> cached[64];
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64)
         return 148;
-    if (cached[dev] == 0) {
-        int n = 0;
+    int n = cached[dev].load(std::memory_order_relaxed);
+    if (n == 0) {
         if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
             n = 148;
-        cached[dev] = n;
+        cached[dev].store(n, std::memory_order_relaxed);
     }
-    return cached[dev];
+    return n;
 }
 
 // Plan of one decode call: the work split of the persistent decode kernel and the
