@@ -20,15 +20,19 @@
  *
  * General conventions
  *  - Every pointer is caller-owned; the library allocates nothing and keeps no
- *    state between calls.  Pointers named *_host are host memory; all others are
- *    device memory of the current CUDA device.
+ *    problem state between calls (only per-device lookups such as the SM count,
+ *    safe under concurrent host threads).  Pointers named *_host are host memory;
+ *    all others are device memory of the current CUDA device.
  *  - Device work is enqueued on `stream`, asynchronously; no call synchronises
  *    the host except lla_status_fetch.  No exception crosses the ABI.
  *  - Arrays are dense and row-major in the index order written next to them.
  *    Storage type "T" is the `dtype` of lla_dims (fp32 or bf16); codec tensors
  *    other than W_down are always fp32.  bf16 values are rounded to nearest-even.
- *  - Return value: LLA_OK or one of the negative LLA_ERR_* codes below; on an
- *    error nothing has been enqueued.  Device pointers must be 16-byte aligned.
+ *  - Return value: LLA_OK or one of the negative LLA_ERR_* codes below.  On an
+ *    argument error (LLA_ERR_INVALID, _UNSUPPORTED, _MISALIGNED, _WORKSPACE) nothing
+ *    has been enqueued; LLA_ERR_CUDA reports a failed launch or copy, and grids of
+ *    the same call launched before it may already be enqueued.  Device pointers
+ *    must be 16-byte aligned.
  */
 #ifndef LLA_H_
 #define LLA_H_
