@@ -52,6 +52,9 @@ MUTANTS = {
     "residual_first_loop_block_only": ("W_up + (int64_t)t * r * Dp", "W_up"),
     "residual_norm_of_rebuilt": ("n2 += xi[t * Dp + k] * xi[t * Dp + k];", "n2 += x_hat[k] * x_hat[k];"),
     "residual_squared": ("err[i] = sqrt(e2);", "err[i] = e2;"),
+    "residual_encodes_with_up_projection": ("oracle_encode(1, W, r, xi, mu, W_down, c);",
+                                            "oracle_encode(1, W, r, xi, mu, W_up, c);"),
+    "residual_up_block_stride": ("W_up + (int64_t)t * r * Dp", "W_up + (int64_t)t * Dp"),
     "decoupled_drops_rope_term": ("l[i] = scale * (dn + dr);", "l[i] = scale * dn;"),
     "decoupled_query_not_rotated": ("rope_rotate(d_r, style, base, q_pos, qr);", ""),
     "decoupled_rope_term_unscaled": ("l[i] = scale * (dn + dr);", "l[i] = scale * dn + dr;"),
@@ -91,6 +94,7 @@ def _pins():
         (P.test_residual_energy_on_calibration_set_is_the_svd_tail, {"r": 5}),
         (P.test_residual_of_in_span_and_orthogonal_offsets, {}),
         (P.test_residual_is_homogeneous_in_the_centred_vector, {}),
+        (P.test_residual_with_differently_scaled_down_and_up_projections, {}),
     ]
     for v in P.VARIANTS:
         pins += [

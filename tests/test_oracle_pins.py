@@ -635,6 +635,26 @@ def test_residual_of_in_span_and_orthogonal_offsets():
     np.testing.assert_allclose(norm_out, np.linalg.norm(mu + v, axis=1), rtol=1e-13)
 
 
+def test_residual_with_differently_scaled_down_and_up_projections():
+    """W_down = alpha Q_r and W_up,t = beta (t-block of Q_r)^T with Q_r orthonormal: for
+    x = mu + a Q_r^T + v (v orthogonal to the span) the definition gives
+    ||x - x_hat||^2 = (1 - alpha beta)^2 ||a||^2 + ||v||^2, which tells the two projections'
+    roles apart (SVD codecs, where W_up = W_down^T, cannot)."""
+    T, d, r, alpha, beta = 3, 8, 5, 2.0, 0.25
+    rng = np.random.default_rng(66)
+    Q, _ = np.linalg.qr(rng.standard_normal((T * d, T * d)))
+    Qr = Q[:, :r]
+    Wd = alpha * Qr
+    Wu = beta * Qr.reshape(T, d, r).transpose(0, 2, 1)
+    mu = rng.standard_normal(T * d)
+    a = rng.standard_normal((9, r))
+    b = rng.standard_normal((9, T * d - r))
+    x = mu + a @ Qr.T + b @ Q[:, r:].T
+    err, _ = oracle.codec_residual(x, mu, Wd, Wu)
+    ref = np.sqrt((1 - alpha * beta) ** 2 * (a ** 2).sum(axis=1) + (b ** 2).sum(axis=1))
+    np.testing.assert_allclose(err, ref, rtol=1e-12)
+
+
 def test_residual_is_homogeneous_in_the_centred_vector():
     """x - x_hat is linear in y = x - mu for any codec (W_up need not be W_down^T), so
     scaling y by s scales the residual by |s|."""
