@@ -79,6 +79,16 @@ def parse():
     return ap.parse_args()
 
 
+def rho_label(w) -> str:
+    """Exact compression ratio of a workload as a reduced fraction: 2 T d / (r_k + r_v) per
+    head per layer, with the H heads folded into one latent for LLA-2D."""
+    num = 2 * w.T * w.d * (w.H if w.fold2d else 1)
+    den = w.r_k + w.r_v
+    g = math.gcd(num, den)
+    num, den = num // g, den // g
+    return str(num) if den == 1 else f"{num}/{den}"
+
+
 def measured_peaks():
     try:
         with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
@@ -799,7 +809,7 @@ def main():
         "config": {"workload": w.name + (f"+window{Wn}" if Wn else "") + (f"+ropekey{DRn}" if DRn else ""),
                    "T": w.T, "L_per_step": 1,
                    "H": H, "d": w.d, "window_rows": Wn, "window_bytes_per_step": win_bytes,
-                   "r_k": w.r_k, "r_v": w.r_v, "rho": "64/3", "B": B,
+                   "r_k": w.r_k, "r_v": w.r_v, "rho": rho_label(w), "B": B,
                    "ctx_len": [w.len_lo, w.len_hi], "tokens": S_tot, "Tq": Tq_call, "decode_calls_per_step": len(calls),
                    "variant": args.variant + (" + rope" if args.rope else "")
                               + (f" + decoupled rotary sub-key {DRn}" if DRn else ""), "seg_max": splits,

@@ -48,7 +48,7 @@ EXPORTED = ("lla_cache_bytes", "lla_slot_layout", "lla_codec_bias", "lla_encode"
             "lla_decode_attn_rope", "lla_codec_residual", "lla_decode_attn_decoupled", "lla_decode_attn_timed",
             "lla_codec_fit", "lla_codec_fit_workspace_bytes", "lla_selftest_wait_timeout",
             "lla_decode_decoupled_workspace_bytes",
-            "lla_status_fetch", "lla_status_string")
+            "lla_status_fetch", "lla_status_fetch_static", "lla_status_string")
 STATIC_SCRATCH_BYTES = 8 << 20
 
 
@@ -112,6 +112,7 @@ _lib.lla_decode_workspace_bytes.argtypes = [_P(Dims), _i32, _i32, _i32, _i32, _i
 _lib.lla_decode_workspace_bytes.restype = _sz
 _lib.lla_decode_num_splits.argtypes = [_P(Dims), _i32, _i32, _i32, _i32, _i32]
 _lib.lla_status_fetch.argtypes = [_vp, _vp, _P(_i32)]
+_lib.lla_status_fetch_static.argtypes = [_vp, _P(_i32)]
 _lib.lla_selftest_wait_timeout.argtypes = [_vp, _vp]
 _lib.lla_selftest_wait_timeout.restype = ctypes.c_int
 _lib.lla_status_string.argtypes = [ctypes.c_int]
@@ -120,7 +121,7 @@ for _n in ("lla_cache_bytes", "lla_slot_layout", "lla_codec_bias", "lla_encode",
            "lla_decode_attn_static", "lla_decode_attn_hybrid", "lla_decode_attn_rope", "lla_codec_residual",
            "lla_decode_attn_decoupled", "lla_decode_attn_timed", "lla_codec_fit",
            "lla_decode_num_splits",
-           "lla_status_fetch"):
+           "lla_status_fetch", "lla_status_fetch_static"):
     getattr(_lib, _n).restype = ctypes.c_int
 
 
@@ -354,7 +355,8 @@ def decode_attn_static(dims: Dims, layer: int, t0: int, Tq: int, q, cache: Cache
                        lse=None, variant: int = ABSORB, num_splits: int = 0, stream=None) -> None:
     """lla_decode_attn without a workspace argument: for callers that cannot allocate
     device memory.  The scratch is an 8 MiB array inside the library, shared by every
-    call (serialise calls that could overlap on the GPU)."""
+    call (serialise calls that could overlap on the GPU).  Device-side errors land in
+    the array's status word: read them with :func:`status_fetch_static`."""
     _check(_lib.lla_decode_attn_static(ctypes.byref(dims), layer, t0, Tq, _ptr(q), ctypes.byref(cache),
                                        _ptr(seq_start), _ptr(ctx_lens), B, max_ctx,
                                        ctypes.byref(codec), float(softmax_scale), variant, num_splits,
@@ -371,4 +373,12 @@ def selftest_wait_timeout(workspace, stream=None) -> None:
 def status_fetch(workspace, stream=None) -> int:
     v = _i32(0)
     _check(_lib.lla_status_fetch(_ptr(workspace), _stream(stream), ctypes.byref(v)), "lla_status_fetch")
+    return int(v.value)
+
+
+def status_fetch_static(stream=None) -> int:
+    """Read and clear the status word of decode_attn_static's library-owned array on the
+    current device (synchronises the stream)."""
+    v = _i32(0)
+    _check(_lib.lla_status_fetch_static(_stream(stream), ctypes.byref(v)), "lla_status_fetch_static")
     return int(v.value)

@@ -39,15 +39,35 @@ def is_stale() -> bool:
 
 
 def build(force: bool = False, verbose: bool = False, extra=()) -> str:
+    """Compile every .cu to an object (in parallel, under a temporary folder) and link them
+    into liblla.so with relocatable device code off (each kernel lives in one file)."""
     if not force and not is_stale():
         return LIB
+    import concurrent.futures
+    import shutil
+    import tempfile
     nvcc = os.environ.get("NVCC", "nvcc")
-    tmp = LIB + f".tmp{os.getpid()}"
-    cmd = [nvcc, *NVCC_FLAGS, *extra, "-I", os.path.join(ROOT, "include"), *sources(), "-o", tmp]
-    if verbose:
-        print(" ".join(cmd), flush=True)
-    subprocess.check_call(cmd)
-    os.replace(tmp, LIB)
+    compile_flags = [f for f in NVCC_FLAGS if f != "-shared"]
+    objdir = tempfile.mkdtemp(prefix="lla_build_")
+    try:
+        objs = [os.path.join(objdir, os.path.basename(s)[:-3] + ".o") for s in sources()]
+        cmds = [[nvcc, *compile_flags, *extra, "-I", os.path.join(ROOT, "include"), "-c", s, "-o", o]
+                for s, o in zip(sources(), objs)]
+
+        def run(cmd):
+            if verbose:
+                print(" ".join(cmd), flush=True)
+            subprocess.check_call(cmd)
+
+        with concurrent.futures.ThreadPoolExecutor(max_workers=min(len(cmds), os.cpu_count() or 4)) as ex:
+            for f in [ex.submit(run, c) for c in cmds]:
+                f.result()
+        tmp = LIB + f".tmp{os.getpid()}"
+        link = [nvcc, "-shared", "-gencode", "arch=compute_100a,code=sm_100a", *objs, "-o", tmp]
+        run(link)
+        os.replace(tmp, LIB)
+    finally:
+        shutil.rmtree(objdir, ignore_errors=True)
     return LIB
 
 

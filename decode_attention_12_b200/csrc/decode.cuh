@@ -77,4 +77,13 @@ cudaError_t launch_decode_reconstruct(const DecodeArgs &a, cudaStream_t stream);
 bool decode_window_supported(int dtype, int d);
 cudaError_t launch_decode_window(const DecodeArgs &a, int dtype, cudaStream_t stream);
 
+// lla_decode_attn that, once its arguments have passed every check, clears the first
+// word of `workspace` (the sticky device status) on `stream` before its launches; a
+// refused call queues nothing.
+int decode_attn_clearing_status(const lla_dims *dims, int32_t layer, int32_t t0, int32_t Tq, const void *q,
+                                const lla_cache *cache, const int64_t *seq_start, const int32_t *ctx_lens,
+                                int32_t B, int32_t max_ctx, const lla_codec *codec, float softmax_scale,
+                                int32_t variant, int32_t num_splits, void *out, float *lse, void *workspace,
+                                size_t ws_bytes, lla_stream_t stream);
+
 } // namespace lla

@@ -355,7 +355,7 @@ int decode_call(const lla_dims *dims, int32_t layer, int32_t t0, int32_t Tq, con
                 int32_t max_ctx, const lla_codec *codec, const lla_window *window, const lla_rope *rope,
                 float softmax_scale, int32_t variant, int32_t num_splits, void *out, float *lse,
                 void *workspace, size_t ws_bytes, lla_stream_t stream, const lla_decoupled *dec = nullptr,
-                lla_event_t ev_start = nullptr, lla_event_t ev_end = nullptr)
+                lla_event_t ev_start = nullptr, lla_event_t ev_end = nullptr, bool clear_status = false)
 {
     int rc = check_dims(dims);
     if (rc != LLA_OK)
@@ -363,8 +363,14 @@ int decode_call(const lla_dims *dims, int32_t layer, int32_t t0, int32_t Tq, con
     if (layer < 0 || layer >= dims->L || t0 < 0 || Tq < 1 || t0 + (int64_t)Tq > dims->T || B < 0 ||
         max_ctx < 0 || num_splits < 0 || (variant != LLA_ABSORB && variant != LLA_RECONSTRUCT))
         return LLA_ERR_INVALID;
-    if (B == 0)
-        return LLA_OK;
+    if (B == 0) { // nothing to compute; a status word the caller asked to clear is cleared
+        if (!clear_status)
+            return LLA_OK;
+        if (workspace == nullptr || !aligned16(workspace))
+            return LLA_ERR_INVALID;
+        return cudaMemsetAsync(workspace, 0, sizeof(int32_t), (cudaStream_t)stream) == cudaSuccess ? LLA_OK
+                                                                                                   : LLA_ERR_CUDA;
+    }
     if (q == nullptr || cache == nullptr || cache->k == nullptr || cache->v == nullptr || cache->slots < 0 ||
         seq_start == nullptr || ctx_lens == nullptr || codec == nullptr || codec->W_up_k == nullptr ||
         codec->W_up_v == nullptr || codec->mu_k == nullptr || codec->mu_v == nullptr || out == nullptr)
@@ -473,6 +479,9 @@ int decode_call(const lla_dims *dims, int32_t layer, int32_t t0, int32_t Tq, con
     a.Tq_all = Tq;
     a.tq_off = 0;
     cudaStream_t s = (cudaStream_t)stream;
+    // every check has passed: only now is anything queued on the caller's stream
+    if (clear_status && cudaMemsetAsync(workspace, 0, sizeof(int32_t), s) != cudaSuccess)
+        return LLA_ERR_CUDA;
     cudaError_t err = cudaSuccess;
     // hybrid form: the window pass runs after the decode grid, before the combine
     auto window_pass = [&](const DecodeArgs &ac) -> cudaError_t {
@@ -562,6 +571,17 @@ int decode_call(const lla_dims *dims, int32_t layer, int32_t t0, int32_t Tq, con
 }
 
 } // namespace
+
+int lla::decode_attn_clearing_status(const lla_dims *dims, int32_t layer, int32_t t0, int32_t Tq, const void *q,
+                                     const lla_cache *cache, const int64_t *seq_start, const int32_t *ctx_lens,
+                                     int32_t B, int32_t max_ctx, const lla_codec *codec, float softmax_scale,
+                                     int32_t variant, int32_t num_splits, void *out, float *lse, void *workspace,
+                                     size_t ws_bytes, lla_stream_t stream)
+{
+    return decode_call(dims, layer, t0, Tq, q, cache, seq_start, ctx_lens, B, max_ctx, codec, nullptr, nullptr,
+                       softmax_scale, variant, num_splits, out, lse, workspace, ws_bytes, stream, nullptr, nullptr,
+                       nullptr, true);
+}
 
 extern "C" {
 

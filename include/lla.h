@@ -364,8 +364,14 @@ size_t lla_decode_decoupled_workspace_bytes(const lla_dims *dims, int32_t B, int
  *    any stream capture.
  *  - A problem that needs more scratch than LLA_STATIC_SCRATCH_BYTES (compare
  *    lla_decode_workspace_bytes) is rejected with LLA_ERR_WORKSPACE before any launch.
- *  - All calls share the one array, which keeps the last call's contents; each call
- *    clears the array's status word (a 4-byte memset on `stream`) before its launches.
+ *  - The looked-up address belongs to the context it was looked up in; a call made in
+ *    a new context of the device (after cudaDeviceReset, say) looks it up again.
+ *  - All calls share the one array, which keeps the last call's contents.  A call whose
+ *    arguments pass every check clears the array's status word (a 4-byte memset on
+ *    `stream`) before its launches; a refused call queues nothing and leaves the word as
+ *    it was.  Device-side errors of the call (a context longer than max_ctx:
+ *    LLA_ERR_INVALID; a bounded wait that gave up: LLA_ERR_DEVICE_TIMEOUT) land in that
+ *    word: read them with lla_status_fetch_static before the next static call clears it.
  *    Calls that overlap on the GPU (other streams, or unordered host threads) race on
  *    the array: the caller must serialise them.                                            */
 #define LLA_STATIC_SCRATCH_BYTES (8u << 20)
@@ -374,6 +380,10 @@ int lla_decode_attn_static(const lla_dims *dims, int32_t layer, int32_t t0, int3
                            const int32_t *ctx_lens, int32_t B, int32_t max_ctx,
                            const lla_codec *codec, float softmax_scale, int32_t variant,
                            int32_t num_splits, void *out, float *lse, lla_stream_t stream);
+/* Status word of lla_decode_attn_static's array on the current device: synchronises
+ * `stream`, copies the word to *status_host and clears it (as lla_status_fetch does for
+ * a caller-owned workspace).  Allocates nothing.                                          */
+int lla_status_fetch_static(lla_stream_t stream, int32_t *status_host);
 
 /* ---- status ---------------------------------------------------------------------------
  * Kernels never trap.  A decode kernel that gives up a bounded wait records

@@ -362,25 +362,3 @@ def decode_layer(variant, q, c_K, c_V, seq_start, ctx_lens, W_up_K, mu_K, W_up_V
         with ThreadPoolExecutor(max_workers=threads) as ex:
             list(ex.map(run, units))
     return o, lse
-
-
-def encode_rows(x, mu, W_down, threads=None, chunk=4096):
-    """Encode many rows on a thread pool (same arithmetic as :func:`encode`)."""
-    x = np.asarray(x)
-    n = x.shape[0]
-    if threads is None:
-        threads = os.cpu_count() or 1
-    parts = [(i, min(n, i + chunk)) for i in range(0, n, chunk)]
-    out = np.empty((n, np.asarray(W_down).shape[1]))
-
-    def run(p):
-        a, b = p
-        out[a:b] = encode(x[a:b], mu, W_down)
-
-    if threads <= 1 or len(parts) == 1:
-        for p in parts:
-            run(p)
-    else:
-        with ThreadPoolExecutor(max_workers=threads) as ex:
-            list(ex.map(run, parts))
-    return out

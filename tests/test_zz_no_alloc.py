@@ -71,3 +71,34 @@ def test_static_scratch_rejects_problems_beyond_its_size():
                                p["seq_start"], p["ctx_lens"], 64, 4096, codec_of(p), 1.0, out,
                                None, num_splits=64)
     assert ei.value.code == lla.LLA_ERR_WORKSPACE
+
+
+def test_static_scratch_reports_device_errors_and_clears_them_per_call():
+    """A context longer than max_ctx is a device-side error (LLA_ERR_INVALID in the status
+    word).  The static call's word is read with status_fetch_static; a call refused on the
+    host queues nothing and leaves the word alone; the next accepted call clears it."""
+    w = S.shrink(S.WORKLOADS["ouro1.4b-layer"], B=2, len_lo=300, len_hi=500)
+    p = S.decode_inputs(w, 0, DEV)
+    dims = dims_of(w)
+    B = len(p["lens"])
+    cache = lla.make_cache(p["k"], p["v"], p["slots"])
+    out = torch.full((B, 4, w.H, w.d), float("nan"), dtype=torch.float32, device=DEV)
+    lla.status_fetch_static()                      # start from a clear word
+    # every context is longer than the max_ctx the scratch was planned for
+    assert int(p["lens"].min()) > 100
+    lla.decode_attn_static(dims, 0, 0, 4, p["q"], cache, p["seq_start"], p["ctx_lens"], B, 100,
+                           codec_of(p), 1.0, out, None)
+    torch.cuda.synchronize()
+    # refused on the host (no query): nothing is queued, the word keeps the error
+    with pytest.raises(lla.LLAError) as ei:
+        lla.decode_attn_static(dims, 0, 0, 4, None, cache, p["seq_start"], p["ctx_lens"], B,
+                               int(p["lens"].max()), codec_of(p), 1.0, out, None)
+    assert ei.value.code == lla.LLA_ERR_INVALID
+    assert lla.status_fetch_static() == lla.LLA_ERR_INVALID
+    assert lla.status_fetch_static() == 0          # the fetch cleared it
+    # an accepted call with the right max_ctx: status clear, results right
+    got = _static_call(p, w, 0, 4, p["q"])
+    assert lla.status_fetch_static() == 0
+    ref = run_decode(p, w, 0, 0, 4, 1.0, q=p["q"])
+    assert ref[2] == 0
+    _assert_same(got[0], got[1], ref[0], ref[1])
