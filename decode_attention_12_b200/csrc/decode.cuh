@@ -72,6 +72,12 @@ bool decode_mma2d_supported(int dtype, int r_k, int r_v, int fold, int H);
 int decode_mma2d_loops_per_pass(int H);
 cudaError_t launch_decode_absorb_2d(const DecodeArgs &a, cudaStream_t stream);
 cudaError_t launch_decode_reconstruct(const DecodeArgs &a, cudaStream_t stream);
+// Reconstruct form on tcgen05 tensor cores: one latent read serves up to
+// decode_recon_tc_loops_per_pass() loop queries (a.Tq per launch); d = 128, bf16.
+bool decode_recon_tc_supported(int dtype, int r_k, int r_v, int d, int fold, int B, bool rope);
+int decode_recon_tc_loops_per_pass();
+int decode_recon_tc_smem_bytes(int r_k, int r_v, bool rope, int lp, int B);
+cudaError_t launch_decode_recon_tc(const DecodeArgs &a, cudaStream_t stream);
 // Hybrid form: attention of every loop query over its exact window rows, written to
 // a.win_part for the combine to merge (launched between the decode and the combine).
 bool decode_window_supported(int dtype, int d);

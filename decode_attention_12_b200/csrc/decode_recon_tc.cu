@@ -1,0 +1,824 @@
+// decode_recon_tc.cu -- LLA decode attention, reconstruct-on-read form (and the faithful
+// read with rotary embedding), on tcgen05 tensor cores with tensor-memory accumulators.
+//
+// "Looped Latent Attention: Cross-Loop KV Compression for Looped Transformers": Pith
+// review page, "What carries the argument" (Eq. 3: loop t reads x_hat_t = c W_up,t + mu_t)
+// and arXiv abstract (K/V vectors are reconstructed only when attention reads them); the
+// faithful read rotates query and rebuilt key at their positions after reconstruction
+// (Pith verdict record, key_machinery; RoFormer's rotation).
+//
+// One latent tile of 128 tokens is read from HBM once and serves every loop query t of
+// the pass (up to 4).  Per (tile, loop) step, on the tensor cores (one issuing thread):
+//     K_hat   [128 tok x d] = C_K . W_up,t^K        M = tokens, N = d, K = r_k  (TMEM)
+//     V_hat^T [d x 128 tok] = W_up,t^V^T . C_V^T    M = d, N = tokens, K = r_v  (TMEM)
+//     O^T     [d x 16]      = V_hat^T . P^T         kind::tf32, A read straight from TMEM
+// W_up,t enters as bf16 hi + lo parts (two MMAs, products exact in fp32), so K_hat and
+// V_hat carry about 16 mantissa bits of W_up; the P.V_hat MMA reads V_hat as tf32 (10
+// bits) and p as tf32 hi + lo parts.  mu_t^V is left out of V_hat and added once per
+// record (sum_n p_n (v_hat_n - mu) + mu sum_n p_n); the score term q . mu_t^K is a
+// constant per (unit, loop) -- with rotation the key's mean turns with the key, so there
+// K_hat takes mu_t^K from one more MMA (a ones column times mu's hi/lo parts).
+//
+// Scores, softmax and output accumulation run on 4 warps, one tensor-memory lane quarter
+// each: thread r owns token row r of K_hat (its score is a 128-long dot product in
+// registers, packed fp32x2 FMAs), keeps a warp-local running max per loop and writes p
+// into rows 2w (hi) and 2w + 1 (lo) of P, so the P.V_hat MMA returns one column pair per
+// warp and no cross-warp reduction is needed per step; the same thread, as lane d of the
+// O^T accumulator, folds each step's column pairs into per-warp output sums with the
+// warps' rescale factors.  Records (acc, m, l) are merged across warps at segment ends
+// and have the layout of the other reconstruct kernels, so the combine is shared.
+//
+// Faithful read: a query at position p and the rebuilt key of token n = n0 + r (tile row
+// r) give <R(p) q, R(n) k> = <R(p - n0) q, R(r) k>: the query is turned once per tile by
+// (p - n0) (angles in double precision), and every thread keeps cos/sin(r w_i) of its row
+// in registers for the whole kernel.  Component pairs (i, i + d/2) sit in one thread: the
+// rows of W_up,t^K, q and mu_t^K are staged pair-major (identity for the half-split
+// pairing, even-first for RoFormer's interleaved one).
+//
+// Work split: the token stream of all (head, sequence) units in head-major order is cut
+// into equal shares, one per CTA (one CTA per SM), so a CTA's share mostly stays within
+// one head and W_up is staged rarely.  Every wait is bounded; a timeout records
+// LLA_ERR_DEVICE_TIMEOUT and the CTA winds down (tensor memory is always released).
+#include "mma_common.cuh"
+#include "tc_common.cuh"
+
+namespace lla {
+namespace {
+using namespace mma;
+
+constexpr int kD = 128;         // head dimension served
+constexpr int kTile = 128;      // tokens per latent tile (M of the K_hat MMA)
+constexpr int kMaxLoops = 4;    // loop queries per pass
+constexpr int kSoftWarps = 4;   // warps 0-3: scores, softmax, output
+constexpr int kProducerWarp = 4, kMmaWarp = 5;
+constexpr int kThreads = 6 * 32;
+constexpr int kSoftThreads = kSoftWarps * 32;
+constexpr float kRescale = 8.0f; // lazy rescale margin (log2 units)
+
+// tensor-memory columns
+constexpr uint32_t kTmemCols = 512;
+constexpr uint32_t kColK = 0;    // K_hat [128 tokens (lanes)][128 d] fp32
+constexpr uint32_t kColV = 128;  // V_hat^T [128 d (lanes)][128 tokens] fp32, two buffers
+constexpr uint32_t kColO = 384;  // O^T [128 d (lanes)][16] fp32, two buffers
+
+constexpr int kPRows = 16;                 // N of the P.V_hat MMA
+constexpr int kPSlab = kPRows * 128;       // 32 tokens (128 B of tf32) x 16 rows, 128B swizzle
+constexpr int kPBuf = 4 * kPSlab;          // 128 tokens
+
+// barriers after the ring's full[NST] and empty[NST]
+enum {
+    BKFULL = 0, BKEMPTY, BVFULL0, BVFULL1, BPFULL0, BPFULL1, BOFULL0, BOFULL1, BOEMPTY0, BOEMPTY1, BWREADY,
+    BDRAIN, BCOUNT
+};
+
+struct RLayout {
+    uint32_t nst, stage, wk, wv, wk_part, wv_part, pbuf, ones, muk_t, qv, qt4, qtn, muk, muv, qmu, alpha, mrg, omg,
+        bar, misc, scr, pref, total;
+};
+
+__host__ __device__ inline uint32_t round_up(uint32_t x, uint32_t a) { return (x + a - 1) / a * a; }
+
+// Shared-memory layout (byte offsets from a 1024-aligned base) for lp loops per pass and
+// B sequences.  Every operand tile starts on a 1024-byte boundary.
+template <int RK, int RV, bool ROPE> __host__ __device__ inline RLayout rlayout(int lp, int B)
+{
+    using LK = TileLayout<RK, kTile>;
+    using LV = TileLayout<RV, kTile>;
+    RLayout L;
+    L.nst = (RK + RV) >= 64 ? 3 : 4;
+    L.stage = align1024(LK::BYTES + LV::BYTES);
+    uint32_t o = L.nst * L.stage;
+    L.wk_part = kD * RK * 2;
+    L.wv_part = kD * RV * 2;
+    L.wk = o;
+    o += lp * 2 * L.wk_part;
+    L.wv = o;
+    o += lp * 2 * L.wv_part;
+    L.pbuf = o;
+    o += 2 * kPBuf;
+    L.ones = o;
+    o += ROPE ? kTile * 32 : 0;
+    L.muk_t = o;
+    o += ROPE ? lp * kD * 32 : 0;
+    L.qv = o;
+    o += lp * kD * 4;
+    L.qt4 = o;
+    o += ROPE ? 2 * lp * 32 * 16 : 0;
+    L.qtn = o;
+    o += ROPE ? 2 * lp * 32 * 8 : 0;
+    L.muk = o;
+    o += lp * kD * 4;
+    L.muv = o;
+    o += lp * kD * 4;
+    L.qmu = o;
+    o += 16;
+    L.alpha = o;
+    o += 4 * kSoftWarps * 4;
+    L.mrg = o;
+    o += kSoftWarps * kMaxLoops * 2 * 4;
+    L.omg = round_up(o, 8);
+    o = L.omg + (ROPE ? kD / 2 * 8 : 0);
+    L.bar = round_up(o, 8);
+    o = L.bar + (2 * L.nst + BCOUNT) * 8;
+    L.misc = o;
+    o += 16;
+    L.scr = round_up(o, 8);
+    o = L.scr + (kThreads / 32 + 1) * 8;
+    L.pref = o;
+    o += 8 * (B + 1);
+    L.total = o;
+    return L;
+}
+
+// Kernel row of d-index k on the key side: pair i is (row i, row i + d/2).
+__device__ __forceinline__ int pair_row(int k, int style)
+{
+    return style == LLA_ROPE_INTERLEAVED ? (k & 1) * (kD / 2) + (k >> 1) : k;
+}
+
+// Walks a CTA's share of the head-major token stream (position p: head p / S, token
+// p mod S of the concatenated sequences), unit segment by unit segment, tile by tile.
+// The record slot of a segment is j = share - first share of its unit, as in the
+// sequence-major walk of the other kernels, so the combine reads it the same way.
+template <int TILE> struct HeadWalk {
+    int64_t pos, end, chunk, S, seq0;
+    int32_t b, h, n, seg_end, u, j, n_u;
+    bool in_seg;
+
+    __device__ void start(int64_t p, int64_t e, int64_t ch, int64_t s_tot)
+    {
+        pos = p;
+        end = e;
+        chunk = ch;
+        S = s_tot;
+        b = 0;
+        in_seg = false;
+    }
+    __device__ bool next(const int64_t *pref, const int64_t *starts, int B, int H, TileDesc &d)
+    {
+        if (!in_seg) {
+            if (pos >= end)
+                return false;
+            h = (int)(pos / S);
+            const int64_t q = pos - (int64_t)h * S;
+            if (!(pref[b] <= q && q < pref[b + 1])) {
+                if (b + 2 <= B && pref[b + 1] <= q && q < pref[b + 2]) {
+                    ++b;
+                } else { // largest b with pref[b] <= q (skips empty sequences)
+                    int lo = 0, hi = B - 1;
+                    while (lo < hi) {
+                        const int mid = (lo + hi + 1) >> 1;
+                        if (pref[mid] <= q)
+                            lo = mid;
+                        else
+                            hi = mid - 1;
+                    }
+                    b = lo;
+                }
+            }
+            const int len = (int)(pref[b + 1] - pref[b]);
+            seq0 = starts[b];
+            n = (int)(q - pref[b]);
+            const int64_t take = min((int64_t)(len - n), end - pos);
+            seg_end = n + (int)take;
+            pos += take;
+            u = b * H + h;
+            const int64_t U = (int64_t)h * S + pref[b]; // unit start in the stream
+            const int64_t c_first = U / chunk, c_last = (U + len - 1) / chunk;
+            j = (int)(blockIdx.x - c_first);
+            n_u = (int)(c_last - c_first + 1);
+            in_seg = true;
+            d.flags = 1;
+        } else {
+            d.flags = 0;
+        }
+        d.row = seq0 + n;
+        d.b = b;
+        d.h = h;
+        d.n0 = n;
+        d.rows = min(TILE, seg_end - n);
+        d.u = u;
+        d.j = j;
+        d.n_u = n_u;
+        n += d.rows;
+        if (n >= seg_end) {
+            d.flags |= 2;
+            in_seg = false;
+        }
+        return true;
+    }
+};
+
+__device__ __forceinline__ float2 f2(uint32_t x, uint32_t y) { return make_float2(__uint_as_float(x), __uint_as_float(y)); }
+
+template <int RK, int RV, bool ROPE>
+__global__ void __launch_bounds__(kThreads, 1)
+    decode_recon_tc_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant__ CUtensorMap map_v,
+                           const DecodeArgs a)
+{
+    using LK = TileLayout<RK, kTile>;
+    using LV = TileLayout<RV, kTile>;
+    using L16 = TileLayout<16, kTile>;
+    extern __shared__ uint8_t smem_raw[];
+    // aligned by arithmetic on the shared array itself, so accesses stay shared-space loads
+    uint8_t *smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
+    const int lp = a.Tq;
+    const RLayout Ly = rlayout<RK, RV, ROPE>(lp, a.B);
+    const uint32_t sbase = smem_u32(smem);
+    const uint32_t bar0 = sbase + Ly.bar;
+    const uint32_t nst = Ly.nst;
+    volatile int *misc = reinterpret_cast<volatile int *>(smem + Ly.misc); // [0] error, [1] tmem, [2] issued
+    int64_t *pref = reinterpret_cast<int64_t *>(smem + Ly.pref);
+    float *alpha = reinterpret_cast<float *>(smem + Ly.alpha); // [4 steps][4 warps]
+    float *mrg = reinterpret_cast<float *>(smem + Ly.mrg);     // [4 warps][4 loops][m, l]
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int B = a.B, H = a.H;
+    auto full_bar = [&](int st) { return bar0 + 8u * st; };
+    auto empty_bar = [&](int st) { return bar0 + 8u * (nst + st); };
+    auto bar = [&](int k) { return bar0 + 8u * (2 * nst + k); };
+
+    if (tid == 0) {
+        for (uint32_t st = 0; st < nst; ++st) {
+            mbar_init(full_bar(st), 1);  // producer's expect_tx + TMA bytes
+            mbar_init(empty_bar(st), 1); // the tile's last MMAs completed (commit)
+        }
+        mbar_init(bar(BKFULL), 1);
+        mbar_init(bar(BKEMPTY), kSoftWarps);
+        mbar_init(bar(BVFULL0), 1);
+        mbar_init(bar(BVFULL1), 1);
+        mbar_init(bar(BPFULL0), kSoftWarps);
+        mbar_init(bar(BPFULL1), kSoftWarps);
+        mbar_init(bar(BOFULL0), 1);
+        mbar_init(bar(BOFULL1), 1);
+        mbar_init(bar(BOEMPTY0), kSoftWarps);
+        mbar_init(bar(BOEMPTY1), kSoftWarps);
+        mbar_init(bar(BWREADY), 1);
+        mbar_init(bar(BDRAIN), 1);
+        misc[0] = 0;
+        misc[2] = 0;
+        fence_barrier_init();
+    }
+    if (warp == kMmaWarp)
+        tc::alloc(reinterpret_cast<uint32_t *>(smem + Ly.misc + 4), kTmemCols);
+    // P buffers start (and, outside each warp's own two rows, stay) zero
+    for (int e = tid; e < 2 * kPBuf / 16; e += kThreads)
+        reinterpret_cast<uint4 *>(smem + Ly.pbuf)[e] = make_uint4(0u, 0u, 0u, 0u);
+    if (ROPE) {
+        // ones tile [128 rows][16]: columns 0 and 1 are 1 (they meet mu's hi and lo parts)
+        const __nv_bfloat162 one2 = __floats2bfloat162_rn(1.f, 1.f);
+        for (int r = tid; r < kTile; r += kThreads) {
+            uint4 c0 = make_uint4(*reinterpret_cast<const uint32_t *>(&one2), 0u, 0u, 0u);
+            *reinterpret_cast<uint4 *>(smem + Ly.ones + L16::off(r, 0)) = c0;
+            *reinterpret_cast<uint4 *>(smem + Ly.ones + L16::off(r, 1)) = make_uint4(0u, 0u, 0u, 0u);
+        }
+        double *omg = reinterpret_cast<double *>(smem + Ly.omg);
+        for (int i = tid; i < kD / 2; i += kThreads)
+            omg[i] = pow((double)a.rope_base, -2.0 * i / kD);
+    }
+    fence_proxy_async_smem(); // generic writes above are read by the tensor cores
+    tc::fence_before();
+    block_length_prefix<kThreads>(a.ctx_lens, B, pref, reinterpret_cast<int64_t *>(smem + Ly.scr));
+    tc::fence_after();
+    const uint32_t tmem = (uint32_t)misc[1];
+    // The combine grid may take SM slots as this grid's CTAs exit; it reads nothing of
+    // ours before its own programmatic-launch wait.
+    grid_launch_dependents();
+    int64_t s0, s1, chunk;
+    cta_share(pref, B, H, a.chunk_min, s0, s1, chunk);
+    const int64_t S_tot = pref[B];
+
+    if (s0 < s1 && warp == kProducerWarp) {
+        // ================= producer: one lane streams the latent tiles =================
+        if (lane == 0) {
+            HeadWalk<kTile> walk;
+            walk.start(s0, s1, chunk, S_tot);
+            TileDesc d;
+            int issued = 0;
+            while (walk.next(pref, a.seq_start, B, H, d)) {
+                const int i = issued, st = i % (int)nst;
+                if (i >= (int)nst && !mbar_wait_bounded(empty_bar(st), ((i / nst) - 1) & 1)) {
+                    misc[0] = 1;
+                    break;
+                }
+                if (misc[0])
+                    break;
+                const uint32_t sk = sbase + st * Ly.stage, sv = sk + LK::BYTES;
+                const int nbox = (d.rows + kBox - 1) / kBox;
+                fence_proxy_async_smem();
+                mbar_arrive_expect_tx(full_bar(st), nbox * kBox * (RK + RV) * 2);
+                const int y0 = (int)((int64_t)d.h * a.slots + d.row);
+                for (int bx = 0; bx < nbox; ++bx) {
+                    tma_load_2d(sk + bx * kBox * LK::TB, &map_k, 0, y0 + bx * kBox, full_bar(st));
+                    tma_load_2d(sv + bx * kBox * LV::TB, &map_v, 0, y0 + bx * kBox, full_bar(st));
+                }
+                ++issued;
+            }
+            misc[2] = issued;
+        }
+    } else if (s0 < s1 && warp == kMmaWarp) {
+        // ================= MMA issuer: lane 0 issues, the warp waits and zeroes =================
+        constexpr uint32_t kIdKV = tc::idesc(tc::kFmtBf16, 128, 128);
+        constexpr uint32_t kIdPV = tc::idesc(tc::kFmtTf32, 128, kPRows);
+        bool err = false;
+        auto wait_all = [&](uint32_t b, uint32_t parity) -> bool {
+            bool ok = !err && misc[0] == 0 && mbar_wait_bounded(b, parity);
+            ok = __all_sync(0xffffffffu, ok);
+            if (!ok) {
+                err = true;
+                misc[0] = 1;
+            }
+            return ok;
+        };
+        // O^T of step sp: V_hat^T (TMEM) . P^T, 16 k-steps of 8 tokens
+        auto issue_pv = [&](int sp) {
+            const int bb = sp & 1;
+            if (!wait_all(bar(BPFULL0 + bb), (sp >> 1) & 1) || !wait_all(bar(BVFULL0 + bb), (sp >> 1) & 1))
+                return;
+            if (sp >= 2 && !wait_all(bar(BOEMPTY0 + bb), ((sp - 2) >> 1) & 1))
+                return;
+            tc::fence_after();
+            if (lane == 0) {
+                const uint32_t pb = sbase + Ly.pbuf + bb * kPBuf;
+#pragma unroll
+                for (int j = 0; j < kTile / 8; ++j)
+                    tc::mma_tf32_ts(tmem + kColO + 16 * bb, tmem + kColV + 128 * bb + 8 * j,
+                                    tc::smem_desc(pb + (j >> 2) * kPSlab + (j & 3) * 32, 128), kIdPV, j > 0);
+                tc::commit(bar(BOFULL0 + bb));
+            }
+            __syncwarp();
+        };
+        HeadWalk<kTile> walk;
+        walk.start(s0, s1, chunk, S_tot);
+        TileDesc d;
+        int s = 0, ti = 0, wc = 0, prev_h = -1;
+        while (!err && walk.next(pref, a.seq_start, B, H, d)) {
+            const int st = ti % (int)nst;
+            const bool wchange = (d.flags & 1) && d.h != prev_h;
+            if (!wait_all(full_bar(st), (ti / nst) & 1))
+                break;
+            const uint32_t sk = sbase + st * Ly.stage, sv = sk + LK::BYTES;
+            if (d.rows < kTile) { // rows past the segment: zeros, never stale or NaN data
+                LK::zero_rows(smem + st * Ly.stage, d.rows, kTile, lane);
+                LV::zero_rows(smem + st * Ly.stage + LK::BYTES, d.rows, kTile, lane);
+                fence_proxy_async_smem();
+                __syncwarp();
+            }
+            for (int t = 0; t < lp && !err; ++t) {
+                if (t == 0 && wchange) {
+                    // the staging of a new head's W_up waits for every MMA of the old one
+                    if (s >= 1)
+                        issue_pv(s - 1);
+                    if (!wait_all(bar(BWREADY), wc & 1))
+                        break;
+                    ++wc;
+                    prev_h = d.h;
+                }
+                if (s >= 1 && !wait_all(bar(BKEMPTY), (s - 1) & 1))
+                    break;
+                if (s >= 2 && !wait_all(bar(BOFULL0 + (s & 1)), ((s - 2) >> 1) & 1))
+                    break; // P.V_hat of step s - 2 has read this V_hat^T buffer
+                tc::fence_after();
+                if (lane == 0) {
+                    const uint32_t wk = sbase + Ly.wk + t * 2 * Ly.wk_part;
+                    const uint32_t wv = sbase + Ly.wv + t * 2 * Ly.wv_part;
+#pragma unroll
+                    for (int kk = 0; kk < RK / 16; ++kk)
+#pragma unroll
+                        for (int hl = 0; hl < 2; ++hl)
+                            tc::mma_bf16(tmem + kColK, tc::smem_desc(sk + 32 * kk, 2 * RK),
+                                         tc::smem_desc(wk + hl * Ly.wk_part + 32 * kk, 2 * RK), kIdKV, (kk | hl) != 0);
+                    if (ROPE)
+                        tc::mma_bf16(tmem + kColK, tc::smem_desc(sbase + Ly.ones, 32),
+                                     tc::smem_desc(sbase + Ly.muk_t + t * kD * 32, 32), kIdKV, 1);
+                    tc::commit(bar(BKFULL));
+                    const uint32_t vcol = tmem + kColV + 128 * (s & 1);
+#pragma unroll
+                    for (int kk = 0; kk < RV / 16; ++kk)
+#pragma unroll
+                        for (int hl = 0; hl < 2; ++hl)
+                            tc::mma_bf16(vcol, tc::smem_desc(wv + hl * Ly.wv_part + 32 * kk, 2 * RV),
+                                         tc::smem_desc(sv + 32 * kk, 2 * RV), kIdKV, (kk | hl) != 0);
+                    tc::commit(bar(BVFULL0 + (s & 1)));
+                    if (t == lp - 1)
+                        tc::commit(empty_bar(st)); // the tile's stage is free once these complete
+                }
+                __syncwarp();
+                if (!(t == 0 && wchange) && s >= 1)
+                    issue_pv(s - 1);
+                ++s;
+            }
+            ++ti;
+        }
+        if (!err && s >= 1)
+            issue_pv(s - 1);
+    } else if (s0 < s1 && warp < kSoftWarps) {
+        // ================= scores, softmax, output: thread r = token row r / lane d =================
+        const int r = tid;
+        const uint32_t trow = tmem + ((uint32_t)(32 * warp) << 16);
+        bool err = false;
+        auto wait_all = [&](uint32_t b, uint32_t parity) -> bool {
+            bool ok = !err && misc[0] == 0 && mbar_wait_bounded(b, parity);
+            ok = __all_sync(0xffffffffu, ok);
+            if (!ok) {
+                err = true;
+                misc[0] = 1;
+            }
+            return ok;
+        };
+        // rotation of this thread's row r: (cos, sin)(r w_i) for pairs 2c and 2c + 1
+        float2 rc[ROPE ? 32 : 1], rs[ROPE ? 32 : 1];
+        if (ROPE) {
+            const float lb = log2f(a.rope_base);
+#pragma unroll
+            for (int c = 0; c < 32; ++c) {
+                float s0_, c0_, s1_, c1_;
+                sincosf((float)r * exp2f(-2.0f * (float)(2 * c) / (float)kD * lb), &s0_, &c0_);
+                sincosf((float)r * exp2f(-2.0f * (float)(2 * c + 1) / (float)kD * lb), &s1_, &c1_);
+                rc[c] = make_float2(c0_, c1_);
+                rs[c] = make_float2(s0_, s1_);
+            }
+        }
+        float m[kMaxLoops], l[kMaxLoops], oacc[kMaxLoops][kSoftWarps];
+        const float *qv = reinterpret_cast<const float *>(smem + Ly.qv);
+        const float *qmu = reinterpret_cast<const float *>(smem + Ly.qmu);
+        const float *muv = reinterpret_cast<const float *>(smem + Ly.muv);
+
+        // O^T of step sp (loop tp): fold each warp's column pair into its output sum
+        auto readout = [&](int sp, int tp) {
+            uint32_t o8[8];
+            const bool ok = wait_all(bar(BOFULL0 + (sp & 1)), (sp >> 1) & 1);
+            if (ok) {
+                tc::fence_after();
+                tc::ld_x8(trow + kColO + 16 * (sp & 1), o8);
+                tc::wait_ld();
+                tc::fence_before();
+            }
+            __syncwarp();
+            if (lane == 0)
+                mbar_arrive(bar(BOEMPTY0 + (sp & 1)));
+            if (!ok)
+                return;
+            const float *al = alpha + (sp & 3) * kSoftWarps;
+#pragma unroll
+            for (int t = 0; t < kMaxLoops; ++t)
+                if (t == tp) {
+#pragma unroll
+                    for (int w = 0; w < kSoftWarps; ++w)
+                        oacc[t][w] = fmaf(oacc[t][w], al[w],
+                                          __uint_as_float(o8[2 * w]) + __uint_as_float(o8[2 * w + 1]));
+                }
+        };
+        // segment end: merge the warps' states into one record per loop
+        auto flush = [&](const TileDesc &dd) {
+#pragma unroll
+            for (int t = 0; t < kMaxLoops; ++t) {
+                if (t < lp) {
+                    float lq = l[t];
+#pragma unroll
+                    for (int off = 16; off > 0; off >>= 1)
+                        lq += __shfl_xor_sync(0xffffffffu, lq, off);
+                    if (lane == 0) {
+                        mrg[(warp * kMaxLoops + t) * 2] = m[t];
+                        mrg[(warp * kMaxLoops + t) * 2 + 1] = lq;
+                    }
+                }
+            }
+            asm volatile("bar.sync 1, %0;" ::"r"(kSoftThreads) : "memory");
+            if (misc[0] == 0 && dd.j < a.seg_max) {
+#pragma unroll
+                for (int t = 0; t < kMaxLoops; ++t) {
+                    if (t < lp) {
+                        float M = -INFINITY;
+#pragma unroll
+                        for (int w = 0; w < kSoftWarps; ++w)
+                            M = fmaxf(M, mrg[(w * kMaxLoops + t) * 2]);
+                        float L = 0.f, acc = 0.f;
+#pragma unroll
+                        for (int w = 0; w < kSoftWarps; ++w) {
+                            const float mw = mrg[(w * kMaxLoops + t) * 2];
+                            if (mw != -INFINITY) {
+                                const float e = fast_exp2(mw - M);
+                                L = fmaf(e, mrg[(w * kMaxLoops + t) * 2 + 1], L);
+                                acc = fmaf(e, oacc[t][w], acc);
+                            }
+                        }
+                        acc = fmaf(L, muv[t * kD + r], acc); // mu_t^V, left out of V_hat
+                        float *rec = a.part + (((int64_t)dd.u * a.Tq_all + a.tq_off + t) * a.seg_max + dd.j) *
+                                                  part_stride(kD);
+                        rec[r] = acc;
+                        if (r == 0) {
+                            rec[kD] = M;
+                            rec[kD + 1] = L;
+                        }
+                    }
+                }
+                if (r == 0 && dd.j == 0)
+                    a.counts[dd.u] = dd.n_u;
+            } else if (r == 0 && dd.j >= a.seg_max) {
+                report_status(a.status, LLA_ERR_INVALID); // a context longer than max_ctx
+            }
+            asm volatile("bar.sync 1, %0;" ::"r"(kSoftThreads) : "memory"); // mrg free again
+        };
+
+        HeadWalk<kTile> walk;
+        walk.start(s0, s1, chunk, S_tot);
+        TileDesc d, dseg;
+        int s = 0, tile = 0, pend = -1, pend_t = 0, prev_h = -1;
+        int32_t qpos = 0;
+        while (walk.next(pref, a.seq_start, B, H, d)) {
+            if (d.flags & 1) {
+                // ---- new unit segment: close the previous one, stage this one's inputs
+                if (pend >= 0) {
+                    readout(pend, pend_t);
+                    pend = -1;
+                    flush(dseg);
+                }
+                dseg = d;
+                const bool wchange = d.h != prev_h;
+                const int style = a.rope_style;
+                for (int t = 0; t < lp; ++t) {
+                    const int tl = a.t0 + a.tq_off + t;
+                    const int64_t gi = ((int64_t)d.h * a.T + tl);
+                    if (wchange) {
+                        // W_up,t^K^T and W_up,t^V^T as bf16 hi/lo K-major tiles (rows = d)
+                        const float *wk = a.W_up_k + gi * RK * kD;
+                        const float *wv = a.W_up_v + gi * RV * kD;
+                        uint8_t *dk = smem + Ly.wk + t * 2 * Ly.wk_part;
+                        uint8_t *dv = smem + Ly.wv + t * 2 * Ly.wv_part;
+                        for (int e = r; e < RK * kD; e += kSoftThreads) {
+                            const int j = e / kD, k = e - j * kD;
+                            const int row = ROPE ? pair_row(k, style) : k;
+                            const float x = wk[e];
+                            const __nv_bfloat16 hi = __float2bfloat16_rn(x);
+                            const __nv_bfloat16 lo = __float2bfloat16_rn(x - __bfloat162float(hi));
+                            const uint32_t off = LK::off(row, j >> 3) + (j & 7) * 2;
+                            *reinterpret_cast<__nv_bfloat16 *>(dk + off) = hi;
+                            *reinterpret_cast<__nv_bfloat16 *>(dk + Ly.wk_part + off) = lo;
+                        }
+                        for (int e = r; e < RV * kD; e += kSoftThreads) {
+                            const int j = e / kD, k = e - j * kD;
+                            const float x = wv[e];
+                            const __nv_bfloat16 hi = __float2bfloat16_rn(x);
+                            const __nv_bfloat16 lo = __float2bfloat16_rn(x - __bfloat162float(hi));
+                            const uint32_t off = LV::off(k, j >> 3) + (j & 7) * 2;
+                            *reinterpret_cast<__nv_bfloat16 *>(dv + off) = hi;
+                            *reinterpret_cast<__nv_bfloat16 *>(dv + Ly.wv_part + off) = lo;
+                        }
+                        const float mk = a.mu_k[gi * kD + r];
+                        const int row = ROPE ? pair_row(r, style) : r;
+                        reinterpret_cast<float *>(smem + Ly.muk)[t * kD + row] = mk;
+                        reinterpret_cast<float *>(smem + Ly.muv)[t * kD + r] = a.mu_v[gi * kD + r];
+                        if (ROPE) { // mu_t^K as the B tile of the ones MMA: columns 0, 1 = hi, lo
+                            const __nv_bfloat16 hi = __float2bfloat16_rn(mk);
+                            const __nv_bfloat16 lo = __float2bfloat16_rn(mk - __bfloat162float(hi));
+                            const __nv_bfloat162 hl = __halves2bfloat162(hi, lo);
+                            uint8_t *mt = smem + Ly.muk_t + t * kD * 32;
+                            *reinterpret_cast<uint4 *>(mt + L16::off(row, 0)) =
+                                make_uint4(*reinterpret_cast<const uint32_t *>(&hl), 0u, 0u, 0u);
+                            *reinterpret_cast<uint4 *>(mt + L16::off(row, 1)) = make_uint4(0u, 0u, 0u, 0u);
+                        }
+                    }
+                    // scaled query of this (sequence, head) and loop, in the kernel's row order
+                    const __nv_bfloat16 *qrow =
+                        static_cast<const __nv_bfloat16 *>(a.q) + (((int64_t)d.b * a.Tq_all + a.tq_off + t) * H + d.h) * kD;
+                    reinterpret_cast<float *>(smem + Ly.qv)[t * kD + (ROPE ? pair_row(r, style) : r)] =
+                        __bfloat162float(qrow[r]) * a.scale * kLog2e;
+                }
+                if (wchange)
+                    fence_proxy_async_smem(); // W and mu tiles are read by the tensor cores
+                asm volatile("bar.sync 1, %0;" ::"r"(kSoftThreads) : "memory");
+                if (wchange && r == 0)
+                    mbar_arrive(bar(BWREADY));
+                prev_h = d.h;
+                if (!ROPE && warp < lp) { // constant score term q . mu_t^K (log2 units)
+                    const float *mk = reinterpret_cast<const float *>(smem + Ly.muk) + warp * kD;
+                    float qm = 0.f;
+                    for (int k = lane; k < kD; k += 32)
+                        qm = fmaf(qv[warp * kD + k], mk[k], qm);
+#pragma unroll
+                    for (int off = 16; off > 0; off >>= 1)
+                        qm += __shfl_xor_sync(0xffffffffu, qm, off);
+                    if (lane == 0)
+                        reinterpret_cast<float *>(smem + Ly.qmu)[warp] = qm;
+                }
+                if (ROPE)
+                    qpos = a.q_pos[d.b];
+                asm volatile("bar.sync 1, %0;" ::"r"(kSoftThreads) : "memory");
+#pragma unroll
+                for (int t = 0; t < kMaxLoops; ++t) {
+                    m[t] = -INFINITY;
+                    l[t] = 0.f;
+#pragma unroll
+                    for (int w = 0; w < kSoftWarps; ++w)
+                        oacc[t][w] = 0.f;
+                }
+            }
+            const int qb = tile & 1;
+            if (ROPE) {
+                // the tile's query: R((p - n0) w) q, pairs 2c and 2c + 1 of loop t
+                const int c = r & 31, t = r >> 5;
+                if (t < lp) {
+                    const double *omg = reinterpret_cast<const double *>(smem + Ly.omg);
+                    const int64_t rel = (int64_t)qpos - d.n0;
+                    float qa2[2], qb2[2];
+#pragma unroll
+                    for (int e = 0; e < 2; ++e) {
+                        const int i = 2 * c + e;
+                        const double ang = (double)rel * omg[i];
+                        const float red = (float)(ang - 6.283185307179586 * rint(ang * 0.15915494309189535));
+                        float sn, cs;
+                        sincosf(red, &sn, &cs);
+                        const float x = qv[t * kD + i], y = qv[t * kD + i + kD / 2];
+                        qa2[e] = x * cs - y * sn;
+                        qb2[e] = x * sn + y * cs;
+                    }
+                    reinterpret_cast<float4 *>(smem + Ly.qt4)[(qb * lp + t) * 32 + c] =
+                        make_float4(qa2[0], qa2[1], qb2[0], qb2[1]);
+                    reinterpret_cast<float2 *>(smem + Ly.qtn)[(qb * lp + t) * 32 + c] = make_float2(-qa2[0], -qa2[1]);
+                }
+                asm volatile("bar.sync 1, %0;" ::"r"(kSoftThreads) : "memory");
+            }
+#pragma unroll
+            for (int t = 0; t < kMaxLoops; ++t) {
+                if (t >= lp)
+                    break;
+                // ---- step s: scores of loop t for this thread's token row
+                float sc = -INFINITY;
+                const bool ok = wait_all(bar(BKFULL), s & 1);
+                if (ok) {
+                    tc::fence_after();
+                    float2 acc = make_float2(0.f, 0.f);
+                    if (!ROPE) {
+                        uint32_t kr[128];
+                        tc::ld_x32(trow + kColK, *reinterpret_cast<uint32_t(*)[32]>(kr));
+                        tc::ld_x32(trow + kColK + 32, *reinterpret_cast<uint32_t(*)[32]>(kr + 32));
+                        tc::ld_x32(trow + kColK + 64, *reinterpret_cast<uint32_t(*)[32]>(kr + 64));
+                        tc::ld_x32(trow + kColK + 96, *reinterpret_cast<uint32_t(*)[32]>(kr + 96));
+                        tc::wait_ld();
+                        tc::fence_before();
+                        __syncwarp();
+                        if (lane == 0)
+                            mbar_arrive(bar(BKEMPTY));
+                        const float4 *q4 = reinterpret_cast<const float4 *>(qv + t * kD);
+#pragma unroll
+                        for (int c = 0; c < kD / 4; ++c) {
+                            const float4 qq = q4[c];
+                            acc = __ffma2_rn(make_float2(qq.x, qq.y), f2(kr[4 * c], kr[4 * c + 1]), acc);
+                            acc = __ffma2_rn(make_float2(qq.z, qq.w), f2(kr[4 * c + 2], kr[4 * c + 3]), acc);
+                        }
+                        sc = acc.x + acc.y + qmu[t];
+                    } else {
+                        const float4 *q4 = reinterpret_cast<const float4 *>(smem + Ly.qt4) + (qb * lp + t) * 32;
+                        const float2 *qn = reinterpret_cast<const float2 *>(smem + Ly.qtn) + (qb * lp + t) * 32;
+#pragma unroll
+                        for (int qt = 0; qt < 4; ++qt) { // pairs 16 qt .. 16 qt + 15
+                            uint32_t ka[16], kb[16];
+                            tc::ld_x16(trow + kColK + 16 * qt, ka);
+                            tc::ld_x16(trow + kColK + kD / 2 + 16 * qt, kb);
+                            tc::wait_ld();
+                            if (qt == 3) {
+                                tc::fence_before();
+                                __syncwarp();
+                                if (lane == 0)
+                                    mbar_arrive(bar(BKEMPTY));
+                            }
+#pragma unroll
+                            for (int cc = 0; cc < 8; ++cc) {
+                                const int c = 8 * qt + cc;
+                                const float4 qq = q4[c];
+                                const float2 qa = make_float2(qq.x, qq.y), qbv = make_float2(qq.z, qq.w);
+                                // x (qa cos + qb sin) + y (qb cos - qa sin), two pairs at once
+                                const float2 t1 = __ffma2_rn(qa, rc[c], __fmul2_rn(qbv, rs[c]));
+                                const float2 t2 = __ffma2_rn(qbv, rc[c], __fmul2_rn(qn[c], rs[c]));
+                                acc = __ffma2_rn(f2(ka[2 * cc], ka[2 * cc + 1]), t1, acc);
+                                acc = __ffma2_rn(f2(kb[2 * cc], kb[2 * cc + 1]), t2, acc);
+                            }
+                        }
+                        sc = acc.x + acc.y;
+                    }
+                } else {
+                    __syncwarp();
+                    if (lane == 0)
+                        mbar_arrive(bar(BKEMPTY));
+                }
+                if (r >= d.rows)
+                    sc = -INFINITY;
+                // ---- online softmax, warp-local max (lazy rescale)
+                float mx = sc;
+#pragma unroll
+                for (int off = 16; off > 0; off >>= 1)
+                    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
+                float al = 1.f;
+                if (mx > m[t] + kRescale) {
+                    al = fast_exp2(m[t] - mx);
+                    m[t] = mx;
+                    l[t] *= al;
+                }
+                const float p = sc == -INFINITY ? 0.f : fast_exp2(sc - m[t]);
+                l[t] += p;
+                const float p_hi = __uint_as_float(__float_as_uint(p) & 0xffffe000u); // tf32-exact part
+                const float p_lo = p - p_hi;
+                // P rows 2w (hi) and 2w + 1 (lo), token column r, slab w (128B swizzle)
+                uint8_t *pb = smem + Ly.pbuf + (s & 1) * kPBuf + warp * kPSlab;
+                const int ch = lane >> 2;
+                const int n0 = 2 * warp, n1 = 2 * warp + 1;
+                *reinterpret_cast<float *>(pb + n0 * 128 + ((ch ^ (n0 & 7)) << 4) + (lane & 3) * 4) = p_hi;
+                *reinterpret_cast<float *>(pb + n1 * 128 + ((ch ^ (n1 & 7)) << 4) + (lane & 3) * 4) = p_lo;
+                if (lane == 0)
+                    alpha[(s & 3) * kSoftWarps + warp] = al;
+                fence_proxy_async_smem();
+                __syncwarp();
+                if (lane == 0)
+                    mbar_arrive(bar(BPFULL0 + (s & 1)));
+                // ---- the previous step's output
+                if (pend >= 0)
+                    readout(pend, pend_t);
+                pend = s;
+                pend_t = t;
+                ++s;
+            }
+            ++tile;
+        }
+        if (pend >= 0) {
+            readout(pend, pend_t);
+            flush(dseg);
+        }
+    }
+    // ---- teardown: every MMA complete before tensor memory is released
+    __syncwarp();
+    __syncthreads();
+    if (warp == kMmaWarp) {
+        if (lane == 0)
+            tc::commit(bar(BDRAIN));
+        __syncwarp();
+        (void)mbar_wait_bounded(bar(BDRAIN), 0);
+        __syncwarp();
+        tc::fence_after();
+        tc::dealloc(tmem, kTmemCols);
+    }
+    if (misc[0] != 0 && warp == kProducerWarp && lane == 0) {
+        report_status(a.status, LLA_ERR_DEVICE_TIMEOUT);
+        const int issued = misc[2];
+        for (int i = issued - (int)nst < 0 ? 0 : issued - (int)nst; i < issued; ++i)
+            (void)mbar_wait_bounded(full_bar(i % nst), (i / nst) & 1);
+    }
+}
+
+template <int RK, int RV, bool ROPE> cudaError_t launch_rtc(const DecodeArgs &a, cudaStream_t stream)
+{
+    CUtensorMap mk, mkt, mv, mvt;
+    if (!plane_maps(&mk, &mkt, a.k, RK, (int64_t)a.H * a.slots) ||
+        !plane_maps(&mv, &mvt, a.v, RV, (int64_t)a.H * a.slots))
+        return cudaErrorInvalidValue;
+    if (a.Tq < 1 || a.Tq > kMaxLoops)
+        return cudaErrorInvalidValue;
+    auto kern = decode_recon_tc_kernel<RK, RV, ROPE>;
+    const int smem = (int)rlayout<RK, RV, ROPE>(a.Tq, a.B).total + 1024;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e != cudaSuccess)
+        return e;
+    int dev = 0, sms = 148;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    // tail maps only: ranks up to 32 are one 32- or 64-byte box column
+    kern<<<sms, kThreads, smem, stream>>>(mkt, mvt, a);
+    return cudaGetLastError();
+}
+
+} // namespace
+
+int decode_recon_tc_smem_bytes(int r_k, int r_v, bool rope, int lp, int B)
+{
+#define LLA_RTC_SMEM(RK, RV) \
+    if (r_k == RK && r_v == RV) \
+        return (int)(rope ? rlayout<RK, RV, true>(lp, B).total : rlayout<RK, RV, false>(lp, B).total) + 1024;
+    LLA_RTC_SMEM(16, 32)
+    LLA_RTC_SMEM(16, 16)
+    LLA_RTC_SMEM(32, 32)
+#undef LLA_RTC_SMEM
+    return -1;
+}
+
+bool decode_recon_tc_supported(int dtype, int r_k, int r_v, int d, int fold, int B, bool rope)
+{
+    if (dtype != LLA_BF16 || d != kD || fold != LLA_PER_HEAD || tensor_map_encoder() == nullptr)
+        return false;
+    const int smem = decode_recon_tc_smem_bytes(r_k, r_v, rope, kMaxLoops, B);
+    return smem > 0 && smem <= 227 * 1024;
+}
+
+int decode_recon_tc_loops_per_pass() { return kMaxLoops; }
+
+cudaError_t launch_decode_recon_tc(const DecodeArgs &a, cudaStream_t stream)
+{
+#define LLA_RTC_CASE(RK, RV) \
+    if (a.r_k == RK && a.r_v == RV) \
+        return a.q_pos != nullptr ? launch_rtc<RK, RV, true>(a, stream) : launch_rtc<RK, RV, false>(a, stream);
+    LLA_RTC_CASE(16, 32)
+    LLA_RTC_CASE(16, 16)
+    LLA_RTC_CASE(32, 32)
+#undef LLA_RTC_CASE
+    return cudaErrorNotSupported;
+}
+
+} // namespace lla

@@ -487,6 +487,26 @@ int decode_call(const lla_dims *dims, int32_t layer, int32_t t0, int32_t Tq, con
     auto window_pass = [&](const DecodeArgs &ac) -> cudaError_t {
         return window != nullptr ? launch_decode_window(ac, dims->dtype, s) : cudaSuccess;
     };
+    if (variant == LLA_RECONSTRUCT &&
+        decode_recon_tc_supported(dims->dtype, dims->r_k, dims->r_v, dims->d_head, dims->fold, B, rope != nullptr)) {
+        // tensor-memory kernel: one pass over the latents per (up to 4) loop queries
+        const int per = decode_recon_tc_loops_per_pass();
+        for (int32_t c = 0; c < Tq && err == cudaSuccess; c += per) {
+            DecodeArgs ac = a;
+            ac.tq_off = c;
+            ac.Tq = Tq - c < per ? Tq - c : per;
+            err = mark(c == 0 ? e0 : nullptr);
+            if (err == cudaSuccess)
+                err = launch_decode_recon_tc(ac, s);
+            if (err == cudaSuccess && c + per >= Tq)
+                err = mark(e1);
+        }
+        if (err == cudaSuccess)
+            err = window_pass(a);
+        if (err == cudaSuccess)
+            err = launch_decode_combine(a, dims->dtype, dims->out_dtype, s);
+        return err == cudaSuccess ? LLA_OK : LLA_ERR_CUDA;
+    }
     if (variant == LLA_RECONSTRUCT) {
         // one pass over the latents per loop query, then one merge of all records
         for (int32_t c = 0; c < Tq && err == cudaSuccess; ++c) {

@@ -1,0 +1,129 @@
+// tc_common.cuh -- tcgen05 (5th-generation tensor core) helpers for the sm_100a kernels
+// that keep their accumulators in tensor memory: shared-memory operand descriptors for
+// the swizzled K-major layouts, instruction descriptors, MMA issue (operands in shared
+// memory, or A in tensor memory), commits, tensor-memory loads and allocation.
+#pragma once
+
+#include "common.cuh"
+
+namespace lla {
+namespace tc {
+
+// Layout codes of the shared-memory descriptor (bits 61-63) for K-major operands whose
+// rows are 32, 64 or 128 bytes with the matching swizzle (8-row atoms).
+constexpr int kSw128 = 2, kSw64 = 4, kSw32 = 6;
+
+// Swizzle code for operand rows of `row_bytes` bytes.
+__host__ __device__ constexpr int swizzle_of(int row_bytes)
+{
+    return row_bytes == 32 ? kSw32 : (row_bytes == 64 ? kSw64 : kSw128);
+}
+
+// Descriptor of a K-major operand tile starting at shared address `addr`: rows of
+// `row_bytes` bytes (32, 64 or 128), 8-row groups `8 * row_bytes` apart.  Moving the start
+// by 32 bytes inside a row selects the next 16 bf16 (or 8 tf32) values of K; the swizzle
+// is applied to the resulting addresses, the same way the TMA wrote them.
+__device__ __forceinline__ uint64_t smem_desc(uint32_t addr, int row_bytes)
+{
+    uint64_t d = 0;
+    d |= (uint64_t)((addr >> 4) & 0x3FFFu);                      // start address
+    d |= (uint64_t)1 << 16;                                       // leading offset (unused here)
+    d |= (uint64_t)(((uint32_t)(8 * row_bytes) >> 4) & 0x3FFFu) << 32; // stride offset: 8 rows
+    d |= (uint64_t)1 << 46;                                       // descriptor version (sm_100)
+    d |= (uint64_t)swizzle_of(row_bytes) << 61;                   // swizzle mode
+    return d;
+}
+
+constexpr int kFmtBf16 = 1, kFmtTf32 = 2;
+
+// Instruction descriptor: fp32 accumulator, A and B of format `fmt` (both K-major),
+// M x N tile.  kind::f16 takes kFmtBf16, kind::tf32 takes kFmtTf32.
+__host__ __device__ constexpr uint32_t idesc(int fmt, int m, int n)
+{
+    return (1u << 4) | ((uint32_t)fmt << 7) | ((uint32_t)fmt << 10) | ((uint32_t)(n >> 3) << 17) |
+           ((uint32_t)(m >> 4) << 24);
+}
+
+__device__ __forceinline__ void fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
+
+// D (tensor memory) (+)= A (shared) . B (shared), bf16 inputs.
+__device__ __forceinline__ void mma_bf16(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t id,
+                                         uint32_t accumulate)
+{
+    asm volatile(
+        "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "l"(a_desc), "l"(b_desc), "r"(id), "r"(accumulate)
+        : "memory");
+}
+
+// D (tensor memory) (+)= A (tensor memory, 32-bit values read as tf32) . B (shared, tf32).
+__device__ __forceinline__ void mma_tf32_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t id,
+                                            uint32_t accumulate)
+{
+    asm volatile(
+        "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::tf32 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "r"(a_tmem), "l"(b_desc), "r"(id), "r"(accumulate)
+        : "memory");
+}
+
+// Arrive once on `bar` when every tcgen05 operation this thread issued so far completes.
+__device__ __forceinline__ void commit(uint32_t bar)
+{
+    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar)
+                 : "memory");
+}
+
+// Tensor-memory loads: thread i of the warp reads lane (warp's lane quarter) + i, N
+// consecutive 32-bit columns from `taddr` on.  Complete after wait_ld().
+__device__ __forceinline__ void ld_x32(uint32_t taddr, uint32_t (&r)[32])
+{
+    asm volatile("tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, "
+                 "%12, %13, %14, %15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, "
+                 "%30, %31}, [%32];"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+                   "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
+                   "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]),
+                   "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]),
+                   "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+                 : "r"(taddr));
+}
+
+__device__ __forceinline__ void ld_x16(uint32_t taddr, uint32_t (&r)[16])
+{
+    asm volatile("tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, "
+                 "%12, %13, %14, %15}, [%16];"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+                   "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
+                   "=r"(r[14]), "=r"(r[15])
+                 : "r"(taddr));
+}
+
+__device__ __forceinline__ void ld_x8(uint32_t taddr, uint32_t (&r)[8])
+{
+    asm volatile("tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%8];"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+                   "=r"(r[7])
+                 : "r"(taddr));
+}
+
+__device__ __forceinline__ void wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
+
+// Whole-warp allocation of `cols` tensor-memory columns; the base address lands in *dst.
+__device__ __forceinline__ void alloc(uint32_t *dst, uint32_t cols)
+{
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(dst)),
+                 "r"(cols)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+}
+
+__device__ __forceinline__ void dealloc(uint32_t taddr, uint32_t cols)
+{
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(cols) : "memory");
+}
+
+} // namespace tc
+} // namespace lla

@@ -56,3 +56,28 @@ def test_lla2d_small_rank_both_variants(variant):
     assert st == 0
     o_ref, l_ref = oracle_decode(p, w, 0, 0, 4, 1.0, variant="reconstruct")
     assert_attn_close(out, lse, o_ref, l_ref)
+
+
+@pytest.mark.parametrize("Tq,t0", [(6, 1), (5, 0)])
+def test_reconstruct_more_loop_queries_than_one_latent_pass(Tq, t0):
+    """Eight loops: a call with 5 or 6 loop queries reads the latents in two passes (4 + the
+    rest); both passes' records meet in the one combine."""
+    w = S.shrink(S.WORKLOADS["ouro1.4b-layer"], name="rec-T8", T=8, B=6, len_lo=200, len_hi=2500)
+    p = S.decode_inputs(w, 0, DEV, Tq=Tq, perturb=0.1)
+    out, lse, st = run_decode(p, w, 0, t0, Tq, 1.0, variant=REC)
+    assert st == 0
+    o_ref, l_ref = oracle_decode(p, w, 0, t0, Tq, 1.0, variant="reconstruct")
+    assert_attn_close(out, lse, o_ref, l_ref)
+
+
+@pytest.mark.parametrize("rk,rv", [(16, 32), (32, 32), (16, 16)])
+def test_reconstruct_large_logits_and_ranks(rk, rv):
+    """Softmax scale 30: sharp rows stress the running max and the precision of the rebuilt
+    keys (W_up enters the tensor cores as bf16 hi + lo parts)."""
+    w = S.shrink(S.WORKLOADS["ouro1.4b-layer"], name=f"rec-big-{rk}-{rv}", r_k=rk, r_v=rv, B=5,
+                 len_lo=130, len_hi=2100)
+    p = S.decode_inputs(w, 0, DEV)
+    out, lse, st = run_decode(p, w, 0, 0, 4, 30.0, variant=REC)
+    assert st == 0
+    o_ref, l_ref = oracle_decode(p, w, 0, 0, 4, 30.0, variant="reconstruct")
+    assert_attn_close(out, lse, o_ref, l_ref)
