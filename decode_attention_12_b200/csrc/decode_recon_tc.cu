@@ -8,32 +8,34 @@
 // (Pith verdict record, key_machinery; RoFormer's rotation).
 //
 // One latent tile of 128 tokens is read from HBM once and serves every loop query t of
-// the pass (up to 4).  Per (tile, loop) step, on the tensor cores (one issuing thread):
-//     K_hat   [128 tok x d] = C_K . W_up,t^K        M = tokens, N = d, K = r_k  (TMEM)
-//     V_hat^T [d x 128 tok] = W_up,t^V^T . C_V^T    M = d, N = tokens, K = r_v  (TMEM)
-//     O^T     [d x 16]      = V_hat^T . P^T         kind::tf32, A read straight from TMEM
-// W_up,t enters as bf16 hi + lo parts (two MMAs, products exact in fp32), so K_hat and
-// V_hat carry about 16 mantissa bits of W_up; the P.V_hat MMA reads V_hat as tf32 (10
-// bits) and p as tf32 hi + lo parts.  mu_t^V is left out of V_hat and added once per
-// record (sum_n p_n (v_hat_n - mu) + mu sum_n p_n); the score term q . mu_t^K is a
-// constant per (unit, loop) -- with rotation the key's mean turns with the key, so there
-// K_hat takes mu_t^K from one more MMA (a ones column times mu's hi/lo parts).
+// the pass (up to 4).  Per (tile, loop) step one thread issues, on the tensor cores,
+//     K_hat   [128 tok x d] = C_K . W_up,t^K       M = tokens, N = d, K = r_k
+//     V_hat^T [d x 128 tok] = W_up,t^V^T . C_V^T   M = d, N = tokens, K = r_v
+// into tensor memory.  W_up,t enters as bf16 hi + lo parts (two MMAs whose products are
+// exact in the fp32 accumulator), so the rebuilt vectors carry about 16 mantissa bits of
+// W_up against exact bf16 latents.  mu_t^V is left out of V_hat and added once per record
+// (sum_n p_n (v_hat_n - mu) + mu sum_n p_n); the score term q . mu_t^K is one constant per
+// (unit, loop) -- with rotation the key's mean turns with the key, so there K_hat takes
+// mu_t^K from one more MMA (a ones column against mu's hi/lo parts).
 //
-// Scores, softmax and output accumulation run on 4 warps, one tensor-memory lane quarter
-// each: thread r owns token row r of K_hat (its score is a 128-long dot product in
-// registers, packed fp32x2 FMAs), keeps a warp-local running max per loop and writes p
-// into rows 2w (hi) and 2w + 1 (lo) of P, so the P.V_hat MMA returns one column pair per
-// warp and no cross-warp reduction is needed per step; the same thread, as lane d of the
-// O^T accumulator, folds each step's column pairs into per-warp output sums with the
-// warps' rescale factors.  Records (acc, m, l) are merged across warps at segment ends
-// and have the layout of the other reconstruct kernels, so the combine is shared.
+// Two warpgroups of 4 warps take alternate steps, each with its own K_hat and V_hat^T
+// buffers (4 x 128 of the 512 tensor-memory columns), so one group's scores overlap the
+// other's output sums and the tensor cores' next rebuild.  Within a group, thread r:
+//   * reads token row r of K_hat (its score is a d-long dot product in registers, packed
+//     fp32x2 FMAs, several independent chains), keeps a warp-local running max per loop
+//     (lazy rescale) and writes p to shared memory;
+//   * after the group's barrier reads row r of V_hat^T -- the d-index r of every token --
+//     and forms the 32-token partial sums sum_n p_n v_hat_n[r] of each warp's tokens,
+//     folded into per-warp output sums with the warps' rescale factors.
+// Records (acc, m, l) are merged across the 8 warps at segment ends and have the layout
+// of the other reconstruct kernels, so the combine is shared.
 //
 // Faithful read: a query at position p and the rebuilt key of token n = n0 + r (tile row
-// r) give <R(p) q, R(n) k> = <R(p - n0) q, R(r) k>: the query is turned once per tile by
-// (p - n0) (angles in double precision), and every thread keeps cos/sin(r w_i) of its row
-// in registers for the whole kernel.  Component pairs (i, i + d/2) sit in one thread: the
-// rows of W_up,t^K, q and mu_t^K are staged pair-major (identity for the half-split
-// pairing, even-first for RoFormer's interleaved one).
+// r) give <R(p) q, R(n) k> = <R(p - n0) q, R(r) k>: each group turns the query once per
+// tile by (p - n0) (angles in double precision), and every thread keeps cos/sin(r w_i) of
+// its row in registers for the whole kernel.  Component pairs (i, i + d/2) sit in one
+// thread: the rows of W_up,t^K, q and mu_t^K are staged pair-major (identity for the
+// half-split pairing, even-first for RoFormer's interleaved one).
 //
 // Work split: the token stream of all (head, sequence) units in head-major order is cut
 // into equal shares, one per CTA (one CTA per SM), so a CTA's share mostly stays within
@@ -49,31 +51,29 @@ using namespace mma;
 constexpr int kD = 128;         // head dimension served
 constexpr int kTile = 128;      // tokens per latent tile (M of the K_hat MMA)
 constexpr int kMaxLoops = 4;    // loop queries per pass
-constexpr int kSoftWarps = 4;   // warps 0-3: scores, softmax, output
-constexpr int kProducerWarp = 4, kMmaWarp = 5;
-constexpr int kThreads = 6 * 32;
-constexpr int kSoftThreads = kSoftWarps * 32;
+constexpr int kGroups = 2;      // softmax warpgroups, alternate steps
+constexpr int kGroupThreads = 128;
+constexpr int kSoftThreads = kGroups * kGroupThreads;
+constexpr int kProducerWarp = 8, kMmaWarp = 9; // warps 10, 11 complete the third warpgroup
+constexpr int kThreads = 12 * 32;
+// Register split (setmaxnreg): launched at 168 per thread (384 x 168 = 64,512 of the SM's
+// 65,536), the producer/MMA warpgroup gives back to 40 and the two softmax warpgroups take
+// 232: 2 x 128 x 232 + 128 x 40 = 64,512, exactly the launch's total.
+constexpr int kLaunchRegs = 168, kSoftRegs = 232, kIssueRegs = 40;
+static_assert(2 * 128 * kSoftRegs + 128 * kIssueRegs <= kThreads * kLaunchRegs, "register split exceeds the launch");
 constexpr float kRescale = 8.0f; // lazy rescale margin (log2 units)
 
-// tensor-memory columns
+// tensor-memory columns: K_hat of group g at 128 g, V_hat^T of group g at 256 + 128 g
 constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t kColK = 0;    // K_hat [128 tokens (lanes)][128 d] fp32
-constexpr uint32_t kColV = 128;  // V_hat^T [128 d (lanes)][128 tokens] fp32, two buffers
-constexpr uint32_t kColO = 384;  // O^T [128 d (lanes)][16] fp32, two buffers
-
-constexpr int kPRows = 16;                 // N of the P.V_hat MMA
-constexpr int kPSlab = kPRows * 128;       // 32 tokens (128 B of tf32) x 16 rows, 128B swizzle
-constexpr int kPBuf = 4 * kPSlab;          // 128 tokens
+__device__ __forceinline__ uint32_t col_k(int g) { return 128u * g; }
+__device__ __forceinline__ uint32_t col_v(int g) { return 256u + 128u * g; }
 
 // barriers after the ring's full[NST] and empty[NST]
-enum {
-    BKFULL = 0, BKEMPTY, BVFULL0, BVFULL1, BPFULL0, BPFULL1, BOFULL0, BOFULL1, BOEMPTY0, BOEMPTY1, BWREADY,
-    BDRAIN, BCOUNT
-};
+enum { BKFULL0 = 0, BKFULL1, BKEMPTY0, BKEMPTY1, BVFULL0, BVFULL1, BVEMPTY0, BVEMPTY1, BWREADY, BDRAIN, BCOUNT };
 
 struct RLayout {
-    uint32_t nst, stage, wk, wv, wk_part, wv_part, pbuf, ones, muk_t, qv, qt4, qtn, muk, muv, qmu, alpha, mrg, omg,
-        bar, misc, scr, pref, total;
+    uint32_t nst, stage, wk, wv, wk_part, wv_part, ones, muk_t, qv, qt4, qtn, muk, muv, pv, alpha, xch, qmu, mrg,
+        omg, bar, misc, scr, pref, total;
 };
 
 __host__ __device__ inline uint32_t round_up(uint32_t x, uint32_t a) { return (x + a - 1) / a * a; }
@@ -94,28 +94,30 @@ template <int RK, int RV, bool ROPE> __host__ __device__ inline RLayout rlayout(
     o += lp * 2 * L.wk_part;
     L.wv = o;
     o += lp * 2 * L.wv_part;
-    L.pbuf = o;
-    o += 2 * kPBuf;
     L.ones = o;
     o += ROPE ? kTile * 32 : 0;
     L.muk_t = o;
     o += ROPE ? lp * kD * 32 : 0;
-    L.qv = o;
+    L.qv = o;                       // [lp][d] scaled query (kernel row order)
     o += lp * kD * 4;
-    L.qt4 = o;
-    o += ROPE ? 2 * lp * 32 * 16 : 0;
-    L.qtn = o;
-    o += ROPE ? 2 * lp * 32 * 8 : 0;
-    L.muk = o;
+    L.qt4 = o;                      // [group][2 tiles][lp][32] turned query, pairs 2c, 2c+1
+    o += ROPE ? kGroups * 2 * lp * 32 * 16 : 0;
+    L.qtn = o;                      // [group][2 tiles][lp][32] minus its first parts
+    o += ROPE ? kGroups * 2 * lp * 32 * 8 : 0;
+    L.muk = o;                      // [lp][d]
     o += lp * kD * 4;
-    L.muv = o;
+    L.muv = o;                      // [lp][d]
+    o += lp * kD * 4;
+    L.pv = o;                       // [group][2][128] softmax weights of a step
+    o += kGroups * 2 * kTile * 4;
+    L.alpha = o;                    // [group][2][4 warps] rescale factors of a step
+    o += kGroups * 2 * 4 * 4;
+    L.xch = o;                      // [lp][d] group 1's share of a record
     o += lp * kD * 4;
     L.qmu = o;
     o += 16;
-    L.alpha = o;
-    o += 4 * kSoftWarps * 4;
-    L.mrg = o;
-    o += kSoftWarps * kMaxLoops * 2 * 4;
+    L.mrg = o;                      // [8 warps][4 loops][m, l]
+    o += 8 * kMaxLoops * 2 * 4;
     L.omg = round_up(o, 8);
     o = L.omg + (ROPE ? kD / 2 * 8 : 0);
     L.bar = round_up(o, 8);
@@ -211,6 +213,13 @@ template <int TILE> struct HeadWalk {
 
 __device__ __forceinline__ float2 f2(uint32_t x, uint32_t y) { return make_float2(__uint_as_float(x), __uint_as_float(y)); }
 
+__device__ __forceinline__ void group_sync(int g)
+{
+    asm volatile("bar.sync %0, %1;" ::"r"(1 + g), "r"(kGroupThreads) : "memory");
+}
+__device__ __forceinline__ void soft_sync() { asm volatile("bar.sync 3, %0;" ::"r"(kSoftThreads) : "memory"); }
+__device__ __forceinline__ void all_sync() { asm volatile("bar.sync 4, %0;" ::"r"(kThreads) : "memory"); }
+
 template <int RK, int RV, bool ROPE>
 __global__ void __launch_bounds__(kThreads, 1)
     decode_recon_tc_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant__ CUtensorMap map_v,
@@ -229,8 +238,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t nst = Ly.nst;
     volatile int *misc = reinterpret_cast<volatile int *>(smem + Ly.misc); // [0] error, [1] tmem, [2] issued
     int64_t *pref = reinterpret_cast<int64_t *>(smem + Ly.pref);
-    float *alpha = reinterpret_cast<float *>(smem + Ly.alpha); // [4 steps][4 warps]
-    float *mrg = reinterpret_cast<float *>(smem + Ly.mrg);     // [4 warps][4 loops][m, l]
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int B = a.B, H = a.H;
     auto full_bar = [&](int st) { return bar0 + 8u * st; };
@@ -242,16 +249,12 @@ __global__ void __launch_bounds__(kThreads, 1)
             mbar_init(full_bar(st), 1);  // producer's expect_tx + TMA bytes
             mbar_init(empty_bar(st), 1); // the tile's last MMAs completed (commit)
         }
-        mbar_init(bar(BKFULL), 1);
-        mbar_init(bar(BKEMPTY), kSoftWarps);
-        mbar_init(bar(BVFULL0), 1);
-        mbar_init(bar(BVFULL1), 1);
-        mbar_init(bar(BPFULL0), kSoftWarps);
-        mbar_init(bar(BPFULL1), kSoftWarps);
-        mbar_init(bar(BOFULL0), 1);
-        mbar_init(bar(BOFULL1), 1);
-        mbar_init(bar(BOEMPTY0), kSoftWarps);
-        mbar_init(bar(BOEMPTY1), kSoftWarps);
+        for (int g = 0; g < kGroups; ++g) {
+            mbar_init(bar(BKFULL0 + g), 1);
+            mbar_init(bar(BKEMPTY0 + g), 4); // one arrival per warp of the group
+            mbar_init(bar(BVFULL0 + g), 1);
+            mbar_init(bar(BVEMPTY0 + g), 4);
+        }
         mbar_init(bar(BWREADY), 1);
         mbar_init(bar(BDRAIN), 1);
         misc[0] = 0;
@@ -260,22 +263,19 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     if (warp == kMmaWarp)
         tc::alloc(reinterpret_cast<uint32_t *>(smem + Ly.misc + 4), kTmemCols);
-    // P buffers start (and, outside each warp's own two rows, stay) zero
-    for (int e = tid; e < 2 * kPBuf / 16; e += kThreads)
-        reinterpret_cast<uint4 *>(smem + Ly.pbuf)[e] = make_uint4(0u, 0u, 0u, 0u);
     if (ROPE) {
         // ones tile [128 rows][16]: columns 0 and 1 are 1 (they meet mu's hi and lo parts)
         const __nv_bfloat162 one2 = __floats2bfloat162_rn(1.f, 1.f);
         for (int r = tid; r < kTile; r += kThreads) {
-            uint4 c0 = make_uint4(*reinterpret_cast<const uint32_t *>(&one2), 0u, 0u, 0u);
-            *reinterpret_cast<uint4 *>(smem + Ly.ones + L16::off(r, 0)) = c0;
+            *reinterpret_cast<uint4 *>(smem + Ly.ones + L16::off(r, 0)) =
+                make_uint4(*reinterpret_cast<const uint32_t *>(&one2), 0u, 0u, 0u);
             *reinterpret_cast<uint4 *>(smem + Ly.ones + L16::off(r, 1)) = make_uint4(0u, 0u, 0u, 0u);
         }
         double *omg = reinterpret_cast<double *>(smem + Ly.omg);
         for (int i = tid; i < kD / 2; i += kThreads)
             omg[i] = pow((double)a.rope_base, -2.0 * i / kD);
+        fence_proxy_async_smem(); // the ones tile is read by the tensor cores
     }
-    fence_proxy_async_smem(); // generic writes above are read by the tensor cores
     tc::fence_before();
     block_length_prefix<kThreads>(a.ctx_lens, B, pref, reinterpret_cast<int64_t *>(smem + Ly.scr));
     tc::fence_after();
@@ -286,8 +286,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     int64_t s0, s1, chunk;
     cta_share(pref, B, H, a.chunk_min, s0, s1, chunk);
     const int64_t S_tot = pref[B];
-
-    if (s0 < s1 && warp == kProducerWarp) {
+    if (warp >= 8) {
+      // ======== third warpgroup: producer warp, MMA warp, two idle warps ========
+      asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kIssueRegs));
+      if (s0 < s1 && warp == kProducerWarp) {
         // ================= producer: one lane streams the latent tiles =================
         if (lane == 0) {
             HeadWalk<kTile> walk;
@@ -315,10 +317,9 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             misc[2] = issued;
         }
-    } else if (s0 < s1 && warp == kMmaWarp) {
+      } else if (s0 < s1 && warp == kMmaWarp) {
         // ================= MMA issuer: lane 0 issues, the warp waits and zeroes =================
         constexpr uint32_t kIdKV = tc::idesc(tc::kFmtBf16, 128, 128);
-        constexpr uint32_t kIdPV = tc::idesc(tc::kFmtTf32, 128, kPRows);
         bool err = false;
         auto wait_all = [&](uint32_t b, uint32_t parity) -> bool {
             bool ok = !err && misc[0] == 0 && mbar_wait_bounded(b, parity);
@@ -329,31 +330,19 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             return ok;
         };
-        // O^T of step sp: V_hat^T (TMEM) . P^T, 16 k-steps of 8 tokens
-        auto issue_pv = [&](int sp) {
-            const int bb = sp & 1;
-            if (!wait_all(bar(BPFULL0 + bb), (sp >> 1) & 1) || !wait_all(bar(BVFULL0 + bb), (sp >> 1) & 1))
-                return;
-            if (sp >= 2 && !wait_all(bar(BOEMPTY0 + bb), ((sp - 2) >> 1) & 1))
-                return;
-            tc::fence_after();
-            if (lane == 0) {
-                const uint32_t pb = sbase + Ly.pbuf + bb * kPBuf;
-#pragma unroll
-                for (int j = 0; j < kTile / 8; ++j)
-                    tc::mma_tf32_ts(tmem + kColO + 16 * bb, tmem + kColV + 128 * bb + 8 * j,
-                                    tc::smem_desc(pb + (j >> 2) * kPSlab + (j & 3) * 32, 128), kIdPV, j > 0);
-                tc::commit(bar(BOFULL0 + bb));
-            }
-            __syncwarp();
-        };
         HeadWalk<kTile> walk;
         walk.start(s0, s1, chunk, S_tot);
         TileDesc d;
         int s = 0, ti = 0, wc = 0, prev_h = -1;
         while (!err && walk.next(pref, a.seq_start, B, H, d)) {
             const int st = ti % (int)nst;
-            const bool wchange = (d.flags & 1) && d.h != prev_h;
+            if ((d.flags & 1) && d.h != prev_h) {
+                // a new head's W_up: staged once every MMA of the old one has been consumed
+                if (!wait_all(bar(BWREADY), wc & 1))
+                    break;
+                ++wc;
+                prev_h = d.h;
+            }
             if (!wait_all(full_bar(st), (ti / nst) & 1))
                 break;
             const uint32_t sk = sbase + st * Ly.stage, sv = sk + LK::BYTES;
@@ -363,58 +352,68 @@ __global__ void __launch_bounds__(kThreads, 1)
                 fence_proxy_async_smem();
                 __syncwarp();
             }
-            for (int t = 0; t < lp && !err; ++t) {
-                if (t == 0 && wchange) {
-                    // the staging of a new head's W_up waits for every MMA of the old one
-                    if (s >= 1)
-                        issue_pv(s - 1);
-                    if (!wait_all(bar(BWREADY), wc & 1))
-                        break;
-                    ++wc;
-                    prev_h = d.h;
-                }
-                if (s >= 1 && !wait_all(bar(BKEMPTY), (s - 1) & 1))
+            for (int t = 0; t < lp && !err; ++t, ++s) {
+                const int g = s & 1, use = s >> 1; // group g's use number of its buffers
+                if (use >= 1 && !wait_all(bar(BKEMPTY0 + g), (use - 1) & 1))
                     break;
-                if (s >= 2 && !wait_all(bar(BOFULL0 + (s & 1)), ((s - 2) >> 1) & 1))
-                    break; // P.V_hat of step s - 2 has read this V_hat^T buffer
                 tc::fence_after();
                 if (lane == 0) {
                     const uint32_t wk = sbase + Ly.wk + t * 2 * Ly.wk_part;
-                    const uint32_t wv = sbase + Ly.wv + t * 2 * Ly.wv_part;
 #pragma unroll
                     for (int kk = 0; kk < RK / 16; ++kk)
 #pragma unroll
                         for (int hl = 0; hl < 2; ++hl)
-                            tc::mma_bf16(tmem + kColK, tc::smem_desc(sk + 32 * kk, 2 * RK),
+                            tc::mma_bf16(tmem + col_k(g), tc::smem_desc(sk + 32 * kk, 2 * RK),
                                          tc::smem_desc(wk + hl * Ly.wk_part + 32 * kk, 2 * RK), kIdKV, (kk | hl) != 0);
                     if (ROPE)
-                        tc::mma_bf16(tmem + kColK, tc::smem_desc(sbase + Ly.ones, 32),
+                        tc::mma_bf16(tmem + col_k(g), tc::smem_desc(sbase + Ly.ones, 32),
                                      tc::smem_desc(sbase + Ly.muk_t + t * kD * 32, 32), kIdKV, 1);
-                    tc::commit(bar(BKFULL));
-                    const uint32_t vcol = tmem + kColV + 128 * (s & 1);
+                    tc::commit(bar(BKFULL0 + g));
+                }
+                __syncwarp();
+                if (use >= 1 && !wait_all(bar(BVEMPTY0 + g), (use - 1) & 1))
+                    break;
+                tc::fence_after();
+                if (lane == 0) {
+                    const uint32_t wv = sbase + Ly.wv + t * 2 * Ly.wv_part;
 #pragma unroll
                     for (int kk = 0; kk < RV / 16; ++kk)
 #pragma unroll
                         for (int hl = 0; hl < 2; ++hl)
-                            tc::mma_bf16(vcol, tc::smem_desc(wv + hl * Ly.wv_part + 32 * kk, 2 * RV),
+                            tc::mma_bf16(tmem + col_v(g), tc::smem_desc(wv + hl * Ly.wv_part + 32 * kk, 2 * RV),
                                          tc::smem_desc(sv + 32 * kk, 2 * RV), kIdKV, (kk | hl) != 0);
-                    tc::commit(bar(BVFULL0 + (s & 1)));
+                    tc::commit(bar(BVFULL0 + g));
                     if (t == lp - 1)
                         tc::commit(empty_bar(st)); // the tile's stage is free once these complete
                 }
                 __syncwarp();
-                if (!(t == 0 && wchange) && s >= 1)
-                    issue_pv(s - 1);
-                ++s;
             }
             ++ti;
         }
-        if (!err && s >= 1)
-            issue_pv(s - 1);
-    } else if (s0 < s1 && warp < kSoftWarps) {
-        // ================= scores, softmax, output: thread r = token row r / lane d =================
-        const int r = tid;
-        const uint32_t trow = tmem + ((uint32_t)(32 * warp) << 16);
+      }
+      __syncwarp();
+      all_sync(); // the softmax groups have consumed every MMA result
+      if (warp == kMmaWarp) { // every MMA complete before tensor memory is released
+          if (lane == 0)
+              tc::commit(bar(BDRAIN));
+          __syncwarp();
+          (void)mbar_wait_bounded(bar(BDRAIN), 0);
+          __syncwarp();
+          tc::fence_after();
+          tc::dealloc(tmem, kTmemCols);
+      }
+      if (misc[0] != 0 && warp == kProducerWarp && lane == 0) {
+          report_status(a.status, LLA_ERR_DEVICE_TIMEOUT);
+          const int issued = misc[2];
+          for (int i = issued - (int)nst < 0 ? 0 : issued - (int)nst; i < issued; ++i)
+              (void)mbar_wait_bounded(full_bar(i % nst), (i / nst) & 1);
+      }
+    } else {
+      // ======== two groups of 4 warps, alternate steps: thread r = token row r / d-index r ========
+      asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kSoftRegs));
+      if (s0 < s1) {
+        const int g = warp >> 2, wq = warp & 3, r = tid & 127;
+        const uint32_t tq = tmem + ((uint32_t)(32 * wq) << 16); // this warp's lane quarter
         bool err = false;
         auto wait_all = [&](uint32_t b, uint32_t parity) -> bool {
             bool ok = !err && misc[0] == 0 && mbar_wait_bounded(b, parity);
@@ -431,44 +430,21 @@ __global__ void __launch_bounds__(kThreads, 1)
             const float lb = log2f(a.rope_base);
 #pragma unroll
             for (int c = 0; c < 32; ++c) {
-                float s0_, c0_, s1_, c1_;
-                sincosf((float)r * exp2f(-2.0f * (float)(2 * c) / (float)kD * lb), &s0_, &c0_);
-                sincosf((float)r * exp2f(-2.0f * (float)(2 * c + 1) / (float)kD * lb), &s1_, &c1_);
-                rc[c] = make_float2(c0_, c1_);
-                rs[c] = make_float2(s0_, s1_);
+                float sa, ca, sb, cb;
+                sincosf((float)r * exp2f(-2.0f * (float)(2 * c) / (float)kD * lb), &sa, &ca);
+                sincosf((float)r * exp2f(-2.0f * (float)(2 * c + 1) / (float)kD * lb), &sb, &cb);
+                rc[c] = make_float2(ca, cb);
+                rs[c] = make_float2(sa, sb);
             }
         }
-        float m[kMaxLoops], l[kMaxLoops], oacc[kMaxLoops][kSoftWarps];
+        float m[kMaxLoops], l[kMaxLoops], oacc[kMaxLoops][4];
         const float *qv = reinterpret_cast<const float *>(smem + Ly.qv);
         const float *qmu = reinterpret_cast<const float *>(smem + Ly.qmu);
         const float *muv = reinterpret_cast<const float *>(smem + Ly.muv);
+        float *mrg = reinterpret_cast<float *>(smem + Ly.mrg);
+        float *xch = reinterpret_cast<float *>(smem + Ly.xch);
 
-        // O^T of step sp (loop tp): fold each warp's column pair into its output sum
-        auto readout = [&](int sp, int tp) {
-            uint32_t o8[8];
-            const bool ok = wait_all(bar(BOFULL0 + (sp & 1)), (sp >> 1) & 1);
-            if (ok) {
-                tc::fence_after();
-                tc::ld_x8(trow + kColO + 16 * (sp & 1), o8);
-                tc::wait_ld();
-                tc::fence_before();
-            }
-            __syncwarp();
-            if (lane == 0)
-                mbar_arrive(bar(BOEMPTY0 + (sp & 1)));
-            if (!ok)
-                return;
-            const float *al = alpha + (sp & 3) * kSoftWarps;
-#pragma unroll
-            for (int t = 0; t < kMaxLoops; ++t)
-                if (t == tp) {
-#pragma unroll
-                    for (int w = 0; w < kSoftWarps; ++w)
-                        oacc[t][w] = fmaf(oacc[t][w], al[w],
-                                          __uint_as_float(o8[2 * w]) + __uint_as_float(o8[2 * w + 1]));
-                }
-        };
-        // segment end: merge the warps' states into one record per loop
+        // segment end: merge the 8 warps' states into one record per loop
         auto flush = [&](const TileDesc &dd) {
 #pragma unroll
             for (int t = 0; t < kMaxLoops; ++t) {
@@ -483,59 +459,73 @@ __global__ void __launch_bounds__(kThreads, 1)
                     }
                 }
             }
-            asm volatile("bar.sync 1, %0;" ::"r"(kSoftThreads) : "memory");
-            if (misc[0] == 0 && dd.j < a.seg_max) {
+            soft_sync();
+            float M[kMaxLoops], part[kMaxLoops];
+#pragma unroll
+            for (int t = 0; t < kMaxLoops; ++t) {
+                M[t] = -INFINITY;
+                part[t] = 0.f;
+                if (t < lp) {
+#pragma unroll
+                    for (int w = 0; w < 8; ++w)
+                        M[t] = fmaxf(M[t], mrg[(w * kMaxLoops + t) * 2]);
+#pragma unroll
+                    for (int w = 0; w < 4; ++w) { // this group's warps
+                        const float mw = mrg[((4 * g + w) * kMaxLoops + t) * 2];
+                        if (mw != -INFINITY)
+                            part[t] = fmaf(fast_exp2(mw - M[t]), oacc[t][w], part[t]);
+                    }
+                    if (g == 1)
+                        xch[t * kD + r] = part[t];
+                }
+            }
+            soft_sync();
+            if (g == 0 && misc[0] == 0 && dd.j < a.seg_max) {
 #pragma unroll
                 for (int t = 0; t < kMaxLoops; ++t) {
                     if (t < lp) {
-                        float M = -INFINITY;
+                        float L = 0.f;
 #pragma unroll
-                        for (int w = 0; w < kSoftWarps; ++w)
-                            M = fmaxf(M, mrg[(w * kMaxLoops + t) * 2]);
-                        float L = 0.f, acc = 0.f;
-#pragma unroll
-                        for (int w = 0; w < kSoftWarps; ++w) {
+                        for (int w = 0; w < 8; ++w) {
                             const float mw = mrg[(w * kMaxLoops + t) * 2];
-                            if (mw != -INFINITY) {
-                                const float e = fast_exp2(mw - M);
-                                L = fmaf(e, mrg[(w * kMaxLoops + t) * 2 + 1], L);
-                                acc = fmaf(e, oacc[t][w], acc);
-                            }
+                            if (mw != -INFINITY)
+                                L = fmaf(fast_exp2(mw - M[t]), mrg[(w * kMaxLoops + t) * 2 + 1], L);
                         }
-                        acc = fmaf(L, muv[t * kD + r], acc); // mu_t^V, left out of V_hat
+                        // + L mu_t^V: the mean left out of V_hat
+                        const float acc = fmaf(L, muv[t * kD + r], part[t] + xch[t * kD + r]);
                         float *rec = a.part + (((int64_t)dd.u * a.Tq_all + a.tq_off + t) * a.seg_max + dd.j) *
                                                   part_stride(kD);
                         rec[r] = acc;
                         if (r == 0) {
-                            rec[kD] = M;
+                            rec[kD] = M[t];
                             rec[kD + 1] = L;
                         }
                     }
                 }
                 if (r == 0 && dd.j == 0)
                     a.counts[dd.u] = dd.n_u;
-            } else if (r == 0 && dd.j >= a.seg_max) {
+            } else if (g == 0 && r == 0 && dd.j >= a.seg_max) {
                 report_status(a.status, LLA_ERR_INVALID); // a context longer than max_ctx
             }
-            asm volatile("bar.sync 1, %0;" ::"r"(kSoftThreads) : "memory"); // mrg free again
+            soft_sync(); // mrg and xch free again
         };
 
         HeadWalk<kTile> walk;
         walk.start(s0, s1, chunk, S_tot);
         TileDesc d, dseg;
-        int s = 0, tile = 0, pend = -1, pend_t = 0, prev_h = -1;
+        bool have_seg = false;
+        int s = 0, tile = 0, prev_h = -1;
         int32_t qpos = 0;
         while (walk.next(pref, a.seq_start, B, H, d)) {
             if (d.flags & 1) {
                 // ---- new unit segment: close the previous one, stage this one's inputs
-                if (pend >= 0) {
-                    readout(pend, pend_t);
-                    pend = -1;
+                if (have_seg)
                     flush(dseg);
-                }
                 dseg = d;
+                have_seg = true;
                 const bool wchange = d.h != prev_h;
                 const int style = a.rope_style;
+                const int st_ = tid; // 0 .. 255 over both groups
                 for (int t = 0; t < lp; ++t) {
                     const int tl = a.t0 + a.tq_off + t;
                     const int64_t gi = ((int64_t)d.h * a.T + tl);
@@ -545,7 +535,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                         const float *wv = a.W_up_v + gi * RV * kD;
                         uint8_t *dk = smem + Ly.wk + t * 2 * Ly.wk_part;
                         uint8_t *dv = smem + Ly.wv + t * 2 * Ly.wv_part;
-                        for (int e = r; e < RK * kD; e += kSoftThreads) {
+                        for (int e = st_; e < RK * kD; e += kSoftThreads) {
                             const int j = e / kD, k = e - j * kD;
                             const int row = ROPE ? pair_row(k, style) : k;
                             const float x = wk[e];
@@ -555,7 +545,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                             *reinterpret_cast<__nv_bfloat16 *>(dk + off) = hi;
                             *reinterpret_cast<__nv_bfloat16 *>(dk + Ly.wk_part + off) = lo;
                         }
-                        for (int e = r; e < RV * kD; e += kSoftThreads) {
+                        for (int e = st_; e < RV * kD; e += kSoftThreads) {
                             const int j = e / kD, k = e - j * kD;
                             const float x = wv[e];
                             const __nv_bfloat16 hi = __float2bfloat16_rn(x);
@@ -564,30 +554,33 @@ __global__ void __launch_bounds__(kThreads, 1)
                             *reinterpret_cast<__nv_bfloat16 *>(dv + off) = hi;
                             *reinterpret_cast<__nv_bfloat16 *>(dv + Ly.wv_part + off) = lo;
                         }
-                        const float mk = a.mu_k[gi * kD + r];
-                        const int row = ROPE ? pair_row(r, style) : r;
-                        reinterpret_cast<float *>(smem + Ly.muk)[t * kD + row] = mk;
-                        reinterpret_cast<float *>(smem + Ly.muv)[t * kD + r] = a.mu_v[gi * kD + r];
-                        if (ROPE) { // mu_t^K as the B tile of the ones MMA: columns 0, 1 = hi, lo
-                            const __nv_bfloat16 hi = __float2bfloat16_rn(mk);
-                            const __nv_bfloat16 lo = __float2bfloat16_rn(mk - __bfloat162float(hi));
-                            const __nv_bfloat162 hl = __halves2bfloat162(hi, lo);
-                            uint8_t *mt = smem + Ly.muk_t + t * kD * 32;
-                            *reinterpret_cast<uint4 *>(mt + L16::off(row, 0)) =
-                                make_uint4(*reinterpret_cast<const uint32_t *>(&hl), 0u, 0u, 0u);
-                            *reinterpret_cast<uint4 *>(mt + L16::off(row, 1)) = make_uint4(0u, 0u, 0u, 0u);
+                        if (g == 0) {
+                            const float mk = a.mu_k[gi * kD + r];
+                            const int row = ROPE ? pair_row(r, style) : r;
+                            reinterpret_cast<float *>(smem + Ly.muk)[t * kD + row] = mk;
+                            reinterpret_cast<float *>(smem + Ly.muv)[t * kD + r] = a.mu_v[gi * kD + r];
+                            if (ROPE) { // mu_t^K as the B tile of the ones MMA: columns 0, 1 = hi, lo
+                                const __nv_bfloat16 hi = __float2bfloat16_rn(mk);
+                                const __nv_bfloat16 lo = __float2bfloat16_rn(mk - __bfloat162float(hi));
+                                const __nv_bfloat162 hl = __halves2bfloat162(hi, lo);
+                                uint8_t *mt = smem + Ly.muk_t + t * kD * 32;
+                                *reinterpret_cast<uint4 *>(mt + L16::off(row, 0)) =
+                                    make_uint4(*reinterpret_cast<const uint32_t *>(&hl), 0u, 0u, 0u);
+                                *reinterpret_cast<uint4 *>(mt + L16::off(row, 1)) = make_uint4(0u, 0u, 0u, 0u);
+                            }
                         }
                     }
-                    // scaled query of this (sequence, head) and loop, in the kernel's row order
-                    const __nv_bfloat16 *qrow =
-                        static_cast<const __nv_bfloat16 *>(a.q) + (((int64_t)d.b * a.Tq_all + a.tq_off + t) * H + d.h) * kD;
-                    reinterpret_cast<float *>(smem + Ly.qv)[t * kD + (ROPE ? pair_row(r, style) : r)] =
-                        __bfloat162float(qrow[r]) * a.scale * kLog2e;
+                    if (g == 1) { // scaled query of this (sequence, head) and loop, kernel row order
+                        const __nv_bfloat16 *qrow = static_cast<const __nv_bfloat16 *>(a.q) +
+                                                    (((int64_t)d.b * a.Tq_all + a.tq_off + t) * H + d.h) * kD;
+                        reinterpret_cast<float *>(smem + Ly.qv)[t * kD + (ROPE ? pair_row(r, style) : r)] =
+                            __bfloat162float(qrow[r]) * a.scale * kLog2e;
+                    }
                 }
                 if (wchange)
                     fence_proxy_async_smem(); // W and mu tiles are read by the tensor cores
-                asm volatile("bar.sync 1, %0;" ::"r"(kSoftThreads) : "memory");
-                if (wchange && r == 0)
+                soft_sync();
+                if (wchange && tid == 0)
                     mbar_arrive(bar(BWREADY));
                 prev_h = d.h;
                 if (!ROPE && warp < lp) { // constant score term q . mu_t^K (log2 units)
@@ -603,19 +596,21 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
                 if (ROPE)
                     qpos = a.q_pos[d.b];
-                asm volatile("bar.sync 1, %0;" ::"r"(kSoftThreads) : "memory");
+                soft_sync();
 #pragma unroll
                 for (int t = 0; t < kMaxLoops; ++t) {
                     m[t] = -INFINITY;
                     l[t] = 0.f;
 #pragma unroll
-                    for (int w = 0; w < kSoftWarps; ++w)
+                    for (int w = 0; w < 4; ++w)
                         oacc[t][w] = 0.f;
                 }
             }
-            const int qb = tile & 1;
-            if (ROPE) {
-                // the tile's query: R((p - n0) w) q, pairs 2c and 2c + 1 of loop t
+            // does this group take any step of the tile?
+            const bool mine = lp > 1 || (s & 1) == g;
+            const int tb = tile & 1;
+            if (ROPE && mine) {
+                // the tile's query: R((p - n0) w) q, pairs 2c and 2c + 1 of loop t (this group's copy)
                 const int c = r & 31, t = r >> 5;
                 if (t < lp) {
                     const double *omg = reinterpret_cast<const double *>(smem + Ly.omg);
@@ -632,74 +627,83 @@ __global__ void __launch_bounds__(kThreads, 1)
                         qa2[e] = x * cs - y * sn;
                         qb2[e] = x * sn + y * cs;
                     }
-                    reinterpret_cast<float4 *>(smem + Ly.qt4)[(qb * lp + t) * 32 + c] =
-                        make_float4(qa2[0], qa2[1], qb2[0], qb2[1]);
-                    reinterpret_cast<float2 *>(smem + Ly.qtn)[(qb * lp + t) * 32 + c] = make_float2(-qa2[0], -qa2[1]);
+                    const int qi = ((g * 2 + tb) * lp + t) * 32 + c;
+                    reinterpret_cast<float4 *>(smem + Ly.qt4)[qi] = make_float4(qa2[0], qa2[1], qb2[0], qb2[1]);
+                    reinterpret_cast<float2 *>(smem + Ly.qtn)[qi] = make_float2(-qa2[0], -qa2[1]);
                 }
-                asm volatile("bar.sync 1, %0;" ::"r"(kSoftThreads) : "memory");
+                group_sync(g);
             }
 #pragma unroll
             for (int t = 0; t < kMaxLoops; ++t) {
                 if (t >= lp)
                     break;
-                // ---- step s: scores of loop t for this thread's token row
+                const int ss = s + t;
+                if ((ss & 1) != g)
+                    continue;
+                const int use = ss >> 1;
+                const int pb = use & 1; // this group's p / alpha buffer of the step
+                // ---- scores of loop t for this thread's token row
                 float sc = -INFINITY;
-                const bool ok = wait_all(bar(BKFULL), s & 1);
-                if (ok) {
+                if (wait_all(bar(BKFULL0 + g), use & 1)) {
                     tc::fence_after();
-                    float2 acc = make_float2(0.f, 0.f);
                     if (!ROPE) {
                         uint32_t kr[128];
-                        tc::ld_x32(trow + kColK, *reinterpret_cast<uint32_t(*)[32]>(kr));
-                        tc::ld_x32(trow + kColK + 32, *reinterpret_cast<uint32_t(*)[32]>(kr + 32));
-                        tc::ld_x32(trow + kColK + 64, *reinterpret_cast<uint32_t(*)[32]>(kr + 64));
-                        tc::ld_x32(trow + kColK + 96, *reinterpret_cast<uint32_t(*)[32]>(kr + 96));
+                        tc::ld_x32(tq + col_k(g), *reinterpret_cast<uint32_t(*)[32]>(kr));
+                        tc::ld_x32(tq + col_k(g) + 32, *reinterpret_cast<uint32_t(*)[32]>(kr + 32));
+                        tc::ld_x32(tq + col_k(g) + 64, *reinterpret_cast<uint32_t(*)[32]>(kr + 64));
+                        tc::ld_x32(tq + col_k(g) + 96, *reinterpret_cast<uint32_t(*)[32]>(kr + 96));
                         tc::wait_ld();
                         tc::fence_before();
                         __syncwarp();
                         if (lane == 0)
-                            mbar_arrive(bar(BKEMPTY));
+                            mbar_arrive(bar(BKEMPTY0 + g));
                         const float4 *q4 = reinterpret_cast<const float4 *>(qv + t * kD);
+                        float2 acc[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f),
+                                         make_float2(0.f, 0.f)};
 #pragma unroll
                         for (int c = 0; c < kD / 4; ++c) {
                             const float4 qq = q4[c];
-                            acc = __ffma2_rn(make_float2(qq.x, qq.y), f2(kr[4 * c], kr[4 * c + 1]), acc);
-                            acc = __ffma2_rn(make_float2(qq.z, qq.w), f2(kr[4 * c + 2], kr[4 * c + 3]), acc);
+                            acc[c & 3] = __ffma2_rn(make_float2(qq.x, qq.y), f2(kr[4 * c], kr[4 * c + 1]), acc[c & 3]);
+                            acc[c & 3] =
+                                __ffma2_rn(make_float2(qq.z, qq.w), f2(kr[4 * c + 2], kr[4 * c + 3]), acc[c & 3]);
                         }
-                        sc = acc.x + acc.y + qmu[t];
+                        sc = ((acc[0].x + acc[0].y) + (acc[1].x + acc[1].y)) +
+                             ((acc[2].x + acc[2].y) + (acc[3].x + acc[3].y)) + qmu[t];
                     } else {
-                        const float4 *q4 = reinterpret_cast<const float4 *>(smem + Ly.qt4) + (qb * lp + t) * 32;
-                        const float2 *qn = reinterpret_cast<const float2 *>(smem + Ly.qtn) + (qb * lp + t) * 32;
+                        const int qi = ((g * 2 + tb) * lp + t) * 32;
+                        const float4 *q4 = reinterpret_cast<const float4 *>(smem + Ly.qt4) + qi;
+                        const float2 *qn = reinterpret_cast<const float2 *>(smem + Ly.qtn) + qi;
+                        float2 acc[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
 #pragma unroll
                         for (int qt = 0; qt < 4; ++qt) { // pairs 16 qt .. 16 qt + 15
                             uint32_t ka[16], kb[16];
-                            tc::ld_x16(trow + kColK + 16 * qt, ka);
-                            tc::ld_x16(trow + kColK + kD / 2 + 16 * qt, kb);
+                            tc::ld_x16(tq + col_k(g) + 16 * qt, ka);
+                            tc::ld_x16(tq + col_k(g) + kD / 2 + 16 * qt, kb);
                             tc::wait_ld();
                             if (qt == 3) {
                                 tc::fence_before();
                                 __syncwarp();
                                 if (lane == 0)
-                                    mbar_arrive(bar(BKEMPTY));
+                                    mbar_arrive(bar(BKEMPTY0 + g));
                             }
 #pragma unroll
                             for (int cc = 0; cc < 8; ++cc) {
                                 const int c = 8 * qt + cc;
                                 const float4 qq = q4[c];
-                                const float2 qa = make_float2(qq.x, qq.y), qbv = make_float2(qq.z, qq.w);
+                                const float2 qa = make_float2(qq.x, qq.y), qb = make_float2(qq.z, qq.w);
                                 // x (qa cos + qb sin) + y (qb cos - qa sin), two pairs at once
-                                const float2 t1 = __ffma2_rn(qa, rc[c], __fmul2_rn(qbv, rs[c]));
-                                const float2 t2 = __ffma2_rn(qbv, rc[c], __fmul2_rn(qn[c], rs[c]));
-                                acc = __ffma2_rn(f2(ka[2 * cc], ka[2 * cc + 1]), t1, acc);
-                                acc = __ffma2_rn(f2(kb[2 * cc], kb[2 * cc + 1]), t2, acc);
+                                const float2 t1 = __ffma2_rn(qa, rc[c], __fmul2_rn(qb, rs[c]));
+                                const float2 t2 = __ffma2_rn(qb, rc[c], __fmul2_rn(qn[c], rs[c]));
+                                acc[cc & 1] = __ffma2_rn(f2(ka[2 * cc], ka[2 * cc + 1]), t1, acc[cc & 1]);
+                                acc[cc & 1] = __ffma2_rn(f2(kb[2 * cc], kb[2 * cc + 1]), t2, acc[cc & 1]);
                             }
                         }
-                        sc = acc.x + acc.y;
+                        sc = (acc[0].x + acc[0].y) + (acc[1].x + acc[1].y);
                     }
                 } else {
                     __syncwarp();
                     if (lane == 0)
-                        mbar_arrive(bar(BKEMPTY));
+                        mbar_arrive(bar(BKEMPTY0 + g));
                 }
                 if (r >= d.rows)
                     sc = -INFINITY;
@@ -716,51 +720,55 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
                 const float p = sc == -INFINITY ? 0.f : fast_exp2(sc - m[t]);
                 l[t] += p;
-                const float p_hi = __uint_as_float(__float_as_uint(p) & 0xffffe000u); // tf32-exact part
-                const float p_lo = p - p_hi;
-                // P rows 2w (hi) and 2w + 1 (lo), token column r, slab w (128B swizzle)
-                uint8_t *pb = smem + Ly.pbuf + (s & 1) * kPBuf + warp * kPSlab;
-                const int ch = lane >> 2;
-                const int n0 = 2 * warp, n1 = 2 * warp + 1;
-                *reinterpret_cast<float *>(pb + n0 * 128 + ((ch ^ (n0 & 7)) << 4) + (lane & 3) * 4) = p_hi;
-                *reinterpret_cast<float *>(pb + n1 * 128 + ((ch ^ (n1 & 7)) << 4) + (lane & 3) * 4) = p_lo;
+                float *pw = reinterpret_cast<float *>(smem + Ly.pv) + (g * 2 + pb) * kTile;
+                float *aw = reinterpret_cast<float *>(smem + Ly.alpha) + (g * 2 + pb) * 4;
+                pw[r] = p;
                 if (lane == 0)
-                    alpha[(s & 3) * kSoftWarps + warp] = al;
-                fence_proxy_async_smem();
-                __syncwarp();
-                if (lane == 0)
-                    mbar_arrive(bar(BPFULL0 + (s & 1)));
-                // ---- the previous step's output
-                if (pend >= 0)
-                    readout(pend, pend_t);
-                pend = s;
-                pend_t = t;
-                ++s;
+                    aw[wq] = al;
+                group_sync(g);
+                // ---- output: partial sums of each warp's 32 tokens at d-index r
+                float2 part[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f),
+                                  make_float2(0.f, 0.f)};
+                if (wait_all(bar(BVFULL0 + g), use & 1)) {
+                    tc::fence_after();
+                    uint32_t vr[128];
+                    tc::ld_x32(tq + col_v(g), *reinterpret_cast<uint32_t(*)[32]>(vr));
+                    tc::ld_x32(tq + col_v(g) + 32, *reinterpret_cast<uint32_t(*)[32]>(vr + 32));
+                    tc::ld_x32(tq + col_v(g) + 64, *reinterpret_cast<uint32_t(*)[32]>(vr + 64));
+                    tc::ld_x32(tq + col_v(g) + 96, *reinterpret_cast<uint32_t(*)[32]>(vr + 96));
+                    tc::wait_ld();
+                    tc::fence_before();
+                    __syncwarp();
+                    if (lane == 0)
+                        mbar_arrive(bar(BVEMPTY0 + g));
+                    const float4 *p4 = reinterpret_cast<const float4 *>(pw);
+#pragma unroll
+                    for (int c = 0; c < 8; ++c) {
+#pragma unroll
+                        for (int w = 0; w < 4; ++w) {
+                            const float4 pp = p4[8 * w + c];
+                            const int n = 32 * w + 4 * c;
+                            part[w] = __ffma2_rn(make_float2(pp.x, pp.y), f2(vr[n], vr[n + 1]), part[w]);
+                            part[w] = __ffma2_rn(make_float2(pp.z, pp.w), f2(vr[n + 2], vr[n + 3]), part[w]);
+                        }
+                    }
+                } else {
+                    __syncwarp();
+                    if (lane == 0)
+                        mbar_arrive(bar(BVEMPTY0 + g));
+                }
+#pragma unroll
+                for (int w = 0; w < 4; ++w)
+                    oacc[t][w] = fmaf(oacc[t][w], aw[w], part[w].x + part[w].y);
             }
+            s += lp;
             ++tile;
         }
-        if (pend >= 0) {
-            readout(pend, pend_t);
+        if (have_seg)
             flush(dseg);
-        }
-    }
-    // ---- teardown: every MMA complete before tensor memory is released
-    __syncwarp();
-    __syncthreads();
-    if (warp == kMmaWarp) {
-        if (lane == 0)
-            tc::commit(bar(BDRAIN));
-        __syncwarp();
-        (void)mbar_wait_bounded(bar(BDRAIN), 0);
-        __syncwarp();
-        tc::fence_after();
-        tc::dealloc(tmem, kTmemCols);
-    }
-    if (misc[0] != 0 && warp == kProducerWarp && lane == 0) {
-        report_status(a.status, LLA_ERR_DEVICE_TIMEOUT);
-        const int issued = misc[2];
-        for (int i = issued - (int)nst < 0 ? 0 : issued - (int)nst; i < issued; ++i)
-            (void)mbar_wait_bounded(full_bar(i % nst), (i / nst) & 1);
+      }
+      __syncwarp();
+      all_sync();
     }
 }
 
