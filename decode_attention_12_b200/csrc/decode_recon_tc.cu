@@ -57,9 +57,9 @@ constexpr int kSoftThreads = kGroups * kGroupThreads;
 constexpr int kProducerWarp = 8, kMmaWarp = 9; // warps 10, 11 complete the third warpgroup
 constexpr int kThreads = 12 * 32;
 // Register split (setmaxnreg): launched at 168 per thread (384 x 168 = 64,512 of the SM's
-// 65,536), the producer/MMA warpgroup gives back to 40 and the two softmax warpgroups take
-// 232: 2 x 128 x 232 + 128 x 40 = 64,512, exactly the launch's total.
-constexpr int kLaunchRegs = 168, kSoftRegs = 232, kIssueRegs = 40;
+// 65,536), the producer/MMA warpgroup gives back to 104 and the two softmax warpgroups take
+// 200: 2 x 128 x 200 + 128 x 104 = 64,512, exactly the launch's total.
+constexpr int kLaunchRegs = 168, kSoftRegs = 200, kIssueRegs = 104;
 static_assert(2 * 128 * kSoftRegs + 128 * kIssueRegs <= kThreads * kLaunchRegs, "register split exceeds the launch");
 constexpr float kRescale = 8.0f; // lazy rescale margin (log2 units)
 
@@ -72,7 +72,7 @@ __device__ __forceinline__ uint32_t col_v(int g) { return 256u + 128u * g; }
 enum { BKFULL0 = 0, BKFULL1, BKEMPTY0, BKEMPTY1, BVFULL0, BVFULL1, BVEMPTY0, BVEMPTY1, BWREADY, BDRAIN, BCOUNT };
 
 struct RLayout {
-    uint32_t nst, stage, wk, wv, wk_part, wv_part, ones, muk_t, qv, qt4, qtn, muk, muv, pv, alpha, xch, qmu, mrg,
+    uint32_t nst, stage, wk, wv, wk_part, wv_part, ones, muk_t, qv, qt4, muk, muv, pv, alpha, xch, qmu, mrg,
         omg, bar, misc, scr, pref, total;
 };
 
@@ -100,17 +100,15 @@ template <int RK, int RV, bool ROPE> __host__ __device__ inline RLayout rlayout(
     o += ROPE ? lp * kD * 32 : 0;
     L.qv = o;                       // [lp][d] scaled query (kernel row order)
     o += lp * kD * 4;
-    L.qt4 = o;                      // [group][2 tiles][lp][32] turned query, pairs 2c, 2c+1
-    o += ROPE ? kGroups * 2 * lp * 32 * 16 : 0;
-    L.qtn = o;                      // [group][2 tiles][lp][32] minus its first parts
-    o += ROPE ? kGroups * 2 * lp * 32 * 8 : 0;
+    L.qt4 = o;                      // [group][lp][4 row offsets][32] turned query, pairs 2c, 2c+1
+    o += ROPE ? kGroups * lp * 4 * 32 * 16 : 0;
     L.muk = o;                      // [lp][d]
     o += lp * kD * 4;
     L.muv = o;                      // [lp][d]
     o += lp * kD * 4;
     L.pv = o;                       // [group][2][128] softmax weights of a step
     o += kGroups * 2 * kTile * 4;
-    L.alpha = o;                    // [group][2][4 warps] rescale factors of a step
+    L.alpha = o;                    // [group][2][4 warps] max references of a step
     o += kGroups * 2 * 4 * 4;
     L.xch = o;                      // [lp][d] group 1's share of a record
     o += lp * kD * 4;
@@ -318,77 +316,80 @@ __global__ void __launch_bounds__(kThreads, 1)
             misc[2] = issued;
         }
       } else if (s0 < s1 && warp == kMmaWarp) {
-        // ================= MMA issuer: lane 0 issues, the warp waits and zeroes =================
-        constexpr uint32_t kIdKV = tc::idesc(tc::kFmtBf16, 128, 128);
-        bool err = false;
-        auto wait_all = [&](uint32_t b, uint32_t parity) -> bool {
-            bool ok = !err && misc[0] == 0 && mbar_wait_bounded(b, parity);
-            ok = __all_sync(0xffffffffu, ok);
-            if (!ok) {
-                err = true;
-                misc[0] = 1;
-            }
-            return ok;
-        };
-        HeadWalk<kTile> walk;
-        walk.start(s0, s1, chunk, S_tot);
-        TileDesc d;
-        int s = 0, ti = 0, wc = 0, prev_h = -1;
-        while (!err && walk.next(pref, a.seq_start, B, H, d)) {
-            const int st = ti % (int)nst;
-            if ((d.flags & 1) && d.h != prev_h) {
-                // a new head's W_up: staged once every MMA of the old one has been consumed
-                if (!wait_all(bar(BWREADY), wc & 1))
-                    break;
-                ++wc;
-                prev_h = d.h;
-            }
-            if (!wait_all(full_bar(st), (ti / nst) & 1))
-                break;
-            const uint32_t sk = sbase + st * Ly.stage, sv = sk + LK::BYTES;
-            if (d.rows < kTile) { // rows past the segment: zeros, never stale or NaN data
-                LK::zero_rows(smem + st * Ly.stage, d.rows, kTile, lane);
-                LV::zero_rows(smem + st * Ly.stage + LK::BYTES, d.rows, kTile, lane);
-                fence_proxy_async_smem();
-                __syncwarp();
-            }
-            for (int t = 0; t < lp && !err; ++t, ++s) {
-                const int g = s & 1, use = s >> 1; // group g's use number of its buffers
-                if (use >= 1 && !wait_all(bar(BKEMPTY0 + g), (use - 1) & 1))
-                    break;
-                tc::fence_after();
-                if (lane == 0) {
-                    const uint32_t wk = sbase + Ly.wk + t * 2 * Ly.wk_part;
-#pragma unroll
-                    for (int kk = 0; kk < RK / 16; ++kk)
-#pragma unroll
-                        for (int hl = 0; hl < 2; ++hl)
-                            tc::mma_bf16(tmem + col_k(g), tc::smem_desc(sk + 32 * kk, 2 * RK),
-                                         tc::smem_desc(wk + hl * Ly.wk_part + 32 * kk, 2 * RK), kIdKV, (kk | hl) != 0);
-                    if (ROPE)
-                        tc::mma_bf16(tmem + col_k(g), tc::smem_desc(sbase + Ly.ones, 32),
-                                     tc::smem_desc(sbase + Ly.muk_t + t * kD * 32, 32), kIdKV, 1);
-                    tc::commit(bar(BKFULL0 + g));
+        // ================= MMA issuer: the whole warp runs the loop, one elected lane issues =================
+        // Shared-memory descriptors are formed once; moving a descriptor's start address by
+        // `bytes` adds bytes / 16 to its low field (every operand lies below 256 KB).
+        {
+            constexpr uint32_t kIdKV = tc::idesc(tc::kFmtBf16, 128, 128);
+            const uint64_t dK0 = tc::smem_desc(sbase, 2 * RK);                // latent K tile of stage 0
+            const uint64_t dV0 = tc::smem_desc(sbase + LK::BYTES, 2 * RV);    // latent V tile of stage 0
+            const uint64_t dWk = tc::smem_desc(sbase + Ly.wk, 2 * RK);        // W_up^K^T parts
+            const uint64_t dWv = tc::smem_desc(sbase + Ly.wv, 2 * RV);        // W_up^V^T parts
+            const uint64_t dOnes = tc::smem_desc(sbase + Ly.ones, 32);
+            const uint64_t dMu = tc::smem_desc(sbase + Ly.muk_t, 32);
+            const uint32_t stage_units = Ly.stage >> 4, wk_units = Ly.wk_part >> 4, wv_units = Ly.wv_part >> 4;
+            bool err = false;
+            auto wait_all = [&](uint32_t b, uint32_t parity) -> bool {
+                bool ok = !err && misc[0] == 0 && mbar_wait_bounded(b, parity);
+                ok = __all_sync(0xffffffffu, ok);
+                if (!ok) {
+                    err = true;
+                    misc[0] = 1;
                 }
-                __syncwarp();
-                if (use >= 1 && !wait_all(bar(BVEMPTY0 + g), (use - 1) & 1))
-                    break;
-                tc::fence_after();
-                if (lane == 0) {
-                    const uint32_t wv = sbase + Ly.wv + t * 2 * Ly.wv_part;
-#pragma unroll
-                    for (int kk = 0; kk < RV / 16; ++kk)
-#pragma unroll
-                        for (int hl = 0; hl < 2; ++hl)
-                            tc::mma_bf16(tmem + col_v(g), tc::smem_desc(wv + hl * Ly.wv_part + 32 * kk, 2 * RV),
-                                         tc::smem_desc(sv + 32 * kk, 2 * RV), kIdKV, (kk | hl) != 0);
-                    tc::commit(bar(BVFULL0 + g));
-                    if (t == lp - 1)
-                        tc::commit(empty_bar(st)); // the tile's stage is free once these complete
+                return ok;
+            };
+            HeadWalk<kTile> walk;
+            walk.start(s0, s1, chunk, S_tot);
+            TileDesc d;
+            int s = 0, ti = 0, wc = 0, prev_h = -1;
+            while (!err && walk.next(pref, a.seq_start, B, H, d)) {
+                const int st = ti % (int)nst;
+                if ((d.flags & 1) && d.h != prev_h) {
+                    // a new head's W_up: staged once every MMA of the old one has been consumed
+                    if (!wait_all(bar(BWREADY), wc & 1))
+                        break;
+                    ++wc;
+                    prev_h = d.h;
                 }
-                __syncwarp();
+                if (!wait_all(full_bar(st), (ti / nst) & 1))
+                    break;
+                if (d.rows < kTile) { // rows past the segment: zeros, never stale or NaN data
+                    LK::zero_rows(smem + st * Ly.stage, d.rows, kTile, lane);
+                    LV::zero_rows(smem + st * Ly.stage + LK::BYTES, d.rows, kTile, lane);
+                    fence_proxy_async_smem();
+                    __syncwarp();
+                }
+                const uint64_t dK = dK0 + st * stage_units, dV = dV0 + st * stage_units;
+                for (int t = 0; t < lp && !err; ++t, ++s) {
+                    const int g = s & 1, use = s >> 1; // group g's use number of its buffers
+                    // the group has read both buffers of its previous step (V after K)
+                    if (use >= 1 && !wait_all(bar(BVEMPTY0 + g), (use - 1) & 1))
+                        break;
+                    tc::fence_after();
+                    const uint64_t wk = dWk + 2 * t * wk_units, wv = dWv + 2 * t * wv_units;
+                    const uint32_t dk_t = tmem + col_k(g), dv_t = tmem + col_v(g);
+                    if (tc::elect_one()) {
+#pragma unroll
+                        for (int kk = 0; kk < RK / 16; ++kk)
+#pragma unroll
+                            for (int hl = 0; hl < 2; ++hl)
+                                tc::mma_bf16(dk_t, dK + 2 * kk, wk + hl * wk_units + 2 * kk, kIdKV, (kk | hl) != 0);
+                        if (ROPE)
+                            tc::mma_bf16(dk_t, dOnes, dMu + t * (kD * 32 / 16), kIdKV, 1);
+                        tc::commit(bar(BKFULL0 + g));
+#pragma unroll
+                        for (int kk = 0; kk < RV / 16; ++kk)
+#pragma unroll
+                            for (int hl = 0; hl < 2; ++hl)
+                                tc::mma_bf16(dv_t, wv + hl * wv_units + 2 * kk, dV + 2 * kk, kIdKV, (kk | hl) != 0);
+                        tc::commit(bar(BVFULL0 + g));
+                        if (t == lp - 1)
+                            tc::commit(empty_bar(st)); // the tile's stage is free once these complete
+                    }
+                    __syncwarp();
+                }
+                ++ti;
             }
-            ++ti;
         }
       }
       __syncwarp();
@@ -409,11 +410,18 @@ __global__ void __launch_bounds__(kThreads, 1)
               (void)mbar_wait_bounded(full_bar(i % nst), (i / nst) & 1);
       }
     } else {
-      // ======== two groups of 4 warps, alternate steps: thread r = token row r / d-index r ========
+      // ======== two groups of 4 warps, alternate steps ========
+      // Tensor memory is read in 16-lane x 256-bit fragments: lane t of a warp holds rows
+      // rq, rq + 8, rq + 16, rq + 24 (rq = t / 4) of the warp's 32-lane quarter and columns
+      // 8 i + 2 j + {0, 1} (j = t % 4, i = 0..15), so a query or weight pair it loads from
+      // shared memory serves four rows, and a row's sum closes over the 4 lanes of a quad.
       asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kSoftRegs));
       if (s0 < s1) {
         const int g = warp >> 2, wq = warp & 3, r = tid & 127;
+        const int j = lane & 3, rq = lane >> 2;
         const uint32_t tq = tmem + ((uint32_t)(32 * wq) << 16); // this warp's lane quarter
+        // tile row / d-index of the thread's k-th row (k = 2 h + e: half h, +8 e)
+        auto row_of = [&](int k) { return 32 * wq + 16 * (k >> 1) + 8 * (k & 1) + rq; };
         bool err = false;
         auto wait_all = [&](uint32_t b, uint32_t parity) -> bool {
             bool ok = !err && misc[0] == 0 && mbar_wait_bounded(b, parity);
@@ -424,19 +432,27 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             return ok;
         };
-        // rotation of this thread's row r: (cos, sin)(r w_i) for pairs 2c and 2c + 1
-        float2 rc[ROPE ? 32 : 1], rs[ROPE ? 32 : 1];
+        auto quad_sum = [&](float x) {
+            x += __shfl_xor_sync(0xffffffffu, x, 1);
+            return x + __shfl_xor_sync(0xffffffffu, x, 2);
+        };
+        // rotation of the thread's base row b0 = 32 wq + rq: (cos, sin)(b0 w_P) for the pairs
+        // P = 8 i + 2 j + {0, 1}, i = 0..7 (rows b0 + 8 k turn the query instead)
+        float2 rc[ROPE ? 8 : 1], rs[ROPE ? 8 : 1];
         if (ROPE) {
             const float lb = log2f(a.rope_base);
+            const float b0 = (float)(32 * wq + rq);
 #pragma unroll
-            for (int c = 0; c < 32; ++c) {
+            for (int i = 0; i < 8; ++i) {
                 float sa, ca, sb, cb;
-                sincosf((float)r * exp2f(-2.0f * (float)(2 * c) / (float)kD * lb), &sa, &ca);
-                sincosf((float)r * exp2f(-2.0f * (float)(2 * c + 1) / (float)kD * lb), &sb, &cb);
-                rc[c] = make_float2(ca, cb);
-                rs[c] = make_float2(sa, sb);
+                sincosf(b0 * exp2f(-2.0f * (float)(8 * i + 2 * j) / (float)kD * lb), &sa, &ca);
+                sincosf(b0 * exp2f(-2.0f * (float)(8 * i + 2 * j + 1) / (float)kD * lb), &sb, &cb);
+                rc[i] = make_float2(ca, cb);
+                rs[i] = make_float2(sa, sb);
             }
         }
+        // per loop: the group's running max (uniform), this thread's share of the sum of
+        // weights (the rows it writes), output sums of its 4 d-rows
         float m[kMaxLoops], l[kMaxLoops], oacc[kMaxLoops][4];
         const float *qv = reinterpret_cast<const float *>(smem + Ly.qv);
         const float *qmu = reinterpret_cast<const float *>(smem + Ly.qmu);
@@ -444,7 +460,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         float *mrg = reinterpret_cast<float *>(smem + Ly.mrg);
         float *xch = reinterpret_cast<float *>(smem + Ly.xch);
 
-        // segment end: merge the 8 warps' states into one record per loop
+        // segment end: merge the two groups' states into one record per loop
         auto flush = [&](const TileDesc &dd) {
 #pragma unroll
             for (int t = 0; t < kMaxLoops; ++t) {
@@ -460,23 +476,18 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
             }
             soft_sync();
-            float M[kMaxLoops], part[kMaxLoops];
+            float M[kMaxLoops], wg[kMaxLoops];
 #pragma unroll
             for (int t = 0; t < kMaxLoops; ++t) {
                 M[t] = -INFINITY;
-                part[t] = 0.f;
+                wg[t] = 0.f;
                 if (t < lp) {
-#pragma unroll
-                    for (int w = 0; w < 8; ++w)
-                        M[t] = fmaxf(M[t], mrg[(w * kMaxLoops + t) * 2]);
-#pragma unroll
-                    for (int w = 0; w < 4; ++w) { // this group's warps
-                        const float mw = mrg[((4 * g + w) * kMaxLoops + t) * 2];
-                        if (mw != -INFINITY)
-                            part[t] = fmaf(fast_exp2(mw - M[t]), oacc[t][w], part[t]);
-                    }
+                    const float m0 = mrg[(0 * kMaxLoops + t) * 2], m1 = mrg[(4 * kMaxLoops + t) * 2];
+                    M[t] = fmaxf(m0, m1);
+                    const float mine = g == 0 ? m0 : m1;
+                    wg[t] = mine == -INFINITY ? 0.f : fast_exp2(mine - M[t]);
                     if (g == 1)
-                        xch[t * kD + r] = part[t];
+                        xch[t * kD + row_of(j)] = wg[t] * oacc[t][j];
                 }
             }
             soft_sync();
@@ -491,11 +502,12 @@ __global__ void __launch_bounds__(kThreads, 1)
                             if (mw != -INFINITY)
                                 L = fmaf(fast_exp2(mw - M[t]), mrg[(w * kMaxLoops + t) * 2 + 1], L);
                         }
+                        const int d = row_of(j);
                         // + L mu_t^V: the mean left out of V_hat
-                        const float acc = fmaf(L, muv[t * kD + r], part[t] + xch[t * kD + r]);
+                        const float acc = fmaf(L, muv[t * kD + d], fmaf(wg[t], oacc[t][j], xch[t * kD + d]));
                         float *rec = a.part + (((int64_t)dd.u * a.Tq_all + a.tq_off + t) * a.seg_max + dd.j) *
                                                   part_stride(kD);
-                        rec[r] = acc;
+                        rec[d] = acc;
                         if (r == 0) {
                             rec[kD] = M[t];
                             rec[kD + 1] = L;
@@ -514,7 +526,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         walk.start(s0, s1, chunk, S_tot);
         TileDesc d, dseg;
         bool have_seg = false;
-        int s = 0, tile = 0, prev_h = -1;
+        int s = 0, prev_h = -1;
         int32_t qpos = 0;
         while (walk.next(pref, a.seq_start, B, H, d)) {
             if (d.flags & 1) {
@@ -525,7 +537,6 @@ __global__ void __launch_bounds__(kThreads, 1)
                 have_seg = true;
                 const bool wchange = d.h != prev_h;
                 const int style = a.rope_style;
-                const int st_ = tid; // 0 .. 255 over both groups
                 for (int t = 0; t < lp; ++t) {
                     const int tl = a.t0 + a.tq_off + t;
                     const int64_t gi = ((int64_t)d.h * a.T + tl);
@@ -535,22 +546,22 @@ __global__ void __launch_bounds__(kThreads, 1)
                         const float *wv = a.W_up_v + gi * RV * kD;
                         uint8_t *dk = smem + Ly.wk + t * 2 * Ly.wk_part;
                         uint8_t *dv = smem + Ly.wv + t * 2 * Ly.wv_part;
-                        for (int e = st_; e < RK * kD; e += kSoftThreads) {
-                            const int j = e / kD, k = e - j * kD;
+                        for (int e = tid; e < RK * kD; e += kSoftThreads) {
+                            const int jj = e / kD, k = e - jj * kD;
                             const int row = ROPE ? pair_row(k, style) : k;
                             const float x = wk[e];
                             const __nv_bfloat16 hi = __float2bfloat16_rn(x);
                             const __nv_bfloat16 lo = __float2bfloat16_rn(x - __bfloat162float(hi));
-                            const uint32_t off = LK::off(row, j >> 3) + (j & 7) * 2;
+                            const uint32_t off = LK::off(row, jj >> 3) + (jj & 7) * 2;
                             *reinterpret_cast<__nv_bfloat16 *>(dk + off) = hi;
                             *reinterpret_cast<__nv_bfloat16 *>(dk + Ly.wk_part + off) = lo;
                         }
-                        for (int e = st_; e < RV * kD; e += kSoftThreads) {
-                            const int j = e / kD, k = e - j * kD;
+                        for (int e = tid; e < RV * kD; e += kSoftThreads) {
+                            const int jj = e / kD, k = e - jj * kD;
                             const float x = wv[e];
                             const __nv_bfloat16 hi = __float2bfloat16_rn(x);
                             const __nv_bfloat16 lo = __float2bfloat16_rn(x - __bfloat162float(hi));
-                            const uint32_t off = LV::off(k, j >> 3) + (j & 7) * 2;
+                            const uint32_t off = LV::off(k, jj >> 3) + (jj & 7) * 2;
                             *reinterpret_cast<__nv_bfloat16 *>(dv + off) = hi;
                             *reinterpret_cast<__nv_bfloat16 *>(dv + Ly.wv_part + off) = lo;
                         }
@@ -602,34 +613,33 @@ __global__ void __launch_bounds__(kThreads, 1)
                     m[t] = -INFINITY;
                     l[t] = 0.f;
 #pragma unroll
-                    for (int w = 0; w < 4; ++w)
-                        oacc[t][w] = 0.f;
+                    for (int k = 0; k < 4; ++k)
+                        oacc[t][k] = 0.f;
                 }
             }
             // does this group take any step of the tile?
             const bool mine = lp > 1 || (s & 1) == g;
-            const int tb = tile & 1;
             if (ROPE && mine) {
-                // the tile's query: R((p - n0) w) q, pairs 2c and 2c + 1 of loop t (this group's copy)
-                const int c = r & 31, t = r >> 5;
-                if (t < lp) {
-                    const double *omg = reinterpret_cast<const double *>(smem + Ly.omg);
-                    const int64_t rel = (int64_t)qpos - d.n0;
+                // the tile's query, once per row offset 8 v (v = 0..3) of the thread rows:
+                // R((p - n0 - 8 v) w) q for pairs 2c, 2c + 1; entry [loop][v][couple c]
+                const double *omg = reinterpret_cast<const double *>(smem + Ly.omg);
+                float4 *qt = reinterpret_cast<float4 *>(smem + Ly.qt4) + g * lp * 4 * 32;
+                for (int e = r; e < lp * 4 * 32; e += kGroupThreads) {
+                    const int c = e & 31, v = (e >> 5) & 3, t = e >> 7;
+                    const int64_t rel = (int64_t)qpos - d.n0 - 8 * v;
                     float qa2[2], qb2[2];
 #pragma unroll
-                    for (int e = 0; e < 2; ++e) {
-                        const int i = 2 * c + e;
+                    for (int ee = 0; ee < 2; ++ee) {
+                        const int i = 2 * c + ee;
                         const double ang = (double)rel * omg[i];
                         const float red = (float)(ang - 6.283185307179586 * rint(ang * 0.15915494309189535));
                         float sn, cs;
                         sincosf(red, &sn, &cs);
                         const float x = qv[t * kD + i], y = qv[t * kD + i + kD / 2];
-                        qa2[e] = x * cs - y * sn;
-                        qb2[e] = x * sn + y * cs;
+                        qa2[ee] = x * cs - y * sn;
+                        qb2[ee] = x * sn + y * cs;
                     }
-                    const int qi = ((g * 2 + tb) * lp + t) * 32 + c;
-                    reinterpret_cast<float4 *>(smem + Ly.qt4)[qi] = make_float4(qa2[0], qa2[1], qb2[0], qb2[1]);
-                    reinterpret_cast<float2 *>(smem + Ly.qtn)[qi] = make_float2(-qa2[0], -qa2[1]);
+                    qt[e] = make_float4(qa2[0], qa2[1], qb2[0], qb2[1]);
                 }
                 group_sync(g);
             }
@@ -641,115 +651,148 @@ __global__ void __launch_bounds__(kThreads, 1)
                 if ((ss & 1) != g)
                     continue;
                 const int use = ss >> 1;
-                const int pb = use & 1; // this group's p / alpha buffer of the step
-                // ---- scores of loop t for this thread's token row
-                float sc = -INFINITY;
+                const int pb = use & 1; // this group's weight / reference buffer of the step
+                // ---- scores of loop t for the thread's 4 token rows
+                float sc[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
                 if (wait_all(bar(BKFULL0 + g), use & 1)) {
                     tc::fence_after();
+                    float2 acc[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f),
+                                     make_float2(0.f, 0.f)};
                     if (!ROPE) {
-                        uint32_t kr[128];
-                        tc::ld_x32(tq + col_k(g), *reinterpret_cast<uint32_t(*)[32]>(kr));
-                        tc::ld_x32(tq + col_k(g) + 32, *reinterpret_cast<uint32_t(*)[32]>(kr + 32));
-                        tc::ld_x32(tq + col_k(g) + 64, *reinterpret_cast<uint32_t(*)[32]>(kr + 64));
-                        tc::ld_x32(tq + col_k(g) + 96, *reinterpret_cast<uint32_t(*)[32]>(kr + 96));
-                        tc::wait_ld();
-                        tc::fence_before();
-                        __syncwarp();
-                        if (lane == 0)
-                            mbar_arrive(bar(BKEMPTY0 + g));
-                        const float4 *q4 = reinterpret_cast<const float4 *>(qv + t * kD);
-                        float2 acc[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f),
-                                         make_float2(0.f, 0.f)};
+                        float2 qp[16]; // q pairs at columns 8 i + 2 j
+                        const float2 *q2 = reinterpret_cast<const float2 *>(qv + t * kD + 2 * j);
 #pragma unroll
-                        for (int c = 0; c < kD / 4; ++c) {
-                            const float4 qq = q4[c];
-                            acc[c & 3] = __ffma2_rn(make_float2(qq.x, qq.y), f2(kr[4 * c], kr[4 * c + 1]), acc[c & 3]);
-                            acc[c & 3] =
-                                __ffma2_rn(make_float2(qq.z, qq.w), f2(kr[4 * c + 2], kr[4 * c + 3]), acc[c & 3]);
-                        }
-                        sc = ((acc[0].x + acc[0].y) + (acc[1].x + acc[1].y)) +
-                             ((acc[2].x + acc[2].y) + (acc[3].x + acc[3].y)) + qmu[t];
-                    } else {
-                        const int qi = ((g * 2 + tb) * lp + t) * 32;
-                        const float4 *q4 = reinterpret_cast<const float4 *>(smem + Ly.qt4) + qi;
-                        const float2 *qn = reinterpret_cast<const float2 *>(smem + Ly.qtn) + qi;
-                        float2 acc[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
+                        for (int i = 0; i < 16; ++i)
+                            qp[i] = q2[4 * i];
 #pragma unroll
-                        for (int qt = 0; qt < 4; ++qt) { // pairs 16 qt .. 16 qt + 15
-                            uint32_t ka[16], kb[16];
-                            tc::ld_x16(tq + col_k(g) + 16 * qt, ka);
-                            tc::ld_x16(tq + col_k(g) + kD / 2 + 16 * qt, kb);
+                        for (int h = 0; h < 2; ++h) {
+                            uint32_t kr[64];
+                            tc::ld_16x256b_x16(tq + ((uint32_t)(16 * h) << 16) + col_k(g), kr);
                             tc::wait_ld();
-                            if (qt == 3) {
+                            if (h == 1) {
                                 tc::fence_before();
                                 __syncwarp();
                                 if (lane == 0)
                                     mbar_arrive(bar(BKEMPTY0 + g));
                             }
 #pragma unroll
-                            for (int cc = 0; cc < 8; ++cc) {
-                                const int c = 8 * qt + cc;
-                                const float4 qq = q4[c];
-                                const float2 qa = make_float2(qq.x, qq.y), qb = make_float2(qq.z, qq.w);
-                                // x (qa cos + qb sin) + y (qb cos - qa sin), two pairs at once
-                                const float2 t1 = __ffma2_rn(qa, rc[c], __fmul2_rn(qb, rs[c]));
-                                const float2 t2 = __ffma2_rn(qb, rc[c], __fmul2_rn(qn[c], rs[c]));
-                                acc[cc & 1] = __ffma2_rn(f2(ka[2 * cc], ka[2 * cc + 1]), t1, acc[cc & 1]);
-                                acc[cc & 1] = __ffma2_rn(f2(kb[2 * cc], kb[2 * cc + 1]), t2, acc[cc & 1]);
+                            for (int i = 0; i < 16; ++i) {
+                                acc[2 * h] = __ffma2_rn(qp[i], f2(kr[4 * i], kr[4 * i + 1]), acc[2 * h]);
+                                acc[2 * h + 1] = __ffma2_rn(qp[i], f2(kr[4 * i + 2], kr[4 * i + 3]), acc[2 * h + 1]);
                             }
                         }
-                        sc = (acc[0].x + acc[0].y) + (acc[1].x + acc[1].y);
+#pragma unroll
+                        for (int k = 0; k < 4; ++k)
+                            sc[k] = quad_sum(acc[k].x + acc[k].y) + qmu[t];
+                    } else {
+                        // row k = 2 h + e uses the query turned by its row offset 8 k
+                        const float4 *qt = reinterpret_cast<const float4 *>(smem + Ly.qt4) + (g * lp + t) * 4 * 32;
+#pragma unroll
+                        for (int h = 0; h < 2; ++h) {
+                            uint32_t kr[64];
+                            tc::ld_16x256b_x16(tq + ((uint32_t)(16 * h) << 16) + col_k(g), kr);
+                            tc::wait_ld();
+                            if (h == 1) {
+                                tc::fence_before();
+                                __syncwarp();
+                                if (lane == 0)
+                                    mbar_arrive(bar(BKEMPTY0 + g));
+                            }
+#pragma unroll
+                            for (int e = 0; e < 2; ++e) {
+                                const int k = 2 * h + e;
+#pragma unroll
+                                for (int i = 0; i < 8; ++i) { // pairs 8 i + 2 j + {0, 1}: columns i, i + 8
+                                    const float4 qq = qt[k * 32 + 4 * i + j];
+                                    const float2 qa = make_float2(qq.x, qq.y), qb = make_float2(qq.z, qq.w);
+                                    const float2 qas = __fmul2_rn(qa, rs[i]);
+                                    // x (qa cos + qb sin) + y (qb cos - qa sin)
+                                    const float2 t1 = __ffma2_rn(qa, rc[i], __fmul2_rn(qb, rs[i]));
+                                    const float2 t2 = __ffma2_rn(qb, rc[i], make_float2(-qas.x, -qas.y));
+                                    acc[k] = __ffma2_rn(f2(kr[4 * i + 2 * e], kr[4 * i + 2 * e + 1]), t1, acc[k]);
+                                    acc[k] = __ffma2_rn(f2(kr[4 * (i + 8) + 2 * e], kr[4 * (i + 8) + 2 * e + 1]), t2,
+                                                        acc[k]);
+                                }
+                            }
+                        }
+#pragma unroll
+                        for (int k = 0; k < 4; ++k)
+                            sc[k] = quad_sum(acc[k].x + acc[k].y);
                     }
                 } else {
                     __syncwarp();
                     if (lane == 0)
                         mbar_arrive(bar(BKEMPTY0 + g));
                 }
-                if (r >= d.rows)
-                    sc = -INFINITY;
-                // ---- online softmax, warp-local max (lazy rescale)
-                float mx = sc;
 #pragma unroll
-                for (int off = 16; off > 0; off >>= 1)
+                for (int k = 0; k < 4; ++k)
+                    if (row_of(k) >= d.rows)
+                        sc[k] = -INFINITY;
+                // ---- online softmax: each warp picks a reference (the group's running max, or
+                // its own max when that is more than the margin higher), the group reconciles
+                float mx = fmaxf(fmaxf(sc[0], sc[1]), fmaxf(sc[2], sc[3]));
+#pragma unroll
+                for (int off = 4; off < 32; off <<= 1)
                     mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
-                float al = 1.f;
-                if (mx > m[t] + kRescale) {
-                    al = fast_exp2(m[t] - mx);
-                    m[t] = mx;
-                    l[t] *= al;
-                }
-                const float p = sc == -INFINITY ? 0.f : fast_exp2(sc - m[t]);
-                l[t] += p;
+                const float ref = mx > m[t] + kRescale ? mx : m[t];
+                float p[4];
+#pragma unroll
+                for (int k = 0; k < 4; ++k)
+                    p[k] = sc[k] == -INFINITY ? 0.f : fast_exp2(sc[k] - ref);
+                const float pmine = j == 0 ? p[0] : j == 1 ? p[1] : j == 2 ? p[2] : p[3];
                 float *pw = reinterpret_cast<float *>(smem + Ly.pv) + (g * 2 + pb) * kTile;
-                float *aw = reinterpret_cast<float *>(smem + Ly.alpha) + (g * 2 + pb) * 4;
-                pw[r] = p;
+                float *rw = reinterpret_cast<float *>(smem + Ly.alpha) + (g * 2 + pb) * 4;
+                pw[row_of(j)] = pmine;
                 if (lane == 0)
-                    aw[wq] = al;
+                    rw[wq] = ref;
                 group_sync(g);
-                // ---- output: partial sums of each warp's 32 tokens at d-index r
-                float2 part[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f),
+                const float4 rf = *reinterpret_cast<const float4 *>(rw);
+                const float Mn = fmaxf(fmaxf(rf.x, rf.y), fmaxf(rf.z, rf.w));
+                float f[4] = {1.f, 1.f, 1.f, 1.f};
+                if (Mn != -INFINITY && !(rf.x == Mn && rf.y == Mn && rf.z == Mn && rf.w == Mn)) {
+                    f[0] = fast_exp2(rf.x - Mn);
+                    f[1] = fast_exp2(rf.y - Mn);
+                    f[2] = fast_exp2(rf.z - Mn);
+                    f[3] = fast_exp2(rf.w - Mn);
+                }
+                if (Mn > m[t]) { // the group's max rose: rescale what was summed so far
+                    const float al = fast_exp2(m[t] - Mn);
+                    l[t] *= al;
+#pragma unroll
+                    for (int k = 0; k < 4; ++k)
+                        oacc[t][k] *= al;
+                    m[t] = Mn;
+                }
+                const float fmine = wq == 0 ? f[0] : wq == 1 ? f[1] : wq == 2 ? f[2] : f[3];
+                l[t] = fmaf(fmine, pmine, l[t]);
+                // ---- output: sum over the tile's tokens of p v_hat at the thread's 4 d-rows
+                float2 pacc[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f),
                                   make_float2(0.f, 0.f)};
                 if (wait_all(bar(BVFULL0 + g), use & 1)) {
                     tc::fence_after();
-                    uint32_t vr[128];
-                    tc::ld_x32(tq + col_v(g), *reinterpret_cast<uint32_t(*)[32]>(vr));
-                    tc::ld_x32(tq + col_v(g) + 32, *reinterpret_cast<uint32_t(*)[32]>(vr + 32));
-                    tc::ld_x32(tq + col_v(g) + 64, *reinterpret_cast<uint32_t(*)[32]>(vr + 64));
-                    tc::ld_x32(tq + col_v(g) + 96, *reinterpret_cast<uint32_t(*)[32]>(vr + 96));
-                    tc::wait_ld();
-                    tc::fence_before();
-                    __syncwarp();
-                    if (lane == 0)
-                        mbar_arrive(bar(BVEMPTY0 + g));
-                    const float4 *p4 = reinterpret_cast<const float4 *>(pw);
+                    float2 pp[16]; // weight pairs of tokens 8 i + 2 j, on the common reference
+                    const float2 *p2 = reinterpret_cast<const float2 *>(pw + 2 * j);
 #pragma unroll
-                    for (int c = 0; c < 8; ++c) {
+                    for (int i = 0; i < 16; ++i) {
+                        const float fi = f[i >> 2];
+                        const float2 x = p2[4 * i];
+                        pp[i] = make_float2(x.x * fi, x.y * fi);
+                    }
 #pragma unroll
-                        for (int w = 0; w < 4; ++w) {
-                            const float4 pp = p4[8 * w + c];
-                            const int n = 32 * w + 4 * c;
-                            part[w] = __ffma2_rn(make_float2(pp.x, pp.y), f2(vr[n], vr[n + 1]), part[w]);
-                            part[w] = __ffma2_rn(make_float2(pp.z, pp.w), f2(vr[n + 2], vr[n + 3]), part[w]);
+                    for (int h = 0; h < 2; ++h) {
+                        uint32_t vr[64];
+                        tc::ld_16x256b_x16(tq + ((uint32_t)(16 * h) << 16) + col_v(g), vr);
+                        tc::wait_ld();
+                        if (h == 1) {
+                            tc::fence_before();
+                            __syncwarp();
+                            if (lane == 0)
+                                mbar_arrive(bar(BVEMPTY0 + g));
+                        }
+#pragma unroll
+                        for (int i = 0; i < 16; ++i) {
+                            pacc[2 * h] = __ffma2_rn(pp[i], f2(vr[4 * i], vr[4 * i + 1]), pacc[2 * h]);
+                            pacc[2 * h + 1] = __ffma2_rn(pp[i], f2(vr[4 * i + 2], vr[4 * i + 3]), pacc[2 * h + 1]);
                         }
                     }
                 } else {
@@ -758,11 +801,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                         mbar_arrive(bar(BVEMPTY0 + g));
                 }
 #pragma unroll
-                for (int w = 0; w < 4; ++w)
-                    oacc[t][w] = fmaf(oacc[t][w], aw[w], part[w].x + part[w].y);
+                for (int k = 0; k < 4; ++k)
+                    oacc[t][k] += quad_sum(pacc[k].x + pacc[k].y);
             }
             s += lp;
-            ++tile;
         }
         if (have_seg)
             flush(dseg);

@@ -32,17 +32,18 @@ template <int R, int TILE> struct TileLayout {
         const int cc = c - 8 * NBLK;
         return (uint32_t)(NBLK * TILE * 128 + row * TB + 16 * (cc ^ ((row * TB >> 7) & (TB / 16 - 1))));
     }
-    // zero rows [r0, r1) of the tile (all column blocks), lane-strided over one warp
-    __device__ static __forceinline__ void zero_rows(uint8_t *tile, int r0, int r1, int lane)
+    // zero rows [r0, r1) of the tile (all column blocks), strided over `n` threads (a warp's
+    // lanes by default; n = 1: one thread does it all)
+    __device__ static __forceinline__ void zero_rows(uint8_t *tile, int r0, int r1, int lane, int n = 32)
     {
         for (int blk = 0; blk < NBLK; ++blk) {
             uint4 *z = reinterpret_cast<uint4 *>(tile + blk * TILE * 128 + r0 * 128);
-            for (int e = lane; e < (r1 - r0) * 8; e += 32)
+            for (int e = lane; e < (r1 - r0) * 8; e += n)
                 z[e] = make_uint4(0u, 0u, 0u, 0u);
         }
         if (TAIL) {
             uint4 *z = reinterpret_cast<uint4 *>(tile + NBLK * TILE * 128 + r0 * TB);
-            for (int e = lane; e < (r1 - r0) * TB / 16; e += 32)
+            for (int e = lane; e < (r1 - r0) * TB / 16; e += n)
                 z[e] = make_uint4(0u, 0u, 0u, 0u);
         }
     }

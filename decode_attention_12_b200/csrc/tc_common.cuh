@@ -36,6 +36,16 @@ __device__ __forceinline__ uint64_t smem_desc(uint32_t addr, int row_bytes)
 
 constexpr int kFmtBf16 = 1, kFmtTf32 = 2;
 
+// True in exactly one lane of the (converged) warp: the lane that issues a tcgen05
+// operation while the whole warp runs the issuing loop with warp-uniform values.
+__device__ __forceinline__ bool elect_one()
+{
+    uint32_t pred = 0;
+    asm volatile("{\n\t.reg .pred P;\n\telect.sync _|P, 0xffffffff;\n\tselp.u32 %0, 1, 0, P;\n\t}"
+                 : "=r"(pred));
+    return pred != 0;
+}
+
 // Instruction descriptor: fp32 accumulator, A and B of format `fmt` (both K-major),
 // M x N tile.  kind::f16 takes kFmtBf16, kind::tf32 takes kFmtTf32.
 __host__ __device__ constexpr uint32_t idesc(int fmt, int m, int n)
@@ -106,6 +116,28 @@ __device__ __forceinline__ void ld_x8(uint32_t taddr, uint32_t (&r)[8])
     asm volatile("tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%8];"
                  : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
                    "=r"(r[7])
+                 : "r"(taddr));
+}
+
+// 16-lane x 256-bit fragments, repeated 16 times along the columns: thread t of the warp
+// receives, for i = 0..15, r[4i + 0..1] = (lane t/4, columns 8i + 2(t%4) + 0..1) and
+// r[4i + 2..3] = (lane t/4 + 8, the same columns), lanes counted from `taddr`'s lane.
+__device__ __forceinline__ void ld_16x256b_x16(uint32_t taddr, uint32_t (&r)[64])
+{
+    asm volatile("tcgen05.ld.sync.aligned.16x256b.x16.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, "
+                 "%12, %13, %14, %15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, "
+                 "%30, %31, %32, %33, %34, %35, %36, %37, %38, %39, %40, %41, %42, %43, %44, %45, %46, %47, "
+                 "%48, %49, %50, %51, %52, %53, %54, %55, %56, %57, %58, %59, %60, %61, %62, %63}, [%64];"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+                   "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
+                   "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]),
+                   "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]),
+                   "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31]), "=r"(r[32]), "=r"(r[33]), "=r"(r[34]),
+                   "=r"(r[35]), "=r"(r[36]), "=r"(r[37]), "=r"(r[38]), "=r"(r[39]), "=r"(r[40]), "=r"(r[41]),
+                   "=r"(r[42]), "=r"(r[43]), "=r"(r[44]), "=r"(r[45]), "=r"(r[46]), "=r"(r[47]), "=r"(r[48]),
+                   "=r"(r[49]), "=r"(r[50]), "=r"(r[51]), "=r"(r[52]), "=r"(r[53]), "=r"(r[54]), "=r"(r[55]),
+                   "=r"(r[56]), "=r"(r[57]), "=r"(r[58]), "=r"(r[59]), "=r"(r[60]), "=r"(r[61]), "=r"(r[62]),
+                   "=r"(r[63])
                  : "r"(taddr));
 }
 
