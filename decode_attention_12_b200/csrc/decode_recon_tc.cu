@@ -52,15 +52,18 @@ constexpr int kD = 128;         // head dimension served
 constexpr int kTile = 128;      // tokens per latent tile (M of the K_hat MMA)
 constexpr int kMaxLoops = 4;    // loop queries per pass
 constexpr int kGroups = 2;      // softmax warpgroups, alternate steps
-constexpr int kGroupThreads = 128;
-constexpr int kSoftThreads = kGroups * kGroupThreads;
-constexpr int kProducerWarp = 8, kMmaWarp = 9; // warps 10, 11 complete the third warpgroup
-constexpr int kThreads = 12 * 32;
-// Register split (setmaxnreg): launched at 168 per thread (384 x 168 = 64,512 of the SM's
-// 65,536), the producer/MMA warpgroup gives back to 104 and the two softmax warpgroups take
-// 200: 2 x 128 x 200 + 128 x 104 = 64,512, exactly the launch's total.
-constexpr int kLaunchRegs = 168, kSoftRegs = 200, kIssueRegs = 104;
-static_assert(2 * 128 * kSoftRegs + 128 * kIssueRegs <= kThreads * kLaunchRegs, "register split exceeds the launch");
+constexpr int kGroupWarps = 8;  // two per tensor-memory lane quarter, one per 16-lane half
+constexpr int kGroupThreads = kGroupWarps * 32;
+constexpr int kSoftWarps = kGroups * kGroupWarps;
+constexpr int kSoftThreads = kSoftWarps * 32;
+constexpr int kProducerWarp = kSoftWarps, kMmaWarp = kSoftWarps + 1; // + 2 idle warps: a fifth warpgroup
+constexpr int kThreads = (kSoftWarps + 4) * 32;
+// Register split (setmaxnreg): 640 threads launch with 96 registers each (61,440 of the
+// SM's 65,536); the producer/MMA warpgroup gives back to 56 and the four softmax warpgroups
+// take 104: 512 x 104 + 128 x 56 = 60,416.  The host checks the count the kernel was built
+// with before enabling it, so a split above the launch's total never runs.
+constexpr int kSoftRegs = 104, kIssueRegs = 56;
+constexpr int kSplitRegs = kSoftThreads * kSoftRegs + 128 * kIssueRegs;
 constexpr float kRescale = 8.0f; // lazy rescale margin (log2 units)
 
 // tensor-memory columns: K_hat of group g at 128 g, V_hat^T of group g at 256 + 128 g
@@ -100,22 +103,22 @@ template <int RK, int RV, bool ROPE> __host__ __device__ inline RLayout rlayout(
     o += ROPE ? lp * kD * 32 : 0;
     L.qv = o;                       // [lp][d] scaled query (kernel row order)
     o += lp * kD * 4;
-    L.qt4 = o;                      // [group][lp][4 row offsets][32] turned query, pairs 2c, 2c+1
-    o += ROPE ? kGroups * lp * 4 * 32 * 16 : 0;
+    L.qt4 = o;                      // [group][lp][2 row offsets][32] turned query, pairs 2c, 2c+1
+    o += ROPE ? kGroups * lp * 2 * 32 * 16 : 0;
     L.muk = o;                      // [lp][d]
     o += lp * kD * 4;
     L.muv = o;                      // [lp][d]
     o += lp * kD * 4;
     L.pv = o;                       // [group][2][128] softmax weights of a step
     o += kGroups * 2 * kTile * 4;
-    L.alpha = o;                    // [group][2][4 warps] max references of a step
-    o += kGroups * 2 * 4 * 4;
+    L.alpha = o;                    // [group][2][8 warps] max references of a step
+    o += kGroups * 2 * kGroupWarps * 4;
     L.xch = o;                      // [lp][d] group 1's share of a record
     o += lp * kD * 4;
     L.qmu = o;
     o += 16;
-    L.mrg = o;                      // [8 warps][4 loops][m, l]
-    o += 8 * kMaxLoops * 2 * 4;
+    L.mrg = o;                      // [16 warps][4 loops][m, l]
+    o += kSoftWarps * kMaxLoops * 2 * 4;
     L.omg = round_up(o, 8);
     o = L.omg + (ROPE ? kD / 2 * 8 : 0);
     L.bar = round_up(o, 8);
@@ -249,9 +252,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         for (int g = 0; g < kGroups; ++g) {
             mbar_init(bar(BKFULL0 + g), 1);
-            mbar_init(bar(BKEMPTY0 + g), 4); // one arrival per warp of the group
+            mbar_init(bar(BKEMPTY0 + g), kGroupWarps); // one arrival per warp of the group
             mbar_init(bar(BVFULL0 + g), 1);
-            mbar_init(bar(BVEMPTY0 + g), 4);
+            mbar_init(bar(BVEMPTY0 + g), kGroupWarps);
         }
         mbar_init(bar(BWREADY), 1);
         mbar_init(bar(BDRAIN), 1);
@@ -284,8 +287,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     int64_t s0, s1, chunk;
     cta_share(pref, B, H, a.chunk_min, s0, s1, chunk);
     const int64_t S_tot = pref[B];
-    if (warp >= 8) {
-      // ======== third warpgroup: producer warp, MMA warp, two idle warps ========
+    if (warp >= kSoftWarps) {
+      // ======== fifth warpgroup: producer warp, MMA warp, two idle warps ========
       asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kIssueRegs));
       if (s0 < s1 && warp == kProducerWarp) {
         // ================= producer: one lane streams the latent tiles =================
@@ -410,18 +413,19 @@ __global__ void __launch_bounds__(kThreads, 1)
               (void)mbar_wait_bounded(full_bar(i % nst), (i / nst) & 1);
       }
     } else {
-      // ======== two groups of 4 warps, alternate steps ========
-      // Tensor memory is read in 16-lane x 256-bit fragments: lane t of a warp holds rows
-      // rq, rq + 8, rq + 16, rq + 24 (rq = t / 4) of the warp's 32-lane quarter and columns
-      // 8 i + 2 j + {0, 1} (j = t % 4, i = 0..15), so a query or weight pair it loads from
-      // shared memory serves four rows, and a row's sum closes over the 4 lanes of a quad.
+      // ======== two groups of 8 warps, alternate steps ========
+      // Tensor memory is read in 16-lane x 256-bit fragments.  Warp (wq, hh) of a group owns
+      // lanes 32 wq + 16 hh .. + 15 of the buffers; its lane t holds rows rq and rq + 8
+      // (rq = t / 4) of those 16 and columns 8 i + 2 j + {0, 1} (j = t % 4), so a query or
+      // weight pair it loads from shared memory serves two rows, and a row's sum closes over
+      // the 4 lanes of a quad.
       asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kSoftRegs));
       if (s0 < s1) {
-        const int g = warp >> 2, wq = warp & 3, r = tid & 127;
-        const int j = lane & 3, rq = lane >> 2;
-        const uint32_t tq = tmem + ((uint32_t)(32 * wq) << 16); // this warp's lane quarter
-        // tile row / d-index of the thread's k-th row (k = 2 h + e: half h, +8 e)
-        auto row_of = [&](int k) { return 32 * wq + 16 * (k >> 1) + 8 * (k & 1) + rq; };
+        const int g = warp / kGroupWarps, gw = warp % kGroupWarps, wq = gw & 3, hh = gw >> 2;
+        const int r = tid % kGroupThreads, j = lane & 3, rq = lane >> 2;
+        const int tb = 2 * wq + hh;                      // this warp's 16-row block of the tile
+        const uint32_t tq = tmem + ((uint32_t)(32 * wq + 16 * hh) << 16);
+        auto row_of = [&](int e) { return 16 * tb + 8 * e + rq; }; // tile row / d-index of row e
         bool err = false;
         auto wait_all = [&](uint32_t b, uint32_t parity) -> bool {
             bool ok = !err && misc[0] == 0 && mbar_wait_bounded(b, parity);
@@ -436,12 +440,12 @@ __global__ void __launch_bounds__(kThreads, 1)
             x += __shfl_xor_sync(0xffffffffu, x, 1);
             return x + __shfl_xor_sync(0xffffffffu, x, 2);
         };
-        // rotation of the thread's base row b0 = 32 wq + rq: (cos, sin)(b0 w_P) for the pairs
-        // P = 8 i + 2 j + {0, 1}, i = 0..7 (rows b0 + 8 k turn the query instead)
+        // rotation of the thread's base row b0 = 16 tb + rq: (cos, sin)(b0 w_P) for the pairs
+        // P = 8 i + 2 j + {0, 1}, i = 0..7 (row b0 + 8 takes a query turned 8 steps further)
         float2 rc[ROPE ? 8 : 1], rs[ROPE ? 8 : 1];
         if (ROPE) {
             const float lb = log2f(a.rope_base);
-            const float b0 = (float)(32 * wq + rq);
+            const float b0 = (float)(16 * tb + rq);
 #pragma unroll
             for (int i = 0; i < 8; ++i) {
                 float sa, ca, sb, cb;
@@ -452,8 +456,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
         }
         // per loop: the group's running max (uniform), this thread's share of the sum of
-        // weights (the rows it writes), output sums of its 4 d-rows
-        float m[kMaxLoops], l[kMaxLoops], oacc[kMaxLoops][4];
+        // weights (the row it writes), output sums of its 2 d-rows
+        float m[kMaxLoops], l[kMaxLoops], oacc[kMaxLoops][2];
         const float *qv = reinterpret_cast<const float *>(smem + Ly.qv);
         const float *qmu = reinterpret_cast<const float *>(smem + Ly.qmu);
         const float *muv = reinterpret_cast<const float *>(smem + Ly.muv);
@@ -482,12 +486,12 @@ __global__ void __launch_bounds__(kThreads, 1)
                 M[t] = -INFINITY;
                 wg[t] = 0.f;
                 if (t < lp) {
-                    const float m0 = mrg[(0 * kMaxLoops + t) * 2], m1 = mrg[(4 * kMaxLoops + t) * 2];
+                    const float m0 = mrg[(0 * kMaxLoops + t) * 2], m1 = mrg[(kGroupWarps * kMaxLoops + t) * 2];
                     M[t] = fmaxf(m0, m1);
                     const float mine = g == 0 ? m0 : m1;
                     wg[t] = mine == -INFINITY ? 0.f : fast_exp2(mine - M[t]);
-                    if (g == 1)
-                        xch[t * kD + row_of(j)] = wg[t] * oacc[t][j];
+                    if (g == 1 && j < 2)
+                        xch[t * kD + row_of(j)] = wg[t] * (j == 0 ? oacc[t][0] : oacc[t][1]);
                 }
             }
             soft_sync();
@@ -497,17 +501,19 @@ __global__ void __launch_bounds__(kThreads, 1)
                     if (t < lp) {
                         float L = 0.f;
 #pragma unroll
-                        for (int w = 0; w < 8; ++w) {
+                        for (int w = 0; w < kSoftWarps; ++w) {
                             const float mw = mrg[(w * kMaxLoops + t) * 2];
                             if (mw != -INFINITY)
                                 L = fmaf(fast_exp2(mw - M[t]), mrg[(w * kMaxLoops + t) * 2 + 1], L);
                         }
-                        const int d = row_of(j);
-                        // + L mu_t^V: the mean left out of V_hat
-                        const float acc = fmaf(L, muv[t * kD + d], fmaf(wg[t], oacc[t][j], xch[t * kD + d]));
                         float *rec = a.part + (((int64_t)dd.u * a.Tq_all + a.tq_off + t) * a.seg_max + dd.j) *
                                                   part_stride(kD);
-                        rec[d] = acc;
+                        if (j < 2) {
+                            const int d = row_of(j);
+                            // + L mu_t^V: the mean left out of V_hat
+                            rec[d] = fmaf(L, muv[t * kD + d],
+                                          fmaf(wg[t], j == 0 ? oacc[t][0] : oacc[t][1], xch[t * kD + d]));
+                        }
                         if (r == 0) {
                             rec[kD] = M[t];
                             rec[kD + 1] = L;
@@ -528,6 +534,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         bool have_seg = false;
         int s = 0, prev_h = -1;
         int32_t qpos = 0;
+        const int st_ = tid; // 0 .. kSoftThreads - 1
         while (walk.next(pref, a.seq_start, B, H, d)) {
             if (d.flags & 1) {
                 // ---- new unit segment: close the previous one, stage this one's inputs
@@ -546,7 +553,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                         const float *wv = a.W_up_v + gi * RV * kD;
                         uint8_t *dk = smem + Ly.wk + t * 2 * Ly.wk_part;
                         uint8_t *dv = smem + Ly.wv + t * 2 * Ly.wv_part;
-                        for (int e = tid; e < RK * kD; e += kSoftThreads) {
+                        for (int e = st_; e < RK * kD; e += kSoftThreads) {
                             const int jj = e / kD, k = e - jj * kD;
                             const int row = ROPE ? pair_row(k, style) : k;
                             const float x = wk[e];
@@ -556,7 +563,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                             *reinterpret_cast<__nv_bfloat16 *>(dk + off) = hi;
                             *reinterpret_cast<__nv_bfloat16 *>(dk + Ly.wk_part + off) = lo;
                         }
-                        for (int e = tid; e < RV * kD; e += kSoftThreads) {
+                        for (int e = st_; e < RV * kD; e += kSoftThreads) {
                             const int jj = e / kD, k = e - jj * kD;
                             const float x = wv[e];
                             const __nv_bfloat16 hi = __float2bfloat16_rn(x);
@@ -565,11 +572,12 @@ __global__ void __launch_bounds__(kThreads, 1)
                             *reinterpret_cast<__nv_bfloat16 *>(dv + off) = hi;
                             *reinterpret_cast<__nv_bfloat16 *>(dv + Ly.wv_part + off) = lo;
                         }
-                        if (g == 0) {
-                            const float mk = a.mu_k[gi * kD + r];
-                            const int row = ROPE ? pair_row(r, style) : r;
+                        if (st_ < kD) {
+                            const int k = st_;
+                            const float mk = a.mu_k[gi * kD + k];
+                            const int row = ROPE ? pair_row(k, style) : k;
                             reinterpret_cast<float *>(smem + Ly.muk)[t * kD + row] = mk;
-                            reinterpret_cast<float *>(smem + Ly.muv)[t * kD + r] = a.mu_v[gi * kD + r];
+                            reinterpret_cast<float *>(smem + Ly.muv)[t * kD + k] = a.mu_v[gi * kD + k];
                             if (ROPE) { // mu_t^K as the B tile of the ones MMA: columns 0, 1 = hi, lo
                                 const __nv_bfloat16 hi = __float2bfloat16_rn(mk);
                                 const __nv_bfloat16 lo = __float2bfloat16_rn(mk - __bfloat162float(hi));
@@ -581,11 +589,12 @@ __global__ void __launch_bounds__(kThreads, 1)
                             }
                         }
                     }
-                    if (g == 1) { // scaled query of this (sequence, head) and loop, kernel row order
+                    if (st_ >= kD && st_ < 2 * kD) { // scaled query of this (sequence, head) and loop
+                        const int k = st_ - kD;
                         const __nv_bfloat16 *qrow = static_cast<const __nv_bfloat16 *>(a.q) +
                                                     (((int64_t)d.b * a.Tq_all + a.tq_off + t) * H + d.h) * kD;
-                        reinterpret_cast<float *>(smem + Ly.qv)[t * kD + (ROPE ? pair_row(r, style) : r)] =
-                            __bfloat162float(qrow[r]) * a.scale * kLog2e;
+                        reinterpret_cast<float *>(smem + Ly.qv)[t * kD + (ROPE ? pair_row(k, style) : k)] =
+                            __bfloat162float(qrow[k]) * a.scale * kLog2e;
                     }
                 }
                 if (wchange)
@@ -612,20 +621,19 @@ __global__ void __launch_bounds__(kThreads, 1)
                 for (int t = 0; t < kMaxLoops; ++t) {
                     m[t] = -INFINITY;
                     l[t] = 0.f;
-#pragma unroll
-                    for (int k = 0; k < 4; ++k)
-                        oacc[t][k] = 0.f;
+                    oacc[t][0] = oacc[t][1] = 0.f;
                 }
             }
             // does this group take any step of the tile?
             const bool mine = lp > 1 || (s & 1) == g;
             if (ROPE && mine) {
-                // the tile's query, once per row offset 8 v (v = 0..3) of the thread rows:
-                // R((p - n0 - 8 v) w) q for pairs 2c, 2c + 1; entry [loop][v][couple c]
+                // the tile's query, once per row offset 8 v (v = 0, 1) within a 16-row block:
+                // R((p - n0 - 8 v) w) q for pairs 2c, 2c + 1; entry [loop][v][couple c]; the
+                // block offset 16 tb sits in the thread's own rotation
                 const double *omg = reinterpret_cast<const double *>(smem + Ly.omg);
-                float4 *qt = reinterpret_cast<float4 *>(smem + Ly.qt4) + g * lp * 4 * 32;
-                for (int e = r; e < lp * 4 * 32; e += kGroupThreads) {
-                    const int c = e & 31, v = (e >> 5) & 3, t = e >> 7;
+                float4 *qt = reinterpret_cast<float4 *>(smem + Ly.qt4) + g * lp * 2 * 32;
+                for (int e = r; e < lp * 2 * 32; e += kGroupThreads) {
+                    const int c = e & 31, v = (e >> 5) & 1, t = e >> 6;
                     const int64_t rel = (int64_t)qpos - d.n0 - 8 * v;
                     float qa2[2], qb2[2];
 #pragma unroll
@@ -652,47 +660,43 @@ __global__ void __launch_bounds__(kThreads, 1)
                     continue;
                 const int use = ss >> 1;
                 const int pb = use & 1; // this group's weight / reference buffer of the step
-                // ---- scores of loop t for the thread's 4 token rows
-                float sc[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+                // ---- scores of loop t for the thread's 2 token rows
+                float sc[2] = {-INFINITY, -INFINITY};
                 if (wait_all(bar(BKFULL0 + g), use & 1)) {
                     tc::fence_after();
-                    float2 acc[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f),
-                                     make_float2(0.f, 0.f)};
+                    float2 acc[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
                     if (!ROPE) {
-                        float2 qp[16]; // q pairs at columns 8 i + 2 j
-                        const float2 *q2 = reinterpret_cast<const float2 *>(qv + t * kD + 2 * j);
+                        const float2 *q2 = reinterpret_cast<const float2 *>(qv + t * kD + 2 * j); // q pairs
 #pragma unroll
-                        for (int i = 0; i < 16; ++i)
-                            qp[i] = q2[4 * i];
-#pragma unroll
-                        for (int h = 0; h < 2; ++h) {
-                            uint32_t kr[64];
-                            tc::ld_16x256b_x16(tq + ((uint32_t)(16 * h) << 16) + col_k(g), kr);
+                        for (int c = 0; c < 2; ++c) { // columns 64 c .. 64 c + 63
+                            uint32_t kr[32];
+                            tc::ld_16x256b_x8(tq + col_k(g) + 64 * c, kr);
                             tc::wait_ld();
-                            if (h == 1) {
+                            if (c == 1) {
                                 tc::fence_before();
                                 __syncwarp();
                                 if (lane == 0)
                                     mbar_arrive(bar(BKEMPTY0 + g));
                             }
 #pragma unroll
-                            for (int i = 0; i < 16; ++i) {
-                                acc[2 * h] = __ffma2_rn(qp[i], f2(kr[4 * i], kr[4 * i + 1]), acc[2 * h]);
-                                acc[2 * h + 1] = __ffma2_rn(qp[i], f2(kr[4 * i + 2], kr[4 * i + 3]), acc[2 * h + 1]);
+                            for (int i = 0; i < 8; ++i) {
+                                const float2 qq = q2[4 * (8 * c + i)];
+                                acc[0] = __ffma2_rn(qq, f2(kr[4 * i], kr[4 * i + 1]), acc[0]);
+                                acc[1] = __ffma2_rn(qq, f2(kr[4 * i + 2], kr[4 * i + 3]), acc[1]);
                             }
                         }
-#pragma unroll
-                        for (int k = 0; k < 4; ++k)
-                            sc[k] = quad_sum(acc[k].x + acc[k].y) + qmu[t];
+                        sc[0] = quad_sum(acc[0].x + acc[0].y) + qmu[t];
+                        sc[1] = quad_sum(acc[1].x + acc[1].y) + qmu[t];
                     } else {
-                        // row k = 2 h + e uses the query turned by its row offset 8 k
-                        const float4 *qt = reinterpret_cast<const float4 *>(smem + Ly.qt4) + (g * lp + t) * 4 * 32;
+                        // row e uses the query turned by its row offset 8 e
+                        const float4 *qt = reinterpret_cast<const float4 *>(smem + Ly.qt4) + (g * lp + t) * 2 * 32;
 #pragma unroll
-                        for (int h = 0; h < 2; ++h) {
-                            uint32_t kr[64];
-                            tc::ld_16x256b_x16(tq + ((uint32_t)(16 * h) << 16) + col_k(g), kr);
+                        for (int c = 0; c < 2; ++c) { // pairs 32 c .. 32 c + 31: columns i and i + 8
+                            uint32_t ka[16], kb[16];
+                            tc::ld_16x256b_x4(tq + col_k(g) + 32 * c, ka);
+                            tc::ld_16x256b_x4(tq + col_k(g) + kD / 2 + 32 * c, kb);
                             tc::wait_ld();
-                            if (h == 1) {
+                            if (c == 1) {
                                 tc::fence_before();
                                 __syncwarp();
                                 if (lane == 0)
@@ -700,99 +704,96 @@ __global__ void __launch_bounds__(kThreads, 1)
                             }
 #pragma unroll
                             for (int e = 0; e < 2; ++e) {
-                                const int k = 2 * h + e;
 #pragma unroll
-                                for (int i = 0; i < 8; ++i) { // pairs 8 i + 2 j + {0, 1}: columns i, i + 8
-                                    const float4 qq = qt[k * 32 + 4 * i + j];
+                                for (int ii = 0; ii < 4; ++ii) {
+                                    const int i = 4 * c + ii;
+                                    const float4 qq = qt[e * 32 + 4 * i + j];
                                     const float2 qa = make_float2(qq.x, qq.y), qb = make_float2(qq.z, qq.w);
                                     const float2 qas = __fmul2_rn(qa, rs[i]);
                                     // x (qa cos + qb sin) + y (qb cos - qa sin)
                                     const float2 t1 = __ffma2_rn(qa, rc[i], __fmul2_rn(qb, rs[i]));
                                     const float2 t2 = __ffma2_rn(qb, rc[i], make_float2(-qas.x, -qas.y));
-                                    acc[k] = __ffma2_rn(f2(kr[4 * i + 2 * e], kr[4 * i + 2 * e + 1]), t1, acc[k]);
-                                    acc[k] = __ffma2_rn(f2(kr[4 * (i + 8) + 2 * e], kr[4 * (i + 8) + 2 * e + 1]), t2,
-                                                        acc[k]);
+                                    acc[e] = __ffma2_rn(f2(ka[4 * ii + 2 * e], ka[4 * ii + 2 * e + 1]), t1, acc[e]);
+                                    acc[e] = __ffma2_rn(f2(kb[4 * ii + 2 * e], kb[4 * ii + 2 * e + 1]), t2, acc[e]);
                                 }
                             }
                         }
-#pragma unroll
-                        for (int k = 0; k < 4; ++k)
-                            sc[k] = quad_sum(acc[k].x + acc[k].y);
+                        sc[0] = quad_sum(acc[0].x + acc[0].y);
+                        sc[1] = quad_sum(acc[1].x + acc[1].y);
                     }
                 } else {
                     __syncwarp();
                     if (lane == 0)
                         mbar_arrive(bar(BKEMPTY0 + g));
                 }
-#pragma unroll
-                for (int k = 0; k < 4; ++k)
-                    if (row_of(k) >= d.rows)
-                        sc[k] = -INFINITY;
+                if (row_of(0) >= d.rows)
+                    sc[0] = -INFINITY;
+                if (row_of(1) >= d.rows)
+                    sc[1] = -INFINITY;
                 // ---- online softmax: each warp picks a reference (the group's running max, or
                 // its own max when that is more than the margin higher), the group reconciles
-                float mx = fmaxf(fmaxf(sc[0], sc[1]), fmaxf(sc[2], sc[3]));
+                float mx = fmaxf(sc[0], sc[1]);
 #pragma unroll
                 for (int off = 4; off < 32; off <<= 1)
                     mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
                 const float ref = mx > m[t] + kRescale ? mx : m[t];
-                float p[4];
-#pragma unroll
-                for (int k = 0; k < 4; ++k)
-                    p[k] = sc[k] == -INFINITY ? 0.f : fast_exp2(sc[k] - ref);
-                const float pmine = j == 0 ? p[0] : j == 1 ? p[1] : j == 2 ? p[2] : p[3];
+                const float sm_ = j == 0 ? sc[0] : sc[1];
+                const float pmine = sm_ == -INFINITY ? 0.f : fast_exp2(sm_ - ref); // rows j = 0, 1 write
                 float *pw = reinterpret_cast<float *>(smem + Ly.pv) + (g * 2 + pb) * kTile;
-                float *rw = reinterpret_cast<float *>(smem + Ly.alpha) + (g * 2 + pb) * 4;
-                pw[row_of(j)] = pmine;
+                float *rw = reinterpret_cast<float *>(smem + Ly.alpha) + (g * 2 + pb) * kGroupWarps;
+                if (j < 2)
+                    pw[row_of(j)] = pmine;
                 if (lane == 0)
-                    rw[wq] = ref;
+                    rw[tb] = ref;
                 group_sync(g);
-                const float4 rf = *reinterpret_cast<const float4 *>(rw);
-                const float Mn = fmaxf(fmaxf(rf.x, rf.y), fmaxf(rf.z, rf.w));
-                float f[4] = {1.f, 1.f, 1.f, 1.f};
-                if (Mn != -INFINITY && !(rf.x == Mn && rf.y == Mn && rf.z == Mn && rf.w == Mn)) {
-                    f[0] = fast_exp2(rf.x - Mn);
-                    f[1] = fast_exp2(rf.y - Mn);
-                    f[2] = fast_exp2(rf.z - Mn);
-                    f[3] = fast_exp2(rf.w - Mn);
+                const float4 ra = *reinterpret_cast<const float4 *>(rw), rb = *reinterpret_cast<const float4 *>(rw + 4);
+                const float Mn = fmaxf(fmaxf(fmaxf(ra.x, ra.y), fmaxf(ra.z, ra.w)), fmaxf(fmaxf(rb.x, rb.y), fmaxf(rb.z, rb.w)));
+                float f[8] = {1.f, 1.f, 1.f, 1.f, 1.f, 1.f, 1.f, 1.f};
+                const bool same = ra.x == Mn && ra.y == Mn && ra.z == Mn && ra.w == Mn && rb.x == Mn && rb.y == Mn &&
+                                  rb.z == Mn && rb.w == Mn;
+                if (Mn != -INFINITY && !same) {
+                    f[0] = fast_exp2(ra.x - Mn);
+                    f[1] = fast_exp2(ra.y - Mn);
+                    f[2] = fast_exp2(ra.z - Mn);
+                    f[3] = fast_exp2(ra.w - Mn);
+                    f[4] = fast_exp2(rb.x - Mn);
+                    f[5] = fast_exp2(rb.y - Mn);
+                    f[6] = fast_exp2(rb.z - Mn);
+                    f[7] = fast_exp2(rb.w - Mn);
                 }
                 if (Mn > m[t]) { // the group's max rose: rescale what was summed so far
                     const float al = fast_exp2(m[t] - Mn);
                     l[t] *= al;
-#pragma unroll
-                    for (int k = 0; k < 4; ++k)
-                        oacc[t][k] *= al;
+                    oacc[t][0] *= al;
+                    oacc[t][1] *= al;
                     m[t] = Mn;
                 }
-                const float fmine = wq == 0 ? f[0] : wq == 1 ? f[1] : wq == 2 ? f[2] : f[3];
-                l[t] = fmaf(fmine, pmine, l[t]);
-                // ---- output: sum over the tile's tokens of p v_hat at the thread's 4 d-rows
-                float2 pacc[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f),
-                                  make_float2(0.f, 0.f)};
+                if (j < 2)
+                    l[t] = fmaf(f[tb], pmine, l[t]);
+                // ---- output: sum over the tile's tokens of p v_hat at the thread's 2 d-rows
+                float2 pacc[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
                 if (wait_all(bar(BVFULL0 + g), use & 1)) {
                     tc::fence_after();
-                    float2 pp[16]; // weight pairs of tokens 8 i + 2 j, on the common reference
-                    const float2 *p2 = reinterpret_cast<const float2 *>(pw + 2 * j);
+                    const float2 *p2 = reinterpret_cast<const float2 *>(pw + 2 * j); // tokens 8 i + 2 j
 #pragma unroll
-                    for (int i = 0; i < 16; ++i) {
-                        const float fi = f[i >> 2];
-                        const float2 x = p2[4 * i];
-                        pp[i] = make_float2(x.x * fi, x.y * fi);
-                    }
-#pragma unroll
-                    for (int h = 0; h < 2; ++h) {
-                        uint32_t vr[64];
-                        tc::ld_16x256b_x16(tq + ((uint32_t)(16 * h) << 16) + col_v(g), vr);
+                    for (int c = 0; c < 2; ++c) { // tokens 64 c .. 64 c + 63
+                        uint32_t vr[32];
+                        tc::ld_16x256b_x8(tq + col_v(g) + 64 * c, vr);
                         tc::wait_ld();
-                        if (h == 1) {
+                        if (c == 1) {
                             tc::fence_before();
                             __syncwarp();
                             if (lane == 0)
                                 mbar_arrive(bar(BVEMPTY0 + g));
                         }
 #pragma unroll
-                        for (int i = 0; i < 16; ++i) {
-                            pacc[2 * h] = __ffma2_rn(pp[i], f2(vr[4 * i], vr[4 * i + 1]), pacc[2 * h]);
-                            pacc[2 * h + 1] = __ffma2_rn(pp[i], f2(vr[4 * i + 2], vr[4 * i + 3]), pacc[2 * h + 1]);
+                        for (int i = 0; i < 8; ++i) {
+                            const int ti = 8 * c + i; // tokens 8 ti + 2 j: 16-row block ti / 2
+                            float2 pq = p2[4 * ti];
+                            if (!same)
+                                pq = make_float2(pq.x * f[ti >> 1], pq.y * f[ti >> 1]);
+                            pacc[0] = __ffma2_rn(pq, f2(vr[4 * i], vr[4 * i + 1]), pacc[0]);
+                            pacc[1] = __ffma2_rn(pq, f2(vr[4 * i + 2], vr[4 * i + 3]), pacc[1]);
                         }
                     }
                 } else {
@@ -800,9 +801,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                     if (lane == 0)
                         mbar_arrive(bar(BVEMPTY0 + g));
                 }
-#pragma unroll
-                for (int k = 0; k < 4; ++k)
-                    oacc[t][k] += quad_sum(pacc[k].x + pacc[k].y);
+                oacc[t][0] += quad_sum(pacc[0].x + pacc[0].y);
+                oacc[t][1] += quad_sum(pacc[1].x + pacc[1].y);
             }
             s += lp;
         }
@@ -849,12 +849,31 @@ int decode_recon_tc_smem_bytes(int r_k, int r_v, bool rope, int lp, int B)
     return -1;
 }
 
+// Registers per thread the kernel instantiation launches with (0 when unknown).
+static int rtc_launch_regs(int r_k, int r_v, bool rope)
+{
+    cudaFuncAttributes fa;
+    cudaError_t e = cudaErrorInvalidValue;
+#define LLA_RTC_REGS(RK, RV) \
+    if (r_k == RK && r_v == RV) \
+        e = rope ? cudaFuncGetAttributes(&fa, decode_recon_tc_kernel<RK, RV, true>) \
+                 : cudaFuncGetAttributes(&fa, decode_recon_tc_kernel<RK, RV, false>);
+    LLA_RTC_REGS(16, 32)
+    LLA_RTC_REGS(16, 16)
+    LLA_RTC_REGS(32, 32)
+#undef LLA_RTC_REGS
+    return e == cudaSuccess ? fa.numRegs : 0;
+}
+
 bool decode_recon_tc_supported(int dtype, int r_k, int r_v, int d, int fold, int B, bool rope)
 {
     if (dtype != LLA_BF16 || d != kD || fold != LLA_PER_HEAD || tensor_map_encoder() == nullptr)
         return false;
     const int smem = decode_recon_tc_smem_bytes(r_k, r_v, rope, kMaxLoops, B);
-    return smem > 0 && smem <= 227 * 1024;
+    if (smem <= 0 || smem > 227 * 1024)
+        return false;
+    // setmaxnreg redistributes the registers the CTA was launched with: the split must fit
+    return rtc_launch_regs(r_k, r_v, rope) * kThreads >= kSplitRegs;
 }
 
 int decode_recon_tc_loops_per_pass() { return kMaxLoops; }
