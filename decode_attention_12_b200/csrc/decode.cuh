@@ -63,6 +63,9 @@ cudaError_t launch_absorb_prologue(const DecodeArgs &a, int dtype, cudaStream_t 
 cudaError_t launch_decode_combine(const DecodeArgs &a, int dtype, int out_dtype, cudaStream_t stream);
 bool decode_absorb_supported(int dtype, int r_k, int r_v, int d, int fold);
 bool decode_mma_supported(int dtype, int r_k, int r_v, int fold, int Tq);
+// loop queries one pass of the tensor-core kernel serves (two m16 row tiles; 16 with a
+// decoupled rotary sub-key)
+int decode_mma_loops_per_pass(int d_rope);
 bool decode_mma_rope_supported(int dtype, int r_k, int r_v, int d_rope, int fold);
 cudaError_t launch_decode_absorb_mma(const DecodeArgs &a, int ctas, cudaStream_t stream);
 bool decode_reconstruct_supported(int dtype, int r_k, int r_v, int d);

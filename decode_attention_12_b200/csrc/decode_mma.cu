@@ -30,11 +30,15 @@ using namespace mma;
 // Pith verdict record's decoupled RoPE for the absorbed variant); its tile sits beside
 // the key tile and adds DR / 16 k16 steps to the score MMA, with the rotated rotary query
 // part appended to q_tilde (rows of RK + DR).
-template <int RK, int RV, int NW, int DR = 0> struct MCfg {
+// RT row tiles: the loop queries of a pass fill RT m16 tiles (RT = 2: up to 32 queries), each
+// taken by its own NW consumer warps over the same staged latent tile, so one read of the
+// latents serves them all.
+template <int RK, int RV, int NW, int DR = 0, int RT = 1> struct MCfg {
     static constexpr int TILE = 32 * NW;
-    static constexpr int THREADS = (NW + 1) * 32;
-    static constexpr int CONSUMERS = NW * 32;
-    static constexpr int STAGES = (RK + RV + DR) * 2 * TILE > 24 * 1024 ? 2 : 3;
+    static constexpr int CW = NW * RT; // consumer warps
+    static constexpr int THREADS = (CW + 1) * 32;
+    static constexpr int CONSUMERS = CW * 32;
+    static constexpr int STAGES = RT > 1 ? 3 : ((RK + RV + DR) * 2 * TILE > 24 * 1024 ? 2 : 3);
     using LK = TileLayout<RK, TILE>;
     using LV = TileLayout<RV, TILE>;
     using LR = TileLayout<(DR > 0 ? DR : 16), TILE>;
@@ -44,25 +48,25 @@ template <int RK, int RV, int NW, int DR = 0> struct MCfg {
     static constexpr int NTV = RV / 8;  // n8 tiles of the output
     static constexpr int K_BYTES = LK::BYTES, V_BYTES = LV::BYTES, R_BYTES = DR > 0 ? LR::BYTES : 0;
     static constexpr int Q_OFF = K_BYTES + V_BYTES + R_BYTES;
-    static constexpr int Q_BYTES = 16 * RKT * 4;
+    static constexpr int Q_BYTES = 16 * RT * RKT * 4;
     static constexpr int STAGE = align1024(Q_OFF + Q_BYTES);
     static constexpr int RING = STAGES * STAGE;
-    static constexpr int MRG_OFF = RING;                              // [NW][16][RV + 2]
-    static constexpr int BAR_OFF = (MRG_OFF + NW * 16 * (RV + 2) * 4 + 15) & ~15; // full[S], empty[S]
+    static constexpr int MRG_OFF = RING;                              // [NW][16 RT][RV + 2]
+    static constexpr int BAR_OFF = (MRG_OFF + NW * 16 * RT * (RV + 2) * 4 + 15) & ~15; // full[S], empty[S]
     static constexpr int MISC_OFF = BAR_OFF + 2 * STAGES * 8;
-    static constexpr int SCR_OFF = (MISC_OFF + 16 + 15) & ~15;        // int64 [NW + 1]
-    static constexpr int PREF_OFF = SCR_OFF + (NW + 1) * 8;           // int64 [B + 1]
+    static constexpr int SCR_OFF = (MISC_OFF + 16 + 15) & ~15;        // int64 [CW + 2]
+    static constexpr int PREF_OFF = SCR_OFF + (CW + 2) * 8;           // int64 [B + 1]
 };
 
 // TQ16: the tile carries more than 8 loop queries, so fragment rows g + 8 are real.
-template <int RK, int RV, bool TQ16, int NW, int DR>
+template <int RK, int RV, bool TQ16, int NW, int DR, int RT = 1>
 __device__ __forceinline__ void decode_mma_body(const CUtensorMap *map_k, const CUtensorMap *map_kt,
                                                 const CUtensorMap *map_v, const CUtensorMap *map_vt,
                                                 const CUtensorMap *map_r, const CUtensorMap *map_rt,
                                                 const DecodeArgs &a)
 {
-    using C = MCfg<RK, RV, NW, DR>;
-    constexpr int kWarps = NW, kThreads = C::THREADS, kConsumers = C::CONSUMERS, kTile = C::TILE;
+    using C = MCfg<RK, RV, NW, DR, RT>;
+    constexpr int kWarps = C::CW, kThreads = C::THREADS, kConsumers = C::CONSUMERS, kTile = C::TILE;
     constexpr int kStages = C::STAGES;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
@@ -156,6 +160,9 @@ __device__ __forceinline__ void decode_mma_body(const CUtensorMap *map_k, const 
         }
     } else {
         // ================= consumer warps =================
+        // warp = rt * NW + tw: token group tw (32 tokens of the tile), row tile rt (queries
+        // 16 rt .. 16 rt + 15)
+        const int tw = warp % NW, rt = warp / NW;
         uint32_t qa[C::KS + C::KSR][2][4]; // q_tilde A fragments, [k16 step][hi/lo][a0..a3]
         float o[C::NTV][4];       // output accumulator fragments (rows g, g + 8)
         float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.f, l1 = 0.f;
@@ -172,7 +179,7 @@ __device__ __forceinline__ void decode_mma_body(const CUtensorMap *map_k, const 
                 // from beyond the segment, or never written): their p is 0, but 0 * NaN is NaN
                 // in the MMA, so that warp zeroes those value rows.
                 const int r0 = d.rows, r1 = (d.rows + 31) & ~31;
-                if (r0 < r1 && warp == (r0 >> 5)) {
+                if (r0 < r1 && tw == (r0 >> 5)) { // (each row tile's warp zeroes the same rows)
                     C::LV::zero_rows(smem + stage * C::STAGE + C::K_BYTES, r0, r1, lane);
                     __syncwarp();
                 }
@@ -184,8 +191,8 @@ __device__ __forceinline__ void decode_mma_body(const CUtensorMap *map_k, const 
                         const int c0 = 16 * kk + 2 * tq;
                         float x[4][2];
 #pragma unroll
-                        for (int r = 0; r < 2; ++r) { // rows g, g + 8
-                            const int row = g + 8 * r;
+                        for (int r = 0; r < 2; ++r) { // rows g, g + 8 of the row tile
+                            const int row = 16 * rt + g + 8 * r;
                             const bool in = row < Tq;
                             x[r][0] = in ? qs[row * QL + c0] : 0.f;
                             x[r][1] = in ? qs[row * QL + c0 + 1] : 0.f;
@@ -203,7 +210,7 @@ __device__ __forceinline__ void decode_mma_body(const CUtensorMap *map_k, const 
                     m0 = m1 = -INFINITY;
                     l0 = l1 = 0.f;
                 }
-                const int tbase = warp * 32; // this warp's 32 tokens of the tile
+                const int tbase = tw * 32; // this warp's 32 tokens of the tile
                 if (tbase < d.rows) {
                     // ---- a2: scores for 32 tokens (4 n8 tiles)
                     float s[4][4];
@@ -334,10 +341,10 @@ __device__ __forceinline__ void decode_mma_body(const CUtensorMap *map_k, const 
                 lq0 += __shfl_xor_sync(0xffffffffu, lq0, 2);
                 float lq1 = l1 + __shfl_xor_sync(0xffffffffu, l1, 1);
                 lq1 += __shfl_xor_sync(0xffffffffu, lq1, 2);
-                float *mw = mrg + warp * 16 * (RV + 2);
+                float *mw = mrg + tw * 16 * RT * (RV + 2); // [token group][query row][RV + 2]
 #pragma unroll
                 for (int r = 0; r < 2; ++r) {
-                    const int row = g + 8 * r;
+                    const int row = 16 * rt + g + 8 * r;
                     if (row < Tq) {
 #pragma unroll
                         for (int j = 0; j < C::NTV; ++j) {
@@ -356,17 +363,17 @@ __device__ __forceinline__ void decode_mma_body(const CUtensorMap *map_k, const 
                         const int row = idx / (RV + 2), jj = idx - row * (RV + 2);
                         float M = -INFINITY;
 #pragma unroll
-                        for (int w = 0; w < kWarps; ++w)
-                            M = fmaxf(M, mrg[(w * 16 + row) * (RV + 2) + RV]);
+                        for (int w = 0; w < NW; ++w)
+                            M = fmaxf(M, mrg[(w * 16 * RT + row) * (RV + 2) + RV]);
                         float val = 0.f;
                         if (jj == RV) {
                             val = M;
                         } else {
 #pragma unroll
-                            for (int w = 0; w < kWarps; ++w) {
-                                const float mwv = mrg[(w * 16 + row) * (RV + 2) + RV];
+                            for (int w = 0; w < NW; ++w) {
+                                const float mwv = mrg[(w * 16 * RT + row) * (RV + 2) + RV];
                                 if (mwv != -INFINITY)
-                                    val += fast_exp2(mwv - M) * mrg[(w * 16 + row) * (RV + 2) + jj];
+                                    val += fast_exp2(mwv - M) * mrg[(w * 16 * RT + row) * (RV + 2) + jj];
                             }
                         }
                         a.part[(((int64_t)d.u * a.Tq_all + a.tq_off + row) * a.seg_max + d.j) * part_stride(RV) + jj] =
@@ -392,13 +399,13 @@ __device__ __forceinline__ void decode_mma_body(const CUtensorMap *map_k, const 
     }
 }
 
-template <int RK, int RV, bool TQ16, int NW, int MINB>
-__global__ void __launch_bounds__((NW + 1) * 32, MINB)
+template <int RK, int RV, bool TQ16, int NW, int MINB, int RT = 1>
+__global__ void __launch_bounds__((NW * RT + 1) * 32, MINB)
     decode_absorb_mma_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant__ CUtensorMap map_kt,
                              const __grid_constant__ CUtensorMap map_v, const __grid_constant__ CUtensorMap map_vt,
                              const DecodeArgs a)
 {
-    decode_mma_body<RK, RV, TQ16, NW, 0>(&map_k, &map_kt, &map_v, &map_vt, nullptr, nullptr, a);
+    decode_mma_body<RK, RV, TQ16, NW, 0, RT>(&map_k, &map_kt, &map_v, &map_vt, nullptr, nullptr, a);
 }
 
 // With the decoupled rotary sub-key plane (two more tensor maps).
@@ -413,10 +420,10 @@ __global__ void __launch_bounds__((NW + 1) * 32, MINB)
 }
 
 // ---- host ------------------------------------------------------------------------------
-template <int RK, int RV, bool TQ16, int NW, int MINB, int DR>
+template <int RK, int RV, bool TQ16, int NW, int MINB, int DR, int RT = 1>
 cudaError_t launch_mma_t(const DecodeArgs &a, int ctas, cudaStream_t stream)
 {
-    using C = MCfg<RK, RV, NW, DR>;
+    using C = MCfg<RK, RV, NW, DR, RT>;
     const int Hs = a.fold ? 1 : a.H;
     CUtensorMap mk, mkt, mv, mvt, mr, mrt;
     if (!plane_maps(&mk, &mkt, a.k, RK, (int64_t)Hs * a.slots) ||
@@ -427,7 +434,7 @@ cudaError_t launch_mma_t(const DecodeArgs &a, int ctas, cudaStream_t stream)
     if constexpr (DR > 0)
         kern = (const void *)decode_absorb_mma_rope_kernel<RK, RV, TQ16, NW, MINB, DR>;
     else
-        kern = (const void *)decode_absorb_mma_kernel<RK, RV, TQ16, NW, MINB>;
+        kern = (const void *)decode_absorb_mma_kernel<RK, RV, TQ16, NW, MINB, RT>;
     const int smem = C::PREF_OFF + 8 * (a.B + 1) + 1024;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess)
@@ -457,7 +464,7 @@ cudaError_t launch_mma_t(const DecodeArgs &a, int ctas, cudaStream_t stream)
         return cudaLaunchKernelEx(&cfg, decode_absorb_mma_rope_kernel<RK, RV, TQ16, NW, MINB, DR>, mk, mkt, mv, mvt,
                                   mr, mrt, a);
     else
-        return cudaLaunchKernelEx(&cfg, decode_absorb_mma_kernel<RK, RV, TQ16, NW, MINB>, mk, mkt, mv, mvt, a);
+        return cudaLaunchKernelEx(&cfg, decode_absorb_mma_kernel<RK, RV, TQ16, NW, MINB, RT>, mk, mkt, mv, mvt, a);
 }
 
 // Small ranks: 128-token tiles, 4 consumer warps, 4 CTAs per SM.  Ranks >= 64: 64-token
@@ -468,15 +475,22 @@ cudaError_t launch_mma(const DecodeArgs &a, int ctas, cudaStream_t stream)
     constexpr bool big = RK >= 64 || RV >= 64;
     // a 64-wide rotary sub-key adds 32 registers of q_tilde fragments: 3 CTAs per SM
     constexpr int NW = big ? 2 : 4, MINB = big ? 2 : (DR >= 64 ? 3 : 4);
+    if constexpr (DR == 0) {
+        // 17 .. 32 loop queries: two row tiles over one staged latent tile (one pass)
+        if (a.Tq > 16)
+            return launch_mma_t<RK, RV, true, NW, big ? 1 : 2, 0, 2>(a, ctas, stream);
+    }
     return a.Tq > 8 ? launch_mma_t<RK, RV, true, NW, MINB, DR>(a, ctas, stream)
                     : launch_mma_t<RK, RV, false, NW, MINB, DR>(a, ctas, stream);
 }
 
 } // namespace
 
+int decode_mma_loops_per_pass(int d_rope) { return d_rope > 0 ? 16 : 32; }
+
 bool decode_mma_supported(int dtype, int r_k, int r_v, int fold, int Tq)
 {
-    (void)Tq; // more than 16 loop queries run as passes of 16
+    (void)Tq; // more than decode_mma_loops_per_pass() loop queries run as several passes
     const bool pair = (r_k == 16 && r_v == 32) || (r_k == 16 && r_v == 16) || (r_k == 32 && r_v == 32) ||
                       (r_k == 64 && r_v == 128) || (r_k == 96 && r_v == 160) || (r_k == 128 && r_v == 128);
     return dtype == LLA_BF16 && pair && tensor_map_encoder() != nullptr;

@@ -548,17 +548,18 @@ int decode_call(const lla_dims *dims, int32_t layer, int32_t t0, int32_t Tq, con
         return err == cudaSuccess ? LLA_OK : LLA_ERR_CUDA;
     }
     if (use_mma) {
-        // tensor-core kernel: up to 16 loop queries (one m16 tile) per pass over the latents
-        for (int32_t c = 0; c < Tq && err == cudaSuccess; c += 16) {
+        // tensor-core kernel: up to 32 loop queries (two m16 row tiles) per pass over the latents
+        const int per = decode_mma_loops_per_pass(a.d_rope);
+        for (int32_t c = 0; c < Tq && err == cudaSuccess; c += per) {
             DecodeArgs ac = a;
             ac.tq_off = c;
-            ac.Tq = Tq - c < 16 ? Tq - c : 16;
+            ac.Tq = Tq - c < per ? Tq - c : per;
             err = launch_absorb_prologue(ac, dims->dtype, s);
             if (err == cudaSuccess && c == 0)
                 err = mark(e0);
             if (err == cudaSuccess)
                 err = launch_decode_absorb_mma(ac, 0, s);
-            if (err == cudaSuccess && c + 16 >= Tq)
+            if (err == cudaSuccess && c + per >= Tq)
                 err = mark(e1);
             if (err == cudaSuccess)
                 err = window_pass(ac);

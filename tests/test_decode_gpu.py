@@ -202,3 +202,28 @@ def test_more_than_eight_loop_queries_small_ranks(Tq, t0):
     assert st == 0
     o_ref, l_ref = oracle_decode(p, w, 0, t0, Tq, 1.0)
     assert_attn_close(out, lse, o_ref, l_ref)
+
+
+@pytest.mark.parametrize("T,Tq,t0", [(24, 20, 2), (32, 32, 0), (40, 37, 1)])
+def test_two_row_tiles_in_one_latent_pass_small_ranks(T, Tq, t0):
+    """17 to 32 loop queries fill two m16 row tiles that share each staged latent tile (one
+    read of the latents); 37 queries take a second pass of 5."""
+    w = S.shrink(S.WORKLOADS["ouro1.4b-layer"], name=f"T{T}", T=T, L=1, B=5, len_lo=60, len_hi=1700)
+    p = S.decode_inputs(w, 0, "cuda", Tq=Tq)
+    out, lse, st = run_decode(p, w, 0, t0, Tq, 1.0)
+    assert st == 0
+    o_ref, l_ref = oracle_decode(p, w, 0, t0, Tq, 1.0)
+    assert_attn_close(out, lse, o_ref, l_ref)
+
+
+def test_two_row_tiles_big_ranks_ragged():
+    """Ranks 96/160 (64-token tiles, two consumer warps per row tile), 17 loop queries and
+    ragged contexts including empty and one-token sequences."""
+    lens = [0, 1, 63, 64, 65, 700, 1500]
+    w = S.shrink(S.WORKLOADS["deep-T32"], name="T32-ragged", L=1, B=len(lens))
+    p = S.decode_inputs(w, 0, "cuda", Tq=17, lens=lens, gap=2)
+    out, lse, st = run_decode(p, w, 0, 9, 17, 1.0)
+    assert st == 0
+    o_ref, l_ref = oracle_decode(p, w, 0, 9, 17, 1.0)
+    assert_attn_close(out, lse, o_ref, l_ref)
+    assert torch.all(out[0] == 0) and torch.all(torch.isneginf(lse[0]))
