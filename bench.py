@@ -74,6 +74,9 @@ def parse():
     ap.add_argument("--window", type=int, default=0,
                     help="hybrid form: W exact window rows per sequence (all in use) besides the "
                          "latents; 0 = latents only")
+    ap.add_argument("--layers", type=int, default=0,
+                    help="layers one decode step reads (0: every layer of the workload -- a whole-model "
+                         "step; the rotary, decoupled and window forms read the first layer only)")
     ap.add_argument("--model-order", action="store_true",
                     help="one decode call per loop (Tq = 1, t = 0..T-1) instead of all loops fused")
     return ap.parse_args()
@@ -276,8 +279,10 @@ def run_encode_phase(args, dev):
     w = S.WORKLOADS[args.workload]
     n_seq = args.encode_seqs or w.B
     n_tok = n_seq * w.len_hi
-    layer = w.L - 1
-    p = S.decode_inputs(w, layer, dev, lens=[1], Tq=1)
+    # layers encoded per step (a prefill writes every layer's latents): one call covers them all
+    nl = min(args.layers, w.L) if args.layers > 0 else w.L
+    layers = list(range(nl))
+    p = S.decode_inputs(w, layers, dev, lens=[1], Tq=1)
     dims = lla.make_dims(w.T, w.L, w.H, w.d, w.r_k, w.r_v, int(w.fold2d),
                          lla.F32 if w.dtype == "f32" else lla.BF16)
     bias_k = torch.zeros(w.L, w.heads_stored, w.r_k, device=dev)
@@ -288,13 +293,16 @@ def run_encode_phase(args, dev):
     ck = torch.empty(w.L, w.heads_stored, n_tok, w.r_k, dtype=w.torch_dtype, device=dev)
     cv = torch.empty(w.L, w.heads_stored, n_tok, w.r_v, dtype=w.torch_dtype, device=dev)
     cache = lla.make_cache(ck, cv, n_tok)
-    xk = S.draw_encode_tokens(w, layer, "k", n_tok, dev)
-    xv = S.draw_encode_tokens(w, layer, "v", n_tok, dev)
+    xk = torch.empty(nl, n_tok, w.T, w.H, w.d, dtype=w.torch_dtype, device=dev)
+    xv = torch.empty_like(xk)
+    for l in layers:  # drawn layer by layer into place (no stacked copy)
+        xk[l].copy_(S.draw_encode_tokens(w, l, "k", n_tok, dev))
+        xv[l].copy_(S.draw_encode_tokens(w, l, "v", n_tok, dev))
     slot_idx = torch.arange(n_tok, device=dev)
     stream = torch.cuda.current_stream(dev)
 
     def step():
-        lla.encode(dims, layer, 1, xk, xv, n_tok, slot_idx, codec, cache, stream=stream)
+        lla.encode(dims, 0, nl, xk, xv, n_tok, slot_idx, codec, cache, stream=stream)
 
     for _ in range(args.warmup):
         step()
@@ -312,18 +320,18 @@ def run_encode_phase(args, dev):
     assert lla.status_fetch(None) == 0
     ms = e0.elapsed_time(e1) / args.steps
     e = w.elem_bytes
-    bytes_moved = 2 * n_tok * w.H * w.T * w.d * e + n_tok * w.heads_stored * (w.r_k + w.r_v) * e
-    flops = 2.0 * n_tok * w.heads_stored * w.W * (w.r_k + w.r_v)
+    bytes_moved = nl * (2 * n_tok * w.H * w.T * w.d * e + n_tok * w.heads_stored * (w.r_k + w.r_v) * e)
+    flops = 2.0 * nl * n_tok * w.heads_stored * w.W * (w.r_k + w.r_v)
     peaks, kind = measured_peaks()
     gbs = bytes_moved / (ms * 1e-3) / 1e9
     tfl = flops / (ms * 1e-3) / 1e12
     print(json.dumps({
-        "metric": "LLA prefill encode GB/s (one layer, K and V)", "value": gbs, "unit": "GB/s",
+        "metric": "LLA prefill encode GB/s (K and V of every layer)", "value": gbs, "unit": "GB/s",
         "n_gpus": 1, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
         "higher_is_better": True, "dtype": "bf16 x bf16 -> f32" if w.dtype == "bf16" else "f32",
         "data": "synthetic",
-        "config": {"workload": w.name, "tokens": n_tok, "H": w.H, "T": w.T, "d": w.d, "r_k": w.r_k,
-                   "r_v": w.r_v, "fold2d": w.fold2d},
+        "config": {"workload": w.name, "tokens": n_tok, "layers": nl, "H": w.H, "T": w.T, "d": w.d,
+                   "r_k": w.r_k, "r_v": w.r_v, "rho": rho_label(w), "fold2d": w.fold2d},
         "roofline": {"bound": "hbm", "achieved": gbs, "peak": float(peaks["hbm_gbs"]), "unit": "GB/s",
                      "frac": gbs / float(peaks["hbm_gbs"]), "peak_kind": kind},
         "tensor": {"achieved_tflops": tfl, "peak_tflops": float(peaks.get("bf16_tflops", 1590.0)),
@@ -496,7 +504,11 @@ def main():
         return
     w = S.WORKLOADS[args.workload]
     Tq = w.T
-    p = S.decode_inputs(w, 0, dev, gap=1)          # one free slot per sequence for the new token
+    # layers a step reads: a whole-model decode step walks every layer of the workload
+    one_layer = bool(args.rope or args.decoupled or args.window)
+    nl = 1 if one_layer else (min(args.layers, w.L) if args.layers > 0 else w.L)
+    layers = list(range(nl))
+    p = S.decode_inputs(w, layers, dev, gap=1)     # one free slot per sequence for the new token
     dims = lla.make_dims(w.T, w.L, w.H, w.d, w.r_k, w.r_v, int(w.fold2d),
                          lla.F32 if w.dtype == "f32" else lla.BF16)
     B, H = w.B, w.H
@@ -512,10 +524,13 @@ def main():
     # independent cache replicas, rotated per step so that no step finds latents in L2: at
     # least enough that the replicas together span twice the 126 MB L2 (small planes, such
     # as the LLA-2D layer's 25 MB, need more than the default 3)
-    plane_bytes = (p["k"][0].numel() + p["v"][0].numel()) * p["k"].element_size()  # the layer a step reads
-    R = max(1, args.replicas, math.ceil(2 * L2_BYTES / max(plane_bytes, 1)) if args.replicas > 1 else 1)
-    # (a step reads layer 0 only, so the extra replicas hold that layer alone)
-    reps = [(p["k"], p["v"])] + [(p["k"][:1].clone(), p["v"][:1].clone()) for _ in range(R - 1)]
+    plane_bytes = (p["k"][0].numel() + p["v"][0].numel()) * p["k"].element_size()  # one layer's latents
+    step_plane_bytes = nl * plane_bytes                                           # what a step reads
+    R = max(1, args.replicas, math.ceil(2 * L2_BYTES / max(step_plane_bytes, 1)) if args.replicas > 1 else 1)
+    if nl > 1 and step_plane_bytes >= 2 * L2_BYTES:
+        R = 1  # a whole-model step streams far more than L2 holds: no replica needed
+    # (the extra replicas hold the layers a step reads)
+    reps = [(p["k"], p["v"])] + [(p["k"][:nl].clone(), p["v"][:nl].clone()) for _ in range(R - 1)]
     caches = [lla.make_cache(k, v, p["slots"]) for k, v in reps]
     # hybrid form: every sequence holds a full window of W exact rows (steady state)
     Wn = max(0, args.window)
@@ -525,8 +540,9 @@ def main():
         wreps = [(win["win_k"], win["win_v"])] + [(win["win_k"].clone(), win["win_v"].clone())
                                                   for _ in range(R - 1)]
         windows = [lla.make_window(k, v, win["win_len"], Wn, B) for k, v in wreps]
-    x_k = S.draw_encode_tokens(w, 0, "k", B, dev, seed_tag="new")
-    x_v = S.draw_encode_tokens(w, 0, "v", B, dev, seed_tag="new")
+    # the finished tokens' stacked K/V of every layer the step reads: [layers][B][T][H][d]
+    x_k = torch.stack([S.draw_encode_tokens(w, l, "k", B, dev, seed_tag="new") for l in layers])
+    x_v = torch.stack([S.draw_encode_tokens(w, l, "v", B, dev, seed_tag="new") for l in layers])
     new_slot = (p["seq_start"] + p["ctx_lens"].to(torch.int64)).contiguous()
     if args.rope:
         args.variant = "reconstruct"
@@ -536,7 +552,8 @@ def main():
     # decode calls of one step: all T loop queries fused (t0 = 0, Tq = T), or in model
     # order one call per loop (t0 = t, Tq = 1) with each loop's queries and outputs in
     # buffers of their own
-    calls = [(t, 1) for t in range(w.T)] if args.model_order else [(0, w.T)]
+    loop_calls = [(t, 1) for t in range(w.T)] if args.model_order else [(0, w.T)]
+    calls = [(l, t0, n) for l in layers for t0, n in loop_calls]  # (layer, t0, Tq) per decode call
     # decoupled rotary sub-key planes (drawn unrotated: rotation does not change the timing)
     DRn = max(0, args.decoupled)
     if DRn:
@@ -544,12 +561,15 @@ def main():
         kr0 = S.rope_subkeys(w, 0, p["slots"], DRn, dev).to(w.torch_dtype).unsqueeze(0)
         k_ropes = [kr0] + [kr0.clone() for _ in range(R - 1)]
         q_rope = S.rope_queries(w, B, w.T, DRn, dev)
-        q_ropes = [q_rope[:, t0:t0 + n].contiguous() for t0, n in calls]
-    Tq_call = calls[0][1]
+        q_ropes = [q_rope[:, t0:t0 + n].contiguous() for _, t0, n in calls]
+    Tq_call = calls[0][2]
     q_full = p["q"]
-    qs = [q_full[:, t0:t0 + n].contiguous() for t0, n in calls]
-    outs = [torch.empty(B, n, H, w.d, dtype=torch.float32, device=dev) for _, n in calls]
-    lses = [torch.empty(B, n, H, dtype=torch.float32, device=dev) for _, n in calls]
+    # each layer's queries (the first layer's are the drawn inputs' own)
+    q_layers = [q_full] + [S.draw_queries(B, w.T, H, w.d, S.seed_of(w.name, "q", l), dev, w.torch_dtype)
+                           for l in layers[1:]]
+    qs = [q_layers[l][:, t0:t0 + n].contiguous() for l, t0, n in calls]
+    outs = [torch.empty(B, n, H, w.d, dtype=torch.float32, device=dev) for _, _, n in calls]
+    lses = [torch.empty(B, n, H, dtype=torch.float32, device=dev) for _, _, n in calls]
     q, out, lse = q_full, outs[0], lses[0]
     if DRn:
         ws_bytes = lla.decode_decoupled_workspace_bytes(dims, B, Tq_call, max_ctx, DRn, args.num_splits)
@@ -561,32 +581,32 @@ def main():
     splits = lla.decode_num_splits(dims, B, Tq_call, max_ctx, variant, args.num_splits)
 
     def decode(i, q_in=None, out_buf=None, lse_buf=None):
-        for c, (t0, n) in enumerate(calls):
+        for c, (layer, t0, n) in enumerate(calls):
             if DRn:
-                lla.decode_attn_decoupled(dims, 0, t0, n, (q_in or qs)[c], caches[i % R], p["seq_start"],
+                lla.decode_attn_decoupled(dims, layer, t0, n, (q_in or qs)[c], caches[i % R], p["seq_start"],
                                           p["ctx_lens"], B, max_ctx, codec, k_ropes[i % R],
                                           q_ropes[c], DRn,
                                           rope, 1.0, (out_buf or outs)[c], (lse_buf or lses)[c], ws, ws_bytes,
                                           num_splits=args.num_splits, stream=stream)
                 continue
             if rope is not None:
-                lla.decode_attn_rope(dims, 0, t0, n, (q_in or qs)[c], caches[i % R], p["seq_start"],
+                lla.decode_attn_rope(dims, layer, t0, n, (q_in or qs)[c], caches[i % R], p["seq_start"],
                                      p["ctx_lens"], B, max_ctx, codec, rope, 1.0, (out_buf or outs)[c],
                                      (lse_buf or lses)[c], ws, ws_bytes, num_splits=args.num_splits,
                                      stream=stream)
                 continue
             if Wn:
-                lla.decode_attn_hybrid(dims, 0, t0, n, (q_in or qs)[c], caches[i % R], p["seq_start"],
+                lla.decode_attn_hybrid(dims, layer, t0, n, (q_in or qs)[c], caches[i % R], p["seq_start"],
                                        p["ctx_lens"], B, max_ctx, codec, windows[i % R], 1.0,
                                        (out_buf or outs)[c], (lse_buf or lses)[c], ws, ws_bytes,
                                        variant=variant, num_splits=args.num_splits, stream=stream)
                 continue
-            lla.decode_attn(dims, 0, t0, n, (q_in or qs)[c], caches[i % R], p["seq_start"], p["ctx_lens"], B,
+            lla.decode_attn(dims, layer, t0, n, (q_in or qs)[c], caches[i % R], p["seq_start"], p["ctx_lens"], B,
                             max_ctx, codec, 1.0, (out_buf or outs)[c], (lse_buf or lses)[c], ws, ws_bytes,
                             variant=variant, num_splits=args.num_splits, stream=stream)
 
     def encode(i, xk=x_k, xv=x_v, strm=None):
-        lla.encode(dims, 0, 1, xk, xv, B, new_slot, codec, caches[i % R],
+        lla.encode(dims, 0, nl, xk, xv, B, new_slot, codec, caches[i % R],
                    stream=strm if strm is not None else stream)
 
     # The encode of the finished tokens writes each sequence's next slot, which no decode
@@ -645,7 +665,7 @@ def main():
     step_bytes += len(calls) * S_tot * w.heads_stored * DRn * w.elem_bytes
     ms_step = ms_total / args.steps
     value = world * step_bytes / (ms_step * 1e-3) / 1e9
-    reads = world * S_tot * Tq / (ms_step * 1e-3)       # (token, layer, loop) reads per second
+    reads = world * S_tot * Tq * nl / (ms_step * 1e-3)  # (token, layer, loop) reads per second
     peaks, peak_kind = measured_peaks()
     peak = float(peaks["hbm_gbs"])
     mean_dec_ms = float(np.mean(decode_ms))
@@ -659,7 +679,7 @@ def main():
     if args.variant == "reconstruct":
         # the reconstruct form rebuilds K_hat and V_hat on tensor cores: per (token, head,
         # loop) 2 d (r_k + r_v) flop for the rebuild and 4 d for the score and the P.V sum
-        flop = S_tot * w.heads_stored * Tq * (2 * w.d * (w.r_k + w.r_v) + 4 * w.d) * (w.H if w.fold2d else 1)
+        flop = nl * S_tot * w.heads_stored * Tq * (2 * w.d * (w.r_k + w.r_v) + 4 * w.d) * (w.H if w.fold2d else 1)
         tf_peak = float(peaks.get("bf16_tflops_sustained", peaks.get("bf16_tflops", 1590.0)))
         tfl = flop / (mean_dec_ms * 1e-3) / 1e12
         roofline = {"bound": "tensor", "achieved": tfl, "peak": tf_peak, "unit": "TFLOP/s",
@@ -683,8 +703,8 @@ def main():
                 e_b.record(stream)
         torch.cuda.synchronize()
         for i, step_ev in enumerate(kev):
-            for c, (t0, n) in enumerate(calls):
-                lla.decode_attn_timed(dims, 0, t0, n, qs[c], caches[i % R], p["seq_start"], p["ctx_lens"], B,
+            for c, (layer, t0, n) in enumerate(calls):
+                lla.decode_attn_timed(dims, layer, t0, n, qs[c], caches[i % R], p["seq_start"], p["ctx_lens"], B,
                                       max_ctx, codec, 1.0, outs[c], lses[c], ws, ws_bytes, step_ev[c][0],
                                       step_ev[c][1], variant=variant, num_splits=args.num_splits, stream=stream)
             encode(i)
@@ -807,18 +827,20 @@ def main():
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": "f32", "storage_dtype": w.dtype, "data": "synthetic",
         "config": {"workload": w.name + (f"+window{Wn}" if Wn else "") + (f"+ropekey{DRn}" if DRn else ""),
-                   "T": w.T, "L_per_step": 1,
+                   "T": w.T, "L": w.L, "L_per_step": nl,
                    "H": H, "d": w.d, "window_rows": Wn, "window_bytes_per_step": win_bytes,
                    "r_k": w.r_k, "r_v": w.r_v, "rho": rho_label(w), "B": B,
                    "ctx_len": [w.len_lo, w.len_hi], "tokens": S_tot, "Tq": Tq_call, "decode_calls_per_step": len(calls),
                    "variant": args.variant + (" + rope" if args.rope else "")
                               + (f" + decoupled rotary sub-key {DRn}" if DRn else ""), "seg_max": splits,
-                   "step": (f"{len(calls)} x decode_attn(Tq = 1, one loop each, model order)"
-                            if args.model_order else f"decode_attn(all {w.T} loop queries fused)")
-                           + (f" with {Wn} exact window rows per sequence (decode_attn_hybrid)" if Wn else "")
-                           + " + encode(B new tokens)",
-                   "l2": f"{R} rotating cache replicas; the layer read per step is {plane_bytes / 1e6:.0f} MB "
-                         f"({R * plane_bytes / 1e6:.0f} MB together, L2 is 126 MB); "
+                   "step": (f"{nl} layer(s) x "
+                            + (f"{len(loop_calls)} x decode_attn(Tq = 1, one loop each, model order)"
+                               if args.model_order else f"decode_attn(all {w.T} loop queries fused)")
+                            + (f" with {Wn} exact window rows per sequence (decode_attn_hybrid)" if Wn else "")
+                            + f" + encode(B new tokens, {nl} layer(s))"),
+                   "l2": (f"{R} rotating cache replicas" if R > 1 else "no replicas (the step streams far more than L2)")
+                         + f"; one layer's latents are {plane_bytes / 1e6:.0f} MB, a step reads {nl} layer(s) "
+                         f"({R * step_plane_bytes / 1e6:.0f} MB of replicas together, L2 is 126 MB); "
                          f"{step_bytes / 1e6:.0f} MB read per step",
                    "parallelism": f"replicas x{world}"},
         "token_loop_reads_per_s": reads,
