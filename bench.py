@@ -42,9 +42,11 @@ PROFILE_TRAFFIC = {
     "rope": os.path.join(ROOT, "profiles", "decode_reconstruct_rope.ouro1.4b-layer.json"),
 }
 KERNEL_SOURCES = {
-    "absorb": ("decode_mma.cu", "mma_common.cuh", "decode_sched.cuh", "decode.cuh", "common.cuh"),
-    "reconstruct": ("decode_reconstruct.cu", "mma_common.cuh", "decode_sched.cuh", "decode.cuh", "common.cuh"),
-    "rope": ("decode_reconstruct.cu", "mma_common.cuh", "decode_sched.cuh", "decode.cuh", "common.cuh"),
+    "absorb": ("decode_mma.cu", "mma_common.cuh", "tmap.cuh", "decode_sched.cuh", "decode.cuh", "common.cuh"),
+    "reconstruct": ("decode_recon_tc.cu", "tc_common.cuh", "mma_common.cuh", "tmap.cuh", "decode_sched.cuh",
+                    "decode.cuh", "common.cuh"),
+    "rope": ("decode_recon_tc.cu", "tc_common.cuh", "mma_common.cuh", "tmap.cuh", "decode_sched.cuh",
+             "decode.cuh", "common.cuh"),
 }
 
 
@@ -624,9 +626,14 @@ def main():
             ev_b.record(stream)
         stream.wait_stream(s_enc)
 
-    # per decode call: prologue + decode + combine (reconstruct: one decode pass per loop
-    # query + combine); the encode of K and V is one launch
-    per_call = (3 if args.variant == "absorb" else Tq_call + 1) + (1 if Wn else 0)  # + window pass
+    # per decode call: prologue + decode + combine for each pass over the latents (32 loop
+    # queries per pass, 16 with a rotary sub-key, 64 / H for LLA-2D), reconstruct: one decode
+    # pass per 4 loop queries + combine; + the window pass; the encode of K and V is one launch
+    if args.variant == "absorb":
+        per_pass = 16 if DRn else (max(1, 64 // w.H) if w.fold2d else 32)
+        per_call = 3 * -(-Tq_call // per_pass) + (1 if Wn else 0)
+    else:
+        per_call = -(-Tq_call // 4) + 1 + (1 if Wn else 0)
     launches_per_step = per_call * len(calls) + 1
     # ---- warm-up, then the device-timed region ------------------------------------------------
     sampler = ClockSampler(local).start()
@@ -685,7 +692,7 @@ def main():
         roofline = {"bound": "tensor", "achieved": tfl, "peak": tf_peak, "unit": "TFLOP/s",
                     "frac": tfl / tf_peak, "peak_kind": peak_kind + " (sustained bf16)",
                     "traffic": profiled_traffic(S_tot * w.heads_stored, "rope" if args.rope else args.variant),
-                    "timed": "one decode call (one reconstruct pass per loop query + combine), "
+                    "timed": "one decode call (one reconstruct pass per 4 loop queries + combine), "
                              "CUDA events per call on the launch stream",
                     "algorithmic_flop_per_step": flop, "hbm_gbs": achieved, "hbm_frac": achieved / peak}
 

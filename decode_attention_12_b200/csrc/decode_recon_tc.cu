@@ -18,17 +18,20 @@
 // (unit, loop) -- with rotation the key's mean turns with the key, so there K_hat takes
 // mu_t^K from one more MMA (a ones column against mu's hi/lo parts).
 //
-// Two warpgroups of 4 warps take alternate steps, each with its own K_hat and V_hat^T
+// Two groups of 8 warps take alternate steps, each with its own K_hat and V_hat^T
 // buffers (4 x 128 of the 512 tensor-memory columns), so one group's scores overlap the
-// other's output sums and the tensor cores' next rebuild.  Within a group, thread r:
-//   * reads token row r of K_hat (its score is a d-long dot product in registers, packed
-//     fp32x2 FMAs, several independent chains), keeps a warp-local running max per loop
-//     (lazy rescale) and writes p to shared memory;
-//   * after the group's barrier reads row r of V_hat^T -- the d-index r of every token --
-//     and forms the 32-token partial sums sum_n p_n v_hat_n[r] of each warp's tokens,
-//     folded into per-warp output sums with the warps' rescale factors.
-// Records (acc, m, l) are merged across the 8 warps at segment ends and have the layout
-// of the other reconstruct kernels, so the combine is shared.
+// other's output sums and the tensor cores' next rebuild.  Tensor memory is read in
+// 16-lane x 256-bit fragments: each warp of a group owns a 16-row block of the buffers,
+// and its lane holds two rows (rq and rq + 8 of the block, rq = lane / 4) and a quarter of
+// their columns, so each shared-memory operand a lane loads serves two rows and a row's
+// dot product closes over the 4 lanes of a quad.  Per step a warp:
+//   * forms the scores of its 16 token rows of K_hat against the loop's query, picks a
+//     warp reference (the group's running max, or its own max when that is more than a
+//     lazy-rescale margin higher) and writes p to shared memory;
+//   * after the group's barrier reconciles the 8 warps' references and reads its 16
+//     d-rows of V_hat^T, forming sum_n p_n v_hat_n[d] over all 128 tokens of the tile.
+// Records (acc, m, l) are merged across the two groups at segment ends and have the
+// layout of the other reconstruct kernels, so the combine is shared.
 //
 // Faithful read: a query at position p and the rebuilt key of token n = n0 + r (tile row
 // r) give <R(p) q, R(n) k> = <R(p - n0) q, R(r) k>: each group turns the query once per

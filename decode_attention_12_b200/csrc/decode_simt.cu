@@ -570,8 +570,16 @@ template <int RG, int SPEC> struct RecBatch {
 // REC: records carry d-wide outputs of the reconstruct form (mu and the q.mu_t^K score term
 // already included), so the output is the merged record itself.  RG = record width / 128,
 // rounded up.  WIN: hybrid form, merge the window part (a.win_part) as well.
+// Resident CTAs per SM the registers are sized for: 4 (64 registers) only for the plain
+// bf16 form; wide record batches, the window merge and fp32 inputs get 2 (128 registers)
+// so that nothing spills -- their grids (H x Tq x B / 8 CTAs) are far below 2 per SM anyway.
+template <typename T, bool WIN, int RG, int SPEC> constexpr int combine_min_blocks()
+{
+    return RG == 1 && !WIN && SPEC == kSpecRecords && sizeof(T) == 2 ? 4 : 2;
+}
+
 template <typename T, typename O, bool REC, int RG, bool WIN, int SPEC>
-__global__ void __launch_bounds__(kCombineThreads, RG == 1 && !WIN && SPEC == kSpecRecords ? 4 : RG == 1 ? 3 : 2)
+__global__ void __launch_bounds__(kCombineThreads, (combine_min_blocks<T, WIN, RG, SPEC>()))
     decode_combine_kernel(const DecodeArgs a)
 {
     extern __shared__ __align__(16) float csm[];
