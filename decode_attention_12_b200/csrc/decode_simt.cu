@@ -347,100 +347,122 @@ cudaError_t launch_tq(const DecodeArgs &a, int ctas, cudaStream_t stream)
 
 // ---------------------------------------------------------------------------------
 // a1: q_tilde[u][tq_off + t][j] = scale * log2(e) * sum_k q[b][t][h][k] W_up,t^K[j][k]
-// Batched per (head, loop query, chunk of 32 sequences): the loop's W_up,t^K slice of
-// the head (r_k x d, LLA-2D: head h's columns) is staged in shared memory once and
-// serves all 32 sequences.  Thread (sequence, j) runs a d-long dot product.
+// One CTA per (head h, loop query t, chunk of 8 sequences).  Lane l of a warp owns the
+// components k = 128 c + 4 l .. + 3 of the reduction axis: the 8 query rows sit in its
+// registers and each W_up,t^K row (r_k rows, LLA-2D: head h's columns) is read from
+// global memory once per CTA as coalesced 16-byte loads, a warp taking every 8th row.
+// A row's 8 partial sums are closed across the warp by recursive halving (9 shuffles),
+// leaving sequence lane / 4's sum in lanes 4 (lane / 4) .. + 3.  d is covered in
+// passes of 256 components; the results gather in shared memory and leave as whole
+// q_tilde rows.
 // ---------------------------------------------------------------------------------
-// Copy a rows x cols fp32 matrix (16-byte aligned rows of stride src_ld floats) into
-// shared memory (row stride dst_ld) with all of a thread's loads issued before its stores.
-template <int NT>
-__device__ __forceinline__ void stage_f32(float *dst, int dst_ld, const float *src, int64_t src_ld, int rows, int cols)
+constexpr int kBatchSeqs = 8;    // sequences per combine CTA (one warp each)
+constexpr int kPrologueSeqs = 8; // sequences per prologue CTA (the 8 partial sums of a lane)
+constexpr int kPrologueThreads = 256;
+constexpr int kPrologueWarps = kPrologueThreads / 32;
+constexpr int kProloguePass = 256; // components of the reduction axis per pass (2 x 128)
+
+// Sum over the warp of s[0..7] (one partial per sequence): returns the total of sequence
+// lane / 4 (the same in the 4 lanes of a quad).
+__device__ __forceinline__ float warp_sum8(float (&s)[8], int lane)
 {
-    const int c4 = cols >> 2, n = rows * c4;
-    for (int base = threadIdx.x; base < n; base += 4 * NT) {
-        float4 v[4];
+    const bool b4 = lane & 16, b3 = lane & 8, b2 = lane & 4;
+    float h4[4], h2[2];
 #pragma unroll
-        for (int u = 0; u < 4; ++u) {
-            const int e = base + u * NT;
-            if (e < n) {
-                const int r = e / c4, c = e - r * c4;
-                v[u] = *reinterpret_cast<const float4 *>(src + r * src_ld + 4 * c);
-            }
-        }
-#pragma unroll
-        for (int u = 0; u < 4; ++u) {
-            const int e = base + u * NT;
-            if (e < n) {
-                const int r = e / c4, c = e - r * c4;
-                float *o = dst + r * dst_ld + 4 * c;
-                o[0] = v[u].x, o[1] = v[u].y, o[2] = v[u].z, o[3] = v[u].w;
-            }
-        }
+    for (int i = 0; i < 4; ++i) { // keep sequences 4 b4 + i, hand over the other half
+        const float keep = b4 ? s[i + 4] : s[i], give = b4 ? s[i] : s[i + 4];
+        h4[i] = keep + __shfl_xor_sync(0xffffffffu, give, 16);
     }
+#pragma unroll
+    for (int i = 0; i < 2; ++i) {
+        const float keep = b3 ? h4[i + 2] : h4[i], give = b3 ? h4[i] : h4[i + 2];
+        h2[i] = keep + __shfl_xor_sync(0xffffffffu, give, 8);
+    }
+    float v = (b2 ? h2[1] : h2[0]) + __shfl_xor_sync(0xffffffffu, b2 ? h2[0] : h2[1], 4);
+    v += __shfl_xor_sync(0xffffffffu, v, 2);
+    return v + __shfl_xor_sync(0xffffffffu, v, 1);
 }
 
-constexpr int kBatchSeqs = 8;    // sequences per combine CTA (one warp each)
-constexpr int kPrologueSeqs = 8; // sequences per prologue CTA
-constexpr int kPrologueThreads = 128;
+// 4 consecutive query components as floats (bf16: one 8-byte load; fp32: one 16-byte load)
+template <typename T> __device__ __forceinline__ float4 load4(const T *p);
+template <> __device__ __forceinline__ float4 load4<float>(const float *p)
+{
+    return *reinterpret_cast<const float4 *>(p);
+}
+template <> __device__ __forceinline__ float4 load4<__nv_bfloat16>(const __nv_bfloat16 *p)
+{
+    const uint2 u = *reinterpret_cast<const uint2 *>(p);
+    return make_float4(bf16_lo(u.x), bf16_hi(u.x), bf16_lo(u.y), bf16_hi(u.y));
+}
+
+__device__ __forceinline__ float dot4(float4 a, float4 b, float s)
+{
+    return fmaf(a.x, b.x, fmaf(a.y, b.y, fmaf(a.z, b.z, fmaf(a.w, b.w, s))));
+}
 
 // ROPEQ: also append the rotated rotary query part (decoupled sub-key form).
 template <typename T, bool ROPEQ>
 __global__ void __launch_bounds__(kPrologueThreads) absorb_prologue_kernel(const DecodeArgs a)
 {
-    extern __shared__ float psm[];
-    grid_launch_dependents(); // the decode grid may start streaming latents right away
+    extern __shared__ float psm[]; // [kPrologueSeqs][r_k]: q_tilde rows of the chunk
+    grid_launch_dependents();      // the decode grid may start streaming latents right away
     const int h = blockIdx.x, t = blockIdx.y, b0 = blockIdx.z * kPrologueSeqs;
-    const int RK = a.r_k, d = a.d, ldw = d + 1;
-    float *W = psm;                       // [RK][d + 1]
-    float *qs = W + RK * ldw;             // [kPrologueSeqs][d]
+    const int RK = a.r_k, d = a.d;
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int tg = a.t0 + a.tq_off + t;
     const int ld = a.fold ? a.H * d : d;
     const float *wsrc = a.W_up_k + (a.fold ? (int64_t)tg * RK * ld + (int64_t)h * d
                                            : ((int64_t)h * a.T + tg) * RK * ld);
-    stage_f32<kPrologueThreads>(W, ldw, wsrc, ld, RK, d);
     const int nb = min(kPrologueSeqs, a.B - b0);
-    {
-        // query rows of the chunk, 16-byte loads (8 bf16 or 4 fp32), all issued first
-        constexpr int V = 16 / (int)sizeof(T);
-        const int dv = d / V, n = nb * dv;
-        for (int base = threadIdx.x; base < n; base += 2 * kPrologueThreads) {
-            uint4 raw[2];
+    const T *qbase = static_cast<const T *>(a.q) + ((int64_t)b0 * a.Tq_all + a.tq_off + t) * a.H * d + (int64_t)h * d;
+    const int64_t qstride = (int64_t)a.Tq_all * a.H * d; // next sequence
+    for (int k0 = 0; k0 < d; k0 += kProloguePass) {
+        // this lane's components of the pass: k0 + 128 c + 4 lane, c = 0, 1
+        float4 qv[kPrologueSeqs][2];
+        bool kin[2];
 #pragma unroll
-            for (int u = 0; u < 2; ++u) {
-                const int e = base + u * kPrologueThreads;
-                if (e < n) {
-                    const int bl = e / dv, c = e - bl * dv;
-                    raw[u] = *reinterpret_cast<const uint4 *>(
-                        static_cast<const T *>(a.q) + (((int64_t)(b0 + bl) * a.Tq_all + a.tq_off + t) * a.H + h) * d + V * c);
+        for (int c = 0; c < 2; ++c) {
+            const int k = k0 + 128 * c + 4 * lane;
+            kin[c] = k < d;
+#pragma unroll
+            for (int b = 0; b < kPrologueSeqs; ++b)
+                qv[b][c] = kin[c] && b < nb ? load4<T>(qbase + b * qstride + k) : make_float4(0.f, 0.f, 0.f, 0.f);
+        }
+        // rows j = warp, warp + 8, ...; two rows' loads in flight per step
+        for (int j0 = warp; j0 < RK; j0 += 2 * kPrologueWarps) {
+            float4 w[2][2];
+#pragma unroll
+            for (int r = 0; r < 2; ++r) {
+                const int j = j0 + r * kPrologueWarps;
+#pragma unroll
+                for (int c = 0; c < 2; ++c) {
+                    const int k = k0 + 128 * c + 4 * lane;
+                    w[r][c] = j < RK && kin[c] ? *reinterpret_cast<const float4 *>(wsrc + (int64_t)j * ld + k)
+                                               : make_float4(0.f, 0.f, 0.f, 0.f);
                 }
             }
 #pragma unroll
-            for (int u = 0; u < 2; ++u) {
-                const int e = base + u * kPrologueThreads;
-                if (e < n) {
-                    const int bl = e / dv, c = e - bl * dv;
-                    const T *vals = reinterpret_cast<const T *>(&raw[u]);
+            for (int r = 0; r < 2; ++r) {
+                const int j = j0 + r * kPrologueWarps;
+                float s[kPrologueSeqs];
 #pragma unroll
-                    for (int k = 0; k < V; ++k)
-                        qs[bl * d + V * c + k] = Elem<T>::to_f(vals[k]);
+                for (int b = 0; b < kPrologueSeqs; ++b)
+                    s[b] = dot4(qv[b][1], w[r][1], dot4(qv[b][0], w[r][0], 0.f));
+                const float tot = warp_sum8(s, lane); // uniform control flow: every lane shuffles
+                if (j < RK && (lane & 3) == 0) {
+                    float *dst = psm + (lane >> 2) * RK + j;
+                    *dst = k0 == 0 ? tot : *dst + tot; // the same lane owns (sequence, j) in every pass
                 }
             }
         }
     }
     __syncthreads();
-    for (int o = threadIdx.x; o < nb * RK; o += kPrologueThreads) {
-        const int bl = o / RK, j = o - bl * RK;
-        const float *qr = qs + bl * d;
-        const float *wr = W + j * ldw;
-        float s0 = 0.f, s1 = 0.f, s2 = 0.f, s3 = 0.f;
-        for (int k = 0; k < d; k += 4) {
-            s0 = fmaf(qr[k], wr[k], s0);
-            s1 = fmaf(qr[k + 1], wr[k + 1], s1);
-            s2 = fmaf(qr[k + 2], wr[k + 2], s2);
-            s3 = fmaf(qr[k + 3], wr[k + 3], s3);
-        }
+    const float sc = a.scale * kLog2e;
+    const int qt_ld = RK + a.d_rope;
+    for (int e = threadIdx.x; e < nb * RK; e += kPrologueThreads) {
+        const int bl = e / RK, j = e - bl * RK;
         const int64_t u = (int64_t)(b0 + bl) * a.H + h;
-        a.qt[(u * a.Tq_all + a.tq_off + t) * (RK + a.d_rope) + j] = ((s0 + s1) + (s2 + s3)) * a.scale * kLog2e;
+        a.qt[(u * a.Tq_all + a.tq_off + t) * qt_ld + j] = psm[bl * RK + j] * sc;
     }
     if (ROPEQ) {
         // decoupled rotary part: q_rope rotated at the query position, appended to q_tilde;
@@ -458,8 +480,7 @@ __global__ void __launch_bounds__(kPrologueThreads) absorb_prologue_kernel(const
             float sn, cs;
             sincosf(red, &sn, &cs);
             const int64_t u = (int64_t)b * a.H + h;
-            float *dst = a.qt + (u * a.Tq_all + a.tq_off + t) * (RK + dr) + RK;
-            const float sc = a.scale * kLog2e;
+            float *dst = a.qt + (u * a.Tq_all + a.tq_off + t) * qt_ld + RK;
             dst[ia] = (xa * cs - xb * sn) * sc;
             dst[ib] = (xa * sn + xb * cs) * sc;
         }
@@ -467,18 +488,18 @@ __global__ void __launch_bounds__(kPrologueThreads) absorb_prologue_kernel(const
 }
 
 // ---------------------------------------------------------------------------------
-// a4: cross-segment combine + output projection.  One warp per (sequence b, head h,
-// loop query t); a CTA holds 8 sequences of one (h, t) and stages W_up,t^V (r_v x d)
-// in shared memory once:
+// a4: cross-segment combine + output projection.  A CTA holds 8 sequences of one
+// (head h, loop query t); warp w merges the records of sequence b0 + w:
 //   M = max_s m_s,  L = sum_s l_s 2^(m_s - M),  o_lat = sum_s acc_s 2^(m_s - M) / L,
 //   lse = ln2 (M + log2 L) + scale * q . mu_t^K   (-inf and out = 0 for an empty context)
-//   out[b] = o_lat W_up,t^V + mu_t^V.
+// (lane c owns record columns 4c + 128 i), then the CTA projects all 8 at once:
+//   out[b] = o_lat W_up,t^V + mu_t^V,
+// W_up,t^V (r_v x d) read once into shared memory by bulk copies.
 // Latency design: everything that does not come from the decode grid (W_up,t^V,
-// mu_t^V, mu_t^K, q, ctx_lens) is fetched before the programmatic-launch wait; after
+// mu_t^V, mu_t^K, q, ctx_lens) is requested before the programmatic-launch wait; after
 // it, the unit's record count and its first kSpecRecords records are loaded in one
 // round (slots past the count lie inside the workspace and are ignored), so the
 // combine adds two dependent global-load latencies to the end of the decode.
-// Lane c owns record / output columns 4c + 128 i (16-byte groups).
 // ---------------------------------------------------------------------------------
 constexpr int kCombineThreads = 256; // 8 warps: one sequence each
 constexpr int kSpecRecords = 4;      // records fetched before the count is known
@@ -589,8 +610,14 @@ __global__ void __launch_bounds__(kCombineThreads, (combine_min_blocks<T, WIN, R
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int b = b0 + warp;
     const bool active = b < a.B;
-    float *W = csm;          // [RV][d]
-    float *muv = W + RV * d; // [d]
+    // shared memory of the projection: W_up,t^V [RV][d] | mu_t^V [d] | o_lat [8][RV + 4] |
+    // per sequence (valid, fa, fw, -) [8][4] | mbarrier of the W copy
+    const int osl = RV + 4; // row stride of o_lat: 8 rows fall in distinct 16-byte bank groups
+    float *W = csm;
+    float *muv = W + RV * d;
+    float *os = muv + d;
+    float *sq = os + kBatchSeqs * osl;
+    const uint32_t wbar = smem_u32(sq + kBatchSeqs * 4);
     const int tg = a.t0 + t;
     const int ld = a.fold ? a.H * d : d;
     const int64_t wbase = a.fold ? (int64_t)tg * RV * ld + (int64_t)h * d : ((int64_t)h * a.T + tg) * RV * ld;
@@ -599,7 +626,20 @@ __global__ void __launch_bounds__(kCombineThreads, (combine_min_blocks<T, WIN, R
 
     // ---- inputs of the call (not written by the decode grid)
     if (!REC) {
-        stage_f32<kCombineThreads>(W, d, a.W_up_v + wbase, ld, RV, d);
+        // W_up,t^V rows (d fp32 each, 16-byte aligned) come in by bulk copies issued by
+        // warp 0; they land while the records are merged
+        if (threadIdx.x == 0) {
+            mbar_init(wbar, 1);
+            fence_barrier_init();
+        }
+        __syncthreads();
+        if (warp == 0) {
+            if (lane == 0)
+                mbar_arrive_expect_tx(wbar, (uint32_t)(RV * d * 4));
+            __syncwarp();
+            for (int j = lane; j < RV; j += 32)
+                bulk_copy_g2s(smem_u32(W + j * d), a.W_up_v + wbase + (int64_t)j * ld, (uint32_t)(d * 4), wbar);
+        }
         for (int k = threadIdx.x; k < d; k += kCombineThreads)
             muv[k] = a.mu_v[mbase + k];
     }
@@ -630,7 +670,7 @@ __global__ void __launch_bounds__(kCombineThreads, (combine_min_blocks<T, WIN, R
     float4 wo0 = make_float4(0.f, 0.f, 0.f, 0.f);
     if (win && active) {
         wl = wrec[d];
-        if (4 * lane < d)
+        if (REC && 4 * lane < d)
             wo0 = Vec4<float>::load(wrec + 4 * lane);
     }
 
@@ -673,8 +713,8 @@ __global__ void __launch_bounds__(kCombineThreads, (combine_min_blocks<T, WIN, R
     if (active && lane == 0 && a.lse != nullptr)
         a.lse[((int64_t)b * a.Tq_all + t) * a.H + h] = lse;
 
-    O *orow = static_cast<O *>(a.out) + (((int64_t)b * a.Tq_all + t) * a.H + h) * d;
     if (REC) {
+        O *orow = static_cast<O *>(a.out) + (((int64_t)b * a.Tq_all + t) * a.H + h) * d;
         if (active) {
 #pragma unroll
             for (int g = 0; g < RG; ++g) {
@@ -689,37 +729,69 @@ __global__ void __launch_bounds__(kCombineThreads, (combine_min_blocks<T, WIN, R
         }
         return;
     }
-    __syncthreads(); // W_up,t^V and mu_t^V staged
-    if (!active)
+
+    // ---- projection out[b] = o_lat[b] W_up,t^V + mu_t^V for the CTA's 8 sequences at once:
+    // warp w owns the column groups cg = 4 (w + 8 i) + lane % 4 (4 columns each) and lane
+    // l works for sequence l / 4, so a W row's 16 columns of a warp are one shared-memory
+    // wavefront serving 8 sequences
+    const bool valid = active && L > 0.f;
+#pragma unroll
+    for (int g = 0; g < RG; ++g) {
+        const int c = 4 * lane + 128 * g;
+        if (c < RV)
+            *reinterpret_cast<float4 *>(os + warp * osl + c) = valid ? acc[g] : make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+    if (lane == 0)
+        *reinterpret_cast<float4 *>(sq + 4 * warp) = make_float4(valid ? 1.f : 0.f, fa, fw, 0.f);
+    const bool landed = mbar_wait_bounded(wbar, 0);
+    if (__syncthreads_or(!landed)) { // o_lat, flags and W all in place, or a copy never landed
+        if (threadIdx.x == 0)
+            report_status(a.status, LLA_ERR_DEVICE_TIMEOUT);
         return;
-    const bool valid = L > 0.f;
-    for (int c = 4 * lane, gi = 0; gi < kMaxOutGroups && c - 4 * lane < d; c += 128, ++gi) {
-        // every lane takes part in the shuffles; lanes past d only skip the math
-        const bool mine = c < d;
-        float4 o = valid && mine ? *reinterpret_cast<const float4 *>(muv + c) : make_float4(0.f, 0.f, 0.f, 0.f);
-        if (valid) {
-            // o_lat[j] sits in lane (j / 4) % 32, group j / 128, component j % 4
+    }
+    const int bs = lane >> 2, qd = lane & 3, sb = b0 + bs;
+    const float4 flags = *reinterpret_cast<const float4 *>(sq + 4 * bs);
+    const int ncg = d >> 2;
+    float4 o4[kMaxOutGroups];
+#pragma unroll
+    for (int i = 0; i < kMaxOutGroups; ++i)
+        o4[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (flags.x != 0.f) {
+        const float *orow = os + bs * osl;
 #pragma unroll 2
-            for (int j4 = 0; j4 < RV; j4 += 4) {
-                const int src = (j4 >> 2) & 31;
-                const float4 sel = (RG > 1 && j4 >= 128) ? acc[RG - 1] : acc[0];
-                const float ox = __shfl_sync(0xffffffffu, sel.x, src);
-                const float oy = __shfl_sync(0xffffffffu, sel.y, src);
-                const float oz = __shfl_sync(0xffffffffu, sel.z, src);
-                const float ow = __shfl_sync(0xffffffffu, sel.w, src);
-                if (mine) {
-                    const float *wr = W + j4 * d + c;
-                    o = f4_fma(ox, *reinterpret_cast<const float4 *>(wr), o);
-                    o = f4_fma(oy, *reinterpret_cast<const float4 *>(wr + d), o);
-                    o = f4_fma(oz, *reinterpret_cast<const float4 *>(wr + 2 * d), o);
-                    o = f4_fma(ow, *reinterpret_cast<const float4 *>(wr + 3 * d), o);
+        for (int j = 0; j < RV; j += 4) {
+            const float4 ov = *reinterpret_cast<const float4 *>(orow + j);
+#pragma unroll
+            for (int i = 0; i < kMaxOutGroups; ++i) {
+                const int cg = 4 * (warp + 8 * i) + qd;
+                if (cg < ncg) {
+                    const float *wc = W + j * d + 4 * cg;
+                    o4[i] = f4_fma(ov.x, *reinterpret_cast<const float4 *>(wc), o4[i]);
+                    o4[i] = f4_fma(ov.y, *reinterpret_cast<const float4 *>(wc + d), o4[i]);
+                    o4[i] = f4_fma(ov.z, *reinterpret_cast<const float4 *>(wc + 2 * d), o4[i]);
+                    o4[i] = f4_fma(ov.w, *reinterpret_cast<const float4 *>(wc + 3 * d), o4[i]);
                 }
             }
         }
-        if (win && mine)
-            o = f4_fma(fw, gi == 0 ? wo0 : Vec4<float>::load(wrec + c), f4_scale(fa, o));
-        if (mine)
+    }
+    if (sb >= a.B)
+        return;
+    O *orow = static_cast<O *>(a.out) + (((int64_t)sb * a.Tq_all + t) * a.H + h) * d;
+    const float *wrow = win ? a.win_part + (((int64_t)sb * a.H + h) * a.Tq_all + t) * part_stride(d) : nullptr;
+#pragma unroll
+    for (int i = 0; i < kMaxOutGroups; ++i) {
+        const int cg = 4 * (warp + 8 * i) + qd;
+        if (cg < ncg) {
+            const int c = 4 * cg;
+            float4 o = o4[i];
+            if (flags.x != 0.f) {
+                const float4 m = *reinterpret_cast<const float4 *>(muv + c);
+                o = make_float4(o.x + m.x, o.y + m.y, o.z + m.z, o.w + m.w);
+            }
+            if (win)
+                o = f4_fma(flags.z, Vec4<float>::load(wrow + c), f4_scale(flags.y, o));
             Vec4<O>::store(orow + c, o);
+        }
     }
 }
 
@@ -755,7 +827,7 @@ cudaError_t launch_decode_absorb(const DecodeArgs &a, int dtype, int ctas, cudaS
 cudaError_t launch_absorb_prologue(const DecodeArgs &a, int dtype, cudaStream_t stream)
 {
     dim3 grid(a.H, a.Tq, (a.B + kPrologueSeqs - 1) / kPrologueSeqs);
-    const size_t smem = sizeof(float) * ((size_t)a.r_k * (a.d + 1) + (size_t)kPrologueSeqs * a.d);
+    const size_t smem = sizeof(float) * (size_t)kPrologueSeqs * a.r_k; // q_tilde rows of the chunk
     if (smem > 200 * 1024)
         return cudaErrorInvalidValue;
     if (dtype == LLA_BF16) {
@@ -811,7 +883,10 @@ cudaError_t launch_decode_combine(const DecodeArgs &a, int dtype, int out_dtype,
     const int rv = a.recon ? a.d : a.r_v;
     if (rv > 256 || a.d > 128 * kMaxOutGroups || rv % 4 != 0 || a.d % 4 != 0)
         return cudaErrorInvalidValue; // a lane holds 16-byte groups of a record / output row
-    const size_t smem = a.recon ? 16 : sizeof(float) * ((size_t)rv * a.d + a.d);
+    // W_up,t^V + mu_t^V + o_lat rows + per-sequence flags + the copy's mbarrier
+    const size_t smem = a.recon ? 16
+                                : sizeof(float) * ((size_t)rv * a.d + a.d + (size_t)kBatchSeqs * (rv + 4) +
+                                                   4 * kBatchSeqs) + 16;
     if (smem > 200 * 1024)
         return cudaErrorInvalidValue;
     using BF = __nv_bfloat16;
