@@ -74,11 +74,6 @@ bool decode_reconstruct_supported(int dtype, int r_k, int r_v, int d);
 bool decode_mma2d_supported(int dtype, int r_k, int r_v, int fold, int H);
 int decode_mma2d_loops_per_pass(int H);
 cudaError_t launch_decode_absorb_2d(const DecodeArgs &a, cudaStream_t stream);
-// tcgen05 absorbed form for passes with many query rows per latent tile (LLA-2D r 64/128,
-// per head r 96/160 with more than 16 loop queries)
-bool decode_absorb_tc_supported(int dtype, int r_k, int r_v, int d_rope, int fold, int H, int B);
-int decode_absorb_tc_loops_per_pass(int fold, int H);
-cudaError_t launch_decode_absorb_tc(const DecodeArgs &a, cudaStream_t stream);
 cudaError_t launch_decode_reconstruct(const DecodeArgs &a, cudaStream_t stream);
 // Reconstruct form on tcgen05 tensor cores: one latent read serves up to
 // decode_recon_tc_loops_per_pass() loop queries (a.Tq per launch); d = 128, bf16.

@@ -525,29 +525,6 @@ int decode_call(const lla_dims *dims, int32_t layer, int32_t t0, int32_t Tq, con
             err = launch_decode_combine(a, dims->dtype, dims->out_dtype, s);
         return err == cudaSuccess ? LLA_OK : LLA_ERR_CUDA;
     }
-    if (variant == LLA_ABSORB && (dims->fold == LLA_FOLD_2D || Tq > 16) &&
-        decode_absorb_tc_supported(dims->dtype, dims->r_k, dims->r_v, a.d_rope, dims->fold, dims->H, B)) {
-        // tensor-memory kernel: every latent tile serves up to 64 query rows (LLA-2D: all
-        // heads of a sequence x the pass's loops; per head: up to 32 loop queries)
-        const int per = decode_absorb_tc_loops_per_pass(dims->fold, dims->H);
-        for (int32_t c = 0; c < Tq && err == cudaSuccess; c += per) {
-            DecodeArgs ac = a;
-            ac.tq_off = c;
-            ac.Tq = Tq - c < per ? Tq - c : per;
-            err = launch_absorb_prologue(ac, dims->dtype, s);
-            if (err == cudaSuccess && c == 0)
-                err = mark(e0);
-            if (err == cudaSuccess)
-                err = launch_decode_absorb_tc(ac, s);
-            if (err == cudaSuccess && c + per >= Tq)
-                err = mark(e1);
-            if (err == cudaSuccess)
-                err = window_pass(ac);
-            if (err == cudaSuccess)
-                err = launch_decode_combine(ac, dims->dtype, dims->out_dtype, s);
-        }
-        return err == cudaSuccess ? LLA_OK : LLA_ERR_CUDA;
-    }
     if (decode_mma2d_supported(dims->dtype, dims->r_k, dims->r_v, dims->fold, dims->H)) {
         // LLA-2D: all heads of a sequence share each latent tile; passes of H * loops <= 64
         // query rows
