@@ -111,14 +111,15 @@ def kernel_source_hash(variant="absorb"):
     return h.hexdigest()[:16]
 
 
-def profiled_traffic(units_per_launch, variant="absorb"):
-    """DRAM bytes per launch from the committed ncu summary, or None if stale/absent."""
+def profiled_traffic(units_per_launch, variant="absorb", workload=WORKLOAD):
+    """DRAM bytes per launch from the committed ncu summary, or None if stale, absent, or
+    captured on another workload (other ranks run other kernel instantiations)."""
     try:
         with open(PROFILE_TRAFFIC[variant]) as f:
             prof = json.load(f)
     except (OSError, ValueError):
         return None
-    if prof.get("source_hash") != kernel_source_hash(variant):
+    if prof.get("source_hash") != kernel_source_hash(variant) or prof.get("workload") != workload:
         return None
     per_unit = prof["dram_bytes_per_launch"] / prof["units_per_launch"]
     return per_unit * units_per_launch
@@ -679,7 +680,7 @@ def main():
     achieved = step_bytes / (mean_dec_ms * 1e-3) / 1e9
     roofline = {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                 "frac": achieved / peak, "peak_kind": peak_kind,
-                "traffic": profiled_traffic(S_tot * w.heads_stored, args.variant),
+                "traffic": profiled_traffic(S_tot * w.heads_stored, args.variant, w.name),
                 "timed": "one lla_decode_attn call (q_tilde prologue + decode + combine "
                          "kernels), CUDA events per call on the launch stream",
                 "algorithmic_bytes_per_launch": step_bytes}
@@ -691,7 +692,7 @@ def main():
         tfl = flop / (mean_dec_ms * 1e-3) / 1e12
         roofline = {"bound": "tensor", "achieved": tfl, "peak": tf_peak, "unit": "TFLOP/s",
                     "frac": tfl / tf_peak, "peak_kind": peak_kind + " (sustained bf16)",
-                    "traffic": profiled_traffic(S_tot * w.heads_stored, "rope" if args.rope else args.variant),
+                    "traffic": profiled_traffic(S_tot * w.heads_stored, "rope" if args.rope else args.variant, w.name),
                     "timed": "one decode call (one reconstruct pass per 4 loop queries + combine), "
                              "CUDA events per call on the launch stream",
                     "algorithmic_flop_per_step": flop, "hbm_gbs": achieved, "hbm_frac": achieved / peak}

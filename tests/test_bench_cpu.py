@@ -119,10 +119,12 @@ def test_profiled_traffic_scales_per_unit_and_rejects_stale_profiles(tmp_path, m
     import bench
     path = tmp_path / "prof.json"
     prof = {"source_hash": bench.kernel_source_hash("absorb"), "dram_bytes_per_launch": 3.0e8,
-            "units_per_launch": 1.0e6}
+            "units_per_launch": 1.0e6, "workload": bench.WORKLOAD}
     path.write_text(json.dumps(prof))
     monkeypatch.setitem(bench.PROFILE_TRAFFIC, "absorb", str(path))
     assert bench.profiled_traffic(2.0e6, "absorb") == pytest.approx(6.0e8)
+    # another workload runs another kernel instantiation: no scaled guess
+    assert bench.profiled_traffic(2.0e6, "absorb", "rho4-prefill") is None
     prof["source_hash"] = "0" * 16                            # taken on other kernel sources
     path.write_text(json.dumps(prof))
     assert bench.profiled_traffic(2.0e6, "absorb") is None
@@ -141,6 +143,8 @@ def test_committed_traffic_summaries_are_well_formed():
             prof = json.load(f)
         assert prof["units_per_launch"] > 0 and prof["dram_bytes_per_launch"] > 0
         assert len(prof["source_hash"]) == 16
+        import lla_synth
+        assert prof["workload"] in lla_synth.WORKLOADS
 
 
 def test_measured_peaks_fall_back_when_the_file_is_absent(tmp_path, monkeypatch):
