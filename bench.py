@@ -36,13 +36,13 @@ METRIC = "LLA decode latent-cache GB/s & token-loop reads/s (% of HBM roofline) 
 WORKLOAD = "ouro1.4b-layer"
 SPEC_HBM_GBS = 8000.0
 L2_BYTES = 126 * 1000 * 1000
-PROFILE_TRAFFIC = {
-    "absorb": os.path.join(ROOT, "profiles", "decode_absorb_mma.ouro1.4b-layer.json"),
-    "reconstruct": os.path.join(ROOT, "profiles", "decode_reconstruct.ouro1.4b-layer.json"),
-    "rope": os.path.join(ROOT, "profiles", "decode_reconstruct_rope.ouro1.4b-layer.json"),
-}
+# committed ncu traffic summaries: profiles/<kernel>.<workload>.json, one per (decode kernel,
+# workload) captured; the LLA-2D workloads run their own kernel
+PROFILE_KERNEL = {"absorb": "decode_absorb_mma", "absorb2d": "decode_absorb_2d", "reconstruct": "decode_reconstruct",
+                  "rope": "decode_reconstruct_rope"}
 KERNEL_SOURCES = {
     "absorb": ("decode_mma.cu", "mma_common.cuh", "tmap.cuh", "decode_sched.cuh", "decode.cuh", "common.cuh"),
+    "absorb2d": ("decode_mma2d.cu", "mma_common.cuh", "tmap.cuh", "decode_sched.cuh", "decode.cuh", "common.cuh"),
     "reconstruct": ("decode_recon_tc.cu", "tc_common.cuh", "mma_common.cuh", "tmap.cuh", "decode_sched.cuh",
                     "decode.cuh", "common.cuh"),
     "rope": ("decode_recon_tc.cu", "tc_common.cuh", "mma_common.cuh", "tmap.cuh", "decode_sched.cuh",
@@ -111,11 +111,15 @@ def kernel_source_hash(variant="absorb"):
     return h.hexdigest()[:16]
 
 
+def profile_path(variant, workload=WORKLOAD):
+    return os.path.join(ROOT, "profiles", f"{PROFILE_KERNEL[variant]}.{workload}.json")
+
+
 def profiled_traffic(units_per_launch, variant="absorb", workload=WORKLOAD):
-    """DRAM bytes per launch from the committed ncu summary, or None if stale, absent, or
-    captured on another workload (other ranks run other kernel instantiations)."""
+    """DRAM bytes per launch from the committed ncu summary of this kernel on this workload,
+    or None if stale (taken on other sources) or absent."""
     try:
-        with open(PROFILE_TRAFFIC[variant]) as f:
+        with open(profile_path(variant, workload)) as f:
             prof = json.load(f)
     except (OSError, ValueError):
         return None
@@ -680,7 +684,9 @@ def main():
     achieved = step_bytes / (mean_dec_ms * 1e-3) / 1e9
     roofline = {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                 "frac": achieved / peak, "peak_kind": peak_kind,
-                "traffic": profiled_traffic(S_tot * w.heads_stored, args.variant, w.name),
+                "traffic": profiled_traffic(S_tot * w.heads_stored,
+                                            "absorb2d" if w.fold2d and args.variant == "absorb" else args.variant,
+                                            w.name),
                 "timed": "one lla_decode_attn call (q_tilde prologue + decode + combine "
                          "kernels), CUDA events per call on the launch stream",
                 "algorithmic_bytes_per_launch": step_bytes}

@@ -121,7 +121,8 @@ def test_profiled_traffic_scales_per_unit_and_rejects_stale_profiles(tmp_path, m
     prof = {"source_hash": bench.kernel_source_hash("absorb"), "dram_bytes_per_launch": 3.0e8,
             "units_per_launch": 1.0e6, "workload": bench.WORKLOAD}
     path.write_text(json.dumps(prof))
-    monkeypatch.setitem(bench.PROFILE_TRAFFIC, "absorb", str(path))
+    monkeypatch.setattr(bench, "profile_path", lambda variant, workload=bench.WORKLOAD:
+                        str(path) if workload == bench.WORKLOAD else str(tmp_path / "none.json"))
     assert bench.profiled_traffic(2.0e6, "absorb") == pytest.approx(6.0e8)
     # another workload runs another kernel instantiation: no scaled guess
     assert bench.profiled_traffic(2.0e6, "absorb", "rho4-prefill") is None
@@ -130,21 +131,26 @@ def test_profiled_traffic_scales_per_unit_and_rejects_stale_profiles(tmp_path, m
     assert bench.profiled_traffic(2.0e6, "absorb") is None
     path.write_text("not json")
     assert bench.profiled_traffic(2.0e6, "absorb") is None
-    monkeypatch.setitem(bench.PROFILE_TRAFFIC, "absorb", str(tmp_path / "absent.json"))
+    path.unlink()
     assert bench.profiled_traffic(2.0e6, "absorb") is None
 
 
 def test_committed_traffic_summaries_are_well_formed():
     """Each committed traffic summary names the hash of the sources it was taken on; the
     bench reports traffic only while they match (otherwise null)."""
+    import glob
     import bench
-    for variant, path in bench.PROFILE_TRAFFIC.items():
+    paths = glob.glob(os.path.join(bench.ROOT, "profiles", "*.json"))
+    assert paths
+    for path in paths:
         with open(path) as f:
             prof = json.load(f)
         assert prof["units_per_launch"] > 0 and prof["dram_bytes_per_launch"] > 0
         assert len(prof["source_hash"]) == 16
         import lla_synth
         assert prof["workload"] in lla_synth.WORKLOADS
+        kernel, workload = os.path.basename(path)[:-5].split(".", 1)
+        assert kernel in bench.PROFILE_KERNEL.values() and workload == prof["workload"]
 
 
 def test_measured_peaks_fall_back_when_the_file_is_absent(tmp_path, monkeypatch):
