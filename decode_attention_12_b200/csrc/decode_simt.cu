@@ -353,14 +353,19 @@ cudaError_t launch_tq(const DecodeArgs &a, int ctas, cudaStream_t stream)
 // global memory once per CTA as coalesced 16-byte loads, a warp taking every 8th row.
 // A row's 8 partial sums are closed across the warp by recursive halving (9 shuffles),
 // leaving sequence lane / 4's sum in lanes 4 (lane / 4) .. + 3.  d is covered in
-// passes of 256 components; the results gather in shared memory and leave as whole
-// q_tilde rows.
+// passes of 128 NCH components (NCH = 1 for d <= 128, so only the registers a head needs
+// are held); the results gather in shared memory and leave as whole q_tilde rows.
 // ---------------------------------------------------------------------------------
-constexpr int kBatchSeqs = 8;    // sequences per combine CTA (one warp each)
+// sequences per combine CTA (one warp each): 16 when W_up,t^V is large enough that staging
+// it once for more sequences pays, else 8 (smaller CTAs take SM slots sooner at the
+// decode grid's tail)
+constexpr int kBatchSmall = 8, kBatchLarge = 16;
 constexpr int kPrologueSeqs = 8; // sequences per prologue CTA (the 8 partial sums of a lane)
 constexpr int kPrologueThreads = 256;
 constexpr int kPrologueWarps = kPrologueThreads / 32;
-constexpr int kProloguePass = 256; // components of the reduction axis per pass (2 x 128)
+// W rows a warp keeps in flight per step: the kernel is bound by load latency, so a warp
+// requests 8 rows (4 when a lane holds two 128-wide chunks) before it sums any of them
+template <int NCH> constexpr int prologue_rows() { return NCH == 1 ? 8 : 4; }
 
 // Sum over the warp of s[0..7] (one partial per sequence): returns the total of sequence
 // lane / 4 (the same in the 4 lanes of a quad).
@@ -401,8 +406,8 @@ __device__ __forceinline__ float dot4(float4 a, float4 b, float s)
 }
 
 // ROPEQ: also append the rotated rotary query part (decoupled sub-key form).
-template <typename T, bool ROPEQ>
-__global__ void __launch_bounds__(kPrologueThreads) absorb_prologue_kernel(const DecodeArgs a)
+template <typename T, bool ROPEQ, int NCH>
+__global__ void __launch_bounds__(kPrologueThreads, 2) absorb_prologue_kernel(const DecodeArgs a)
 {
     extern __shared__ float psm[]; // [kPrologueSeqs][r_k]: q_tilde rows of the chunk
     grid_launch_dependents();      // the decode grid may start streaming latents right away
@@ -416,40 +421,47 @@ __global__ void __launch_bounds__(kPrologueThreads) absorb_prologue_kernel(const
     const int nb = min(kPrologueSeqs, a.B - b0);
     const T *qbase = static_cast<const T *>(a.q) + ((int64_t)b0 * a.Tq_all + a.tq_off + t) * a.H * d + (int64_t)h * d;
     const int64_t qstride = (int64_t)a.Tq_all * a.H * d; // next sequence
-    for (int k0 = 0; k0 < d; k0 += kProloguePass) {
-        // this lane's components of the pass: k0 + 128 c + 4 lane, c = 0, 1
-        float4 qv[kPrologueSeqs][2];
-        bool kin[2];
+    for (int k0 = 0; k0 < d; k0 += 128 * NCH) {
+        // this lane's components of the pass: k0 + 128 c + 4 lane, c < NCH
+        float4 qv[kPrologueSeqs][NCH];
+        bool kin[NCH];
 #pragma unroll
-        for (int c = 0; c < 2; ++c) {
+        for (int c = 0; c < NCH; ++c) {
             const int k = k0 + 128 * c + 4 * lane;
             kin[c] = k < d;
 #pragma unroll
             for (int b = 0; b < kPrologueSeqs; ++b)
                 qv[b][c] = kin[c] && b < nb ? load4<T>(qbase + b * qstride + k) : make_float4(0.f, 0.f, 0.f, 0.f);
         }
-        // rows j = warp, warp + 8, ...; two rows' loads in flight per step
-        for (int j0 = warp; j0 < RK; j0 += 2 * kPrologueWarps) {
-            float4 w[2][2];
+        // rows j = warp, warp + 8, ...; R rows' loads in flight per step
+        constexpr int R = prologue_rows<NCH>();
+        for (int j0 = warp; j0 < RK; j0 += R * kPrologueWarps) {
+            float4 w[R][NCH];
 #pragma unroll
-            for (int r = 0; r < 2; ++r) {
+            for (int r = 0; r < R; ++r) {
                 const int j = j0 + r * kPrologueWarps;
 #pragma unroll
-                for (int c = 0; c < 2; ++c) {
+                for (int c = 0; c < NCH; ++c) {
                     const int k = k0 + 128 * c + 4 * lane;
                     w[r][c] = j < RK && kin[c] ? *reinterpret_cast<const float4 *>(wsrc + (int64_t)j * ld + k)
                                                : make_float4(0.f, 0.f, 0.f, 0.f);
                 }
             }
 #pragma unroll
-            for (int r = 0; r < 2; ++r) {
+            for (int r = 0; r < R; ++r) {
                 const int j = j0 + r * kPrologueWarps;
+                if (j >= RK)
+                    break; // warp-uniform: no sums (and no shuffles) for rows past r_k
                 float s[kPrologueSeqs];
 #pragma unroll
-                for (int b = 0; b < kPrologueSeqs; ++b)
-                    s[b] = dot4(qv[b][1], w[r][1], dot4(qv[b][0], w[r][0], 0.f));
+                for (int b = 0; b < kPrologueSeqs; ++b) {
+                    s[b] = 0.f;
+#pragma unroll
+                    for (int c = 0; c < NCH; ++c)
+                        s[b] = dot4(qv[b][c], w[r][c], s[b]);
+                }
                 const float tot = warp_sum8(s, lane); // uniform control flow: every lane shuffles
-                if (j < RK && (lane & 3) == 0) {
+                if ((lane & 3) == 0) {
                     float *dst = psm + (lane >> 2) * RK + j;
                     *dst = k0 == 0 ? tot : *dst + tot; // the same lane owns (sequence, j) in every pass
                 }
@@ -488,11 +500,11 @@ __global__ void __launch_bounds__(kPrologueThreads) absorb_prologue_kernel(const
 }
 
 // ---------------------------------------------------------------------------------
-// a4: cross-segment combine + output projection.  A CTA holds 8 sequences of one
+// a4: cross-segment combine + output projection.  A CTA holds NSEQ sequences of one
 // (head h, loop query t); warp w merges the records of sequence b0 + w:
 //   M = max_s m_s,  L = sum_s l_s 2^(m_s - M),  o_lat = sum_s acc_s 2^(m_s - M) / L,
 //   lse = ln2 (M + log2 L) + scale * q . mu_t^K   (-inf and out = 0 for an empty context)
-// (lane c owns record columns 4c + 128 i), then the CTA projects all 8 at once:
+// (lane c owns record columns 4c + 128 i), then the CTA projects all of them at once:
 //   out[b] = o_lat W_up,t^V + mu_t^V,
 // W_up,t^V (r_v x d) read once into shared memory by bulk copies.
 // Latency design: everything that does not come from the decode grid (W_up,t^V,
@@ -501,7 +513,7 @@ __global__ void __launch_bounds__(kPrologueThreads) absorb_prologue_kernel(const
 // round (slots past the count lie inside the workspace and are ignored), so the
 // combine adds two dependent global-load latencies to the end of the decode.
 // ---------------------------------------------------------------------------------
-constexpr int kCombineThreads = 256; // 8 warps: one sequence each
+
 constexpr int kSpecRecords = 4;      // records fetched before the count is known
 constexpr int kMaxOutGroups = 4;     // d <= 512
 
@@ -591,18 +603,19 @@ template <int RG, int SPEC> struct RecBatch {
 // REC: records carry d-wide outputs of the reconstruct form (mu and the q.mu_t^K score term
 // already included), so the output is the merged record itself.  RG = record width / 128,
 // rounded up.  WIN: hybrid form, merge the window part (a.win_part) as well.
-// Resident CTAs per SM the registers are sized for: 4 (64 registers) only for the plain
-// bf16 form; wide record batches, the window merge and fp32 inputs get 2 (128 registers)
-// so that nothing spills -- their grids (H x Tq x B / 8 CTAs) are far below 2 per SM anyway.
-template <typename T, bool WIN, int RG, int SPEC> constexpr int combine_min_blocks()
+// Registers per thread the launch bounds allow: 64 only for the plain bf16 form; wide record
+// batches, the window merge and fp32 inputs get 128 so that nothing spills -- their grids
+// (H x Tq x B / NSEQ CTAs) are far below that many CTAs per SM anyway.
+template <typename T, bool WIN, int RG, int SPEC, int NSEQ> constexpr int combine_min_blocks()
 {
-    return RG == 1 && !WIN && SPEC == kSpecRecords && sizeof(T) == 2 ? 4 : 2;
+    return (RG == 1 && !WIN && SPEC == kSpecRecords && sizeof(T) == 2 ? 2 : 1) * (NSEQ == kBatchSmall ? 2 : 1);
 }
 
-template <typename T, typename O, bool REC, int RG, bool WIN, int SPEC>
-__global__ void __launch_bounds__(kCombineThreads, (combine_min_blocks<T, WIN, RG, SPEC>()))
+template <typename T, typename O, bool REC, int RG, bool WIN, int SPEC, int NSEQ>
+__global__ void __launch_bounds__(32 * NSEQ, (combine_min_blocks<T, WIN, RG, SPEC, NSEQ>()))
     decode_combine_kernel(const DecodeArgs a)
 {
+    constexpr int kBatchSeqs = NSEQ, kCombineThreads = 32 * NSEQ;
     extern __shared__ __align__(16) float csm[];
     const int h = blockIdx.x, tl = blockIdx.y, b0 = blockIdx.z * kBatchSeqs;
     const int t = a.tq_off + tl; // indexes q / out / lse / records
@@ -730,10 +743,11 @@ __global__ void __launch_bounds__(kCombineThreads, (combine_min_blocks<T, WIN, R
         return;
     }
 
-    // ---- projection out[b] = o_lat[b] W_up,t^V + mu_t^V for the CTA's 8 sequences at once:
-    // warp w owns the column groups cg = 4 (w + 8 i) + lane % 4 (4 columns each) and lane
-    // l works for sequence l / 4, so a W row's 16 columns of a warp are one shared-memory
-    // wavefront serving 8 sequences
+    // ---- projection out[b] = o_lat[b] W_up,t^V + mu_t^V for the CTA's NSEQ sequences at
+    // once: lane l works for sequence l / (32 / NSEQ) and column group l % (32 / NSEQ) of
+    // the warp's; warp w owns the groups (32 / NSEQ) (w + NSEQ i) + l % (32 / NSEQ) (4
+    // columns each), so a W row's columns of a warp are one shared-memory wavefront
+    // serving all NSEQ sequences
     const bool valid = active && L > 0.f;
 #pragma unroll
     for (int g = 0; g < RG; ++g) {
@@ -749,7 +763,8 @@ __global__ void __launch_bounds__(kCombineThreads, (combine_min_blocks<T, WIN, R
             report_status(a.status, LLA_ERR_DEVICE_TIMEOUT);
         return;
     }
-    const int bs = lane >> 2, qd = lane & 3, sb = b0 + bs;
+    constexpr int GPL = 32 / NSEQ; // column groups per warp and W row
+    const int bs = lane / GPL, qd = lane % GPL, sb = b0 + bs;
     const float4 flags = *reinterpret_cast<const float4 *>(sq + 4 * bs);
     const int ncg = d >> 2;
     float4 o4[kMaxOutGroups];
@@ -763,7 +778,7 @@ __global__ void __launch_bounds__(kCombineThreads, (combine_min_blocks<T, WIN, R
             const float4 ov = *reinterpret_cast<const float4 *>(orow + j);
 #pragma unroll
             for (int i = 0; i < kMaxOutGroups; ++i) {
-                const int cg = 4 * (warp + 8 * i) + qd;
+                const int cg = GPL * (warp + NSEQ * i) + qd;
                 if (cg < ncg) {
                     const float *wc = W + j * d + 4 * cg;
                     o4[i] = f4_fma(ov.x, *reinterpret_cast<const float4 *>(wc), o4[i]);
@@ -780,7 +795,7 @@ __global__ void __launch_bounds__(kCombineThreads, (combine_min_blocks<T, WIN, R
     const float *wrow = win ? a.win_part + (((int64_t)sb * a.H + h) * a.Tq_all + t) * part_stride(d) : nullptr;
 #pragma unroll
     for (int i = 0; i < kMaxOutGroups; ++i) {
-        const int cg = 4 * (warp + 8 * i) + qd;
+        const int cg = GPL * (warp + NSEQ * i) + qd;
         if (cg < ncg) {
             const int c = 4 * cg;
             float4 o = o4[i];
@@ -830,32 +845,38 @@ cudaError_t launch_absorb_prologue(const DecodeArgs &a, int dtype, cudaStream_t 
     const size_t smem = sizeof(float) * (size_t)kPrologueSeqs * a.r_k; // q_tilde rows of the chunk
     if (smem > 200 * 1024)
         return cudaErrorInvalidValue;
-    if (dtype == LLA_BF16) {
-        auto k = a.d_rope > 0 ? absorb_prologue_kernel<__nv_bfloat16, true> : absorb_prologue_kernel<__nv_bfloat16, false>;
-        cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-        k<<<grid, kPrologueThreads, smem, stream>>>(a);
-    } else {
-        auto k = a.d_rope > 0 ? absorb_prologue_kernel<float, true> : absorb_prologue_kernel<float, false>;
-        cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-        k<<<grid, kPrologueThreads, smem, stream>>>(a);
-    }
+    auto pick = [&](auto tag) {
+        using T = decltype(tag);
+        if (a.d <= 128)
+            return a.d_rope > 0 ? absorb_prologue_kernel<T, true, 1> : absorb_prologue_kernel<T, false, 1>;
+        return a.d_rope > 0 ? absorb_prologue_kernel<T, true, 2> : absorb_prologue_kernel<T, false, 2>;
+    };
+    auto k = dtype == LLA_BF16 ? pick(__nv_bfloat16{}) : pick(float{});
+    cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    k<<<grid, kPrologueThreads, smem, stream>>>(a);
     return cudaGetLastError();
 }
 
-template <typename T, typename O, int RG, int SPEC>
-static cudaError_t launch_combine_t(const DecodeArgs &a, size_t smem, cudaStream_t stream)
+template <typename T, typename O, int RG, int SPEC, int NSEQ>
+static cudaError_t launch_combine_n(const DecodeArgs &a, cudaStream_t stream)
 {
+    const int rv = a.recon ? a.d : a.r_v;
+    // W_up,t^V + mu_t^V + o_lat rows + per-sequence flags + the copy's mbarrier
+    const size_t smem = a.recon ? 16
+                                : sizeof(float) * ((size_t)rv * a.d + a.d + (size_t)NSEQ * (rv + 4) + 4 * NSEQ) + 16;
+    if (smem > 200 * 1024)
+        return cudaErrorInvalidValue;
     const bool win = a.win_part != nullptr;
-    auto k = a.recon ? (win ? decode_combine_kernel<T, O, true, RG, true, SPEC>
-                            : decode_combine_kernel<T, O, true, RG, false, SPEC>)
-                     : (win ? decode_combine_kernel<T, O, false, RG, true, SPEC>
-                            : decode_combine_kernel<T, O, false, RG, false, SPEC>);
+    auto k = a.recon ? (win ? decode_combine_kernel<T, O, true, RG, true, SPEC, NSEQ>
+                            : decode_combine_kernel<T, O, true, RG, false, SPEC, NSEQ>)
+                     : (win ? decode_combine_kernel<T, O, false, RG, true, SPEC, NSEQ>
+                            : decode_combine_kernel<T, O, false, RG, false, SPEC, NSEQ>);
     cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess)
         return e;
     cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(a.H, a.Tq, (a.B + kBatchSeqs - 1) / kBatchSeqs);
-    cfg.blockDim = dim3(kCombineThreads);
+    cfg.gridDim = dim3(a.H, a.Tq, (a.B + NSEQ - 1) / NSEQ);
+    cfg.blockDim = dim3(32 * NSEQ);
     cfg.dynamicSmemBytes = smem;
     cfg.stream = stream;
     cudaLaunchAttribute attr[1];
@@ -866,16 +887,25 @@ static cudaError_t launch_combine_t(const DecodeArgs &a, size_t smem, cudaStream
     return cudaLaunchKernelEx(&cfg, k, a);
 }
 
+template <typename T, typename O, int RG, int SPEC>
+static cudaError_t launch_combine_t(const DecodeArgs &a, cudaStream_t stream)
+{
+    // a W_up,t^V of 32 KB or more is worth staging once for 16 sequences
+    const bool large = !a.recon && (size_t)a.r_v * a.d * sizeof(float) >= 32 * 1024;
+    return large ? launch_combine_n<T, O, RG, SPEC, kBatchLarge>(a, stream)
+                 : launch_combine_n<T, O, RG, SPEC, kBatchSmall>(a, stream);
+}
+
 template <typename T, typename O>
-static cudaError_t launch_combine_rg(const DecodeArgs &a, int rv, size_t smem, cudaStream_t stream)
+static cudaError_t launch_combine_rg(const DecodeArgs &a, int rv, cudaStream_t stream)
 {
     // many record slots per unit (LLA-2D's short shares, long contexts): 8 records per load
     // round instead of 4, so fewer dependent rounds; the small batch keeps the register count
     // (and the CTAs resident beside a finishing decode grid) when a unit has <= 4 records
     if (rv > 128)
-        return launch_combine_t<T, O, 2, kSpecRecords>(a, smem, stream);
-    return a.seg_max > kSpecRecords ? launch_combine_t<T, O, 1, 2 * kSpecRecords>(a, smem, stream)
-                                    : launch_combine_t<T, O, 1, kSpecRecords>(a, smem, stream);
+        return launch_combine_t<T, O, 2, kSpecRecords>(a, stream);
+    return a.seg_max > kSpecRecords ? launch_combine_t<T, O, 1, 2 * kSpecRecords>(a, stream)
+                                    : launch_combine_t<T, O, 1, kSpecRecords>(a, stream);
 }
 
 cudaError_t launch_decode_combine(const DecodeArgs &a, int dtype, int out_dtype, cudaStream_t stream)
@@ -883,20 +913,14 @@ cudaError_t launch_decode_combine(const DecodeArgs &a, int dtype, int out_dtype,
     const int rv = a.recon ? a.d : a.r_v;
     if (rv > 256 || a.d > 128 * kMaxOutGroups || rv % 4 != 0 || a.d % 4 != 0)
         return cudaErrorInvalidValue; // a lane holds 16-byte groups of a record / output row
-    // W_up,t^V + mu_t^V + o_lat rows + per-sequence flags + the copy's mbarrier
-    const size_t smem = a.recon ? 16
-                                : sizeof(float) * ((size_t)rv * a.d + a.d + (size_t)kBatchSeqs * (rv + 4) +
-                                                   4 * kBatchSeqs) + 16;
-    if (smem > 200 * 1024)
-        return cudaErrorInvalidValue;
     using BF = __nv_bfloat16;
     if (dtype == LLA_BF16 && out_dtype == LLA_BF16)
-        return launch_combine_rg<BF, BF>(a, rv, smem, stream);
+        return launch_combine_rg<BF, BF>(a, rv, stream);
     if (dtype == LLA_BF16)
-        return launch_combine_rg<BF, float>(a, rv, smem, stream);
+        return launch_combine_rg<BF, float>(a, rv, stream);
     if (out_dtype == LLA_BF16)
-        return launch_combine_rg<float, BF>(a, rv, smem, stream);
-    return launch_combine_rg<float, float>(a, rv, smem, stream);
+        return launch_combine_rg<float, BF>(a, rv, stream);
+    return launch_combine_rg<float, float>(a, rv, stream);
 }
 
 } // namespace lla
