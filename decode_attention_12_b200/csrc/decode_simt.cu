@@ -908,6 +908,20 @@ static cudaError_t launch_combine_rg(const DecodeArgs &a, int rv, cudaStream_t s
                                     : launch_combine_t<T, O, 1, kSpecRecords>(a, stream);
 }
 
+// The combine holds W_up,t^V (r_v x d fp32) in shared memory for its CTA's sequences:
+// shapes whose W does not fit are refused before anything is queued.
+bool decode_combine_supported(int r_v, int d, bool recon)
+{
+    const int rv = recon ? d : r_v;
+    if (rv > 256 || d > 128 * kMaxOutGroups || rv % 4 != 0 || d % 4 != 0)
+        return false;
+    if (recon)
+        return true;
+    const int nseq = (size_t)r_v * d * sizeof(float) >= 32 * 1024 ? kBatchLarge : kBatchSmall;
+    const size_t smem = sizeof(float) * ((size_t)rv * d + d + (size_t)nseq * (rv + 4) + 4 * nseq) + 16;
+    return smem <= 200 * 1024;
+}
+
 cudaError_t launch_decode_combine(const DecodeArgs &a, int dtype, int out_dtype, cudaStream_t stream)
 {
     const int rv = a.recon ? a.d : a.r_v;

@@ -418,7 +418,7 @@ int decode_call(const lla_dims *dims, int32_t layer, int32_t t0, int32_t Tq, con
     const bool use_mma = decode_mma_supported(dims->dtype, dims->r_k, dims->r_v, dims->fold, Tq);
     if (!use_mma && !decode_absorb_supported(dims->dtype, dims->r_k, dims->r_v, dims->d_head, dims->fold))
         return LLA_ERR_UNSUPPORTED;
-    if (B > 16384)
+    if (B > 16384 || !decode_combine_supported(dims->r_v, dims->d_head, variant == LLA_RECONSTRUCT))
         return LLA_ERR_UNSUPPORTED;
 
     const int Hs = heads_stored(dims);

@@ -211,8 +211,10 @@ int lla_codec_residual(const lla_dims *dims, int32_t layer0, int32_t n_layers, c
  *   workspace   device scratch of at least lla_decode_workspace_bytes(...) bytes; its
  *               contents need not be initialised (the first word, the status, must be
  *               zero -- lla_status_fetch leaves it so)
- * Errors: LLA_ERR_INVALID (dims, loop range, Tq < 1, pointers), LLA_ERR_UNSUPPORTED,
- * LLA_ERR_MISALIGNED, LLA_ERR_WORKSPACE, LLA_ERR_CUDA.                                  */
+ * Errors: LLA_ERR_INVALID (dims, loop range, Tq < 1, pointers), LLA_ERR_UNSUPPORTED (no
+ * kernel for the ranks / dtype, B > 16384, d_head > 512, or an absorbed-form W_up,t^V of
+ * r_v x d_head fp32 too large for the combine's shared memory -- about 190 KB; nothing is
+ * queued then), LLA_ERR_MISALIGNED, LLA_ERR_WORKSPACE, LLA_ERR_CUDA.                    */
 int lla_decode_attn(const lla_dims *dims, int32_t layer, int32_t t0, int32_t Tq,
                     const void *q, const lla_cache *cache, const int64_t *seq_start,
                     const int32_t *ctx_lens, int32_t B, int32_t max_ctx,

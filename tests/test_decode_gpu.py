@@ -227,3 +227,35 @@ def test_two_row_tiles_big_ranks_ragged():
     o_ref, l_ref = oracle_decode(p, w, 0, 9, 17, 1.0)
     assert_attn_close(out, lse, o_ref, l_ref)
     assert torch.all(out[0] == 0) and torch.all(torch.isneginf(lse[0]))
+
+
+# ---- head dimensions other than 128 ------------------------------------------------------
+@pytest.mark.parametrize("d", [64, 96, 192, 256, 512])
+@pytest.mark.parametrize("rk,rv", [(16, 32), (96, 160)])
+def test_head_dims_prologue_and_projection(d, rk, rv):
+    """The q_tilde prologue covers d in 128-wide register chunks (several passes for d > 256)
+    and the combine projects d / 4 column groups over its warps; both depend on d."""
+    w = S.shrink(S.WORKLOADS["ouro1.4b-layer"], name=f"d{d}-{rk}-{rv}", d=d, r_k=rk, r_v=rv, H=4, B=5,
+                 len_lo=60, len_hi=700)
+    p = S.decode_inputs(w, 0, DEV)
+    scale = 1.0 / np.sqrt(d)
+    if rv * d * 4 > 190 * 1024:  # W_up,t^V too large for the combine: refused, nothing queued
+        with pytest.raises(lla.LLAError) as e:
+            run_decode(p, w, 0, 0, 4, scale)
+        assert e.value.code == lla.LLA_ERR_UNSUPPORTED
+        return
+    out, lse, st = run_decode(p, w, 0, 0, 4, scale)
+    assert st == 0
+    o_ref, l_ref = oracle_decode(p, w, 0, 0, 4, scale)
+    assert_attn_close(out, lse, o_ref, l_ref)
+
+
+def test_head_dim_256_deep_loops_sixteen_sequence_combine():
+    """32 loop queries (two row tiles) at d = 256: W_up,t^V of 160 KB, staged once per 16
+    sequences by the combine; 17 sequences so a second, partial combine CTA exists."""
+    w = S.shrink(S.WORKLOADS["deep-T32"], name="d256-T32", d=256, H=2, L=1, B=17, len_lo=40, len_hi=600)
+    p = S.decode_inputs(w, 0, DEV, Tq=32)
+    out, lse, st = run_decode(p, w, 0, 0, 32, 1.0 / 16)
+    assert st == 0
+    o_ref, l_ref = oracle_decode(p, w, 0, 0, 32, 1.0 / 16)
+    assert_attn_close(out, lse, o_ref, l_ref)
