@@ -650,8 +650,18 @@ __global__ void __launch_bounds__(32 * NSEQ, (combine_min_blocks<T, WIN, RG, SPE
             if (lane == 0)
                 mbar_arrive_expect_tx(wbar, (uint32_t)(RV * d * 4));
             __syncwarp();
-            for (int j = lane; j < RV; j += 32)
-                bulk_copy_g2s(smem_u32(W + j * d), a.W_up_v + wbase + (int64_t)j * ld, (uint32_t)(d * 4), wbar);
+            if (!a.fold) {
+                // per-head layout: the (head, loop) block is contiguous -- a few large copies
+                constexpr uint32_t kPiece = 64 * 1024;
+                const uint32_t total = (uint32_t)(RV * d * 4);
+                for (uint32_t o = (uint32_t)lane * kPiece; o < total; o += 32u * kPiece)
+                    bulk_copy_g2s(smem_u32(W) + o, reinterpret_cast<const uint8_t *>(a.W_up_v + wbase) + o,
+                                  total - o < kPiece ? total - o : kPiece, wbar);
+            } else {
+                // LLA-2D: head h's d columns of each folded row
+                for (int j = lane; j < RV; j += 32)
+                    bulk_copy_g2s(smem_u32(W + j * d), a.W_up_v + wbase + (int64_t)j * ld, (uint32_t)(d * 4), wbar);
+            }
         }
         for (int k = threadIdx.x; k < d; k += kCombineThreads)
             muv[k] = a.mu_v[mbase + k];
