@@ -130,6 +130,8 @@ def test_decode_argument_errors():
     assert _rc(dims=lla.make_dims(4, 1, 16, 128, 0, 32)) == lla.LLA_ERR_INVALID
     assert _rc(dims=lla.make_dims(4, 1, 16, 128, 12, 32)) == lla.LLA_ERR_UNSUPPORTED  # 24 B rows
     assert _rc(dims=lla.make_dims(4, 1, 16, 128, 16, 32, 0, 5)) == lla.LLA_ERR_INVALID
+    # d_head above the combine's 512 columns: refused before anything is queued
+    assert _rc(dims=lla.make_dims(4, 1, 16, 1024, 16, 32)) == lla.LLA_ERR_UNSUPPORTED
     assert _rc(B=0) == 0  # nothing to do, nothing launched
 
 
