@@ -60,7 +60,6 @@ constexpr int kDecodeCtasPerSm = 4;
 cudaError_t launch_decode_absorb(const DecodeArgs &a, int dtype, int ctas, cudaStream_t stream,
                                  bool *supported);
 cudaError_t launch_absorb_prologue(const DecodeArgs &a, int dtype, cudaStream_t stream);
-bool decode_combine_supported(int r_v, int d, bool recon);
 cudaError_t launch_decode_combine(const DecodeArgs &a, int dtype, int out_dtype, cudaStream_t stream);
 bool decode_absorb_supported(int dtype, int r_k, int r_v, int d, int fold);
 bool decode_mma_supported(int dtype, int r_k, int r_v, int fold, int Tq);

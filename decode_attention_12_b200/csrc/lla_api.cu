@@ -9,6 +9,11 @@
 #include "decode.cuh"
 #include "encode.cuh"
 
+namespace lla {
+// decode_simt.cu: whether the combine can hold W_up,t^V for this shape
+bool decode_combine_supported(int r_v, int d, bool recon);
+} // namespace lla
+
 using namespace lla;
 
 namespace {
